@@ -1,0 +1,64 @@
+"""Message-passing convolution and its CSR segmentation in float64 (oracle side; test
+infrastructure only).
+
+e3nn course, "Curriculum at a glance", lesson 06a: the point convolution forms, for each edge,
+the tensor product of the edge's spherical harmonics (scaled by radial weights) with the
+sender's features, and sums the messages over each receiver's neighbours.  "Modular v2106
+point models" (Scope) divides by sqrt(num_neighbors); the E3J summary, section E.2.2, names the
+receiver-ordered CSR aggregation that the GPU path uses.  Here the sum is the literal
+definition: messages are accumulated with ``np.add.at`` in the input edge order.
+
+Edge i -> j has sender ``src = i`` and receiver ``dst = j`` (lesson 05a: r_ij = r_j - r_i).
+"""
+
+import numpy as np
+
+from .tp import tp_backward, tp_forward
+
+
+def csr_build(n_nodes, src, dst):
+    """Receiver (dst) CSR and sender (src) CSR of an edge list.
+
+    perm_dst: stable argsort of dst (original edge ids in dst-sorted order).
+    row_ptr_dst[n]..row_ptr_dst[n+1]: positions of node n's in-edges in that order.
+    perm_src: stable argsort by src of the dst-sorted list (positions in dst-sorted order).
+    row_ptr_src: the same offsets per sender.
+    Ties keep input order (stable), which makes every array unique.
+    """
+    src = np.asarray(src, dtype=np.int64)
+    dst = np.asarray(dst, dtype=np.int64)
+    perm_dst = np.argsort(dst, kind="stable")
+    row_ptr_dst = np.concatenate([[0], np.cumsum(np.bincount(dst, minlength=n_nodes))])
+    perm_src = np.argsort(src[perm_dst], kind="stable")
+    row_ptr_src = np.concatenate([[0], np.cumsum(np.bincount(src, minlength=n_nodes))])
+    return (perm_dst.astype(np.int32), row_ptr_dst.astype(np.int32),
+            perm_src.astype(np.int32), row_ptr_src.astype(np.int32))
+
+
+def conv_forward(plan, n_nodes, src, dst, x, y, w, scale, chunk=4096):
+    """out[n] = scale * sum_{e: dst_e = n} TP(x[src_e], y_e, w_e)."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros((n_nodes, plan.irreps_out.dim))
+    n_edges = len(src)
+    for s in range(0, n_edges, chunk):
+        e = slice(s, min(s + chunk, n_edges))
+        msg = tp_forward(plan, x[src[e]], y[e], w[e])
+        np.add.at(out, dst[e], msg)
+    return scale * out
+
+
+def conv_backward(plan, n_nodes, src, dst, x, y, w, grad_out, scale, chunk=4096):
+    """(dx [N, dim1], dy [E, dim2], dw [E, weight_numel]) for conv_forward."""
+    x = np.asarray(x, dtype=np.float64)
+    g = np.asarray(grad_out, dtype=np.float64)
+    n_edges = len(src)
+    dx = np.zeros_like(x)
+    dy = np.zeros((n_edges, plan.irreps_in2.dim))
+    dw = np.zeros((n_edges, plan.weight_numel))
+    for s in range(0, n_edges, chunk):
+        e = slice(s, min(s + chunk, n_edges))
+        ddx, ddy, ddw = tp_backward(plan, x[src[e]], y[e], w[e], g[dst[e]])
+        np.add.at(dx, src[e], scale * ddx)
+        dy[e] = scale * ddy
+        dw[e] = scale * ddw
+    return dx, dy, dw

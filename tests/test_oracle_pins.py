@@ -1,0 +1,407 @@
+"""Pins of the float64 oracle to facts that do not come from the oracle itself: closed forms
+and textbook values, a library routine (sympy's Clebsch-Gordan), symmetry (rotations and
+reflections), orthogonality, multilinearity, finite differences and brute force."""
+
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.cg import complex_cg, real_basis_change, real_cg
+from oracle.sh import real_sh, real_sh_all
+from tests.conftest import rel_err
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rand_rot(rng):
+    q, r = np.linalg.qr(rng.standard_normal((3, 3)))
+    q = q * np.sign(np.diag(r))
+    if np.linalg.det(q) < 0:
+        q[:, 0] = -q[:, 0]
+    return q
+
+
+def wigner_real(l, R, rng):
+    """D^l(R) in the real-harmonic basis, fitted from Y(R r) = D Y(r) on random points
+    (exact up to rounding: the harmonics of one degree span a (2l+1)-dim space)."""
+    r = rng.standard_normal((4 * (2 * l + 1) + 8, 3))
+    A = real_sh(l, r)
+    B = real_sh(l, r @ R.T)
+    D, *_ = np.linalg.lstsq(A, B, rcond=None)
+    return D.T
+
+
+# ------------------------------------------------------------------------ harmonics ---
+def test_sh_closed_forms_low_degree():
+    rng = np.random.default_rng(0)
+    v = rng.standard_normal((50, 3))
+    u = v / np.linalg.norm(v, axis=1, keepdims=True)
+    x, y, z = u.T
+    np.testing.assert_allclose(real_sh(0, v)[:, 0], 1.0, atol=1e-15)
+    np.testing.assert_allclose(real_sh(1, v), math.sqrt(3) * np.stack([y, z, x], 1), atol=1e-14)
+    s15, s5 = math.sqrt(15), math.sqrt(5)
+    y2 = np.stack([s15 * x * y, s15 * y * z, s5 / 2 * (3 * z * z - 1), s15 * x * z, s15 / 2 * (x * x - y * y)], 1)
+    np.testing.assert_allclose(real_sh(2, v), y2, atol=1e-13)
+    # textbook real harmonics of degree 3 (orthonormal table times sqrt(4 pi))
+    y3 = np.stack([
+        math.sqrt(70) / 4 * y * (3 * x * x - y * y),
+        math.sqrt(105) * x * y * z,
+        math.sqrt(42) / 4 * y * (5 * z * z - 1),
+        math.sqrt(7) / 2 * z * (5 * z * z - 3),
+        math.sqrt(42) / 4 * x * (5 * z * z - 1),
+        math.sqrt(105) / 2 * z * (x * x - y * y),
+        math.sqrt(70) / 4 * x * (x * x - 3 * y * y),
+    ], 1)
+    np.testing.assert_allclose(real_sh(3, v), y3, atol=1e-13)
+
+
+@pytest.mark.parametrize("l", range(5))
+def test_sh_norm_parity_and_scale_invariance(l):
+    rng = np.random.default_rng(l)
+    v = rng.standard_normal((40, 3))
+    Y = real_sh(l, v)
+    np.testing.assert_allclose((Y * Y).sum(1), 2 * l + 1, rtol=1e-13)
+    np.testing.assert_allclose(real_sh(l, -v), (-1) ** l * Y, atol=1e-13)
+    np.testing.assert_allclose(real_sh(l, 3.7 * v), Y, atol=1e-13)
+
+
+@pytest.mark.parametrize("l", range(1, 5))
+def test_sh_harmonic(l):
+    # r^l Y_lm(r) is a harmonic polynomial: its Laplacian vanishes (central differences)
+    rng = np.random.default_rng(10 + l)
+    p = rng.standard_normal((10, 3))
+    h = 1e-3
+    f = lambda q: np.linalg.norm(q, axis=1, keepdims=True) ** l * real_sh(l, q)
+    lap = sum(f(p + h * e) + f(p - h * e) - 2 * f(p) for e in np.eye(3)) / h ** 2
+    assert np.abs(lap).max() < 1e-5 * max(1.0, np.abs(f(p)).max())
+
+
+def test_sh_zero_vector():
+    Y = real_sh_all(3, np.zeros((2, 3)))
+    assert Y[0, 0] == 1.0 and np.all(Y[:, 1:] == 0.0)
+
+
+@pytest.mark.parametrize("l", range(4))
+def test_sh_equivariance_and_wigner_homomorphism(l):
+    rng = np.random.default_rng(20 + l)
+    R1, R2 = rand_rot(rng), rand_rot(rng)
+    D1, D2, D12 = wigner_real(l, R1, rng), wigner_real(l, R2, rng), wigner_real(l, R1 @ R2, rng)
+    v = rng.standard_normal((30, 3))
+    np.testing.assert_allclose(real_sh(l, v @ R1.T), real_sh(l, v) @ D1.T, atol=1e-12)
+    np.testing.assert_allclose(D1 @ D1.T, np.eye(2 * l + 1), atol=1e-12)
+    np.testing.assert_allclose(D12, D1 @ D2, atol=1e-12)
+    if l == 1:
+        P = np.array([[0, 1, 0], [0, 0, 1], [1, 0, 0]], dtype=float)  # (x,y,z) -> (y,z,x)
+        np.testing.assert_allclose(D1, P @ R1 @ P.T, atol=1e-12)
+
+
+# ------------------------------------------------------------------ Clebsch-Gordan ---
+def test_complex_cg_matches_sympy():
+    from sympy.physics.quantum.cg import CG
+    for l1, l2 in itertools.product(range(4), range(4)):
+        for l3 in range(abs(l1 - l2), l1 + l2 + 1):
+            for m1 in range(-l1, l1 + 1):
+                for m2 in range(-l2, l2 + 1):
+                    m3 = m1 + m2
+                    if abs(m3) > l3:
+                        continue
+                    ref = float(CG(l1, m1, l2, m2, l3, m3).doit())
+                    assert abs(complex_cg(l1, m1, l2, m2, l3, m3) - ref) < 1e-14
+
+
+def test_complex_cg_textbook_values():
+    assert abs(complex_cg(1, 1, 1, -1, 0, 0) - 1 / math.sqrt(3)) < 1e-15
+    assert abs(complex_cg(1, 0, 1, 0, 0, 0) + 1 / math.sqrt(3)) < 1e-15
+    assert abs(complex_cg(1, 1, 1, 0, 2, 1) - 1 / math.sqrt(2)) < 1e-15
+    assert abs(complex_cg(1, 0, 1, 0, 2, 0) - math.sqrt(2 / 3)) < 1e-15
+    assert abs(complex_cg(1, 0, 1, 0, 1, 0)) < 1e-15
+
+
+def test_real_basis_change_is_unitary_and_real_sh_follows():
+    for l in range(5):
+        U = real_basis_change(l)
+        np.testing.assert_allclose(U @ U.conj().T, np.eye(2 * l + 1), atol=1e-15)
+
+
+def _golden_1x1():
+    vals = {0: np.zeros((3, 3, 1)), 1: np.zeros((3, 3, 3)), 2: np.zeros((3, 3, 5))}
+    with open(os.path.join(GOLDEN, "one_times_one.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            l3, m1, m2, m3, a, b = (int(t) for t in line.split())
+            vals[l3][m1 + 1, m2 + 1, m3 + l3] = math.copysign(math.sqrt(abs(a) / b), a)
+    return vals
+
+
+def test_real_cg_1x1_is_dot_cross_symtraceless():
+    gold = _golden_1x1()
+    for l3 in range(3):
+        np.testing.assert_allclose(real_cg(1, 1, l3), gold[l3], atol=1e-15)
+    rng = np.random.default_rng(3)
+    a, b = rng.standard_normal(3), rng.standard_normal(3)
+    P = [1, 2, 0]  # (y, z, x) order of the real basis
+    ar, br = a[P], b[P]
+    np.testing.assert_allclose(np.einsum("i,j,ijk->k", ar, br, real_cg(1, 1, 0)), [a @ b / math.sqrt(3)], atol=1e-14)
+    np.testing.assert_allclose(np.einsum("i,j,ijk->k", ar, br, real_cg(1, 1, 1)), np.cross(a, b)[P] / math.sqrt(6),
+                               atol=1e-14)
+
+
+@pytest.mark.parametrize("l1,l2", list(itertools.product(range(4), range(4))))
+def test_real_cg_orthogonality(l1, l2):
+    for l3 in range(abs(l1 - l2), l1 + l2 + 1):
+        for l3b in range(abs(l1 - l2), l1 + l2 + 1):
+            g = np.einsum("ijk,ijl->kl", real_cg(l1, l2, l3), real_cg(l1, l2, l3b))
+            ref = np.eye(2 * l3 + 1) / (2 * l3 + 1) if l3 == l3b else np.zeros((2 * l3 + 1, 2 * l3b + 1))
+            np.testing.assert_allclose(g, ref, atol=1e-14)
+
+
+@pytest.mark.parametrize("l1,l2", list(itertools.product(range(4), range(4))))
+def test_real_cg_equivariance(l1, l2):
+    rng = np.random.default_rng(100 + 4 * l1 + l2)
+    R = rand_rot(rng)
+    D1, D2 = wigner_real(l1, R, rng), wigner_real(l2, R, rng)
+    for l3 in range(abs(l1 - l2), l1 + l2 + 1):
+        D3 = wigner_real(l3, R, rng)
+        C = real_cg(l1, l2, l3)
+        # f(D1 a, D2 b) = D3 f(a, b) with f(a, b)_k = sum_ij C[i, j, k] a_i b_j
+        lhs = np.einsum("ia,jb,ijk->abk", D1, D2, C)
+        rhs = np.einsum("kc,abc->abk", D3, C)
+        np.testing.assert_allclose(lhs, rhs, atol=1e-12)
+
+
+@pytest.mark.parametrize("l1,l2", [(1, 1), (1, 2), (2, 2), (2, 3), (3, 3)])
+def test_real_cg_gaunt_property(l1, l2):
+    # for even l1+l2+l3, contracting C with Y^l1(r) Y^l2(r) gives a multiple of Y^l3(r)
+    rng = np.random.default_rng(7)
+    v = rng.standard_normal((25, 3))
+    for l3 in range(abs(l1 - l2), l1 + l2 + 1, 2):
+        f = np.einsum("ni,nj,ijk->nk", real_sh(l1, v), real_sh(l2, v), real_cg(l1, l2, l3))
+        Y3 = real_sh(l3, v)
+        c = (f * Y3).sum() / (Y3 * Y3).sum()
+        assert abs(c) > 1e-3
+        np.testing.assert_allclose(f, c * Y3, atol=1e-12)
+
+
+# --------------------------------------------------------------- tensor product ---
+def brute_tp(plan, x, y, w):
+    """Pure-Python loops over every index of the definition (tiny inputs only)."""
+    out = np.zeros((x.shape[0], plan.irreps_out.dim))
+    o1s, o2s, o3s = plan.irreps_in1.offsets(), plan.irreps_in2.offsets(), plan.irreps_out.offsets()
+    for b in range(x.shape[0]):
+        for p, ins in enumerate(plan.instructions):
+            a, c = plan.irreps_in1[ins.i_in1], plan.irreps_out[ins.i_out]
+            bb = plan.irreps_in2[ins.i_in2]
+            C = real_cg(a.l, bb.l, c.l)
+            for u in range(a.mul):
+                for v in range(bb.mul):
+                    wt = w[b, plan.weight_offsets[p] + u * bb.mul + v]
+                    for i in range(2 * a.l + 1):
+                        for j in range(2 * bb.l + 1):
+                            for k in range(2 * c.l + 1):
+                                out[b, o3s[ins.i_out] + u * (2 * c.l + 1) + k] += (
+                                    plan.alphas[p] * wt * C[i, j, k]
+                                    * x[b, o1s[ins.i_in1] + u * (2 * a.l + 1) + i]
+                                    * y[b, o2s[ins.i_in2] + v * (2 * bb.l + 1) + j])
+    return out
+
+
+def test_tp_matches_brute_force_loops():
+    rng = np.random.default_rng(5)
+    plan = oracle.make_plan("2x0e+2x1o+2x2e", "1x0e+1x1o+1x2e", lmax_out=2)
+    x = rng.standard_normal((3, plan.irreps_in1.dim))
+    y = rng.standard_normal((3, plan.irreps_in2.dim))
+    w = rng.standard_normal((3, plan.weight_numel))
+    np.testing.assert_allclose(oracle.tp_forward(plan, x, y, w), brute_tp(plan, x, y, w), atol=1e-13)
+
+
+def test_tp_multiplicity_two_inputs_brute_force():
+    # uvu with mul_y = 2 (sum over v with one weight per (u, v)) and a collapsed output
+    rng = np.random.default_rng(6)
+    plan = oracle.make_plan("2x1o", "2x1o", "2x0e+2x1e", instructions=[(0, 0, 0), (0, 0, 1)])
+    x = rng.standard_normal((2, plan.irreps_in1.dim))
+    y = rng.standard_normal((2, plan.irreps_in2.dim))
+    w = rng.standard_normal((2, plan.weight_numel))
+    np.testing.assert_allclose(oracle.tp_forward(plan, x, y, w), brute_tp(plan, x, y, w), atol=1e-13)
+
+
+def test_tp_scalar_path():
+    plan = oracle.make_plan("3x0e", "1x0e", lmax_out=0)
+    rng = np.random.default_rng(1)
+    x, y, w = rng.standard_normal((4, 3)), rng.standard_normal((4, 1)), rng.standard_normal((4, 3))
+    np.testing.assert_allclose(oracle.tp_forward(plan, x, y, w), x * y * w, atol=1e-15)
+
+
+def test_default_path_enumeration_counts():
+    p0 = oracle.make_plan("8x0e+8x1o", "1x0e+1x1o+1x2e", lmax_out=2)
+    assert [(plan_l(p0, i)) for i in range(p0.n_paths)] == [
+        (0, 0, 0), (0, 1, 1), (0, 2, 2), (1, 0, 1), (1, 1, 0), (1, 1, 1), (1, 1, 2), (1, 2, 1), (1, 2, 2)]
+    assert p0.irreps_out.dim == 29 * 8
+    p2 = oracle.make_plan("64x0e+64x1o+64x2e", "1x0e+1x1o+1x2e+1x3o", lmax_out=2)
+    assert p2.n_paths == 18 and p2.irreps_out.dim == 64 * 64
+    p3 = oracle.make_plan("128x0e+128x1o+128x2e+128x3o", "1x0e+1x1o+1x2e+1x3o", lmax_out=3)
+    assert p3.n_paths == 34 and p3.irreps_out.dim == 156 * 128
+    # parity rule: 1o x 1o -> 1e (pseudovector)
+    assert str(p0.irreps_out).split(" + ")[5] == "8x1e"
+
+
+def plan_l(plan, p):
+    ins = plan.instructions[p]
+    return plan.irreps_in1[ins.i_in1].l, plan.irreps_in2[ins.i_in2].l, plan.irreps_out[ins.i_out].l
+
+
+def test_instruction_validation():
+    with pytest.raises(ValueError):
+        oracle.make_plan("1x1o", "1x1o", "1x0o", instructions=[(0, 0, 0)])  # parity
+    with pytest.raises(ValueError):
+        oracle.make_plan("1x1o", "1x1o", "1x3e", instructions=[(0, 0, 0)])  # triangle
+    with pytest.raises(ValueError):
+        oracle.parse_irreps("3x1q")
+
+
+def _rep(plan_irreps, Ds, parity_flip, x):
+    """Apply the O(3) element (R, or -R when parity_flip) to features in mul_ir layout."""
+    out = np.empty_like(x)
+    for ir, off in zip(plan_irreps, plan_irreps.offsets()):
+        d = 2 * ir.l + 1
+        blk = x[:, off:off + ir.dim].reshape(x.shape[0], ir.mul, d)
+        s = ir.p if parity_flip else 1
+        out[:, off:off + ir.dim] = (s * blk @ Ds[ir.l].T).reshape(x.shape[0], -1)
+    return out
+
+
+@pytest.mark.parametrize("flip", [False, True])
+def test_tp_equivariance_o3(flip):
+    rng = np.random.default_rng(11 + flip)
+    plan = oracle.make_plan("3x0e+3x1o+3x2e+3x3o", "1x0e+1x1o+1x2e+1x3o", lmax_out=3)
+    R = rand_rot(rng)
+    Ds = {l: wigner_real(l, R, rng) for l in range(4)}
+    v = rng.standard_normal((5, 3))
+    x = rng.standard_normal((5, plan.irreps_in1.dim))
+    w = rng.standard_normal((5, plan.weight_numel))
+    g = -R if flip else R
+    y, y_rot = real_sh_all(3, v), real_sh_all(3, v @ g.T)
+    out = oracle.tp_forward(plan, x, y, w)
+    out_rot = oracle.tp_forward(plan, _rep(plan.irreps_in1, Ds, flip, x), y_rot, w)
+    np.testing.assert_allclose(out_rot, _rep(plan.irreps_out, Ds, flip, out), atol=1e-12)
+
+
+def test_tp_backward_euler_identities_and_fd():
+    rng = np.random.default_rng(12)
+    plan = oracle.make_plan("2x0e+2x1o+2x2e", "1x0e+1x1o+1x2e+1x3o", lmax_out=2)
+    B = 4
+    x = rng.standard_normal((B, plan.irreps_in1.dim))
+    y = rng.standard_normal((B, plan.irreps_in2.dim))
+    w = rng.standard_normal((B, plan.weight_numel))
+    g = rng.standard_normal((B, plan.irreps_out.dim))
+    dx, dy, dw = oracle.tp_backward(plan, x, y, w, g)
+    L = float((g * oracle.tp_forward(plan, x, y, w)).sum())
+    # the map is linear in each input separately: <grad, input> = L (Euler)
+    for d, t in ((dx, x), (dy, y), (dw, w)):
+        assert abs(float((d * t).sum()) - L) < 1e-11 * max(1.0, abs(L))
+    # central differences along random directions (exact for a linear function up to rounding)
+    h = 1e-3
+    for which, d in ((0, dx), (1, dy), (2, dw)):
+        args = [x, y, w]
+        dirn = rng.standard_normal(args[which].shape)
+        plus = list(args)
+        minus = list(args)
+        plus[which] = args[which] + h * dirn
+        minus[which] = args[which] - h * dirn
+        fd = ((g * oracle.tp_forward(plan, *plus)).sum() - (g * oracle.tp_forward(plan, *minus)).sum()) / (2 * h)
+        assert abs(fd - (d * dirn).sum()) < 1e-9 * max(1.0, abs(fd))
+
+
+# ------------------------------------------------------------------- convolution ---
+def small_graph(seed, n=40, e=300):
+    rng = np.random.default_rng(seed)
+    src = rng.integers(0, n, e).astype(np.int32)
+    dst = rng.integers(0, n, e).astype(np.int32)
+    return rng, src, dst
+
+
+def test_csr_bit_exact_against_loops():
+    rng, src, dst = small_graph(1)
+    n = 40
+    perm_dst, rp_dst, perm_src, rp_src = oracle.csr_build(n, src, dst)
+    # brute force: receivers ascending, ties in input order
+    ref = [e for v in range(n) for e in range(len(dst)) if dst[e] == v]
+    assert perm_dst.tolist() == ref
+    srt = src[perm_dst]
+    ref_s = [i for v in range(n) for i in range(len(srt)) if srt[i] == v]
+    assert perm_src.tolist() == ref_s
+    assert rp_dst[0] == 0 and rp_dst[-1] == len(dst) and np.all(np.diff(rp_dst) >= 0)
+    assert rp_dst.tolist() == [sum(1 for d in dst if d < v) for v in range(n + 1)]
+    assert rp_src.tolist() == [sum(1 for s in src if s < v) for v in range(n + 1)]
+
+
+def test_conv_edge_order_invariance_isolated_and_empty():
+    rng, src, dst = small_graph(2)
+    n = 40
+    dst[dst == 7] = 8  # node 7 has no in-edges
+    plan = oracle.make_plan("2x0e+2x1o", "1x0e+1x1o+1x2e", lmax_out=2)
+    x = rng.standard_normal((n, plan.irreps_in1.dim))
+    v = rng.standard_normal((len(src), 3))
+    y = real_sh_all(2, v)
+    w = rng.standard_normal((len(src), plan.weight_numel))
+    out = oracle.conv_forward(plan, n, src, dst, x, y, w, 0.5)
+    p = rng.permutation(len(src))
+    out2 = oracle.conv_forward(plan, n, src[p], dst[p], x, y[p], w[p], 0.5)
+    np.testing.assert_allclose(out2, out, atol=1e-13)
+    assert np.all(out[7] == 0.0)
+    e0 = np.zeros(0, dtype=np.int32)
+    z = oracle.conv_forward(plan, n, e0, e0, x, y[:0], w[:0], 0.5)
+    assert z.shape == out.shape and np.all(z == 0.0)
+    # sum over edges: equals the per-edge products accumulated by receiver with loops
+    ref = np.zeros_like(out)
+    msg = oracle.tp_forward(plan, x[src], y, w)
+    for e in range(len(src)):
+        ref[dst[e]] += 0.5 * msg[e]
+    np.testing.assert_allclose(out, ref, atol=1e-13)
+
+
+def test_conv_equivariance_rotated_positions():
+    rng = np.random.default_rng(13)
+    n = 12
+    pos = rng.uniform(0, 3, (n, 3))
+    src, dst = np.nonzero(np.ones((n, n)) - np.eye(n))
+    src, dst = src.astype(np.int32), dst.astype(np.int32)
+    plan = oracle.make_plan("2x0e+2x1o+2x2e", "1x0e+1x1o+1x2e+1x3o", lmax_out=2)
+    x = rng.standard_normal((n, plan.irreps_in1.dim))
+    w = rng.standard_normal((len(src), plan.weight_numel))
+    R = rand_rot(rng)
+    Ds = {l: wigner_real(l, R, rng) for l in range(4)}
+    vec = pos[dst] - pos[src]
+    out = oracle.conv_forward(plan, n, src, dst, x, real_sh_all(3, vec), w, 1.0)
+    out_r = oracle.conv_forward(plan, n, src, dst, _rep(plan.irreps_in1, Ds, False, x),
+                                real_sh_all(3, (pos @ R.T)[dst] - (pos @ R.T)[src]), w, 1.0)
+    np.testing.assert_allclose(out_r, _rep(plan.irreps_out, Ds, False, out), atol=1e-12)
+
+
+def test_conv_backward_euler_and_fd():
+    rng, src, dst = small_graph(3, n=15, e=80)
+    n = 15
+    plan = oracle.make_plan("2x0e+2x1o+2x2e", "1x0e+1x1o+1x2e+1x3o", lmax_out=2)
+    x = rng.standard_normal((n, plan.irreps_in1.dim))
+    y = real_sh_all(3, rng.standard_normal((len(src), 3)))
+    w = rng.standard_normal((len(src), plan.weight_numel))
+    g = rng.standard_normal((n, plan.irreps_out.dim))
+    s = 0.3
+    dx, dy, dw = oracle.conv_backward(plan, n, src, dst, x, y, w, g, s)
+    L = float((g * oracle.conv_forward(plan, n, src, dst, x, y, w, s)).sum())
+    for d, t in ((dx, x), (dy, y), (dw, w)):
+        assert abs(float((d * t).sum()) - L) < 1e-11 * max(1.0, abs(L))
+    h = 1e-3
+    for which, d in ((0, dx), (1, dy), (2, dw)):
+        args = [x, y, w]
+        dirn = rng.standard_normal(args[which].shape)
+        pl, mi = list(args), list(args)
+        pl[which] = args[which] + h * dirn
+        mi[which] = args[which] - h * dirn
+        f = lambda a: float((g * oracle.conv_forward(plan, n, src, dst, a[0], a[1], a[2], s)).sum())
+        fd = (f(pl) - f(mi)) / (2 * h)
+        assert abs(fd - float((d * dirn).sum())) < 1e-9 * max(1.0, abs(fd))
