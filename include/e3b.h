@@ -1,0 +1,230 @@
+/*
+ * e3b.h -- C ABI of the B200 (sm_100a) library for the channelwise ("uvu") Clebsch-Gordan
+ * tensor product and the message-passing convolution built on it.
+ *
+ * Sources for what each call computes:
+ *   [TP]   e3nn course, "Curriculum at a glance", lesson 03a (Clebsch-Gordan decomposition,
+ *          parity rule p3 = p1 p2, triangle rule) and lesson 03b (weighted tensor product
+ *          x (x)_w y, instructions, connection modes, counting weights).
+ *   [IRR]  same page, lesson 02a (irreps strings "16x0e + 8x1o", memory layout); lesson 12a
+ *          (mul_ir layout; a mismatch silently gives wrong numbers).
+ *   [SH]   same page, lesson 02b (Y^l(R r) = D^l(R) Y^l(r), parity (-1)^l, normalisations);
+ *          "Modular v2106 point models", Scope (component-normalised harmonics).
+ *   [CONV] same course page, lesson 06a (point convolution m_ij = (R(|r_ij|) Y(r_ij)) (x)_w h_j,
+ *          summed over neighbours) and lesson 05a (edge i -> j, r_ij = r_j - r_i);
+ *          "Modular v2106 point models", Scope (1/sqrt(num_neighbors) normalisation);
+ *          E3J (Peltre et al., "E3J: An Efficient and Open-Source Backend for Euclidean
+ *          Equivariant Operations on GPU and TPU"), section E.2.2 (CSR receiver aggregation
+ *          without atomics) and section C.2 (deterministic aggregation).
+ *   [BWD]  E3J, section E.1 (reverse mode by transposing the linearised operation).
+ *   [CG]   E3J, section G.2 (top-spin vector from a triangular system, then the lowering
+ *          operator) -- the construction the library uses for its coefficient table.
+ *
+ * Conventions shared by every call
+ *   - Tensors are dense, row-major, contiguous, in the mul_ir layout [IRR]: irrep blocks in
+ *     order; inside a block [u][m] with m = -l..l fastest.  Every pointer must be 16-byte
+ *     aligned.  The caller owns all memory; the library owns only plans.
+ *   - Device pointers unless stated; every compute call is asynchronous on `stream` (a
+ *     cudaStream_t passed as void*; NULL means the legacy default stream).
+ *   - The element type of every float tensor is the plan's dtype (float or double).
+ *   - Weights w are [B or E, weight_numel], path-major in instruction order, then channel u
+ *     (uvu with mul_in2 = 1: one weight per (path, u)).  E3_W_SHARED: one row [weight_numel].
+ *   - Real spherical harmonics use m = -l..l with the z axis as the pole and no
+ *     Condon-Shortley phase, so Y^1 = sqrt(3) (y, z, x) / |r| under component normalisation.
+ *   - Real CG tensors have Frobenius norm 1 per path; sign: positive C[0,0,0] when
+ *     l1+l2+l3 is even, else a positive first nonzero entry in lexicographic (m1,m2,m3) order.
+ *     1 (x) 1 then gives +dot/sqrt(3), +cross/sqrt(6) and the symmetric traceless product.
+ *   - Path weight alpha_p defaults to sqrt((2 l3 + 1) / (mul_in2 * n_out)), n_out = number of
+ *     instructions writing the same output block (uncollapsed: sqrt(2 l3 + 1)).
+ *   - Errors are returned before any launch when they can be seen on the host; the message
+ *     is available from e3_last_error().  Errors seen on the device (an index out of range,
+ *     a bounded wait that gave up) are recorded in one status word per device, shared by
+ *     every call on that device, and read (and cleared) by e3_device_status(); the offending
+ *     edge is skipped, never dereferenced.
+ *   - Results are deterministic: the same inputs give bitwise the same outputs (no atomics
+ *     on floating-point data).
+ */
+#ifndef E3B_H
+#define E3B_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define E3_API __attribute__((visibility("default")))
+#else
+#define E3_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  E3_OK = 0,
+  E3_ERR_INVALID_ARG = 1,  /* NULL/misaligned pointer, negative size, bad enum */
+  E3_ERR_IRREPS_PARSE = 2, /* malformed irreps string */
+  E3_ERR_INSTRUCTION = 3,  /* triangle rule, parity rule, index range, multiplicity */
+  E3_ERR_UNSUPPORTED = 4,  /* valid request with no compiled kernel (mode, degrees, layout) */
+  E3_ERR_SHAPE = 5,        /* sizes that do not fit (e.g. row_ptr[N] != E, too many edges) */
+  E3_ERR_INDEX = 6,        /* device: an index out of range was seen (checked kernels) */
+  E3_ERR_CUDA = 7,         /* a CUDA runtime call failed */
+  E3_ERR_TIMEOUT = 8       /* device: a bounded wait gave up */
+} e3_status;
+
+typedef enum { E3_F32 = 0, E3_F64 = 1 } e3_dtype;
+
+/* Connection modes of lesson 03b [TP].  Only E3_UVU has kernels; others -> UNSUPPORTED. */
+typedef enum { E3_UVU = 0, E3_UVW = 1, E3_UUU = 2, E3_UUW = 3 } e3_mode;
+
+/* SH normalisations of lesson 02b [SH]: component (sum_m Y^2 = 2l+1), integral
+ * (component / sqrt(4 pi)), norm (component / sqrt(2l+1)).  Used only with edge vectors. */
+typedef enum { E3_SH_COMPONENT = 0, E3_SH_INTEGRAL = 1, E3_SH_NORM = 2 } e3_sh_norm;
+
+typedef enum { E3_W_PER_SAMPLE = 0, E3_W_SHARED = 1 } e3_weight_mode;
+
+/* One instruction of lesson 03b [TP]: couple irrep i_in1 of input 1 with irrep i_in2 of
+ * input 2 into irrep i_out of the output.  path_weight < 0 selects the default alpha_p. */
+typedef struct {
+  int32_t i_in1, i_in2, i_out;
+  int32_t has_weight; /* must be 1 for the compiled kernels */
+  double path_weight;
+} e3_instruction;
+
+typedef struct e3_plan e3_plan;
+
+/* ---------------------------------------------------------------- plans (host, once) --- */
+
+/* Build a plan [TP][IRR][CG].
+ *   irreps_in1  node features, e.g. "64x0e+64x1o+64x2e".  Kernels need one irrep per degree
+ *               l = 0..Lx in ascending order (any parities), one common multiplicity C with
+ *               C % 4 == 0, Lx <= 3.
+ *   irreps_in2  edge attributes, e.g. "1x0e+1x1o+1x2e+1x3o": multiplicity 1, l = 0..Ly, Ly <= 3.
+ *   irreps_out  with n_instr == 0: a filter listing the output irreps allowed (multiplicities
+ *               ignored; NULL or "" = all); instructions are then enumerated as
+ *               for i1, for i2, for l3 = |l1-l2| .. l1+l2 with (l3, p1 p2) in the filter,
+ *               each with its own output block of multiplicity C ("uncollapsed").
+ *               With n_instr > 0: the output irreps that the instructions index.
+ *   instr       n_instr explicit instructions (may be NULL when n_instr == 0).
+ * The compiled kernels cover the full enumeration for (Lx, Ly, Lo) in the set listed by
+ * e3_supported(); an explicit list must equal that enumeration (alphas may differ).
+ * The CG table is generated here by the ladder construction and uploaded to the current
+ * device on first use.  The plan is bound to the current CUDA device.
+ * Returns IRREPS_PARSE, INSTRUCTION, UNSUPPORTED, INVALID_ARG or CUDA on failure. */
+E3_API e3_status e3_plan_create(const char* irreps_in1, const char* irreps_in2, const char* irreps_out,
+                         const e3_instruction* instr, int32_t n_instr, e3_mode mode,
+                         e3_dtype dtype, e3_weight_mode wmode, e3_plan** plan);
+
+E3_API e3_status e3_plan_destroy(e3_plan* plan);
+
+/* Sizes per sample: dims of x, y, out (floats), weight_numel, number of paths.  Any output
+ * pointer may be NULL. */
+E3_API e3_status e3_plan_info(const e3_plan* plan, int64_t* dim_in1, int64_t* dim_in2, int64_t* dim_out,
+                       int64_t* weight_numel, int32_t* n_paths);
+
+/* The output irreps as a string ("64x0e+64x1o+...") written into buf (NUL-terminated);
+ * *needed receives the length including the NUL.  buf may be NULL to query the length. */
+E3_API e3_status e3_plan_irreps_out(const e3_plan* plan, char* buf, size_t buf_len, size_t* needed);
+
+/* Per path: (l1, l2, l3) into lls[3*p..3*p+2] and alpha_p into alpha[p] (host arrays of
+ * n_paths entries; either may be NULL). */
+E3_API e3_status e3_plan_paths(const e3_plan* plan, int32_t* lls, double* alpha);
+
+/* Synchronise `stream`, return the current device's status word (E3_OK, E3_ERR_INDEX or
+ * E3_ERR_TIMEOUT; the first error recorded since the last read) and clear it. */
+E3_API e3_status e3_device_status(void* stream);
+
+/* Real CG table as generated for the plan's kernels: dense [2l1+1][2l2+1][2l3+1] doubles
+ * for (l1, l2, l3), written to out (host).  Exposed for table-against-table checks. */
+E3_API e3_status e3_cg_dense(int32_t l1, int32_t l2, int32_t l3, double* out);
+
+/* Space-separated list "Lx,Ly,Lo ..." of degree triples with compiled kernels. */
+E3_API const char* e3_supported(void);
+
+/* ------------------------------------------------------------ tensor product (no graph) --- */
+
+/* out[b] = TP(x[b], y[b], w[b]) for b < B [TP].
+ *   x [B, dim_in1], y [B, dim_in2], w [B, weight_numel] (or [weight_numel] if shared),
+ *   out [B, dim_out] (overwritten).  B == 0 is a no-op.  B < 2^31. */
+E3_API e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x, const void* y,
+                        const void* w, void* out, void* stream);
+
+/* Gradients of <grad_out, TP(x, y, w)> by transposition [BWD].  Each of grad_x [B, dim_in1],
+ * grad_y [B, dim_in2], grad_w [B, weight_numel] may be NULL to skip it; outputs are
+ * overwritten.  E3_W_SHARED plans are not supported for the backward. */
+E3_API e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* x, const void* y,
+                         const void* w, const void* grad_out, void* grad_x, void* grad_y,
+                         void* grad_w, void* stream);
+
+/* ------------------------------------------------------------------ harmonics --- */
+
+/* Real spherical harmonics Y^0..Y^lmax of n vectors [SH]: out[i] = [Y^0 | Y^1 | ... ] with
+ * (lmax+1)^2 values per vector, normalisation sh_norm; vec [n, 3] (any stride-3 layout,
+ * element-aligned), out [n, (lmax+1)^2].  A zero vector gives Y^0 = 1 (scaled by the
+ * normalisation) and Y^{l>0} = 0.  lmax <= 3.  n == 0 is a no-op. */
+E3_API e3_status e3_spherical_harmonics(int32_t lmax, int64_t n, const void* vec, e3_sh_norm sh_norm,
+                                 e3_dtype dtype, void* out, void* stream);
+
+/* ------------------------------------------------------------------ CSR segmentation --- */
+
+/* Bytes of device workspace that e3_csr_build needs for N nodes and E edges. */
+E3_API e3_status e3_csr_workspace_size(int64_t N, int64_t E, size_t* bytes);
+
+/* Receiver and sender CSR of an edge list [CONV] (integer-only, bit-exact):
+ *   perm_dst[E]      original edge ids in receiver order, ties in input order (stable);
+ *   row_ptr_dst[N+1] node n's in-edges are positions row_ptr_dst[n] .. row_ptr_dst[n+1]-1;
+ *   perm_src[E]      positions in receiver order, sorted stably by sender;
+ *   row_ptr_src[N+1] node n's out-edges are perm_src[row_ptr_src[n] .. row_ptr_src[n+1]-1].
+ * src, dst: int32 [E] in [0, N).  An id out of range records E3_ERR_INDEX in the device
+ * status word (e3_device_status) and the outputs are then unspecified.  workspace: device
+ * buffer of at least e3_csr_workspace_size bytes, 256-byte aligned.  N, E < 2^31. */
+E3_API e3_status e3_csr_build(int64_t N, int64_t E, const int32_t* src, const int32_t* dst,
+                       int32_t* perm_dst, int32_t* row_ptr_dst, int32_t* perm_src,
+                       int32_t* row_ptr_src, void* workspace, size_t ws_bytes, void* stream);
+
+/* Rows of `in` gathered by `perm`: out[i, :] = in[perm[i], :] for i < n_rows, each row
+ * row_bytes bytes (multiple of 4).  Used once per topology to put edge arrays into receiver
+ * order.  perm entries must lie in [0, n_in_rows). */
+E3_API e3_status e3_gather_rows(int64_t n_rows, int64_t n_in_rows, int64_t row_bytes,
+                         const int32_t* perm, const void* in, void* out, void* stream);
+
+/* ----------------------------------------------------------------------- convolution --- */
+
+/* out[n] = out_scale * sum_{e : dst_e = n} TP(x[src_e], Y_e, w_e)   [CONV][TP]
+ * Edge arrays are in receiver order (apply perm_dst once per topology):
+ *   row_ptr_dst [N+1] (row_ptr_dst[0] == 0, row_ptr_dst[N] == E, non-decreasing);
+ *   src [E] int32 in [0, N);
+ *   exactly one of y [E, dim_in2] (given harmonics) or edge_vec [E, 3] (r_j - r_i, harmonics
+ *   computed in registers with normalisation sh_norm; requires irreps_in2 = 1x0+1x1+..);
+ *   w [E, weight_numel] (or [weight_numel] if shared); x [N, dim_in1]; out [N, dim_out]
+ *   (overwritten; nodes without in-edges get zero rows).  E == 0 zero-fills out.
+ * No atomics: each output row is reduced by one CTA in edge order.  An src id or row_ptr
+ * entry out of range records E3_ERR_INDEX in the device status word and that edge is
+ * skipped.  N, E < 2^31. */
+E3_API e3_status e3_conv_forward(const e3_plan* plan, int64_t N, int64_t E, const int32_t* row_ptr_dst,
+                          const int32_t* src, const void* x, const void* y, const void* edge_vec,
+                          e3_sh_norm sh_norm, const void* w, double out_scale, void* out,
+                          void* stream);
+
+/* Gradients of <grad_out, conv_forward(...)> [BWD][CONV] with respect to
+ *   grad_x [N, dim_in1]: sum over each node's out-edges (sender CSR: row_ptr_src, perm_src);
+ *   grad_y [E, dim_in2]: per edge, with respect to the harmonics (also when they were
+ *                        computed from edge_vec);
+ *   grad_w [E, weight_numel]: per edge.
+ * Any gradient pointer may be NULL to skip it.  Other arguments as e3_conv_forward; dst [E]
+ * is the receiver of each (receiver-ordered) edge.  Shared weights are not supported. */
+E3_API e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E, const int32_t* row_ptr_dst,
+                           const int32_t* src, const int32_t* dst, const int32_t* row_ptr_src,
+                           const int32_t* perm_src, const void* x, const void* y,
+                           const void* edge_vec, e3_sh_norm sh_norm, const void* w,
+                           const void* grad_out, double out_scale, void* grad_x, void* grad_y,
+                           void* grad_w, void* stream);
+
+/* Message of the last non-OK status returned on the calling thread ("" if none). */
+E3_API const char* e3_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* E3B_H */

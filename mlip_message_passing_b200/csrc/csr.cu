@@ -1,0 +1,275 @@
+// Receiver / sender CSR segmentation of an edge list, and a row gather, for sm_100a.
+//
+// E3J, section E.2.2: the convolution aggregates messages per receiver over a CSR adjacency
+// so that no atomics are needed; section C.2: aggregation must be deterministic.  The
+// segmentation here is integer-only and bit-exact: perm_dst is the stable sort of the edges
+// by receiver, perm_src the stable sort of that order by sender, and the row pointers are
+// exclusive prefix sums of the degree counts.
+//
+// The stable sorts are least-significant-digit radix sorts with 8-bit digits over the
+// ceil(log2 N) bits that a node id can use.  Each pass: per-tile digit counts, one exclusive
+// scan over the (digit, tile) table in digit-major order, then a scatter in which every tile
+// ranks its elements stably (tile rounds of 256 elements in input order, warp-level match of
+// equal digits, per-warp counts combined in warp order).  Counting uses integer atomics in
+// shared memory only; ranks never depend on thread scheduling, so the output is unique.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+
+namespace e3b {
+
+constexpr int RS_THREADS = 256;
+constexpr int RS_ROUNDS = 8;  // rounds of 256 elements per tile
+constexpr int RS_TILE = RS_THREADS * RS_ROUNDS;
+constexpr int RS_RADIX = 256;
+
+__device__ __forceinline__ void rs_error(int* status, int code) { atomicCAS(status, 0, code); }
+
+// key of element i: keys[gather ? gather[i] : i]
+__device__ __forceinline__ uint32_t rs_key(const int32_t* __restrict__ keys, const int32_t* __restrict__ gather,
+                                           int64_t i) {
+  const int64_t j = gather ? int64_t(__ldg(gather + i)) : i;
+  return uint32_t(__ldg(keys + j));
+}
+
+// counts[d * n_tiles + tile] = number of elements of `tile` whose digit is d
+__global__ void __launch_bounds__(RS_THREADS) rs_count(const int32_t* __restrict__ keys,
+                                                       const int32_t* __restrict__ gather, int64_t n,
+                                                       int shift, int n_tiles, int32_t* __restrict__ counts) {
+  __shared__ int32_t h[RS_RADIX];
+  h[threadIdx.x] = 0;
+  __syncthreads();
+  const int64_t base = int64_t(blockIdx.x) * RS_TILE;
+  for (int r = 0; r < RS_ROUNDS; ++r) {
+    const int64_t i = base + int64_t(r) * RS_THREADS + threadIdx.x;
+    if (i < n) atomicAdd(&h[(rs_key(keys, gather, i) >> shift) & 0xff], 1);
+  }
+  __syncthreads();
+  counts[int64_t(threadIdx.x) * n_tiles + blockIdx.x] = h[threadIdx.x];
+}
+
+// In-place exclusive scan of a[0..n) by one CTA of 1024 threads (chunked serial sums, then a
+// block scan of the chunk totals).  total (optional) receives the sum.
+__global__ void __launch_bounds__(1024) exclusive_scan_1cta(int32_t* __restrict__ a, int64_t n,
+                                                            int32_t* __restrict__ total) {
+  __shared__ int32_t part[1024];
+  const int t = threadIdx.x;
+  const int64_t chunk = (n + 1023) / 1024;
+  const int64_t b = t * chunk, e = b + chunk < n ? b + chunk : n;
+  int32_t s = 0;
+  for (int64_t i = b; i < e; ++i) s += a[i];
+  part[t] = s;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const int32_t v = t >= off ? part[t - off] : 0;
+    __syncthreads();
+    part[t] += v;
+    __syncthreads();
+  }
+  int32_t run = part[t] - s;  // exclusive prefix of this chunk
+  for (int64_t i = b; i < e; ++i) {
+    const int32_t v = a[i];
+    a[i] = run;
+    run += v;
+  }
+  if (total != nullptr && t == 1023) *total = part[1023];
+}
+
+// Stable scatter of one pass.  offsets: exclusive scan of counts (digit-major).
+__global__ void __launch_bounds__(RS_THREADS) rs_scatter(const int32_t* __restrict__ keys,
+                                                         const int32_t* __restrict__ gather,
+                                                         const int32_t* __restrict__ vals_in, int64_t n, int shift,
+                                                         int n_tiles, const int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ keys_out,
+                                                         int32_t* __restrict__ vals_out) {
+  __shared__ int32_t run[RS_RADIX];              // running count per digit in this tile
+  __shared__ int32_t wc[RS_THREADS / 32][RS_RADIX];  // per-warp counts of the current round
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  run[t] = offsets[int64_t(t) * n_tiles + blockIdx.x];
+  const int64_t base = int64_t(blockIdx.x) * RS_TILE;
+  for (int r = 0; r < RS_ROUNDS; ++r) {
+    for (int q = t; q < (RS_THREADS / 32) * RS_RADIX; q += RS_THREADS) (&wc[0][0])[q] = 0;
+    __syncthreads();
+    const int64_t i = base + int64_t(r) * RS_THREADS + t;
+    const bool ok = i < n;
+    uint32_t key = 0;
+    int d = RS_RADIX;  // sentinel: no element
+    if (ok) {
+      key = rs_key(keys, gather, i);
+      d = int((key >> shift) & 0xff);
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, d);
+    const int rank_in_warp = __popc(peers & ((1u << lane) - 1u));
+    if (ok && rank_in_warp == 0) wc[warp][d] = __popc(peers);
+    __syncthreads();
+    if (ok) {
+      int32_t pos = run[d] + rank_in_warp;
+      for (int w = 0; w < warp; ++w) pos += wc[w][d];
+      if (keys_out) keys_out[pos] = int32_t(key);
+      vals_out[pos] = vals_in ? __ldg(vals_in + i) : int32_t(i);
+    }
+    __syncthreads();
+    {
+      int32_t add = 0;
+      for (int w = 0; w < RS_THREADS / 32; ++w) add += wc[w][t];
+      run[t] += add;
+    }
+    __syncthreads();
+  }
+}
+
+// degree counts (row_ptr[id] += 1); ids outside [0, N) are reported and skipped
+__global__ void degree_count(const int32_t* __restrict__ ids, int64_t n, int64_t N, int32_t* __restrict__ row_ptr,
+                             int* status) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int32_t v = __ldg(ids + i);
+    if (v < 0 || v >= N) {
+      rs_error(status, E3_ERR_INDEX);
+      continue;
+    }
+    atomicAdd(row_ptr + v, 1);
+  }
+}
+
+__global__ void gather_rows_kernel(int64_t n_rows, int64_t n_in_rows, int64_t row_words, bool vec16,
+                                   const int32_t* __restrict__ perm, const uint32_t* __restrict__ in,
+                                   uint32_t* __restrict__ out, int* status) {
+  const int64_t per_row = vec16 ? row_words / 4 : row_words;
+  const int64_t total = n_rows * per_row;
+  for (int64_t q = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; q < total; q += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = q / per_row, c = q % per_row;
+    const int32_t s = __ldg(perm + r);
+    if (s < 0 || s >= n_in_rows) {
+      rs_error(status, E3_ERR_INDEX);
+      continue;
+    }
+    if (vec16)
+      reinterpret_cast<uint4*>(out)[r * per_row + c] = __ldg(reinterpret_cast<const uint4*>(in) + int64_t(s) * per_row + c);
+    else
+      out[r * row_words + c] = __ldg(in + int64_t(s) * row_words + c);
+  }
+}
+
+// ------------------------------------------------------------------------ host side ---
+static int64_t n_tiles_of(int64_t E) { return (E + RS_TILE - 1) / RS_TILE; }
+static size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+static size_t csr_ws_bytes(int64_t E) {
+  const int64_t nt = n_tiles_of(E) > 0 ? n_tiles_of(E) : 1;
+  return 4 * align256(sizeof(int32_t) * size_t(E > 0 ? E : 1)) + align256(sizeof(int32_t) * size_t(RS_RADIX) * nt);
+}
+
+static int key_bits(int64_t N) {
+  int b = 1;
+  while ((int64_t(1) << b) < N) ++b;
+  return b;
+}
+
+// Stable sort of element indices 0..n by key(i); writes the sorted indices to vals_final.
+static e3_status radix_sort(const int32_t* keys, const int32_t* gather, int64_t n, int bits, int32_t* vals_final,
+                            int32_t* ka, int32_t* va, int32_t* kb, int32_t* vb, int32_t* counts, cudaStream_t s) {
+  const int n_tiles = int(n_tiles_of(n));
+  const int passes = (bits + 7) / 8;
+  const int32_t* kin = keys;
+  const int32_t* gin = gather;
+  const int32_t* vin = nullptr;
+  for (int p = 0; p < passes; ++p) {
+    const bool last = p == passes - 1;
+    int32_t* kout = last ? nullptr : (p % 2 == 0 ? ka : kb);
+    int32_t* vout = last ? vals_final : (p % 2 == 0 ? va : vb);
+    rs_count<<<n_tiles, RS_THREADS, 0, s>>>(kin, gin, n, 8 * p, n_tiles, counts);
+    exclusive_scan_1cta<<<1, 1024, 0, s>>>(counts, int64_t(RS_RADIX) * n_tiles, nullptr);
+    rs_scatter<<<n_tiles, RS_THREADS, 0, s>>>(kin, gin, vin, n, 8 * p, n_tiles, counts, kout, vout);
+    kin = kout;
+    gin = nullptr;
+    vin = vout;
+  }
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "radix sort launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+}  // namespace e3b
+
+using namespace e3b;
+
+extern "C" e3_status e3_csr_workspace_size(int64_t N, int64_t E, size_t* bytes) {
+  clear_error();
+  if (bytes == nullptr) return fail(E3_ERR_INVALID_ARG, "bytes is NULL");
+  if (N < 0 || E < 0 || N >= (int64_t(1) << 31) || E >= (int64_t(1) << 31))
+    return fail(E3_ERR_SHAPE, "N or E out of range");
+  *bytes = csr_ws_bytes(E);
+  return E3_OK;
+}
+
+extern "C" e3_status e3_csr_build(int64_t N, int64_t E, const int32_t* src, const int32_t* dst, int32_t* perm_dst,
+                                  int32_t* row_ptr_dst, int32_t* perm_src, int32_t* row_ptr_src, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+  clear_error();
+  if (N < 0 || E < 0 || N >= (int64_t(1) << 31) || E >= (int64_t(1) << 31))
+    return fail(E3_ERR_SHAPE, "N or E out of range");
+  if (row_ptr_dst == nullptr || row_ptr_src == nullptr) return fail(E3_ERR_INVALID_ARG, "row_ptr array is NULL");
+  if (E > 0 && (src == nullptr || dst == nullptr || perm_dst == nullptr || perm_src == nullptr))
+    return fail(E3_ERR_INVALID_ARG, "edge array is NULL");
+  if (E > 0 && N == 0) return fail(E3_ERR_SHAPE, "edges without nodes");
+  if (E > 0 && (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+    return fail(E3_ERR_INVALID_ARG, "workspace is NULL or not 256-byte aligned");
+  if (E > 0 && ws_bytes < csr_ws_bytes(E))
+    return fail(E3_ERR_SHAPE, "workspace of %zu bytes, need %zu", ws_bytes, csr_ws_bytes(E));
+  int* status = nullptr;
+  e3_status st = device_status_ptr(&status);
+  if (st != E3_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaMemsetAsync(row_ptr_dst, 0, sizeof(int32_t) * size_t(N + 1), s);
+  if (err == cudaSuccess) err = cudaMemsetAsync(row_ptr_src, 0, sizeof(int32_t) * size_t(N + 1), s);
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "memset failed: %s", cudaGetErrorString(err));
+  if (E == 0) return E3_OK;
+  const int blocks = int(std::min<int64_t>((E + 255) / 256, 148 * 8));
+  degree_count<<<blocks, 256, 0, s>>>(dst, E, N, row_ptr_dst, status);
+  degree_count<<<blocks, 256, 0, s>>>(src, E, N, row_ptr_src, status);
+  // row_ptr[n] = c_n for n < N and row_ptr[N] = 0: one exclusive scan over N + 1 entries
+  // gives row_ptr[n] = sum_{m < n} c_m and row_ptr[N] = E
+  exclusive_scan_1cta<<<1, 1024, 0, s>>>(row_ptr_dst, N + 1, nullptr);
+  exclusive_scan_1cta<<<1, 1024, 0, s>>>(row_ptr_src, N + 1, nullptr);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "count launch failed: %s", cudaGetErrorString(err));
+
+  char* ws = static_cast<char*>(workspace);
+  const size_t eb = align256(sizeof(int32_t) * size_t(E));
+  int32_t* ka = reinterpret_cast<int32_t*>(ws);
+  int32_t* va = reinterpret_cast<int32_t*>(ws + eb);
+  int32_t* kb = reinterpret_cast<int32_t*>(ws + 2 * eb);
+  int32_t* vb = reinterpret_cast<int32_t*>(ws + 3 * eb);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + 4 * eb);
+  const int bits = key_bits(N);
+  st = radix_sort(dst, nullptr, E, bits, perm_dst, ka, va, kb, vb, counts, s);
+  if (st != E3_OK) return st;
+  st = radix_sort(src, perm_dst, E, bits, perm_src, ka, va, kb, vb, counts, s);
+  return st;
+}
+
+extern "C" e3_status e3_gather_rows(int64_t n_rows, int64_t n_in_rows, int64_t row_bytes, const int32_t* perm,
+                                    const void* in, void* out, void* stream) {
+  clear_error();
+  if (n_rows < 0 || n_in_rows < 0 || row_bytes < 0 || row_bytes % 4 != 0)
+    return fail(E3_ERR_SHAPE, "bad sizes (row_bytes must be a multiple of 4)");
+  if (n_rows == 0 || row_bytes == 0) return E3_OK;
+  if (perm == nullptr || in == nullptr || out == nullptr) return fail(E3_ERR_INVALID_ARG, "NULL pointer");
+  if ((reinterpret_cast<uintptr_t>(in) & 3u) || (reinterpret_cast<uintptr_t>(out) & 3u))
+    return fail(E3_ERR_INVALID_ARG, "in/out not 4-byte aligned");
+  int* status = nullptr;
+  e3_status st = device_status_ptr(&status);
+  if (st != E3_OK) return st;
+  const bool vec16 = row_bytes % 16 == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+  const int64_t words = row_bytes / 4;
+  const int64_t total = n_rows * (vec16 ? words / 4 : words);
+  const int blocks = int(std::min<int64_t>((total + 255) / 256, 148 * 16));
+  gather_rows_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      n_rows, n_in_rows, words, vec16, perm, static_cast<const uint32_t*>(in), static_cast<uint32_t*>(out), status);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "gather launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}

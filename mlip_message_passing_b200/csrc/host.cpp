@@ -1,0 +1,687 @@
+// Host side of the library: irreps strings, instruction validation, the Clebsch-Gordan table
+// (ladder construction), plans, and argument checking for every C-ABI entry point that
+// launches work.  No CUDA kernels live here.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <complex>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "cg_pattern.h"
+#include "internal.h"
+
+namespace e3b {
+
+// ------------------------------------------------------------------------- errors ---
+static thread_local std::string g_last_error;
+
+e3_status fail(e3_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+void clear_error() { g_last_error.clear(); }
+
+// ------------------------------------------------------------------ irreps strings ---
+// e3nn course, "Curriculum at a glance", lesson 02a: terms "<mul>x<l><p>" joined by '+';
+// a bare "<l><p>" has multiplicity 1.
+struct IrrepT {
+  int mul, l, p;
+};
+
+static bool parse_irreps(const char* s, std::vector<IrrepT>* out, std::string* why) {
+  out->clear();
+  if (s == nullptr) {
+    *why = "NULL irreps string";
+    return false;
+  }
+  const char* c = s;
+  auto skip = [&] {
+    while (*c == ' ' || *c == '\t') ++c;
+  };
+  skip();
+  if (*c == '\0') {
+    *why = "empty irreps string";
+    return false;
+  }
+  while (true) {
+    skip();
+    long a = -1, b = -1;
+    if (*c < '0' || *c > '9') {
+      *why = std::string("expected a digit at '") + c + "'";
+      return false;
+    }
+    a = 0;
+    while (*c >= '0' && *c <= '9') {
+      a = a * 10 + (*c - '0');
+      if (a > 1000000) {
+        *why = "number too large";
+        return false;
+      }
+      ++c;
+    }
+    skip();
+    if (*c == 'x') {
+      ++c;
+      skip();
+      if (*c < '0' || *c > '9') {
+        *why = std::string("expected a degree after 'x' at '") + c + "'";
+        return false;
+      }
+      b = 0;
+      while (*c >= '0' && *c <= '9') {
+        b = b * 10 + (*c - '0');
+        if (b > 1000) {
+          *why = "degree too large";
+          return false;
+        }
+        ++c;
+      }
+    } else {
+      b = a;
+      a = 1;
+    }
+    if (*c != 'e' && *c != 'o') {
+      *why = std::string("expected parity 'e' or 'o' at '") + c + "'";
+      return false;
+    }
+    if (a <= 0) {
+      *why = "multiplicity must be positive";
+      return false;
+    }
+    out->push_back({int(a), int(b), *c == 'e' ? 1 : -1});
+    ++c;
+    skip();
+    if (*c == '\0') break;
+    if (*c != '+') {
+      *why = std::string("expected '+' at '") + c + "'";
+      return false;
+    }
+    ++c;
+  }
+  return true;
+}
+
+static std::string irreps_to_string(const std::vector<IrrepT>& v) {
+  std::string s;
+  for (size_t i = 0; i < v.size(); ++i) {
+    if (i) s += "+";
+    s += std::to_string(v[i].mul) + "x" + std::to_string(v[i].l) + (v[i].p > 0 ? "e" : "o");
+  }
+  return s;
+}
+
+// ------------------------------------------------------ CG: the ladder construction ---
+// E3J, section G.2: the top-spin vector |l3, l3> of V_l1 (x) V_l2 solves J+ v = 0 restricted
+// to m1 + m2 = l3, a two-term (triangular) recurrence; the lower vectors follow by applying
+// J- = J1- + J2- and normalising.  The standard angular-momentum matrix elements are
+//   J+ |j m> = sqrt(j(j+1) - m(m+1)) |j m+1>,   J- |j m> = sqrt(j(j+1) - m(m-1)) |j m-1>.
+// The complex-basis result is then moved to the real basis of the harmonics (the same change
+// of basis that defines the real harmonics from the complex ones), normalised to Frobenius
+// norm 1 and given the sign of the library convention (see e3b.h).
+
+static double jp(int j, int m) { return std::sqrt(double(j * (j + 1) - m * (m + 1))); }
+static double jm(int j, int m) { return std::sqrt(double(j * (j + 1) - m * (m - 1))); }
+
+// cc[(m1+l1)][(m2+l2)][(m3+l3)]: coefficient of |m1>|m2> in |l3 m3>, Condon-Shortley phase.
+static std::vector<double> complex_cg_ladder(int l1, int l2, int l3) {
+  const int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1;
+  std::vector<double> cc(size_t(d1) * d2 * d3, 0.0);
+  auto at = [&](int m1, int m2, int m3) -> double& {
+    return cc[(size_t(m1 + l1) * d2 + (m2 + l2)) * d3 + (m3 + l3)];
+  };
+  // top state: a[m1] with m2 = l3 - m1; a_{m1+1} = -a_{m1} jp(l1, m1) / jp(l2, l3 - m1 - 1)
+  const int lo = std::max(-l1, l3 - l2), hi = std::min(l1, l3 + l2);
+  std::vector<double> a(size_t(hi - lo + 1), 0.0);
+  a[0] = 1.0;
+  for (int m1 = lo; m1 < hi; ++m1) a[m1 + 1 - lo] = -a[m1 - lo] * jp(l1, m1) / jp(l2, l3 - m1 - 1);
+  double nrm = 0.0;
+  for (double v : a) nrm += v * v;
+  nrm = std::sqrt(nrm);
+  const double sgn = a[hi - lo] >= 0 ? 1.0 : -1.0;  // <l1 l1; l2 l3-l1 | l3 l3> > 0
+  for (int m1 = lo; m1 <= hi; ++m1) at(m1, l3 - m1, l3) = sgn * a[m1 - lo] / nrm;
+  // lowering
+  for (int m3 = l3; m3 > -l3; --m3) {
+    const double inv = 1.0 / jm(l3, m3);
+    for (int m1 = -l1; m1 <= l1; ++m1)
+      for (int m2 = -l2; m2 <= l2; ++m2) {
+        const double v = at(m1, m2, m3);
+        if (v == 0.0) continue;
+        if (m1 > -l1) at(m1 - 1, m2, m3 - 1) += v * jm(l1, m1) * inv;
+        if (m2 > -l2) at(m1, m2 - 1, m3 - 1) += v * jm(l2, m2) * inv;
+      }
+  }
+  return cc;
+}
+
+// U with Y_real = U Y_complex for the real harmonics of e3b.h (m>0: cos, m<0: sin, no
+// Condon-Shortley phase), rows real m, columns complex m.
+static std::vector<std::complex<double>> real_from_complex(int l) {
+  const int d = 2 * l + 1;
+  std::vector<std::complex<double>> U(size_t(d) * d, 0.0);
+  const double r = 1.0 / std::sqrt(2.0);
+  for (int m = -l; m <= l; ++m) {
+    auto u = [&](int mc) -> std::complex<double>& { return U[size_t(m + l) * d + (mc + l)]; };
+    if (m > 0) {
+      u(-m) = r;
+      u(m) = ((m & 1) ? -r : r);
+    } else if (m == 0) {
+      u(0) = 1.0;
+    } else {
+      const int k = -m;
+      u(-k) = std::complex<double>(0.0, r);
+      u(k) = std::complex<double>(0.0, (k & 1) ? r : -r);
+    }
+  }
+  return U;
+}
+
+std::vector<double> real_cg_ladder(int l1, int l2, int l3) {
+  const int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1;
+  const std::vector<double> cc = complex_cg_ladder(l1, l2, l3);
+  const auto U1 = real_from_complex(l1), U2 = real_from_complex(l2), U3 = real_from_complex(l3);
+  // C_R[i][j][k] = sum conj(U1[i][a]) conj(U2[j][b]) U3[k][c] cc[a][b][c]
+  std::vector<std::complex<double>> cr(size_t(d1) * d2 * d3, 0.0);
+  for (int i = 0; i < d1; ++i)
+    for (int j = 0; j < d2; ++j)
+      for (int k = 0; k < d3; ++k) {
+        std::complex<double> s = 0.0;
+        for (int a = 0; a < d1; ++a) {
+          const auto u1 = std::conj(U1[size_t(i) * d1 + a]);
+          if (u1 == 0.0) continue;
+          for (int b = 0; b < d2; ++b) {
+            const auto u2 = std::conj(U2[size_t(j) * d2 + b]);
+            if (u2 == 0.0) continue;
+            for (int c = 0; c < d3; ++c) {
+              const double v = cc[(size_t(a) * d2 + b) * d3 + c];
+              if (v == 0.0) continue;
+              s += u1 * u2 * U3[size_t(k) * d3 + c] * v;
+            }
+          }
+        }
+        cr[(size_t(i) * d2 + j) * d3 + k] = s;
+      }
+  double re = 0.0, im = 0.0;
+  for (const auto& z : cr) {
+    re = std::max(re, std::fabs(z.real()));
+    im = std::max(im, std::fabs(z.imag()));
+  }
+  const bool use_re = re >= im;
+  std::vector<double> t(cr.size());
+  double nrm = 0.0;
+  for (size_t q = 0; q < cr.size(); ++q) {
+    t[q] = use_re ? cr[q].real() : cr[q].imag();
+    nrm += t[q] * t[q];
+  }
+  nrm = std::sqrt(nrm);
+  for (double& v : t) v /= nrm;
+  double ref = 0.0;
+  if (((l1 + l2 + l3) & 1) == 0) {
+    ref = t[(size_t(l1) * d2 + l2) * d3 + l3];
+  } else {
+    for (double v : t)
+      if (std::fabs(v) > 1e-12) {
+        ref = v;
+        break;
+      }
+  }
+  if (ref < 0)
+    for (double& v : t) v = -v;
+  for (double& v : t)
+    if (std::fabs(v) < 1e-15) v = 0.0;
+  return t;
+}
+
+const std::vector<double>& packed_cg_table() {
+  static std::vector<double> table;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    table.assign(CG_TABLE_SIZE, 0.0);
+    for (int l1 = 0; l1 <= E3_LMAX; ++l1)
+      for (int l2 = 0; l2 <= E3_LMAX; ++l2)
+        for (int l3 = 0; l3 <= E3_LMAX; ++l3) {
+          if (!triangle(l1, l2, l3)) continue;
+          const auto t = real_cg_ladder(l1, l2, l3);
+          const int d2 = 2 * l2 + 1, d3 = 2 * l3 + 1;
+          for (int m1 = -l1; m1 <= l1; ++m1)
+            for (int m2 = -l2; m2 <= l2; ++m2)
+              for (int m3 = -l3; m3 <= l3; ++m3) {
+                const double v = t[(size_t(m1 + l1) * d2 + (m2 + l2)) * d3 + (m3 + l3)];
+                const int idx = cg_index(l1, l2, l3, m1, m2, m3);
+                if (idx >= 0) {
+                  table[idx] = v;
+                } else if (std::fabs(v) > 1e-12) {
+                  // the selection rules of cg_pattern.h would be wrong; never expected
+                  std::fprintf(stderr, "e3b: CG entry outside pattern (%d %d %d | %d %d %d) = %g\n",
+                               l1, l2, l3, m1, m2, m3, v);
+                }
+              }
+        }
+  });
+  return table;
+}
+
+// ------------------------------------------------------------- compiled path sets ---
+static const int kSupported[][3] = {{1, 1, 2}, {1, 2, 2}, {2, 3, 2}, {3, 3, 3}};
+
+bool degrees_supported(int LX, int LY, int LO) {
+  for (const auto& s : kSupported)
+    if (s[0] == LX && s[1] == LY && s[2] == LO) return true;
+  return false;
+}
+
+const char* supported_list() {
+  static std::string s;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    for (const auto& t : kSupported) {
+      if (!s.empty()) s += " ";
+      s += std::to_string(t[0]) + "," + std::to_string(t[1]) + "," + std::to_string(t[2]);
+    }
+  });
+  return s.c_str();
+}
+
+}  // namespace e3b
+
+using namespace e3b;
+
+// ===================================================================== C ABI: plans ===
+
+extern "C" const char* e3_last_error(void) { return e3b::g_last_error.c_str(); }
+
+extern "C" const char* e3_supported(void) { return supported_list(); }
+
+extern "C" e3_status e3_cg_dense(int32_t l1, int32_t l2, int32_t l3, double* out) {
+  clear_error();
+  if (out == nullptr) return fail(E3_ERR_INVALID_ARG, "e3_cg_dense: out is NULL");
+  if (l1 < 0 || l2 < 0 || l3 < 0 || l1 > E3_LMAX || l2 > E3_LMAX || l3 > E3_LMAX)
+    return fail(E3_ERR_UNSUPPORTED, "e3_cg_dense: degrees must lie in [0, %d]", E3_LMAX);
+  if (!triangle(l1, l2, l3)) return fail(E3_ERR_INSTRUCTION, "e3_cg_dense: triangle rule violated");
+  const auto t = real_cg_ladder(l1, l2, l3);
+  std::memcpy(out, t.data(), t.size() * sizeof(double));
+  return E3_OK;
+}
+
+extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_in2,
+                                    const char* irreps_out, const e3_instruction* instr,
+                                    int32_t n_instr, e3_mode mode, e3_dtype dtype,
+                                    e3_weight_mode wmode, e3_plan** plan_out) {
+  clear_error();
+  if (plan_out == nullptr) return fail(E3_ERR_INVALID_ARG, "plan output pointer is NULL");
+  *plan_out = nullptr;
+  if (dtype != E3_F32 && dtype != E3_F64) return fail(E3_ERR_INVALID_ARG, "bad dtype %d", int(dtype));
+  if (wmode != E3_W_PER_SAMPLE && wmode != E3_W_SHARED)
+    return fail(E3_ERR_INVALID_ARG, "bad weight mode %d", int(wmode));
+  if (mode != E3_UVU && mode != E3_UVW && mode != E3_UUU && mode != E3_UUW)
+    return fail(E3_ERR_INVALID_ARG, "bad connection mode %d", int(mode));
+  if (n_instr < 0 || (n_instr > 0 && instr == nullptr))
+    return fail(E3_ERR_INVALID_ARG, "bad instruction list");
+
+  std::vector<IrrepT> ir1, ir2, irf;
+  std::string why;
+  if (!parse_irreps(irreps_in1, &ir1, &why)) return fail(E3_ERR_IRREPS_PARSE, "irreps_in1: %s", why.c_str());
+  if (!parse_irreps(irreps_in2, &ir2, &why)) return fail(E3_ERR_IRREPS_PARSE, "irreps_in2: %s", why.c_str());
+  const bool have_out = irreps_out != nullptr && irreps_out[strspn(irreps_out, " \t")] != '\0';
+  if (have_out && !parse_irreps(irreps_out, &irf, &why))
+    return fail(E3_ERR_IRREPS_PARSE, "irreps_out: %s", why.c_str());
+  if (n_instr > 0 && !have_out)
+    return fail(E3_ERR_INSTRUCTION, "explicit instructions need irreps_out");
+
+  // instructions: (i1, i2, i_out, alpha_override); output irreps
+  struct Ins {
+    int i1, i2, io;
+    double pw;
+  };
+  std::vector<Ins> ins;
+  std::vector<IrrepT> out_irreps;
+  if (n_instr == 0) {
+    for (int i1 = 0; i1 < int(ir1.size()); ++i1)
+      for (int i2 = 0; i2 < int(ir2.size()); ++i2) {
+        const auto &a = ir1[i1], &b = ir2[i2];
+        for (int l3 = std::abs(a.l - b.l); l3 <= a.l + b.l; ++l3) {
+          const int p3 = a.p * b.p;
+          bool ok = !have_out;
+          for (const auto& f : irf) ok = ok || (f.l == l3 && f.p == p3);
+          if (!ok) continue;
+          ins.push_back({i1, i2, int(out_irreps.size()), -1.0});
+          out_irreps.push_back({a.mul, l3, p3});  // uvu: output channel u of x
+        }
+      }
+    if (ins.empty()) return fail(E3_ERR_INSTRUCTION, "no allowed path between the inputs and the output filter");
+  } else {
+    out_irreps = irf;
+    for (int q = 0; q < n_instr; ++q) {
+      const auto& s = instr[q];
+      if (s.i_in1 < 0 || s.i_in1 >= int(ir1.size()) || s.i_in2 < 0 || s.i_in2 >= int(ir2.size()) ||
+          s.i_out < 0 || s.i_out >= int(out_irreps.size()))
+        return fail(E3_ERR_INSTRUCTION, "instruction %d: index out of range", q);
+      const auto &a = ir1[s.i_in1], &b = ir2[s.i_in2], &c = out_irreps[s.i_out];
+      if (!triangle(a.l, b.l, c.l))
+        return fail(E3_ERR_INSTRUCTION, "instruction %d: triangle rule |l1-l2| <= l3 <= l1+l2 fails (%d,%d,%d)",
+                    q, a.l, b.l, c.l);
+      if (c.p != a.p * b.p)
+        return fail(E3_ERR_INSTRUCTION, "instruction %d: parity rule p3 = p1 p2 fails", q);
+      if (mode == E3_UVU && c.mul != a.mul)
+        return fail(E3_ERR_INSTRUCTION, "instruction %d: uvu needs mul_out == mul_in1", q);
+      if (!s.has_weight)
+        return fail(E3_ERR_UNSUPPORTED, "instruction %d: paths without weights have no kernel", q);
+      ins.push_back({s.i_in1, s.i_in2, s.i_out, s.path_weight});
+    }
+  }
+  if (mode != E3_UVU) return fail(E3_ERR_UNSUPPORTED, "only the uvu connection mode has kernels");
+
+  // layout the kernels are compiled for
+  const int C = ir1[0].mul;
+  for (int i = 0; i < int(ir1.size()); ++i)
+    if (ir1[i].l != i || ir1[i].mul != C)
+      return fail(E3_ERR_UNSUPPORTED,
+                  "irreps_in1 must be Cx0+Cx1+..+CxLx (one block per degree, ascending, common multiplicity)");
+  for (int i = 0; i < int(ir2.size()); ++i)
+    if (ir2[i].l != i || ir2[i].mul != 1)
+      return fail(E3_ERR_UNSUPPORTED, "irreps_in2 must be 1x0+1x1+..+1xLy");
+  const int LX = int(ir1.size()) - 1, LY = int(ir2.size()) - 1;
+  if (C % 4 != 0 || !((C / 4) <= 32 ? (32 % (C / 4) == 0) : ((C / 4) % 32 == 0)))
+    return fail(E3_ERR_UNSUPPORTED, "multiplicity %d: kernels need C in {4, 8, 16, 32, 64} or a multiple of 128", C);
+  int LO = 0;
+  for (const auto& s : ins) LO = std::max(LO, out_irreps[s.io].l);
+  if (LX > E3_LMAX || LY > E3_LMAX || LO > E3_LMAX)
+    return fail(E3_ERR_UNSUPPORTED, "degrees above %d have no kernel", E3_LMAX);
+  // the instruction list must be the full enumeration for (LX, LY, LO), uncollapsed, with
+  // output blocks in instruction order
+  const int P = n_paths(LX, LY, LO);
+  bool same = int(ins.size()) == P && int(out_irreps.size()) == P;
+  for (int p = 0; same && p < P; ++p) {
+    same = ir1[ins[p].i1].l == path_l(LX, LY, LO, p, 0) && ir2[ins[p].i2].l == path_l(LX, LY, LO, p, 1) &&
+           out_irreps[ins[p].io].l == path_l(LX, LY, LO, p, 2) && ins[p].io == p;
+  }
+  if (!same)
+    return fail(E3_ERR_UNSUPPORTED,
+                "kernels need every path with l3 <= %d, one output block per instruction in order", LO);
+  if (!degrees_supported(LX, LY, LO))
+    return fail(E3_ERR_UNSUPPORTED, "(Lx, Ly, Lo) = (%d, %d, %d) is not compiled; compiled: %s", LX, LY, LO,
+                supported_list());
+
+  auto* plan = new (std::nothrow) e3_plan();
+  if (plan == nullptr) return fail(E3_ERR_INVALID_ARG, "out of host memory");
+  if (cudaGetDevice(&plan->device) != cudaSuccess) {
+    delete plan;
+    return fail(E3_ERR_CUDA, "cudaGetDevice failed");
+  }
+  plan->dtype = dtype;
+  plan->wmode = wmode;
+  plan->C = C;
+  plan->LX = LX;
+  plan->LY = LY;
+  plan->LO = LO;
+  plan->n_paths = P;
+  std::vector<int> n_out(out_irreps.size(), 0);
+  for (const auto& s : ins) n_out[s.io] += 1;
+  for (int p = 0; p < P; ++p) {
+    const auto &b = ir2[ins[p].i2], &c = out_irreps[ins[p].io];
+    plan->l1.push_back(ir1[ins[p].i1].l);
+    plan->l2.push_back(b.l);
+    plan->l3.push_back(c.l);
+    plan->alpha.push_back(ins[p].pw >= 0 ? ins[p].pw : std::sqrt((2.0 * c.l + 1.0) / (b.mul * n_out[ins[p].io])));
+  }
+  for (const auto& a : ir1) plan->dim1 += int64_t(a.mul) * (2 * a.l + 1);
+  for (const auto& b : ir2) plan->dim2 += int64_t(b.mul) * (2 * b.l + 1);
+  for (const auto& c : out_irreps) plan->dim_out += int64_t(c.mul) * (2 * c.l + 1);
+  plan->weight_numel = int64_t(P) * C;
+  plan->irreps_out = irreps_to_string(out_irreps);
+  packed_cg_table();
+  const e3_status st = ensure_device_tables();
+  if (st != E3_OK) {
+    delete plan;
+    return st;
+  }
+  *plan_out = plan;
+  return E3_OK;
+}
+
+extern "C" e3_status e3_plan_destroy(e3_plan* plan) {
+  clear_error();
+  delete plan;
+  return E3_OK;
+}
+
+extern "C" e3_status e3_plan_info(const e3_plan* plan, int64_t* dim_in1, int64_t* dim_in2, int64_t* dim_out,
+                                  int64_t* weight_numel, int32_t* n_paths_out) {
+  clear_error();
+  if (plan == nullptr) return fail(E3_ERR_INVALID_ARG, "plan is NULL");
+  if (dim_in1) *dim_in1 = plan->dim1;
+  if (dim_in2) *dim_in2 = plan->dim2;
+  if (dim_out) *dim_out = plan->dim_out;
+  if (weight_numel) *weight_numel = plan->weight_numel;
+  if (n_paths_out) *n_paths_out = plan->n_paths;
+  return E3_OK;
+}
+
+extern "C" e3_status e3_plan_irreps_out(const e3_plan* plan, char* buf, size_t buf_len, size_t* needed) {
+  clear_error();
+  if (plan == nullptr) return fail(E3_ERR_INVALID_ARG, "plan is NULL");
+  const size_t n = plan->irreps_out.size() + 1;
+  if (needed) *needed = n;
+  if (buf != nullptr) {
+    if (buf_len < n) return fail(E3_ERR_SHAPE, "buffer of %zu bytes, need %zu", buf_len, n);
+    std::memcpy(buf, plan->irreps_out.c_str(), n);
+  }
+  return E3_OK;
+}
+
+extern "C" e3_status e3_plan_paths(const e3_plan* plan, int32_t* lls, double* alpha) {
+  clear_error();
+  if (plan == nullptr) return fail(E3_ERR_INVALID_ARG, "plan is NULL");
+  for (int p = 0; p < plan->n_paths; ++p) {
+    if (lls) {
+      lls[3 * p] = plan->l1[p];
+      lls[3 * p + 1] = plan->l2[p];
+      lls[3 * p + 2] = plan->l3[p];
+    }
+    if (alpha) alpha[p] = plan->alpha[p];
+  }
+  return E3_OK;
+}
+
+extern "C" e3_status e3_device_status(void* stream) {
+  clear_error();
+  int* d = nullptr;
+  e3_status st = device_status_ptr(&d);
+  if (st != E3_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  if (cudaMemcpyAsync(&h, d, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemsetAsync(d, 0, sizeof(int), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+    return fail(E3_ERR_CUDA, "reading the device status word failed: %s", cudaGetErrorString(cudaGetLastError()));
+  if (h == E3_OK) return E3_OK;
+  return fail(static_cast<e3_status>(h), "device reported %s",
+              h == E3_ERR_INDEX ? "an index out of range" : (h == E3_ERR_TIMEOUT ? "a wait that gave up" : "an error"));
+}
+
+// ========================================================= C ABI: compute entry points ===
+
+static bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+static e3_status check_plan_device(const e3_plan* plan) {
+  if (plan == nullptr) return fail(E3_ERR_INVALID_ARG, "plan is NULL");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(E3_ERR_CUDA, "cudaGetDevice failed");
+  if (dev != plan->device)
+    return fail(E3_ERR_INVALID_ARG, "plan belongs to device %d but device %d is current", plan->device, dev);
+  return E3_OK;
+}
+
+#define E3_REQ(ptr, name)                                                        \
+  do {                                                                           \
+    if ((ptr) == nullptr) return fail(E3_ERR_INVALID_ARG, "%s is NULL", name);   \
+    if (misaligned(ptr)) return fail(E3_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+  } while (0)
+#define E3_OPT(ptr, name)                                                        \
+  do {                                                                           \
+    if ((ptr) != nullptr && misaligned(ptr))                                     \
+      return fail(E3_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);        \
+  } while (0)
+
+extern "C" e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x, const void* y, const void* w,
+                                   void* out, void* stream) {
+  clear_error();
+  e3_status st = check_plan_device(plan);
+  if (st != E3_OK) return st;
+  if (B < 0 || B >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "B = %lld out of range", (long long)B);
+  if (B == 0) return E3_OK;
+  E3_REQ(x, "x");
+  E3_REQ(y, "y");
+  E3_REQ(w, "w");
+  E3_REQ(out, "out");
+  FwdArgs a{};
+  a.n_rows = B;
+  a.x = x;
+  a.y = y;
+  a.vec = nullptr;
+  a.sh_norm = E3_SH_COMPONENT;
+  a.w = w;
+  a.w_stride = plan->wmode == E3_W_SHARED ? 0 : plan->weight_numel;
+  a.scale = 1.0;
+  a.out = out;
+  a.stream = stream;
+  return launch_forward(plan, a, false);
+}
+
+extern "C" e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* x, const void* y, const void* w,
+                                    const void* grad_out, void* grad_x, void* grad_y, void* grad_w,
+                                    void* stream) {
+  clear_error();
+  e3_status st = check_plan_device(plan);
+  if (st != E3_OK) return st;
+  if (plan->wmode == E3_W_SHARED) return fail(E3_ERR_UNSUPPORTED, "backward with shared weights has no kernel");
+  if (B < 0 || B >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "B = %lld out of range", (long long)B);
+  if (B == 0) return E3_OK;
+  E3_REQ(x, "x");
+  E3_REQ(y, "y");
+  E3_REQ(w, "w");
+  E3_REQ(grad_out, "grad_out");
+  E3_OPT(grad_x, "grad_x");
+  E3_OPT(grad_y, "grad_y");
+  E3_OPT(grad_w, "grad_w");
+  if (!grad_x && !grad_y && !grad_w) return E3_OK;
+  BwdArgs a{};
+  a.n_nodes = B;
+  a.n_edges = B;
+  a.x = x;
+  a.y = y;
+  a.sh_norm = E3_SH_COMPONENT;
+  a.w = w;
+  a.grad_out = grad_out;
+  a.scale = 1.0;
+  a.grad_x = grad_x;
+  a.grad_y = grad_y;
+  a.grad_w = grad_w;
+  a.stream = stream;
+  return launch_backward(plan, a, false);
+}
+
+static e3_status check_conv_common(const e3_plan* plan, int64_t N, int64_t E, const void* y, const void* vec,
+                                   e3_sh_norm sh_norm) {
+  if (N < 0 || N >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N = %lld out of range", (long long)N);
+  if (E < 0 || E >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "E = %lld out of range", (long long)E);
+  if ((y == nullptr) == (vec == nullptr)) return fail(E3_ERR_INVALID_ARG, "give exactly one of y and edge_vec");
+  if (vec != nullptr && (sh_norm < E3_SH_COMPONENT || sh_norm > E3_SH_NORM))
+    return fail(E3_ERR_INVALID_ARG, "bad sh_norm %d", int(sh_norm));
+  if (vec != nullptr && (reinterpret_cast<uintptr_t>(vec) % (plan->dtype == E3_F64 ? 8 : 4)) != 0)
+    return fail(E3_ERR_INVALID_ARG, "edge_vec is not aligned to its element size");
+  return E3_OK;
+}
+
+extern "C" e3_status e3_conv_forward(const e3_plan* plan, int64_t N, int64_t E, const int32_t* row_ptr_dst,
+                                     const int32_t* src, const void* x, const void* y, const void* edge_vec,
+                                     e3_sh_norm sh_norm, const void* w, double out_scale, void* out,
+                                     void* stream) {
+  clear_error();
+  e3_status st = check_plan_device(plan);
+  if (st != E3_OK) return st;
+  st = check_conv_common(plan, N, E, y, edge_vec, sh_norm);
+  if (st != E3_OK) return st;
+  if (N == 0) return E3_OK;
+  E3_REQ(out, "out");
+  if (row_ptr_dst == nullptr) return fail(E3_ERR_INVALID_ARG, "row_ptr_dst is NULL");
+  if (E > 0) {
+    E3_REQ(x, "x");
+    E3_REQ(w, "w");
+    E3_OPT(y, "y");
+    if (src == nullptr) return fail(E3_ERR_INVALID_ARG, "src is NULL");
+  }
+  if (!std::isfinite(out_scale)) return fail(E3_ERR_INVALID_ARG, "out_scale is not finite");
+  FwdArgs a{};
+  a.n_rows = N;
+  a.n_edges = E;
+  a.row_ptr = row_ptr_dst;
+  a.src = src;
+  a.x = x;
+  a.y = y;
+  a.vec = edge_vec;
+  a.sh_norm = sh_norm;
+  a.w = w;
+  a.w_stride = plan->wmode == E3_W_SHARED ? 0 : plan->weight_numel;
+  a.scale = out_scale;
+  a.out = out;
+  a.stream = stream;
+  return launch_forward(plan, a, true);
+}
+
+extern "C" e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E, const int32_t* row_ptr_dst,
+                                      const int32_t* src, const int32_t* dst, const int32_t* row_ptr_src,
+                                      const int32_t* perm_src, const void* x, const void* y, const void* edge_vec,
+                                      e3_sh_norm sh_norm, const void* w, const void* grad_out, double out_scale,
+                                      void* grad_x, void* grad_y, void* grad_w, void* stream) {
+  clear_error();
+  (void)row_ptr_dst;
+  (void)src;
+  e3_status st = check_plan_device(plan);
+  if (st != E3_OK) return st;
+  if (plan->wmode == E3_W_SHARED) return fail(E3_ERR_UNSUPPORTED, "backward with shared weights has no kernel");
+  st = check_conv_common(plan, N, E, y, edge_vec, sh_norm);
+  if (st != E3_OK) return st;
+  E3_OPT(grad_x, "grad_x");
+  E3_OPT(grad_y, "grad_y");
+  E3_OPT(grad_w, "grad_w");
+  if (!grad_x && !grad_y && !grad_w) return E3_OK;
+  if (N == 0) return E3_OK;
+  if (row_ptr_src == nullptr) return fail(E3_ERR_INVALID_ARG, "row_ptr_src is NULL");
+  if (E > 0) {
+    E3_REQ(x, "x");
+    E3_REQ(w, "w");
+    E3_REQ(grad_out, "grad_out");
+    E3_OPT(y, "y");
+    if (dst == nullptr || perm_src == nullptr) return fail(E3_ERR_INVALID_ARG, "dst or perm_src is NULL");
+  }
+  if (!std::isfinite(out_scale)) return fail(E3_ERR_INVALID_ARG, "out_scale is not finite");
+  BwdArgs a{};
+  a.n_nodes = N;
+  a.n_edges = E;
+  a.row_ptr_src = row_ptr_src;
+  a.perm_src = perm_src;
+  a.dst = dst;
+  a.x = x;
+  a.y = y;
+  a.vec = edge_vec;
+  a.sh_norm = sh_norm;
+  a.w = w;
+  a.grad_out = grad_out;
+  a.scale = out_scale;
+  a.grad_x = grad_x;
+  a.grad_y = grad_y;
+  a.grad_w = grad_w;
+  a.stream = stream;
+  return launch_backward(plan, a, true);
+}

@@ -1,0 +1,889 @@
+// Kernels for the channelwise ("uvu") Clebsch-Gordan tensor product and the message-passing
+// convolution, forward and backward, for sm_100a.
+//
+// What is computed (e3nn course, "Curriculum at a glance", lessons 03a/03b/06a; E3J, sections
+// E.1 and E.2.2): for an edge e with sender s, receiver n, harmonics Y_e and weights w_e,
+//     msg[p, u, m3] = alpha_p * w[e, p, u] * sum_{m1, m2} C_p[m1, m2, m3] x[s, l1(p), u, m1] Y_e[l2(p), m2]
+//     out[n]        = scale * sum_{e : dst_e = n} msg_e
+// and the transposes of this trilinear map for the backward pass.
+//
+// Work decomposition (B200: FP32 FMA issue is the co-bottleneck with HBM for l <= 3):
+//   * A_p[m1, m3] = sum_m2 C_p[m1, m2, m3] Y[m2] is formed once per edge and path in registers;
+//     the CG values come from __constant__ memory at compile-time offsets, so they enter the
+//     FFMA as constant-bank operands and cost no load instruction.  Only the structural
+//     nonzeros of C and of A are visited (selection rules in cg_pattern.h).
+//   * A thread owns 4 consecutive channels x one compile-time group of paths, so one A entry
+//     feeds 4 FMAs and the accumulators (<= 80) stay in registers.
+//   * Channels are the fastest thread index; when C/4 < 32 the remaining lanes of a warp take
+//     different edges of the same receiver ("slices") and are summed with a fixed butterfly at
+//     the end, so the reduction order is fixed and the result is bitwise repeatable.
+//   * Forward: one CTA per (receiver, path group); the receiver's in-edges are consecutive in
+//     memory (receiver CSR), so the weight rows stream contiguously and x[src] rows are
+//     gathered from L2.  No atomics, no [E, dim_out] message tensor.
+//   * Backward: one CTA per sender with one warp per path group, walking the sender CSR;
+//     A is recomputed, never stored; grad_w and grad_y are edge-local writes; grad_x is
+//     reduced in registers and shared memory in a fixed order.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <type_traits>
+
+#include "cg_pattern.h"
+#include "internal.h"
+
+namespace e3b {
+
+// Each translation unit that includes this header gets its own copy of the coefficient
+// tables (internal linkage); upload_tables() fills the copy of the including unit.
+static __constant__ float c_cg32[CG_TABLE_SIZE];
+static __constant__ double c_cg64[CG_TABLE_SIZE];
+
+constexpr int MAXP = 64;  // paths per plan (34 at l <= 3)
+constexpr int K = 4;      // channels per thread
+
+template <typename T>
+struct CGT;
+template <>
+struct CGT<float> {
+  template <int I>
+  static __device__ __forceinline__ float get() {
+    static_assert(I >= 0 && I < CG_TABLE_SIZE, "CG index");
+    return c_cg32[I];
+  }
+};
+template <>
+struct CGT<double> {
+  template <int I>
+  static __device__ __forceinline__ double get() {
+    static_assert(I >= 0 && I < CG_TABLE_SIZE, "CG index");
+    return c_cg64[I];
+  }
+};
+
+template <int B, int E, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (B < E) {
+    f(std::integral_constant<int, B>());
+    static_for<B + 1, E>(f);
+  }
+}
+
+template <int N, int I = 0, typename F>
+__device__ __forceinline__ void dispatch(int g, F&& f) {
+  if constexpr (I < N) {
+    if (g == I)
+      f(std::integral_constant<int, I>());
+    else
+      dispatch<N, I + 1>(g, f);
+  }
+}
+
+__device__ __forceinline__ void record_error(int* status, int code) { atomicCAS(status, 0, code); }
+
+__device__ __forceinline__ float rsqrt_t(float v) { return rsqrtf(v); }
+__device__ __forceinline__ double rsqrt_t(double v) { return rsqrt(v); }
+
+// --------------------------------------------------------------------- configuration ---
+template <int LX_, int LY_, int LO_, typename T_>
+struct Cfg {
+  static constexpr int LX = LX_, LY = LY_, LO = LO_;
+  using T = T_;
+  static constexpr int P = n_paths(LX, LY, LO);
+  static constexpr int G = n_groups(LX, LY, LO);
+  static constexpr int NY = (LY + 1) * (LY + 1);
+  static constexpr int NX = (LX + 1) * (LX + 1);
+  static constexpr int NO = out_dim_per_channel(LX, LY, LO);
+  static_assert(P <= MAXP, "too many paths");
+};
+
+template <class CF, int GI>
+struct Grp {
+  static constexpr int LX = CF::LX, LY = CF::LY, LO = CF::LO;
+  static constexpr int PB = group_begin(LX, LY, LO, GI);
+  static constexpr int PE = group_begin(LX, LY, LO, GI + 1);
+  static constexpr int NP = PE - PB;
+  static_assert(NP >= 1, "empty path group");
+  static constexpr int L1A = path_l(LX, LY, LO, PB, 0);
+  static constexpr int L1B = path_l(LX, LY, LO, PE - 1, 0);
+  static constexpr int XB = L1A * L1A;                    // first per-channel x index used
+  static constexpr int NXG = (L1B + 1) * (L1B + 1) - XB;  // per-channel x values used
+  static constexpr int OB = path_out_off(LX, LY, LO, PB);
+  static constexpr int NOG = path_out_off(LX, LY, LO, PE) - OB;
+};
+
+template <class CF, int P>
+struct PathC {
+  static constexpr int L1 = path_l(CF::LX, CF::LY, CF::LO, P, 0);
+  static constexpr int L2 = path_l(CF::LX, CF::LY, CF::LO, P, 1);
+  static constexpr int L3 = path_l(CF::LX, CF::LY, CF::LO, P, 2);
+  static constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1;
+  static constexpr int OUT = path_out_off(CF::LX, CF::LY, CF::LO, P);  // per-channel offset
+};
+
+// A_p[m1, m3] for one (m1, m3): sum over the pattern m2 of C[m1, m2, m3] * Y[l2, m2].
+template <typename T, int L1, int L2, int L3, int M1, int M3, int NY>
+__device__ __forceinline__ T a_entry(const T (&Y)[NY]) {
+  T v = T(0);
+  static_for<-L2, L2 + 1>([&](auto m2c) {
+    constexpr int M2 = decltype(m2c)::value;
+    if constexpr (cg_nz(L1, L2, L3, M1, M2, M3)) {
+      constexpr int I = cg_index(L1, L2, L3, M1, M2, M3);
+      v = fma(CGT<T>::template get<I>(), Y[L2 * L2 + L2 + M2], v);
+    }
+  });
+  return v;
+}
+
+// ----------------------------------------------------------------- memory helpers ---
+// 16-byte vector moves between global memory and register arrays.
+template <typename T, int N>
+__device__ __forceinline__ void ld16(T (&r)[N], const T* __restrict__ p, bool stream) {
+  if constexpr (std::is_same<T, float>::value) {
+    static_assert(N % 4 == 0, "float chunk");
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const float4 v = stream ? __ldcs(reinterpret_cast<const float4*>(p) + i)
+                              : __ldg(reinterpret_cast<const float4*>(p) + i);
+      r[4 * i] = v.x;
+      r[4 * i + 1] = v.y;
+      r[4 * i + 2] = v.z;
+      r[4 * i + 3] = v.w;
+    }
+  } else {
+    static_assert(N % 2 == 0, "double chunk");
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const double2 v = stream ? __ldcs(reinterpret_cast<const double2*>(p) + i)
+                               : __ldg(reinterpret_cast<const double2*>(p) + i);
+      r[2 * i] = v.x;
+      r[2 * i + 1] = v.y;
+    }
+  }
+}
+
+template <typename T, int N>
+__device__ __forceinline__ void st16(T* __restrict__ p, const T (&r)[N]) {
+  if constexpr (std::is_same<T, float>::value) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i)
+      __stcs(reinterpret_cast<float4*>(p) + i, make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) __stcs(reinterpret_cast<double2*>(p) + i, make_double2(r[2 * i], r[2 * i + 1]));
+  }
+}
+
+// x values of the group's degree range for channels 4cb..4cb+3 of row `row`:
+// xr[k][j] = x[row, block l, channel 4cb+k, m] with j = l*l + (m + l) - XB.
+template <class CF, class GR, typename T>
+__device__ __forceinline__ void load_x(T (&xr)[K][GR::NXG], const T* __restrict__ xrow, int C, int cb) {
+  static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
+    constexpr int L = decltype(lc)::value;
+    constexpr int D = 2 * L + 1;
+    T t[K * D];
+    ld16(t, xrow + size_t(C) * (L * L) + size_t(4 * cb) * D, false);
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+#pragma unroll
+      for (int m = 0; m < D; ++m) xr[k][L * L - GR::XB + m] = t[k * D + m];
+  });
+}
+
+// weights of the group's paths for channels 4cb..4cb+3: wr[k][q] = w[row, PB + q, 4cb + k]
+template <class GR, typename T>
+__device__ __forceinline__ void load_w(T (&wr)[K][GR::NP], const T* __restrict__ wrow, int C, int cb) {
+#pragma unroll
+  for (int q = 0; q < GR::NP; ++q) {
+    T t[K];
+    ld16(t, wrow + size_t(GR::PB + q) * C + 4 * cb, true);
+#pragma unroll
+    for (int k = 0; k < K; ++k) wr[k][q] = t[k];
+  }
+}
+
+// ------------------------------------------------------------ spherical harmonics ---
+// Real harmonics, component normalisation (sum_m Y_lm^2 = 2l+1 on the unit sphere), m = -l..l,
+// z the pole, no Condon-Shortley phase (e3nn course, lesson 02b).  Polynomials in the unit
+// vector (x, y, z); r = 0 gives Y^0 = 1 and zero for l > 0.
+template <int LY, typename T>
+__device__ __forceinline__ void sh_eval(T vx, T vy, T vz, int norm, T (&Y)[(LY + 1) * (LY + 1)]) {
+  Y[0] = T(1);
+  if constexpr (LY >= 1) {
+    const T r2 = vx * vx + vy * vy + vz * vz;
+    const T inv = r2 > T(0) ? rsqrt_t(r2) : T(0);
+    const T x = vx * inv, y = vy * inv, z = vz * inv;
+    const T s3 = T(1.7320508075688772935);
+    Y[1] = s3 * y;
+    Y[2] = s3 * z;
+    Y[3] = s3 * x;
+    if constexpr (LY >= 2) {
+      const T s15 = T(3.8729833462074168852), s5h = T(1.1180339887498948482);
+      Y[4] = s15 * x * y;
+      Y[5] = s15 * y * z;
+      Y[6] = s5h * (T(2) * z * z - x * x - y * y);
+      Y[7] = s15 * x * z;
+      Y[8] = T(0.5) * s15 * (x * x - y * y);
+      if constexpr (LY >= 3) {
+        const T c70 = T(2.0916500663351888699);   // sqrt(70)/4
+        const T c105 = T(10.246950765959598383);  // sqrt(105)
+        const T c42 = T(1.6201851746019650147);   // sqrt(42)/4
+        const T c7 = T(1.3228756555322952953);    // sqrt(7)/2
+        const T x2 = x * x, y2 = y * y, z2 = z * z;
+        const T f = T(4) * z2 - x2 - y2;            // 5 z^2 - r^2 on the sphere
+        Y[9] = c70 * y * (T(3) * x2 - y2);
+        Y[10] = c105 * x * y * z;
+        Y[11] = c42 * y * f;
+        Y[12] = c7 * z * (T(2) * z2 - T(3) * x2 - T(3) * y2);
+        Y[13] = c42 * x * f;
+        Y[14] = T(0.5) * c105 * z * (x2 - y2);
+        Y[15] = c70 * x * (x2 - T(3) * y2);
+      }
+    }
+    // zero vector: every l > 0 component is already 0 through inv = 0
+  }
+  if (norm == E3_SH_INTEGRAL) {
+    const T c = T(0.28209479177387814347);  // 1/sqrt(4 pi)
+#pragma unroll
+    for (int i = 0; i < (LY + 1) * (LY + 1); ++i) Y[i] *= c;
+  } else if (norm == E3_SH_NORM) {
+#pragma unroll
+    for (int l = 1; l <= LY; ++l) {
+      const T c = rsqrt_t(T(2 * l + 1));
+#pragma unroll
+      for (int m = 0; m < 2 * l + 1; ++m) Y[l * l + m] *= c;
+    }
+  }
+}
+
+template <class CF, typename T>
+__device__ __forceinline__ void load_y(T (&Y)[CF::NY], const T* __restrict__ y, const T* __restrict__ vec,
+                                       int norm, int64_t e) {
+  if (y != nullptr) {
+#pragma unroll
+    for (int i = 0; i < CF::NY; ++i) Y[i] = __ldg(y + e * CF::NY + i);
+  } else {
+    const T vx = __ldg(vec + 3 * e), vy = __ldg(vec + 3 * e + 1), vz = __ldg(vec + 3 * e + 2);
+    sh_eval<CF::LY, T>(vx, vy, vz, norm, Y);
+  }
+}
+
+// ========================================================================== forward ===
+struct KFwd {
+  const int32_t* row_ptr;
+  const int32_t* src;
+  const void* x;
+  const void* y;
+  const void* vec;
+  const void* w;
+  void* out;
+  int64_t n_rows, n_edges, w_stride;
+  int C, sh_norm, n_chunks;
+  int* status;
+  double pscale[MAXP];  // scale * alpha_p
+};
+
+template <class CF, int GI>
+struct FwdAcc {
+  using T = typename CF::T;
+  using GR = Grp<CF, GI>;
+  T acc[K][GR::NOG];
+
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+#pragma unroll
+      for (int o = 0; o < GR::NOG; ++o) acc[k][o] = T(0);
+  }
+
+  // acc += w (x) A x for one edge
+  __device__ __forceinline__ void edge(const T (&xr)[K][GR::NXG], const T (&wr)[K][GR::NP], const T (&Y)[CF::NY]) {
+    static_for<GR::PB, GR::PE>([&](auto pc) {
+      constexpr int P = decltype(pc)::value;
+      using PC = PathC<CF, P>;
+      constexpr int L1 = PC::L1, L2 = PC::L2, L3 = PC::L3, D1 = PC::D1, D3 = PC::D3;
+      constexpr int XO = L1 * L1 - GR::XB, OO = PC::OUT - GR::OB, PW = P - GR::PB;
+      if constexpr (D1 < D3) {
+        // scale x by the weight first (fewer multiplies), then acc += A^T xs
+        T xs[K][D1];
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+#pragma unroll
+          for (int m1 = 0; m1 < D1; ++m1) xs[k][m1] = wr[k][PW] * xr[k][XO + m1];
+        static_for<0, D3>([&](auto m3c) {
+          constexpr int M3I = decltype(m3c)::value;
+          T a[D1];
+          static_for<0, D1>([&](auto m1c) {
+            constexpr int M1I = decltype(m1c)::value;
+            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3))
+              a[M1I] = a_entry<T, L1, L2, L3, M1I - L1, M3I - L3>(Y);
+          });
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            T t = acc[k][OO + M3I];
+            static_for<0, D1>([&](auto m1c) {
+              constexpr int M1I = decltype(m1c)::value;
+              if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) t = fma(a[M1I], xs[k][M1I], t);
+            });
+            acc[k][OO + M3I] = t;
+          }
+        });
+      } else {
+        // t = A^T x, then acc += w t
+        static_for<0, D3>([&](auto m3c) {
+          constexpr int M3I = decltype(m3c)::value;
+          T a[D1];
+          static_for<0, D1>([&](auto m1c) {
+            constexpr int M1I = decltype(m1c)::value;
+            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3))
+              a[M1I] = a_entry<T, L1, L2, L3, M1I - L1, M3I - L3>(Y);
+          });
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            T t = T(0);
+            static_for<0, D1>([&](auto m1c) {
+              constexpr int M1I = decltype(m1c)::value;
+              if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) t = fma(a[M1I], xr[k][XO + M1I], t);
+            });
+            acc[k][OO + M3I] = fma(wr[k][PW], t, acc[k][OO + M3I]);
+          }
+        });
+      }
+    });
+  }
+
+  // out[row, path blocks of the group, channels 4cb..] = pscale_p * acc
+  __device__ __forceinline__ void store(T* __restrict__ orow, int C, int cb, const double* pscale) {
+    static_for<GR::PB, GR::PE>([&](auto pc) {
+      constexpr int P = decltype(pc)::value;
+      using PC = PathC<CF, P>;
+      constexpr int D3 = PC::D3, OO = PC::OUT - GR::OB;
+      const T s = T(pscale[P]);
+      T t[K * D3];
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int m = 0; m < D3; ++m) t[k * D3 + m] = s * acc[k][OO + m];
+      st16(orow + size_t(C) * PC::OUT + size_t(4 * cb) * D3, t);
+    });
+  }
+};
+
+template <class CF, int GI, bool CONV>
+__device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit) {
+  using T = typename CF::T;
+  using GR = Grp<CF, GI>;
+  const int C = a.C, CB = C >> 2;
+  const int lane = threadIdx.x;
+  const int cb = CB >= 32 ? lane : lane % CB;
+  const int slice = CB >= 32 ? 0 : lane / CB;
+  const int NS = CB >= 32 ? 1 : 32 / CB;
+  const T* __restrict__ x = static_cast<const T*>(a.x);
+  const T* __restrict__ y = static_cast<const T*>(a.y);
+  const T* __restrict__ vec = static_cast<const T*>(a.vec);
+  const T* __restrict__ w = static_cast<const T*>(a.w);
+  T* __restrict__ out = static_cast<T*>(a.out);
+  const size_t xrow = size_t(CF::NX) * C;
+  const size_t orow = size_t(CF::NO) * C;
+
+  FwdAcc<CF, GI> f;
+  T xr[K][GR::NXG], wr[K][GR::NP], Y[CF::NY];
+  if constexpr (CONV) {
+    const int64_t n = unit;
+    int64_t e0 = a.row_ptr[n], e1 = a.row_ptr[n + 1];
+    if (e0 < 0 || e1 < e0 || e1 > a.n_edges) {
+      if (lane == 0) record_error(a.status, E3_ERR_INDEX);
+      e0 = e1 = 0;
+    }
+    f.zero();
+    for (int64_t e = e0 + slice; e < e1; e += NS) {
+      const int32_t s = __ldg(a.src + e);
+      if (uint32_t(s) >= uint32_t(a.n_rows)) {
+        record_error(a.status, E3_ERR_INDEX);
+        continue;
+      }
+      load_w<GR>(wr, w + e * a.w_stride, C, cb);
+      load_x<CF, GR>(xr, x + size_t(s) * xrow, C, cb);
+      load_y<CF>(Y, y, vec, a.sh_norm, e);
+      f.edge(xr, wr, Y);
+    }
+    // sum the slices (lanes cb, cb + CB, ...) in a fixed butterfly order
+    if (CB < 32) {
+      for (int off = CB; off < 32; off <<= 1)
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+#pragma unroll
+          for (int o = 0; o < GR::NOG; ++o) f.acc[k][o] += __shfl_xor_sync(0xffffffffu, f.acc[k][o], off);
+    }
+    if (slice == 0) f.store(out + size_t(n) * orow, C, cb, a.pscale);
+  } else {
+    // tensor product: each slice takes its own sample
+    const int64_t n_units = (a.n_rows + NS - 1) / NS;
+    for (int64_t u = unit; u < n_units; u += a.n_chunks) {
+      const int64_t b = u * NS + slice;
+      if (b >= a.n_rows) continue;
+      f.zero();
+      load_w<GR>(wr, w + b * a.w_stride, C, cb);
+      load_x<CF, GR>(xr, x + size_t(b) * xrow, C, cb);
+      load_y<CF>(Y, y, vec, a.sh_norm, b);
+      f.edge(xr, wr, Y);
+      f.store(out + size_t(b) * orow, C, cb, a.pscale);
+    }
+  }
+}
+
+template <class CF, bool CONV>
+__global__ void __launch_bounds__(256) fwd_kernel(const __grid_constant__ KFwd a) {
+  const int g = int(blockIdx.x % CF::G);
+  const int64_t unit = blockIdx.x / CF::G;
+  dispatch<CF::G>(g, [&](auto gi) { fwd_group<CF, decltype(gi)::value, CONV>(a, unit); });
+}
+
+// ========================================================================= backward ===
+struct KBwd {
+  const int32_t* row_ptr_src;
+  const int32_t* perm_src;
+  const int32_t* dst;
+  const void* x;
+  const void* y;
+  const void* vec;
+  const void* w;
+  const void* grad_out;
+  void* grad_x;
+  void* grad_y;
+  void* grad_w;
+  int64_t n_nodes, n_edges;
+  int C, sh_norm, n_chunks;
+  int* status;
+  double scale;
+  double alpha[MAXP];
+};
+
+constexpr int BWD_WINDOW = 8;  // edge steps between grad_y flushes
+
+template <class CF, int GI>
+struct BwdPart {
+  using T = typename CF::T;
+  using GR = Grp<CF, GI>;
+  T dx[K][GR::NXG];
+
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+#pragma unroll
+      for (int j = 0; j < GR::NXG; ++j) dx[k][j] = T(0);
+  }
+
+  // One edge.  gr: grad_out of the receiver for the group's outputs.  Accumulates dx (scale
+  // applied later), returns the unreduced grad_y contribution of this thread's channels in dY,
+  // and writes grad_w (scaled) when gw != nullptr.
+  __device__ __forceinline__ void edge(const T (&xr)[K][GR::NXG], const T (&wr)[K][GR::NP],
+                                       const T (&Y)[CF::NY], const T (&gr)[K][GR::NOG], T (&dY)[CF::NY],
+                                       bool want_dy, T* __restrict__ gw, int C, int cb, const double* alpha,
+                                       T scale) {
+#pragma unroll
+    for (int i = 0; i < CF::NY; ++i) dY[i] = T(0);
+    static_for<GR::PB, GR::PE>([&](auto pc) {
+      constexpr int P = decltype(pc)::value;
+      using PC = PathC<CF, P>;
+      constexpr int L1 = PC::L1, L2 = PC::L2, L3 = PC::L3, D1 = PC::D1, D3 = PC::D3;
+      constexpr int XO = L1 * L1 - GR::XB, OO = PC::OUT - GR::OB, PW = P - GR::PB;
+      const T al = T(alpha[P]);
+      T wa[K];
+#pragma unroll
+      for (int k = 0; k < K; ++k) wa[k] = al * wr[k][PW];
+      // t[k][m1] = sum_m3 A[m1, m3] g[k][m3]
+      T t[K][D1];
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int m1 = 0; m1 < D1; ++m1) t[k][m1] = T(0);
+      static_for<0, D3>([&](auto m3c) {
+        constexpr int M3I = decltype(m3c)::value;
+        T a[D1];
+        static_for<0, D1>([&](auto m1c) {
+          constexpr int M1I = decltype(m1c)::value;
+          if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) a[M1I] = a_entry<T, L1, L2, L3, M1I - L1, M3I - L3>(Y);
+        });
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+          static_for<0, D1>([&](auto m1c) {
+            constexpr int M1I = decltype(m1c)::value;
+            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) t[k][M1I] = fma(a[M1I], gr[k][OO + M3I], t[k][M1I]);
+          });
+      });
+      // grad_w[e, p, u] = scale * alpha_p * sum_m1 x[u, m1] t[u, m1]
+      if (gw != nullptr) {
+        T o[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          T s = T(0);
+#pragma unroll
+          for (int m1 = 0; m1 < D1; ++m1) s = fma(xr[k][XO + m1], t[k][m1], s);
+          o[k] = scale * al * s;
+        }
+        st16(gw + size_t(P) * C + 4 * cb, o);
+      }
+      // grad_x += alpha_p w t
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int m1 = 0; m1 < D1; ++m1) dx[k][XO + m1] = fma(wa[k], t[k][m1], dx[k][XO + m1]);
+      // grad_y[m2] += sum_{m1, m3} C[m1, m2, m3] Z[m1, m3],  Z = sum_k alpha_p w_k x_k[m1] g_k[m3]
+      if (want_dy) {
+        T xw[K][D1];
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+#pragma unroll
+          for (int m1 = 0; m1 < D1; ++m1) xw[k][m1] = wa[k] * xr[k][XO + m1];
+        static_for<0, D1>([&](auto m1c) {
+          constexpr int M1I = decltype(m1c)::value;
+          static_for<0, D3>([&](auto m3c) {
+            constexpr int M3I = decltype(m3c)::value;
+            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) {
+              T z = T(0);
+#pragma unroll
+              for (int k = 0; k < K; ++k) z = fma(xw[k][M1I], gr[k][OO + M3I], z);
+              static_for<-L2, L2 + 1>([&](auto m2c) {
+                constexpr int M2 = decltype(m2c)::value;
+                if constexpr (cg_nz(L1, L2, L3, M1I - L1, M2, M3I - L3)) {
+                  constexpr int I = cg_index(L1, L2, L3, M1I - L1, M2, M3I - L3);
+                  dY[L2 * L2 + L2 + M2] = fma(CGT<T>::template get<I>(), z, dY[L2 * L2 + L2 + M2]);
+                }
+              });
+            }
+          });
+        });
+      }
+    });
+  }
+};
+
+// grad_out values of the group's outputs for channels 4cb..4cb+3 of row `grow`
+template <class CF, class GR, typename T>
+__device__ __forceinline__ void load_g(T (&gr)[K][GR::NOG], const T* __restrict__ grow, int C, int cb) {
+  static_for<GR::PB, GR::PE>([&](auto pc) {
+    constexpr int P = decltype(pc)::value;
+    using PC = PathC<CF, P>;
+    constexpr int D3 = PC::D3, OO = PC::OUT - GR::OB;
+    T t[K * D3];
+    ld16(t, grow + size_t(C) * PC::OUT + size_t(4 * cb) * D3, false);
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+#pragma unroll
+      for (int m = 0; m < D3; ++m) gr[k][OO + m] = t[k * D3 + m];
+  });
+}
+
+template <class CF, int GI, bool CONV>
+__device__ __forceinline__ void bwd_group(const KBwd& a, int64_t unit, unsigned char* smem_raw) {
+  using T = typename CF::T;
+  using GR = Grp<CF, GI>;
+  const int C = a.C, CB = C >> 2;
+  const int WPG = CB >= 32 ? CB / 32 : 1;  // warps per group
+  const int NW = CF::G * WPG;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wg = warp % WPG;
+  const int cb = CB >= 32 ? wg * 32 + lane : lane % CB;
+  const int slice = CB >= 32 ? 0 : lane / CB;
+  const int NS = CB >= 32 ? 1 : 32 / CB;
+  const bool lead = CB >= 32 ? (lane == 0) : (cb == 0);  // writes the slice's grad_y partial
+  const T* __restrict__ x = static_cast<const T*>(a.x);
+  const T* __restrict__ y = static_cast<const T*>(a.y);
+  const T* __restrict__ vec = static_cast<const T*>(a.vec);
+  const T* __restrict__ w = static_cast<const T*>(a.w);
+  const T* __restrict__ g = static_cast<const T*>(a.grad_out);
+  T* __restrict__ gx = static_cast<T*>(a.grad_x);
+  T* __restrict__ gy = static_cast<T*>(a.grad_y);
+  T* __restrict__ gwp = static_cast<T*>(a.grad_w);
+  const size_t xrow = size_t(CF::NX) * C;
+  const size_t orow = size_t(CF::NO) * C;
+  const size_t wrow = size_t(CF::P) * C;
+  const T scale = T(a.scale);
+  const bool want_dy = gy != nullptr;
+
+  // smem: dys[BWD_WINDOW * NS][NW][NY] grad_y partials, eidx[BWD_WINDOW * NS] edge ids,
+  //       dxs[NSX][NX * C] grad_x rows (NSX = 1 for the convolution, NS for the product)
+  const int NSLOT = BWD_WINDOW * NS;
+  T* dys = reinterpret_cast<T*>(smem_raw);
+  int64_t* eidx = reinterpret_cast<int64_t*>(dys + size_t(NSLOT) * NW * CF::NY);
+  T* dxs = reinterpret_cast<T*>(eidx + NSLOT);
+
+  BwdPart<CF, GI> bp;
+  T xr[K][GR::NXG], wr[K][GR::NP], Y[CF::NY], gr[K][GR::NOG], dY[CF::NY];
+
+  // flush the grad_y partials of the current window: sum over warps in a fixed order
+  auto flush_dy = [&](int nslots) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < nslots * CF::NY; i += blockDim.x) {
+      const int sl = i / CF::NY, m = i % CF::NY;
+      const int64_t e = eidx[sl];
+      if (e < 0) continue;
+      T s = T(0);
+      for (int ww = 0; ww < NW; ++ww) s += dys[(size_t(sl) * NW + ww) * CF::NY + m];
+      gy[e * CF::NY + m] = scale * s;
+    }
+    __syncthreads();
+  };
+  auto put_dy = [&](int sl, int64_t e) {
+    // reduce over the channel lanes of this slice (butterfly), leader stores
+    if (want_dy) {
+      const int lim = CB >= 32 ? 32 : CB;
+      for (int off = 1; off < lim; off <<= 1)
+#pragma unroll
+        for (int i = 0; i < CF::NY; ++i) dY[i] += __shfl_xor_sync(0xffffffffu, dY[i], off);
+      if (lead) {
+#pragma unroll
+        for (int i = 0; i < CF::NY; ++i) dys[(size_t(sl) * NW + warp) * CF::NY + i] = dY[i];
+        if (warp == 0) eidx[sl] = e;
+      }
+    }
+  };
+
+  if constexpr (CONV) {
+    const int64_t n = unit;
+    int64_t j0 = a.row_ptr_src[n], j1 = a.row_ptr_src[n + 1];
+    if (j0 < 0 || j1 < j0 || j1 > a.n_edges) {
+      if (threadIdx.x == 0) record_error(a.status, E3_ERR_INDEX);
+      j0 = j1 = 0;
+    }
+    bp.zero();
+    load_x<CF, GR>(xr, x + size_t(n) * xrow, C, cb);
+    const int64_t deg = j1 - j0;
+    const int64_t steps = (deg + NS - 1) / NS;
+    for (int64_t st0 = 0; st0 < steps; st0 += BWD_WINDOW) {
+      const int nst = int(steps - st0 < BWD_WINDOW ? steps - st0 : BWD_WINDOW);
+      for (int si = 0; si < nst; ++si) {
+        const int64_t jj = (st0 + si) * NS + slice;
+        const int sl = si * NS + slice;
+        int64_t e = -1;
+        bool ok = jj < deg;
+        int32_t d = 0;
+        if (ok) {
+          e = __ldg(a.perm_src + j0 + jj);
+          if (e < 0 || e >= a.n_edges) {
+            ok = false;
+            e = -1;
+            record_error(a.status, E3_ERR_INDEX);
+          } else {
+            d = __ldg(a.dst + e);
+            if (uint32_t(d) >= uint32_t(a.n_nodes)) {
+              ok = false;
+              e = -1;
+              record_error(a.status, E3_ERR_INDEX);
+            }
+          }
+        }
+        if (ok) {
+          load_w<GR>(wr, w + e * wrow, C, cb);
+          load_y<CF>(Y, y, vec, a.sh_norm, e);
+          load_g<CF, GR>(gr, g + size_t(d) * orow, C, cb);
+          bp.edge(xr, wr, Y, gr, dY, want_dy, gwp ? gwp + e * wrow : nullptr, C, cb, a.alpha, scale);
+        } else {
+#pragma unroll
+          for (int i = 0; i < CF::NY; ++i) dY[i] = T(0);
+        }
+        put_dy(sl, e);
+      }
+      if (want_dy) flush_dy(nst * NS);
+    }
+    // grad_x: sum slices (butterfly), then groups in order through shared memory
+    if (gx != nullptr) {
+      if (CB < 32) {
+        for (int off = CB; off < 32; off <<= 1)
+#pragma unroll
+          for (int k = 0; k < K; ++k)
+#pragma unroll
+            for (int j = 0; j < GR::NXG; ++j) bp.dx[k][j] += __shfl_xor_sync(0xffffffffu, bp.dx[k][j], off);
+      }
+      for (int i = threadIdx.x; i < CF::NX * C; i += blockDim.x) dxs[i] = T(0);
+      for (int gg = 0; gg < CF::G; ++gg) {
+        __syncthreads();
+        if (gg == GI && slice == 0) {
+          static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
+            constexpr int L = decltype(lc)::value;
+            constexpr int D = 2 * L + 1;
+#pragma unroll
+            for (int k = 0; k < K; ++k)
+#pragma unroll
+              for (int m = 0; m < D; ++m) dxs[C * (L * L) + (4 * cb + k) * D + m] += bp.dx[k][L * L - GR::XB + m];
+          });
+        }
+      }
+      __syncthreads();
+      for (int i = threadIdx.x; i < CF::NX * C; i += blockDim.x) gx[size_t(n) * xrow + i] = scale * dxs[i];
+    }
+  } else {
+    // tensor product: slice = sample within the step; NS samples per step
+    const int64_t n_units = (a.n_nodes + NS - 1) / NS;
+    for (int64_t u = unit; u < n_units; u += a.n_chunks) {
+      const int64_t b = u * NS + slice;
+      const bool ok = b < a.n_nodes;
+      bp.zero();
+      if (ok) {
+        load_x<CF, GR>(xr, x + size_t(b) * xrow, C, cb);
+        load_w<GR>(wr, w + b * wrow, C, cb);
+        load_y<CF>(Y, y, vec, a.sh_norm, b);
+        load_g<CF, GR>(gr, g + size_t(b) * orow, C, cb);
+        bp.edge(xr, wr, Y, gr, dY, want_dy, gwp ? gwp + b * wrow : nullptr, C, cb, a.alpha, scale);
+      } else {
+#pragma unroll
+        for (int i = 0; i < CF::NY; ++i) dY[i] = T(0);
+      }
+      put_dy(slice, ok ? b : -1);
+      if (want_dy) flush_dy(NS);
+      if (gx != nullptr) {
+        for (int i = threadIdx.x; i < NS * CF::NX * C; i += blockDim.x) dxs[i] = T(0);
+        for (int gg = 0; gg < CF::G; ++gg) {
+          __syncthreads();
+          if (gg == GI) {
+            static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
+              constexpr int L = decltype(lc)::value;
+              constexpr int D = 2 * L + 1;
+#pragma unroll
+              for (int k = 0; k < K; ++k)
+#pragma unroll
+                for (int m = 0; m < D; ++m)
+                  dxs[size_t(slice) * CF::NX * C + C * (L * L) + (4 * cb + k) * D + m] += bp.dx[k][L * L - GR::XB + m];
+            });
+          }
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < NS * CF::NX * C; i += blockDim.x) {
+          const int64_t bb = u * NS + i / (CF::NX * C);
+          if (bb < a.n_nodes) gx[size_t(bb) * xrow + i % (CF::NX * C)] = scale * dxs[i];
+        }
+        __syncthreads();
+      }
+    }
+  }
+}
+
+template <class CF, bool CONV>
+__global__ void __launch_bounds__(320) bwd_kernel(const __grid_constant__ KBwd a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int C = a.C, CB = C >> 2;
+  const int WPG = CB >= 32 ? CB / 32 : 1;
+  const int gi = int(threadIdx.x >> 5) / WPG;
+  dispatch<CF::G>(gi, [&](auto g) { bwd_group<CF, decltype(g)::value, CONV>(a, blockIdx.x, smem_raw); });
+}
+
+template <class CF>
+static size_t bwd_smem_bytes(int C, bool conv) {
+  using T = typename CF::T;
+  const int CB = C / 4;
+  const int WPG = CB >= 32 ? CB / 32 : 1, NS = CB >= 32 ? 1 : 32 / CB;
+  const int NW = CF::G * WPG, NSLOT = BWD_WINDOW * NS;
+  size_t b = sizeof(T) * size_t(NSLOT) * NW * CF::NY + sizeof(int64_t) * NSLOT;
+  b = (b + 15) & ~size_t(15);
+  b += sizeof(T) * size_t(conv ? 1 : NS) * CF::NX * C;
+  return b;
+}
+
+// =================================================================== host launchers ===
+template <class CF>
+e3_status launch_fwd_cfg(const e3_plan* plan, const FwdArgs& h, bool conv) {
+  KFwd a{};
+  a.row_ptr = h.row_ptr;
+  a.src = h.src;
+  a.x = h.x;
+  a.y = h.y;
+  a.vec = h.vec;
+  a.w = h.w;
+  a.out = h.out;
+  a.n_rows = h.n_rows;
+  a.n_edges = h.n_edges;
+  a.w_stride = h.w_stride;
+  a.C = plan->C;
+  a.sh_norm = h.sh_norm;
+  e3_status st = device_status_ptr(&a.status);
+  if (st != E3_OK) return st;
+  for (int p = 0; p < plan->n_paths; ++p) a.pscale[p] = h.scale * plan->alpha[p];
+  const int CB = plan->C / 4;
+  const int threads = CB >= 32 ? CB : 32;
+  const int NS = CB >= 32 ? 1 : 32 / CB;
+  int64_t units;
+  if (conv) {
+    units = h.n_rows;
+    a.n_chunks = 0;
+  } else {
+    const int64_t n_units = (h.n_rows + NS - 1) / NS;
+    units = std::min<int64_t>(n_units, int64_t(sm_count()) * 32);
+    a.n_chunks = int(units);
+  }
+  const int64_t blocks = units * CF::G;
+  if (blocks >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "grid too large");
+  cudaStream_t s = static_cast<cudaStream_t>(h.stream);
+  if (conv)
+    fwd_kernel<CF, true><<<unsigned(blocks), threads, 0, s>>>(a);
+  else
+    fwd_kernel<CF, false><<<unsigned(blocks), threads, 0, s>>>(a);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "forward launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+template <class CF>
+e3_status launch_bwd_cfg(const e3_plan* plan, const BwdArgs& h, bool conv) {
+  KBwd a{};
+  a.row_ptr_src = h.row_ptr_src;
+  a.perm_src = h.perm_src;
+  a.dst = h.dst;
+  a.x = h.x;
+  a.y = h.y;
+  a.vec = h.vec;
+  a.w = h.w;
+  a.grad_out = h.grad_out;
+  a.grad_x = h.grad_x;
+  a.grad_y = h.grad_y;
+  a.grad_w = h.grad_w;
+  a.n_nodes = h.n_nodes;
+  a.n_edges = h.n_edges;
+  a.C = plan->C;
+  a.sh_norm = h.sh_norm;
+  a.scale = h.scale;
+  e3_status st = device_status_ptr(&a.status);
+  if (st != E3_OK) return st;
+  for (int p = 0; p < plan->n_paths; ++p) a.alpha[p] = plan->alpha[p];
+  const int CB = plan->C / 4;
+  const int WPG = CB >= 32 ? CB / 32 : 1;
+  const int NS = CB >= 32 ? 1 : 32 / CB;
+  const int threads = 32 * WPG * CF::G;
+  if (threads > 320) return fail(E3_ERR_UNSUPPORTED, "backward needs %d threads per CTA (max 320)", threads);
+  const size_t smem = bwd_smem_bytes<CF>(plan->C, conv);
+  if (smem > 200 * 1024) return fail(E3_ERR_UNSUPPORTED, "backward needs %zu bytes of shared memory", smem);
+  int64_t blocks;
+  if (conv) {
+    blocks = h.n_nodes;
+    a.n_chunks = 0;
+  } else {
+    const int64_t n_units = (h.n_nodes + NS - 1) / NS;
+    blocks = std::min<int64_t>(n_units, int64_t(sm_count()) * 16);
+    a.n_chunks = int(blocks);
+  }
+  if (blocks >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "grid too large");
+  cudaStream_t s = static_cast<cudaStream_t>(h.stream);
+  cudaError_t err;
+  if (conv) {
+    err = cudaFuncSetAttribute(bwd_kernel<CF, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err == cudaSuccess) bwd_kernel<CF, true><<<unsigned(blocks), threads, smem, s>>>(a);
+  } else {
+    err = cudaFuncSetAttribute(bwd_kernel<CF, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err == cudaSuccess) bwd_kernel<CF, false><<<unsigned(blocks), threads, smem, s>>>(a);
+  }
+  if (err == cudaSuccess) err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "backward launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+
+// Fill this unit's copy of the coefficient tables on the current device.
+static inline cudaError_t upload_tables(const double* t64, const float* t32) {
+  cudaError_t err = cudaMemcpyToSymbol(c_cg64, t64, sizeof(double) * CG_TABLE_SIZE);
+  if (err == cudaSuccess) err = cudaMemcpyToSymbol(c_cg32, t32, sizeof(float) * CG_TABLE_SIZE);
+  return err;
+}
+
+}  // namespace e3b

@@ -1,0 +1,22 @@
+// Kernels of the (1, 2, 2) path set: x degrees 0..1, harmonics 0..2, outputs up to 2.
+#include "kernels.cuh"
+
+namespace e3b {
+
+e3_status upload_tables_l122(const double* t64, const float* t32) {
+  const cudaError_t err = upload_tables(t64, t32);
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uploading the CG table failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+e3_status launch_fwd_l122(const e3_plan* plan, const FwdArgs& a, bool conv) {
+  if (plan->dtype == E3_F32) return launch_fwd_cfg<Cfg<1, 2, 2, float>>(plan, a, conv);
+  return launch_fwd_cfg<Cfg<1, 2, 2, double>>(plan, a, conv);
+}
+
+e3_status launch_bwd_l122(const e3_plan* plan, const BwdArgs& a, bool conv) {
+  if (plan->dtype == E3_F32) return launch_bwd_cfg<Cfg<1, 2, 2, float>>(plan, a, conv);
+  return launch_bwd_cfg<Cfg<1, 2, 2, double>>(plan, a, conv);
+}
+
+}  // namespace e3b

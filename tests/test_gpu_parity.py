@@ -1,0 +1,385 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle on the same seeded
+inputs.  fp32 results must match to an infinity-norm relative error <= 1e-5, fp64 results to
+<= 1e-12; CSR index arrays must match bit for bit."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mlip_message_passing_b200 import workloads as W
+from tests.conftest import rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-5, torch.float64: 1e-12}
+NP = {torch.float32: np.float32, torch.float64: np.float64}
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def e3b():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from mlip_message_passing_b200 import e3b
+    return e3b
+
+
+def oplan(mul, lx, ly, lo):
+    return oracle.make_plan(W.irreps_str(mul, lx), W.sh_irreps(ly), lmax_out=lo)
+
+
+def gplan(e3b, mul, lx, ly, lo, dtype):
+    return e3b.Plan(W.irreps_str(mul, lx), W.sh_irreps(ly), lmax_out=lo, dtype=dtype)
+
+
+def t(a, dtype=None):
+    x = torch.as_tensor(np.ascontiguousarray(a))
+    if dtype is not None:
+        x = x.to(dtype)
+    return x.to(DEV)
+
+
+def h(x):
+    return x.detach().cpu().numpy().astype(np.float64)
+
+
+# ------------------------------------------------------------------------- plans ---
+def test_plan_matches_oracle_enumeration(e3b):
+    for mul, lx, ly, lo in [(8, 1, 2, 2), (64, 2, 3, 2), (128, 3, 3, 3), (4, 1, 1, 2)]:
+        p, q = gplan(e3b, mul, lx, ly, lo, torch.float32), oplan(mul, lx, ly, lo)
+        assert p.irreps_out.replace(" ", "") == str(q.irreps_out).replace(" ", "")
+        assert p.weight_numel == q.weight_numel and p.dim_out == q.irreps_out.dim
+        np.testing.assert_allclose(p.alphas, q.alphas, rtol=1e-15)
+
+
+# --------------------------------------------------------------------- harmonics ---
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+@pytest.mark.parametrize("norm", ["component", "integral", "norm"])
+def test_spherical_harmonics(e3b, dtype, norm):
+    rng = np.random.default_rng(0)
+    v = rng.standard_normal((5000, 3)).astype(NP[dtype])
+    v[7] = 0.0
+    got = h(e3b.spherical_harmonics(3, t(v), sh_norm=norm))
+    ref = oracle.real_sh_all(3, v.astype(np.float64))
+    if norm == "integral":
+        ref = ref / math.sqrt(4 * math.pi)
+    elif norm == "norm":
+        ref = ref / np.sqrt(np.concatenate([[2 * l + 1] * (2 * l + 1) for l in range(4)]))
+    assert rel_err(got, ref) < (2e-6 if dtype == torch.float32 else 1e-14)
+
+
+# ------------------------------------------------------------- tensor product ---
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+def test_tp_small_forward_backward(e3b, dtype):
+    cfg = W.CONFIGS["tp_small"]
+    mul, lx, ly, lo = cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
+    d = W.tp_inputs(cfg["B"], mul, lx, ly, lo, cfg["seed"], cfg["vectors"], dtype=NP[dtype])
+    y = oracle.real_sh_all(ly, d["vec"]).astype(NP[dtype])
+    p, q = gplan(e3b, mul, lx, ly, lo, dtype), oplan(mul, lx, ly, lo)
+    out = e3b.tp_forward(p, t(d["x"]), t(y), t(d["w"]))
+    ref = oracle.tp_forward(q, d["x"], y, d["w"])
+    assert rel_err(h(out), ref) <= TOL[dtype]
+    g = np.random.default_rng(9).standard_normal(ref.shape).astype(NP[dtype])
+    gx, gy, gw = e3b.tp_backward(p, t(d["x"]), t(y), t(d["w"]), t(g))
+    rx, ry, rw = oracle.tp_backward(q, d["x"], y, d["w"], g)
+    assert rel_err(h(gx), rx) <= TOL[dtype]
+    assert rel_err(h(gy), ry) <= TOL[dtype]
+    assert rel_err(h(gw), rw) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("B", [1, 2, 17, 33])
+def test_tp_ragged_batches(e3b, B):
+    # batches that leave part of a warp's sample slices idle
+    d = W.tp_inputs(B, 8, 1, 2, 2, 3, dtype=np.float32)
+    y = oracle.real_sh_all(2, d["vec"]).astype(np.float32)
+    p, q = gplan(e3b, 8, 1, 2, 2, torch.float32), oplan(8, 1, 2, 2)
+    assert rel_err(h(e3b.tp_forward(p, t(d["x"]), t(y), t(d["w"]))), oracle.tp_forward(q, d["x"], y, d["w"])) <= 1e-5
+    g = np.random.default_rng(B).standard_normal((B, q.irreps_out.dim)).astype(np.float32)
+    res = e3b.tp_backward(p, t(d["x"]), t(y), t(d["w"]), t(g))
+    for a, b in zip(res, oracle.tp_backward(q, d["x"], y, d["w"], g)):
+        assert rel_err(h(a), b) <= 1e-5
+
+
+def test_tp_shared_weights(e3b):
+    d = W.tp_inputs(300, 8, 1, 2, 2, 4, dtype=np.float32)
+    y = oracle.real_sh_all(2, d["vec"]).astype(np.float32)
+    p = e3b.Plan(W.irreps_str(8, 1), W.sh_irreps(2), lmax_out=2, shared_weights=True)
+    q = oracle.make_plan(W.irreps_str(8, 1), W.sh_irreps(2), lmax_out=2, shared_weights=True)
+    w = d["w"][0]
+    assert rel_err(h(e3b.tp_forward(p, t(d["x"]), t(y), t(w))), oracle.tp_forward(q, d["x"], y, w)) <= 1e-5
+
+
+def test_tp_batched_full_size_sampled(e3b):
+    cfg = W.CONFIGS["tp_batched"]
+    mul, lx, ly, lo = cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
+    d = W.tp_inputs(cfg["B"], mul, lx, ly, lo, cfg["seed"], cfg["vectors"])
+    vec = t(d["vec"], torch.float32)
+    p, q = gplan(e3b, mul, lx, ly, lo, torch.float32), oplan(mul, lx, ly, lo)
+    y = e3b.spherical_harmonics(ly, vec)  # the library's own harmonics feed the product
+    x, w = t(d["x"]), t(d["w"])
+    out = e3b.tp_forward(p, x, y, w)
+    rows = np.unique(np.concatenate([[0, cfg["B"] - 1], np.random.default_rng(0).integers(0, cfg["B"], 1500)]))
+    yh = h(y)[rows]
+    ref = oracle.tp_forward(q, d["x"][rows], yh, d["w"][rows])
+    assert rel_err(h(out[torch.as_tensor(rows, device=DEV)]), ref) <= 1e-5
+    g = torch.randn_like(out)
+    gx, gy, gw = e3b.tp_backward(p, x, y, w, g)
+    ri = torch.as_tensor(rows, device=DEV)
+    rx, ry, rw = oracle.tp_backward(q, d["x"][rows], yh, d["w"][rows], h(g[ri]))
+    assert rel_err(h(gx[ri]), rx) <= 1e-5
+    assert rel_err(h(gy[ri]), ry) <= 1e-5
+    assert rel_err(h(gw[ri]), rw) <= 1e-5
+
+
+# --------------------------------------------------------------------------- CSR ---
+def _csr_case(e3b, n, src, dst):
+    ref = oracle.csr_build(n, src, dst)
+    got = e3b.csr_build(n, t(src), t(dst))
+    for a, b in zip(got, ref):
+        assert a.dtype == torch.int32
+        assert np.array_equal(a.cpu().numpy(), b)
+
+
+def test_csr_bit_exact(e3b):
+    g = W.graph_inputs(3000, 4, 0, 0, 0, seed=2)
+    _csr_case(e3b, 3000, g["src"], g["dst"])
+    rng = np.random.default_rng(1)
+    for n, e in [(1, 0), (1, 5), (7, 1), (300, 5000), (70000, 9000), (5, 4099)]:
+        src = rng.integers(0, n, e).astype(np.int32)
+        dst = rng.integers(0, n, e).astype(np.int32)
+        _csr_case(e3b, n, src, dst)
+    # a hub receiver with many duplicates (ties must keep input order)
+    dst = np.zeros(20000, dtype=np.int32)
+    dst[::3] = 5
+    src = rng.integers(0, 9, 20000).astype(np.int32)
+    _csr_case(e3b, 9, src, dst)
+
+
+def test_csr_out_of_range_is_reported(e3b):
+    src = np.array([0, 1, 2, 7], dtype=np.int32)
+    dst = np.array([1, 2, 0, 1], dtype=np.int32)
+    e3b.csr_build(3, t(src), t(dst))
+    with pytest.raises(e3b.E3Error) as ei:
+        e3b.device_status()
+    assert ei.value.status == e3b.E3_ERR_INDEX
+    e3b.device_status()  # cleared
+
+
+# ------------------------------------------------------------------- convolution ---
+def conv_setup(e3b, n_nodes, mul, lx, ly, lo, seed, dtype, weights="host"):
+    g = W.graph_inputs(n_nodes, mul, lx, ly, lo, seed, dtype=NP[dtype], weights=weights, device=DEV)
+    graph = e3b.Graph(n_nodes, t(g["src"]), t(g["dst"]))
+    w_dev = g["w"] if weights == "torch" else t(g["w"])
+    return g, graph, w_dev
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+@pytest.mark.parametrize("mode", ["y", "vec"])
+def test_conv_forward_backward_full(e3b, dtype, mode):
+    # a small water box: several CTAs per SM, ragged degrees (about 52 +- 7)
+    n, mul, lx, ly, lo = 400, 64, 2, 3, 2
+    g, graph, w = conv_setup(e3b, n, mul, lx, ly, lo, 21, dtype)
+    p, q = gplan(e3b, mul, lx, ly, lo, dtype), oplan(mul, lx, ly, lo)
+    Y = oracle.real_sh_all(ly, g["vec"].astype(np.float64)).astype(NP[dtype])
+    s = 1 / math.sqrt(52)
+    wr = graph.to_receiver_order(w)
+    kw = dict(y=graph.to_receiver_order(t(Y))) if mode == "y" else dict(edge_vec=graph.to_receiver_order(t(g["vec"])))
+    out = e3b.conv_forward(p, graph, t(g["x"]), wr, out_scale=s, **kw)
+    ref = oracle.conv_forward(q, n, g["src"], g["dst"], g["x"], Y, g["w"], s)
+    assert rel_err(h(out), ref) <= TOL[dtype]
+    go = W.grad_out(n, q.irreps_out.dim, 5, dtype=NP[dtype])
+    gx, gy, gw = e3b.conv_backward(p, graph, t(g["x"]), wr, t(go), out_scale=s, **kw)
+    rx, ry, rw = oracle.conv_backward(q, n, g["src"], g["dst"], g["x"], Y, g["w"], go, s)
+    perm = graph.perm_dst.cpu().numpy()
+    assert rel_err(h(gx), rx) <= TOL[dtype]
+    assert rel_err(h(gy), ry[perm]) <= TOL[dtype]
+    assert rel_err(h(gw), rw[perm]) <= TOL[dtype]
+
+
+def test_conv_small_multiplicity_and_degrees(e3b):
+    # C = 8 (16 edge slices per warp) on the (1, 2, 2) path set and C = 4 on (1, 1, 2)
+    for mul, lx, ly, lo in [(8, 1, 2, 2), (4, 1, 1, 2), (32, 2, 3, 2)]:
+        n = 400
+        g = W.graph_inputs(n, mul, lx, ly, lo, 8, dtype=np.float32)
+        graph = e3b.Graph(n, t(g["src"]), t(g["dst"]))
+        p, q = gplan(e3b, mul, lx, ly, lo, torch.float32), oplan(mul, lx, ly, lo)
+        vec = graph.to_receiver_order(t(g["vec"]))
+        wr = graph.to_receiver_order(t(g["w"]))
+        Y = oracle.real_sh_all(ly, g["vec"].astype(np.float64))
+        out = e3b.conv_forward(p, graph, t(g["x"]), wr, edge_vec=vec, out_scale=0.2)
+        assert rel_err(h(out), oracle.conv_forward(q, n, g["src"], g["dst"], g["x"], Y, g["w"], 0.2)) <= 1e-5
+        go = W.grad_out(n, q.irreps_out.dim, 6)
+        res = e3b.conv_backward(p, graph, t(g["x"]), wr, t(go), edge_vec=vec, out_scale=0.2)
+        ref = oracle.conv_backward(q, n, g["src"], g["dst"], g["x"], Y, g["w"], go, 0.2)
+        perm = graph.perm_dst.cpu().numpy()
+        assert rel_err(h(res[0]), ref[0]) <= 1e-5
+        assert rel_err(h(res[1]), ref[1][perm]) <= 1e-5
+        assert rel_err(h(res[2]), ref[2][perm]) <= 1e-5
+
+
+def test_conv_edge_cases(e3b):
+    p = gplan(e3b, 8, 1, 2, 2, torch.float32)
+    q = oplan(8, 1, 2, 2)
+    rng = np.random.default_rng(3)
+    # no edges at all: zero rows, no kernel reads of edge arrays
+    n = 5
+    graph = e3b.Graph(n, t(np.zeros(0, np.int32)), t(np.zeros(0, np.int32)))
+    x = t(rng.standard_normal((n, p.dim_in1)).astype(np.float32))
+    out = e3b.conv_forward(p, graph, x, torch.zeros((0, p.weight_numel), device=DEV),
+                           edge_vec=torch.zeros((0, 3), device=DEV))
+    assert out.shape == (n, p.dim_out) and torch.all(out == 0)
+    gx, gy, gw = e3b.conv_backward(p, graph, x, torch.zeros((0, p.weight_numel), device=DEV),
+                                   torch.ones((n, p.dim_out), device=DEV), edge_vec=torch.zeros((0, 3), device=DEV))
+    assert torch.all(gx == 0) and gy.shape[0] == 0 and gw.shape[0] == 0
+    # isolated receivers and senders, a single edge, a hub receiver with 300 in-edges
+    src = np.array([0, 2, 2, 3] + [1] * 300, dtype=np.int32)
+    dst = np.array([1, 1, 3, 0] + [4] * 300, dtype=np.int32)
+    n = 6  # node 5 is isolated
+    vec = rng.standard_normal((len(src), 3)).astype(np.float32)
+    w = rng.standard_normal((len(src), p.weight_numel)).astype(np.float32)
+    x = rng.standard_normal((n, p.dim_in1)).astype(np.float32)
+    graph = e3b.Graph(n, t(src), t(dst))
+    out = e3b.conv_forward(p, graph, t(x), graph.to_receiver_order(t(w)), edge_vec=graph.to_receiver_order(t(vec)))
+    Y = oracle.real_sh_all(2, vec.astype(np.float64))
+    ref = oracle.conv_forward(q, n, src, dst, x, Y, w, 1.0)
+    assert rel_err(h(out), ref) <= 1e-5 and torch.all(out[5] == 0) and torch.all(out[2] == 0)
+
+
+def test_conv_bad_index_is_reported_not_dereferenced(e3b):
+    p = gplan(e3b, 8, 1, 2, 2, torch.float32)
+    n = 4
+    src = np.array([0, 1, 2, 3], dtype=np.int32)
+    dst = np.array([1, 2, 3, 0], dtype=np.int32)
+    graph = e3b.Graph(n, t(src), t(dst))
+    graph.src[2] = 1000  # corrupt one sender id after the CSR was built
+    x = torch.randn(n, p.dim_in1, device=DEV)
+    w = torch.randn(4, p.weight_numel, device=DEV)
+    out = e3b.conv_forward(p, graph, x, w, edge_vec=torch.randn(4, 3, device=DEV))
+    with pytest.raises(e3b.E3Error) as ei:
+        e3b.device_status()
+    assert ei.value.status == e3b.E3_ERR_INDEX
+    assert torch.isfinite(out).all()
+    e3b.device_status()
+
+
+def test_conv_deterministic(e3b):
+    g, graph, w = conv_setup(e3b, 400, 64, 2, 3, 2, 22, torch.float32)
+    p = gplan(e3b, 64, 2, 3, 2, torch.float32)
+    vec, wr, x = graph.to_receiver_order(t(g["vec"])), graph.to_receiver_order(w), t(g["x"])
+    a = e3b.conv_forward(p, graph, x, wr, edge_vec=vec, out_scale=0.1)
+    b = e3b.conv_forward(p, graph, x, wr, edge_vec=vec, out_scale=0.1)
+    assert torch.equal(a, b)
+    go = torch.randn_like(a)
+    r1 = e3b.conv_backward(p, graph, x, wr, go, edge_vec=vec, out_scale=0.1)
+    r2 = e3b.conv_backward(p, graph, x, wr, go, edge_vec=vec, out_scale=0.1)
+    for u, v in zip(r1, r2):
+        assert torch.equal(u, v)
+
+
+def test_conv_waterbox_full_size_sampled(e3b):
+    """The benchmark's workload and launch configuration (3000 nodes, ~156k edges, 64 channels,
+    harmonics from edge vectors), checked on sampled receivers, senders and edges."""
+    cfg = W.CONFIGS["conv_waterbox"]
+    n, mul, lx, ly, lo = cfg["N"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
+    g, graph, w = conv_setup(e3b, n, mul, lx, ly, lo, cfg["seed"], torch.float32)
+    p, q = gplan(e3b, mul, lx, ly, lo, torch.float32), oplan(mul, lx, ly, lo)
+    s = 1 / math.sqrt(52)
+    vec, wr, x = graph.to_receiver_order(t(g["vec"])), graph.to_receiver_order(w), t(g["x"])
+    out = e3b.conv_forward(p, graph, x, wr, edge_vec=vec, out_scale=s)
+    rng = np.random.default_rng(0)
+    nodes = np.unique(np.concatenate([[0, n - 1], rng.integers(0, n, 150)]))
+    sel = np.flatnonzero(np.isin(g["dst"], nodes))
+    Y = oracle.real_sh_all(ly, g["vec"][sel].astype(np.float64))
+    full = oracle.conv_forward(q, n, g["src"][sel], g["dst"][sel], g["x"], Y, g["w"][sel], s)
+    assert rel_err(h(out)[nodes], full[nodes]) <= 1e-5
+    # backward: grad_x of sampled senders (all their out-edges), grad_y / grad_w of sampled edges
+    go = W.grad_out(n, q.irreps_out.dim, W.CONFIGS["conv_waterbox_bwd"]["grad_seed"])
+    gx, gy, gw = e3b.conv_backward(p, graph, x, wr, t(go), edge_vec=vec, out_scale=s)
+    senders = np.unique(np.concatenate([[0, n - 1], rng.integers(0, n, 80)]))
+    sel = np.flatnonzero(np.isin(g["src"], senders))
+    Y = oracle.real_sh_all(ly, g["vec"][sel].astype(np.float64))
+    rx, ry, rw = oracle.conv_backward(q, n, g["src"][sel], g["dst"][sel], g["x"], Y, g["w"][sel], go, s)
+    assert rel_err(h(gx)[senders], rx[senders]) <= 1e-5
+    inv = np.empty_like(graph.perm_dst.cpu().numpy())
+    inv[graph.perm_dst.cpu().numpy()] = np.arange(len(inv))
+    pos = torch.as_tensor(inv[sel], device=DEV)
+    assert rel_err(h(gy[pos]), ry) <= 1e-5
+    assert rel_err(h(gw[pos]), rw) <= 1e-5
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+def test_conv_large_sampled(e3b, dtype):
+    """24000 nodes, ~1.26M edges, 128 channels, l <= 3: 256 sampled receivers."""
+    cfg = W.CONFIGS["conv_large"]
+    n, mul, lx, ly, lo = cfg["N"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
+    torch.cuda.empty_cache()
+    g, graph, w = conv_setup(e3b, n, mul, lx, ly, lo, cfg["seed"], dtype, weights="torch")
+    p, q = gplan(e3b, mul, lx, ly, lo, dtype), oplan(mul, lx, ly, lo)
+    s = 1 / math.sqrt(52)
+    vec, x = graph.to_receiver_order(t(g["vec"])), t(g["x"])
+    wr = graph.to_receiver_order(w)
+    out = e3b.conv_forward(p, graph, x, wr, edge_vec=vec, out_scale=s)
+    nodes = np.sort(np.random.default_rng(1).choice(n, 256, replace=False))
+    sel = np.flatnonzero(np.isin(g["dst"], nodes))
+    w_sel = h(w[torch.as_tensor(sel, device=DEV)])
+    Y = oracle.real_sh_all(ly, g["vec"][sel].astype(np.float64))
+    ref = oracle.conv_forward(q, n, g["src"][sel], g["dst"][sel], g["x"], Y, w_sel, s)
+    assert rel_err(h(out[torch.as_tensor(nodes, device=DEV)]), ref[nodes]) <= TOL[dtype]
+    del w, wr, out
+    torch.cuda.empty_cache()
+
+
+def test_conv_backward_finite_differences_subgraph(e3b):
+    """fp64 on the 50 nodes nearest to node 0 of the water box (every edge among them):
+    the kernel gradients equal central differences of the kernel forward and the oracle."""
+    cfg = W.CONFIGS["conv_waterbox"]
+    g = W.graph_inputs(cfg["N"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"], cfg["seed"], dtype=np.float64)
+    nodes, eids, s_src, s_dst = W.subgraph_nearest(g["pos"], g["side"], g["src"], g["dst"], 0, 50)
+    n = len(nodes)
+    x = g["x"][nodes]
+    w = g["w"][eids]
+    vec = g["vec"][eids]
+    p = gplan(e3b, 64, 2, 3, 2, torch.float64)
+    q = oplan(64, 2, 3, 2)
+    graph = e3b.Graph(n, t(s_src), t(s_dst))
+    Y = oracle.real_sh_all(3, vec)
+    Yr, wr = graph.to_receiver_order(t(Y)), graph.to_receiver_order(t(w))
+    go = np.random.default_rng(4).standard_normal((n, p.dim_out))
+    s = 1 / math.sqrt(52)
+    gx, gy, gw = e3b.conv_backward(p, graph, t(x), wr, t(go), y=Yr, out_scale=s)
+    rng = np.random.default_rng(5)
+    hstep = 1e-4
+
+    def L(xx, yy, ww):
+        return float((t(go) * e3b.conv_forward(p, graph, xx, ww, y=yy, out_scale=s)).sum())
+
+    for which, grad in ((0, gx), (1, gy), (2, gw)):
+        base = [t(x), Yr, wr]
+        d = torch.as_tensor(rng.standard_normal(tuple(base[which].shape)), device=DEV)
+        plus, minus = list(base), list(base)
+        plus[which] = base[which] + hstep * d
+        minus[which] = base[which] - hstep * d
+        fd = (L(*plus) - L(*minus)) / (2 * hstep)
+        an = float((grad * d).sum())
+        assert abs(fd - an) <= 1e-8 * max(1.0, abs(an))
+    rx, ry, rw = oracle.conv_backward(q, n, s_src, s_dst, x, Y, w, go, s)
+    perm = graph.perm_dst.cpu().numpy()
+    assert rel_err(h(gx), rx) <= 1e-12
+    assert rel_err(h(gy), ry[perm]) <= 1e-12
+    assert rel_err(h(gw), rw[perm]) <= 1e-12
+
+
+def test_autograd_wrapper(e3b):
+    g, graph, w = conv_setup(e3b, 200, 32, 2, 3, 2, 9, torch.float32)
+    p = gplan(e3b, 32, 2, 3, 2, torch.float32)
+    Y = graph.to_receiver_order(e3b.spherical_harmonics(3, t(g["vec"])))
+    x = t(g["x"]).requires_grad_()
+    y = Y.clone().requires_grad_()
+    wr = graph.to_receiver_order(w).requires_grad_()
+    out = e3b.conv(p, graph, x, y, wr, 0.3)
+    go = torch.randn_like(out)
+    out.backward(go)
+    gx, gy, gw = e3b.conv_backward(p, graph, x.detach(), wr.detach(), go, y=Y, out_scale=0.3)
+    assert torch.equal(x.grad, gx) and torch.equal(y.grad, gy) and torch.equal(wr.grad, gw)

@@ -1,0 +1,109 @@
+"""Host-side checks of the C-ABI library that need no GPU: every declared symbol is exported,
+argument validation returns the documented status before any launch, and the library's CG
+table (ladder construction) equals the oracle's (Racah formula) -- two independent generators."""
+
+import ctypes
+import itertools
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "e3b.h")
+
+
+@pytest.fixture(scope="module")
+def e3b():
+    from mlip_message_passing_b200 import e3b
+    return e3b
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^E3_API\s+[\w\s\*]+?\b(e3_\w+)\s*\(", txt, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol(e3b):
+    decl = declared_symbols()
+    assert len(decl) >= 15
+    raw = ctypes.CDLL(e3b.LIB_PATH)
+    for name in decl:
+        assert hasattr(raw, name), name
+    assert sorted(e3b.SYMBOLS) == decl
+
+
+def test_ladder_cg_equals_racah_cg(e3b):
+    import oracle
+    for l1, l2 in itertools.product(range(4), range(4)):
+        for l3 in range(abs(l1 - l2), min(l1 + l2, 3) + 1):
+            lib = e3b.cg_dense(l1, l2, l3).numpy()
+            np.testing.assert_allclose(lib, oracle.real_cg(l1, l2, l3), atol=1e-14, rtol=0)
+
+
+def test_cg_dense_errors(e3b):
+    out = (ctypes.c_double * 64)()
+    assert e3b.lib.e3_cg_dense(1, 1, 3, out) == e3b.E3_ERR_INSTRUCTION
+    assert e3b.lib.e3_cg_dense(4, 0, 4, out) == e3b.E3_ERR_UNSUPPORTED
+    assert e3b.lib.e3_cg_dense(1, 1, 1, None) == e3b.E3_ERR_INVALID_ARG
+
+
+def _create(e3b, a, b, c=None, instr=None, mode=0, dtype=0, wmode=0):
+    h = ctypes.c_void_p()
+    arr, n = None, 0
+    if instr is not None:
+        n = len(instr)
+        arr = (e3b.Instruction * n)(*[e3b.Instruction(i, j, k, 1, -1.0) for i, j, k in instr])
+    st = e3b.lib.e3_plan_create(a.encode(), b.encode(), None if c is None else c.encode(), arr, n, mode, dtype,
+                                wmode, ctypes.byref(h))
+    return st, e3b.lib.e3_last_error().decode()
+
+
+@pytest.mark.parametrize("a,b,code", [
+    ("8x0e+8x1q", "1x0e", "IRREPS_PARSE"),
+    ("8x0e+", "1x0e", "IRREPS_PARSE"),
+    ("", "1x0e", "IRREPS_PARSE"),
+    ("8x0e", "x1o", "IRREPS_PARSE"),
+])
+def test_plan_parse_errors(e3b, a, b, code):
+    st, msg = _create(e3b, a, b)
+    assert e3b.STATUS_NAMES[st] == code and msg
+
+
+def test_plan_instruction_errors(e3b):
+    st, msg = _create(e3b, "8x1o", "1x1o", "8x0o", instr=[(0, 0, 0)])
+    assert st == e3b.E3_ERR_INSTRUCTION and "parity" in msg
+    st, msg = _create(e3b, "8x1o", "1x1o", "8x3e", instr=[(0, 0, 0)])
+    assert st == e3b.E3_ERR_INSTRUCTION and "triangle" in msg
+    st, msg = _create(e3b, "8x1o", "1x1o", "8x0e", instr=[(0, 1, 0)])
+    assert st == e3b.E3_ERR_INSTRUCTION and "range" in msg
+    st, msg = _create(e3b, "8x1o", "1x1o", "4x0e", instr=[(0, 0, 0)])
+    assert st == e3b.E3_ERR_INSTRUCTION
+
+
+def test_plan_unsupported(e3b):
+    # uvw mode, unsupported layouts, degrees without compiled kernels
+    assert _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", mode=1)[0] == e3b.E3_ERR_UNSUPPORTED
+    assert _create(e3b, "8x0e+4x1o", "1x0e+1x1o+1x2e")[0] == e3b.E3_ERR_UNSUPPORTED
+    assert _create(e3b, "8x1o+8x0e", "1x0e+1x1o+1x2e")[0] == e3b.E3_ERR_UNSUPPORTED
+    assert _create(e3b, "6x0e+6x1o", "1x0e+1x1o+1x2e")[0] == e3b.E3_ERR_UNSUPPORTED
+    assert _create(e3b, "8x0e+8x1o+8x2e+8x3o+8x4e", "1x0e+1x1o")[0] == e3b.E3_ERR_UNSUPPORTED
+    # an output filter that drops a path of the enumeration
+    st, msg = _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", "1x0e+1x1o+1x2e")
+    assert st == e3b.E3_ERR_UNSUPPORTED and "every path" in msg
+    assert _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", dtype=7)[0] == e3b.E3_ERR_INVALID_ARG
+
+
+def test_supported_list(e3b):
+    s = e3b.supported()
+    assert (1, 2, 2) in s and (2, 3, 2) in s and (3, 3, 3) in s
+
+
+def test_csr_workspace_and_argument_errors(e3b):
+    n = ctypes.c_size_t()
+    assert e3b.lib.e3_csr_workspace_size(3000, 156278, ctypes.byref(n)) == e3b.E3_OK and n.value > 4 * 156278 * 4
+    assert e3b.lib.e3_csr_workspace_size(-1, 5, ctypes.byref(n)) == e3b.E3_ERR_SHAPE
+    assert e3b.lib.e3_gather_rows(4, 4, 6, None, None, None, None) == e3b.E3_ERR_SHAPE
+    assert e3b.lib.e3_spherical_harmonics(4, 10, None, 0, 0, None, None) == e3b.E3_ERR_UNSUPPORTED
+    assert e3b.lib.e3_tp_forward(None, 1, None, None, None, None, None) == e3b.E3_ERR_INVALID_ARG
