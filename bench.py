@@ -1,0 +1,375 @@
+"""Benchmark of the channelwise CG tensor-product convolution (forward + backward) on B200.
+
+Default workload (``conv_waterbox``): the water-box-like graph of 3000 nodes at 0.1 atoms/A^3
+with a 5 A cutoff (~156k directed edges), node features 64x0e+64x1o+64x2e fp32, harmonics of
+degree <= 3 evaluated in the kernel from edge vectors, output degrees <= 2 (18 paths,
+uncollapsed), per-edge weights from the radial MLP fixture, aggregation scale 1/sqrt(52).
+One step = conv forward + conv backward (grad_x, grad_y, grad_w) through the C ABI.
+
+Output: one JSON line on rank 0 (see the fields below).  ``--impl reference`` times the float64
+CPU oracle on a bounded sample of the same workload instead.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "edges/sec and achieved HBM GB/s (% of B200 peak) for TP-conv fwd and fwd+bwd"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="conv_waterbox", choices=["conv_waterbox", "conv_large"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mlip_message_passing_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        ent = d[workload][kernel]
+        if ent.get("src_hash") != kernel_source_hash():
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def workload_spec(name):
+    from mlip_message_passing_b200 import workloads as W
+    cfg = dict(W.CONFIGS[name])
+    mul, lx, ly, lo = cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
+    return cfg, W.irreps_str(mul, lx), W.sh_irreps(ly)
+
+
+def algorithmic_bytes(N, E, mul, lx, ly, lo, esize=4):
+    """Each unique tensor read or written once (edge vectors as input, int32 indices)."""
+    from mlip_message_passing_b200 import workloads as W
+    P = W.n_paths(lx, ly, lo)
+    dx, dy, do, wn = mul * (lx + 1) ** 2, (ly + 1) ** 2, W.out_dim(mul, lx, ly, lo), P * mul
+    fwd = E * (wn * esize + 3 * esize + 4) + N * (dx * esize + do * esize + 4) + 4
+    bwd = E * (2 * wn * esize + 3 * esize + dy * esize + 8) + N * (do * esize + 2 * dx * esize + 4) + 4
+    return fwd, bwd
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"e3b_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}",
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx = max(mx, float(parts[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[3:7]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.remove(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_sample(cfg, irreps_x, irreps_y, n_edges_target, seed=0):
+    """The oracle (float64 CPU) on the in-edges of random receivers: (edges, seconds fwd+bwd)."""
+    import oracle
+    from mlip_message_passing_b200 import workloads as W
+    g = W.graph_inputs(cfg["N"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"], cfg["seed"])
+    plan = oracle.make_plan(irreps_x, irreps_y, lmax_out=cfg["lo"])
+    rng = np.random.default_rng(seed)
+    nodes = rng.permutation(cfg["N"])
+    deg = np.bincount(g["dst"], minlength=cfg["N"])
+    take = nodes[:max(1, int(np.searchsorted(np.cumsum(deg[nodes]), n_edges_target)))]
+    sel = np.flatnonzero(np.isin(g["dst"], take))
+    go = W.grad_out(cfg["N"], plan.irreps_out.dim, cfg.get("grad_seed", 4))
+    s = 1.0 / math.sqrt(52.0)
+    t0 = time.perf_counter()
+    Y = oracle.real_sh_all(cfg["ly"], g["vec"][sel].astype(np.float64))
+    oracle.conv_forward(plan, cfg["N"], g["src"][sel], g["dst"][sel], g["x"], Y, g["w"][sel], s)
+    oracle.conv_backward(plan, cfg["N"], g["src"][sel], g["dst"][sel], g["x"], Y, g["w"][sel], go, s)
+    return len(sel), time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg, irreps_x, irreps_y = workload_spec(args.workload)
+    budget = 8000  # edges per step: a few seconds of CPU work per step
+    per_step, tot_e, tot_t = [], 0, 0.0
+    for k in range(args.warmup + args.steps):
+        e, t = oracle_sample(cfg, irreps_x, irreps_y, budget, seed=k)
+        if k >= args.warmup:
+            tot_e += e
+            tot_t += t
+    v = tot_e / tot_t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "edges/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload + "_fwd_bwd", "nodes": cfg["N"],
+                                        "sample": f"in-edges of random receivers, ~{budget} edges per step"},
+        "cpu_baseline": {"value": v, "unit": "edges/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"~{budget} edges per step (fwd+bwd), {args.steps} steps"},
+        "e2e": {"value": v, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+    from mlip_message_passing_b200 import e3b, workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    cfg, irreps_x, irreps_y = workload_spec(args.workload)
+    N, mul, lx, ly, lo = cfg["N"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
+    # weak scaling: every rank owns an independent box of the same size (its own seed)
+    g = W.graph_inputs(N, mul, lx, ly, lo, cfg["seed"] + 1000 * rank, weights="torch", device=dev)
+    plan = e3b.Plan(irreps_x, irreps_y, lmax_out=lo)
+    graph = e3b.Graph(N, torch.as_tensor(g["src"], device=dev), torch.as_tensor(g["dst"], device=dev))
+    E = graph.n_edges
+    x = torch.as_tensor(g["x"], device=dev)
+    vec = graph.to_receiver_order(torch.as_tensor(g["vec"], device=dev))
+    w = graph.to_receiver_order(g["w"])
+    del g
+    go = torch.as_tensor(W.grad_out(N, plan.dim_out, cfg.get("grad_seed", 4)), device=dev)
+    s = 1.0 / math.sqrt(52.0)
+    out = torch.empty((N, plan.dim_out), device=dev)
+    gx = torch.empty_like(x)
+    gy = torch.empty((E, plan.dim_in2), device=dev)
+    gw = torch.empty_like(w)
+    stream = torch.cuda.current_stream()
+    ev = []
+
+    def step(record):
+        if record:
+            a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            a.record(stream)
+        e3b.lib.e3_conv_forward(plan.handle, N, E, e3b._ptr(graph.row_ptr_dst), e3b._ptr(graph.src), e3b._ptr(x),
+                                None, e3b._ptr(vec), 0, e3b._ptr(w), s, e3b._ptr(out), e3b._stream())
+        if record:
+            b.record(stream)
+        e3b.lib.e3_conv_backward(plan.handle, N, E, e3b._ptr(graph.row_ptr_dst), e3b._ptr(graph.src),
+                                 e3b._ptr(graph.dst), e3b._ptr(graph.row_ptr_src), e3b._ptr(graph.perm_src),
+                                 e3b._ptr(x), None, e3b._ptr(vec), 0, e3b._ptr(w), e3b._ptr(go), s, e3b._ptr(gx),
+                                 e3b._ptr(gy), e3b._ptr(gw), e3b._stream())
+        if record:
+            c.record(stream)
+            ev.append((a, b, c))
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    e3b.device_status()
+    launches_per_step = 2
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    with ClockSampler(local) as clk:
+        barrier()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        t1.record(stream)
+        barrier()
+    ms_total = t0.elapsed_time(t1)
+    fwd_ms = statistics.fmean(a.elapsed_time(b) for a, b, c in ev)
+    bwd_ms = statistics.fmean(b.elapsed_time(c) for a, b, c in ev)
+    e3b.device_status()
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = E * world / (ms_step * 1e-3)
+
+    # end to end through the public API: inputs from pinned host memory, results back to host
+    e2e = None
+    if not args.no_e2e:
+        hx = x.cpu().pin_memory()
+        hvec = vec.cpu().pin_memory()
+        hw = w.cpu().pin_memory()
+        hgo = go.cpu().pin_memory()
+        hout = torch.empty(out.shape, pin_memory=True)
+        hgx = torch.empty(gx.shape, pin_memory=True)
+        hgy = torch.empty(gy.shape, pin_memory=True)
+        hgw = torch.empty(gw.shape, pin_memory=True)
+        dx_, dvec_, dw_, dgo_ = (torch.empty_like(t) for t in (x, vec, w, go))
+
+        def e2e_step():
+            for d_, h_ in ((dx_, hx), (dvec_, hvec), (dw_, hw), (dgo_, hgo)):
+                d_.copy_(h_, non_blocking=True)
+            o = e3b.conv_forward(plan, graph, dx_, dw_, edge_vec=dvec_, out_scale=s)
+            r = e3b.conv_backward(plan, graph, dx_, dw_, dgo_, edge_vec=dvec_, out_scale=s)
+            for h_, d_ in ((hout, o), (hgx, r[0]), (hgy, r[1]), (hgw, r[2])):
+                h_.copy_(d_, non_blocking=True)
+
+        e2e_steps = max(1, min(args.steps, 5))
+        e2e_step()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        barrier()
+        e_ms = a.elapsed_time(b) / e2e_steps
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(t.numel() * t.element_size() for t in (hx, hvec, hw, hgo))
+        d2h = sum(t.numel() * t.element_size() for t in (hout, hgx, hgy, hgw))
+        e2e = {"value": E * world / (e_ms * 1e-3), "unit": "edges/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    fb, bb = algorithmic_bytes(N, E, mul, lx, ly, lo)
+    peak, peak_kind = hbm_peak()
+    fwd_gbs, bwd_gbs = fb / (fwd_ms * 1e-3) / 1e9, bb / (bwd_ms * 1e-3) / 1e9
+    dom = "conv_backward" if bwd_ms >= fwd_ms else "conv_forward"
+    dom_gbs, dom_bytes = (bwd_gbs, bb) if dom == "conv_backward" else (fwd_gbs, fb)
+    cpu = None
+    if not args.no_cpu_baseline:
+        e_s, t_s = oracle_sample(cfg, irreps_x, irreps_y, 40000)
+        cpu = {"value": e_s / t_s, "unit": "edges/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"float64 oracle fwd+bwd on the {e_s} in-edges of random receivers of the same graph "
+                         f"({t_s:.1f} s)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{args.workload}_fwd_bwd", "nodes_per_gpu": N, "edges_per_gpu": E,
+                   "irreps_x": irreps_x, "irreps_sh": irreps_y, "lmax_out": lo, "paths": plan.n_paths,
+                   "sh_from": "edge vectors (in-kernel)", "out_scale": "1/sqrt(52)", "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2: the streamed weights are "
+                         f"{w.numel() * 4 / 1e6:.0f} MB per launch (L2 126 MB)"},
+        "fwd": {"ms": fwd_ms, "edges_per_s": E / (fwd_ms * 1e-3), "GBps": fwd_gbs, "frac_of_hbm": fwd_gbs / peak,
+                "algorithmic_bytes": fb},
+        "bwd": {"ms": bwd_ms, "edges_per_s": E / (bwd_ms * 1e-3), "GBps": bwd_gbs, "frac_of_hbm": bwd_gbs / peak,
+                "algorithmic_bytes": bb},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": dom_gbs / peak, "peak_kind": peak_kind,
+                     "traffic": traffic_for(dom, args.workload), "algorithmic_bytes": dom_bytes},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -595,7 +595,7 @@ static e3_status check_conv_common(const e3_plan* plan, int64_t N, int64_t E, co
                                    e3_sh_norm sh_norm) {
   if (N < 0 || N >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N = %lld out of range", (long long)N);
   if (E < 0 || E >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "E = %lld out of range", (long long)E);
-  if ((y == nullptr) == (vec == nullptr)) return fail(E3_ERR_INVALID_ARG, "give exactly one of y and edge_vec");
+  if (E > 0 && (y == nullptr) == (vec == nullptr)) return fail(E3_ERR_INVALID_ARG, "give exactly one of y and edge_vec");
   if (vec != nullptr && (sh_norm < E3_SH_COMPONENT || sh_norm > E3_SH_NORM))
     return fail(E3_ERR_INVALID_ARG, "bad sh_norm %d", int(sh_norm));
   if (vec != nullptr && (reinterpret_cast<uintptr_t>(vec) % (plan->dtype == E3_F64 ? 8 : 4)) != 0)

@@ -280,7 +280,7 @@ struct KFwd {
   const void* w;
   void* out;
   int64_t n_rows, n_edges, w_stride;
-  int C, sh_norm, n_chunks;
+  int C, sh_norm, n_chunks, stages;
   int* status;
   double pscale[MAXP];  // scale * alpha_p
 };
@@ -371,45 +371,273 @@ struct FwdAcc {
   }
 };
 
-template <class CF, int GI, bool CONV>
-__device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit) {
+// ------------------------------------------------------------ async copy machinery ---
+// One thread per CTA streams the weight and x slices of upcoming edges into a ring of shared
+// memory stages with cp.async.bulk (1-D TMA, no multicast); completion is tracked by one
+// mbarrier per stage (transaction bytes).  Every wait is bounded: after WAIT_LIMIT polls the
+// kernel records E3_ERR_TIMEOUT and stops issuing work.
+constexpr long long WAIT_LIMIT = 1ll << 24;
+constexpr int FWD_WIN = 96;  // in-edges whose sender ids and harmonics are staged at once
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_addr(dst)),
+               "l"(src), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
+}
+// bounded wait; false after WAIT_LIMIT polls (the error is recorded)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+  for (long long i = 0; i < WAIT_LIMIT; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  record_error(status, E3_ERR_TIMEOUT);
+  return false;
+}
+
+template <typename T, int N>
+__device__ __forceinline__ void lds16(T (&r)[N], const T* p) {
+  if constexpr (std::is_same<T, float>::value) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const float4 v = reinterpret_cast<const float4*>(p)[i];
+      r[4 * i] = v.x;
+      r[4 * i + 1] = v.y;
+      r[4 * i + 2] = v.z;
+      r[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const double2 v = reinterpret_cast<const double2*>(p)[i];
+      r[2 * i] = v.x;
+      r[2 * i + 1] = v.y;
+    }
+  }
+}
+
+// Byte sizes of one edge's slices for group GI: weights of the group's paths (all channels)
+// and x blocks l1 in [L1A, L1B] (all channels); both are contiguous in global memory.
+template <class CF, int GI>
+struct FwdSlice {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
-  const int C = a.C, CB = C >> 2;
-  const int lane = threadIdx.x;
-  const int cb = CB >= 32 ? lane : lane % CB;
-  const int slice = CB >= 32 ? 0 : lane / CB;
-  const int NS = CB >= 32 ? 1 : 32 / CB;
-  const T* __restrict__ x = static_cast<const T*>(a.x);
+  static __host__ __device__ constexpr uint32_t wbytes(int C) { return uint32_t(GR::NP) * C * sizeof(T); }
+  static __host__ __device__ constexpr uint32_t xbytes(int C) { return uint32_t(GR::NXG) * C * sizeof(T); }
+};
+
+template <class CF, int I = 0>
+__host__ __device__ constexpr uint32_t max_slice_bytes(int C) {
+  if constexpr (I >= CF::G) {
+    return 0;
+  } else {
+    const uint32_t a = FwdSlice<CF, I>::wbytes(C) + FwdSlice<CF, I>::xbytes(C);
+    const uint32_t b = max_slice_bytes<CF, I + 1>(C);
+    return a > b ? a : b;
+  }
+}
+
+// Shared memory of the forward CTA.
+template <class CF>
+struct FwdSmem {
+  using T = typename CF::T;
+  static constexpr int NYP = (CF::NY + 3) & ~3;  // harmonics row padded to 16 bytes (float)
+  static __host__ __device__ size_t ysh_off() { return 0; }
+  static __host__ __device__ size_t src_off() { return sizeof(T) * size_t(FWD_WIN) * NYP; }
+  static __host__ __device__ size_t bar_off() { return src_off() + sizeof(int32_t) * FWD_WIN; }
+  static __host__ __device__ size_t stage_off(int S) { return (bar_off() + 8 * size_t(S) + 127) & ~size_t(127); }
+  static __host__ __device__ size_t stage_bytes(int C, int NS) { return size_t(NS) * max_slice_bytes<CF>(C); }
+  static __host__ __device__ size_t total(int C, int NS, int S) { return stage_off(S) + size_t(S) * stage_bytes(C, NS); }
+};
+
+// Stage sender ids (checked) and harmonics of edges [e0 + ws, e0 + ws + cnt) into shared
+// memory.  Shared by every path group, so it is kept out of line (one copy of the code).
+template <class CF, bool CONV>
+__device__ __noinline__ void fwd_stage_window(const KFwd& a, int64_t e0, int64_t ws, int cnt,
+                                              typename CF::T* ysh, int32_t* src_s) {
+  using T = typename CF::T;
+  constexpr int NYP = FwdSmem<CF>::NYP;
   const T* __restrict__ y = static_cast<const T*>(a.y);
   const T* __restrict__ vec = static_cast<const T*>(a.vec);
+  for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+    const int64_t e = e0 + ws + i;
+    if constexpr (CONV) {
+      const int32_t s = __ldg(a.src + e);
+      const bool ok = uint32_t(s) < uint32_t(a.n_rows);
+      if (!ok) record_error(a.status, E3_ERR_INDEX);
+      src_s[i] = ok ? s : -1;
+    }
+    T Yl[CF::NY];
+    load_y<CF>(Yl, y, vec, a.sh_norm, e);
+#pragma unroll
+    for (int m = 0; m < CF::NY; ++m) ysh[i * NYP + m] = Yl[m];
+  }
+}
+
+template <class CF, int GI, bool CONV>
+__device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned char* smem) {
+  using T = typename CF::T;
+  using GR = Grp<CF, GI>;
+  using SM = FwdSmem<CF>;
+  constexpr int NYP = SM::NYP;
+  const int C = a.C, CB = C >> 2;
+  const int tid = threadIdx.x;
+  const int cb = CB >= 32 ? tid : tid % CB;
+  const int slice = CB >= 32 ? 0 : tid / CB;
+  const int NS = CB >= 32 ? 1 : 32 / CB;
+  const int S = a.stages;
+  const T* __restrict__ x = static_cast<const T*>(a.x);
   const T* __restrict__ w = static_cast<const T*>(a.w);
   T* __restrict__ out = static_cast<T*>(a.out);
-  const size_t xrow = size_t(CF::NX) * C;
-  const size_t orow = size_t(CF::NO) * C;
+  const size_t xrow = size_t(CF::NX) * C, orow = size_t(CF::NO) * C;
+  const uint32_t WB = FwdSlice<CF, GI>::wbytes(C), XB = FwdSlice<CF, GI>::xbytes(C);
+  const uint32_t SLOT = WB + XB;
+  const size_t STAGE = SM::stage_bytes(C, NS);
 
-  FwdAcc<CF, GI> f;
-  T xr[K][GR::NXG], wr[K][GR::NP], Y[CF::NY];
+  T* ysh = reinterpret_cast<T*>(smem + SM::ysh_off());
+  int32_t* src_s = reinterpret_cast<int32_t*>(smem + SM::src_off());
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::bar_off());
+  unsigned char* stages = smem + SM::stage_off(S);
+
+  // segment of rows handled by this CTA
+  int64_t e0, e1;
   if constexpr (CONV) {
-    const int64_t n = unit;
-    int64_t e0 = a.row_ptr[n], e1 = a.row_ptr[n + 1];
+    e0 = a.row_ptr[unit];
+    e1 = a.row_ptr[unit + 1];
     if (e0 < 0 || e1 < e0 || e1 > a.n_edges) {
-      if (lane == 0) record_error(a.status, E3_ERR_INDEX);
+      if (tid == 0) record_error(a.status, E3_ERR_INDEX);
       e0 = e1 = 0;
     }
-    f.zero();
-    for (int64_t e = e0 + slice; e < e1; e += NS) {
-      const int32_t s = __ldg(a.src + e);
-      if (uint32_t(s) >= uint32_t(a.n_rows)) {
-        record_error(a.status, E3_ERR_INDEX);
-        continue;
+  } else {
+    const int64_t per = (a.n_rows + a.n_chunks - 1) / a.n_chunks;
+    e0 = unit * per;
+    e1 = e0 + per < a.n_rows ? e0 + per : a.n_rows;
+    if (e0 > e1) e0 = e1;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  FwdAcc<CF, GI> f;
+  f.zero();
+  T xr[K][GR::NXG], wr[K][GR::NP], Y[CF::NY];
+  uint32_t issued = 0;  // steps issued so far (all windows), drives stage index and parity
+  uint32_t consumed = 0;
+  bool alive = true;
+  const int64_t deg = e1 - e0;
+
+  for (int64_t ws = 0; ws < deg && alive; ws += FWD_WIN) {
+    const int cnt = int(deg - ws < FWD_WIN ? deg - ws : FWD_WIN);
+    fwd_stage_window<CF, CONV>(a, e0, ws, cnt, ysh, src_s);
+    __syncthreads();
+    const int steps = (cnt + NS - 1) / NS;
+    // producer: stage `st` of this window -> ring slot issued % S
+    auto issue = [&](int st) {
+      const uint32_t slot = issued % S;
+      uint64_t* bar = &bars[slot];
+      unsigned char* dst = stages + size_t(slot) * STAGE;
+      uint32_t bytes = 0;
+      for (int j = 0; j < NS; ++j) {
+        const int r = st * NS + j;
+        if (r < cnt && (!CONV || src_s[r] >= 0)) bytes += SLOT;
       }
-      load_w<GR>(wr, w + e * a.w_stride, C, cb);
-      load_x<CF, GR>(xr, x + size_t(s) * xrow, C, cb);
-      load_y<CF>(Y, y, vec, a.sh_norm, e);
-      f.edge(xr, wr, Y);
+      mbar_arrive_expect_tx(bar, bytes);
+      for (int j = 0; j < NS; ++j) {
+        const int r = st * NS + j;
+        if (r >= cnt) break;
+        const int64_t e = e0 + ws + r;
+        int64_t xr_row = e;
+        if constexpr (CONV) {
+          if (src_s[r] < 0) continue;
+          xr_row = src_s[r];
+        }
+        bulk_load(dst + size_t(j) * SLOT, w + e * a.w_stride + size_t(GR::PB) * C, WB, bar);
+        bulk_load(dst + size_t(j) * SLOT + WB, x + size_t(xr_row) * xrow + size_t(GR::XB) * C, XB, bar);
+      }
+      ++issued;
+    };
+    if (tid == 0)
+      for (int st = 0; st < S && st < steps; ++st) issue(st);
+    // `issued` is only advanced by thread 0; every thread tracks the same count
+    if (tid != 0) issued += uint32_t(S < steps ? S : steps);
+
+    for (int st = 0; st < steps; ++st) {
+      const uint32_t slot = consumed % S, parity = (consumed / S) & 1u;
+      const bool ok = mbar_wait(&bars[slot], parity, a.status);
+      if (__syncthreads_or(!ok)) {  // uniform decision: no thread leaves the barrier loop alone
+        alive = false;
+        break;
+      }
+      ++consumed;
+      const int r = st * NS + slice;
+      const bool mine = r < cnt && (!CONV || src_s[r] >= 0);
+      if (mine) {
+        const T* sl = reinterpret_cast<const T*>(stages + size_t(slot) * STAGE + size_t(slice) * SLOT);
+        // weights of the group's paths for channels 4cb..4cb+3
+#pragma unroll
+        for (int q = 0; q < GR::NP; ++q) {
+          T t4[K];
+          lds16(t4, sl + size_t(q) * C + 4 * cb);
+#pragma unroll
+          for (int k = 0; k < K; ++k) wr[k][q] = t4[k];
+        }
+        const T* xs = sl + WB / sizeof(T);
+        static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
+          constexpr int L = decltype(lc)::value;
+          constexpr int D = 2 * L + 1;
+          T t[K * D];
+          lds16(t, xs + size_t(C) * (L * L - GR::XB) + size_t(4 * cb) * D);
+#pragma unroll
+          for (int k = 0; k < K; ++k)
+#pragma unroll
+            for (int m = 0; m < D; ++m) xr[k][L * L - GR::XB + m] = t[k * D + m];
+        });
+        {
+          T yp[NYP];
+          lds16(yp, ysh + r * NYP);
+#pragma unroll
+          for (int m = 0; m < CF::NY; ++m) Y[m] = yp[m];
+        }
+        if constexpr (!CONV) f.zero();
+        f.edge(xr, wr, Y);
+        if constexpr (!CONV) f.store(out + size_t(e0 + ws + r) * orow, C, cb, a.pscale);
+      }
+      __syncthreads();  // every thread is done with this stage
+      if (tid == 0 && st + S < steps) issue(st + S);
+      if (tid != 0 && st + S < steps) ++issued;
     }
-    // sum the slices (lanes cb, cb + CB, ...) in a fixed butterfly order
+    __syncthreads();  // window staging buffers are reused by the next window
+  }
+  if (!alive) {
+    // a wait gave up: let the copies in flight land (bounded) before the CTA exits
+    if (tid == 0)
+      while (consumed < issued) {
+        mbar_wait(&bars[consumed % S], (consumed / S) & 1u, a.status);
+        ++consumed;
+      }
+    __syncthreads();
+    return;
+  }
+  if constexpr (CONV) {
     if (CB < 32) {
       for (int off = CB; off < 32; off <<= 1)
 #pragma unroll
@@ -417,28 +645,19 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit) {
 #pragma unroll
           for (int o = 0; o < GR::NOG; ++o) f.acc[k][o] += __shfl_xor_sync(0xffffffffu, f.acc[k][o], off);
     }
-    if (slice == 0) f.store(out + size_t(n) * orow, C, cb, a.pscale);
-  } else {
-    // tensor product: each slice takes its own sample
-    const int64_t n_units = (a.n_rows + NS - 1) / NS;
-    for (int64_t u = unit; u < n_units; u += a.n_chunks) {
-      const int64_t b = u * NS + slice;
-      if (b >= a.n_rows) continue;
-      f.zero();
-      load_w<GR>(wr, w + b * a.w_stride, C, cb);
-      load_x<CF, GR>(xr, x + size_t(b) * xrow, C, cb);
-      load_y<CF>(Y, y, vec, a.sh_norm, b);
-      f.edge(xr, wr, Y);
-      f.store(out + size_t(b) * orow, C, cb, a.pscale);
-    }
+    if (slice == 0) f.store(out + size_t(unit) * orow, C, cb, a.pscale);
   }
 }
 
 template <class CF, bool CONV>
 __global__ void __launch_bounds__(256) fwd_kernel(const __grid_constant__ KFwd a) {
-  const int g = int(blockIdx.x % CF::G);
-  const int64_t unit = blockIdx.x / CF::G;
-  dispatch<CF::G>(g, [&](auto gi) { fwd_group<CF, decltype(gi)::value, CONV>(a, unit); });
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  // group-major order: CTAs are started roughly in index order, so the CTAs resident on an SM
+  // at any time run the same path group and share its (large, fully unrolled) code
+  const int64_t units = int64_t(gridDim.x) / CF::G;
+  const int g = int(blockIdx.x / units);
+  const int64_t unit = blockIdx.x % units;
+  dispatch<CF::G>(g, [&](auto gi) { fwd_group<CF, decltype(gi)::value, CONV>(a, unit, smem_raw); });
 }
 
 // ========================================================================= backward ===
@@ -804,23 +1023,35 @@ e3_status launch_fwd_cfg(const e3_plan* plan, const FwdArgs& h, bool conv) {
   const int CB = plan->C / 4;
   const int threads = CB >= 32 ? CB : 32;
   const int NS = CB >= 32 ? 1 : 32 / CB;
+  // ring depth: as deep as 3 stages while the CTAs that fit by registers also fit in shared memory
+  auto kern = conv ? fwd_kernel<CF, true> : fwd_kernel<CF, false>;
+  cudaFuncAttributes fa{};
+  cudaError_t err = cudaFuncGetAttributes(&fa, kern);
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(err));
+  const int regs = fa.numRegs > 0 ? fa.numRegs : 255;
+  int ctas = 65536 / (((regs + 7) & ~7) * ((threads + 31) & ~31));
+  ctas = std::max(1, std::min(ctas, 32));
+  const size_t budget = size_t(225) * 1024 / ctas;
+  int S = 3;
+  while (S > 2 && FwdSmem<CF>::total(plan->C, NS, S) + 1024 > budget) --S;
+  a.stages = S;
+  const size_t smem = FwdSmem<CF>::total(plan->C, NS, S);
+  if (smem > size_t(227) * 1024) return fail(E3_ERR_UNSUPPORTED, "forward needs %zu bytes of shared memory", smem);
   int64_t units;
   if (conv) {
     units = h.n_rows;
     a.n_chunks = 0;
   } else {
     const int64_t n_units = (h.n_rows + NS - 1) / NS;
-    units = std::min<int64_t>(n_units, int64_t(sm_count()) * 32);
+    units = std::min<int64_t>(n_units, int64_t(sm_count()) * ctas);
     a.n_chunks = int(units);
   }
   const int64_t blocks = units * CF::G;
   if (blocks >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "grid too large");
-  cudaStream_t s = static_cast<cudaStream_t>(h.stream);
-  if (conv)
-    fwd_kernel<CF, true><<<unsigned(blocks), threads, 0, s>>>(a);
-  else
-    fwd_kernel<CF, false><<<unsigned(blocks), threads, 0, s>>>(a);
-  const cudaError_t err = cudaGetLastError();
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
+  kern<<<unsigned(blocks), threads, smem, static_cast<cudaStream_t>(h.stream)>>>(a);
+  err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "forward launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
 }

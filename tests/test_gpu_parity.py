@@ -372,7 +372,7 @@ def test_conv_backward_finite_differences_subgraph(e3b):
 
 
 def test_autograd_wrapper(e3b):
-    g, graph, w = conv_setup(e3b, 200, 32, 2, 3, 2, 9, torch.float32)
+    g, graph, w = conv_setup(e3b, 400, 32, 2, 3, 2, 9, torch.float32)
     p = gplan(e3b, 32, 2, 3, 2, torch.float32)
     Y = graph.to_receiver_order(e3b.spherical_harmonics(3, t(g["vec"])))
     x = t(g["x"]).requires_grad_()
