@@ -182,6 +182,26 @@ E3_API e3_status e3_csr_build(int64_t N, int64_t E, const int32_t* src, const in
                        int32_t* perm_dst, int32_t* row_ptr_dst, int32_t* perm_src,
                        int32_t* row_ptr_src, void* workspace, size_t ws_bytes, void* stream);
 
+/* No counterpart in the paper: a library convenience.  Same result as e3_csr_build, but the
+ * scratch lives in a fixed device array owned by the library, so the caller passes no
+ * workspace and nothing is allocated.  It exists for callers that cannot allocate device
+ * memory at the point where they build a graph: code running inside a CUDA stream capture
+ * (cudaMalloc is not allowed there), code embedded in a host program whose device memory is
+ * all owned by its own pool or arena, and loops that must avoid the implicit device
+ * synchronisation of cudaMalloc / cudaFree.
+ *   - Limit: E <= E3_CSR_STATIC_MAX_EDGES; larger E returns E3_ERR_SHAPE before any launch.
+ *     The array (about 16.5 MiB) is held on every device that loads the library until exit.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     and sets up the device status word; make that first call before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU (different streams, or
+ *     different host threads without ordering) race and give undefined results.  Nothing in
+ *     the array needs to start at zero: every pass overwrites what it reads.
+ *   - Errors as e3_csr_build. */
+#define E3_CSR_STATIC_MAX_EDGES (1 << 20)
+E3_API e3_status e3_csr_build_static(int64_t N, int64_t E, const int32_t* src, const int32_t* dst,
+                                     int32_t* perm_dst, int32_t* row_ptr_dst, int32_t* perm_src,
+                                     int32_t* row_ptr_src, void* stream);
+
 /* Rows of `in` gathered by `perm`: out[i, :] = in[perm[i], :] for i < n_rows, each row
  * row_bytes bytes (multiple of 4).  Used once per topology to put edge arrays into receiver
  * order.  perm entries must lie in [0, n_in_rows). */

@@ -15,6 +15,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "internal.h"
 
@@ -272,4 +273,59 @@ extern "C" e3_status e3_gather_rows(int64_t n_rows, int64_t n_in_rows, int64_t r
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "gather launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
+}
+
+// ------------------------------------------------------------ no-allocation variant ---
+// e3_csr_build_static: the same CSR build with its scratch in a fixed device array that the
+// library owns, for callers that cannot allocate device memory themselves.  The array is
+// sized for E3_CSR_STATIC_MAX_EDGES edges and lives on every device that loads the library
+// until the process exits.
+namespace e3b {
+
+constexpr size_t static_align256(size_t b) { return (b + 255) & ~size_t(255); }
+constexpr size_t kStaticTiles = (size_t(E3_CSR_STATIC_MAX_EDGES) + RS_TILE - 1) / RS_TILE;
+constexpr size_t kStaticScratchBytes =
+    4 * static_align256(sizeof(int32_t) * size_t(E3_CSR_STATIC_MAX_EDGES)) +
+    static_align256(sizeof(int32_t) * size_t(RS_RADIX) * kStaticTiles);
+
+static __device__ __align__(256) unsigned char g_csr_scratch[kStaticScratchBytes];
+
+static std::mutex g_scratch_mutex;
+static void* g_scratch_ptr[64] = {};
+
+// Device address of g_csr_scratch on the current device (looked up once per device; the
+// name g_csr_scratch is only a host-side stand-in and must never be passed to a kernel).
+static e3_status static_scratch(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(E3_ERR_CUDA, "cudaGetDevice failed");
+  if (dev < 0 || dev >= 64) return fail(E3_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t err = cudaGetSymbolAddress(&p, g_csr_scratch);
+    if (err != cudaSuccess || p == nullptr)
+      return fail(E3_ERR_CUDA, "cudaGetSymbolAddress(csr scratch) failed: %s", cudaGetErrorString(err));
+    g_scratch_ptr[dev] = p;
+  }
+  *ptr = g_scratch_ptr[dev];
+  return E3_OK;
+}
+
+}  // namespace e3b
+
+extern "C" e3_status e3_csr_build_static(int64_t N, int64_t E, const int32_t* src, const int32_t* dst,
+                                         int32_t* perm_dst, int32_t* row_ptr_dst, int32_t* perm_src,
+                                         int32_t* row_ptr_src, void* stream) {
+  clear_error();
+  if (E > int64_t(E3_CSR_STATIC_MAX_EDGES))
+    return fail(E3_ERR_SHAPE, "e3_csr_build_static: %lld edges exceed the built-in scratch limit of %d edges; "
+                "use e3_csr_build with a caller-provided workspace", (long long)E, E3_CSR_STATIC_MAX_EDGES);
+  if (E < 0 || N < 0) return fail(E3_ERR_SHAPE, "N or E out of range");
+  if (csr_ws_bytes(E) > kStaticScratchBytes)
+    return fail(E3_ERR_SHAPE, "e3_csr_build_static: scratch too small for %lld edges", (long long)E);
+  void* ws = nullptr;
+  const e3_status st = static_scratch(&ws);
+  if (st != E3_OK) return st;
+  return e3_csr_build(N, E, src, dst, perm_dst, row_ptr_dst, perm_src, row_ptr_src, ws, kStaticScratchBytes,
+                      stream);
 }

@@ -25,7 +25,7 @@ SYMBOLS = [
     "e3_plan_create", "e3_plan_destroy", "e3_plan_info", "e3_plan_irreps_out", "e3_plan_paths",
     "e3_device_status", "e3_cg_dense", "e3_supported", "e3_tp_forward", "e3_tp_backward",
     "e3_spherical_harmonics", "e3_csr_workspace_size", "e3_csr_build", "e3_gather_rows",
-    "e3_conv_forward", "e3_conv_backward", "e3_last_error",
+    "e3_conv_forward", "e3_conv_backward", "e3_last_error", "e3_csr_build_static",
 ]
 
 
@@ -62,6 +62,7 @@ def _load():
         "e3_spherical_harmonics": [I32, I64, VP, ctypes.c_int, ctypes.c_int, VP, VP],
         "e3_csr_workspace_size": [I64, I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_csr_build": [I64, I64, VP, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP],
+        "e3_csr_build_static": [I64, I64, VP, VP, VP, VP, VP, VP, VP],
         "e3_gather_rows": [I64, I64, I64, VP, VP, VP, VP],
         "e3_conv_forward": [VP, I64, I64, VP, VP, VP, VP, VP, ctypes.c_int, VP, D, VP, VP],
         "e3_conv_backward": [VP, I64, I64, VP, VP, VP, VP, VP, VP, VP, VP, ctypes.c_int, VP, VP, D, VP, VP, VP,
