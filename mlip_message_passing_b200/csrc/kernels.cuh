@@ -674,141 +674,239 @@ struct KBwd {
   void* grad_y;
   void* grad_w;
   int64_t n_nodes, n_edges;
-  int C, sh_norm, n_chunks;
+  int C, sh_norm, n_chunks, stages;
   int* status;
   double scale;
   double alpha[MAXP];
 };
 
-constexpr int BWD_WINDOW = 8;  // edge steps between grad_y flushes
-
+// Which path groups touch x block l1 / harmonics block l2 (the first toucher stores, later
+// groups accumulate; blocks no group touches are zero-filled by group 0).
+template <class CF>
+__host__ __device__ constexpr int first_group_l1(int l) {
+  for (int g = 0; g < CF::G; ++g)
+    for (int p = group_begin(CF::LX, CF::LY, CF::LO, g); p < group_begin(CF::LX, CF::LY, CF::LO, g + 1); ++p)
+      if (path_l(CF::LX, CF::LY, CF::LO, p, 0) == l) return g;
+  return -1;
+}
+template <class CF>
+__host__ __device__ constexpr int first_group_l2(int l) {
+  for (int g = 0; g < CF::G; ++g)
+    for (int p = group_begin(CF::LX, CF::LY, CF::LO, g); p < group_begin(CF::LX, CF::LY, CF::LO, g + 1); ++p)
+      if (path_l(CF::LX, CF::LY, CF::LO, p, 1) == l) return g;
+  return -1;
+}
 template <class CF, int GI>
-struct BwdPart {
+__host__ __device__ constexpr bool group_has_l2(int l) {
+  for (int p = group_begin(CF::LX, CF::LY, CF::LO, GI); p < group_begin(CF::LX, CF::LY, CF::LO, GI + 1); ++p)
+    if (path_l(CF::LX, CF::LY, CF::LO, p, 1) == l) return true;
+  return false;
+}
+
+constexpr int BWD_WIN = 64;  // out-edges whose ids and harmonics are staged at once
+
+// Byte sizes of one edge's staged slices in the backward of group GI: weights of the group's
+// paths, grad_out of the receiver for the group's outputs, and (tensor product only) the x slice.
+template <class CF, int GI>
+struct BwdSlice {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
-  T dx[K][GR::NXG];
-
-  __device__ __forceinline__ void zero() {
-#pragma unroll
-    for (int k = 0; k < K; ++k)
-#pragma unroll
-      for (int j = 0; j < GR::NXG; ++j) dx[k][j] = T(0);
+  static __host__ __device__ constexpr uint32_t wbytes(int C) { return uint32_t(GR::NP) * C * sizeof(T); }
+  static __host__ __device__ constexpr uint32_t gbytes(int C) { return uint32_t(GR::NOG) * C * sizeof(T); }
+  static __host__ __device__ constexpr uint32_t xbytes(int C, bool conv) {
+    return conv ? 0u : uint32_t(GR::NXG) * C * sizeof(T);
   }
+  static __host__ __device__ constexpr uint32_t slot(int C, bool conv) { return wbytes(C) + gbytes(C) + xbytes(C, conv); }
+};
 
-  // One edge.  gr: grad_out of the receiver for the group's outputs.  Accumulates dx (scale
-  // applied later), returns the unreduced grad_y contribution of this thread's channels in dY,
-  // and writes grad_w (scaled) when gw != nullptr.
-  __device__ __forceinline__ void edge(const T (&xr)[K][GR::NXG], const T (&wr)[K][GR::NP],
-                                       const T (&Y)[CF::NY], const T (&gr)[K][GR::NOG], T (&dY)[CF::NY],
-                                       bool want_dy, T* __restrict__ gw, int C, int cb, const double* alpha,
-                                       T scale) {
-#pragma unroll
-    for (int i = 0; i < CF::NY; ++i) dY[i] = T(0);
-    static_for<GR::PB, GR::PE>([&](auto pc) {
-      constexpr int P = decltype(pc)::value;
-      using PC = PathC<CF, P>;
-      constexpr int L1 = PC::L1, L2 = PC::L2, L3 = PC::L3, D1 = PC::D1, D3 = PC::D3;
-      constexpr int XO = L1 * L1 - GR::XB, OO = PC::OUT - GR::OB, PW = P - GR::PB;
-      const T al = T(alpha[P]);
-      T wa[K];
-#pragma unroll
-      for (int k = 0; k < K; ++k) wa[k] = al * wr[k][PW];
-      // t[k][m1] = sum_m3 A[m1, m3] g[k][m3]
-      T t[K][D1];
-#pragma unroll
-      for (int k = 0; k < K; ++k)
-#pragma unroll
-        for (int m1 = 0; m1 < D1; ++m1) t[k][m1] = T(0);
-      static_for<0, D3>([&](auto m3c) {
-        constexpr int M3I = decltype(m3c)::value;
-        T a[D1];
-        static_for<0, D1>([&](auto m1c) {
-          constexpr int M1I = decltype(m1c)::value;
-          if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) a[M1I] = a_entry<T, L1, L2, L3, M1I - L1, M3I - L3>(Y);
-        });
-#pragma unroll
-        for (int k = 0; k < K; ++k)
-          static_for<0, D1>([&](auto m1c) {
-            constexpr int M1I = decltype(m1c)::value;
-            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) t[k][M1I] = fma(a[M1I], gr[k][OO + M3I], t[k][M1I]);
-          });
-      });
-      // grad_w[e, p, u] = scale * alpha_p * sum_m1 x[u, m1] t[u, m1]
-      if (gw != nullptr) {
-        T o[K];
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-          T s = T(0);
-#pragma unroll
-          for (int m1 = 0; m1 < D1; ++m1) s = fma(xr[k][XO + m1], t[k][m1], s);
-          o[k] = scale * al * s;
-        }
-        st16(gw + size_t(P) * C + 4 * cb, o);
-      }
-      // grad_x += alpha_p w t
-#pragma unroll
-      for (int k = 0; k < K; ++k)
-#pragma unroll
-        for (int m1 = 0; m1 < D1; ++m1) dx[k][XO + m1] = fma(wa[k], t[k][m1], dx[k][XO + m1]);
-      // grad_y[m2] += sum_{m1, m3} C[m1, m2, m3] Z[m1, m3],  Z = sum_k alpha_p w_k x_k[m1] g_k[m3]
-      if (want_dy) {
-        T xw[K][D1];
-#pragma unroll
-        for (int k = 0; k < K; ++k)
-#pragma unroll
-          for (int m1 = 0; m1 < D1; ++m1) xw[k][m1] = wa[k] * xr[k][XO + m1];
-        static_for<0, D1>([&](auto m1c) {
-          constexpr int M1I = decltype(m1c)::value;
-          static_for<0, D3>([&](auto m3c) {
-            constexpr int M3I = decltype(m3c)::value;
-            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) {
-              T z = T(0);
-#pragma unroll
-              for (int k = 0; k < K; ++k) z = fma(xw[k][M1I], gr[k][OO + M3I], z);
-              static_for<-L2, L2 + 1>([&](auto m2c) {
-                constexpr int M2 = decltype(m2c)::value;
-                if constexpr (cg_nz(L1, L2, L3, M1I - L1, M2, M3I - L3)) {
-                  constexpr int I = cg_index(L1, L2, L3, M1I - L1, M2, M3I - L3);
-                  dY[L2 * L2 + L2 + M2] = fma(CGT<T>::template get<I>(), z, dY[L2 * L2 + L2 + M2]);
-                }
-              });
-            }
-          });
-        });
-      }
-    });
+template <class CF, int GI>
+struct BwdSmem {
+  using T = typename CF::T;
+  static constexpr int NYP = (CF::NY + 3) & ~3;
+  static __host__ __device__ size_t ysh_off() { return 0; }
+  static __host__ __device__ size_t eid_off() { return sizeof(T) * size_t(BWD_WIN) * NYP; }
+  static __host__ __device__ size_t did_off() { return eid_off() + sizeof(int32_t) * BWD_WIN; }
+  static __host__ __device__ size_t bar_off() { return did_off() + sizeof(int32_t) * BWD_WIN; }
+  static __host__ __device__ size_t stage_off(int S) { return (bar_off() + 8 * size_t(S) + 127) & ~size_t(127); }
+  static __host__ __device__ size_t stage_bytes(int C, int NS, bool conv) {
+    return size_t(NS) * BwdSlice<CF, GI>::slot(C, conv);
+  }
+  static __host__ __device__ size_t total(int C, int NS, int S, bool conv) {
+    return stage_off(S) + size_t(S) * stage_bytes(C, NS, conv);
   }
 };
 
-// grad_out values of the group's outputs for channels 4cb..4cb+3 of row `grow`
-template <class CF, class GR, typename T>
-__device__ __forceinline__ void load_g(T (&gr)[K][GR::NOG], const T* __restrict__ grow, int C, int cb) {
+// Per-edge backward of one path group with grad_out read from shared memory (sg: the group's
+// outputs, channels in mul_ir order).  Accumulates alpha_p w t into dx, returns this thread's
+// unreduced grad_y contribution in dY and writes grad_w (scaled) when gw != nullptr.
+template <class CF, int GI>
+__device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, GI>::NXG],
+                                         const typename CF::T (&wr)[K][Grp<CF, GI>::NP],
+                                         const typename CF::T (&Y)[CF::NY], const typename CF::T* sg,
+                                         typename CF::T (&dx)[K][Grp<CF, GI>::NXG], typename CF::T (&dY)[CF::NY],
+                                         bool want_dy, typename CF::T* __restrict__ gw, int C, int cb,
+                                         const double* alpha, typename CF::T scale) {
+  using T = typename CF::T;
+  using GR = Grp<CF, GI>;
+#pragma unroll
+  for (int i = 0; i < CF::NY; ++i) dY[i] = T(0);
   static_for<GR::PB, GR::PE>([&](auto pc) {
     constexpr int P = decltype(pc)::value;
     using PC = PathC<CF, P>;
-    constexpr int D3 = PC::D3, OO = PC::OUT - GR::OB;
-    T t[K * D3];
-    ld16(t, grow + size_t(C) * PC::OUT + size_t(4 * cb) * D3, false);
+    constexpr int L1 = PC::L1, L2 = PC::L2, L3 = PC::L3, D1 = PC::D1, D3 = PC::D3;
+    constexpr int XO = L1 * L1 - GR::XB, PW = P - GR::PB;
+    T g[K][D3];
+    {
+      T t4[K * D3];
+      lds16(t4, sg + size_t(C) * (PC::OUT - GR::OB) + size_t(4 * cb) * D3);
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int m = 0; m < D3; ++m) g[k][m] = t4[k * D3 + m];
+    }
+    const T al = T(alpha[P]);
+    T wa[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) wa[k] = al * wr[k][PW];
+    // t[k][m1] = sum_m3 A[m1, m3] g[k][m3]
+    T t[K][D1];
 #pragma unroll
     for (int k = 0; k < K; ++k)
 #pragma unroll
-      for (int m = 0; m < D3; ++m) gr[k][OO + m] = t[k * D3 + m];
+      for (int m1 = 0; m1 < D1; ++m1) t[k][m1] = T(0);
+    static_for<0, D3>([&](auto m3c) {
+      constexpr int M3I = decltype(m3c)::value;
+      T a[D1];
+      static_for<0, D1>([&](auto m1c) {
+        constexpr int M1I = decltype(m1c)::value;
+        if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) a[M1I] = a_entry<T, L1, L2, L3, M1I - L1, M3I - L3>(Y);
+      });
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+        static_for<0, D1>([&](auto m1c) {
+          constexpr int M1I = decltype(m1c)::value;
+          if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) t[k][M1I] = fma(a[M1I], g[k][M3I], t[k][M1I]);
+        });
+    });
+    if (gw != nullptr) {  // grad_w[e, p, u] = scale alpha_p sum_m1 x[u, m1] t[u, m1]
+      T o[K];
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        T s = T(0);
+#pragma unroll
+        for (int m1 = 0; m1 < D1; ++m1) s = fma(xr[k][XO + m1], t[k][m1], s);
+        o[k] = scale * al * s;
+      }
+      st16(gw + size_t(P) * C + 4 * cb, o);
+    }
+#pragma unroll
+    for (int k = 0; k < K; ++k)  // grad_x += alpha_p w t
+#pragma unroll
+      for (int m1 = 0; m1 < D1; ++m1) dx[k][XO + m1] = fma(wa[k], t[k][m1], dx[k][XO + m1]);
+    if (want_dy) {  // grad_y[m2] += sum_{m1,m3} C[m1,m2,m3] sum_k alpha_p w_k x_k[m1] g_k[m3]
+      T xw[K][D1];
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int m1 = 0; m1 < D1; ++m1) xw[k][m1] = wa[k] * xr[k][XO + m1];
+      static_for<0, D1>([&](auto m1c) {
+        constexpr int M1I = decltype(m1c)::value;
+        static_for<0, D3>([&](auto m3c) {
+          constexpr int M3I = decltype(m3c)::value;
+          if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) {
+            T z = T(0);
+#pragma unroll
+            for (int k = 0; k < K; ++k) z = fma(xw[k][M1I], g[k][M3I], z);
+            static_for<-L2, L2 + 1>([&](auto m2c) {
+              constexpr int M2 = decltype(m2c)::value;
+              if constexpr (cg_nz(L1, L2, L3, M1I - L1, M2, M3I - L3)) {
+                constexpr int I = cg_index(L1, L2, L3, M1I - L1, M2, M3I - L3);
+                dY[L2 * L2 + L2 + M2] = fma(CGT<T>::template get<I>(), z, dY[L2 * L2 + L2 + M2]);
+              }
+            });
+          }
+        });
+      });
+    }
   });
 }
 
-template <class CF, int GI, bool CONV>
-__device__ __forceinline__ void bwd_group(const KBwd& a, int64_t unit, unsigned char* smem_raw) {
+// Store / accumulate rules of group GI for grad_y blocks (bit l2) and grad_x blocks (bit l1).
+template <class CF, int GI>
+struct BwdMasks {
+  static constexpr unsigned y_store() {
+    unsigned m = 0;
+    for (int l = 0; l <= CF::LY; ++l) m |= (first_group_l2<CF>(l) == GI ? 1u : 0u) << l;
+    return m;
+  }
+  static constexpr unsigned y_acc() {
+    unsigned m = 0;
+    for (int l = 0; l <= CF::LY; ++l) m |= (group_has_l2<CF, GI>(l) && first_group_l2<CF>(l) != GI ? 1u : 0u) << l;
+    return m;
+  }
+  static constexpr unsigned y_zero() {
+    unsigned m = 0;
+    if (GI == 0)
+      for (int l = 0; l <= CF::LY; ++l) m |= (first_group_l2<CF>(l) < 0 ? 1u : 0u) << l;
+    return m;
+  }
+};
+
+__device__ __forceinline__ int block_of(int m) { return m >= 9 ? 3 : (m >= 4 ? 2 : (m >= 1 ? 1 : 0)); }
+
+// grad_x of one row for the group's degree blocks (first toucher stores, later groups add);
+// group 0 also zero-fills the blocks no group touches.
+template <class CF, int GI>
+__device__ __forceinline__ void bwd_put_dx(typename CF::T* __restrict__ row, const typename CF::T (&dx)[K][Grp<CF, GI>::NXG],
+                                           int C, int cb, typename CF::T scale) {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
-  const int C = a.C, CB = C >> 2;
-  const int WPG = CB >= 32 ? CB / 32 : 1;  // warps per group
-  const int NW = CF::G * WPG;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wg = warp % WPG;
-  const int cb = CB >= 32 ? wg * 32 + lane : lane % CB;
-  const int slice = CB >= 32 ? 0 : lane / CB;
-  const int NS = CB >= 32 ? 1 : 32 / CB;
-  const bool lead = CB >= 32 ? (lane == 0) : (cb == 0);  // writes the slice's grad_y partial
+  static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
+    constexpr int L = decltype(lc)::value;
+    constexpr int D = 2 * L + 1;
+    T* p = row + size_t(C) * (L * L) + size_t(4 * cb) * D;
+    T v[K * D];
+    if constexpr (first_group_l1<CF>(L) != GI) ld16(v, p, false);
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+#pragma unroll
+      for (int m = 0; m < D; ++m) {
+        const T s = scale * dx[k][L * L - GR::XB + m];
+        if constexpr (first_group_l1<CF>(L) == GI)
+          v[k * D + m] = s;
+        else
+          v[k * D + m] += s;
+      }
+    st16(p, v);
+  });
+  if constexpr (GI == 0) {
+    static_for<0, CF::LX + 1>([&](auto lc) {
+      constexpr int L = decltype(lc)::value;
+      constexpr int D = 2 * L + 1;
+      if constexpr (first_group_l1<CF>(L) < 0) {
+        T v[K * D];
+#pragma unroll
+        for (int i = 0; i < K * D; ++i) v[i] = T(0);
+        st16(row + size_t(C) * (L * L) + size_t(4 * cb) * D, v);
+      }
+    });
+  }
+}
+
+// Backward of path group GI.  Convolution: one CTA (one warp) per sender, walking its
+// out-edges through the sender CSR; tensor product: one CTA per contiguous sample range.
+template <class CF, int GI, bool CONV>
+__global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a) {
+  using T = typename CF::T;
+  using GR = Grp<CF, GI>;
+  using SM = BwdSmem<CF, GI>;
+  using MK = BwdMasks<CF, GI>;
+  constexpr int NYP = SM::NYP;
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int C = a.C, CB = C >> 2;  // CB <= 32: one warp covers every channel
+  const int lane = threadIdx.x;
+  const int cb = lane % CB, slice = lane / CB, NS = 32 / CB;
+  const int S = a.stages;
   const T* __restrict__ x = static_cast<const T*>(a.x);
   const T* __restrict__ y = static_cast<const T*>(a.y);
   const T* __restrict__ vec = static_cast<const T*>(a.vec);
@@ -817,188 +915,205 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, int64_t unit, unsigned 
   T* __restrict__ gx = static_cast<T*>(a.grad_x);
   T* __restrict__ gy = static_cast<T*>(a.grad_y);
   T* __restrict__ gwp = static_cast<T*>(a.grad_w);
-  const size_t xrow = size_t(CF::NX) * C;
-  const size_t orow = size_t(CF::NO) * C;
-  const size_t wrow = size_t(CF::P) * C;
+  const size_t xrow = size_t(CF::NX) * C, orow = size_t(CF::NO) * C, wrow = size_t(CF::P) * C;
   const T scale = T(a.scale);
   const bool want_dy = gy != nullptr;
+  const uint32_t WB = BwdSlice<CF, GI>::wbytes(C), GB = BwdSlice<CF, GI>::gbytes(C);
+  const uint32_t XB = BwdSlice<CF, GI>::xbytes(C, CONV), SLOT = WB + GB + XB;
+  const size_t STAGE = size_t(NS) * SLOT;
+  T* ysh = reinterpret_cast<T*>(smem + SM::ysh_off());
+  int32_t* eid = reinterpret_cast<int32_t*>(smem + SM::eid_off());
+  int32_t* did = reinterpret_cast<int32_t*>(smem + SM::did_off());
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::bar_off());
+  unsigned char* stages = smem + SM::stage_off(S);
 
-  // smem: dys[BWD_WINDOW * NS][NW][NY] grad_y partials, eidx[BWD_WINDOW * NS] edge ids,
-  //       dxs[NSX][NX * C] grad_x rows (NSX = 1 for the convolution, NS for the product)
-  const int NSLOT = BWD_WINDOW * NS;
-  T* dys = reinterpret_cast<T*>(smem_raw);
-  int64_t* eidx = reinterpret_cast<int64_t*>(dys + size_t(NSLOT) * NW * CF::NY);
-  T* dxs = reinterpret_cast<T*>(eidx + NSLOT);
-
-  BwdPart<CF, GI> bp;
-  T xr[K][GR::NXG], wr[K][GR::NP], Y[CF::NY], gr[K][GR::NOG], dY[CF::NY];
-
-  // flush the grad_y partials of the current window: sum over warps in a fixed order
-  auto flush_dy = [&](int nslots) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < nslots * CF::NY; i += blockDim.x) {
-      const int sl = i / CF::NY, m = i % CF::NY;
-      const int64_t e = eidx[sl];
-      if (e < 0) continue;
-      T s = T(0);
-      for (int ww = 0; ww < NW; ++ww) s += dys[(size_t(sl) * NW + ww) * CF::NY + m];
-      gy[e * CF::NY + m] = scale * s;
-    }
-    __syncthreads();
-  };
-  auto put_dy = [&](int sl, int64_t e) {
-    // reduce over the channel lanes of this slice (butterfly), leader stores
-    if (want_dy) {
-      const int lim = CB >= 32 ? 32 : CB;
-      for (int off = 1; off < lim; off <<= 1)
-#pragma unroll
-        for (int i = 0; i < CF::NY; ++i) dY[i] += __shfl_xor_sync(0xffffffffu, dY[i], off);
-      if (lead) {
-#pragma unroll
-        for (int i = 0; i < CF::NY; ++i) dys[(size_t(sl) * NW + warp) * CF::NY + i] = dY[i];
-        if (warp == 0) eidx[sl] = e;
-      }
-    }
-  };
-
+  int64_t j0, j1;
+  const int64_t n = blockIdx.x;
   if constexpr (CONV) {
-    const int64_t n = unit;
-    int64_t j0 = a.row_ptr_src[n], j1 = a.row_ptr_src[n + 1];
+    j0 = a.row_ptr_src[n];
+    j1 = a.row_ptr_src[n + 1];
     if (j0 < 0 || j1 < j0 || j1 > a.n_edges) {
-      if (threadIdx.x == 0) record_error(a.status, E3_ERR_INDEX);
+      if (lane == 0) record_error(a.status, E3_ERR_INDEX);
       j0 = j1 = 0;
     }
-    bp.zero();
-    load_x<CF, GR>(xr, x + size_t(n) * xrow, C, cb);
-    const int64_t deg = j1 - j0;
-    const int64_t steps = (deg + NS - 1) / NS;
-    for (int64_t st0 = 0; st0 < steps; st0 += BWD_WINDOW) {
-      const int nst = int(steps - st0 < BWD_WINDOW ? steps - st0 : BWD_WINDOW);
-      for (int si = 0; si < nst; ++si) {
-        const int64_t jj = (st0 + si) * NS + slice;
-        const int sl = si * NS + slice;
-        int64_t e = -1;
-        bool ok = jj < deg;
-        int32_t d = 0;
-        if (ok) {
-          e = __ldg(a.perm_src + j0 + jj);
-          if (e < 0 || e >= a.n_edges) {
-            ok = false;
-            e = -1;
-            record_error(a.status, E3_ERR_INDEX);
-          } else {
-            d = __ldg(a.dst + e);
-            if (uint32_t(d) >= uint32_t(a.n_nodes)) {
-              ok = false;
-              e = -1;
-              record_error(a.status, E3_ERR_INDEX);
-            }
-          }
-        }
-        if (ok) {
-          load_w<GR>(wr, w + e * wrow, C, cb);
-          load_y<CF>(Y, y, vec, a.sh_norm, e);
-          load_g<CF, GR>(gr, g + size_t(d) * orow, C, cb);
-          bp.edge(xr, wr, Y, gr, dY, want_dy, gwp ? gwp + e * wrow : nullptr, C, cb, a.alpha, scale);
-        } else {
+  } else {
+    const int64_t per = (a.n_nodes + a.n_chunks - 1) / a.n_chunks;
+    j0 = n * per;
+    j1 = j0 + per < a.n_nodes ? j0 + per : a.n_nodes;
+    if (j0 > j1) j0 = j1;
+  }
+  if (lane == 0) {
+    for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  T xr[K][GR::NXG], dx[K][GR::NXG], wr[K][GR::NP], Y[CF::NY], dY[CF::NY];
 #pragma unroll
-          for (int i = 0; i < CF::NY; ++i) dY[i] = T(0);
-        }
-        put_dy(sl, e);
+  for (int k = 0; k < K; ++k)
+#pragma unroll
+    for (int j = 0; j < GR::NXG; ++j) dx[k][j] = T(0);
+  if constexpr (CONV) load_x<CF, GR>(xr, x + size_t(n) * xrow, C, cb);
+
+  uint32_t issued = 0, consumed = 0;
+  bool alive = true;
+  const int64_t deg = j1 - j0;
+  for (int64_t ws = 0; ws < deg && alive; ws += BWD_WIN) {
+    const int cnt = int(deg - ws < BWD_WIN ? deg - ws : BWD_WIN);
+    for (int i = lane; i < cnt; i += 32) {
+      int64_t e = j0 + ws + i;
+      int64_t d = e;
+      bool ok = true;
+      if constexpr (CONV) {
+        e = __ldg(a.perm_src + e);
+        ok = e >= 0 && e < a.n_edges;
+        d = ok ? __ldg(a.dst + e) : 0;
+        ok = ok && d >= 0 && d < a.n_nodes;
+        if (!ok) record_error(a.status, E3_ERR_INDEX);
       }
-      if (want_dy) flush_dy(nst * NS);
+      eid[i] = ok ? int32_t(e) : -1;
+      did[i] = ok ? int32_t(d) : 0;
+      T Yl[CF::NY];
+      if (ok) {
+        load_y<CF>(Yl, y, vec, a.sh_norm, e);
+      } else {
+#pragma unroll
+        for (int m = 0; m < CF::NY; ++m) Yl[m] = T(0);
+      }
+#pragma unroll
+      for (int m = 0; m < CF::NY; ++m) ysh[i * NYP + m] = Yl[m];
     }
-    // grad_x: sum slices (butterfly), then groups in order through shared memory
-    if (gx != nullptr) {
-      if (CB < 32) {
-        for (int off = CB; off < 32; off <<= 1)
-#pragma unroll
-          for (int k = 0; k < K; ++k)
-#pragma unroll
-            for (int j = 0; j < GR::NXG; ++j) bp.dx[k][j] += __shfl_xor_sync(0xffffffffu, bp.dx[k][j], off);
+    __syncthreads();
+    const int steps = (cnt + NS - 1) / NS;
+    auto issue = [&](int st) {  // thread 0 only
+      const uint32_t slot = issued % S;
+      uint64_t* bar = &bars[slot];
+      unsigned char* dst = stages + size_t(slot) * STAGE;
+      uint32_t bytes = 0;
+      for (int j = 0; j < NS; ++j) {
+        const int r = st * NS + j;
+        if (r < cnt && eid[r] >= 0) bytes += SLOT;
       }
-      for (int i = threadIdx.x; i < CF::NX * C; i += blockDim.x) dxs[i] = T(0);
-      for (int gg = 0; gg < CF::G; ++gg) {
-        __syncthreads();
-        if (gg == GI && slice == 0) {
+      mbar_arrive_expect_tx(bar, bytes);
+      for (int j = 0; j < NS; ++j) {
+        const int r = st * NS + j;
+        if (r >= cnt) break;
+        if (eid[r] < 0) continue;
+        const int64_t e = eid[r];
+        unsigned char* d = dst + size_t(j) * SLOT;
+        bulk_load(d, w + e * wrow + size_t(GR::PB) * C, WB, bar);
+        bulk_load(d + WB, g + size_t(did[r]) * orow + size_t(GR::OB) * C, GB, bar);
+        if constexpr (!CONV) bulk_load(d + WB + GB, x + size_t(e) * xrow + size_t(GR::XB) * C, XB, bar);
+      }
+      ++issued;
+    };
+    if (lane == 0)
+      for (int st = 0; st < S && st < steps; ++st) issue(st);
+    else
+      issued += uint32_t(S < steps ? S : steps);
+
+    for (int st = 0; st < steps; ++st) {
+      const uint32_t slot = consumed % S, parity = (consumed / S) & 1u;
+      const bool ok = mbar_wait(&bars[slot], parity, a.status);
+      if (__syncthreads_or(!ok)) {
+        alive = false;
+        break;
+      }
+      ++consumed;
+      const int r = st * NS + slice;
+      const bool mine = r < cnt && eid[r] >= 0;
+      const int64_t e = mine ? eid[r] : 0;
+      if (mine) {
+        const T* sl = reinterpret_cast<const T*>(stages + size_t(slot) * STAGE + size_t(slice) * SLOT);
+#pragma unroll
+        for (int q = 0; q < GR::NP; ++q) {
+          T t4[K];
+          lds16(t4, sl + size_t(q) * C + 4 * cb);
+#pragma unroll
+          for (int k = 0; k < K; ++k) wr[k][q] = t4[k];
+        }
+        if constexpr (!CONV) {
+          const T* xs = sl + (WB + GB) / sizeof(T);
           static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
             constexpr int L = decltype(lc)::value;
             constexpr int D = 2 * L + 1;
+            T t[K * D];
+            lds16(t, xs + size_t(C) * (L * L - GR::XB) + size_t(4 * cb) * D);
 #pragma unroll
             for (int k = 0; k < K; ++k)
 #pragma unroll
-              for (int m = 0; m < D; ++m) dxs[C * (L * L) + (4 * cb + k) * D + m] += bp.dx[k][L * L - GR::XB + m];
+              for (int m = 0; m < D; ++m) xr[k][L * L - GR::XB + m] = t[k * D + m];
           });
+#pragma unroll
+          for (int k = 0; k < K; ++k)
+#pragma unroll
+            for (int j = 0; j < GR::NXG; ++j) dx[k][j] = T(0);
         }
-      }
-      __syncthreads();
-      for (int i = threadIdx.x; i < CF::NX * C; i += blockDim.x) gx[size_t(n) * xrow + i] = scale * dxs[i];
-    }
-  } else {
-    // tensor product: slice = sample within the step; NS samples per step
-    const int64_t n_units = (a.n_nodes + NS - 1) / NS;
-    for (int64_t u = unit; u < n_units; u += a.n_chunks) {
-      const int64_t b = u * NS + slice;
-      const bool ok = b < a.n_nodes;
-      bp.zero();
-      if (ok) {
-        load_x<CF, GR>(xr, x + size_t(b) * xrow, C, cb);
-        load_w<GR>(wr, w + b * wrow, C, cb);
-        load_y<CF>(Y, y, vec, a.sh_norm, b);
-        load_g<CF, GR>(gr, g + size_t(b) * orow, C, cb);
-        bp.edge(xr, wr, Y, gr, dY, want_dy, gwp ? gwp + b * wrow : nullptr, C, cb, a.alpha, scale);
+        {
+          T yp[NYP];
+          lds16(yp, ysh + r * NYP);
+#pragma unroll
+          for (int m = 0; m < CF::NY; ++m) Y[m] = yp[m];
+        }
+        bwd_edge<CF, GI>(xr, wr, Y, sl + WB / sizeof(T), dx, dY, want_dy, gwp ? gwp + e * wrow : nullptr, C, cb,
+                         a.alpha, scale);
       } else {
 #pragma unroll
-        for (int i = 0; i < CF::NY; ++i) dY[i] = T(0);
+        for (int m = 0; m < CF::NY; ++m) dY[m] = T(0);
       }
-      put_dy(slice, ok ? b : -1);
-      if (want_dy) flush_dy(NS);
-      if (gx != nullptr) {
-        for (int i = threadIdx.x; i < NS * CF::NX * C; i += blockDim.x) dxs[i] = T(0);
-        for (int gg = 0; gg < CF::G; ++gg) {
-          __syncthreads();
-          if (gg == GI) {
-            static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
-              constexpr int L = decltype(lc)::value;
-              constexpr int D = 2 * L + 1;
+      if (want_dy) {
+        // sum over the channel lanes of the slice (fixed butterfly), then lane cb writes
+        // components cb, cb + CB, ... of its slice's edge
+        for (int off = 1; off < CB; off <<= 1)
 #pragma unroll
-              for (int k = 0; k < K; ++k)
+          for (int m = 0; m < CF::NY; ++m) dY[m] += __shfl_xor_sync(0xffffffffu, dY[m], off);
+        if (mine) {
 #pragma unroll
-                for (int m = 0; m < D; ++m)
-                  dxs[size_t(slice) * CF::NX * C + C * (L * L) + (4 * cb + k) * D + m] += bp.dx[k][L * L - GR::XB + m];
-            });
+          for (int m = 0; m < CF::NY; ++m) {
+            if ((m - cb) % CB != 0 || m < cb) continue;
+            const unsigned bit = 1u << block_of(m);
+            T* p = gy + e * CF::NY + m;
+            if (MK::y_store() & bit)
+              *p = scale * dY[m];
+            else if (MK::y_acc() & bit)
+              *p += scale * dY[m];
+            else if (MK::y_zero() & bit)
+              *p = T(0);
           }
         }
-        __syncthreads();
-        for (int i = threadIdx.x; i < NS * CF::NX * C; i += blockDim.x) {
-          const int64_t bb = u * NS + i / (CF::NX * C);
-          if (bb < a.n_nodes) gx[size_t(bb) * xrow + i % (CF::NX * C)] = scale * dxs[i];
-        }
-        __syncthreads();
+      }
+      if constexpr (!CONV) {
+        if (mine && gx != nullptr) bwd_put_dx<CF, GI>(gx + size_t(e) * xrow, dx, C, cb, scale);
+      }
+      __syncthreads();
+      if (st + S < steps) {
+        if (lane == 0)
+          issue(st + S);
+        else
+          ++issued;
       }
     }
+    __syncthreads();
   }
-}
-
-template <class CF, bool CONV>
-__global__ void __launch_bounds__(320) bwd_kernel(const __grid_constant__ KBwd a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int C = a.C, CB = C >> 2;
-  const int WPG = CB >= 32 ? CB / 32 : 1;
-  const int gi = int(threadIdx.x >> 5) / WPG;
-  dispatch<CF::G>(gi, [&](auto g) { bwd_group<CF, decltype(g)::value, CONV>(a, blockIdx.x, smem_raw); });
-}
-
-template <class CF>
-static size_t bwd_smem_bytes(int C, bool conv) {
-  using T = typename CF::T;
-  const int CB = C / 4;
-  const int WPG = CB >= 32 ? CB / 32 : 1, NS = CB >= 32 ? 1 : 32 / CB;
-  const int NW = CF::G * WPG, NSLOT = BWD_WINDOW * NS;
-  size_t b = sizeof(T) * size_t(NSLOT) * NW * CF::NY + sizeof(int64_t) * NSLOT;
-  b = (b + 15) & ~size_t(15);
-  b += sizeof(T) * size_t(conv ? 1 : NS) * CF::NX * C;
-  return b;
+  if (!alive) {
+    if (lane == 0)
+      while (consumed < issued) {
+        mbar_wait(&bars[consumed % S], (consumed / S) & 1u, a.status);
+        ++consumed;
+      }
+    __syncthreads();
+    return;
+  }
+  if constexpr (CONV) {
+    if (gx != nullptr) {
+      for (int off = CB; off < 32; off <<= 1)
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+#pragma unroll
+          for (int j = 0; j < GR::NXG; ++j) dx[k][j] += __shfl_xor_sync(0xffffffffu, dx[k][j], off);
+      if (slice == 0) bwd_put_dx<CF, GI>(gx + size_t(n) * xrow, dx, C, cb, scale);
+    }
+  }
 }
 
 // =================================================================== host launchers ===
@@ -1056,6 +1171,43 @@ e3_status launch_fwd_cfg(const e3_plan* plan, const FwdArgs& h, bool conv) {
   return E3_OK;
 }
 
+// One backward launch per path group, in group order on the caller's stream: a launch only
+// holds its group's code, and grad_x / grad_y blocks shared by several groups are stored by
+// the first and accumulated by the later launches (fixed order: deterministic).
+template <class CF, int GI>
+e3_status launch_bwd_group(KBwd a, bool conv, int64_t blocks, cudaStream_t s) {
+  const int CB = a.C / 4, NS = 32 / CB;
+  auto kern = conv ? bwd_kernel<CF, GI, true> : bwd_kernel<CF, GI, false>;
+  cudaFuncAttributes fa{};
+  cudaError_t err = cudaFuncGetAttributes(&fa, kern);
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(err));
+  const int regs = fa.numRegs > 0 ? fa.numRegs : 255;
+  const int ctas = std::max(1, std::min(32, 65536 / (((regs + 7) & ~7) * 32)));
+  const size_t budget = size_t(225) * 1024 / ctas;
+  int S = 3;
+  while (S > 2 && BwdSmem<CF, GI>::total(a.C, NS, S, conv) + 1024 > budget) --S;
+  a.stages = S;
+  const size_t smem = BwdSmem<CF, GI>::total(a.C, NS, S, conv);
+  if (smem > size_t(227) * 1024) return fail(E3_ERR_UNSUPPORTED, "backward needs %zu bytes of shared memory", smem);
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
+  kern<<<unsigned(blocks), 32, smem, s>>>(a);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "backward launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+template <class CF, int GI = 0>
+e3_status launch_bwd_groups(const KBwd& a, bool conv, int64_t blocks, cudaStream_t s) {
+  if constexpr (GI < CF::G) {
+    const e3_status st = launch_bwd_group<CF, GI>(a, conv, blocks, s);
+    if (st != E3_OK) return st;
+    return launch_bwd_groups<CF, GI + 1>(a, conv, blocks, s);
+  } else {
+    return E3_OK;
+  }
+}
+
 template <class CF>
 e3_status launch_bwd_cfg(const e3_plan* plan, const BwdArgs& h, bool conv) {
   KBwd a{};
@@ -1079,12 +1231,8 @@ e3_status launch_bwd_cfg(const e3_plan* plan, const BwdArgs& h, bool conv) {
   if (st != E3_OK) return st;
   for (int p = 0; p < plan->n_paths; ++p) a.alpha[p] = plan->alpha[p];
   const int CB = plan->C / 4;
-  const int WPG = CB >= 32 ? CB / 32 : 1;
-  const int NS = CB >= 32 ? 1 : 32 / CB;
-  const int threads = 32 * WPG * CF::G;
-  if (threads > 320) return fail(E3_ERR_UNSUPPORTED, "backward needs %d threads per CTA (max 320)", threads);
-  const size_t smem = bwd_smem_bytes<CF>(plan->C, conv);
-  if (smem > 200 * 1024) return fail(E3_ERR_UNSUPPORTED, "backward needs %zu bytes of shared memory", smem);
+  if (CB > 32) return fail(E3_ERR_UNSUPPORTED, "the backward kernels need a multiplicity of at most 128");
+  const int NS = 32 / CB;
   int64_t blocks;
   if (conv) {
     blocks = h.n_nodes;
@@ -1095,20 +1243,9 @@ e3_status launch_bwd_cfg(const e3_plan* plan, const BwdArgs& h, bool conv) {
     a.n_chunks = int(blocks);
   }
   if (blocks >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "grid too large");
-  cudaStream_t s = static_cast<cudaStream_t>(h.stream);
-  cudaError_t err;
-  if (conv) {
-    err = cudaFuncSetAttribute(bwd_kernel<CF, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (err == cudaSuccess) bwd_kernel<CF, true><<<unsigned(blocks), threads, smem, s>>>(a);
-  } else {
-    err = cudaFuncSetAttribute(bwd_kernel<CF, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (err == cudaSuccess) bwd_kernel<CF, false><<<unsigned(blocks), threads, smem, s>>>(a);
-  }
-  if (err == cudaSuccess) err = cudaGetLastError();
-  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "backward launch failed: %s", cudaGetErrorString(err));
-  return E3_OK;
+  if (blocks == 0) return E3_OK;
+  return launch_bwd_groups<CF>(a, conv, blocks, static_cast<cudaStream_t>(h.stream));
 }
-
 
 // Fill this unit's copy of the coefficient tables on the current device.
 static inline cudaError_t upload_tables(const double* t64, const float* t32) {
