@@ -47,16 +47,29 @@ E3_HD constexpr int cg_block_nnz(int l1, int l2, int l3) {
   return n;
 }
 
-// Offset of block (l1, l2, l3) in the packed table; (E3_LMAX+1, 0, 0) gives the table size.
-E3_HD constexpr int cg_block_offset(int l1, int l2, int l3) {
+// Offsets of every block in the packed table, computed once (blocks in lexicographic
+// (l1, l2, l3) order over triangle-valid triples; `total` is the table size).
+struct CGOffsetTable {
+  int off[E3_LMAX + 1][E3_LMAX + 1][E3_LMAX + 1];
+  int total;
+};
+E3_HD constexpr CGOffsetTable make_cg_offsets() {
+  CGOffsetTable t{};
   int off = 0;
   for (int a = 0; a <= E3_LMAX; ++a)
     for (int b = 0; b <= E3_LMAX; ++b)
       for (int c = 0; c <= E3_LMAX; ++c) {
-        if (a == l1 && b == l2 && c == l3) return off;
+        t.off[a][b][c] = off;
         if (triangle(a, b, c)) off += cg_block_nnz(a, b, c);
       }
-  return off;
+  t.total = off;
+  return t;
+}
+constexpr CGOffsetTable kCGOffsets = make_cg_offsets();
+
+// Offset of block (l1, l2, l3) in the packed table; (E3_LMAX+1, 0, 0) gives the table size.
+E3_HD constexpr int cg_block_offset(int l1, int l2, int l3) {
+  return l1 > E3_LMAX ? kCGOffsets.total : kCGOffsets.off[l1][l2][l3];
 }
 
 constexpr int CG_TABLE_SIZE = cg_block_offset(E3_LMAX + 1, 0, 0);
@@ -162,6 +175,41 @@ E3_HD constexpr int n_groups(int LX, int LY, int LO) { return group_scan(LX, LY,
 // First path of group g (g = n_groups gives n_paths).
 E3_HD constexpr int group_begin(int LX, int LY, int LO, int g) {
   return g <= 0 ? 0 : group_scan(LX, LY, LO, g, false);
+}
+
+// Everything the kernels need to know about a path set, computed once per (LX, LY, LO).
+constexpr int MAX_PATHS = 64;
+struct PathTable {
+  int n, ngroups, out_dim;
+  int l1[MAX_PATHS], l2[MAX_PATHS], l3[MAX_PATHS];
+  int out_off[MAX_PATHS + 1];
+  int gbegin[MAX_PATHS + 1];
+};
+E3_HD constexpr PathTable make_path_table(int LX, int LY, int LO) {
+  PathTable t{};
+  for (int l1 = 0; l1 <= LX; ++l1)
+    for (int l2 = 0; l2 <= LY; ++l2)
+      for (int l3 = iabs(l1 - l2); l3 <= l1 + l2 && l3 <= LO; ++l3) {
+        t.l1[t.n] = l1;
+        t.l2[t.n] = l2;
+        t.l3[t.n] = l3;
+        t.out_off[t.n + 1] = t.out_off[t.n] + 2 * l3 + 1;
+        ++t.n;
+      }
+  t.out_dim = t.out_off[t.n];
+  int outs = 0;
+  t.gbegin[0] = 0;
+  t.ngroups = 1;
+  for (int p = 0; p < t.n; ++p) {
+    const int d = 2 * t.l3[p] + 1;
+    if (outs > 0 && outs + d > GROUP_OUT_CAP) {
+      t.gbegin[t.ngroups++] = p;
+      outs = 0;
+    }
+    outs += d;
+  }
+  t.gbegin[t.ngroups] = t.n;
+  return t;
 }
 
 }  // namespace e3b

@@ -91,36 +91,36 @@ template <int LX_, int LY_, int LO_, typename T_>
 struct Cfg {
   static constexpr int LX = LX_, LY = LY_, LO = LO_;
   using T = T_;
-  static constexpr int P = n_paths(LX, LY, LO);
-  static constexpr int G = n_groups(LX, LY, LO);
+  static constexpr PathTable PT = make_path_table(LX, LY, LO);
+  static constexpr int P = PT.n;
+  static constexpr int G = PT.ngroups;
   static constexpr int NY = (LY + 1) * (LY + 1);
   static constexpr int NX = (LX + 1) * (LX + 1);
-  static constexpr int NO = out_dim_per_channel(LX, LY, LO);
+  static constexpr int NO = PT.out_dim;
   static_assert(P <= MAXP, "too many paths");
 };
 
 template <class CF, int GI>
 struct Grp {
-  static constexpr int LX = CF::LX, LY = CF::LY, LO = CF::LO;
-  static constexpr int PB = group_begin(LX, LY, LO, GI);
-  static constexpr int PE = group_begin(LX, LY, LO, GI + 1);
+  static constexpr int PB = CF::PT.gbegin[GI];
+  static constexpr int PE = CF::PT.gbegin[GI + 1];
   static constexpr int NP = PE - PB;
   static_assert(NP >= 1, "empty path group");
-  static constexpr int L1A = path_l(LX, LY, LO, PB, 0);
-  static constexpr int L1B = path_l(LX, LY, LO, PE - 1, 0);
+  static constexpr int L1A = CF::PT.l1[PB];
+  static constexpr int L1B = CF::PT.l1[PE - 1];
   static constexpr int XB = L1A * L1A;                    // first per-channel x index used
   static constexpr int NXG = (L1B + 1) * (L1B + 1) - XB;  // per-channel x values used
-  static constexpr int OB = path_out_off(LX, LY, LO, PB);
-  static constexpr int NOG = path_out_off(LX, LY, LO, PE) - OB;
+  static constexpr int OB = CF::PT.out_off[PB];
+  static constexpr int NOG = CF::PT.out_off[PE] - OB;
 };
 
 template <class CF, int P>
 struct PathC {
-  static constexpr int L1 = path_l(CF::LX, CF::LY, CF::LO, P, 0);
-  static constexpr int L2 = path_l(CF::LX, CF::LY, CF::LO, P, 1);
-  static constexpr int L3 = path_l(CF::LX, CF::LY, CF::LO, P, 2);
+  static constexpr int L1 = CF::PT.l1[P];
+  static constexpr int L2 = CF::PT.l2[P];
+  static constexpr int L3 = CF::PT.l3[P];
   static constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1;
-  static constexpr int OUT = path_out_off(CF::LX, CF::LY, CF::LO, P);  // per-channel offset
+  static constexpr int OUT = CF::PT.out_off[P];  // per-channel offset
 };
 
 // A_p[m1, m3] for one (m1, m3): sum over the pattern m2 of C[m1, m2, m3] * Y[l2, m2].
@@ -685,21 +685,21 @@ struct KBwd {
 template <class CF>
 __host__ __device__ constexpr int first_group_l1(int l) {
   for (int g = 0; g < CF::G; ++g)
-    for (int p = group_begin(CF::LX, CF::LY, CF::LO, g); p < group_begin(CF::LX, CF::LY, CF::LO, g + 1); ++p)
-      if (path_l(CF::LX, CF::LY, CF::LO, p, 0) == l) return g;
+    for (int p = CF::PT.gbegin[g]; p < CF::PT.gbegin[g + 1]; ++p)
+      if (CF::PT.l1[p] == l) return g;
   return -1;
 }
 template <class CF>
 __host__ __device__ constexpr int first_group_l2(int l) {
   for (int g = 0; g < CF::G; ++g)
-    for (int p = group_begin(CF::LX, CF::LY, CF::LO, g); p < group_begin(CF::LX, CF::LY, CF::LO, g + 1); ++p)
-      if (path_l(CF::LX, CF::LY, CF::LO, p, 1) == l) return g;
+    for (int p = CF::PT.gbegin[g]; p < CF::PT.gbegin[g + 1]; ++p)
+      if (CF::PT.l2[p] == l) return g;
   return -1;
 }
 template <class CF, int GI>
 __host__ __device__ constexpr bool group_has_l2(int l) {
-  for (int p = group_begin(CF::LX, CF::LY, CF::LO, GI); p < group_begin(CF::LX, CF::LY, CF::LO, GI + 1); ++p)
-    if (path_l(CF::LX, CF::LY, CF::LO, p, 1) == l) return true;
+  for (int p = CF::PT.gbegin[GI]; p < CF::PT.gbegin[GI + 1]; ++p)
+    if (CF::PT.l2[p] == l) return true;
   return false;
 }
 
@@ -741,7 +741,7 @@ struct BwdSmem {
 // unreduced grad_y contribution in dY and writes grad_w (scaled) when gw != nullptr.
 template <class CF, int GI>
 __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, GI>::NXG],
-                                         const typename CF::T (&wr)[K][Grp<CF, GI>::NP],
+                                         const typename CF::T* sw,
                                          const typename CF::T (&Y)[CF::NY], const typename CF::T* sg,
                                          typename CF::T (&dx)[K][Grp<CF, GI>::NXG], typename CF::T (&dY)[CF::NY],
                                          bool want_dy, typename CF::T* __restrict__ gw, int C, int cb,
@@ -755,6 +755,8 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
     using PC = PathC<CF, P>;
     constexpr int L1 = PC::L1, L2 = PC::L2, L3 = PC::L3, D1 = PC::D1, D3 = PC::D3;
     constexpr int XO = L1 * L1 - GR::XB, PW = P - GR::PB;
+    T wk[K];
+    lds16(wk, sw + size_t(PW) * C + 4 * cb);
     T g[K][D3];
     {
       T t4[K * D3];
@@ -767,7 +769,7 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
     const T al = T(alpha[P]);
     T wa[K];
 #pragma unroll
-    for (int k = 0; k < K; ++k) wa[k] = al * wr[k][PW];
+    for (int k = 0; k < K; ++k) wa[k] = al * wk[k];
     // t[k][m1] = sum_m3 A[m1, m3] g[k][m3]
     T t[K][D1];
 #pragma unroll
@@ -804,6 +806,9 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
 #pragma unroll
       for (int m1 = 0; m1 < D1; ++m1) dx[k][XO + m1] = fma(wa[k], t[k][m1], dx[k][XO + m1]);
     if (want_dy) {  // grad_y[m2] += sum_{m1,m3} C[m1,m2,m3] sum_k alpha_p w_k x_k[m1] g_k[m3]
+      T dyp[2 * L2 + 1];
+#pragma unroll
+      for (int i = 0; i < 2 * L2 + 1; ++i) dyp[i] = T(0);
       T xw[K][D1];
 #pragma unroll
       for (int k = 0; k < K; ++k)
@@ -821,35 +826,83 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
               constexpr int M2 = decltype(m2c)::value;
               if constexpr (cg_nz(L1, L2, L3, M1I - L1, M2, M3I - L3)) {
                 constexpr int I = cg_index(L1, L2, L3, M1I - L1, M2, M3I - L3);
-                dY[L2 * L2 + L2 + M2] = fma(CGT<T>::template get<I>(), z, dY[L2 * L2 + L2 + M2]);
+                dyp[L2 + M2] = fma(CGT<T>::template get<I>(), z, dyp[L2 + M2]);
               }
             });
           }
         });
       });
+#pragma unroll
+      for (int i = 0; i < 2 * L2 + 1; ++i) dY[L2 * L2 + i] += dyp[i];
     }
   });
+}
+
+// grad_y components that group GI produces: every component of each harmonics block l2 that
+// one of its paths uses, ascending; VP = that count rounded up to a power of two.
+template <class CF, int GI>
+struct YUse {
+  struct Tab {
+    int n;
+    int comp[16];
+  };
+  static constexpr Tab make() {
+    Tab t{};
+    for (int l = 0; l <= CF::LY; ++l)
+      if (group_has_l2<CF, GI>(l))
+        for (int i = 0; i < 2 * l + 1; ++i) t.comp[t.n++] = l * l + i;
+    return t;
+  }
+  static constexpr Tab TAB = make();
+  static constexpr int NU = TAB.n;
+  static constexpr int VP = NU <= 1 ? 1 : (NU <= 2 ? 2 : (NU <= 4 ? 4 : (NU <= 8 ? 8 : 16)));
+};
+
+// Sum v[0..VP) over the W lanes of a slice (lane bits below W) by recursive halving: after
+// each level a lane keeps half of its values and adds its partner's copy of that half.  On
+// return v[0..max(VP/W, 1)) hold totals of components base + j (same base for lanes that
+// differ only in the bits below W/VP when VP < W).
+template <typename T, int VP>
+__device__ __forceinline__ int reduce_scatter(T (&v)[VP], int W, int cb) {
+  int base = 0;
+  int len = VP;
+#pragma unroll
+  for (int lvl = 0; lvl < 5; ++lvl) {
+    const int o = W >> (lvl + 1);
+    if (o < 1) break;
+    const bool up = (cb & o) != 0;
+    if (len > 1) {
+      const int half = len / 2;
+#pragma unroll
+      for (int i = 0; i < VP / 2; ++i) {
+        if (i >= half) break;
+        const T send = up ? v[i] : v[i + half];
+        const T keep = up ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+      if (up) base += half;
+      len = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    }
+  }
+  return base;
 }
 
 // Store / accumulate rules of group GI for grad_y blocks (bit l2) and grad_x blocks (bit l1).
 template <class CF, int GI>
 struct BwdMasks {
-  static constexpr unsigned y_store() {
+  static constexpr unsigned YS = [] {
     unsigned m = 0;
     for (int l = 0; l <= CF::LY; ++l) m |= (first_group_l2<CF>(l) == GI ? 1u : 0u) << l;
     return m;
-  }
-  static constexpr unsigned y_acc() {
-    unsigned m = 0;
-    for (int l = 0; l <= CF::LY; ++l) m |= (group_has_l2<CF, GI>(l) && first_group_l2<CF>(l) != GI ? 1u : 0u) << l;
-    return m;
-  }
-  static constexpr unsigned y_zero() {
+  }();
+  static constexpr unsigned YZ = [] {
     unsigned m = 0;
     if (GI == 0)
       for (int l = 0; l <= CF::LY; ++l) m |= (first_group_l2<CF>(l) < 0 ? 1u : 0u) << l;
     return m;
-  }
+  }();
 };
 
 __device__ __forceinline__ int block_of(int m) { return m >= 9 ? 3 : (m >= 4 ? 2 : (m >= 1 ? 1 : 0)); }
@@ -948,7 +1001,7 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
   }
   __syncthreads();
 
-  T xr[K][GR::NXG], dx[K][GR::NXG], wr[K][GR::NP], Y[CF::NY], dY[CF::NY];
+  T xr[K][GR::NXG], dx[K][GR::NXG], Y[CF::NY], dY[CF::NY];
 #pragma unroll
   for (int k = 0; k < K; ++k)
 #pragma unroll
@@ -1025,13 +1078,6 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
       const int64_t e = mine ? eid[r] : 0;
       if (mine) {
         const T* sl = reinterpret_cast<const T*>(stages + size_t(slot) * STAGE + size_t(slice) * SLOT);
-#pragma unroll
-        for (int q = 0; q < GR::NP; ++q) {
-          T t4[K];
-          lds16(t4, sl + size_t(q) * C + 4 * cb);
-#pragma unroll
-          for (int k = 0; k < K; ++k) wr[k][q] = t4[k];
-        }
         if constexpr (!CONV) {
           const T* xs = sl + (WB + GB) / sizeof(T);
           static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
@@ -1055,30 +1101,52 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
 #pragma unroll
           for (int m = 0; m < CF::NY; ++m) Y[m] = yp[m];
         }
-        bwd_edge<CF, GI>(xr, wr, Y, sl + WB / sizeof(T), dx, dY, want_dy, gwp ? gwp + e * wrow : nullptr, C, cb,
+        bwd_edge<CF, GI>(xr, sl, Y, sl + WB / sizeof(T), dx, dY, want_dy, gwp ? gwp + e * wrow : nullptr, C, cb,
                          a.alpha, scale);
       } else {
 #pragma unroll
         for (int m = 0; m < CF::NY; ++m) dY[m] = T(0);
       }
       if (want_dy) {
-        // sum over the channel lanes of the slice (fixed butterfly), then lane cb writes
-        // components cb, cb + CB, ... of its slice's edge
-        for (int off = 1; off < CB; off <<= 1)
+        // sum the group's components over the channel lanes of the slice, then each lane
+        // writes the components it holds (first group of a block stores, later ones add)
+        using YU = YUse<CF, GI>;
+        T v[YU::VP];
+        static_for<0, YU::VP>([&](auto uc) {
+          constexpr int U = decltype(uc)::value;
+          if constexpr (U < YU::NU) {
+            constexpr int M = YU::TAB.comp[U];
+            v[U] = dY[M];
+          } else {
+            v[U] = T(0);
+          }
+        });
+        const int base = reduce_scatter<T, YU::VP>(v, CB, cb);
+        const int held = YU::VP >= CB ? YU::VP / CB : 1;
+        const bool writer = YU::VP >= CB || (cb & (CB / YU::VP - 1)) == 0;
+        if (mine && writer) {
 #pragma unroll
-          for (int m = 0; m < CF::NY; ++m) dY[m] += __shfl_xor_sync(0xffffffffu, dY[m], off);
-        if (mine) {
-#pragma unroll
-          for (int m = 0; m < CF::NY; ++m) {
-            if ((m - cb) % CB != 0 || m < cb) continue;
-            const unsigned bit = 1u << block_of(m);
+          for (int j = 0; j < YU::VP; ++j) {
+            if (j >= held) break;
+            const int u = base + j;
+            if (u >= YU::NU) break;
+            int m = 0;
+            static_for<0, YU::NU>([&](auto qc) {
+              constexpr int Q = decltype(qc)::value;
+              constexpr int MQ = YU::TAB.comp[Q];
+              if (u == Q) m = MQ;
+            });
             T* p = gy + e * CF::NY + m;
-            if (MK::y_store() & bit)
-              *p = scale * dY[m];
-            else if (MK::y_acc() & bit)
-              *p += scale * dY[m];
-            else if (MK::y_zero() & bit)
-              *p = T(0);
+            if (MK::YS & (1u << block_of(m)))
+              *p = scale * v[j];
+            else
+              *p += scale * v[j];
+          }
+          // group 0 also zero-fills harmonics blocks that no path uses
+          if constexpr (MK::YZ != 0u) {
+            if (cb == 0)
+              for (int m = 0; m < CF::NY; ++m)
+                if (MK::YZ & (1u << block_of(m))) gy[e * CF::NY + m] = T(0);
           }
         }
       }
