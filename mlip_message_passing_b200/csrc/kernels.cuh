@@ -462,7 +462,8 @@ struct FwdSmem {
   static __host__ __device__ size_t ysh_off() { return 0; }
   static __host__ __device__ size_t src_off() { return sizeof(T) * size_t(FWD_WIN) * NYP; }
   static __host__ __device__ size_t bar_off() { return src_off() + sizeof(int32_t) * FWD_WIN; }
-  static __host__ __device__ size_t stage_off(int S) { return (bar_off() + 8 * size_t(S) + 127) & ~size_t(127); }
+  static __host__ __device__ size_t flag_off(int S) { return bar_off() + 8 * size_t(S); }
+  static __host__ __device__ size_t stage_off(int S) { return (flag_off(S) + 16 + 127) & ~size_t(127); }
   static __host__ __device__ size_t stage_bytes(int C, int NS) { return size_t(NS) * max_slice_bytes<CF>(C); }
   static __host__ __device__ size_t total(int C, int NS, int S) { return stage_off(S) + size_t(S) * stage_bytes(C, NS); }
 };
@@ -514,6 +515,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
   T* ysh = reinterpret_cast<T*>(smem + SM::ysh_off());
   int32_t* src_s = reinterpret_cast<int32_t*>(smem + SM::src_off());
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::bar_off());
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SM::flag_off(S));
   unsigned char* stages = smem + SM::stage_off(S);
 
   // segment of rows handled by this CTA
@@ -533,6 +535,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
   }
   if (tid == 0) {
     for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+    *s_abort = 0;
     mbar_fence_init();
   }
   __syncthreads();
@@ -540,8 +543,9 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
   FwdAcc<CF, GI> f;
   f.zero();
   T xr[K][GR::NXG], wr[K][GR::NP], Y[CF::NY];
-  uint32_t issued = 0;  // steps issued so far (all windows), drives stage index and parity
-  uint32_t consumed = 0;
+  // ring state: identical in every thread, advanced uniformly
+  int prod_slot = 0, cons_slot = 0;
+  uint32_t cons_phase = 0, issued = 0, consumed = 0;
   bool alive = true;
   const int64_t deg = e1 - e0;
 
@@ -550,46 +554,48 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
     fwd_stage_window<CF, CONV>(a, e0, ws, cnt, ysh, src_s);
     __syncthreads();
     const int steps = (cnt + NS - 1) / NS;
-    // producer: stage `st` of this window -> ring slot issued % S
+    // producer: warp 0; lane 0 posts the expected bytes, then lanes move one slice each
+    // (item 2j: weights of the step's j-th edge, item 2j+1: its x slice)
     auto issue = [&](int st) {
-      const uint32_t slot = issued % S;
-      uint64_t* bar = &bars[slot];
-      unsigned char* dst = stages + size_t(slot) * STAGE;
-      uint32_t bytes = 0;
-      for (int j = 0; j < NS; ++j) {
-        const int r = st * NS + j;
-        if (r < cnt && (!CONV || src_s[r] >= 0)) bytes += SLOT;
-      }
-      mbar_arrive_expect_tx(bar, bytes);
-      for (int j = 0; j < NS; ++j) {
-        const int r = st * NS + j;
-        if (r >= cnt) break;
-        const int64_t e = e0 + ws + r;
-        int64_t xr_row = e;
-        if constexpr (CONV) {
-          if (src_s[r] < 0) continue;
-          xr_row = src_s[r];
+      if (tid < 32) {
+        uint64_t* bar = &bars[prod_slot];
+        unsigned char* dst = stages + size_t(prod_slot) * STAGE;
+        int nv = 0;
+        for (int j = tid; j < NS; j += 32) {
+          const int r = st * NS + j;
+          nv += (r < cnt && (!CONV || src_s[r] >= 0)) ? 1 : 0;
         }
-        bulk_load(dst + size_t(j) * SLOT, w + e * a.w_stride + size_t(GR::PB) * C, WB, bar);
-        bulk_load(dst + size_t(j) * SLOT + WB, x + size_t(xr_row) * xrow + size_t(GR::XB) * C, XB, bar);
+        nv = __reduce_add_sync(0xffffffffu, nv);
+        if (tid == 0) mbar_arrive_expect_tx(bar, uint32_t(nv) * SLOT);
+        __syncwarp();
+        for (int it = tid; it < 2 * NS; it += 32) {
+          const int j = it >> 1;
+          const int r = st * NS + j;
+          if (r >= cnt) continue;
+          const int64_t e = e0 + ws + r;
+          if (it & 1) {
+            int64_t row = e;
+            if constexpr (CONV) row = src_s[r];
+            if (row >= 0) bulk_load(dst + size_t(j) * SLOT + WB, x + size_t(row) * xrow + size_t(GR::XB) * C, XB, bar);
+          } else if (!CONV || src_s[r] >= 0) {
+            bulk_load(dst + size_t(j) * SLOT, w + e * a.w_stride + size_t(GR::PB) * C, WB, bar);
+          }
+        }
       }
+      prod_slot = prod_slot + 1 == S ? 0 : prod_slot + 1;
       ++issued;
     };
-    if (tid == 0)
-      for (int st = 0; st < S && st < steps; ++st) issue(st);
-    // `issued` is only advanced by thread 0; every thread tracks the same count
-    if (tid != 0) issued += uint32_t(S < steps ? S : steps);
+    for (int st = 0; st < S && st < steps; ++st) issue(st);
 
     for (int st = 0; st < steps; ++st) {
-      const uint32_t slot = consumed % S, parity = (consumed / S) & 1u;
-      const bool ok = mbar_wait(&bars[slot], parity, a.status);
-      if (__syncthreads_or(!ok)) {  // uniform decision: no thread leaves the barrier loop alone
-        alive = false;
-        break;
-      }
+      const int slot = cons_slot;
+      const bool ok = mbar_wait(&bars[slot], cons_phase, a.status);
+      if (!ok) *s_abort = 1;
+      cons_slot = cons_slot + 1 == S ? 0 : cons_slot + 1;
+      if (cons_slot == 0) cons_phase ^= 1u;
       ++consumed;
       const int r = st * NS + slice;
-      const bool mine = r < cnt && (!CONV || src_s[r] >= 0);
+      const bool mine = ok && r < cnt && (!CONV || src_s[r] >= 0);
       if (mine) {
         const T* sl = reinterpret_cast<const T*>(stages + size_t(slot) * STAGE + size_t(slice) * SLOT);
         // weights of the group's paths for channels 4cb..4cb+3
@@ -621,19 +627,19 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
         f.edge(xr, wr, Y);
         if constexpr (!CONV) f.store(out + size_t(e0 + ws + r) * orow, C, cb, a.pscale);
       }
-      __syncthreads();  // every thread is done with this stage
-      if (tid == 0 && st + S < steps) issue(st + S);
-      if (tid != 0 && st + S < steps) ++issued;
+      __syncthreads();  // every thread is done with this stage (and sees an abort)
+      if (*s_abort) {
+        alive = false;
+        break;
+      }
+      if (st + S < steps) issue(st + S);
     }
     __syncthreads();  // window staging buffers are reused by the next window
   }
   if (!alive) {
     // a wait gave up: let the copies in flight land (bounded) before the CTA exits
     if (tid == 0)
-      while (consumed < issued) {
-        mbar_wait(&bars[consumed % S], (consumed / S) & 1u, a.status);
-        ++consumed;
-      }
+      for (uint32_t q = consumed - 1; q < issued; ++q) mbar_wait(&bars[q % S], (q / S) & 1u, a.status);
     __syncthreads();
     return;
   }
@@ -727,7 +733,8 @@ struct BwdSmem {
   static __host__ __device__ size_t eid_off() { return sizeof(T) * size_t(BWD_WIN) * NYP; }
   static __host__ __device__ size_t did_off() { return eid_off() + sizeof(int32_t) * BWD_WIN; }
   static __host__ __device__ size_t bar_off() { return did_off() + sizeof(int32_t) * BWD_WIN; }
-  static __host__ __device__ size_t stage_off(int S) { return (bar_off() + 8 * size_t(S) + 127) & ~size_t(127); }
+  static __host__ __device__ size_t flag_off(int S) { return bar_off() + 8 * size_t(S); }
+  static __host__ __device__ size_t stage_off(int S) { return (flag_off(S) + 16 + 127) & ~size_t(127); }
   static __host__ __device__ size_t stage_bytes(int C, int NS, bool conv) {
     return size_t(NS) * BwdSlice<CF, GI>::slot(C, conv);
   }
@@ -978,6 +985,7 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
   int32_t* eid = reinterpret_cast<int32_t*>(smem + SM::eid_off());
   int32_t* did = reinterpret_cast<int32_t*>(smem + SM::did_off());
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::bar_off());
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SM::flag_off(S));
   unsigned char* stages = smem + SM::stage_off(S);
 
   int64_t j0, j1;
@@ -997,6 +1005,7 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
   }
   if (lane == 0) {
     for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+    *s_abort = 0;
     mbar_fence_init();
   }
   __syncthreads();
@@ -1008,7 +1017,8 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
     for (int j = 0; j < GR::NXG; ++j) dx[k][j] = T(0);
   if constexpr (CONV) load_x<CF, GR>(xr, x + size_t(n) * xrow, C, cb);
 
-  uint32_t issued = 0, consumed = 0;
+  int prod_slot = 0, cons_slot = 0;
+  uint32_t cons_phase = 0, issued = 0, consumed = 0;
   bool alive = true;
   const int64_t deg = j1 - j0;
   for (int64_t ws = 0; ws < deg && alive; ws += BWD_WIN) {
@@ -1038,43 +1048,47 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
     }
     __syncthreads();
     const int steps = (cnt + NS - 1) / NS;
-    auto issue = [&](int st) {  // thread 0 only
-      const uint32_t slot = issued % S;
-      uint64_t* bar = &bars[slot];
-      unsigned char* dst = stages + size_t(slot) * STAGE;
-      uint32_t bytes = 0;
-      for (int j = 0; j < NS; ++j) {
+    // producer: lane 0 posts the expected bytes, then lanes move one slice each (per edge:
+    // weights, grad_out of the receiver, and x for the tensor product)
+    constexpr int ITEMS = CONV ? 2 : 3;
+    auto issue = [&](int st) {
+      uint64_t* bar = &bars[prod_slot];
+      unsigned char* dst = stages + size_t(prod_slot) * STAGE;
+      int nv = 0;
+      for (int j = lane; j < NS; j += 32) {
         const int r = st * NS + j;
-        if (r < cnt && eid[r] >= 0) bytes += SLOT;
+        nv += (r < cnt && eid[r] >= 0) ? 1 : 0;
       }
-      mbar_arrive_expect_tx(bar, bytes);
-      for (int j = 0; j < NS; ++j) {
+      nv = __reduce_add_sync(0xffffffffu, nv);
+      if (lane == 0) mbar_arrive_expect_tx(bar, uint32_t(nv) * SLOT);
+      __syncwarp();
+      for (int it = lane; it < ITEMS * NS; it += 32) {
+        const int j = it / ITEMS, kind = it % ITEMS;
         const int r = st * NS + j;
-        if (r >= cnt) break;
-        if (eid[r] < 0) continue;
+        if (r >= cnt || eid[r] < 0) continue;
         const int64_t e = eid[r];
         unsigned char* d = dst + size_t(j) * SLOT;
-        bulk_load(d, w + e * wrow + size_t(GR::PB) * C, WB, bar);
-        bulk_load(d + WB, g + size_t(did[r]) * orow + size_t(GR::OB) * C, GB, bar);
-        if constexpr (!CONV) bulk_load(d + WB + GB, x + size_t(e) * xrow + size_t(GR::XB) * C, XB, bar);
+        if (kind == 0)
+          bulk_load(d, w + e * wrow + size_t(GR::PB) * C, WB, bar);
+        else if (kind == 1)
+          bulk_load(d + WB, g + size_t(did[r]) * orow + size_t(GR::OB) * C, GB, bar);
+        else
+          bulk_load(d + WB + GB, x + size_t(e) * xrow + size_t(GR::XB) * C, XB, bar);
       }
+      prod_slot = prod_slot + 1 == S ? 0 : prod_slot + 1;
       ++issued;
     };
-    if (lane == 0)
-      for (int st = 0; st < S && st < steps; ++st) issue(st);
-    else
-      issued += uint32_t(S < steps ? S : steps);
+    for (int st = 0; st < S && st < steps; ++st) issue(st);
 
     for (int st = 0; st < steps; ++st) {
-      const uint32_t slot = consumed % S, parity = (consumed / S) & 1u;
-      const bool ok = mbar_wait(&bars[slot], parity, a.status);
-      if (__syncthreads_or(!ok)) {
-        alive = false;
-        break;
-      }
+      const int slot = cons_slot;
+      const bool okw = mbar_wait(&bars[slot], cons_phase, a.status);
+      if (!okw) *s_abort = 1;
+      cons_slot = cons_slot + 1 == S ? 0 : cons_slot + 1;
+      if (cons_slot == 0) cons_phase ^= 1u;
       ++consumed;
       const int r = st * NS + slice;
-      const bool mine = r < cnt && eid[r] >= 0;
+      const bool mine = okw && r < cnt && eid[r] >= 0;
       const int64_t e = mine ? eid[r] : 0;
       if (mine) {
         const T* sl = reinterpret_cast<const T*>(stages + size_t(slot) * STAGE + size_t(slice) * SLOT);
@@ -1153,22 +1167,19 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
       if constexpr (!CONV) {
         if (mine && gx != nullptr) bwd_put_dx<CF, GI>(gx + size_t(e) * xrow, dx, C, cb, scale);
       }
-      __syncthreads();
-      if (st + S < steps) {
-        if (lane == 0)
-          issue(st + S);
-        else
-          ++issued;
+      __syncthreads();  // every thread is done with this stage (and sees an abort)
+      if (*s_abort) {
+        alive = false;
+        break;
       }
+      if (st + S < steps) issue(st + S);
     }
     __syncthreads();
   }
   if (!alive) {
+    // a wait gave up: let the copies in flight land (bounded) before the CTA exits
     if (lane == 0)
-      while (consumed < issued) {
-        mbar_wait(&bars[consumed % S], (consumed / S) & 1u, a.status);
-        ++consumed;
-      }
+      for (uint32_t q = consumed - 1; q < issued; ++q) mbar_wait(&bars[q % S], (q / S) & 1u, a.status);
     __syncthreads();
     return;
   }
