@@ -492,13 +492,14 @@ __device__ __noinline__ void fwd_stage_window(const KFwd& a, int64_t e0, int64_t
   }
 }
 
-template <class CF, int GI, bool CONV>
+template <class CF, int GI, bool CONV, int CC>
 __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned char* smem) {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
   using SM = FwdSmem<CF>;
   constexpr int NYP = SM::NYP;
-  const int C = a.C, CB = C >> 2;
+  const int C = CC > 0 ? CC : a.C;  // compile-time for the specialised multiplicities
+  const int CB = C >> 2;
   const int tid = threadIdx.x;
   const int cb = CB >= 32 ? tid : tid % CB;
   const int slice = CB >= 32 ? 0 : tid / CB;
@@ -655,7 +656,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
   }
 }
 
-template <class CF, bool CONV>
+template <class CF, bool CONV, int CC>
 __global__ void __launch_bounds__(256) fwd_kernel(const __grid_constant__ KFwd a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   // group-major order: CTAs are started roughly in index order, so the CTAs resident on an SM
@@ -663,7 +664,7 @@ __global__ void __launch_bounds__(256) fwd_kernel(const __grid_constant__ KFwd a
   const int64_t units = int64_t(gridDim.x) / CF::G;
   const int g = int(blockIdx.x / units);
   const int64_t unit = blockIdx.x % units;
-  dispatch<CF::G>(g, [&](auto gi) { fwd_group<CF, decltype(gi)::value, CONV>(a, unit, smem_raw); });
+  dispatch<CF::G>(g, [&](auto gi) { fwd_group<CF, decltype(gi)::value, CONV, CC>(a, unit, smem_raw); });
 }
 
 // ========================================================================= backward ===
@@ -955,7 +956,7 @@ __device__ __forceinline__ void bwd_put_dx(typename CF::T* __restrict__ row, con
 
 // Backward of path group GI.  Convolution: one CTA (one warp) per sender, walking its
 // out-edges through the sender CSR; tensor product: one CTA per contiguous sample range.
-template <class CF, int GI, bool CONV>
+template <class CF, int GI, bool CONV, int CC>
 __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a) {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
@@ -963,7 +964,8 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
   using MK = BwdMasks<CF, GI>;
   constexpr int NYP = SM::NYP;
   extern __shared__ __align__(128) unsigned char smem[];
-  const int C = a.C, CB = C >> 2;  // CB <= 32: one warp covers every channel
+  const int C = CC > 0 ? CC : a.C;  // compile-time for the specialised multiplicities
+  const int CB = C >> 2;            // CB <= 32: one warp covers every channel
   const int lane = threadIdx.x;
   const int cb = lane % CB, slice = lane / CB, NS = 32 / CB;
   const int S = a.stages;
@@ -1196,8 +1198,8 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
 }
 
 // =================================================================== host launchers ===
-template <class CF>
-e3_status launch_fwd_cfg(const e3_plan* plan, const FwdArgs& h, bool conv) {
+template <class CF, int CC>
+e3_status launch_fwd_cc(const e3_plan* plan, const FwdArgs& h, bool conv) {
   KFwd a{};
   a.row_ptr = h.row_ptr;
   a.src = h.src;
@@ -1218,7 +1220,7 @@ e3_status launch_fwd_cfg(const e3_plan* plan, const FwdArgs& h, bool conv) {
   const int threads = CB >= 32 ? CB : 32;
   const int NS = CB >= 32 ? 1 : 32 / CB;
   // ring depth: as deep as 3 stages while the CTAs that fit by registers also fit in shared memory
-  auto kern = conv ? fwd_kernel<CF, true> : fwd_kernel<CF, false>;
+  auto kern = conv ? fwd_kernel<CF, true, CC> : fwd_kernel<CF, false, CC>;
   cudaFuncAttributes fa{};
   cudaError_t err = cudaFuncGetAttributes(&fa, kern);
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(err));
@@ -1253,10 +1255,10 @@ e3_status launch_fwd_cfg(const e3_plan* plan, const FwdArgs& h, bool conv) {
 // One backward launch per path group, in group order on the caller's stream: a launch only
 // holds its group's code, and grad_x / grad_y blocks shared by several groups are stored by
 // the first and accumulated by the later launches (fixed order: deterministic).
-template <class CF, int GI>
+template <class CF, int GI, int CC>
 e3_status launch_bwd_group(KBwd a, bool conv, int64_t blocks, cudaStream_t s) {
   const int CB = a.C / 4, NS = 32 / CB;
-  auto kern = conv ? bwd_kernel<CF, GI, true> : bwd_kernel<CF, GI, false>;
+  auto kern = conv ? bwd_kernel<CF, GI, true, CC> : bwd_kernel<CF, GI, false, CC>;
   cudaFuncAttributes fa{};
   cudaError_t err = cudaFuncGetAttributes(&fa, kern);
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(err));
@@ -1276,19 +1278,19 @@ e3_status launch_bwd_group(KBwd a, bool conv, int64_t blocks, cudaStream_t s) {
   return E3_OK;
 }
 
-template <class CF, int GI = 0>
+template <class CF, int CC, int GI = 0>
 e3_status launch_bwd_groups(const KBwd& a, bool conv, int64_t blocks, cudaStream_t s) {
   if constexpr (GI < CF::G) {
-    const e3_status st = launch_bwd_group<CF, GI>(a, conv, blocks, s);
+    const e3_status st = launch_bwd_group<CF, GI, CC>(a, conv, blocks, s);
     if (st != E3_OK) return st;
-    return launch_bwd_groups<CF, GI + 1>(a, conv, blocks, s);
+    return launch_bwd_groups<CF, CC, GI + 1>(a, conv, blocks, s);
   } else {
     return E3_OK;
   }
 }
 
-template <class CF>
-e3_status launch_bwd_cfg(const e3_plan* plan, const BwdArgs& h, bool conv) {
+template <class CF, int CC>
+e3_status launch_bwd_cc(const e3_plan* plan, const BwdArgs& h, bool conv) {
   KBwd a{};
   a.row_ptr_src = h.row_ptr_src;
   a.perm_src = h.perm_src;
@@ -1323,7 +1325,42 @@ e3_status launch_bwd_cfg(const e3_plan* plan, const BwdArgs& h, bool conv) {
   }
   if (blocks >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "grid too large");
   if (blocks == 0) return E3_OK;
-  return launch_bwd_groups<CF>(a, conv, blocks, static_cast<cudaStream_t>(h.stream));
+  return launch_bwd_groups<CF, CC>(a, conv, blocks, static_cast<cudaStream_t>(h.stream));
+}
+
+// Multiplicities compiled with C as a constant (all channel address arithmetic folds to
+// immediates); any other multiplicity runs the kernels with C read from the arguments.
+template <class CF>
+constexpr int spec_c(int i) {
+  if constexpr (!std::is_same<typename CF::T, float>::value) {
+    return 0;
+  } else if constexpr (CF::LX == 2 && CF::LY == 3 && CF::LO == 2) {
+    return i == 0 ? 64 : (i == 1 ? 128 : 0);
+  } else if constexpr (CF::LX == 3 && CF::LY == 3 && CF::LO == 3) {
+    return i == 0 ? 128 : 0;
+  } else if constexpr (CF::LX == 1 && CF::LY == 2 && CF::LO == 2) {
+    return i == 0 ? 8 : 0;
+  } else {
+    return 0;
+  }
+}
+
+template <class CF>
+e3_status launch_fwd_cfg(const e3_plan* plan, const FwdArgs& h, bool conv) {
+  if constexpr (spec_c<CF>(0) > 0)
+    if (plan->C == spec_c<CF>(0)) return launch_fwd_cc<CF, spec_c<CF>(0)>(plan, h, conv);
+  if constexpr (spec_c<CF>(1) > 0)
+    if (plan->C == spec_c<CF>(1)) return launch_fwd_cc<CF, spec_c<CF>(1)>(plan, h, conv);
+  return launch_fwd_cc<CF, 0>(plan, h, conv);
+}
+
+template <class CF>
+e3_status launch_bwd_cfg(const e3_plan* plan, const BwdArgs& h, bool conv) {
+  if constexpr (spec_c<CF>(0) > 0)
+    if (plan->C == spec_c<CF>(0)) return launch_bwd_cc<CF, spec_c<CF>(0)>(plan, h, conv);
+  if constexpr (spec_c<CF>(1) > 0)
+    if (plan->C == spec_c<CF>(1)) return launch_bwd_cc<CF, spec_c<CF>(1)>(plan, h, conv);
+  return launch_bwd_cc<CF, 0>(plan, h, conv);
 }
 
 // Fill this unit's copy of the coefficient tables on the current device.
