@@ -354,6 +354,64 @@ struct FwdAcc {
     });
   }
 
+  // The same contraction reading each path's weights and x block from the staged slices just
+  // before use (sw: the group's weight slice, path PB first; sx: x blocks L1A..L1B), so that
+  // only one path's operands are live at a time.
+  __device__ __forceinline__ void edge_smem(const T* sw, const T* sx, const T (&Y)[CF::NY], int C, int cb) {
+    static_for<GR::PB, GR::PE>([&](auto pc) {
+      constexpr int P = decltype(pc)::value;
+      using PC = PathC<CF, P>;
+      constexpr int L1 = PC::L1, L2 = PC::L2, L3 = PC::L3, D1 = PC::D1, D3 = PC::D3;
+      constexpr int OO = PC::OUT - GR::OB;
+      T wk[K];
+      lds16(wk, sw + size_t(P - GR::PB) * C + 4 * cb);
+      T xk[K * D1];
+      lds16(xk, sx + size_t(C) * (L1 * L1 - GR::XB) + size_t(4 * cb) * D1);
+      if constexpr (D1 < D3) {
+        T xs[K][D1];
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+#pragma unroll
+          for (int m1 = 0; m1 < D1; ++m1) xs[k][m1] = wk[k] * xk[k * D1 + m1];
+        static_for<0, D3>([&](auto m3c) {
+          constexpr int M3I = decltype(m3c)::value;
+          T a[D1];
+          static_for<0, D1>([&](auto m1c) {
+            constexpr int M1I = decltype(m1c)::value;
+            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) a[M1I] = a_entry<T, L1, L2, L3, M1I - L1, M3I - L3>(Y);
+          });
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            T t = acc[k][OO + M3I];
+            static_for<0, D1>([&](auto m1c) {
+              constexpr int M1I = decltype(m1c)::value;
+              if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) t = fma(a[M1I], xs[k][M1I], t);
+            });
+            acc[k][OO + M3I] = t;
+          }
+        });
+      } else {
+        static_for<0, D3>([&](auto m3c) {
+          constexpr int M3I = decltype(m3c)::value;
+          T a[D1];
+          static_for<0, D1>([&](auto m1c) {
+            constexpr int M1I = decltype(m1c)::value;
+            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) a[M1I] = a_entry<T, L1, L2, L3, M1I - L1, M3I - L3>(Y);
+          });
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            T t = T(0);
+            static_for<0, D1>([&](auto m1c) {
+              constexpr int M1I = decltype(m1c)::value;
+              if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) t = fma(a[M1I], xk[k * D1 + M1I], t);
+            });
+            acc[k][OO + M3I] = fma(wk[k], t, acc[k][OO + M3I]);
+          }
+        });
+      }
+    });
+  }
+
   // out[row, path blocks of the group, channels 4cb..] = pscale_p * acc
   __device__ __forceinline__ void store(T* __restrict__ orow, int C, int cb, const double* pscale) {
     static_for<GR::PB, GR::PE>([&](auto pc) {
@@ -543,7 +601,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
 
   FwdAcc<CF, GI> f;
   f.zero();
-  T xr[K][GR::NXG], wr[K][GR::NP], Y[CF::NY];
+  T Y[CF::NY];
   // ring state: identical in every thread, advanced uniformly
   int prod_slot = 0, cons_slot = 0;
   uint32_t cons_phase = 0, issued = 0, consumed = 0;
@@ -599,25 +657,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
       const bool mine = ok && r < cnt && (!CONV || src_s[r] >= 0);
       if (mine) {
         const T* sl = reinterpret_cast<const T*>(stages + size_t(slot) * STAGE + size_t(slice) * SLOT);
-        // weights of the group's paths for channels 4cb..4cb+3
-#pragma unroll
-        for (int q = 0; q < GR::NP; ++q) {
-          T t4[K];
-          lds16(t4, sl + size_t(q) * C + 4 * cb);
-#pragma unroll
-          for (int k = 0; k < K; ++k) wr[k][q] = t4[k];
-        }
         const T* xs = sl + WB / sizeof(T);
-        static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
-          constexpr int L = decltype(lc)::value;
-          constexpr int D = 2 * L + 1;
-          T t[K * D];
-          lds16(t, xs + size_t(C) * (L * L - GR::XB) + size_t(4 * cb) * D);
-#pragma unroll
-          for (int k = 0; k < K; ++k)
-#pragma unroll
-            for (int m = 0; m < D; ++m) xr[k][L * L - GR::XB + m] = t[k * D + m];
-        });
         {
           T yp[NYP];
           lds16(yp, ysh + r * NYP);
@@ -625,7 +665,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
           for (int m = 0; m < CF::NY; ++m) Y[m] = yp[m];
         }
         if constexpr (!CONV) f.zero();
-        f.edge(xr, wr, Y);
+        f.edge_smem(sl, xs, Y, C, cb);
         if constexpr (!CONV) f.store(out + size_t(e0 + ws + r) * orow, C, cb, a.pscale);
       }
       __syncthreads();  // every thread is done with this stage (and sees an abort)
@@ -656,8 +696,15 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
   }
 }
 
+// Register budget of the forward: path sets with output degree <= 2 fit in 128 registers per
+// thread (16 resident warps per SM); the l <= 3 set keeps the compiler's choice (spills at 128).
+template <class CF>
+constexpr int fwd_min_blocks() {
+  return CF::LO <= 2 ? 2 : 1;
+}
+
 template <class CF, bool CONV, int CC>
-__global__ void __launch_bounds__(256) fwd_kernel(const __grid_constant__ KFwd a) {
+__global__ void __launch_bounds__(256, fwd_min_blocks<CF>()) fwd_kernel(const __grid_constant__ KFwd a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   // group-major order: CTAs are started roughly in index order, so the CTAs resident on an SM
   // at any time run the same path group and share its (large, fully unrolled) code
@@ -685,6 +732,7 @@ struct KBwd {
   int* status;
   double scale;
   double alpha[MAXP];
+  float alpha_f[MAXP];  // the same path weights rounded once, for the float kernels
 };
 
 // Which path groups touch x block l1 / harmonics block l2 (the first toucher stores, later
@@ -710,7 +758,7 @@ __host__ __device__ constexpr bool group_has_l2(int l) {
   return false;
 }
 
-constexpr int BWD_WIN = 64;  // out-edges whose ids and harmonics are staged at once
+constexpr int BWD_WIN = 32;  // out-edges whose ids and harmonics are staged at once
 
 // Byte sizes of one edge's staged slices in the backward of group GI: weights of the group's
 // paths, grad_out of the receiver for the group's outputs, and (tensor product only) the x slice.
@@ -753,7 +801,7 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
                                          const typename CF::T (&Y)[CF::NY], const typename CF::T* sg,
                                          typename CF::T (&dx)[K][Grp<CF, GI>::NXG], typename CF::T (&dY)[CF::NY],
                                          bool want_dy, typename CF::T* __restrict__ gw, int C, int cb,
-                                         const double* alpha, typename CF::T scale) {
+                                         const double* alpha, const float* alpha_f, typename CF::T scale) {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
 #pragma unroll
@@ -774,7 +822,7 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
 #pragma unroll
         for (int m = 0; m < D3; ++m) g[k][m] = t4[k * D3 + m];
     }
-    const T al = T(alpha[P]);
+    const T al = std::is_same<T, float>::value ? T(alpha_f[P]) : T(alpha[P]);
     T wa[K];
 #pragma unroll
     for (int k = 0; k < K; ++k) wa[k] = al * wk[k];
@@ -1118,7 +1166,7 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
           for (int m = 0; m < CF::NY; ++m) Y[m] = yp[m];
         }
         bwd_edge<CF, GI>(xr, sl, Y, sl + WB / sizeof(T), dx, dY, want_dy, gwp ? gwp + e * wrow : nullptr, C, cb,
-                         a.alpha, scale);
+                         a.alpha, a.alpha_f, scale);
       } else {
 #pragma unroll
         for (int m = 0; m < CF::NY; ++m) dY[m] = T(0);
@@ -1310,7 +1358,10 @@ e3_status launch_bwd_cc(const e3_plan* plan, const BwdArgs& h, bool conv) {
   a.scale = h.scale;
   e3_status st = device_status_ptr(&a.status);
   if (st != E3_OK) return st;
-  for (int p = 0; p < plan->n_paths; ++p) a.alpha[p] = plan->alpha[p];
+  for (int p = 0; p < plan->n_paths; ++p) {
+    a.alpha[p] = plan->alpha[p];
+    a.alpha_f[p] = float(plan->alpha[p]);
+  }
   const int CB = plan->C / 4;
   if (CB > 32) return fail(E3_ERR_UNSUPPORTED, "the backward kernels need a multiplicity of at most 128");
   const int NS = 32 / CB;
