@@ -146,6 +146,26 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def rank_seed(base_seed, rank):
+    """Weak scaling: every rank owns an independent box of the same size, with its own seed."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(value, world, dist=None, device=None):
+    """The job's time is the slowest rank's (all_reduce MAX); identity on one rank."""
+    if world <= 1 or dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(edges_per_rank, world, ms_per_step):
+    """Whole-job edges/s: the edges all ranks processed over the slowest rank's step time."""
+    return edges_per_rank * world / (ms_per_step * 1e-3)
+
+
 def oracle_sample(cfg, irreps_x, irreps_y, n_edges_target, seed=0):
     """The oracle (float64 CPU) on the in-edges of random receivers: (edges, seconds fwd+bwd)."""
     import oracle
@@ -219,7 +239,7 @@ def run_native(args):
     cfg, irreps_x, irreps_y = workload_spec(args.workload)
     N, mul, lx, ly, lo = cfg["N"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
     # weak scaling: every rank owns an independent box of the same size (its own seed)
-    g = W.graph_inputs(N, mul, lx, ly, lo, cfg["seed"] + 1000 * rank, weights="torch", device=dev)
+    g = W.graph_inputs(N, mul, lx, ly, lo, rank_seed(cfg["seed"], rank), weights="torch", device=dev)
     plan = e3b.Plan(irreps_x, irreps_y, lmax_out=lo)
     graph = e3b.Graph(N, torch.as_tensor(g["src"], device=dev), torch.as_tensor(g["dst"], device=dev))
     E = graph.n_edges
@@ -276,12 +296,9 @@ def run_native(args):
     fwd_ms = statistics.fmean(a.elapsed_time(b) for a, b, c in ev)
     bwd_ms = statistics.fmean(b.elapsed_time(c) for a, b, c in ev)
     e3b.device_status()
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, dist, dev)
     ms_step = ms_total / args.steps
-    value = E * world / (ms_step * 1e-3)
+    value = job_throughput(E, world, ms_step)
 
     # end to end through the public API: inputs from pinned host memory, results back to host
     e2e = None
@@ -313,14 +330,10 @@ def run_native(args):
             e2e_step()
         b.record(stream)
         barrier()
-        e_ms = a.elapsed_time(b) / e2e_steps
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world, dist, dev)
         h2d = sum(t.numel() * t.element_size() for t in (hx, hvec, hw, hgo))
         d2h = sum(t.numel() * t.element_size() for t in (hout, hgx, hgy, hgw))
-        e2e = {"value": E * world / (e_ms * 1e-3), "unit": "edges/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_throughput(E, world, e_ms), "unit": "edges/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     if world > 1:
