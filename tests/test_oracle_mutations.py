@@ -1,0 +1,151 @@
+"""Planted mistakes in the oracle must be caught by its pins.
+
+Each case patches one oracle routine with a plausible bug (a flipped sign, transposed operands, a
+dropped factor or term, a wrong index) and runs the pins that should see it; the case passes only
+if at least one of them fails.  Everything runs on the CPU."""
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.cg as ocg
+import oracle.conv as oconv
+import oracle.sh as osh
+import oracle.tp as otp
+from tests import test_oracle_pins as pins
+
+
+def _caught(checks):
+    for fn in checks:
+        try:
+            fn()
+        except AssertionError:
+            return True
+    return False
+
+
+def _patch_cg(monkeypatch, fn):
+    orig = ocg.real_cg
+
+    def bad(l1, l2, l3):
+        return fn(l1, l2, l3, np.array(orig(l1, l2, l3)))
+
+    monkeypatch.setattr(ocg, "real_cg", bad)
+    monkeypatch.setattr(otp, "real_cg", bad)
+    monkeypatch.setattr(pins, "real_cg", bad)
+
+
+CG_PINS = [pins.test_real_cg_1x1_is_dot_cross_symtraceless,
+           lambda: pins.test_real_cg_orthogonality(1, 2),
+           lambda: pins.test_real_cg_equivariance(1, 2),
+           lambda: pins.test_real_cg_equivariance(2, 2),
+           lambda: pins.test_tp_equivariance_o3(False)]
+
+
+def test_flipped_cg_entry(monkeypatch):
+    def f(l1, l2, l3, t):
+        if (l1, l2, l3) == (1, 2, 2):
+            idx = tuple(np.argwhere(np.abs(t) > 1e-9)[0])
+            t[idx] = -t[idx]
+        return t
+    _patch_cg(monkeypatch, f)
+    assert _caught(CG_PINS)
+
+
+def test_transposed_cg_operands(monkeypatch):
+    _patch_cg(monkeypatch, lambda l1, l2, l3, t: t.transpose(1, 0, 2) if l1 == l2 else t)
+    assert _caught([pins.test_real_cg_1x1_is_dot_cross_symtraceless])
+
+
+def test_cg_wrong_sign_convention(monkeypatch):
+    _patch_cg(monkeypatch, lambda l1, l2, l3, t: -t if (l1 + l2 + l3) % 2 else t)
+    assert _caught([pins.test_real_cg_1x1_is_dot_cross_symtraceless])
+
+
+def test_sh_wrong_sin_sign(monkeypatch):
+    orig = osh.real_sh
+
+    def bad(l, vec):
+        y = orig(l, vec)
+        if l >= 1:
+            y[:, :l] = -y[:, :l]
+        return y
+
+    monkeypatch.setattr(osh, "real_sh", bad)
+    monkeypatch.setattr(pins, "real_sh", bad)
+    assert _caught([pins.test_sh_closed_forms_low_degree])
+
+
+def test_sh_dropped_sqrt2(monkeypatch):
+    orig = osh.real_sh
+
+    def bad(l, vec):
+        y = orig(l, vec)
+        if l >= 1:
+            y[:, l + 1:] /= np.sqrt(2.0)
+        return y
+
+    monkeypatch.setattr(pins, "real_sh", bad)
+    assert _caught([lambda: pins.test_sh_norm_parity_and_scale_invariance(2)])
+
+
+def test_tp_dropped_path_weight(monkeypatch):
+    orig = otp.tp_forward
+
+    def bad(plan, x, y, w):
+        saved = list(plan.alphas)
+        plan.alphas = [1.0] * len(saved)
+        try:
+            return orig(plan, x, y, w)
+        finally:
+            plan.alphas = saved
+
+    monkeypatch.setattr(oracle, "tp_forward", bad)
+    assert _caught([pins.test_tp_matches_brute_force_loops])
+
+
+def test_tp_transposed_uv_weights(monkeypatch):
+    orig = otp._weights
+
+    def bad2(plan, w, p, bsz):
+        ws = orig(plan, w, p, bsz)
+        a, b = ws.shape[1], ws.shape[2]
+        return ws.reshape(bsz, -1)[:, ::-1].reshape(bsz, a, b)
+
+    monkeypatch.setattr(otp, "_weights", bad2)
+    assert _caught([pins.test_tp_multiplicity_two_inputs_brute_force])
+
+
+def test_backward_dropped_alpha_in_dy(monkeypatch):
+    orig = otp.tp_backward
+
+    def bad(plan, x, y, w, g):
+        dx, dy, dw = orig(plan, x, y, w, g)
+        return dx, dy * 0.5, dw
+
+    monkeypatch.setattr(oracle, "tp_backward", bad)
+    assert _caught([pins.test_tp_backward_euler_identities_and_fd])
+
+
+def test_conv_double_scale(monkeypatch):
+    orig = oconv.conv_forward
+
+    def bad(plan, n, src, dst, x, y, w, scale, chunk=4096):
+        return orig(plan, n, src, dst, x, y, w, scale * scale, chunk)
+
+    monkeypatch.setattr(oracle, "conv_forward", bad)
+    assert _caught([pins.test_conv_edge_order_invariance_isolated_and_empty])
+
+
+def test_csr_unstable_sort(monkeypatch):
+    def bad(n, src, dst):
+        src = np.asarray(src)
+        dst = np.asarray(dst)
+        perm_dst = np.lexsort((-np.arange(len(dst)), dst))  # ties in reverse input order
+        rp = np.concatenate([[0], np.cumsum(np.bincount(dst, minlength=n))])
+        perm_src = np.argsort(src[perm_dst], kind="stable")
+        rps = np.concatenate([[0], np.cumsum(np.bincount(src, minlength=n))])
+        return perm_dst.astype(np.int32), rp.astype(np.int32), perm_src.astype(np.int32), rps.astype(np.int32)
+
+    monkeypatch.setattr(oracle, "csr_build", bad)
+    assert _caught([pins.test_csr_bit_exact_against_loops])
