@@ -149,33 +149,11 @@ E3_HD constexpr int path_cost(int LX, int LY, int LO, int p) {
   return a_block_nnz(l1, l2, l3) + (d1 < d3 ? d1 : d3);
 }
 
-// Path groups.  One CTA (one warp for C <= 128) runs one group of paths for one receiver,
-// and each thread accumulates 4 channels x the outputs of its group in registers, so a group
-// is capped at GROUP_OUT_CAP outputs per channel.  Groups are contiguous runs of paths in
-// enumeration order, cut greedily when the next path would exceed the cap.
+// Path groups.  Each thread accumulates 4 channels x the outputs of one group of paths in
+// registers, so a group is capped at a number of outputs per channel (the forward and the
+// backward use different caps).  Groups are contiguous runs of paths in enumeration order,
+// cut greedily when the next path would exceed the cap.
 constexpr int GROUP_OUT_CAP = 20;
-
-E3_HD constexpr int group_scan(int LX, int LY, int LO, int g_stop, bool want_count) {
-  const int P = n_paths(LX, LY, LO);
-  int grp = 0, outs = 0;
-  for (int p = 0; p < P; ++p) {
-    const int d = 2 * path_l(LX, LY, LO, p, 2) + 1;
-    if (outs > 0 && outs + d > GROUP_OUT_CAP) {
-      ++grp;
-      outs = 0;
-      if (!want_count && grp == g_stop) return p;
-    }
-    outs += d;
-  }
-  return want_count ? grp + 1 : P;
-}
-
-E3_HD constexpr int n_groups(int LX, int LY, int LO) { return group_scan(LX, LY, LO, 0, true); }
-
-// First path of group g (g = n_groups gives n_paths).
-E3_HD constexpr int group_begin(int LX, int LY, int LO, int g) {
-  return g <= 0 ? 0 : group_scan(LX, LY, LO, g, false);
-}
 
 // Everything the kernels need to know about a path set, computed once per (LX, LY, LO).
 constexpr int MAX_PATHS = 64;
@@ -185,7 +163,7 @@ struct PathTable {
   int out_off[MAX_PATHS + 1];
   int gbegin[MAX_PATHS + 1];
 };
-E3_HD constexpr PathTable make_path_table(int LX, int LY, int LO) {
+E3_HD constexpr PathTable make_path_table(int LX, int LY, int LO, int cap) {
   PathTable t{};
   for (int l1 = 0; l1 <= LX; ++l1)
     for (int l2 = 0; l2 <= LY; ++l2)
@@ -202,7 +180,7 @@ E3_HD constexpr PathTable make_path_table(int LX, int LY, int LO) {
   t.ngroups = 1;
   for (int p = 0; p < t.n; ++p) {
     const int d = 2 * t.l3[p] + 1;
-    if (outs > 0 && outs + d > GROUP_OUT_CAP) {
+    if (outs > 0 && outs + d > cap) {
       t.gbegin[t.ngroups++] = p;
       outs = 0;
     }

@@ -91,7 +91,7 @@ template <int LX_, int LY_, int LO_, typename T_>
 struct Cfg {
   static constexpr int LX = LX_, LY = LY_, LO = LO_;
   using T = T_;
-  static constexpr PathTable PT = make_path_table(LX, LY, LO);
+  static constexpr PathTable PT = make_path_table(LX, LY, LO, GROUP_OUT_CAP);
   static constexpr int P = PT.n;
   static constexpr int G = PT.ngroups;
   static constexpr int NY = (LY + 1) * (LY + 1);
@@ -435,7 +435,7 @@ struct FwdAcc {
 // mbarrier per stage (transaction bytes).  Every wait is bounded: after WAIT_LIMIT polls the
 // kernel records E3_ERR_TIMEOUT and stops issuing work.
 constexpr long long WAIT_LIMIT = 1ll << 24;
-constexpr int FWD_WIN = 96;  // in-edges whose sender ids and harmonics are staged at once
+constexpr int FWD_WIN = 64;  // in-edges whose sender ids and harmonics are staged at once
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -760,8 +760,19 @@ __host__ __device__ constexpr bool group_has_l2(int l) {
 
 constexpr int BWD_WIN = 32;  // out-edges whose ids and harmonics are staged at once
 
+// A group that adds to grad_y blocks an earlier group stored stages the edge's grad_y row with
+// its other slices, so the read-modify-write does not wait on a global load (rows whose byte
+// size is not a multiple of 16 cannot be bulk-copied and are read directly).
+template <class CF, int GI>
+__host__ __device__ constexpr bool bwd_stage_gy() {
+  bool acc = false;
+  for (int l = 0; l <= CF::LY; ++l) acc = acc || (group_has_l2<CF, GI>(l) && first_group_l2<CF>(l) != GI);
+  return acc && (CF::NY * sizeof(typename CF::T)) % 16 == 0;
+}
+
 // Byte sizes of one edge's staged slices in the backward of group GI: weights of the group's
-// paths, grad_out of the receiver for the group's outputs, and (tensor product only) the x slice.
+// paths, grad_out of the receiver for the group's outputs, (tensor product only) the x slice,
+// and the grad_y row when bwd_stage_gy() holds and grad_y is requested.
 template <class CF, int GI>
 struct BwdSlice {
   using T = typename CF::T;
@@ -771,7 +782,12 @@ struct BwdSlice {
   static __host__ __device__ constexpr uint32_t xbytes(int C, bool conv) {
     return conv ? 0u : uint32_t(GR::NXG) * C * sizeof(T);
   }
-  static __host__ __device__ constexpr uint32_t slot(int C, bool conv) { return wbytes(C) + gbytes(C) + xbytes(C, conv); }
+  static __host__ __device__ constexpr uint32_t ybytes(bool dy) {
+    return dy && bwd_stage_gy<CF, GI>() ? uint32_t(CF::NY * sizeof(T)) : 0u;
+  }
+  static __host__ __device__ constexpr uint32_t slot(int C, bool conv, bool dy) {
+    return wbytes(C) + gbytes(C) + xbytes(C, conv) + ybytes(dy);
+  }
 };
 
 template <class CF, int GI>
@@ -784,11 +800,11 @@ struct BwdSmem {
   static __host__ __device__ size_t bar_off() { return did_off() + sizeof(int32_t) * BWD_WIN; }
   static __host__ __device__ size_t flag_off(int S) { return bar_off() + 8 * size_t(S); }
   static __host__ __device__ size_t stage_off(int S) { return (flag_off(S) + 16 + 127) & ~size_t(127); }
-  static __host__ __device__ size_t stage_bytes(int C, int NS, bool conv) {
-    return size_t(NS) * BwdSlice<CF, GI>::slot(C, conv);
+  static __host__ __device__ size_t stage_bytes(int C, int NS, bool conv, bool dy) {
+    return size_t(NS) * BwdSlice<CF, GI>::slot(C, conv, dy);
   }
-  static __host__ __device__ size_t total(int C, int NS, int S, bool conv) {
-    return stage_off(S) + size_t(S) * stage_bytes(C, NS, conv);
+  static __host__ __device__ size_t total(int C, int NS, int S, bool conv, bool dy) {
+    return stage_off(S) + size_t(S) * stage_bytes(C, NS, conv, dy);
   }
 };
 
@@ -1029,7 +1045,8 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
   const T scale = T(a.scale);
   const bool want_dy = gy != nullptr;
   const uint32_t WB = BwdSlice<CF, GI>::wbytes(C), GB = BwdSlice<CF, GI>::gbytes(C);
-  const uint32_t XB = BwdSlice<CF, GI>::xbytes(C, CONV), SLOT = WB + GB + XB;
+  const uint32_t XB = BwdSlice<CF, GI>::xbytes(C, CONV), YB = BwdSlice<CF, GI>::ybytes(want_dy);
+  const uint32_t SLOT = WB + GB + XB + YB;
   const size_t STAGE = size_t(NS) * SLOT;
   T* ysh = reinterpret_cast<T*>(smem + SM::ysh_off());
   int32_t* eid = reinterpret_cast<int32_t*>(smem + SM::eid_off());
@@ -1099,8 +1116,8 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
     __syncthreads();
     const int steps = (cnt + NS - 1) / NS;
     // producer: lane 0 posts the expected bytes, then lanes move one slice each (per edge:
-    // weights, grad_out of the receiver, and x for the tensor product)
-    constexpr int ITEMS = CONV ? 2 : 3;
+    // weights, grad_out of the receiver, x for the tensor product, the grad_y row to add to)
+    constexpr int ITEMS = 4;
     auto issue = [&](int st) {
       uint64_t* bar = &bars[prod_slot];
       unsigned char* dst = stages + size_t(prod_slot) * STAGE;
@@ -1122,8 +1139,10 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
           bulk_load(d, w + e * wrow + size_t(GR::PB) * C, WB, bar);
         else if (kind == 1)
           bulk_load(d + WB, g + size_t(did[r]) * orow + size_t(GR::OB) * C, GB, bar);
-        else
+        else if (kind == 2 && XB > 0)
           bulk_load(d + WB + GB, x + size_t(e) * xrow + size_t(GR::XB) * C, XB, bar);
+        else if (kind == 3 && YB > 0)
+          bulk_load(d + WB + GB + XB, gy + size_t(e) * CF::NY, YB, bar);
       }
       prod_slot = prod_slot + 1 == S ? 0 : prod_slot + 1;
       ++issued;
@@ -1140,8 +1159,8 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
       const int r = st * NS + slice;
       const bool mine = okw && r < cnt && eid[r] >= 0;
       const int64_t e = mine ? eid[r] : 0;
+      const T* sl = reinterpret_cast<const T*>(stages + size_t(slot) * STAGE + size_t(slice) * SLOT);
       if (mine) {
-        const T* sl = reinterpret_cast<const T*>(stages + size_t(slot) * STAGE + size_t(slice) * SLOT);
         if constexpr (!CONV) {
           const T* xs = sl + (WB + GB) / sizeof(T);
           static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
@@ -1203,6 +1222,8 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
             T* p = gy + e * CF::NY + m;
             if (MK::YS & (1u << block_of(m)))
               *p = scale * v[j];
+            else if (YB > 0)
+              *p = sl[(WB + GB + XB) / sizeof(T) + m] + scale * v[j];
             else
               *p += scale * v[j];
           }
@@ -1313,10 +1334,11 @@ e3_status launch_bwd_group(KBwd a, bool conv, int64_t blocks, cudaStream_t s) {
   const int regs = fa.numRegs > 0 ? fa.numRegs : 255;
   const int ctas = std::max(1, std::min(32, 65536 / (((regs + 7) & ~7) * 32)));
   const size_t budget = size_t(225) * 1024 / ctas;
+  const bool dy = a.grad_y != nullptr;
   int S = 3;
-  while (S > 2 && BwdSmem<CF, GI>::total(a.C, NS, S, conv) + 1024 > budget) --S;
+  while (S > 2 && BwdSmem<CF, GI>::total(a.C, NS, S, conv, dy) + 1024 > budget) --S;
   a.stages = S;
-  const size_t smem = BwdSmem<CF, GI>::total(a.C, NS, S, conv);
+  const size_t smem = BwdSmem<CF, GI>::total(a.C, NS, S, conv, dy);
   if (smem > size_t(227) * 1024) return fail(E3_ERR_UNSUPPORTED, "backward needs %zu bytes of shared memory", smem);
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
