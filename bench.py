@@ -253,6 +253,7 @@ def run_native(args):
     gx = torch.empty_like(x)
     gy = torch.empty((E, plan.dim_in2), device=dev)
     gw = torch.empty_like(w)
+    ws = e3b.backward_workspace(N, dev)
     stream = torch.cuda.current_stream()
     ev = []
 
@@ -267,7 +268,7 @@ def run_native(args):
         e3b.lib.e3_conv_backward(plan.handle, N, E, e3b._ptr(graph.row_ptr_dst), e3b._ptr(graph.src),
                                  e3b._ptr(graph.dst), e3b._ptr(graph.row_ptr_src), e3b._ptr(graph.perm_src),
                                  e3b._ptr(x), None, e3b._ptr(vec), 0, e3b._ptr(w), e3b._ptr(go), s, e3b._ptr(gx),
-                                 e3b._ptr(gy), e3b._ptr(gw), e3b._stream())
+                                 e3b._ptr(gy), e3b._ptr(gw), e3b._ptr(ws), ws.numel(), e3b._stream())
         if record:
             c.record(stream)
             ev.append((a, b, c))

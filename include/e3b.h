@@ -149,12 +149,19 @@ E3_API const char* e3_supported(void);
 E3_API e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x, const void* y,
                         const void* w, void* out, void* stream);
 
+/* Bytes of device workspace that e3_tp_backward (n = B) and e3_conv_backward (n = N) need:
+ * a ticket counter and one progress counter per work unit, which order the path groups of a
+ * unit inside one launch.  The backward zeroes it on its stream before use. */
+E3_API e3_status e3_backward_workspace_size(int64_t n, size_t* bytes);
+
 /* Gradients of <grad_out, TP(x, y, w)> by transposition [BWD].  Each of grad_x [B, dim_in1],
  * grad_y [B, dim_in2], grad_w [B, weight_numel] may be NULL to skip it; outputs are
- * overwritten.  E3_W_SHARED plans are not supported for the backward. */
+ * overwritten.  workspace: device buffer of at least e3_backward_workspace_size(B) bytes,
+ * 16-byte aligned, owned by the caller and not used by any other call while this one runs
+ * on its stream.  E3_W_SHARED plans are not supported for the backward. */
 E3_API e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* x, const void* y,
                          const void* w, const void* grad_out, void* grad_x, void* grad_y,
-                         void* grad_w, void* stream);
+                         void* grad_w, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------ harmonics --- */
 
@@ -232,13 +239,17 @@ E3_API e3_status e3_conv_forward(const e3_plan* plan, int64_t N, int64_t E, cons
  *                        computed from edge_vec);
  *   grad_w [E, weight_numel]: per edge.
  * Any gradient pointer may be NULL to skip it.  Other arguments as e3_conv_forward; dst [E]
- * is the receiver of each (receiver-ordered) edge.  Shared weights are not supported. */
+ * is the receiver of each (receiver-ordered) edge.  workspace: as for e3_tp_backward, of at
+ * least e3_backward_workspace_size(N) bytes.  No atomics on the gradients: the path groups of
+ * a sender run in a fixed order, so results are bitwise repeatable.  A group that waits for
+ * its predecessor longer than about a second records E3_ERR_TIMEOUT.  Shared weights are not
+ * supported. */
 E3_API e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E, const int32_t* row_ptr_dst,
                            const int32_t* src, const int32_t* dst, const int32_t* row_ptr_src,
                            const int32_t* perm_src, const void* x, const void* y,
                            const void* edge_vec, e3_sh_norm sh_norm, const void* w,
                            const void* grad_out, double out_scale, void* grad_x, void* grad_y,
-                           void* grad_w, void* stream);
+                           void* grad_w, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Message of the last non-OK status returned on the calling thread ("" if none). */
 E3_API const char* e3_last_error(void);

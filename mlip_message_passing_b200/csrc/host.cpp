@@ -558,9 +558,25 @@ extern "C" e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x
   return launch_forward(plan, a, false);
 }
 
+extern "C" e3_status e3_backward_workspace_size(int64_t n, size_t* bytes) {
+  clear_error();
+  if (bytes == nullptr) return fail(E3_ERR_INVALID_ARG, "bytes is NULL");
+  if (n < 0 || n >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "n = %lld out of range", (long long)n);
+  *bytes = backward_workspace_bytes(n);
+  return E3_OK;
+}
+
+static e3_status check_workspace(int64_t n, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr) return fail(E3_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 16 != 0) return fail(E3_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  if (ws_bytes < backward_workspace_bytes(n))
+    return fail(E3_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", ws_bytes, backward_workspace_bytes(n));
+  return E3_OK;
+}
+
 extern "C" e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* x, const void* y, const void* w,
                                     const void* grad_out, void* grad_x, void* grad_y, void* grad_w,
-                                    void* stream) {
+                                    void* workspace, size_t workspace_bytes, void* stream) {
   clear_error();
   e3_status st = check_plan_device(plan);
   if (st != E3_OK) return st;
@@ -575,7 +591,11 @@ extern "C" e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* 
   E3_OPT(grad_y, "grad_y");
   E3_OPT(grad_w, "grad_w");
   if (!grad_x && !grad_y && !grad_w) return E3_OK;
+  st = check_workspace(B, workspace, workspace_bytes);
+  if (st != E3_OK) return st;
   BwdArgs a{};
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
   a.n_nodes = B;
   a.n_edges = B;
   a.x = x;
@@ -643,7 +663,8 @@ extern "C" e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E,
                                       const int32_t* src, const int32_t* dst, const int32_t* row_ptr_src,
                                       const int32_t* perm_src, const void* x, const void* y, const void* edge_vec,
                                       e3_sh_norm sh_norm, const void* w, const void* grad_out, double out_scale,
-                                      void* grad_x, void* grad_y, void* grad_w, void* stream) {
+                                      void* grad_x, void* grad_y, void* grad_w, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
   clear_error();
   (void)row_ptr_dst;
   (void)src;
@@ -666,7 +687,11 @@ extern "C" e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E,
     if (dst == nullptr || perm_src == nullptr) return fail(E3_ERR_INVALID_ARG, "dst or perm_src is NULL");
   }
   if (!std::isfinite(out_scale)) return fail(E3_ERR_INVALID_ARG, "out_scale is not finite");
+  st = check_workspace(N, workspace, workspace_bytes);
+  if (st != E3_OK) return st;
   BwdArgs a{};
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
   a.n_nodes = N;
   a.n_edges = E;
   a.row_ptr_src = row_ptr_src;

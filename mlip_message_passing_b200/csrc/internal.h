@@ -77,8 +77,12 @@ struct BwdArgs {
   void* grad_x;
   void* grad_y;
   void* grad_w;
+  void* workspace;           // e3_backward_workspace_size(n_nodes) bytes
+  size_t workspace_bytes;
   void* stream;
 };
+// Bytes of backward workspace for n units: 16-byte ticket counter + one int per unit.
+inline size_t backward_workspace_bytes(int64_t n) { return (size_t(16) + 4 * size_t(n) + 255) & ~size_t(255); }
 e3_status launch_backward(const e3_plan* plan, const BwdArgs& a, bool conv);
 
 }  // namespace e3b

@@ -20,9 +20,11 @@
 //   * Forward: one CTA per (receiver, path group); the receiver's in-edges are consecutive in
 //     memory (receiver CSR), so the weight rows stream contiguously and x[src] rows are
 //     gathered from L2.  No atomics, no [E, dim_out] message tensor.
-//   * Backward: one CTA per sender with one warp per path group, walking the sender CSR;
-//     A is recomputed, never stored; grad_w and grad_y are edge-local writes; grad_x is
-//     reduced in registers and shared memory in a fixed order.
+//   * Backward: one one-warp CTA per (sender, path group), walking the sender CSR; A is
+//     recomputed, never stored; grad_w and grad_y are edge-local writes; grad_x is reduced in
+//     registers in a fixed order.  All groups run in one launch; the groups of one sender
+//     are ordered by a per-sender progress counter (the first group to touch a grad_x or
+//     grad_y block stores it, later groups add), so no floating-point atomics are used.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -158,6 +160,30 @@ __device__ __forceinline__ void ld16(T (&r)[N], const T* __restrict__ p, bool st
     for (int i = 0; i < N / 2; ++i) {
       const double2 v = stream ? __ldcs(reinterpret_cast<const double2*>(p) + i)
                                : __ldg(reinterpret_cast<const double2*>(p) + i);
+      r[2 * i] = v.x;
+      r[2 * i + 1] = v.y;
+    }
+  }
+}
+
+// The same through L2 only (coherent): for values another CTA of the same launch wrote.
+template <typename T, int N>
+__device__ __forceinline__ void ld16_l2(T (&r)[N], const T* __restrict__ p) {
+  if constexpr (std::is_same<T, float>::value) {
+    static_assert(N % 4 == 0, "float chunk");
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + i);
+      r[4 * i] = v.x;
+      r[4 * i + 1] = v.y;
+      r[4 * i + 2] = v.z;
+      r[4 * i + 3] = v.w;
+    }
+  } else {
+    static_assert(N % 2 == 0, "double chunk");
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const double2 v = __ldcg(reinterpret_cast<const double2*>(p) + i);
       r[2 * i] = v.x;
       r[2 * i + 1] = v.y;
     }
@@ -728,8 +754,11 @@ struct KBwd {
   void* grad_y;
   void* grad_w;
   int64_t n_nodes, n_edges;
+  int64_t units;        // senders (convolution) or sample ranges (tensor product)
   int C, sh_norm, n_chunks, stages;
   int* status;
+  int* ticket;          // CTA ticket counter (zero at launch)
+  int* done;            // per unit: path groups finished (zero at launch)
   double scale;
   double alpha[MAXP];
   float alpha_f[MAXP];  // the same path weights rounded once, for the float kernels
@@ -991,7 +1020,7 @@ __device__ __forceinline__ void bwd_put_dx(typename CF::T* __restrict__ row, con
     constexpr int D = 2 * L + 1;
     T* p = row + size_t(C) * (L * L) + size_t(4 * cb) * D;
     T v[K * D];
-    if constexpr (first_group_l1<CF>(L) != GI) ld16(v, p, false);
+    if constexpr (first_group_l1<CF>(L) != GI) ld16_l2(v, p);
 #pragma unroll
     for (int k = 0; k < K; ++k)
 #pragma unroll
@@ -1018,16 +1047,47 @@ __device__ __forceinline__ void bwd_put_dx(typename CF::T* __restrict__ row, con
   }
 }
 
-// Backward of path group GI.  Convolution: one CTA (one warp) per sender, walking its
-// out-edges through the sender CSR; tensor product: one CTA per contiguous sample range.
+// Ordering of the path groups of one unit.  Group GI of a unit adds to grad_x / grad_y blocks
+// that groups < GI of the same unit stored, so it starts only once done[unit] == GI (acquire),
+// and publishes done[unit] = GI + 1 after its writes (release).  The CTA that waits drew its
+// ticket after the CTA it waits for (tickets are group-major), so that CTA is resident or
+// finished and the chain ends at group 0: no deadlock, whatever order the hardware schedules
+// CTAs in.  The wait is bounded; on timeout the error is recorded and the group proceeds.
+__device__ __forceinline__ void bwd_wait_turn(const KBwd& a, int64_t unit, int gi) {
+  if (gi > 0 && threadIdx.x == 0) {
+    long long it = 0;
+    int v;
+    while (true) {
+      asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a.done + unit) : "memory");
+      if (v >= gi) break;
+      if (++it >= WAIT_LIMIT) {
+        record_error(a.status, E3_ERR_TIMEOUT);
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  __syncwarp();
+  // later bulk copies (async proxy) read what the earlier group wrote (generic proxy)
+  asm volatile("fence.proxy.async;" ::: "memory");
+}
+
+__device__ __forceinline__ void bwd_end_turn(const KBwd& a, int64_t unit, int gi) {
+  __threadfence();
+  __syncwarp();
+  if (threadIdx.x == 0)
+    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(a.done + unit), "r"(gi + 1) : "memory");
+}
+
+// Backward of path group GI for one unit.  Convolution: one CTA (one warp) per sender,
+// walking its out-edges through the sender CSR; tensor product: one CTA per sample range.
 template <class CF, int GI, bool CONV, int CC>
-__global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a) {
+__device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsigned char* smem) {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
   using SM = BwdSmem<CF, GI>;
   using MK = BwdMasks<CF, GI>;
   constexpr int NYP = SM::NYP;
-  extern __shared__ __align__(128) unsigned char smem[];
   const int C = CC > 0 ? CC : a.C;  // compile-time for the specialised multiplicities
   const int CB = C >> 2;            // CB <= 32: one warp covers every channel
   const int lane = threadIdx.x;
@@ -1056,7 +1116,6 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
   unsigned char* stages = smem + SM::stage_off(S);
 
   int64_t j0, j1;
-  const int64_t n = blockIdx.x;
   if constexpr (CONV) {
     j0 = a.row_ptr_src[n];
     j1 = a.row_ptr_src[n + 1];
@@ -1075,6 +1134,7 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
     *s_abort = 0;
     mbar_fence_init();
   }
+  bwd_wait_turn(a, n, GI);
   __syncthreads();
 
   T xr[K][GR::NXG], dx[K][GR::NXG], Y[CF::NY], dY[CF::NY];
@@ -1225,7 +1285,7 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
             else if (YB > 0)
               *p = sl[(WB + GB + XB) / sizeof(T) + m] + scale * v[j];
             else
-              *p += scale * v[j];
+              *p = __ldcg(p) + scale * v[j];
           }
           // group 0 also zero-fills harmonics blocks that no path uses
           if constexpr (MK::YZ != 0u) {
@@ -1252,6 +1312,7 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
     if (lane == 0)
       for (uint32_t q = consumed - 1; q < issued; ++q) mbar_wait(&bars[q % S], (q / S) & 1u, a.status);
     __syncthreads();
+    bwd_end_turn(a, n, GI);
     return;
   }
   if constexpr (CONV) {
@@ -1264,6 +1325,29 @@ __global__ void __launch_bounds__(32) bwd_kernel(const __grid_constant__ KBwd a)
       if (slice == 0) bwd_put_dx<CF, GI>(gx + size_t(n) * xrow, dx, C, cb, scale);
     }
   }
+  bwd_end_turn(a, n, GI);
+}
+
+// All path groups in one launch: every CTA draws a ticket; tickets are group-major (all units
+// of group 0, then group 1, ...), so at any time the SMs mostly run one group's code and the
+// next group's CTAs fill the SMs that the previous group's last CTAs leave idle.
+// Register budget: the largest float group body alone needs about 168 registers; the bound
+// keeps the merged kernel there (12 resident warps per SM by registers).  Double precision
+// keeps the compiler's choice.
+template <class CF>
+constexpr int bwd_min_blocks() {
+  return std::is_same<typename CF::T, float>::value ? 12 : 1;
+}
+
+template <class CF, bool CONV, int CC>
+__global__ void __launch_bounds__(32, bwd_min_blocks<CF>()) bwd_kernel(const __grid_constant__ KBwd a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  int t = 0;
+  if (threadIdx.x == 0) t = atomicAdd(a.ticket, 1);
+  t = __shfl_sync(0xffffffffu, t, 0);
+  const int g = int(t / a.units);
+  const int64_t n = t % a.units;
+  dispatch<CF::G>(g, [&](auto gc) { bwd_group<CF, decltype(gc)::value, CONV, CC>(a, n, smem); });
 }
 
 // =================================================================== host launchers ===
@@ -1321,41 +1405,13 @@ e3_status launch_fwd_cc(const e3_plan* plan, const FwdArgs& h, bool conv) {
   return E3_OK;
 }
 
-// One backward launch per path group, in group order on the caller's stream: a launch only
-// holds its group's code, and grad_x / grad_y blocks shared by several groups are stored by
-// the first and accumulated by the later launches (fixed order: deterministic).
-template <class CF, int GI, int CC>
-e3_status launch_bwd_group(KBwd a, bool conv, int64_t blocks, cudaStream_t s) {
-  const int CB = a.C / 4, NS = 32 / CB;
-  auto kern = conv ? bwd_kernel<CF, GI, true, CC> : bwd_kernel<CF, GI, false, CC>;
-  cudaFuncAttributes fa{};
-  cudaError_t err = cudaFuncGetAttributes(&fa, kern);
-  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(err));
-  const int regs = fa.numRegs > 0 ? fa.numRegs : 255;
-  const int ctas = std::max(1, std::min(32, 65536 / (((regs + 7) & ~7) * 32)));
-  const size_t budget = size_t(225) * 1024 / ctas;
-  const bool dy = a.grad_y != nullptr;
-  int S = 3;
-  while (S > 2 && BwdSmem<CF, GI>::total(a.C, NS, S, conv, dy) + 1024 > budget) --S;
-  a.stages = S;
-  const size_t smem = BwdSmem<CF, GI>::total(a.C, NS, S, conv, dy);
-  if (smem > size_t(227) * 1024) return fail(E3_ERR_UNSUPPORTED, "backward needs %zu bytes of shared memory", smem);
-  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
-  kern<<<unsigned(blocks), 32, smem, s>>>(a);
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "backward launch failed: %s", cudaGetErrorString(err));
-  return E3_OK;
-}
-
-template <class CF, int CC, int GI = 0>
-e3_status launch_bwd_groups(const KBwd& a, bool conv, int64_t blocks, cudaStream_t s) {
+// Shared memory of the merged backward: the largest of the groups' layouts.
+template <class CF, int GI = 0>
+size_t bwd_smem_max(int C, int NS, int S, bool conv, bool dy) {
   if constexpr (GI < CF::G) {
-    const e3_status st = launch_bwd_group<CF, GI, CC>(a, conv, blocks, s);
-    if (st != E3_OK) return st;
-    return launch_bwd_groups<CF, CC, GI + 1>(a, conv, blocks, s);
+    return std::max(BwdSmem<CF, GI>::total(C, NS, S, conv, dy), bwd_smem_max<CF, GI + 1>(C, NS, S, conv, dy));
   } else {
-    return E3_OK;
+    return 0;
   }
 }
 
@@ -1387,18 +1443,45 @@ e3_status launch_bwd_cc(const e3_plan* plan, const BwdArgs& h, bool conv) {
   const int CB = plan->C / 4;
   if (CB > 32) return fail(E3_ERR_UNSUPPORTED, "the backward kernels need a multiplicity of at most 128");
   const int NS = 32 / CB;
-  int64_t blocks;
+  int64_t units;
   if (conv) {
-    blocks = h.n_nodes;
+    units = h.n_nodes;
     a.n_chunks = 0;
   } else {
     const int64_t n_units = (h.n_nodes + NS - 1) / NS;
-    blocks = std::min<int64_t>(n_units, int64_t(sm_count()) * 16);
-    a.n_chunks = int(blocks);
+    units = std::min<int64_t>(n_units, int64_t(sm_count()) * 16);
+    a.n_chunks = int(units);
   }
+  if (units == 0) return E3_OK;
+  const int64_t blocks = units * CF::G;
   if (blocks >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "grid too large");
-  if (blocks == 0) return E3_OK;
-  return launch_bwd_groups<CF, CC>(a, conv, blocks, static_cast<cudaStream_t>(h.stream));
+  if (h.workspace_bytes < backward_workspace_bytes(units)) return fail(E3_ERR_INVALID_ARG, "workspace too small");
+  a.units = units;
+  a.ticket = static_cast<int*>(h.workspace);
+  a.done = reinterpret_cast<int*>(static_cast<unsigned char*>(h.workspace) + 16);
+  const cudaStream_t s = static_cast<cudaStream_t>(h.stream);
+  cudaError_t err = cudaMemsetAsync(h.workspace, 0, 16 + 4 * size_t(units), s);
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
+
+  auto kern = conv ? bwd_kernel<CF, true, CC> : bwd_kernel<CF, false, CC>;
+  cudaFuncAttributes fa{};
+  err = cudaFuncGetAttributes(&fa, kern);
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(err));
+  const int regs = fa.numRegs > 0 ? fa.numRegs : 255;
+  const int ctas = std::max(1, std::min(32, 65536 / (((regs + 7) & ~7) * 32)));
+  const size_t budget = size_t(225) * 1024 / ctas;
+  const bool dy = a.grad_y != nullptr;
+  int S = 3;
+  while (S > 2 && bwd_smem_max<CF>(a.C, NS, S, conv, dy) + 1024 > budget) --S;
+  a.stages = S;
+  const size_t smem = bwd_smem_max<CF>(a.C, NS, S, conv, dy);
+  if (smem > size_t(227) * 1024) return fail(E3_ERR_UNSUPPORTED, "backward needs %zu bytes of shared memory", smem);
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
+  kern<<<unsigned(blocks), 32, smem, s>>>(a);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "backward launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
 }
 
 // Multiplicities compiled with C as a constant (all channel address arithmetic folds to

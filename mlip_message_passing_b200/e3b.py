@@ -26,6 +26,7 @@ SYMBOLS = [
     "e3_device_status", "e3_cg_dense", "e3_supported", "e3_tp_forward", "e3_tp_backward",
     "e3_spherical_harmonics", "e3_csr_workspace_size", "e3_csr_build", "e3_gather_rows",
     "e3_conv_forward", "e3_conv_backward", "e3_last_error", "e3_csr_build_static",
+    "e3_backward_workspace_size",
 ]
 
 
@@ -58,7 +59,8 @@ def _load():
         "e3_cg_dense": [I32, I32, I32, ctypes.POINTER(D)],
         "e3_supported": [],
         "e3_tp_forward": [VP, I64, VP, VP, VP, VP, VP],
-        "e3_tp_backward": [VP, I64, VP, VP, VP, VP, VP, VP, VP, VP],
+        "e3_tp_backward": [VP, I64, VP, VP, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP],
+        "e3_backward_workspace_size": [I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_spherical_harmonics": [I32, I64, VP, ctypes.c_int, ctypes.c_int, VP, VP],
         "e3_csr_workspace_size": [I64, I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_csr_build": [I64, I64, VP, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP],
@@ -66,7 +68,7 @@ def _load():
         "e3_gather_rows": [I64, I64, I64, VP, VP, VP, VP],
         "e3_conv_forward": [VP, I64, I64, VP, VP, VP, VP, VP, ctypes.c_int, VP, D, VP, VP],
         "e3_conv_backward": [VP, I64, I64, VP, VP, VP, VP, VP, VP, VP, VP, ctypes.c_int, VP, VP, D, VP, VP, VP,
-                             VP],
+                             VP, ctypes.c_size_t, VP],
         "e3_last_error": [],
     }
     for name, args in sig.items():
@@ -218,9 +220,17 @@ def tp_backward(plan, x, y, w, grad_out, need_x=True, need_y=True, need_w=True):
     gx = torch.empty_like(x) if need_x else None
     gy = torch.empty_like(y) if need_y else None
     gw = torch.empty_like(w) if need_w else None
+    ws = backward_workspace(B, dev)
     _check(lib.e3_tp_backward(plan.handle, B, _ptr(x), _ptr(y), _ptr(w), _ptr(grad_out), _ptr(gx), _ptr(gy),
-                              _ptr(gw), _stream()))
+                              _ptr(gw), _ptr(ws), ws.numel(), _stream()))
     return gx, gy, gw
+
+
+def backward_workspace(n, device):
+    """Device workspace for e3_tp_backward (n = B) / e3_conv_backward (n = N), from torch's allocator."""
+    nbytes = ctypes.c_size_t()
+    _check(lib.e3_backward_workspace_size(n, ctypes.byref(nbytes)))
+    return torch.empty(nbytes.value, dtype=torch.uint8, device=device)
 
 
 def spherical_harmonics(lmax, vec, sh_norm="component", out=None):
@@ -325,10 +335,11 @@ def conv_backward(plan, graph, x, w, grad_out, y=None, edge_vec=None, sh_norm="c
     gx = torch.empty_like(x) if need_x else None
     gy = torch.empty((E, plan.dim_in2), dtype=dt, device=dev) if need_y else None
     gw = torch.empty_like(w) if need_w else None
+    ws = backward_workspace(N, dev)
     _check(lib.e3_conv_backward(plan.handle, N, E, _ptr(graph.row_ptr_dst), _ptr(graph.src), _ptr(graph.dst),
                                 _ptr(graph.row_ptr_src), _ptr(graph.perm_src), _ptr(x), _ptr(y), _ptr(edge_vec),
                                 _SH_NORMS[sh_norm], _ptr(w), _ptr(grad_out), float(out_scale), _ptr(gx),
-                                _ptr(gy), _ptr(gw), _stream()))
+                                _ptr(gy), _ptr(gw), _ptr(ws), ws.numel(), _stream()))
     return gx, gy, gw
 
 

@@ -247,6 +247,33 @@ def test_conv_edge_cases(e3b):
     assert rel_err(h(out), ref) <= 1e-5 and torch.all(out[5] == 0) and torch.all(out[2] == 0)
 
 
+def test_backward_workspace_is_checked(e3b):
+    """The backward refuses a missing, misaligned or short workspace before any launch."""
+    p = gplan(e3b, 8, 1, 2, 2, torch.float32)
+    n = 4
+    graph = e3b.Graph(n, t(np.array([0, 1, 2, 3], np.int32)), t(np.array([1, 2, 3, 0], np.int32)))
+    x = torch.randn(n, p.dim_in1, device=DEV)
+    w = torch.randn(4, p.weight_numel, device=DEV)
+    go = torch.randn(n, p.dim_out, device=DEV)
+    vec = torch.randn(4, 3, device=DEV)
+    gx = torch.empty_like(x)
+    ws = e3b.backward_workspace(n, DEV)
+    P = e3b._ptr
+
+    def call(wsp, nbytes):
+        return e3b.lib.e3_conv_backward(p.handle, n, 4, P(graph.row_ptr_dst), P(graph.src), P(graph.dst),
+                                        P(graph.row_ptr_src), P(graph.perm_src), P(x), None, P(vec), 0, P(w),
+                                        P(go), 1.0, P(gx), None, None, wsp, nbytes, e3b._stream())
+
+    assert call(None, ws.numel()) == e3b.E3_ERR_INVALID_ARG
+    assert call(P(ws[8:]), ws.numel() - 8) == e3b.E3_ERR_INVALID_ARG
+    assert call(P(ws), 16) == e3b.E3_ERR_INVALID_ARG
+    assert call(P(ws), ws.numel()) == e3b.E3_OK
+    torch.cuda.synchronize()
+    ref, _, _ = e3b.conv_backward(p, graph, x, w, go, edge_vec=vec, need_y=False, need_w=False)
+    assert torch.equal(gx, ref)
+
+
 def test_conv_bad_index_is_reported_not_dereferenced(e3b):
     p = gplan(e3b, 8, 1, 2, 2, torch.float32)
     n = 4

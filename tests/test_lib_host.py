@@ -107,3 +107,13 @@ def test_csr_workspace_and_argument_errors(e3b):
     assert e3b.lib.e3_gather_rows(4, 4, 6, None, None, None, None) == e3b.E3_ERR_SHAPE
     assert e3b.lib.e3_spherical_harmonics(4, 10, None, 0, 0, None, None) == e3b.E3_ERR_UNSUPPORTED
     assert e3b.lib.e3_tp_forward(None, 1, None, None, None, None, None) == e3b.E3_ERR_INVALID_ARG
+
+
+def test_backward_workspace_size(e3b):
+    n = ctypes.c_size_t()
+    for units in (0, 1, 3000, 1 << 20):
+        assert e3b.lib.e3_backward_workspace_size(units, ctypes.byref(n)) == e3b.E3_OK
+        assert n.value >= 16 + 4 * units and n.value % 256 == 0
+    assert e3b.lib.e3_backward_workspace_size(-1, ctypes.byref(n)) == e3b.E3_ERR_SHAPE
+    assert e3b.lib.e3_backward_workspace_size(1 << 31, ctypes.byref(n)) == e3b.E3_ERR_SHAPE
+    assert e3b.lib.e3_backward_workspace_size(5, None) == e3b.E3_ERR_INVALID_ARG
