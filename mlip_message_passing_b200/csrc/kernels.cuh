@@ -458,9 +458,11 @@ struct FwdAcc {
 // ------------------------------------------------------------ async copy machinery ---
 // One thread per CTA streams the weight and x slices of upcoming edges into a ring of shared
 // memory stages with cp.async.bulk (1-D TMA, no multicast); completion is tracked by one
-// mbarrier per stage (transaction bytes).  Every wait is bounded: after WAIT_LIMIT polls the
-// kernel records E3_ERR_TIMEOUT and stops issuing work.
+// mbarrier per stage (transaction bytes).  Every wait is bounded: after WAIT_NS nanoseconds
+// of the global timer (WAIT_LIMIT polls for the progress counters of the backward) the kernel
+// records E3_ERR_TIMEOUT and stops issuing work.
 constexpr long long WAIT_LIMIT = 1ll << 24;
+constexpr unsigned long long WAIT_NS = 1000000000ull;
 constexpr int FWD_WIN = 64;  // in-edges whose sender ids and harmonics are staged at once
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -473,14 +475,30 @@ __device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
       : "r"(smem_addr(bar)), "r"(parity)
       : "memory");
   return ok != 0;
+}
+// try_wait with a suspend-time hint: the warp is parked until the phase completes or about
+// 20 microseconds pass, instead of polling.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(20000u)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
 }
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -488,10 +506,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                "l"(src), "r"(bytes), "r"(smem_addr(bar))
                : "memory");
 }
-// bounded wait; false after WAIT_LIMIT polls (the error is recorded)
+// bounded wait; false after WAIT_NS (the error is recorded).  The common case -- the copy
+// landed while the previous stage was being consumed -- costs one test.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
-  for (long long i = 0; i < WAIT_LIMIT; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  do {
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+  } while (global_ns() - t0 < WAIT_NS);
   record_error(status, E3_ERR_TIMEOUT);
   return false;
 }
