@@ -930,14 +930,19 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
 #pragma unroll
       for (int m1 = 0; m1 < D1; ++m1) dx[k][XO + m1] = fma(wa[k], t[k][m1], dx[k][XO + m1]);
     if (want_dy) {  // grad_y[m2] += sum_{m1,m3} C[m1,m2,m3] sum_k alpha_p w_k x_k[m1] g_k[m3]
-      T dyp[2 * L2 + 1];
+      // the weight scales the shorter of the x and grad_out blocks
+      constexpr bool SX = D1 <= D3;
+      T xw[K][SX ? D1 : 1], gw_[K][SX ? 1 : D3];
 #pragma unroll
-      for (int i = 0; i < 2 * L2 + 1; ++i) dyp[i] = T(0);
-      T xw[K][D1];
+      for (int k = 0; k < K; ++k) {
+        if constexpr (SX) {
 #pragma unroll
-      for (int k = 0; k < K; ++k)
+          for (int m1 = 0; m1 < D1; ++m1) xw[k][m1] = wa[k] * xr[k][XO + m1];
+        } else {
 #pragma unroll
-        for (int m1 = 0; m1 < D1; ++m1) xw[k][m1] = wa[k] * xr[k][XO + m1];
+          for (int m3 = 0; m3 < D3; ++m3) gw_[k][m3] = wa[k] * g[k][m3];
+        }
+      }
       static_for<0, D1>([&](auto m1c) {
         constexpr int M1I = decltype(m1c)::value;
         static_for<0, D3>([&](auto m3c) {
@@ -945,19 +950,22 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
           if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) {
             T z = T(0);
 #pragma unroll
-            for (int k = 0; k < K; ++k) z = fma(xw[k][M1I], g[k][M3I], z);
+            for (int k = 0; k < K; ++k) {
+              if constexpr (SX)
+                z = fma(xw[k][M1I], g[k][M3I], z);
+              else
+                z = fma(xr[k][XO + M1I], gw_[k][M3I], z);
+            }
             static_for<-L2, L2 + 1>([&](auto m2c) {
               constexpr int M2 = decltype(m2c)::value;
               if constexpr (cg_nz(L1, L2, L3, M1I - L1, M2, M3I - L3)) {
                 constexpr int I = cg_index(L1, L2, L3, M1I - L1, M2, M3I - L3);
-                dyp[L2 + M2] = fma(CGT<T>::template get<I>(), z, dyp[L2 + M2]);
+                dY[L2 * L2 + L2 + M2] = fma(CGT<T>::template get<I>(), z, dY[L2 * L2 + L2 + M2]);
               }
             });
           }
         });
       });
-#pragma unroll
-      for (int i = 0; i < 2 * L2 + 1; ++i) dY[L2 * L2 + i] += dyp[i];
     }
   });
 }
@@ -980,15 +988,32 @@ struct YUse {
   static constexpr Tab TAB = make();
   static constexpr int NU = TAB.n;
   static constexpr int VP = NU <= 1 ? 1 : (NU <= 2 ? 2 : (NU <= 4 ? 4 : (NU <= 8 ? 8 : 16)));
+  static constexpr bool CONTIG = [] {
+    for (int i = 0; i < TAB.n; ++i)
+      if (TAB.comp[i] != TAB.comp[0] + i) return false;
+    return true;
+  }();
+  // harmonics component of used index u (u < NU)
+  static __device__ __forceinline__ int comp_of(int u) {
+    if constexpr (CONTIG) {
+      return TAB.comp[0] + u;
+    } else {
+      int m = 0;
+      static_for<0, NU>([&](auto qc) {
+        constexpr int Q = decltype(qc)::value;
+        if (u == Q) m = TAB.comp[Q];
+      });
+      return m;
+    }
+  }
 };
 
 // Sum v[0..VP) over the W lanes of a slice (lane bits below W) by recursive halving: after
 // each level a lane keeps half of its values and adds its partner's copy of that half.  On
-// return v[0..max(VP/W, 1)) hold totals of components base + j (same base for lanes that
-// differ only in the bits below W/VP when VP < W).
+// return v[0..max(VP/W, 1)) hold totals of components reduce_scatter_base(W, cb) + j (the same
+// base for lanes that differ only in the bits below W/VP when VP < W).
 template <typename T, int VP>
-__device__ __forceinline__ int reduce_scatter(T (&v)[VP], int W, int cb) {
-  int base = 0;
+__device__ __forceinline__ void reduce_scatter(T (&v)[VP], int W, int cb) {
   int len = VP;
 #pragma unroll
   for (int lvl = 0; lvl < 5; ++lvl) {
@@ -1004,11 +1029,22 @@ __device__ __forceinline__ int reduce_scatter(T (&v)[VP], int W, int cb) {
         const T keep = up ? v[i + half] : v[i];
         v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
       }
-      if (up) base += half;
       len = half;
     } else {
       v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
     }
+  }
+}
+
+// First component a lane holds after reduce_scatter (fixed per lane).
+template <int VP>
+__device__ __forceinline__ int reduce_scatter_base(int W, int cb) {
+  int base = 0, len = VP;
+  for (int lvl = 0; lvl < 5; ++lvl) {
+    const int o = W >> (lvl + 1);
+    if (o < 1 || len <= 1) break;
+    len /= 2;
+    if (cb & o) base += len;
   }
   return base;
 }
@@ -1166,6 +1202,10 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsign
 #pragma unroll
     for (int j = 0; j < GR::NXG; ++j) dx[k][j] = T(0);
   if constexpr (CONV) load_x<CF, GR>(xr, x + size_t(n) * xrow, C, cb);
+  // grad_y components this lane writes after the per-edge reduction (fixed per lane)
+  const int ybase = reduce_scatter_base<YUse<CF, GI>::VP>(CB, cb);
+  const int yheld = YUse<CF, GI>::VP >= CB ? YUse<CF, GI>::VP / CB : 1;
+  const bool ywriter = YUse<CF, GI>::VP >= CB || (cb & (CB / YUse<CF, GI>::VP - 1)) == 0;
 
   int prod_slot = 0, cons_slot = 0;
   uint32_t cons_phase = 0, issued = 0, consumed = 0;
@@ -1287,21 +1327,14 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsign
             v[U] = T(0);
           }
         });
-        const int base = reduce_scatter<T, YU::VP>(v, CB, cb);
-        const int held = YU::VP >= CB ? YU::VP / CB : 1;
-        const bool writer = YU::VP >= CB || (cb & (CB / YU::VP - 1)) == 0;
-        if (mine && writer) {
+        reduce_scatter<T, YU::VP>(v, CB, cb);
+        if (mine && ywriter) {
 #pragma unroll
           for (int j = 0; j < YU::VP; ++j) {
-            if (j >= held) break;
-            const int u = base + j;
+            if (j >= yheld) break;
+            const int u = ybase + j;
             if (u >= YU::NU) break;
-            int m = 0;
-            static_for<0, YU::NU>([&](auto qc) {
-              constexpr int Q = decltype(qc)::value;
-              constexpr int MQ = YU::TAB.comp[Q];
-              if (u == Q) m = MQ;
-            });
+            const int m = YU::comp_of(u);
             T* p = gy + e * CF::NY + m;
             if (MK::YS & (1u << block_of(m)))
               *p = scale * v[j];
