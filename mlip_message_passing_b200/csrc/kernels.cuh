@@ -662,33 +662,24 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
     fwd_stage_window<CF, CONV>(a, e0, ws, cnt, ysh, src_s);
     __syncthreads();
     const int steps = (cnt + NS - 1) / NS;
-    // producer: warp 0; lane 0 posts the expected bytes, then lanes move one slice each
-    // (item 2j: weights of the step's j-th edge, item 2j+1: its x slice)
+    // producer: thread 0 posts the expected bytes, then thread j (< edges in the step) copies
+    // the weights and the x slice of the step's j-th edge.  An edge whose sender id is out of
+    // range copies row 0 instead (the edge is skipped by the consumer), so the byte count of
+    // a stage depends only on its number of edges.
     auto issue = [&](int st) {
-      if (tid < 32) {
-        uint64_t* bar = &bars[prod_slot];
-        unsigned char* dst = stages + size_t(prod_slot) * STAGE;
-        int nv = 0;
-        for (int j = tid; j < NS; j += 32) {
-          const int r = st * NS + j;
-          nv += (r < cnt && (!CONV || src_s[r] >= 0)) ? 1 : 0;
-        }
-        nv = __reduce_add_sync(0xffffffffu, nv);
-        if (tid == 0) mbar_arrive_expect_tx(bar, uint32_t(nv) * SLOT);
-        __syncwarp();
-        for (int it = tid; it < 2 * NS; it += 32) {
-          const int j = it >> 1;
-          const int r = st * NS + j;
-          if (r >= cnt) continue;
-          const int64_t e = e0 + ws + r;
-          if (it & 1) {
-            int64_t row = e;
-            if constexpr (CONV) row = src_s[r];
-            if (row >= 0) bulk_load(dst + size_t(j) * SLOT + WB, x + size_t(row) * xrow + size_t(GR::XB) * C, XB, bar);
-          } else if (!CONV || src_s[r] >= 0) {
-            bulk_load(dst + size_t(j) * SLOT, w + e * a.w_stride + size_t(GR::PB) * C, WB, bar);
-          }
-        }
+      uint64_t* bar = &bars[prod_slot];
+      unsigned char* dst = stages + size_t(prod_slot) * STAGE;
+      const int nv = min(NS, cnt - st * NS);
+      if (tid == 0) mbar_arrive_expect_tx(bar, uint32_t(nv) * SLOT);
+      __syncwarp();
+      if (tid < nv) {
+        const int r = st * NS + tid;
+        const int64_t e = e0 + ws + r;
+        int64_t row = e;
+        if constexpr (CONV) row = max(src_s[r], 0);
+        unsigned char* d = dst + size_t(tid) * SLOT;
+        bulk_load(d, w + e * a.w_stride + size_t(GR::PB) * C, WB, bar);
+        bulk_load(d + WB, x + size_t(row) * xrow + size_t(GR::XB) * C, XB, bar);
       }
       prod_slot = prod_slot + 1 == S ? 0 : prod_slot + 1;
       ++issued;
@@ -1238,34 +1229,25 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsign
     }
     __syncthreads();
     const int steps = (cnt + NS - 1) / NS;
-    // producer: lane 0 posts the expected bytes, then lanes move one slice each (per edge:
-    // weights, grad_out of the receiver, x for the tensor product, the grad_y row to add to)
-    constexpr int ITEMS = 4;
+    // producer: lane 0 posts the expected bytes, then lane j (< edges in the step) copies the
+    // slices of the step's j-th edge: weights, grad_out of the receiver, x for the tensor
+    // product, the grad_y row to add to.  An edge with an id out of range copies edge 0 /
+    // node 0 instead (the consumer skips it), so a stage's byte count depends only on its
+    // number of edges.
     auto issue = [&](int st) {
       uint64_t* bar = &bars[prod_slot];
       unsigned char* dst = stages + size_t(prod_slot) * STAGE;
-      int nv = 0;
-      for (int j = lane; j < NS; j += 32) {
-        const int r = st * NS + j;
-        nv += (r < cnt && eid[r] >= 0) ? 1 : 0;
-      }
-      nv = __reduce_add_sync(0xffffffffu, nv);
+      const int nv = min(NS, cnt - st * NS);
       if (lane == 0) mbar_arrive_expect_tx(bar, uint32_t(nv) * SLOT);
       __syncwarp();
-      for (int it = lane; it < ITEMS * NS; it += 32) {
-        const int j = it / ITEMS, kind = it % ITEMS;
-        const int r = st * NS + j;
-        if (r >= cnt || eid[r] < 0) continue;
-        const int64_t e = eid[r];
-        unsigned char* d = dst + size_t(j) * SLOT;
-        if (kind == 0)
-          bulk_load(d, w + e * wrow + size_t(GR::PB) * C, WB, bar);
-        else if (kind == 1)
-          bulk_load(d + WB, g + size_t(did[r]) * orow + size_t(GR::OB) * C, GB, bar);
-        else if (kind == 2 && XB > 0)
-          bulk_load(d + WB + GB, x + size_t(e) * xrow + size_t(GR::XB) * C, XB, bar);
-        else if (kind == 3 && YB > 0)
-          bulk_load(d + WB + GB + XB, gy + size_t(e) * CF::NY, YB, bar);
+      if (lane < nv) {
+        const int r = st * NS + lane;
+        const int64_t e = max(eid[r], 0);
+        unsigned char* d = dst + size_t(lane) * SLOT;
+        bulk_load(d, w + e * wrow + size_t(GR::PB) * C, WB, bar);
+        bulk_load(d + WB, g + size_t(did[r]) * orow + size_t(GR::OB) * C, GB, bar);
+        if (XB > 0) bulk_load(d + WB + GB, x + size_t(e) * xrow + size_t(GR::XB) * C, XB, bar);
+        if (YB > 0) bulk_load(d + WB + GB + XB, gy + size_t(e) * CF::NY, YB, bar);
       }
       prod_slot = prod_slot + 1 == S ? 0 : prod_slot + 1;
       ++issued;
