@@ -987,12 +987,14 @@ struct YUse {
   // harmonics component of used index u (u < NU)
   static __device__ __forceinline__ int comp_of(int u) {
     if constexpr (CONTIG) {
-      return TAB.comp[0] + u;
+      constexpr int C0 = TAB.comp[0];
+      return C0 + u;
     } else {
       int m = 0;
       static_for<0, NU>([&](auto qc) {
         constexpr int Q = decltype(qc)::value;
-        if (u == Q) m = TAB.comp[Q];
+        constexpr int MQ = TAB.comp[Q];
+        if (u == Q) m = MQ;
       });
       return m;
     }
@@ -1508,9 +1510,13 @@ e3_status launch_bwd_cc(const e3_plan* plan, const BwdArgs& h, bool conv) {
   const int regs = fa.numRegs > 0 ? fa.numRegs : 255;
   const int ctas = std::max(1, std::min(32, 65536 / (((regs + 7) & ~7) * 32)));
   const size_t budget = size_t(225) * 1024 / ctas;
+  // Ring depth: two stages when they cost no resident CTAs, else one.  A backward step is
+  // long enough that more resident warps hide the copy latency better than a second stage
+  // does (measured on the water-box workload: 8 CTAs/SM with two stages are slower than 12
+  // with one).
   const bool dy = a.grad_y != nullptr;
-  int S = 3;
-  while (S > 2 && bwd_smem_max<CF>(a.C, NS, S, conv, dy) + 1024 > budget) --S;
+  int S = 2;
+  while (S > 1 && bwd_smem_max<CF>(a.C, NS, S, conv, dy) + 1024 > budget) --S;
   a.stages = S;
   const size_t smem = bwd_smem_max<CF>(a.C, NS, S, conv, dy);
   if (smem > size_t(227) * 1024) return fail(E3_ERR_UNSUPPORTED, "backward needs %zu bytes of shared memory", smem);
