@@ -506,6 +506,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                "l"(src), "r"(bytes), "r"(smem_addr(bar))
                : "memory");
 }
+// Bring [p, p + bytes) into L2 ahead of its bulk copy (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // bounded wait; false after WAIT_NS (the error is recorded).  The common case -- the copy
 // landed while the previous stage was being consumed -- costs one test.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
@@ -1257,6 +1262,12 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsign
     for (int st = 0; st < S && st < steps; ++st) issue(st);
 
     for (int st = 0; st < steps; ++st) {
+      {
+        // the weight rows of the edges the next copy will fetch go to L2 now, so that copy
+        // does not wait on DRAM
+        const int rp = (st + S) * NS + lane;
+        if (lane < NS && rp < cnt) prefetch_l2(w + max(eid[rp], 0) * wrow + size_t(GR::PB) * C, WB);
+      }
       const int slot = cons_slot;
       const bool okw = mbar_wait(&bars[slot], cons_phase, a.status);
       if (!okw) *s_abort = 1;
