@@ -67,3 +67,61 @@ def real_sh(l, vec):
 def real_sh_all(lmax, vec):
     """Concatenated [Y^0 | Y^1 | ... | Y^lmax] -> [n, (lmax+1)^2] (irreps 1x0e+1x1o+...)."""
     return np.concatenate([real_sh(l, vec) for l in range(lmax + 1)], axis=1)
+
+
+def real_sh_grad(l, vec):
+    """Jacobian d Y^l / d vec of the component-normalised harmonics -> [n, 2l+1, 3].
+
+    Y depends on vec only through u = vec/|vec|, so dY/dvec = (1/r) (I - u u^T) grad_u F(u) for
+    any smooth F that equals Y on the unit sphere.  F is the formula of ``real_sh`` read as a
+    function of independent (x, y, z):
+        F_lm = N_lm * P_l^{(|m|)}(z) * A_m(x, y),   A_m = Re / Im (x + i y)^{|m|}, A_0 = 1,
+        dF/dx = N P^{(|m|)}(z) * Re / Im (|m| (x + i y)^{|m|-1}),
+        dF/dy = N P^{(|m|)}(z) * Re / Im (i |m| (x + i y)^{|m|-1}),
+        dF/dz = N P^{(|m|+1)}(z) * A_m.
+    At vec = 0 (where Y is set to Y^0 = 1, Y^{l>0} = 0) the gradient is defined as 0.
+    """
+    vec = np.asarray(vec, dtype=np.float64)
+    n = vec.shape[0]
+    out = np.zeros((n, 2 * l + 1, 3))
+    if l == 0:
+        return out
+    r = np.sqrt(np.sum(vec * vec, axis=1))
+    nz = r > 0
+    u = np.zeros_like(vec)
+    u[nz] = vec[nz] / r[nz, None]
+    x, y, z = u[:, 0], u[:, 1], u[:, 2]
+    pl = np.polynomial.polynomial.Polynomial(_legendre_coeffs(l))
+    xy = x + 1j * y
+    gu = np.zeros((n, 2 * l + 1, 3))
+    for m in range(-l, l + 1):
+        am = abs(m)
+        dp = pl.deriv(am) if am > 0 else pl
+        dp1 = pl.deriv(am + 1)
+        norm = sqrt((2 * l + 1) * factorial(l - am) / factorial(l + am))
+        if m != 0:
+            norm *= sqrt(2.0)
+        if m == 0:
+            ang, dax, day = np.ones(n), np.zeros(n), np.zeros(n)
+        else:
+            trig = xy ** am
+            dtrig = am * xy ** (am - 1)
+            pick = (lambda c: c.real) if m > 0 else (lambda c: c.imag)
+            ang, dax, day = pick(trig), pick(dtrig), pick(1j * dtrig)
+        gu[:, m + l, 0] = norm * dp(z) * dax
+        gu[:, m + l, 1] = norm * dp(z) * day
+        gu[:, m + l, 2] = norm * dp1(z) * ang
+    # project out the radial part and scale by 1/r
+    radial = np.einsum("nmk,nk->nm", gu, u)
+    out[nz] = (gu[nz] - radial[nz][:, :, None] * u[nz][:, None, :]) / r[nz, None, None]
+    return out
+
+
+def real_sh_all_grad(lmax, vec):
+    """Jacobian of ``real_sh_all`` -> [n, (lmax+1)^2, 3]."""
+    return np.concatenate([real_sh_grad(l, vec) for l in range(lmax + 1)], axis=1)
+
+
+def sh_backward(lmax, vec, grad_y):
+    """grad_vec[i] = sum_m grad_y[i, m] dY_m(vec_i)/dvec_i for the concatenated harmonics."""
+    return np.einsum("nm,nmk->nk", np.asarray(grad_y, dtype=np.float64), real_sh_all_grad(lmax, vec))

@@ -149,3 +149,36 @@ def test_csr_unstable_sort(monkeypatch):
 
     monkeypatch.setattr(oracle, "csr_build", bad)
     assert _caught([pins.test_csr_bit_exact_against_loops])
+
+
+SH_GRAD_PINS = [lambda: pins.test_sh_grad_matches_central_differences(2),
+                lambda: pins.test_sh_grad_matches_central_differences(3),
+                pins.test_sh_grad_closed_form_l1,
+                lambda: pins.test_sh_grad_radial_scaling_and_rotation(2)]
+
+
+def _patch_sh_grad(monkeypatch, src_old, src_new):
+    """Recompile real_sh_grad with one line changed."""
+    import inspect
+    import textwrap
+    src = textwrap.dedent(inspect.getsource(osh.real_sh_grad))
+    assert src_old in src
+    ns = dict(vars(osh))
+    exec(compile(src.replace(src_old, src_new), "mutant", "exec"), ns)
+    monkeypatch.setattr(osh, "real_sh_grad", ns["real_sh_grad"])
+    monkeypatch.setattr(oracle, "real_sh_grad", ns["real_sh_grad"])
+
+
+def test_sh_grad_without_radial_projection(monkeypatch):
+    _patch_sh_grad(monkeypatch, "(gu[nz] - radial[nz][:, :, None] * u[nz][:, None, :])", "gu[nz]")
+    assert _caught(SH_GRAD_PINS)
+
+
+def test_sh_grad_y_derivative_missing_i(monkeypatch):
+    _patch_sh_grad(monkeypatch, "pick(1j * dtrig)", "pick(dtrig)")
+    assert _caught(SH_GRAD_PINS)
+
+
+def test_sh_grad_wrong_legendre_derivative(monkeypatch):
+    _patch_sh_grad(monkeypatch, "dp1 = pl.deriv(am + 1)", "dp1 = pl.deriv(am)")
+    assert _caught(SH_GRAD_PINS)

@@ -99,6 +99,58 @@ def test_sh_equivariance_and_wigner_homomorphism(l):
         np.testing.assert_allclose(D1, P @ R1 @ P.T, atol=1e-12)
 
 
+@pytest.mark.parametrize("l", [0, 1, 2, 3])
+def test_sh_grad_matches_central_differences(l):
+    """The analytic Jacobian against central differences of real_sh (an independent
+    computation; h = 1e-6: truncation below 1e-9 down to |v| = 0.2, rounding ~1e-10)."""
+    rng = np.random.default_rng(40 + l)
+    v = rng.standard_normal((40, 3)) * rng.uniform(0.5, 3.0, (40, 1))
+    J = oracle.real_sh_grad(l, v)
+    h = 1e-6
+    fd = np.zeros_like(J)
+    for k in range(3):
+        e = np.zeros(3)
+        e[k] = h
+        fd[:, :, k] = (real_sh(l, v + e) - real_sh(l, v - e)) / (2 * h)
+    assert np.max(np.abs(J - fd)) <= 1e-8
+
+
+def test_sh_grad_closed_form_l1():
+    """Y^1 = sqrt(3) (y, z, x) / r, so dY_(i)/dv = sqrt(3) (e_i / r - v_i v / r^3)."""
+    rng = np.random.default_rng(44)
+    v = rng.standard_normal((20, 3))
+    r = np.linalg.norm(v, axis=1)
+    J = oracle.real_sh_grad(1, v)
+    for comp, axis in enumerate((1, 2, 0)):
+        ref = -v[:, axis, None] * v / r[:, None] ** 3
+        ref[:, axis] += 1 / r
+        np.testing.assert_allclose(J[:, comp, :], math.sqrt(3) * ref, atol=1e-13)
+
+
+@pytest.mark.parametrize("l", [1, 2, 3])
+def test_sh_grad_radial_scaling_and_rotation(l):
+    """Y(c v) = Y(v): the Jacobian is orthogonal to v and scales as 1/c; Y(R v) = D Y(v):
+    J(R v) R = D J(v)."""
+    rng = np.random.default_rng(50 + l)
+    v = rng.standard_normal((25, 3))
+    J = oracle.real_sh_grad(l, v)
+    assert np.max(np.abs(np.einsum("nmk,nk->nm", J, v))) <= 1e-12
+    np.testing.assert_allclose(oracle.real_sh_grad(l, 2.5 * v), J / 2.5, atol=1e-13)
+    R = rand_rot(rng)
+    D = wigner_real(l, R, rng)
+    lhs = np.einsum("nmk,kj->nmj", oracle.real_sh_grad(l, v @ R.T), R)
+    rhs = np.einsum("ab,nbk->nak", D, J)
+    np.testing.assert_allclose(lhs, rhs, atol=1e-11)
+
+
+def test_sh_grad_zero_vector_and_backward_contraction():
+    v = np.array([[0.0, 0.0, 0.0], [0.3, -1.2, 0.7]])
+    J = oracle.real_sh_all_grad(3, v)
+    assert J.shape == (2, 16, 3) and np.all(J[0] == 0) and np.all(J[1, 0] == 0)
+    g = np.random.default_rng(45).standard_normal((2, 16))
+    np.testing.assert_allclose(oracle.sh_backward(3, v, g), np.einsum("nm,nmk->nk", g, J), atol=1e-15)
+
+
 # ------------------------------------------------------------------ Clebsch-Gordan ---
 def test_complex_cg_matches_sympy():
     from sympy.physics.quantum.cg import CG
