@@ -337,12 +337,32 @@ def run_native(args):
         e2e = {"value": job_throughput(E, world, e_ms), "unit": "edges/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
+    # gradient with respect to the edge vectors (harmonics backward: turns the backward's grad_y
+    # into forces on the edge vectors), outside the step, each launch after an L2 flush
+    gvec = torch.empty_like(vec)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sh_times = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e3b.lib.e3_spherical_harmonics_backward(ly, E, e3b._ptr(vec), 0, e3b._ptr(gy), 0, e3b._ptr(gvec),
+                                                e3b._stream())
+        b.record(stream)
+        if i >= args.warmup:
+            sh_times.append((a, b))
+    torch.cuda.synchronize()
+    e3b.device_status()
+    sh_ms = statistics.fmean(a.elapsed_time(b) for a, b in sh_times)
+    del flush
+
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
     fb, bb = algorithmic_bytes(N, E, mul, lx, ly, lo)
+    shb = E * (12 + 4 * (ly + 1) ** 2 + 12)
     peak, peak_kind = hbm_peak()
     fwd_gbs, bwd_gbs = fb / (fwd_ms * 1e-3) / 1e9, bb / (bwd_ms * 1e-3) / 1e9
     dom = "conv_backward" if bwd_ms >= fwd_ms else "conv_forward"
@@ -366,6 +386,10 @@ def run_native(args):
                 "algorithmic_bytes": fb},
         "bwd": {"ms": bwd_ms, "edges_per_s": E / (bwd_ms * 1e-3), "GBps": bwd_gbs, "frac_of_hbm": bwd_gbs / peak,
                 "algorithmic_bytes": bb},
+        "sh_bwd": {"ms": sh_ms, "edges_per_s": E / (sh_ms * 1e-3), "GBps": shb / (sh_ms * 1e-3) / 1e9,
+                   "frac_of_hbm": shb / (sh_ms * 1e-3) / 1e9 / peak, "algorithmic_bytes": shb,
+                   "note": "grad wrt edge vectors from grad_y (e3_spherical_harmonics_backward), outside the step, "
+                           "L2 flushed before each launch"},
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
                      "frac": dom_gbs / peak, "peak_kind": peak_kind,
                      "traffic": traffic_for(dom, args.workload), "algorithmic_bytes": dom_bytes},

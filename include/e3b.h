@@ -172,6 +172,19 @@ E3_API e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* x, c
 E3_API e3_status e3_spherical_harmonics(int32_t lmax, int64_t n, const void* vec, e3_sh_norm sh_norm,
                                  e3_dtype dtype, void* out, void* stream);
 
+/* Gradient of the harmonics with respect to the vectors [SH]: for Y = the output of
+ * e3_spherical_harmonics(lmax, n, vec, sh_norm),
+ *   grad_vec[i] = sum_m grad_y[i, m] dY_m(vec_i)/dvec_i,
+ * the chain rule that turns a gradient with respect to the harmonics (e3_conv_backward's grad_y)
+ * into one with respect to edge vectors, hence positions: forces that conserve energy are the
+ * negative gradient of the energy with respect to positions (e3nn course, "Curriculum at a
+ * glance", lesson 07a).  Y depends on the direction only,
+ * so grad_vec is orthogonal to vec and scales as 1/|vec|.  vec [n, 3], grad_y [n, (lmax+1)^2],
+ * grad_vec [n, 3] (overwritten), element-aligned, of `dtype`; a zero vector gets a zero gradient.
+ * lmax <= 3.  n == 0 is a no-op. */
+E3_API e3_status e3_spherical_harmonics_backward(int32_t lmax, int64_t n, const void* vec, e3_sh_norm sh_norm,
+                                          const void* grad_y, e3_dtype dtype, void* grad_vec, void* stream);
+
 /* ------------------------------------------------------------------ CSR segmentation --- */
 
 /* Bytes of device workspace that e3_csr_build needs for N nodes and E edges. */

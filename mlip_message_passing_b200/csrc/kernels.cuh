@@ -231,16 +231,12 @@ __device__ __forceinline__ void load_w(T (&wr)[K][GR::NP], const T* __restrict__
 }
 
 // ------------------------------------------------------------ spherical harmonics ---
-// Real harmonics, component normalisation (sum_m Y_lm^2 = 2l+1 on the unit sphere), m = -l..l,
-// z the pole, no Condon-Shortley phase (e3nn course, lesson 02b).  Polynomials in the unit
-// vector (x, y, z); r = 0 gives Y^0 = 1 and zero for l > 0.
+// Component-normalised harmonics of a unit vector (x, y, z) as polynomials, Y[0] = 1.  T may be
+// a forward-mode dual number: the harmonics backward differentiates this routine.
 template <int LY, typename T>
-__device__ __forceinline__ void sh_eval(T vx, T vy, T vz, int norm, T (&Y)[(LY + 1) * (LY + 1)]) {
+__device__ __forceinline__ void sh_poly(T x, T y, T z, T (&Y)[(LY + 1) * (LY + 1)]) {
   Y[0] = T(1);
   if constexpr (LY >= 1) {
-    const T r2 = vx * vx + vy * vy + vz * vz;
-    const T inv = r2 > T(0) ? rsqrt_t(r2) : T(0);
-    const T x = vx * inv, y = vy * inv, z = vz * inv;
     const T s3 = T(1.7320508075688772935);
     Y[1] = s3 * y;
     Y[2] = s3 * z;
@@ -268,16 +264,37 @@ __device__ __forceinline__ void sh_eval(T vx, T vy, T vz, int norm, T (&Y)[(LY +
         Y[15] = c70 * x * (x2 - T(3) * y2);
       }
     }
-    // zero vector: every l > 0 component is already 0 through inv = 0
   }
-  if (norm == E3_SH_INTEGRAL) {
-    const T c = T(0.28209479177387814347);  // 1/sqrt(4 pi)
+}
+
+// Factor of degree l that turns component-normalised harmonics into normalisation `norm`:
+// integral 1/sqrt(4 pi) for every degree, norm 1/sqrt(2l+1) for l > 0.
+template <typename T>
+__device__ __forceinline__ T sh_norm_factor(int norm, int l) {
+  if (norm == E3_SH_INTEGRAL) return T(0.28209479177387814347);
+  if (norm == E3_SH_NORM && l > 0) return rsqrt_t(T(2 * l + 1));
+  return T(1);
+}
+
+// Real harmonics, component normalisation (sum_m Y_lm^2 = 2l+1 on the unit sphere), m = -l..l,
+// z the pole, no Condon-Shortley phase (e3nn course, lesson 02b), of the direction of (vx, vy,
+// vz), scaled to normalisation `norm`.  r = 0 gives Y^0 = 1 (scaled) and zero for l > 0: every
+// l > 0 polynomial vanishes at the origin.
+template <int LY, typename T>
+__device__ __forceinline__ void sh_eval(T vx, T vy, T vz, int norm, T (&Y)[(LY + 1) * (LY + 1)]) {
+  T x = T(0), y = T(0), z = T(0);
+  if constexpr (LY >= 1) {
+    const T r2 = vx * vx + vy * vy + vz * vz;
+    const T inv = r2 > T(0) ? rsqrt_t(r2) : T(0);
+    x = vx * inv;
+    y = vy * inv;
+    z = vz * inv;
+  }
+  sh_poly<LY, T>(x, y, z, Y);
+  if (norm != E3_SH_COMPONENT) {
 #pragma unroll
-    for (int i = 0; i < (LY + 1) * (LY + 1); ++i) Y[i] *= c;
-  } else if (norm == E3_SH_NORM) {
-#pragma unroll
-    for (int l = 1; l <= LY; ++l) {
-      const T c = rsqrt_t(T(2 * l + 1));
+    for (int l = 0; l <= LY; ++l) {
+      const T c = sh_norm_factor<T>(norm, l);
 #pragma unroll
       for (int m = 0; m < 2 * l + 1; ++m) Y[l * l + m] *= c;
     }

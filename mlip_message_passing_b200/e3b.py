@@ -26,7 +26,7 @@ SYMBOLS = [
     "e3_device_status", "e3_cg_dense", "e3_supported", "e3_tp_forward", "e3_tp_backward",
     "e3_spherical_harmonics", "e3_csr_workspace_size", "e3_csr_build", "e3_gather_rows",
     "e3_conv_forward", "e3_conv_backward", "e3_last_error", "e3_csr_build_static",
-    "e3_backward_workspace_size",
+    "e3_backward_workspace_size", "e3_spherical_harmonics_backward",
 ]
 
 
@@ -62,6 +62,7 @@ def _load():
         "e3_tp_backward": [VP, I64, VP, VP, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP],
         "e3_backward_workspace_size": [I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_spherical_harmonics": [I32, I64, VP, ctypes.c_int, ctypes.c_int, VP, VP],
+        "e3_spherical_harmonics_backward": [I32, I64, VP, ctypes.c_int, VP, ctypes.c_int, VP, VP],
         "e3_csr_workspace_size": [I64, I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_csr_build": [I64, I64, VP, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP],
         "e3_csr_build_static": [I64, I64, VP, VP, VP, VP, VP, VP, VP],
@@ -247,6 +248,39 @@ def spherical_harmonics(lmax, vec, sh_norm="component", out=None):
     return out
 
 
+def spherical_harmonics_backward(lmax, vec, grad_y, sh_norm="component", out=None):
+    """[n, 3] gradient of sum(grad_y * Y(vec)) with respect to vec (e3_spherical_harmonics_backward)."""
+    if vec.dtype not in _DTYPES:
+        raise ValueError("vec must be float32 or float64")
+    n = vec.shape[0]
+    _need(vec, "vec", vec.dtype, (n, 3), vec.device)
+    _need(grad_y, "grad_y", vec.dtype, (n, (lmax + 1) ** 2), vec.device)
+    if out is None:
+        out = torch.empty((n, 3), dtype=vec.dtype, device=vec.device)
+    _need(out, "out", vec.dtype, (n, 3), vec.device)
+    _check(lib.e3_spherical_harmonics_backward(lmax, n, _ptr(vec), _SH_NORMS[sh_norm], _ptr(grad_y),
+                                               _DTYPES[vec.dtype], _ptr(out), _stream()))
+    return out
+
+
+class _ShFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, vec, lmax, sh_norm):
+        ctx.lmax, ctx.sh_norm = lmax, sh_norm
+        ctx.save_for_backward(vec)
+        return spherical_harmonics(lmax, vec, sh_norm)
+
+    @staticmethod
+    def backward(ctx, g):
+        (vec,) = ctx.saved_tensors
+        return spherical_harmonics_backward(ctx.lmax, vec, g.contiguous(), ctx.sh_norm), None, None
+
+
+def sh(lmax, vec, sh_norm="component"):
+    """Differentiable real harmonics of vec [n, 3]."""
+    return _ShFn.apply(vec, lmax, sh_norm)
+
+
 def csr_build(n_nodes, src, dst):
     """(perm_dst, row_ptr_dst, perm_src, row_ptr_src) of an int32 edge list (e3_csr_build)."""
     E = src.shape[0]
@@ -362,3 +396,28 @@ class _ConvFn(torch.autograd.Function):
 def conv(plan, graph, x, y, w, out_scale=1.0):
     """Differentiable convolution with respect to x, y (harmonics) and w."""
     return _ConvFn.apply(x, y, w, plan, graph, out_scale)
+
+
+class _ConvVecFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, vec, w, plan, graph, out_scale, sh_norm):
+        ctx.plan, ctx.graph, ctx.out_scale, ctx.sh_norm = plan, graph, out_scale, sh_norm
+        ctx.save_for_backward(x, vec, w)
+        return conv_forward(plan, graph, x, w, edge_vec=vec, sh_norm=sh_norm, out_scale=out_scale)
+
+    @staticmethod
+    def backward(ctx, g):
+        x, vec, w = ctx.saved_tensors
+        need_vec = ctx.needs_input_grad[1]
+        gx, gy, gw = conv_backward(ctx.plan, ctx.graph, x, w, g.contiguous(), edge_vec=vec, sh_norm=ctx.sh_norm,
+                                   out_scale=ctx.out_scale, need_x=ctx.needs_input_grad[0], need_y=need_vec,
+                                   need_w=ctx.needs_input_grad[2])
+        lmax = int(ctx.plan.dim_in2 ** 0.5 + 0.5) - 1  # harmonics irreps 1x0e+1x1o+... of dim (lmax+1)^2
+        gvec = spherical_harmonics_backward(lmax, vec, gy, ctx.sh_norm) if need_vec else None
+        return gx, gvec, gw, None, None, None, None
+
+
+def conv_vec(plan, graph, x, edge_vec, w, out_scale=1.0, sh_norm="component"):
+    """Differentiable convolution with harmonics computed in the kernels from edge vectors
+    (receiver order): gradients with respect to x, edge_vec (through the harmonics) and w."""
+    return _ConvVecFn.apply(x, edge_vec, w, plan, graph, out_scale, sh_norm)

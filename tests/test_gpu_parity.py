@@ -70,6 +70,34 @@ def test_spherical_harmonics(e3b, dtype, norm):
     assert rel_err(got, ref) < (2e-6 if dtype == torch.float32 else 1e-14)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+@pytest.mark.parametrize("norm", ["component", "integral", "norm"])
+@pytest.mark.parametrize("lmax", [0, 1, 2, 3])
+def test_spherical_harmonics_backward(e3b, dtype, norm, lmax):
+    """grad_vec = sum_m grad_y[m] dY_m/dvec against the oracle's analytic Jacobian."""
+    rng = np.random.default_rng(6 + lmax)
+    n, ny = 3000, (lmax + 1) ** 2
+    v = (rng.standard_normal((n, 3)) * rng.uniform(0.3, 4.0, (n, 1))).astype(NP[dtype])
+    v[5] = 0.0
+    gy = rng.standard_normal((n, ny)).astype(NP[dtype])
+    got = h(e3b.spherical_harmonics_backward(lmax, t(v), t(gy), sh_norm=norm))
+    deg = np.concatenate([[l] * (2 * l + 1) for l in range(lmax + 1)])
+    if norm == "integral":
+        scale = np.full(ny, 1 / math.sqrt(4 * math.pi))
+    elif norm == "norm":
+        scale = 1 / np.sqrt(2 * deg + 1)
+    else:
+        scale = np.ones(ny)
+    ref = oracle.sh_backward(lmax, v.astype(np.float64), gy.astype(np.float64) * scale)
+    assert np.all(got[5] == 0)
+    if lmax == 0:
+        assert np.all(got == 0)
+    else:
+        assert rel_err(got, ref) <= TOL[dtype]
+        # the gradient is orthogonal to the vector (harmonics depend on the direction only)
+        assert np.max(np.abs(np.sum(got * v, axis=1))) <= (1e-4 if dtype == torch.float32 else 1e-11)
+
+
 # ------------------------------------------------------------- tensor product ---
 @pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
 def test_tp_small_forward_backward(e3b, dtype):
@@ -396,6 +424,41 @@ def test_conv_backward_finite_differences_subgraph(e3b):
     assert rel_err(h(gx), rx) <= 1e-12
     assert rel_err(h(gy), ry[perm]) <= 1e-12
     assert rel_err(h(gw), rw[perm]) <= 1e-12
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+def test_conv_vec_gradients(e3b, dtype):
+    """Autograd of the convolution with in-kernel harmonics: gradients with respect to x, the
+    edge vectors (through the harmonics: forces) and w against the oracle, and the edge-vector
+    gradient against central differences of the kernel forward (float64)."""
+    n, mul, lx, ly, lo = 400, 64, 2, 3, 2
+    g, graph, w = conv_setup(e3b, n, mul, lx, ly, lo, 23, dtype)
+    p, q = gplan(e3b, mul, lx, ly, lo, dtype), oplan(mul, lx, ly, lo)
+    s = 1 / math.sqrt(52)
+    vec = graph.to_receiver_order(t(g["vec"])).requires_grad_()
+    x = t(g["x"]).requires_grad_()
+    wr = graph.to_receiver_order(w).requires_grad_()
+    out = e3b.conv_vec(p, graph, x, vec, wr, s)
+    go = np.random.default_rng(8).standard_normal((n, p.dim_out)).astype(NP[dtype])
+    out.backward(t(go))
+    Y = oracle.real_sh_all(ly, g["vec"].astype(np.float64))
+    rx, ry, rw = oracle.conv_backward(q, n, g["src"], g["dst"], g["x"], Y, g["w"], go, s)
+    rvec = oracle.sh_backward(ly, g["vec"].astype(np.float64), ry)
+    perm = graph.perm_dst.cpu().numpy()
+    assert rel_err(h(x.grad), rx) <= TOL[dtype]
+    assert rel_err(h(wr.grad), rw[perm]) <= TOL[dtype]
+    assert rel_err(h(vec.grad), rvec[perm]) <= TOL[dtype]
+    if dtype == torch.float64:
+        d = torch.as_tensor(np.random.default_rng(9).standard_normal(tuple(vec.shape)), device=DEV)
+        hs = 1e-6
+        xd, wd, gt = x.detach(), wr.detach(), t(go)
+
+        def L(vv):
+            return float((gt * e3b.conv_forward(p, graph, xd, wd, edge_vec=vv, out_scale=s)).sum())
+
+        fd = (L(vec.detach() + hs * d) - L(vec.detach() - hs * d)) / (2 * hs)
+        an = float((vec.grad * d).sum())
+        assert abs(fd - an) <= 1e-7 * max(1.0, abs(an))
 
 
 def test_autograd_wrapper(e3b):
