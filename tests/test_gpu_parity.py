@@ -247,6 +247,35 @@ def test_conv_small_multiplicity_and_degrees(e3b):
         assert rel_err(h(res[2]), ref[2][perm]) <= 1e-5
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+def test_conv_l3_mul128_sampled(e3b, dtype):
+    """The l <= 3 path set (34 paths) at multiplicity 128 -- the large-convolution kernels -- on a
+    400-node box: forward on 40 sampled receivers (all their in-edges), backward on 40 sampled
+    senders (all their out-edges: their grad_x and those edges' grad_y, grad_w are exact)."""
+    n, mul, lx, ly, lo = 400, 128, 3, 3, 3
+    g, graph, w = conv_setup(e3b, n, mul, lx, ly, lo, 31, dtype)
+    p, q = gplan(e3b, mul, lx, ly, lo, dtype), oplan(mul, lx, ly, lo)
+    s = 1 / math.sqrt(52)
+    vec, wr = graph.to_receiver_order(t(g["vec"])), graph.to_receiver_order(w)
+    out = e3b.conv_forward(p, graph, t(g["x"]), wr, edge_vec=vec, out_scale=s)
+    go = W.grad_out(n, q.irreps_out.dim, 7, dtype=NP[dtype])
+    gx, gy, gw = e3b.conv_backward(p, graph, t(g["x"]), wr, t(go), edge_vec=vec, out_scale=s)
+    rng = np.random.default_rng(12)
+    recv = np.sort(rng.choice(n, 40, replace=False))
+    sel = np.flatnonzero(np.isin(g["dst"], recv))
+    Y = oracle.real_sh_all(ly, g["vec"][sel].astype(np.float64))
+    ref = oracle.conv_forward(q, n, g["src"][sel], g["dst"][sel], g["x"], Y, g["w"][sel], s)
+    assert rel_err(h(out)[recv], ref[recv]) <= TOL[dtype]
+    send = np.sort(rng.choice(n, 40, replace=False))
+    sel = np.flatnonzero(np.isin(g["src"], send))
+    Y = oracle.real_sh_all(ly, g["vec"][sel].astype(np.float64))
+    rx, ry, rw = oracle.conv_backward(q, n, g["src"][sel], g["dst"][sel], g["x"], Y, g["w"][sel], go, s)
+    pos = np.argsort(graph.perm_dst.cpu().numpy())  # original edge id -> receiver-order position
+    assert rel_err(h(gx)[send], rx[send]) <= TOL[dtype]
+    assert rel_err(h(gy)[pos[sel]], ry) <= TOL[dtype]
+    assert rel_err(h(gw)[pos[sel]], rw) <= TOL[dtype]
+
+
 def test_conv_edge_cases(e3b):
     p = gplan(e3b, 8, 1, 2, 2, torch.float32)
     q = oplan(8, 1, 2, 2)
