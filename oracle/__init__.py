@@ -23,10 +23,11 @@ from .sh import real_sh, real_sh_all, real_sh_grad, real_sh_all_grad, sh_backwar
 from .cg import complex_cg, real_cg, real_basis_change
 from .tp import Instruction, TPPlan, make_plan, tp_forward, tp_backward
 from .conv import csr_build, conv_forward, conv_backward
+from .reorder import morton_codes, morton_order, invert_permutation
 
 __all__ = [
     "Irreps", "parse_irreps", "real_sh", "real_sh_all", "real_sh_grad", "real_sh_all_grad", "sh_backward",
     "complex_cg", "real_cg",
     "real_basis_change", "Instruction", "TPPlan", "make_plan", "tp_forward", "tp_backward",
-    "csr_build", "conv_forward", "conv_backward",
+    "csr_build", "conv_forward", "conv_backward", "morton_codes", "morton_order", "invert_permutation",
 ]

@@ -182,3 +182,18 @@ def test_sh_grad_y_derivative_missing_i(monkeypatch):
 def test_sh_grad_wrong_legendre_derivative(monkeypatch):
     _patch_sh_grad(monkeypatch, "dp1 = pl.deriv(am + 1)", "dp1 = pl.deriv(am)")
     assert _caught(SH_GRAD_PINS)
+
+
+def test_morton_axes_swapped(monkeypatch):
+    import inspect
+    import textwrap
+    import oracle.reorder as ore
+    src = textwrap.dedent(inspect.getsource(ore.morton_codes))
+    ns = dict(vars(ore))
+    exec(compile(src.replace("<< (3 * b + k)", "<< (3 * b + 2 - k)"), "mutant", "exec"), ns)
+    monkeypatch.setattr(ore, "morton_codes", ns["morton_codes"])
+    monkeypatch.setattr(oracle, "morton_codes", ns["morton_codes"])
+    bad_order = lambda pos, lo, ext: np.argsort(ns["morton_codes"](pos, lo, ext), kind="stable").astype(np.int32)
+    monkeypatch.setattr(ore, "morton_order", bad_order)
+    monkeypatch.setattr(oracle, "morton_order", bad_order)
+    assert _caught([pins.test_morton_order_equals_octree_order, pins.test_morton_codes_known_cells_and_clamping])

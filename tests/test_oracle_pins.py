@@ -457,3 +457,45 @@ def test_conv_backward_euler_and_fd():
         f = lambda a: float((g * oracle.conv_forward(plan, n, src, dst, a[0], a[1], a[2], s)).sum())
         fd = (f(pl) - f(mi)) / (2 * h)
         assert abs(fd - float((d * dirn).sum())) < 1e-9 * max(1.0, abs(fd))
+
+
+# ------------------------------------------------------------------- reordering ---
+def _octree_less(qa, qb):
+    """Z-order by recursive octant subdivision: at the coarsest level where the cells differ,
+    the octant index x + 2 y + 4 z decides (an independent formulation of the curve)."""
+    for b in range(oracle.reorder.BITS - 1, -1, -1):
+        oa = sum(((int(qa[k]) >> b) & 1) << k for k in range(3))
+        ob = sum(((int(qb[k]) >> b) & 1) << k for k in range(3))
+        if oa != ob:
+            return -1 if oa < ob else 1
+    return 0
+
+
+def test_morton_order_equals_octree_order():
+    import functools
+    import oracle.reorder  # noqa: F401
+    rng = np.random.default_rng(60)
+    pos = rng.uniform(-2.0, 5.0, (300, 3))
+    lo, ext = (-2.0, -2.0, -2.0), (7.0, 7.0, 7.0)
+    q = oracle.reorder.quantise(pos, lo, ext)
+    ref = sorted(range(len(pos)), key=functools.cmp_to_key(lambda a, b: _octree_less(q[a], q[b]) or (a > b) - (a < b)))
+    assert np.array_equal(oracle.morton_order(pos, lo, ext), np.array(ref, dtype=np.int32))
+
+
+def test_morton_codes_known_cells_and_clamping():
+    import oracle.reorder  # noqa: F401
+    lo, ext = (0.0, 0.0, 0.0), (1024.0, 1024.0, 1024.0)  # one unit per cell
+    pts = np.array([[0.5, 0.5, 0.5], [1.5, 0.5, 0.5], [0.5, 1.5, 0.5], [0.5, 0.5, 1.5], [2.5, 0.5, 0.5],
+                    [1023.9, 1023.9, 1023.9], [-5.0, 2000.0, 0.0]])
+    codes = oracle.morton_codes(pts, lo, ext)
+    # x -> bit 0, y -> bit 1, z -> bit 2, x = 2 -> bit 3; the last cell has all 30 bits set;
+    # out-of-box coordinates clamp to the first / last cell
+    assert list(codes[:5]) == [0, 1, 2, 4, 8]
+    assert codes[5] == (1 << 30) - 1
+    assert codes[6] == oracle.morton_codes(np.array([[0.0, 1023.5, 0.0]]), lo, ext)[0]
+
+
+def test_invert_permutation():
+    perm = np.random.default_rng(61).permutation(50).astype(np.int32)
+    inv = oracle.invert_permutation(perm)
+    assert np.array_equal(perm[inv], np.arange(50)) and np.array_equal(inv[perm], np.arange(50))
