@@ -228,6 +228,33 @@ E3_API e3_status e3_csr_build_static(int64_t N, int64_t E, const int32_t* src, c
 E3_API e3_status e3_gather_rows(int64_t n_rows, int64_t n_in_rows, int64_t row_bytes,
                          const int32_t* perm, const void* in, void* out, void* stream);
 
+/* ------------------------------------------------------------------- node reordering --- */
+
+/* Sparse, irregular gathers bound message passing (Sobek: Streaming Equivariant Tensor Product
+ * Convolutions, abstract); numbering nodes along a space-filling curve makes the senders of
+ * neighbouring receivers neighbours in memory, so gathered rows are reused from L2.  The curve is
+ * the Morton (Z-order) curve: each coordinate of pos[i] is quantised to 10 bits inside the box
+ * [lo, lo + extent) (scale 1024 / extent in double, floor, clamped to [0, 1023]), bit b of axis k
+ * goes to bit 3b + k of a 30-bit code, and perm[i] is the id of the node with the i-th smallest
+ * code (stable: equal codes keep ascending ids; integer-only after the quantisation, bit-exact).
+ * To renumber a graph: inv = inverse of perm; src, dst <- inv[src], inv[dst] (e3_remap_ids);
+ * node rows <- rows[perm] (e3_gather_rows); results come back with rows[inv].
+ *   pos [N, 3] of `dtype`; lo, extent: 3 host doubles (extent > 0); perm [N] int32 (device);
+ *   workspace: device buffer of e3_morton_workspace_size(N) bytes, 256-byte aligned. */
+E3_API e3_status e3_morton_workspace_size(int64_t N, size_t* bytes);
+E3_API e3_status e3_morton_order(int64_t N, const void* pos, e3_dtype dtype, const double* lo,
+                          const double* extent, int32_t* perm, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* inv[perm[i]] = i for a permutation perm of 0..N-1 (device int32 arrays).  Entries out of range
+ * record E3_ERR_INDEX in the device status word and are skipped. */
+E3_API e3_status e3_invert_permutation(int64_t N, const int32_t* perm, int32_t* inv, void* stream);
+
+/* out[i] = map[ids[i]] for i < n, map of N entries (device int32 arrays; out may alias ids).  An id
+ * out of [0, N) records E3_ERR_INDEX and gives -1. */
+E3_API e3_status e3_remap_ids(int64_t n, const int32_t* ids, int64_t N, const int32_t* map, int32_t* out,
+                       void* stream);
+
 /* ----------------------------------------------------------------------- convolution --- */
 
 /* out[n] = out_scale * sum_{e : dst_e = n} TP(x[src_e], Y_e, w_e)   [CONV][TP]

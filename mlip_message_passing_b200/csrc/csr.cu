@@ -14,6 +14,8 @@
 // shared memory only; ranks never depend on thread scheduling, so the output is unique.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -150,6 +152,54 @@ __global__ void gather_rows_kernel(int64_t n_rows, int64_t n_in_rows, int64_t ro
       reinterpret_cast<uint4*>(out)[r * per_row + c] = __ldg(reinterpret_cast<const uint4*>(in) + int64_t(s) * per_row + c);
     else
       out[r * row_words + c] = __ldg(in + int64_t(s) * row_words + c);
+  }
+}
+
+// ------------------------------------------------------------------- node reordering ---
+// Morton (Z-order) code of a position: each coordinate quantised to 10 bits inside the box
+// (scale = 1024 / extent in double, floor, clamp), bit b of axis k goes to bit 3 b + k.
+constexpr int MORTON_BITS = 10;
+template <typename T>
+__global__ void morton_code_kernel(int64_t n, const T* __restrict__ pos, double lo0, double lo1, double lo2,
+                                   double s0, double s1, double s2, int32_t* __restrict__ codes) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const double lo[3] = {lo0, lo1, lo2}, sc[3] = {s0, s1, s2};
+    uint32_t code = 0;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const double f = floor((double(pos[3 * i + k]) - lo[k]) * sc[k]);
+      const uint32_t q = f < 0.0 ? 0u : (f > double((1 << MORTON_BITS) - 1) ? uint32_t((1 << MORTON_BITS) - 1) : uint32_t(f));
+#pragma unroll
+      for (int b = 0; b < MORTON_BITS; ++b) code |= ((q >> b) & 1u) << (3 * b + k);
+    }
+    codes[i] = int32_t(code);
+  }
+}
+
+// inv[perm[i]] = i (entries out of range are reported and skipped)
+__global__ void invert_perm_kernel(int64_t n, const int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                   int* status) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int32_t p = perm[i];
+    if (p < 0 || p >= n) {
+      atomicCAS(status, 0, int(E3_ERR_INDEX));
+      continue;
+    }
+    inv[p] = int32_t(i);
+  }
+}
+
+// out[i] = map[ids[i]] (ids out of range are reported and give -1)
+__global__ void remap_ids_kernel(int64_t n, const int32_t* __restrict__ ids, int64_t N, const int32_t* __restrict__ map,
+                                 int32_t* __restrict__ out, int* status) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int32_t id = ids[i];
+    if (id < 0 || id >= N) {
+      atomicCAS(status, 0, int(E3_ERR_INDEX));
+      out[i] = -1;
+      continue;
+    }
+    out[i] = __ldg(map + id);
   }
 }
 
@@ -328,4 +378,85 @@ extern "C" e3_status e3_csr_build_static(int64_t N, int64_t E, const int32_t* sr
   if (st != E3_OK) return st;
   return e3_csr_build(N, E, src, dst, perm_dst, row_ptr_dst, perm_src, row_ptr_src, ws, kStaticScratchBytes,
                       stream);
+}
+
+// ------------------------------------------------------------------- node reordering ---
+static size_t morton_ws_bytes(int64_t N) { return align256(sizeof(int32_t) * size_t(N > 0 ? N : 1)) + csr_ws_bytes(N); }
+
+extern "C" e3_status e3_morton_workspace_size(int64_t N, size_t* bytes) {
+  clear_error();
+  if (bytes == nullptr) return fail(E3_ERR_INVALID_ARG, "bytes is NULL");
+  if (N < 0 || N >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N out of range");
+  *bytes = morton_ws_bytes(N);
+  return E3_OK;
+}
+
+extern "C" e3_status e3_morton_order(int64_t N, const void* pos, e3_dtype dtype, const double* lo, const double* extent,
+                                     int32_t* perm, void* workspace, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (N < 0 || N >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N out of range");
+  if (dtype != E3_F32 && dtype != E3_F64) return fail(E3_ERR_INVALID_ARG, "bad dtype");
+  if (lo == nullptr || extent == nullptr) return fail(E3_ERR_INVALID_ARG, "lo or extent is NULL");
+  for (int k = 0; k < 3; ++k)
+    if (!(extent[k] > 0.0) || !std::isfinite(extent[k]) || !std::isfinite(lo[k]))
+      return fail(E3_ERR_INVALID_ARG, "box extent must be positive and finite");
+  if (N == 0) return E3_OK;
+  if (pos == nullptr || perm == nullptr) return fail(E3_ERR_INVALID_ARG, "NULL pointer");
+  if (reinterpret_cast<uintptr_t>(pos) % (dtype == E3_F64 ? 8 : 4)) return fail(E3_ERR_INVALID_ARG, "pos not aligned");
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(E3_ERR_INVALID_ARG, "workspace is NULL or not 256-byte aligned");
+  if (ws_bytes < morton_ws_bytes(N)) return fail(E3_ERR_SHAPE, "workspace of %zu bytes, need %zu", ws_bytes, morton_ws_bytes(N));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* codes = reinterpret_cast<int32_t*>(ws);
+  char* sort_ws = ws + align256(sizeof(int32_t) * size_t(N));
+  const size_t eb = align256(sizeof(int32_t) * size_t(N));
+  int32_t* ka = reinterpret_cast<int32_t*>(sort_ws);
+  int32_t* va = reinterpret_cast<int32_t*>(sort_ws + eb);
+  int32_t* kb = reinterpret_cast<int32_t*>(sort_ws + 2 * eb);
+  int32_t* vb = reinterpret_cast<int32_t*>(sort_ws + 3 * eb);
+  int32_t* counts = reinterpret_cast<int32_t*>(sort_ws + 4 * eb);
+  const double scale[3] = {double(1 << MORTON_BITS) / extent[0], double(1 << MORTON_BITS) / extent[1],
+                           double(1 << MORTON_BITS) / extent[2]};
+  const int blocks = int(std::min<int64_t>((N + 255) / 256, 148 * 8));
+  if (dtype == E3_F32)
+    morton_code_kernel<float><<<blocks, 256, 0, s>>>(N, static_cast<const float*>(pos), lo[0], lo[1], lo[2], scale[0],
+                                                     scale[1], scale[2], codes);
+  else
+    morton_code_kernel<double><<<blocks, 256, 0, s>>>(N, static_cast<const double*>(pos), lo[0], lo[1], lo[2],
+                                                      scale[0], scale[1], scale[2], codes);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "morton code launch failed: %s", cudaGetErrorString(err));
+  return radix_sort(codes, nullptr, N, 3 * MORTON_BITS, perm, ka, va, kb, vb, counts, s);
+}
+
+extern "C" e3_status e3_invert_permutation(int64_t N, const int32_t* perm, int32_t* inv, void* stream) {
+  clear_error();
+  if (N < 0 || N >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N out of range");
+  if (N == 0) return E3_OK;
+  if (perm == nullptr || inv == nullptr) return fail(E3_ERR_INVALID_ARG, "NULL pointer");
+  int* status = nullptr;
+  e3_status st = device_status_ptr(&status);
+  if (st != E3_OK) return st;
+  const int blocks = int(std::min<int64_t>((N + 255) / 256, 148 * 8));
+  invert_perm_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(N, perm, inv, status);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "invert launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+extern "C" e3_status e3_remap_ids(int64_t n, const int32_t* ids, int64_t N, const int32_t* map, int32_t* out,
+                                  void* stream) {
+  clear_error();
+  if (n < 0 || N < 0 || n >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "n or N out of range");
+  if (n == 0) return E3_OK;
+  if (ids == nullptr || map == nullptr || out == nullptr) return fail(E3_ERR_INVALID_ARG, "NULL pointer");
+  int* status = nullptr;
+  e3_status st = device_status_ptr(&status);
+  if (st != E3_OK) return st;
+  const int blocks = int(std::min<int64_t>((n + 255) / 256, 148 * 8));
+  remap_ids_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(n, ids, N, map, out, status);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "remap launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
 }

@@ -26,7 +26,8 @@ SYMBOLS = [
     "e3_device_status", "e3_cg_dense", "e3_supported", "e3_tp_forward", "e3_tp_backward",
     "e3_spherical_harmonics", "e3_csr_workspace_size", "e3_csr_build", "e3_gather_rows",
     "e3_conv_forward", "e3_conv_backward", "e3_last_error", "e3_csr_build_static",
-    "e3_backward_workspace_size", "e3_spherical_harmonics_backward",
+    "e3_backward_workspace_size", "e3_spherical_harmonics_backward", "e3_morton_workspace_size",
+    "e3_morton_order", "e3_invert_permutation", "e3_remap_ids",
 ]
 
 
@@ -70,6 +71,11 @@ def _load():
         "e3_conv_forward": [VP, I64, I64, VP, VP, VP, VP, VP, ctypes.c_int, VP, D, VP, VP],
         "e3_conv_backward": [VP, I64, I64, VP, VP, VP, VP, VP, VP, VP, VP, ctypes.c_int, VP, VP, D, VP, VP, VP,
                              VP, ctypes.c_size_t, VP],
+        "e3_morton_workspace_size": [I64, ctypes.POINTER(ctypes.c_size_t)],
+        "e3_morton_order": [I64, VP, ctypes.c_int, ctypes.POINTER(D), ctypes.POINTER(D), VP, VP, ctypes.c_size_t,
+                            VP],
+        "e3_invert_permutation": [I64, VP, VP, VP],
+        "e3_remap_ids": [I64, VP, I64, VP, VP, VP],
         "e3_last_error": [],
     }
     for name, args in sig.items():
@@ -279,6 +285,48 @@ class _ShFn(torch.autograd.Function):
 def sh(lmax, vec, sh_norm="component"):
     """Differentiable real harmonics of vec [n, 3]."""
     return _ShFn.apply(vec, lmax, sh_norm)
+
+
+def morton_order(pos, lo, extent):
+    """int32 [N] node order along the Morton curve of pos [N, 3] inside the box [lo, lo + extent)
+    (e3_morton_order): perm[i] is the id of the i-th node on the curve."""
+    if pos.dtype not in _DTYPES:
+        raise ValueError("pos must be float32 or float64")
+    N = pos.shape[0]
+    _need(pos, "pos", pos.dtype, (N, 3), pos.device)
+    nbytes = ctypes.c_size_t()
+    _check(lib.e3_morton_workspace_size(N, ctypes.byref(nbytes)))
+    ws = torch.empty(nbytes.value, dtype=torch.uint8, device=pos.device)
+    perm = torch.empty(N, dtype=torch.int32, device=pos.device)
+    lo3, ext3 = (ctypes.c_double * 3)(*map(float, lo)), (ctypes.c_double * 3)(*map(float, extent))
+    _check(lib.e3_morton_order(N, _ptr(pos), _DTYPES[pos.dtype], lo3, ext3, _ptr(perm), _ptr(ws), ws.numel(),
+                               _stream()))
+    return perm
+
+
+def invert_permutation(perm):
+    """inv with inv[perm[i]] = i (e3_invert_permutation)."""
+    _need(perm, "perm", torch.int32, (perm.shape[0],), perm.device)
+    inv = torch.empty_like(perm)
+    _check(lib.e3_invert_permutation(perm.shape[0], _ptr(perm), _ptr(inv), _stream()))
+    return inv
+
+
+def remap_ids(ids, mapping):
+    """mapping[ids] for int32 tensors (e3_remap_ids)."""
+    _need(ids, "ids", torch.int32, (ids.shape[0],), ids.device)
+    _need(mapping, "mapping", torch.int32, (mapping.shape[0],), ids.device)
+    out = torch.empty_like(ids)
+    _check(lib.e3_remap_ids(ids.shape[0], _ptr(ids), mapping.shape[0], _ptr(mapping), _ptr(out), _stream()))
+    return out
+
+
+def reorder_graph(pos, lo, extent, src, dst):
+    """Morton renumbering of a graph: (perm, inv, src', dst') with src' = inv[src], dst' = inv[dst].
+    Node rows of the new numbering are rows[perm] (gather_rows); results map back with rows[inv]."""
+    perm = morton_order(pos, lo, extent)
+    inv = invert_permutation(perm)
+    return perm, inv, remap_ids(src, inv), remap_ids(dst, inv)
 
 
 def csr_build(n_nodes, src, dst):

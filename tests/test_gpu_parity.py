@@ -276,6 +276,54 @@ def test_conv_l3_mul128_sampled(e3b, dtype):
     assert rel_err(h(gw)[pos[sel]], rw) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+def test_morton_order_bit_exact(e3b, dtype):
+    """Morton order of positions against the oracle, bit for bit: several sort tiles and a ragged
+    tail, points outside the box (clamped), duplicated positions (ties keep ascending ids)."""
+    rng = np.random.default_rng(70)
+    pos = rng.uniform(-1.0, 11.0, (5003, 3)).astype(NP[dtype])
+    pos[100:140] = pos[7]
+    lo, ext = (0.0, 0.5, -0.25), (10.0, 9.0, 10.5)
+    perm = e3b.morton_order(t(pos), lo, ext)
+    ref = oracle.morton_order(pos.astype(np.float64), lo, ext)
+    assert np.array_equal(perm.cpu().numpy(), ref)
+    inv = e3b.invert_permutation(perm)
+    assert np.array_equal(inv.cpu().numpy(), oracle.invert_permutation(ref))
+    ids = t(rng.integers(0, 5003, 777).astype(np.int32))
+    assert np.array_equal(e3b.remap_ids(ids, inv).cpu().numpy(), oracle.invert_permutation(ref)[ids.cpu().numpy()])
+    e3b.device_status()
+    ids[5] = 5003  # out of range: reported, not dereferenced
+    e3b.remap_ids(ids, inv)
+    with pytest.raises(e3b.E3Error):
+        e3b.device_status()
+
+
+def test_conv_on_morton_renumbered_graph(e3b):
+    """Renumbering nodes along the Morton curve changes no result: the forward is bitwise the
+    permuted original (each receiver keeps its in-edge order); the backward agrees to rounding."""
+    n, mul, lx, ly, lo = 400, 64, 2, 3, 2
+    g, graph, w = conv_setup(e3b, n, mul, lx, ly, lo, 21, torch.float32)
+    p = gplan(e3b, mul, lx, ly, lo, torch.float32)
+    x, vec_e, src, dst = t(g["x"]), t(g["vec"]), t(g["src"]), t(g["dst"])
+    go = t(W.grad_out(n, p.dim_out, 5))
+    out0 = e3b.conv_forward(p, graph, x, graph.to_receiver_order(w), edge_vec=graph.to_receiver_order(vec_e),
+                            out_scale=0.2)
+    b0 = e3b.conv_backward(p, graph, x, graph.to_receiver_order(w), go, edge_vec=graph.to_receiver_order(vec_e),
+                           out_scale=0.2)
+    perm, inv, src2, dst2 = e3b.reorder_graph(t(g["pos"]), (0, 0, 0), (g["side"],) * 3, src, dst)
+    g2 = e3b.Graph(n, src2, dst2)
+    x2, go2 = e3b.gather_rows(perm, x), e3b.gather_rows(perm, go)
+    out2 = e3b.conv_forward(p, g2, x2, g2.to_receiver_order(w), edge_vec=g2.to_receiver_order(vec_e), out_scale=0.2)
+    assert torch.equal(e3b.gather_rows(inv, out2), out0)
+    gx2, gy2, gw2 = e3b.conv_backward(p, g2, x2, g2.to_receiver_order(w), go2, edge_vec=g2.to_receiver_order(vec_e),
+                                      out_scale=0.2)
+    assert rel_err(h(e3b.gather_rows(inv, gx2)), h(b0[0])) <= 1e-5
+    # per-edge gradients: map both back to the original edge order
+    o0, o2 = np.argsort(graph.perm_dst.cpu().numpy()), np.argsort(g2.perm_dst.cpu().numpy())
+    assert rel_err(h(gy2)[o2], h(b0[1])[o0]) <= 1e-5
+    assert rel_err(h(gw2)[o2], h(b0[2])[o0]) <= 1e-5
+
+
 def test_conv_edge_cases(e3b):
     p = gplan(e3b, 8, 1, 2, 2, torch.float32)
     q = oplan(8, 1, 2, 2)
