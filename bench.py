@@ -42,6 +42,7 @@ def parse():
                     help="renumber nodes along the Morton curve of their positions before timing")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-tp", action="store_true", help="skip the tensor-product (no graph) measurement")
     return ap.parse_args()
 
 
@@ -224,6 +225,65 @@ def run_reference(args):
     return 0
 
 
+def measure_tp(args, dev):
+    """Tensor product without a graph (per-sample x, harmonics and weights) on the batched
+    workload, forward and backward, CUDA events; inputs (several GB) are larger than L2."""
+    import torch
+    from mlip_message_passing_b200 import e3b, workloads as W
+
+    cfg = W.CONFIGS["tp_batched"]
+    B, mul, lx, ly, lo = cfg["B"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
+    plan = e3b.Plan(W.irreps_str(mul, lx), W.sh_irreps(ly), lmax_out=lo)
+    gen = torch.Generator(device=dev).manual_seed(cfg["seed"])
+    vec = torch.randn(B, 3, generator=gen, device=dev)
+    vec /= vec.norm(dim=1, keepdim=True)
+    y = e3b.spherical_harmonics(ly, vec)
+    x = torch.randn(B, plan.dim_in1, generator=gen, device=dev)
+    w = torch.randn(B, plan.weight_numel, generator=gen, device=dev)
+    go = torch.randn(B, plan.dim_out, generator=gen, device=dev)
+    out = torch.empty(B, plan.dim_out, device=dev)
+    gx, gy, gw = torch.empty_like(x), torch.empty_like(y), torch.empty_like(w)
+    ws = e3b.backward_workspace(B, dev)
+    stream = torch.cuda.current_stream()
+    P = e3b._ptr
+
+    def fwd():
+        e3b.lib.e3_tp_forward(plan.handle, B, P(x), P(y), P(w), P(out), e3b._stream())
+
+    def bwd():
+        e3b.lib.e3_tp_backward(plan.handle, B, P(x), P(y), P(w), P(go), P(gx), P(gy), P(gw), P(ws), ws.numel(),
+                               e3b._stream())
+
+    res = {}
+    for name, fn in (("fwd", fwd), ("bwd", bwd)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev = []
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        e3b.device_status()
+        res[name] = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    dx, dy, dw, do = plan.dim_in1, plan.dim_in2, plan.weight_numel, plan.dim_out
+    nbytes = {"fwd": 4 * B * (dx + dy + dw + do), "bwd": 4 * B * (2 * dx + 2 * dy + 2 * dw + do)}
+    peak, _ = hbm_peak()
+    line = {"workload": f"tp_batched: B={B}, {W.irreps_str(mul, lx)} x {W.sh_irreps(ly)} -> l<={lo}, "
+                        f"{plan.n_paths} paths, fp32"}
+    for name in ("fwd", "bwd"):
+        ms = res[name]
+        gbs = nbytes[name] / (ms * 1e-3) / 1e9
+        line[name] = {"ms": ms, "samples_per_s": B / (ms * 1e-3), "GBps": gbs, "frac_of_hbm": gbs / peak,
+                      "algorithmic_bytes": nbytes[name]}
+    del x, y, w, go, out, gx, gy, gw, ws
+    torch.cuda.empty_cache()
+    return line
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -368,6 +428,7 @@ def run_native(args):
     if rank != 0:
         return 0
 
+    tp = None if args.no_tp else measure_tp(args, dev)
     fb, bb = algorithmic_bytes(N, E, mul, lx, ly, lo)
     shb = E * (12 + 4 * (ly + 1) ** 2 + 12)
     peak, peak_kind = hbm_peak()
@@ -399,6 +460,7 @@ def run_native(args):
                    "frac_of_hbm": shb / (sh_ms * 1e-3) / 1e9 / peak, "algorithmic_bytes": shb,
                    "note": "grad wrt edge vectors from grad_y (e3_spherical_harmonics_backward), outside the step, "
                            "L2 flushed before each launch"},
+        "tp": tp,
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
                      "frac": dom_gbs / peak, "peak_kind": peak_kind,
                      "traffic": traffic_for(dom, args.workload), "algorithmic_bytes": dom_bytes},
