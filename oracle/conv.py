@@ -9,6 +9,10 @@ receiver-ordered CSR aggregation that the GPU path uses.  Here the sum is the li
 definition: messages are accumulated with ``np.add.at`` in the input edge order.
 
 Edge i -> j has sender ``src = i`` and receiver ``dst = j`` (lesson 05a: r_ij = r_j - r_i).
+
+Padding edges: batches of fixed shape pad the edge list (the E3J summary, sections 3.1.2 and 3.2,
+measures the cost of padding edges that point to a shared padding node).  Here an edge whose sender or
+receiver is -1 is padding: it belongs to no node, contributes nothing and gets zero gradients.
 """
 
 import numpy as np
@@ -27,10 +31,15 @@ def csr_build(n_nodes, src, dst):
     """
     src = np.asarray(src, dtype=np.int64)
     dst = np.asarray(dst, dtype=np.int64)
-    perm_dst = np.argsort(dst, kind="stable")
-    row_ptr_dst = np.concatenate([[0], np.cumsum(np.bincount(dst, minlength=n_nodes))])
-    perm_src = np.argsort(src[perm_dst], kind="stable")
-    row_ptr_src = np.concatenate([[0], np.cumsum(np.bincount(src, minlength=n_nodes))])
+    valid = (src != -1) & (dst != -1)
+    ids = np.flatnonzero(valid)
+    pad = np.flatnonzero(~valid)
+    # valid edges stably by receiver, then the padding edges in input order (outside every row)
+    perm_dst = np.concatenate([ids[np.argsort(dst[ids], kind="stable")], pad])
+    row_ptr_dst = np.concatenate([[0], np.cumsum(np.bincount(dst[ids], minlength=n_nodes))])
+    nv = len(ids)
+    perm_src = np.concatenate([np.argsort(src[perm_dst[:nv]], kind="stable"), np.arange(nv, len(src))])
+    row_ptr_src = np.concatenate([[0], np.cumsum(np.bincount(src[ids], minlength=n_nodes))])
     return (perm_dst.astype(np.int32), row_ptr_dst.astype(np.int32),
             perm_src.astype(np.int32), row_ptr_src.astype(np.int32))
 
@@ -40,8 +49,10 @@ def conv_forward(plan, n_nodes, src, dst, x, y, w, scale, chunk=4096):
     x = np.asarray(x, dtype=np.float64)
     out = np.zeros((n_nodes, plan.irreps_out.dim))
     n_edges = len(src)
+    src, dst = np.asarray(src), np.asarray(dst)
     for s in range(0, n_edges, chunk):
-        e = slice(s, min(s + chunk, n_edges))
+        e = np.arange(s, min(s + chunk, n_edges))
+        e = e[(src[e] != -1) & (dst[e] != -1)]  # padding edges contribute nothing
         msg = tp_forward(plan, x[src[e]], y[e], w[e])
         np.add.at(out, dst[e], msg)
     return scale * out
@@ -55,8 +66,10 @@ def conv_backward(plan, n_nodes, src, dst, x, y, w, grad_out, scale, chunk=4096)
     dx = np.zeros_like(x)
     dy = np.zeros((n_edges, plan.irreps_in2.dim))
     dw = np.zeros((n_edges, plan.weight_numel))
+    src, dst = np.asarray(src), np.asarray(dst)
     for s in range(0, n_edges, chunk):
-        e = slice(s, min(s + chunk, n_edges))
+        e = np.arange(s, min(s + chunk, n_edges))
+        e = e[(src[e] != -1) & (dst[e] != -1)]  # padding edges: zero gradients
         ddx, ddy, ddw = tp_backward(plan, x[src[e]], y[e], w[e], g[dst[e]])
         np.add.at(dx, src[e], scale * ddx)
         dy[e] = scale * ddy

@@ -391,6 +391,49 @@ def test_csr_bit_exact_against_loops():
     assert rp_src.tolist() == [sum(1 for s in src if s < v) for v in range(n + 1)]
 
 
+def test_csr_with_padding_against_loops():
+    """Edges with sender or receiver -1 are padding: outside every row, after the valid edges."""
+    rng, src, dst = small_graph(3)
+    n = 40
+    src, dst = src.copy(), dst.copy()
+    pad = rng.choice(len(src), 25, replace=False)
+    src[pad[:10]] = -1
+    dst[pad[10:20]] = -1
+    src[pad[20:]] = -1
+    dst[pad[20:]] = -1
+    perm_dst, rp_dst, perm_src, rp_src = oracle.csr_build(n, src, dst)
+    valid = [e for e in range(len(src)) if src[e] != -1 and dst[e] != -1]
+    ref = [e for v in range(n) for e in valid if dst[e] == v] + [e for e in range(len(src)) if e not in valid]
+    assert perm_dst.tolist() == ref
+    nv = len(valid)
+    srt = src[perm_dst[:nv]]
+    assert perm_src.tolist() == [i for v in range(n) for i in range(nv) if srt[i] == v] + list(range(nv, len(src)))
+    assert rp_dst.tolist() == [sum(1 for e in valid if dst[e] < v) for v in range(n + 1)]
+    assert rp_src.tolist() == [sum(1 for e in valid if src[e] < v) for v in range(n + 1)]
+
+
+def test_conv_padding_edges_change_nothing():
+    rng, src, dst = small_graph(4)
+    n = 40
+    plan = oracle.make_plan("2x0e+2x1o", "1x0e+1x1o+1x2e", lmax_out=2)
+    x = rng.standard_normal((n, plan.irreps_in1.dim))
+    k = len(src)
+    y = real_sh_all(2, rng.standard_normal((k + 12, 3)))
+    w = rng.standard_normal((k + 12, plan.weight_numel))
+    ps = np.concatenate([src, rng.integers(-1, n, 12)])
+    pd = np.concatenate([dst, np.full(12, -1)])
+    ps[k::3] = -1
+    g = rng.standard_normal((n, plan.irreps_out.dim))
+    np.testing.assert_allclose(oracle.conv_forward(plan, n, ps, pd, x, y, w, 0.5),
+                               oracle.conv_forward(plan, n, src, dst, x, y[:k], w[:k], 0.5), atol=1e-13)
+    dx, dy, dw = oracle.conv_backward(plan, n, ps, pd, x, y, w, g, 0.5)
+    rx, ry, rw = oracle.conv_backward(plan, n, src, dst, x, y[:k], w[:k], g, 0.5)
+    np.testing.assert_allclose(dx, rx, atol=1e-13)
+    np.testing.assert_allclose(dy[:k], ry, atol=1e-13)
+    np.testing.assert_allclose(dw[:k], rw, atol=1e-13)
+    assert np.all(dy[k:] == 0) and np.all(dw[k:] == 0)
+
+
 def test_conv_edge_order_invariance_isolated_and_empty():
     rng, src, dst = small_graph(2)
     n = 40
