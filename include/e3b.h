@@ -195,9 +195,14 @@ E3_API e3_status e3_csr_workspace_size(int64_t N, int64_t E, size_t* bytes);
  *   row_ptr_dst[N+1] node n's in-edges are positions row_ptr_dst[n] .. row_ptr_dst[n+1]-1;
  *   perm_src[E]      positions in receiver order, sorted stably by sender;
  *   row_ptr_src[N+1] node n's out-edges are perm_src[row_ptr_src[n] .. row_ptr_src[n+1]-1].
- * src, dst: int32 [E] in [0, N).  An id out of range records E3_ERR_INDEX in the device
- * status word (e3_device_status) and the outputs are then unspecified.  workspace: device
- * buffer of at least e3_csr_workspace_size bytes, 256-byte aligned.  N, E < 2^31. */
+ * src, dst: int32 [E] in [0, N), or -1 for a padding edge (batches of fixed shape pad the edge
+ * list; the E3J summary, sections 3.1.2 and 3.2, measures what padding edges that point to a
+ * shared padding node cost).  An edge with -1 as sender or receiver belongs to no row: padding
+ * edges follow the valid ones in both orders (input order among themselves), row_ptr_dst[N] and
+ * row_ptr_src[N] count valid edges only, so no kernel walks them and E can stay fixed from step
+ * to step.  Any other id out of range records E3_ERR_INDEX in the device status word
+ * (e3_device_status) and the outputs are then unspecified.  workspace: device buffer of at least
+ * e3_csr_workspace_size bytes, 256-byte aligned.  N, E < 2^31. */
 E3_API e3_status e3_csr_build(int64_t N, int64_t E, const int32_t* src, const int32_t* dst,
                        int32_t* perm_dst, int32_t* row_ptr_dst, int32_t* perm_src,
                        int32_t* row_ptr_src, void* workspace, size_t ws_bytes, void* stream);
@@ -259,7 +264,8 @@ E3_API e3_status e3_remap_ids(int64_t n, const int32_t* ids, int64_t N, const in
 
 /* out[n] = out_scale * sum_{e : dst_e = n} TP(x[src_e], Y_e, w_e)   [CONV][TP]
  * Edge arrays are in receiver order (apply perm_dst once per topology):
- *   row_ptr_dst [N+1] (row_ptr_dst[0] == 0, row_ptr_dst[N] == E, non-decreasing);
+ *   row_ptr_dst [N+1] (row_ptr_dst[0] == 0, non-decreasing; row_ptr_dst[N] <= E, the positions
+ *   from row_ptr_dst[N] on being padding edges, which are not read);
  *   src [E] int32 in [0, N);
  *   exactly one of y [E, dim_in2] (given harmonics) or edge_vec [E, 3] (r_j - r_i, harmonics
  *   computed in registers with normalisation sh_norm; requires irreps_in2 = 1x0+1x1+..);
@@ -279,7 +285,8 @@ E3_API e3_status e3_conv_forward(const e3_plan* plan, int64_t N, int64_t E, cons
  *                        computed from edge_vec);
  *   grad_w [E, weight_numel]: per edge.
  * Any gradient pointer may be NULL to skip it.  Other arguments as e3_conv_forward; dst [E]
- * is the receiver of each (receiver-ordered) edge.  workspace: as for e3_tp_backward, of at
+ * is the receiver of each (receiver-ordered) edge.  Padding positions (from row_ptr_dst[N] on)
+ * get zero grad_y and grad_w rows.  workspace: as for e3_tp_backward, of at
  * least e3_backward_workspace_size(N) bytes.  No atomics on the gradients: the path groups of
  * a sender run in a fixed order, so results are bitwise repeatable.  A group that waits for
  * its predecessor longer than about a second records E3_ERR_TIMEOUT.  Shared weights are not

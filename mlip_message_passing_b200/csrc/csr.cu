@@ -30,16 +30,21 @@ constexpr int RS_RADIX = 256;
 
 __device__ __forceinline__ void rs_error(int* status, int code) { atomicCAS(status, 0, code); }
 
-// key of element i: keys[gather ? gather[i] : i]
-__device__ __forceinline__ uint32_t rs_key(const int32_t* __restrict__ keys, const int32_t* __restrict__ gather,
-                                           int64_t i) {
+// key of element i: keys[j] with j = gather ? gather[i] : i; when `other` is given, an edge whose
+// id in either array is -1 (padding) gets the key `pad` (one past the largest node id), so the
+// stable sort puts padding edges after every valid edge, in element order
+__device__ __forceinline__ uint32_t rs_key(const int32_t* __restrict__ keys, const int32_t* __restrict__ other,
+                                           const int32_t* __restrict__ gather, int64_t i, uint32_t pad) {
   const int64_t j = gather ? int64_t(__ldg(gather + i)) : i;
-  return uint32_t(__ldg(keys + j));
+  const int32_t k = __ldg(keys + j);
+  if (other != nullptr && (k == -1 || __ldg(other + j) == -1)) return pad;
+  return uint32_t(k);
 }
 
 // counts[d * n_tiles + tile] = number of elements of `tile` whose digit is d
 __global__ void __launch_bounds__(RS_THREADS) rs_count(const int32_t* __restrict__ keys,
-                                                       const int32_t* __restrict__ gather, int64_t n,
+                                                       const int32_t* __restrict__ other,
+                                                       const int32_t* __restrict__ gather, uint32_t pad, int64_t n,
                                                        int shift, int n_tiles, int32_t* __restrict__ counts) {
   __shared__ int32_t h[RS_RADIX];
   h[threadIdx.x] = 0;
@@ -47,7 +52,7 @@ __global__ void __launch_bounds__(RS_THREADS) rs_count(const int32_t* __restrict
   const int64_t base = int64_t(blockIdx.x) * RS_TILE;
   for (int r = 0; r < RS_ROUNDS; ++r) {
     const int64_t i = base + int64_t(r) * RS_THREADS + threadIdx.x;
-    if (i < n) atomicAdd(&h[(rs_key(keys, gather, i) >> shift) & 0xff], 1);
+    if (i < n) atomicAdd(&h[(rs_key(keys, other, gather, i, pad) >> shift) & 0xff], 1);
   }
   __syncthreads();
   counts[int64_t(threadIdx.x) * n_tiles + blockIdx.x] = h[threadIdx.x];
@@ -82,7 +87,8 @@ __global__ void __launch_bounds__(1024) exclusive_scan_1cta(int32_t* __restrict_
 
 // Stable scatter of one pass.  offsets: exclusive scan of counts (digit-major).
 __global__ void __launch_bounds__(RS_THREADS) rs_scatter(const int32_t* __restrict__ keys,
-                                                         const int32_t* __restrict__ gather,
+                                                         const int32_t* __restrict__ other,
+                                                         const int32_t* __restrict__ gather, uint32_t pad,
                                                          const int32_t* __restrict__ vals_in, int64_t n, int shift,
                                                          int n_tiles, const int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ keys_out,
@@ -100,7 +106,7 @@ __global__ void __launch_bounds__(RS_THREADS) rs_scatter(const int32_t* __restri
     uint32_t key = 0;
     int d = RS_RADIX;  // sentinel: no element
     if (ok) {
-      key = rs_key(keys, gather, i);
+      key = rs_key(keys, other, gather, i, pad);
       d = int((key >> shift) & 0xff);
     }
     const unsigned peers = __match_any_sync(0xffffffffu, d);
@@ -123,11 +129,13 @@ __global__ void __launch_bounds__(RS_THREADS) rs_scatter(const int32_t* __restri
   }
 }
 
-// degree counts (row_ptr[id] += 1); ids outside [0, N) are reported and skipped
-__global__ void degree_count(const int32_t* __restrict__ ids, int64_t n, int64_t N, int32_t* __restrict__ row_ptr,
-                             int* status) {
+// degree counts (row_ptr[id] += 1); padding edges (-1 in ids or other) are skipped, other ids
+// outside [0, N) are reported and skipped
+__global__ void degree_count(const int32_t* __restrict__ ids, const int32_t* __restrict__ other, int64_t n, int64_t N,
+                             int32_t* __restrict__ row_ptr, int* status) {
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
     const int32_t v = __ldg(ids + i);
+    if (v == -1 || __ldg(other + i) == -1) continue;
     if (v < 0 || v >= N) {
       rs_error(status, E3_ERR_INDEX);
       continue;
@@ -203,6 +211,17 @@ __global__ void remap_ids_kernel(int64_t n, const int32_t* __restrict__ ids, int
   }
 }
 
+// rows [*first_row, n_rows) of 4-byte words set to zero (padding positions after the last row)
+__global__ void zero_tail_kernel(const int32_t* __restrict__ first_row, int64_t n_rows, int64_t row_words,
+                                 uint32_t* __restrict__ p) {
+  const int64_t start = *first_row;
+  if (start < 0 || start >= n_rows) return;
+  const int64_t total = (n_rows - start) * row_words;
+  uint32_t* q = p + start * row_words;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x)
+    q[i] = 0u;
+}
+
 // ------------------------------------------------------------------------ host side ---
 static int64_t n_tiles_of(int64_t E) { return (E + RS_TILE - 1) / RS_TILE; }
 static size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
@@ -218,27 +237,39 @@ static int key_bits(int64_t N) {
   return b;
 }
 
-// Stable sort of element indices 0..n by key(i); writes the sorted indices to vals_final.
-static e3_status radix_sort(const int32_t* keys, const int32_t* gather, int64_t n, int bits, int32_t* vals_final,
-                            int32_t* ka, int32_t* va, int32_t* kb, int32_t* vb, int32_t* counts, cudaStream_t s) {
+// Stable sort of element indices 0..n by key(i) (see rs_key); writes the sorted indices to vals_final.
+static e3_status radix_sort(const int32_t* keys, const int32_t* other, const int32_t* gather, uint32_t pad, int64_t n,
+                            int bits, int32_t* vals_final, int32_t* ka, int32_t* va, int32_t* kb, int32_t* vb,
+                            int32_t* counts, cudaStream_t s) {
   const int n_tiles = int(n_tiles_of(n));
   const int passes = (bits + 7) / 8;
   const int32_t* kin = keys;
+  const int32_t* oin = other;
   const int32_t* gin = gather;
   const int32_t* vin = nullptr;
   for (int p = 0; p < passes; ++p) {
     const bool last = p == passes - 1;
     int32_t* kout = last ? nullptr : (p % 2 == 0 ? ka : kb);
     int32_t* vout = last ? vals_final : (p % 2 == 0 ? va : vb);
-    rs_count<<<n_tiles, RS_THREADS, 0, s>>>(kin, gin, n, 8 * p, n_tiles, counts);
+    rs_count<<<n_tiles, RS_THREADS, 0, s>>>(kin, oin, gin, pad, n, 8 * p, n_tiles, counts);
     exclusive_scan_1cta<<<1, 1024, 0, s>>>(counts, int64_t(RS_RADIX) * n_tiles, nullptr);
-    rs_scatter<<<n_tiles, RS_THREADS, 0, s>>>(kin, gin, vin, n, 8 * p, n_tiles, counts, kout, vout);
-    kin = kout;
+    rs_scatter<<<n_tiles, RS_THREADS, 0, s>>>(kin, oin, gin, pad, vin, n, 8 * p, n_tiles, counts, kout, vout);
+    kin = kout;  // later passes read the (padding-resolved) keys the scatter wrote
+    oin = nullptr;
     gin = nullptr;
     vin = vout;
   }
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "radix sort launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+e3_status zero_rows_after(const int32_t* first_row, int64_t n_rows, int64_t row_bytes, void* ptr, void* stream) {
+  if (n_rows <= 0 || row_bytes <= 0) return E3_OK;
+  zero_tail_kernel<<<148 * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(first_row, n_rows, row_bytes / 4,
+                                                                            static_cast<uint32_t*>(ptr));
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "zero launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
 }
 
@@ -278,8 +309,8 @@ extern "C" e3_status e3_csr_build(int64_t N, int64_t E, const int32_t* src, cons
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "memset failed: %s", cudaGetErrorString(err));
   if (E == 0) return E3_OK;
   const int blocks = int(std::min<int64_t>((E + 255) / 256, 148 * 8));
-  degree_count<<<blocks, 256, 0, s>>>(dst, E, N, row_ptr_dst, status);
-  degree_count<<<blocks, 256, 0, s>>>(src, E, N, row_ptr_src, status);
+  degree_count<<<blocks, 256, 0, s>>>(dst, src, E, N, row_ptr_dst, status);
+  degree_count<<<blocks, 256, 0, s>>>(src, dst, E, N, row_ptr_src, status);
   // row_ptr[n] = c_n for n < N and row_ptr[N] = 0: one exclusive scan over N + 1 entries
   // gives row_ptr[n] = sum_{m < n} c_m and row_ptr[N] = E
   exclusive_scan_1cta<<<1, 1024, 0, s>>>(row_ptr_dst, N + 1, nullptr);
@@ -294,10 +325,10 @@ extern "C" e3_status e3_csr_build(int64_t N, int64_t E, const int32_t* src, cons
   int32_t* kb = reinterpret_cast<int32_t*>(ws + 2 * eb);
   int32_t* vb = reinterpret_cast<int32_t*>(ws + 3 * eb);
   int32_t* counts = reinterpret_cast<int32_t*>(ws + 4 * eb);
-  const int bits = key_bits(N);
-  st = radix_sort(dst, nullptr, E, bits, perm_dst, ka, va, kb, vb, counts, s);
+  const int bits = key_bits(N + 1);  // padding edges take key N
+  st = radix_sort(dst, src, nullptr, uint32_t(N), E, bits, perm_dst, ka, va, kb, vb, counts, s);
   if (st != E3_OK) return st;
-  st = radix_sort(src, perm_dst, E, bits, perm_src, ka, va, kb, vb, counts, s);
+  st = radix_sort(src, dst, perm_dst, uint32_t(N), E, bits, perm_src, ka, va, kb, vb, counts, s);
   return st;
 }
 
@@ -427,7 +458,7 @@ extern "C" e3_status e3_morton_order(int64_t N, const void* pos, e3_dtype dtype,
                                                       scale[0], scale[1], scale[2], codes);
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "morton code launch failed: %s", cudaGetErrorString(err));
-  return radix_sort(codes, nullptr, N, 3 * MORTON_BITS, perm, ka, va, kb, vb, counts, s);
+  return radix_sort(codes, nullptr, nullptr, 0u, N, 3 * MORTON_BITS, perm, ka, va, kb, vb, counts, s);
 }
 
 extern "C" e3_status e3_invert_permutation(int64_t N, const int32_t* perm, int32_t* inv, void* stream) {

@@ -666,7 +666,6 @@ extern "C" e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E,
                                       void* grad_x, void* grad_y, void* grad_w, void* workspace, size_t workspace_bytes,
                                       void* stream) {
   clear_error();
-  (void)row_ptr_dst;
   (void)src;
   e3_status st = check_plan_device(plan);
   if (st != E3_OK) return st;
@@ -677,7 +676,16 @@ extern "C" e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E,
   E3_OPT(grad_y, "grad_y");
   E3_OPT(grad_w, "grad_w");
   if (!grad_x && !grad_y && !grad_w) return E3_OK;
-  if (N == 0) return E3_OK;
+  if (N == 0) {  // without nodes every edge is padding: zero gradients
+    const size_t es = plan->dtype == E3_F64 ? 8 : 4;
+    cudaError_t err = cudaSuccess;
+    if (E > 0 && grad_w != nullptr)
+      err = cudaMemsetAsync(grad_w, 0, size_t(E) * es * plan->weight_numel, static_cast<cudaStream_t>(stream));
+    if (err == cudaSuccess && E > 0 && grad_y != nullptr)
+      err = cudaMemsetAsync(grad_y, 0, size_t(E) * es * plan->dim2, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return fail(E3_ERR_CUDA, "memset failed: %s", cudaGetErrorString(err));
+    return E3_OK;
+  }
   if (row_ptr_src == nullptr) return fail(E3_ERR_INVALID_ARG, "row_ptr_src is NULL");
   if (E > 0) {
     E3_REQ(x, "x");
@@ -694,6 +702,7 @@ extern "C" e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E,
   a.workspace_bytes = workspace_bytes;
   a.n_nodes = N;
   a.n_edges = E;
+  a.row_ptr_dst = row_ptr_dst;
   a.row_ptr_src = row_ptr_src;
   a.perm_src = perm_src;
   a.dst = dst;
@@ -708,5 +717,14 @@ extern "C" e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E,
   a.grad_y = grad_y;
   a.grad_w = grad_w;
   a.stream = stream;
-  return launch_backward(plan, a, true);
+  st = launch_backward(plan, a, true);
+  if (st != E3_OK) return st;
+  // padding edges (receiver-order positions from row_ptr_dst[N] on) get zero gradients
+  const size_t es = plan->dtype == E3_F64 ? 8 : 4;
+  if (E > 0 && grad_w != nullptr) {
+    st = zero_rows_after(row_ptr_dst + N, E, int64_t(es) * plan->weight_numel, grad_w, stream);
+    if (st != E3_OK) return st;
+  }
+  if (E > 0 && grad_y != nullptr) st = zero_rows_after(row_ptr_dst + N, E, int64_t(es) * plan->dim2, grad_y, stream);
+  return st;
 }

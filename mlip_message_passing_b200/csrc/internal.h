@@ -64,6 +64,7 @@ e3_status launch_forward(const e3_plan* plan, const FwdArgs& a, bool conv);
 struct BwdArgs {
   int64_t n_nodes;           // senders (conv) or samples (tp)
   int64_t n_edges;
+  const int32_t* row_ptr_dst; // conv only: row_ptr_dst[N] = first padding position
   const int32_t* row_ptr_src; // conv only
   const int32_t* perm_src;    // conv only
   const int32_t* dst;         // conv only
@@ -84,5 +85,8 @@ struct BwdArgs {
 // Bytes of backward workspace for n units: 16-byte ticket counter + one int per unit.
 inline size_t backward_workspace_bytes(int64_t n) { return (size_t(16) + 4 * size_t(n) + 255) & ~size_t(255); }
 e3_status launch_backward(const e3_plan* plan, const BwdArgs& a, bool conv);
+// Zero rows [*first_row, n_rows) of a row-major array of row_bytes-byte rows (first_row read on
+// the device: the padding positions after the last CSR row).
+e3_status zero_rows_after(const int32_t* first_row, int64_t n_rows, int64_t row_bytes, void* ptr, void* stream);
 
 }  // namespace e3b

@@ -324,6 +324,52 @@ def test_conv_on_morton_renumbered_graph(e3b):
     assert rel_err(h(gw2)[o2], h(b0[2])[o0]) <= 1e-5
 
 
+def test_csr_with_padding_bit_exact(e3b):
+    """Padding edges (-1 as sender, receiver or both) after the valid ones in both orders."""
+    rng = np.random.default_rng(80)
+    n, E = 500, 20000
+    src = rng.integers(0, n, E).astype(np.int32)
+    dst = rng.integers(0, n, E).astype(np.int32)
+    pad = rng.choice(E, 4000, replace=False)
+    src[pad[:1500]] = -1
+    dst[pad[1500:3000]] = -1
+    src[pad[3000:]] = -1
+    dst[pad[3000:]] = -1
+    got = [a.cpu().numpy() for a in e3b.csr_build(n, t(src), t(dst))]
+    e3b.device_status()  # padding is not an error
+    for a, b in zip(got, oracle.csr_build(n, src, dst)):
+        assert np.array_equal(a, b)
+
+
+def test_conv_with_padding_edges(e3b):
+    """A padded water box gives the unpadded results bit for bit; padding edges get zero
+    gradients and no kernel walks them."""
+    n, mul, lx, ly, lo = 400, 64, 2, 3, 2
+    g, graph, w = conv_setup(e3b, n, mul, lx, ly, lo, 21, torch.float32)
+    p = gplan(e3b, mul, lx, ly, lo, torch.float32)
+    rng = np.random.default_rng(81)
+    E = len(g["src"])
+    k = E // 4
+    src_p = np.concatenate([g["src"], rng.integers(-1, n, k).astype(np.int32)])
+    dst_p = np.concatenate([g["dst"], np.full(k, -1, np.int32)])
+    vec_p = np.concatenate([g["vec"], rng.standard_normal((k, 3)).astype(np.float32)])
+    w_p = torch.cat([w, torch.randn(k, p.weight_numel, device=DEV)])
+    gp = e3b.Graph(n, t(src_p), t(dst_p))
+    x, go = t(g["x"]), t(W.grad_out(n, p.dim_out, 5))
+    args = dict(out_scale=0.2)
+    out0 = e3b.conv_forward(p, graph, x, graph.to_receiver_order(w), edge_vec=graph.to_receiver_order(t(g["vec"])),
+                            **args)
+    out1 = e3b.conv_forward(p, gp, x, gp.to_receiver_order(w_p), edge_vec=gp.to_receiver_order(t(vec_p)), **args)
+    assert torch.equal(out0, out1)
+    b0 = e3b.conv_backward(p, graph, x, graph.to_receiver_order(w), go, edge_vec=graph.to_receiver_order(t(g["vec"])),
+                           **args)
+    b1 = e3b.conv_backward(p, gp, x, gp.to_receiver_order(w_p), go, edge_vec=gp.to_receiver_order(t(vec_p)), **args)
+    assert torch.equal(b0[0], b1[0])
+    assert torch.equal(b0[1], b1[1][:E]) and torch.equal(b0[2], b1[2][:E])
+    assert torch.all(b1[1][E:] == 0) and torch.all(b1[2][E:] == 0)
+    e3b.device_status()
+
+
 def test_conv_edge_cases(e3b):
     p = gplan(e3b, 8, 1, 2, 2, torch.float32)
     q = oplan(8, 1, 2, 2)
