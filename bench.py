@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--workload", default="conv_waterbox", choices=["conv_waterbox", "conv_large"])
     ap.add_argument("--reorder", default="none", choices=["none", "morton"],
                     help="renumber nodes along the Morton curve of their positions before timing")
+    ap.add_argument("--padding", type=float, default=0.0,
+                    help="append this fraction of padding edges (ids -1, fixed-shape batches) before timing")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-tp", action="store_true", help="skip the tensor-product (no graph) measurement")
@@ -310,11 +312,19 @@ def run_native(args):
         perm, _, src_t, dst_t = e3b.reorder_graph(torch.as_tensor(g["pos"], device=dev), (0.0, 0.0, 0.0),
                                                   (g["side"],) * 3, src_t, dst_t)
         x, go = e3b.gather_rows(perm, x), e3b.gather_rows(perm, go)
+    vec_t, w_t = torch.as_tensor(g["vec"], device=dev), g["w"]
+    if args.padding > 0:  # padding edges: -1 ids, arbitrary vectors and weights (never read)
+        k = int(round(args.padding * src_t.shape[0]))
+        pad_ids = torch.full((k,), -1, dtype=torch.int32, device=dev)
+        src_t, dst_t = torch.cat([src_t, pad_ids]), torch.cat([dst_t, pad_ids])
+        vec_t = torch.cat([vec_t, torch.ones(k, 3, dtype=vec_t.dtype, device=dev)])
+        w_t = torch.cat([w_t, torch.zeros(k, w_t.shape[1], dtype=w_t.dtype, device=dev)])
     graph = e3b.Graph(N, src_t, dst_t)
     E = graph.n_edges
-    vec = graph.to_receiver_order(torch.as_tensor(g["vec"], device=dev))
-    w = graph.to_receiver_order(g["w"])
-    del g
+    E_work = int(graph.row_ptr_dst[N].item())  # valid edges: the work; padding edges are not
+    vec = graph.to_receiver_order(vec_t)
+    w = graph.to_receiver_order(w_t)
+    del g, vec_t, w_t
     s = 1.0 / math.sqrt(52.0)
     out = torch.empty((N, plan.dim_out), device=dev)
     gx = torch.empty_like(x)
@@ -366,7 +376,7 @@ def run_native(args):
     e3b.device_status()
     ms_total = max_over_ranks(ms_total, world, dist, dev)
     ms_step = ms_total / args.steps
-    value = job_throughput(E, world, ms_step)
+    value = job_throughput(E_work, world, ms_step)
 
     # end to end through the public API: inputs from pinned host memory, results back to host
     e2e = None
@@ -401,7 +411,7 @@ def run_native(args):
         e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world, dist, dev)
         h2d = sum(t.numel() * t.element_size() for t in (hx, hvec, hw, hgo))
         d2h = sum(t.numel() * t.element_size() for t in (hout, hgx, hgy, hgw))
-        e2e = {"value": job_throughput(E, world, e_ms), "unit": "edges/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_throughput(E_work, world, e_ms), "unit": "edges/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     # gradient with respect to the edge vectors (harmonics backward: turns the backward's grad_y
@@ -429,7 +439,7 @@ def run_native(args):
         return 0
 
     tp = None if args.no_tp else measure_tp(args, dev)
-    fb, bb = algorithmic_bytes(N, E, mul, lx, ly, lo)
+    fb, bb = algorithmic_bytes(N, E_work, mul, lx, ly, lo)
     shb = E * (12 + 4 * (ly + 1) ** 2 + 12)
     peak, peak_kind = hbm_peak()
     fwd_gbs, bwd_gbs = fb / (fwd_ms * 1e-3) / 1e9, bb / (bwd_ms * 1e-3) / 1e9
@@ -445,16 +455,17 @@ def run_native(args):
         "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{args.workload}_fwd_bwd", "nodes_per_gpu": N, "edges_per_gpu": E,
+        "config": {"workload": f"{args.workload}_fwd_bwd", "nodes_per_gpu": N, "edges_per_gpu": E_work,
                    "irreps_x": irreps_x, "irreps_sh": irreps_y, "lmax_out": lo, "paths": plan.n_paths,
                    "sh_from": "edge vectors (in-kernel)", "out_scale": "1/sqrt(52)", "parallelism": f"dp{world}",
                    "node_order": "Morton curve of positions" if args.reorder == "morton" else
                                  "as generated (spatially random)",
+                   "padding_edges": f"{args.padding:.0%} of the edges, ids -1" if args.padding > 0 else "none",
                    "l2": "inputs larger than L2: the streamed weights are "
                          f"{w.numel() * 4 / 1e6:.0f} MB per launch (L2 126 MB)"},
-        "fwd": {"ms": fwd_ms, "edges_per_s": E / (fwd_ms * 1e-3), "GBps": fwd_gbs, "frac_of_hbm": fwd_gbs / peak,
+        "fwd": {"ms": fwd_ms, "edges_per_s": E_work / (fwd_ms * 1e-3), "GBps": fwd_gbs, "frac_of_hbm": fwd_gbs / peak,
                 "algorithmic_bytes": fb},
-        "bwd": {"ms": bwd_ms, "edges_per_s": E / (bwd_ms * 1e-3), "GBps": bwd_gbs, "frac_of_hbm": bwd_gbs / peak,
+        "bwd": {"ms": bwd_ms, "edges_per_s": E_work / (bwd_ms * 1e-3), "GBps": bwd_gbs, "frac_of_hbm": bwd_gbs / peak,
                 "algorithmic_bytes": bb},
         "sh_bwd": {"ms": sh_ms, "edges_per_s": E / (sh_ms * 1e-3), "GBps": shb / (sh_ms * 1e-3) / 1e9,
                    "frac_of_hbm": shb / (sh_ms * 1e-3) / 1e9 / peak, "algorithmic_bytes": shb,
