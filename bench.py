@@ -330,7 +330,7 @@ def run_native(args):
     gx = torch.empty_like(x)
     gy = torch.empty((E, plan.dim_in2), device=dev)
     gw = torch.empty_like(w)
-    ws = e3b.backward_workspace(N, dev)
+    ws = e3b.conv_workspace(plan, N, E, dev)
     stream = torch.cuda.current_stream()
     ev = []
 
@@ -339,13 +339,15 @@ def run_native(args):
             a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             a.record(stream)
         e3b.lib.e3_conv_forward(plan.handle, N, E, e3b._ptr(graph.row_ptr_dst), e3b._ptr(graph.src), e3b._ptr(x),
-                                None, e3b._ptr(vec), 0, e3b._ptr(w), s, e3b._ptr(out), e3b._stream())
+                                None, e3b._ptr(vec), 0, e3b._ptr(w), s, e3b._ptr(out), e3b._ptr(graph.topo),
+                                e3b._ptr(ws), ws.numel(), e3b._stream())
         if record:
             b.record(stream)
         e3b.lib.e3_conv_backward(plan.handle, N, E, e3b._ptr(graph.row_ptr_dst), e3b._ptr(graph.src),
                                  e3b._ptr(graph.dst), e3b._ptr(graph.row_ptr_src), e3b._ptr(graph.perm_src),
                                  e3b._ptr(x), None, e3b._ptr(vec), 0, e3b._ptr(w), e3b._ptr(go), s, e3b._ptr(gx),
-                                 e3b._ptr(gy), e3b._ptr(gw), e3b._ptr(ws), ws.numel(), e3b._stream())
+                                 e3b._ptr(gy), e3b._ptr(gw), e3b._ptr(graph.topo), e3b._ptr(ws), ws.numel(),
+                                 e3b._stream())
         if record:
             c.record(stream)
             ev.append((a, b, c))

@@ -149,7 +149,7 @@ E3_API const char* e3_supported(void);
 E3_API e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x, const void* y,
                         const void* w, void* out, void* stream);
 
-/* Bytes of device workspace that e3_tp_backward (n = B) and e3_conv_backward (n = N) need:
+/* Bytes of device workspace that e3_tp_backward needs for n = B samples:
  * a ticket counter and one progress counter per work unit, which order the path groups of a
  * unit inside one launch.  The backward zeroes it on its stream before use. */
 E3_API e3_status e3_backward_workspace_size(int64_t n, size_t* bytes);
@@ -262,6 +262,17 @@ E3_API e3_status e3_remap_ids(int64_t n, const int32_t* ids, int64_t N, const in
 
 /* ----------------------------------------------------------------------- convolution --- */
 
+/* Work units of the convolution for one topology [CONV]: each receiver's in-edges (receiver CSR)
+ * and each sender's out-edges (sender CSR) are cut into segments of at most 256 edges (one for a
+ * row of <= 256 edges, also an empty one) -- the units the convolution's CTAs walk, so that a hub
+ * does not serialise on one CTA.  Build once per topology, after e3_csr_build, and pass the
+ * buffer to every e3_conv_forward / e3_conv_backward of that topology.  topo: device buffer of at
+ * least e3_conv_topology_size(N, E) bytes, 16-byte aligned, owned by the caller.  A row pointer
+ * out of range records E3_ERR_INDEX and gives that row no edges.  Integer-only. */
+E3_API e3_status e3_conv_topology_size(int64_t N, int64_t E, size_t* bytes);
+E3_API e3_status e3_conv_topology_build(int64_t N, int64_t E, const int32_t* row_ptr_dst,
+                                 const int32_t* row_ptr_src, void* topo, size_t topo_bytes, void* stream);
+
 /* out[n] = out_scale * sum_{e : dst_e = n} TP(x[src_e], Y_e, w_e)   [CONV][TP]
  * Edge arrays are in receiver order (apply perm_dst once per topology):
  *   row_ptr_dst [N+1] (row_ptr_dst[0] == 0, non-decreasing; row_ptr_dst[N] <= E, the positions
@@ -271,13 +282,19 @@ E3_API e3_status e3_remap_ids(int64_t n, const int32_t* ids, int64_t N, const in
  *   computed in registers with normalisation sh_norm; requires irreps_in2 = 1x0+1x1+..);
  *   w [E, weight_numel] (or [weight_numel] if shared); x [N, dim_in1]; out [N, dim_out]
  *   (overwritten; nodes without in-edges get zero rows).  E == 0 zero-fills out.
- * No atomics: each output row is reduced by one CTA in edge order.  An src id or row_ptr
- * entry out of range records E3_ERR_INDEX in the device status word and that edge is
- * skipped.  N, E < 2^31. */
+ * No floating-point atomics: each output row is reduced in edge order -- by one CTA, or, for a
+ * row of more than 256 edges, by one CTA per 256-edge segment whose partial sums are added to the
+ * row in segment order (a progress counter per row and path group orders them), so hubs do not
+ * serialise and results stay bitwise repeatable.  topo: the buffer e3_conv_topology_build filled
+ * for this row_ptr_dst (and the matching sender CSR).  workspace: device buffer of at least
+ * e3_conv_workspace_size(plan, N, E) bytes, 16-byte aligned, owned by the caller and not used by
+ * any other call while this one runs on its stream (the call zeroes it).  An src id out of range
+ * records E3_ERR_INDEX in the device status word and that edge is skipped.  N, E < 2^31. */
+E3_API e3_status e3_conv_workspace_size(const e3_plan* plan, int64_t N, int64_t E, size_t* bytes);
 E3_API e3_status e3_conv_forward(const e3_plan* plan, int64_t N, int64_t E, const int32_t* row_ptr_dst,
                           const int32_t* src, const void* x, const void* y, const void* edge_vec,
                           e3_sh_norm sh_norm, const void* w, double out_scale, void* out,
-                          void* stream);
+                          const void* topo, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Gradients of <grad_out, conv_forward(...)> [BWD][CONV] with respect to
  *   grad_x [N, dim_in1]: sum over each node's out-edges (sender CSR: row_ptr_src, perm_src);
@@ -286,8 +303,8 @@ E3_API e3_status e3_conv_forward(const e3_plan* plan, int64_t N, int64_t E, cons
  *   grad_w [E, weight_numel]: per edge.
  * Any gradient pointer may be NULL to skip it.  Other arguments as e3_conv_forward; dst [E]
  * is the receiver of each (receiver-ordered) edge.  Padding positions (from row_ptr_dst[N] on)
- * get zero grad_y and grad_w rows.  workspace: as for e3_tp_backward, of at
- * least e3_backward_workspace_size(N) bytes.  No atomics on the gradients: the path groups of
+ * get zero grad_y and grad_w rows.  Senders with more than 256 out-edges are split into
+ * 256-edge segments like the forward's rows.  topo and workspace: as for e3_conv_forward.  No atomics on the gradients: the path groups of
  * a sender run in a fixed order, so results are bitwise repeatable.  A group that waits for
  * its predecessor longer than about a second records E3_ERR_TIMEOUT.  Shared weights are not
  * supported. */
@@ -296,7 +313,8 @@ E3_API e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E, con
                            const int32_t* perm_src, const void* x, const void* y,
                            const void* edge_vec, e3_sh_norm sh_norm, const void* w,
                            const void* grad_out, double out_scale, void* grad_x, void* grad_y,
-                           void* grad_w, void* workspace, size_t workspace_bytes, void* stream);
+                           void* grad_w, const void* topo, void* workspace, size_t workspace_bytes,
+                           void* stream);
 
 /* Message of the last non-OK status returned on the calling thread ("" if none). */
 E3_API const char* e3_last_error(void);

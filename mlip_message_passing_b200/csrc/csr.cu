@@ -211,6 +211,40 @@ __global__ void remap_ids_kernel(int64_t n, const int32_t* __restrict__ ids, int
   }
 }
 
+// segments per row (at least one, so that every row is written), seg_start[N] = 0 for the scan
+__global__ void seg_count_kernel(int64_t N, const int32_t* __restrict__ row_ptr, int32_t* __restrict__ seg_start) {
+  for (int64_t n = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; n <= N; n += int64_t(gridDim.x) * blockDim.x) {
+    if (n == N) {
+      seg_start[N] = 0;
+      continue;
+    }
+    const int64_t deg = int64_t(row_ptr[n + 1]) - row_ptr[n];
+    seg_start[n] = deg <= SEG_EDGES ? 1 : int32_t((deg + SEG_EDGES - 1) / SEG_EDGES);
+  }
+}
+
+// the units of each row: {row, first edge, end edge, segment} and the row's segment count; the
+// number of units goes to *units.  Rows whose pointers are out of range get empty units.
+__global__ void unit_fill_kernel(int64_t N, int64_t E, const int32_t* __restrict__ row_ptr,
+                                 const int32_t* __restrict__ seg_start, int4* __restrict__ info,
+                                 int32_t* __restrict__ nseg, int32_t* __restrict__ units, int* status) {
+  for (int64_t n = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; n < N; n += int64_t(gridDim.x) * blockDim.x) {
+    int64_t r0 = row_ptr[n], r1 = row_ptr[n + 1];
+    if (r0 < 0 || r1 < r0 || r1 > E) {
+      atomicCAS(status, 0, int(E3_ERR_INDEX));
+      r0 = r1 = 0;
+    }
+    const int32_t u0 = seg_start[n], k = seg_start[n + 1] - u0;
+    for (int32_t s = 0; s < k; ++s) {
+      const int64_t e0 = r0 + int64_t(s) * SEG_EDGES;
+      const int64_t e1 = e0 + SEG_EDGES < r1 ? e0 + SEG_EDGES : r1;
+      info[u0 + s] = make_int4(int(n), int(e0 < e1 ? e0 : e1), int(e1), s);
+      nseg[u0 + s] = k;
+    }
+    if (n == N - 1) *units = seg_start[N];
+  }
+}
+
 // rows [*first_row, n_rows) of 4-byte words set to zero (padding positions after the last row)
 __global__ void zero_tail_kernel(const int32_t* __restrict__ first_row, int64_t n_rows, int64_t row_words,
                                  uint32_t* __restrict__ p) {
@@ -261,6 +295,27 @@ static e3_status radix_sort(const int32_t* keys, const int32_t* other, const int
   }
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "radix sort launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+e3_status build_topo_part(int64_t N, int64_t E, const int32_t* row_ptr, unsigned char* base, const TopoPart& t,
+                          void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* units = reinterpret_cast<int32_t*>(base + t.units);
+  cudaError_t err = cudaMemsetAsync(units, 0, 16, s);
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "memset failed: %s", cudaGetErrorString(err));
+  if (N <= 0) return E3_OK;
+  int* status = nullptr;
+  e3_status st = device_status_ptr(&status);
+  if (st != E3_OK) return st;
+  int32_t* seg_start = reinterpret_cast<int32_t*>(base + t.seg_start);
+  const int blocks = int(std::min<int64_t>((N + 256) / 256, 148 * 8));
+  seg_count_kernel<<<blocks, 256, 0, s>>>(N, row_ptr, seg_start);
+  exclusive_scan_1cta<<<1, 1024, 0, s>>>(seg_start, N + 1, nullptr);
+  unit_fill_kernel<<<blocks, 256, 0, s>>>(N, E, row_ptr, seg_start, reinterpret_cast<int4*>(base + t.info),
+                                          reinterpret_cast<int32_t*>(base + t.nseg), units, status);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "topology launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
 }
 
@@ -490,4 +545,27 @@ extern "C" e3_status e3_remap_ids(int64_t n, const int32_t* ids, int64_t N, cons
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "remap launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
+}
+
+// ------------------------------------------------------------------- convolution units ---
+extern "C" e3_status e3_conv_topology_size(int64_t N, int64_t E, size_t* bytes) {
+  clear_error();
+  if (bytes == nullptr) return fail(E3_ERR_INVALID_ARG, "bytes is NULL");
+  if (N < 0 || E < 0 || N >= (int64_t(1) << 31) || E >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N or E out of range");
+  *bytes = topo_bytes(N, E);
+  return E3_OK;
+}
+
+extern "C" e3_status e3_conv_topology_build(int64_t N, int64_t E, const int32_t* row_ptr_dst, const int32_t* row_ptr_src,
+                                            void* topo, size_t topo_bytes_, void* stream) {
+  clear_error();
+  if (N < 0 || E < 0 || N >= (int64_t(1) << 31) || E >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N or E out of range");
+  if (topo == nullptr || (reinterpret_cast<uintptr_t>(topo) & 15u) != 0)
+    return fail(E3_ERR_INVALID_ARG, "topology buffer is NULL or not 16-byte aligned");
+  if (topo_bytes_ < topo_bytes(N, E)) return fail(E3_ERR_SHAPE, "topology buffer of %zu bytes, need %zu", topo_bytes_, topo_bytes(N, E));
+  if (N > 0 && (row_ptr_dst == nullptr || row_ptr_src == nullptr)) return fail(E3_ERR_INVALID_ARG, "row_ptr array is NULL");
+  unsigned char* base = static_cast<unsigned char*>(topo);
+  e3_status st = build_topo_part(N, E, row_ptr_dst, base, topo_dst(N, E), stream);
+  if (st != E3_OK) return st;
+  return build_topo_part(N, E, row_ptr_src, base, topo_src(N, E), stream);
 }

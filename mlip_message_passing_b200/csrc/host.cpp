@@ -566,6 +566,27 @@ extern "C" e3_status e3_backward_workspace_size(int64_t n, size_t* bytes) {
   return E3_OK;
 }
 
+int e3b::plan_groups(const e3_plan* plan) { return make_path_table(plan->LX, plan->LY, plan->LO, GROUP_OUT_CAP).ngroups; }
+
+extern "C" e3_status e3_conv_workspace_size(const e3_plan* plan, int64_t N, int64_t E, size_t* bytes) {
+  clear_error();
+  if (plan == nullptr || bytes == nullptr) return fail(E3_ERR_INVALID_ARG, "plan or bytes is NULL");
+  if (N < 0 || E < 0 || N >= (int64_t(1) << 31) || E >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N or E out of range");
+  *bytes = conv_counters(N, E, plan_groups(plan)).total;
+  return E3_OK;
+}
+
+static e3_status check_conv_workspace(const e3_plan* plan, int64_t N, int64_t E, const void* topo, const void* ws,
+                                      size_t ws_bytes) {
+  if (topo == nullptr) return fail(E3_ERR_INVALID_ARG, "topology buffer is NULL");
+  if (reinterpret_cast<uintptr_t>(topo) % 16 != 0) return fail(E3_ERR_INVALID_ARG, "topology buffer is not 16-byte aligned");
+  if (ws == nullptr) return fail(E3_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 16 != 0) return fail(E3_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  const size_t need = conv_counters(N, E, plan_groups(plan)).total;
+  if (ws_bytes < need) return fail(E3_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", ws_bytes, need);
+  return E3_OK;
+}
+
 static e3_status check_workspace(int64_t n, const void* ws, size_t ws_bytes) {
   if (ws == nullptr) return fail(E3_ERR_INVALID_ARG, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(ws) % 16 != 0) return fail(E3_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
@@ -626,7 +647,7 @@ static e3_status check_conv_common(const e3_plan* plan, int64_t N, int64_t E, co
 extern "C" e3_status e3_conv_forward(const e3_plan* plan, int64_t N, int64_t E, const int32_t* row_ptr_dst,
                                      const int32_t* src, const void* x, const void* y, const void* edge_vec,
                                      e3_sh_norm sh_norm, const void* w, double out_scale, void* out,
-                                     void* stream) {
+                                     const void* topo, void* workspace, size_t workspace_bytes, void* stream) {
   clear_error();
   e3_status st = check_plan_device(plan);
   if (st != E3_OK) return st;
@@ -642,7 +663,11 @@ extern "C" e3_status e3_conv_forward(const e3_plan* plan, int64_t N, int64_t E, 
     if (src == nullptr) return fail(E3_ERR_INVALID_ARG, "src is NULL");
   }
   if (!std::isfinite(out_scale)) return fail(E3_ERR_INVALID_ARG, "out_scale is not finite");
+  st = check_conv_workspace(plan, N, E, topo, workspace, workspace_bytes);
+  if (st != E3_OK) return st;
   FwdArgs a{};
+  a.topo = topo;
+  a.workspace = workspace;
   a.n_rows = N;
   a.n_edges = E;
   a.row_ptr = row_ptr_dst;
@@ -663,7 +688,8 @@ extern "C" e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E,
                                       const int32_t* src, const int32_t* dst, const int32_t* row_ptr_src,
                                       const int32_t* perm_src, const void* x, const void* y, const void* edge_vec,
                                       e3_sh_norm sh_norm, const void* w, const void* grad_out, double out_scale,
-                                      void* grad_x, void* grad_y, void* grad_w, void* workspace, size_t workspace_bytes,
+                                      void* grad_x, void* grad_y, void* grad_w, const void* topo, void* workspace,
+                                      size_t workspace_bytes,
                                       void* stream) {
   clear_error();
   (void)src;
@@ -695,9 +721,10 @@ extern "C" e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E,
     if (dst == nullptr || perm_src == nullptr) return fail(E3_ERR_INVALID_ARG, "dst or perm_src is NULL");
   }
   if (!std::isfinite(out_scale)) return fail(E3_ERR_INVALID_ARG, "out_scale is not finite");
-  st = check_workspace(N, workspace, workspace_bytes);
+  st = check_conv_workspace(plan, N, E, topo, workspace, workspace_bytes);
   if (st != E3_OK) return st;
   BwdArgs a{};
+  a.topo = topo;
   a.workspace = workspace;
   a.workspace_bytes = workspace_bytes;
   a.n_nodes = N;

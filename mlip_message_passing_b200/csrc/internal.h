@@ -57,6 +57,8 @@ struct FwdArgs {
   int64_t w_stride;          // weight_numel, or 0 for shared weights
   double scale;
   void* out;
+  const void* topo;          // conv only: topology buffer (receiver part used)
+  void* workspace;           // conv only: conv_counters
   void* stream;
 };
 e3_status launch_forward(const e3_plan* plan, const FwdArgs& a, bool conv);
@@ -78,12 +80,59 @@ struct BwdArgs {
   void* grad_x;
   void* grad_y;
   void* grad_w;
-  void* workspace;           // e3_backward_workspace_size(n_nodes) bytes
+  const void* topo;          // conv only: topology buffer (sender part used)
+  void* workspace;           // conv: conv_counters; tp: e3_backward_workspace_size(n_nodes) bytes
   size_t workspace_bytes;
   void* stream;
 };
 // Bytes of backward workspace for n units: 16-byte ticket counter + one int per unit.
 inline size_t backward_workspace_bytes(int64_t n) { return (size_t(16) + 4 * size_t(n) + 255) & ~size_t(255); }
+
+// Row segmentation of the convolution: no CTA walks more than SEG_EDGES edges of one row; a row
+// of deg edges has max(1, ceil(deg / SEG_EDGES)) segments, each a work unit.
+constexpr int64_t SEG_EDGES = 256;
+inline int64_t seg_units_max(int64_t N, int64_t E) { return N + E / SEG_EDGES + 1; }
+inline size_t al16(size_t b) { return (b + 15) & ~size_t(15); }
+
+// Topology buffer (built once per topology by e3_conv_topology_build), one part per direction
+// (receivers: dst, senders: src), each
+//   units (int, padded to 16 B) | info [units_max] int4 {row, first edge, end edge, segment} |
+//   nseg [units_max] int (segments of the unit's row) | seg_start [N + 1] int (scratch)
+struct TopoPart {
+  size_t units, info, nseg, seg_start, end;
+};
+inline TopoPart topo_part(int64_t N, int64_t E, size_t base) {
+  const int64_t U = seg_units_max(N, E);
+  TopoPart t{};
+  t.units = base;
+  t.info = base + 16;
+  t.nseg = t.info + al16(16 * size_t(U));
+  t.seg_start = t.nseg + al16(4 * size_t(U));
+  t.end = t.seg_start + al16(4 * size_t(N + 1));
+  return t;
+}
+inline TopoPart topo_dst(int64_t N, int64_t E) { return topo_part(N, E, 0); }
+inline TopoPart topo_src(int64_t N, int64_t E) { return topo_part(N, E, topo_dst(N, E).end); }
+inline size_t topo_bytes(int64_t N, int64_t E) { return (topo_src(N, E).end + 255) & ~size_t(255); }
+// Fill one direction's part from row_ptr [N + 1] (rows with out-of-range pointers record
+// E3_ERR_INDEX and get empty units); stream-ordered.
+e3_status build_topo_part(int64_t N, int64_t E, const int32_t* row_ptr, unsigned char* base, const TopoPart& t,
+                          void* stream);
+
+// Per-call counters of a convolution launch (zeroed by the call):
+//   ticket (16 B) | flags [units_max * G] int | chain [N] int
+struct ConvCounters {
+  size_t flags, chain, total;
+};
+inline ConvCounters conv_counters(int64_t N, int64_t E, int G) {
+  ConvCounters c{};
+  c.flags = 16;
+  c.chain = c.flags + al16(4 * size_t(seg_units_max(N, E)) * size_t(G));
+  c.total = (c.chain + al16(4 * size_t(N)) + 255) & ~size_t(255);
+  return c;
+}
+// path groups of a plan's kernels
+int plan_groups(const e3_plan* plan);
 e3_status launch_backward(const e3_plan* plan, const BwdArgs& a, bool conv);
 // Zero rows [*first_row, n_rows) of a row-major array of row_bytes-byte rows (first_row read on
 // the device: the padding positions after the last CSR row).

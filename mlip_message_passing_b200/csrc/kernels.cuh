@@ -325,6 +325,14 @@ struct KFwd {
   int64_t n_rows, n_edges, w_stride;
   int C, sh_norm, n_chunks, stages;
   int* status;
+  // convolution: ticket counter and per (row, group) progress counters (zero at launch), the
+  // receiver units of the topology buffer and their number, and the grid's bound on it
+  int* ticket;
+  int* flags;
+  const int4* uinfo;
+  const int32_t* unseg;
+  const int32_t* n_units;
+  int64_t units_max;
   double pscale[MAXP];  // scale * alpha_p
 };
 
@@ -452,6 +460,24 @@ struct FwdAcc {
           }
         });
       }
+    });
+  }
+
+  // out[row, path blocks of the group, channels 4cb..] += pscale_p * acc (a later row segment)
+  __device__ __forceinline__ void store_add(T* __restrict__ orow, int C, int cb, const double* pscale) {
+    static_for<GR::PB, GR::PE>([&](auto pc) {
+      constexpr int P = decltype(pc)::value;
+      using PC = PathC<CF, P>;
+      constexpr int D3 = PC::D3, OO = PC::OUT - GR::OB;
+      const T s = T(pscale[P]);
+      T* p = orow + size_t(C) * PC::OUT + size_t(4 * cb) * D3;
+      T t[K * D3];
+      ld16_l2(t, p);
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int m = 0; m < D3; ++m) t[k * D3 + m] += s * acc[k][OO + m];
+      st16(p, t);
     });
   }
 
@@ -622,7 +648,8 @@ __device__ __noinline__ void fwd_stage_window(const KFwd& a, int64_t e0, int64_t
 }
 
 template <class CF, int GI, bool CONV, int CC>
-__device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned char* smem) {
+__device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, int64_t e0_in, int64_t e1_in, int64_t seg,
+                                          int64_t nseg, unsigned char* smem) {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
   using SM = FwdSmem<CF>;
@@ -648,15 +675,12 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SM::flag_off(S));
   unsigned char* stages = smem + SM::stage_off(S);
 
-  // segment of rows handled by this CTA
+  // edges handled by this CTA: segment `seg` of receiver `unit`'s in-edges (convolution; the
+  // topology build checked the row pointers)
   int64_t e0, e1;
   if constexpr (CONV) {
-    e0 = a.row_ptr[unit];
-    e1 = a.row_ptr[unit + 1];
-    if (e0 < 0 || e1 < e0 || e1 > a.n_edges) {
-      if (tid == 0) record_error(a.status, E3_ERR_INDEX);
-      e0 = e1 = 0;
-    }
+    e0 = e0_in;
+    e1 = e1_in;
   } else {
     const int64_t per = (a.n_rows + a.n_chunks - 1) / a.n_chunks;
     e0 = unit * per;
@@ -739,11 +763,15 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
     }
     __syncthreads();  // window staging buffers are reused by the next window
   }
+  // a row split into segments: its segments add their partial sums in segment order
+  int* seg_flag = (CONV && nseg > 1) ? a.flags + unit * CF::G + GI : nullptr;
   if (!alive) {
     // a wait gave up: let the copies in flight land (bounded) before the CTA exits
     if (tid == 0)
       for (uint32_t q = consumed - 1; q < issued; ++q) mbar_wait(&bars[q % S], (q / S) & 1u, a.status);
     __syncthreads();
+    if (seg_flag != nullptr && tid == 0)  // later segments must not wait for this one in vain
+      asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(seg_flag), "r"(int(seg + 1)) : "memory");
     return;
   }
   if constexpr (CONV) {
@@ -754,7 +782,36 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, unsigned 
 #pragma unroll
           for (int o = 0; o < GR::NOG; ++o) f.acc[k][o] += __shfl_xor_sync(0xffffffffu, f.acc[k][o], off);
     }
-    if (slice == 0) f.store(out + size_t(unit) * orow, C, cb, a.pscale);
+    if (seg_flag == nullptr) {
+      if (slice == 0) f.store(out + size_t(unit) * orow, C, cb, a.pscale);
+    } else {
+      // wait (bounded) until the earlier segments of this row and group have added theirs; the
+      // segment that waits drew a later ticket than those it waits for, so they are resident or
+      // finished
+      if (tid == 0 && seg > 0) {
+        const unsigned long long t0 = global_ns();
+        int v;
+        while (true) {
+          asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(seg_flag) : "memory");
+          if (v >= seg) break;
+          if (global_ns() - t0 > WAIT_NS) {
+            record_error(a.status, E3_ERR_TIMEOUT);
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+      __syncthreads();
+      if (slice == 0) {
+        if (seg == 0)
+          f.store(out + size_t(unit) * orow, C, cb, a.pscale);
+        else
+          f.store_add(out + size_t(unit) * orow, C, cb, a.pscale);
+      }
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(seg_flag), "r"(int(seg + 1)) : "memory");
+    }
   }
 }
 
@@ -768,12 +825,29 @@ constexpr int fwd_min_blocks() {
 template <class CF, bool CONV, int CC>
 __global__ void __launch_bounds__(256, fwd_min_blocks<CF>()) fwd_kernel(const __grid_constant__ KFwd a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  // group-major order: CTAs are started roughly in index order, so the CTAs resident on an SM
-  // at any time run the same path group and share its (large, fully unrolled) code
-  const int64_t units = int64_t(gridDim.x) / CF::G;
-  const int g = int(blockIdx.x / units);
-  const int64_t unit = blockIdx.x % units;
-  dispatch<CF::G>(g, [&](auto gi) { fwd_group<CF, decltype(gi)::value, CONV, CC>(a, unit, smem_raw); });
+  // group-major order, so the CTAs resident on an SM at any time mostly run the same path group
+  // and share its (large, fully unrolled) code
+  if constexpr (CONV) {
+    // a ticket per CTA (tickets follow the order CTAs start in): group, then row segment; a row's
+    // later segments wait for its earlier ones, which hold earlier tickets
+    __shared__ int s_ticket;
+    if (threadIdx.x == 0) s_ticket = atomicAdd(a.ticket, 1);
+    __syncthreads();
+    const int t = s_ticket;
+    const int g = int(t / a.units_max);
+    const int64_t u = t % a.units_max;
+    const int4 inf = a.uinfo[u];  // {row, first edge, end edge, segment}; in bounds for u < units_max
+    const int64_t nseg = a.unseg[u];
+    if (u >= *a.n_units) return;  // the grid covers an upper bound of the units
+    dispatch<CF::G>(g, [&](auto gi) {
+      fwd_group<CF, decltype(gi)::value, CONV, CC>(a, inf.x, inf.y, inf.z, inf.w, nseg, smem_raw);
+    });
+  } else {
+    const int64_t units = int64_t(gridDim.x) / CF::G;
+    const int g = int(blockIdx.x / units);
+    const int64_t unit = blockIdx.x % units;
+    dispatch<CF::G>(g, [&](auto gi) { fwd_group<CF, decltype(gi)::value, CONV, CC>(a, unit, 0, 0, 0, 1, smem_raw); });
+  }
 }
 
 // ========================================================================= backward ===
@@ -795,6 +869,11 @@ struct KBwd {
   int* status;
   int* ticket;          // CTA ticket counter (zero at launch)
   int* done;            // per unit: path groups finished (zero at launch)
+  int* chain;           // convolution, per sender split into segments: (group, segment) pairs that
+                        // have added their grad_x, in group-major order (zero at launch)
+  const int4* uinfo;    // convolution: sender units of the topology buffer
+  const int32_t* unseg;
+  const int32_t* n_units;
   double scale;
   double alpha[MAXP];
   float alpha_f[MAXP];  // the same path weights rounded once, for the float kernels
@@ -1086,7 +1165,7 @@ __device__ __forceinline__ int block_of(int m) { return m >= 9 ? 3 : (m >= 4 ? 2
 // group 0 also zero-fills the blocks no group touches.
 template <class CF, int GI>
 __device__ __forceinline__ void bwd_put_dx(typename CF::T* __restrict__ row, const typename CF::T (&dx)[K][Grp<CF, GI>::NXG],
-                                           int C, int cb, typename CF::T scale) {
+                                           int C, int cb, typename CF::T scale, bool seg0 = true) {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
   static_for<GR::L1A, GR::L1B + 1>([&](auto lc) {
@@ -1094,20 +1173,22 @@ __device__ __forceinline__ void bwd_put_dx(typename CF::T* __restrict__ row, con
     constexpr int D = 2 * L + 1;
     T* p = row + size_t(C) * (L * L) + size_t(4 * cb) * D;
     T v[K * D];
-    if constexpr (first_group_l1<CF>(L) != GI) ld16_l2(v, p);
+    // the first segment of the first group touching block L stores, every later one adds
+    const bool store = first_group_l1<CF>(L) == GI && seg0;
+    if (!store) ld16_l2(v, p);
 #pragma unroll
     for (int k = 0; k < K; ++k)
 #pragma unroll
       for (int m = 0; m < D; ++m) {
         const T s = scale * dx[k][L * L - GR::XB + m];
-        if constexpr (first_group_l1<CF>(L) == GI)
+        if (store)
           v[k * D + m] = s;
         else
           v[k * D + m] += s;
       }
     st16(p, v);
   });
-  if constexpr (GI == 0) {
+  if (GI == 0 && seg0) {
     static_for<0, CF::LX + 1>([&](auto lc) {
       constexpr int L = decltype(lc)::value;
       constexpr int D = 2 * L + 1;
@@ -1156,7 +1237,9 @@ __device__ __forceinline__ void bwd_end_turn(const KBwd& a, int64_t unit, int gi
 // Backward of path group GI for one unit.  Convolution: one CTA (one warp) per sender,
 // walking its out-edges through the sender CSR; tensor product: one CTA per sample range.
 template <class CF, int GI, bool CONV, int CC>
-__device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsigned char* smem) {
+__device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const int64_t n, const int64_t j0_in,
+                                          const int64_t j1_in, const int64_t seg, const int64_t nseg,
+                                          unsigned char* smem) {
   using T = typename CF::T;
   using GR = Grp<CF, GI>;
   using SM = BwdSmem<CF, GI>;
@@ -1189,14 +1272,11 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsign
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SM::flag_off(S));
   unsigned char* stages = smem + SM::stage_off(S);
 
+  // unit u: segment `seg` (of nseg) of sender n's out-edges (convolution), or sample range n
   int64_t j0, j1;
   if constexpr (CONV) {
-    j0 = a.row_ptr_src[n];
-    j1 = a.row_ptr_src[n + 1];
-    if (j0 < 0 || j1 < j0 || j1 > a.n_edges) {
-      if (lane == 0) record_error(a.status, E3_ERR_INDEX);
-      j0 = j1 = 0;
-    }
+    j0 = j0_in;  // the topology build checked the row pointers
+    j1 = j1_in;
   } else {
     const int64_t per = (a.n_nodes + a.n_chunks - 1) / a.n_chunks;
     j0 = n * per;
@@ -1208,7 +1288,7 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsign
     *s_abort = 0;
     mbar_fence_init();
   }
-  bwd_wait_turn(a, n, GI);
+  bwd_wait_turn(a, u, GI);
   __syncthreads();
 
   T xr[K][GR::NXG], dx[K][GR::NXG], Y[CF::NY], dY[CF::NY];
@@ -1375,12 +1455,17 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsign
     }
     __syncthreads();
   }
+  // a sender split into segments adds its grad_x in (group, segment) order through a.chain
+  int* chain = (CONV && nseg > 1) ? a.chain + n : nullptr;
+  const int pos = int(GI * nseg + seg);
   if (!alive) {
     // a wait gave up: let the copies in flight land (bounded) before the CTA exits
     if (lane == 0)
       for (uint32_t q = consumed - 1; q < issued; ++q) mbar_wait(&bars[q % S], (q / S) & 1u, a.status);
     __syncthreads();
-    bwd_end_turn(a, n, GI);
+    if (chain != nullptr && lane == 0)  // later pairs must not wait for this one in vain
+      asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(chain), "r"(pos + 1) : "memory");
+    bwd_end_turn(a, u, GI);
     return;
   }
   if constexpr (CONV) {
@@ -1390,10 +1475,33 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t n, unsign
         for (int k = 0; k < K; ++k)
 #pragma unroll
           for (int j = 0; j < GR::NXG; ++j) dx[k][j] += __shfl_xor_sync(0xffffffffu, dx[k][j], off);
-      if (slice == 0) bwd_put_dx<CF, GI>(gx + size_t(n) * xrow, dx, C, cb, scale);
+      if (chain != nullptr && lane == 0 && pos > 0) {
+        // wait (bounded) for the earlier (group, segment) pairs of this sender; they drew
+        // earlier tickets, so they are resident or finished
+        const unsigned long long t0 = global_ns();
+        int v;
+        while (true) {
+          asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(chain) : "memory");
+          if (v >= pos) break;
+          if (global_ns() - t0 > WAIT_NS) {
+            record_error(a.status, E3_ERR_TIMEOUT);
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+      __syncwarp();
+      if (slice == 0) bwd_put_dx<CF, GI>(gx + size_t(n) * xrow, dx, C, cb, scale, seg == 0);
+      if (chain != nullptr) {
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(chain), "r"(pos + 1) : "memory");
+      }
+    } else if (chain != nullptr && lane == 0) {
+      asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(chain), "r"(pos + 1) : "memory");
     }
   }
-  bwd_end_turn(a, n, GI);
+  bwd_end_turn(a, u, GI);
 }
 
 // All path groups in one launch: every CTA draws a ticket; tickets are group-major (all units
@@ -1414,8 +1522,17 @@ __global__ void __launch_bounds__(32, bwd_min_blocks<CF>()) bwd_kernel(const __g
   if (threadIdx.x == 0) t = atomicAdd(a.ticket, 1);
   t = __shfl_sync(0xffffffffu, t, 0);
   const int g = int(t / a.units);
-  const int64_t n = t % a.units;
-  dispatch<CF::G>(g, [&](auto gc) { bwd_group<CF, decltype(gc)::value, CONV, CC>(a, n, smem); });
+  const int64_t u = t % a.units;
+  if constexpr (CONV) {
+    const int4 inf = a.uinfo[u];  // {sender, first edge, end edge, segment}; in bounds for u < units
+    const int64_t nseg = a.unseg[u];
+    if (u >= *a.n_units) return;  // the grid covers an upper bound of the units
+    dispatch<CF::G>(g, [&](auto gc) {
+      bwd_group<CF, decltype(gc)::value, CONV, CC>(a, u, inf.x, inf.y, inf.z, inf.w, nseg, smem);
+    });
+  } else {
+    dispatch<CF::G>(g, [&](auto gc) { bwd_group<CF, decltype(gc)::value, CONV, CC>(a, u, u, 0, 0, 0, 1, smem); });
+  }
 }
 
 // =================================================================== host launchers ===
@@ -1456,7 +1573,20 @@ e3_status launch_fwd_cc(const e3_plan* plan, const FwdArgs& h, bool conv) {
   if (smem > size_t(227) * 1024) return fail(E3_ERR_UNSUPPORTED, "forward needs %zu bytes of shared memory", smem);
   int64_t units;
   if (conv) {
-    units = h.n_rows;
+    // receiver units from the topology buffer; zeroed ticket and progress counters
+    const TopoPart T = topo_dst(h.n_rows, h.n_edges);
+    const ConvCounters Cn = conv_counters(h.n_rows, h.n_edges, CF::G);
+    const unsigned char* topo = static_cast<const unsigned char*>(h.topo);
+    unsigned char* ws = static_cast<unsigned char*>(h.workspace);
+    a.ticket = reinterpret_cast<int*>(ws);
+    a.flags = reinterpret_cast<int*>(ws + Cn.flags);
+    a.uinfo = reinterpret_cast<const int4*>(topo + T.info);
+    a.unseg = reinterpret_cast<const int32_t*>(topo + T.nseg);
+    a.n_units = reinterpret_cast<const int32_t*>(topo + T.units);
+    a.units_max = seg_units_max(h.n_rows, h.n_edges);
+    cudaError_t e2 = cudaMemsetAsync(ws, 0, Cn.chain, static_cast<cudaStream_t>(h.stream));
+    if (e2 != cudaSuccess) return fail(E3_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e2));
+    units = a.units_max;
     a.n_chunks = 0;
   } else {
     const int64_t n_units = (h.n_rows + NS - 1) / NS;
@@ -1512,24 +1642,38 @@ e3_status launch_bwd_cc(const e3_plan* plan, const BwdArgs& h, bool conv) {
   if (CB > 32) return fail(E3_ERR_UNSUPPORTED, "the backward kernels need a multiplicity of at most 128");
   const int NS = 32 / CB;
   int64_t units;
+  const cudaStream_t s = static_cast<cudaStream_t>(h.stream);
+  unsigned char* ws = static_cast<unsigned char*>(h.workspace);
+  cudaError_t err = cudaSuccess;
   if (conv) {
-    units = h.n_nodes;
+    // units are sender segments of the topology buffer; zeroed ticket and counters
+    const TopoPart T = topo_src(h.n_nodes, h.n_edges);
+    const ConvCounters Cn = conv_counters(h.n_nodes, h.n_edges, CF::G);
+    const unsigned char* topo = static_cast<const unsigned char*>(h.topo);
+    units = seg_units_max(h.n_nodes, h.n_edges);
     a.n_chunks = 0;
+    a.ticket = reinterpret_cast<int*>(ws);
+    a.done = reinterpret_cast<int*>(ws + Cn.flags);
+    a.chain = reinterpret_cast<int*>(ws + Cn.chain);
+    a.uinfo = reinterpret_cast<const int4*>(topo + T.info);
+    a.unseg = reinterpret_cast<const int32_t*>(topo + T.nseg);
+    a.n_units = reinterpret_cast<const int32_t*>(topo + T.units);
+    err = cudaMemsetAsync(ws, 0, Cn.total, s);
+    if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
   } else {
     const int64_t n_units = (h.n_nodes + NS - 1) / NS;
     units = std::min<int64_t>(n_units, int64_t(sm_count()) * 16);
     a.n_chunks = int(units);
+    if (units == 0) return E3_OK;
+    if (h.workspace_bytes < backward_workspace_bytes(units)) return fail(E3_ERR_INVALID_ARG, "workspace too small");
+    a.ticket = reinterpret_cast<int*>(ws);
+    a.done = reinterpret_cast<int*>(ws + 16);
+    err = cudaMemsetAsync(ws, 0, 16 + 4 * size_t(units), s);
+    if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
   }
-  if (units == 0) return E3_OK;
   const int64_t blocks = units * CF::G;
   if (blocks >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "grid too large");
-  if (h.workspace_bytes < backward_workspace_bytes(units)) return fail(E3_ERR_INVALID_ARG, "workspace too small");
   a.units = units;
-  a.ticket = static_cast<int*>(h.workspace);
-  a.done = reinterpret_cast<int*>(static_cast<unsigned char*>(h.workspace) + 16);
-  const cudaStream_t s = static_cast<cudaStream_t>(h.stream);
-  cudaError_t err = cudaMemsetAsync(h.workspace, 0, 16 + 4 * size_t(units), s);
-  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
 
   auto kern = conv ? bwd_kernel<CF, true, CC> : bwd_kernel<CF, false, CC>;
   cudaFuncAttributes fa{};

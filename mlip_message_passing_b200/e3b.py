@@ -27,7 +27,8 @@ SYMBOLS = [
     "e3_spherical_harmonics", "e3_csr_workspace_size", "e3_csr_build", "e3_gather_rows",
     "e3_conv_forward", "e3_conv_backward", "e3_last_error", "e3_csr_build_static",
     "e3_backward_workspace_size", "e3_spherical_harmonics_backward", "e3_morton_workspace_size",
-    "e3_morton_order", "e3_invert_permutation", "e3_remap_ids",
+    "e3_morton_order", "e3_invert_permutation", "e3_remap_ids", "e3_conv_workspace_size",
+    "e3_conv_topology_size", "e3_conv_topology_build",
 ]
 
 
@@ -68,9 +69,13 @@ def _load():
         "e3_csr_build": [I64, I64, VP, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP],
         "e3_csr_build_static": [I64, I64, VP, VP, VP, VP, VP, VP, VP],
         "e3_gather_rows": [I64, I64, I64, VP, VP, VP, VP],
-        "e3_conv_forward": [VP, I64, I64, VP, VP, VP, VP, VP, ctypes.c_int, VP, D, VP, VP],
+        "e3_conv_forward": [VP, I64, I64, VP, VP, VP, VP, VP, ctypes.c_int, VP, D, VP, VP, VP, ctypes.c_size_t,
+                            VP],
+        "e3_conv_workspace_size": [VP, I64, I64, ctypes.POINTER(ctypes.c_size_t)],
+        "e3_conv_topology_size": [I64, I64, ctypes.POINTER(ctypes.c_size_t)],
+        "e3_conv_topology_build": [I64, I64, VP, VP, VP, ctypes.c_size_t, VP],
         "e3_conv_backward": [VP, I64, I64, VP, VP, VP, VP, VP, VP, VP, VP, ctypes.c_int, VP, VP, D, VP, VP, VP,
-                             VP, ctypes.c_size_t, VP],
+                             VP, VP, ctypes.c_size_t, VP],
         "e3_morton_workspace_size": [I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_morton_order": [I64, VP, ctypes.c_int, ctypes.POINTER(D), ctypes.POINTER(D), VP, VP, ctypes.c_size_t,
                             VP],
@@ -233,6 +238,13 @@ def tp_backward(plan, x, y, w, grad_out, need_x=True, need_y=True, need_w=True):
     return gx, gy, gw
 
 
+def conv_workspace(plan, n_nodes, n_edges, device):
+    """Device workspace for e3_conv_forward / e3_conv_backward, from torch's allocator."""
+    nbytes = ctypes.c_size_t()
+    _check(lib.e3_conv_workspace_size(plan.handle, n_nodes, n_edges, ctypes.byref(nbytes)))
+    return torch.empty(nbytes.value, dtype=torch.uint8, device=device)
+
+
 def backward_workspace(n, device):
     """Device workspace for e3_tp_backward (n = B) / e3_conv_backward (n = N), from torch's allocator."""
     nbytes = ctypes.c_size_t()
@@ -373,6 +385,12 @@ class Graph:
         self.perm_dst, self.row_ptr_dst, self.perm_src, self.row_ptr_src = csr_build(self.n_nodes, src, dst)
         self.src = gather_rows(self.perm_dst, src)
         self.dst = gather_rows(self.perm_dst, dst)
+        # the convolution's work units (rows cut into segments), built once for the topology
+        nbytes = ctypes.c_size_t()
+        _check(lib.e3_conv_topology_size(self.n_nodes, self.n_edges, ctypes.byref(nbytes)))
+        self.topo = torch.empty(nbytes.value, dtype=torch.uint8, device=src.device)
+        _check(lib.e3_conv_topology_build(self.n_nodes, self.n_edges, _ptr(self.row_ptr_dst), _ptr(self.row_ptr_src),
+                                          _ptr(self.topo), self.topo.numel(), _stream()))
 
     def to_receiver_order(self, t):
         return gather_rows(self.perm_dst, t.contiguous())
@@ -394,9 +412,10 @@ def conv_forward(plan, graph, x, w, y=None, edge_vec=None, sh_norm="component", 
     if out is None:
         out = torch.empty((N, plan.dim_out), dtype=dt, device=dev)
     _need(out, "out", dt, (N, plan.dim_out), dev)
+    ws = conv_workspace(plan, N, E, dev)
     _check(lib.e3_conv_forward(plan.handle, N, E, _ptr(graph.row_ptr_dst), _ptr(graph.src), _ptr(x), _ptr(y),
                                _ptr(edge_vec), _SH_NORMS[sh_norm], _ptr(w), float(out_scale), _ptr(out),
-                               _stream()))
+                               _ptr(graph.topo), _ptr(ws), ws.numel(), _stream()))
     return out
 
 
@@ -417,11 +436,11 @@ def conv_backward(plan, graph, x, w, grad_out, y=None, edge_vec=None, sh_norm="c
     gx = torch.empty_like(x) if need_x else None
     gy = torch.empty((E, plan.dim_in2), dtype=dt, device=dev) if need_y else None
     gw = torch.empty_like(w) if need_w else None
-    ws = backward_workspace(N, dev)
+    ws = conv_workspace(plan, N, E, dev)
     _check(lib.e3_conv_backward(plan.handle, N, E, _ptr(graph.row_ptr_dst), _ptr(graph.src), _ptr(graph.dst),
                                 _ptr(graph.row_ptr_src), _ptr(graph.perm_src), _ptr(x), _ptr(y), _ptr(edge_vec),
                                 _SH_NORMS[sh_norm], _ptr(w), _ptr(grad_out), float(out_scale), _ptr(gx),
-                                _ptr(gy), _ptr(gw), _ptr(ws), ws.numel(), _stream()))
+                                _ptr(gy), _ptr(gw), _ptr(graph.topo), _ptr(ws), ws.numel(), _stream()))
     return gx, gy, gw
 
 

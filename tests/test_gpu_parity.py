@@ -370,6 +370,40 @@ def test_conv_with_padding_edges(e3b):
     e3b.device_status()
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+def test_conv_hubs_split_into_segments(e3b, dtype):
+    """A receiver with 5000 in-edges and a sender with 5000 out-edges (20 row segments each, added
+    in order by separate CTAs) beside ordinary nodes: forward and backward against the oracle,
+    bitwise equal on a second run."""
+    rng = np.random.default_rng(90)
+    n, mul, lx, ly, lo = 300, 32, 2, 3, 2
+    src = np.concatenate([rng.integers(0, n, 6000), rng.integers(0, n, 5000), np.full(5000, 11)]).astype(np.int32)
+    dst = np.concatenate([rng.integers(0, n, 6000), np.full(5000, 7), rng.integers(0, n, 5000)]).astype(np.int32)
+    E = len(src)
+    p, q = gplan(e3b, mul, lx, ly, lo, dtype), oplan(mul, lx, ly, lo)
+    vec = rng.standard_normal((E, 3))
+    x = rng.standard_normal((n, p.dim_in1))
+    w = rng.standard_normal((E, p.weight_numel)) / 8
+    go = rng.standard_normal((n, p.dim_out))
+    graph = e3b.Graph(n, t(src), t(dst))
+    args = (t(x, dtype), graph.to_receiver_order(t(w, dtype)))
+    kw = dict(edge_vec=graph.to_receiver_order(t(vec, dtype)), out_scale=0.3)
+    out = e3b.conv_forward(p, graph, *args, **kw)
+    gx, gy, gw = e3b.conv_backward(p, graph, *args, t(go, dtype), **kw)
+    Y = oracle.real_sh_all(ly, vec)
+    ref = oracle.conv_forward(q, n, src, dst, x, Y, w, 0.3)
+    rx, ry, rw = oracle.conv_backward(q, n, src, dst, x, Y, w, go, 0.3)
+    perm = graph.perm_dst.cpu().numpy()
+    assert rel_err(h(out), ref) <= TOL[dtype]
+    assert rel_err(h(gx), rx) <= TOL[dtype]
+    assert rel_err(h(gy), ry[perm]) <= TOL[dtype]
+    assert rel_err(h(gw), rw[perm]) <= TOL[dtype]
+    out2 = e3b.conv_forward(p, graph, *args, **kw)
+    gx2, gy2, gw2 = e3b.conv_backward(p, graph, *args, t(go, dtype), **kw)
+    assert torch.equal(out, out2) and torch.equal(gx, gx2) and torch.equal(gy, gy2) and torch.equal(gw, gw2)
+    e3b.device_status()
+
+
 def test_conv_edge_cases(e3b):
     p = gplan(e3b, 8, 1, 2, 2, torch.float32)
     q = oplan(8, 1, 2, 2)
@@ -408,13 +442,13 @@ def test_backward_workspace_is_checked(e3b):
     go = torch.randn(n, p.dim_out, device=DEV)
     vec = torch.randn(4, 3, device=DEV)
     gx = torch.empty_like(x)
-    ws = e3b.backward_workspace(n, DEV)
+    ws = e3b.conv_workspace(p, n, 4, DEV)
     P = e3b._ptr
 
     def call(wsp, nbytes):
         return e3b.lib.e3_conv_backward(p.handle, n, 4, P(graph.row_ptr_dst), P(graph.src), P(graph.dst),
                                         P(graph.row_ptr_src), P(graph.perm_src), P(x), None, P(vec), 0, P(w),
-                                        P(go), 1.0, P(gx), None, None, wsp, nbytes, e3b._stream())
+                                        P(go), 1.0, P(gx), None, None, P(graph.topo), wsp, nbytes, e3b._stream())
 
     assert call(None, ws.numel()) == e3b.E3_ERR_INVALID_ARG
     assert call(P(ws[8:]), ws.numel() - 8) == e3b.E3_ERR_INVALID_ARG
