@@ -17,14 +17,18 @@
 //   * Channels are the fastest thread index; when C/4 < 32 the remaining lanes of a warp take
 //     different edges of the same receiver ("slices") and are summed with a fixed butterfly at
 //     the end, so the reduction order is fixed and the result is bitwise repeatable.
-//   * Forward: one CTA per (receiver, path group); the receiver's in-edges are consecutive in
-//     memory (receiver CSR), so the weight rows stream contiguously and x[src] rows are
-//     gathered from L2.  No atomics, no [E, dim_out] message tensor.
-//   * Backward: one one-warp CTA per (sender, path group), walking the sender CSR; A is
-//     recomputed, never stored; grad_w and grad_y are edge-local writes; grad_x is reduced in
-//     registers in a fixed order.  All groups run in one launch; the groups of one sender
-//     are ordered by a per-sender progress counter (the first group to touch a grad_x or
-//     grad_y block stores it, later groups add), so no floating-point atomics are used.
+//   * Forward: one CTA per (receiver segment, path group); the receiver's in-edges are
+//     consecutive in memory (receiver CSR), so the weight rows stream contiguously and x[src]
+//     rows are gathered from L2.  No floating-point atomics, no [E, dim_out] message tensor.
+//   * Backward: one one-warp CTA per (sender segment, path group), walking the sender CSR; A
+//     is recomputed, never stored; grad_w and grad_y are edge-local writes; grad_x is reduced
+//     in registers in a fixed order.  All groups run in one launch; the groups of one unit are
+//     ordered by a progress counter (the first group to touch a grad_x or grad_y block stores
+//     it, later groups add).
+//   * A row (a receiver's in-edges, a sender's out-edges) of more than SEG_EDGES edges is cut
+//     into segments, each its own unit, so a hub does not serialise on one CTA; the segments'
+//     partial sums join the row in segment order through progress counters.  CTAs take tickets
+//     in start order, and every wait is on a CTA with an earlier ticket: no deadlock.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -216,18 +220,6 @@ __device__ __forceinline__ void load_x(T (&xr)[K][GR::NXG], const T* __restrict_
 #pragma unroll
       for (int m = 0; m < D; ++m) xr[k][L * L - GR::XB + m] = t[k * D + m];
   });
-}
-
-// weights of the group's paths for channels 4cb..4cb+3: wr[k][q] = w[row, PB + q, 4cb + k]
-template <class GR, typename T>
-__device__ __forceinline__ void load_w(T (&wr)[K][GR::NP], const T* __restrict__ wrow, int C, int cb) {
-#pragma unroll
-  for (int q = 0; q < GR::NP; ++q) {
-    T t[K];
-    ld16(t, wrow + size_t(GR::PB + q) * C + 4 * cb, true);
-#pragma unroll
-    for (int k = 0; k < K; ++k) wr[k][q] = t[k];
-  }
 }
 
 // ------------------------------------------------------------ spherical harmonics ---

@@ -117,3 +117,15 @@ def test_backward_workspace_size(e3b):
     assert e3b.lib.e3_backward_workspace_size(-1, ctypes.byref(n)) == e3b.E3_ERR_SHAPE
     assert e3b.lib.e3_backward_workspace_size(1 << 31, ctypes.byref(n)) == e3b.E3_ERR_SHAPE
     assert e3b.lib.e3_backward_workspace_size(5, None) == e3b.E3_ERR_INVALID_ARG
+
+
+def test_conv_topology_and_workspace_sizes(e3b):
+    n = ctypes.c_size_t()
+    assert e3b.lib.e3_conv_topology_size(3000, 156278, ctypes.byref(n)) == e3b.E3_OK
+    # two directions, each: units (N + E/256 + 1) x (16 + 4 bytes) + row offsets (N + 1) x 4 bytes
+    units = 3000 + 156278 // 256 + 1
+    assert n.value >= 2 * (20 * units + 4 * 3001) and n.value % 256 == 0
+    assert e3b.lib.e3_conv_topology_size(-1, 5, ctypes.byref(n)) == e3b.E3_ERR_SHAPE
+    assert e3b.lib.e3_conv_topology_size(5, 5, None) == e3b.E3_ERR_INVALID_ARG
+    assert e3b.lib.e3_conv_topology_build(4, 4, None, None, None, 0, None) == e3b.E3_ERR_INVALID_ARG
+    assert e3b.lib.e3_conv_workspace_size(None, 5, 5, ctypes.byref(n)) == e3b.E3_ERR_INVALID_ARG
