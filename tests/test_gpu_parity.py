@@ -404,6 +404,22 @@ def test_conv_hubs_split_into_segments(e3b, dtype):
     e3b.device_status()
 
 
+def test_conv_forward_multiplicity_256(e3b):
+    """C = 256: two warps per forward CTA (64 lanes of 4 channels) on a small box; the backward
+    reports the multiplicity as unsupported."""
+    n, mul, lx, ly, lo = 400, 256, 1, 2, 2
+    g = W.graph_inputs(n, mul, lx, ly, lo, 14, dtype=np.float32)
+    graph = e3b.Graph(n, t(g["src"]), t(g["dst"]))
+    p, q = gplan(e3b, mul, lx, ly, lo, torch.float32), oplan(mul, lx, ly, lo)
+    vec, wr = graph.to_receiver_order(t(g["vec"])), graph.to_receiver_order(t(g["w"]))
+    out = e3b.conv_forward(p, graph, t(g["x"]), wr, edge_vec=vec, out_scale=0.2)
+    Y = oracle.real_sh_all(ly, g["vec"].astype(np.float64))
+    assert rel_err(h(out), oracle.conv_forward(q, n, g["src"], g["dst"], g["x"], Y, g["w"], 0.2)) <= 1e-5
+    with pytest.raises(e3b.E3Error) as ei:
+        e3b.conv_backward(p, graph, t(g["x"]), wr, torch.zeros_like(out), edge_vec=vec, out_scale=0.2)
+    assert ei.value.status == e3b.E3_ERR_UNSUPPORTED
+
+
 def test_conv_edge_cases(e3b):
     p = gplan(e3b, 8, 1, 2, 2, torch.float32)
     q = oplan(8, 1, 2, 2)
