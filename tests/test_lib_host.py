@@ -129,3 +129,20 @@ def test_conv_topology_and_workspace_sizes(e3b):
     assert e3b.lib.e3_conv_topology_size(5, 5, None) == e3b.E3_ERR_INVALID_ARG
     assert e3b.lib.e3_conv_topology_build(4, 4, None, None, None, 0, None) == e3b.E3_ERR_INVALID_ARG
     assert e3b.lib.e3_conv_workspace_size(None, 5, 5, ctypes.byref(n)) == e3b.E3_ERR_INVALID_ARG
+
+
+def test_c_abi_from_plain_c(e3b, tmp_path):
+    """The header compiles as C (gcc, -std=c11), the library links, host-only calls answer."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    exe = tmp_path / "abi_host"
+    src = os.path.join(ROOT, "tests", "c", "abi_host.c")
+    lib_dir = os.path.dirname(e3b.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), src, "-o", str(exe),
+                        "-L", lib_dir, "-l:libe3b.so", "-Wl,-rpath," + lib_dir, "-lm"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "FAIL" not in r.stdout
