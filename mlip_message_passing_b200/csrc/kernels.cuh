@@ -946,8 +946,10 @@ struct BwdSmem {
 
 // Per-edge backward of one path group with grad_out read from shared memory (sg: the group's
 // outputs, channels in mul_ir order).  Accumulates alpha_p w t into dx, returns this thread's
-// unreduced grad_y contribution in dY and writes grad_w (scaled) when gw != nullptr.
-template <class CF, int GI>
+// unreduced grad_y contribution in dY and writes grad_w (scaled) when gw != nullptr.  FL = 1:
+// grad_w and grad_y are both requested, known at compile time, so that no per-path test
+// separates one path's work from the next in the schedule.
+template <class CF, int GI, int FL>
 __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, GI>::NXG],
                                          const typename CF::T* sw,
                                          const typename CF::T (&Y)[CF::NY], const typename CF::T* sg,
@@ -998,7 +1000,7 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
           if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) t[k][M1I] = fma(a[M1I], g[k][M3I], t[k][M1I]);
         });
     });
-    if (gw != nullptr) {  // grad_w[e, p, u] = scale alpha_p sum_m1 x[u, m1] t[u, m1]
+    if (FL == 1 || gw != nullptr) {  // grad_w[e, p, u] = scale alpha_p sum_m1 x[u, m1] t[u, m1]
       T o[K];
 #pragma unroll
       for (int k = 0; k < K; ++k) {
@@ -1013,7 +1015,7 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
     for (int k = 0; k < K; ++k)  // grad_x += alpha_p w t
 #pragma unroll
       for (int m1 = 0; m1 < D1; ++m1) dx[k][XO + m1] = fma(wa[k], t[k][m1], dx[k][XO + m1]);
-    if (want_dy) {  // grad_y[m2] += sum_{m1,m3} C[m1,m2,m3] sum_k alpha_p w_k x_k[m1] g_k[m3]
+    if (FL == 1 || want_dy) {  // grad_y[m2] += sum_{m1,m3} C[m1,m2,m3] sum_k alpha_p w_k x_k[m1] g_k[m3]
       // the weight scales the shorter of the x and grad_out blocks
       constexpr bool SX = D1 <= D3;
       T xw[K][SX ? D1 : 1], gw_[K][SX ? 1 : D3];
@@ -1228,7 +1230,8 @@ __device__ __forceinline__ void bwd_end_turn(const KBwd& a, int64_t unit, int gi
 
 // Backward of path group GI for one unit.  Convolution: one CTA (one warp) per sender,
 // walking its out-edges through the sender CSR; tensor product: one CTA per sample range.
-template <class CF, int GI, bool CONV, int CC>
+// FL = 1: grad_w and grad_y are both non-null (the caller checked).
+template <class CF, int GI, bool CONV, int CC, int FL>
 __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const int64_t n, const int64_t j0_in,
                                           const int64_t j1_in, const int64_t seg, const int64_t nseg,
                                           unsigned char* smem) {
@@ -1252,7 +1255,7 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const 
   T* __restrict__ gwp = static_cast<T*>(a.grad_w);
   const size_t xrow = size_t(CF::NX) * C, orow = size_t(CF::NO) * C, wrow = size_t(CF::P) * C;
   const T scale = T(a.scale);
-  const bool want_dy = gy != nullptr;
+  const bool want_dy = FL == 1 || gy != nullptr;
   const uint32_t WB = BwdSlice<CF, GI>::wbytes(C), GB = BwdSlice<CF, GI>::gbytes(C);
   const uint32_t XB = BwdSlice<CF, GI>::xbytes(C, CONV), YB = BwdSlice<CF, GI>::ybytes(want_dy);
   const uint32_t SLOT = WB + GB + XB + YB;
@@ -1391,7 +1394,8 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const 
 #pragma unroll
           for (int m = 0; m < CF::NY; ++m) Y[m] = yp[m];
         }
-        bwd_edge<CF, GI>(xr, sl, Y, sl + WB / sizeof(T), dx, dY, want_dy, gwp ? gwp + e * wrow : nullptr, C, cb,
+        bwd_edge<CF, GI, FL>(xr, sl, Y, sl + WB / sizeof(T), dx, dY, want_dy,
+                             (FL == 1 || gwp) ? gwp + e * wrow : nullptr, C, cb,
                          a.alpha, a.alpha_f, scale);
       } else {
 #pragma unroll
@@ -1519,11 +1523,18 @@ __global__ void __launch_bounds__(32, bwd_min_blocks<CF>()) bwd_kernel(const __g
     const int4 inf = a.uinfo[u];  // {sender, first edge, end edge, segment}; in bounds for u < units
     const int64_t nseg = a.unseg[u];
     if (u >= *a.n_units) return;  // the grid covers an upper bound of the units
-    dispatch<CF::G>(g, [&](auto gc) {
-      bwd_group<CF, decltype(gc)::value, CONV, CC>(a, u, inf.x, inf.y, inf.z, inf.w, nseg, smem);
-    });
+    // the specialised multiplicities carry a copy with every gradient requested
+    if (CC > 0 && a.grad_w != nullptr && a.grad_y != nullptr) {
+      dispatch<CF::G>(g, [&](auto gc) {
+        bwd_group<CF, decltype(gc)::value, CONV, CC, (CC > 0 ? 1 : 0)>(a, u, inf.x, inf.y, inf.z, inf.w, nseg, smem);
+      });
+    } else {
+      dispatch<CF::G>(g, [&](auto gc) {
+        bwd_group<CF, decltype(gc)::value, CONV, CC, 0>(a, u, inf.x, inf.y, inf.z, inf.w, nseg, smem);
+      });
+    }
   } else {
-    dispatch<CF::G>(g, [&](auto gc) { bwd_group<CF, decltype(gc)::value, CONV, CC>(a, u, u, 0, 0, 0, 1, smem); });
+    dispatch<CF::G>(g, [&](auto gc) { bwd_group<CF, decltype(gc)::value, CONV, CC, 0>(a, u, u, 0, 0, 0, 1, smem); });
   }
 }
 
