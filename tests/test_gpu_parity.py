@@ -226,6 +226,31 @@ def test_conv_forward_backward_full(e3b, dtype, mode):
     assert rel_err(h(gw), rw[perm]) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("mul", [64, 128])
+def test_conv_backward_gradient_subsets(e3b, mul):
+    """Multiplicities 64 and 128 run a separately compiled backward when grad_w and grad_y are
+    both requested; every other subset runs the general one.  Each subset against the oracle."""
+    n, lx, ly, lo = 400, 2, 3, 2
+    g, graph, w = conv_setup(e3b, n, mul, lx, ly, lo, 23, torch.float32)
+    p, q = gplan(e3b, mul, lx, ly, lo, torch.float32), oplan(mul, lx, ly, lo)
+    Y = oracle.real_sh_all(ly, g["vec"].astype(np.float64))
+    vec = graph.to_receiver_order(t(g["vec"]))
+    wr = graph.to_receiver_order(w)
+    go = W.grad_out(n, q.irreps_out.dim, 9)
+    s = 1 / math.sqrt(52)
+    rx, ry, rw = oracle.conv_backward(q, n, g["src"], g["dst"], g["x"], Y, g["w"], go, s)
+    perm = graph.perm_dst.cpu().numpy()
+    ref = (rx, ry[perm], rw[perm])
+    for need in [(1, 1, 1), (1, 0, 0), (0, 1, 0), (0, 0, 1), (1, 0, 1), (1, 1, 0), (0, 1, 1)]:
+        res = e3b.conv_backward(p, graph, t(g["x"]), wr, t(go), edge_vec=vec, out_scale=s,
+                                need_x=bool(need[0]), need_y=bool(need[1]), need_w=bool(need[2]))
+        for i in range(3):
+            if need[i]:
+                assert rel_err(h(res[i]), ref[i]) <= 1e-5, (need, i)
+            else:
+                assert res[i] is None, (need, i)
+
+
 def test_conv_small_multiplicity_and_degrees(e3b):
     # C = 8 (16 edge slices per warp) on the (1, 2, 2) path set and C = 4 on (1, 1, 2)
     for mul, lx, ly, lo in [(8, 1, 2, 2), (4, 1, 1, 2), (32, 2, 3, 2)]:
