@@ -894,7 +894,7 @@ __host__ __device__ constexpr bool group_has_l2(int l) {
   return false;
 }
 
-constexpr int BWD_WIN = 32;  // out-edges whose ids and harmonics are staged at once
+constexpr int BWD_WIN = 64;  // out-edges whose ids and harmonics are staged at once (a typical sender in one window)
 
 // A group that adds to grad_y blocks an earlier group stored stages the edge's grad_y row with
 // its other slices, so the read-modify-write does not wait on a global load (rows whose byte
