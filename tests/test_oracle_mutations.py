@@ -197,3 +197,46 @@ def test_morton_axes_swapped(monkeypatch):
     monkeypatch.setattr(ore, "morton_order", bad_order)
     monkeypatch.setattr(oracle, "morton_order", bad_order)
     assert _caught([pins.test_morton_order_equals_octree_order, pins.test_morton_codes_known_cells_and_clamping])
+
+
+ALPHA_PINS = [lambda: pins.test_default_path_weight_gives_unit_second_moment("uncollapsed"),
+              lambda: pins.test_default_path_weight_gives_unit_second_moment("collapsed"),
+              lambda: pins.test_default_path_weight_gives_unit_second_moment("mul_y2"),
+              pins.test_default_path_weight_unit_moment_over_the_sphere,
+              pins.test_default_path_weight_closed_forms_1x1]
+
+
+def _patch_alpha(monkeypatch, formula):
+    """Recompute every default path weight of the plans make_plan builds with another formula
+    of (l3, mul_y, n_out)."""
+    orig = otp.make_plan
+
+    def bad(*args, **kwargs):
+        plan = orig(*args, **kwargs)
+        n_out = {}
+        for ins in plan.instructions:
+            n_out[ins.i_out] = n_out.get(ins.i_out, 0) + 1
+        plan.alphas = [formula(plan.irreps_out[ins.i_out].l, plan.irreps_in2[ins.i_in2].mul, n_out[ins.i_out])
+                       if ins.path_weight < 0 else a for ins, a in zip(plan.instructions, plan.alphas)]
+        return plan
+
+    monkeypatch.setattr(otp, "make_plan", bad)
+    monkeypatch.setattr(oracle, "make_plan", bad)
+
+
+@pytest.mark.parametrize("name,formula", [
+    ("inverted", lambda l3, mv, no: np.sqrt(1.0 / ((2 * l3 + 1) * mv * no))),
+    ("no_n_out", lambda l3, mv, no: np.sqrt((2 * l3 + 1) / mv)),
+    ("no_mul_y", lambda l3, mv, no: np.sqrt((2 * l3 + 1) / no)),
+    ("dimension_not_sqrt", lambda l3, mv, no: (2 * l3 + 1) / (mv * no)),
+    ("l3_plus_one", lambda l3, mv, no: np.sqrt((l3 + 1) / (mv * no))),
+])
+def test_wrong_default_path_weight(monkeypatch, name, formula):
+    _patch_alpha(monkeypatch, formula)
+    assert _caught(ALPHA_PINS)
+
+
+def test_right_default_path_weight_passes(monkeypatch):
+    # the harness itself: the stated formula re-applied leaves every pin green
+    _patch_alpha(monkeypatch, lambda l3, mv, no: np.sqrt((2 * l3 + 1) / (mv * no)))
+    assert not _caught(ALPHA_PINS)

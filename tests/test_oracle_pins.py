@@ -288,6 +288,82 @@ def test_tp_scalar_path():
     np.testing.assert_allclose(oracle.tp_forward(plan, x, y, w), x * y * w, atol=1e-15)
 
 
+def _trilinear_coefficients(plan):
+    """T[k, i, j, q] = out_k for x = e_i, y = e_j, w = e_q (the oracle as a black box).  The
+    tensor product is linear in each input, so these basis evaluations fix it completely."""
+    d1, d2, nw, do = plan.irreps_in1.dim, plan.irreps_in2.dim, plan.weight_numel, plan.irreps_out.dim
+    T = np.zeros((do, d1, d2, nw))
+    eye1, eye2 = np.eye(d1), np.eye(d2)
+    for q in range(nw):
+        wq = np.zeros((d1 * d2, nw))
+        wq[:, q] = 1.0
+        xs = np.repeat(eye1, d2, axis=0)
+        ys = np.tile(eye2, (d1, 1))
+        T[:, :, :, q] = oracle.tp_forward(plan, xs, ys, wq).reshape(d1, d2, do).transpose(2, 0, 1)
+    return T
+
+
+@pytest.mark.parametrize("case", ["uncollapsed", "collapsed", "mul_y2"])
+def test_default_path_weight_gives_unit_second_moment(case):
+    """The default path weight alpha_p is fixed by one property (e3nn course, lesson 03b: paths
+    are normalised so that the output keeps the scale of the inputs): when every component of x,
+    y and w is an independent zero-mean unit-variance variable, every output component has second
+    moment 1.  For a trilinear map out_k = sum T[k,i,j,q] x_i y_j w_q that moment is exactly
+    sum_{ijq} T[k,i,j,q]^2, so the check is exact, with T read off the oracle by basis inputs."""
+    if case == "uncollapsed":
+        plan = oracle.make_plan("1x0e+1x1o+1x2e", "1x0e+1x1o+1x2e+1x3o", lmax_out=3)
+    elif case == "collapsed":  # two paths share each output block: n_out = 2
+        plan = oracle.make_plan("1x1o+1x2o", "1x1o", "1x1e+1x2e",
+                                instructions=[(0, 0, 0), (1, 0, 0), (1, 0, 1)])
+    else:  # uvu with two channels of y: sum over v with a weight per (u, v)
+        plan = oracle.make_plan("2x1o", "2x1o+2x2e", "2x0e+2x1e+2x2o+2x3o",
+                                instructions=[(0, 0, 0), (0, 0, 1), (0, 1, 2), (0, 1, 3)])
+    T = _trilinear_coefficients(plan)
+    moment = (T * T).sum(axis=(1, 2, 3))
+    np.testing.assert_allclose(moment, 1.0, rtol=1e-12)
+
+
+def test_default_path_weight_unit_moment_over_the_sphere():
+    """The same property with y the component-normalised harmonics of a direction uniform on the
+    sphere (the convolution's input), averaged exactly by a product quadrature (Gauss-Legendre in
+    cos(theta) times equally spaced phi; exact for the degree-6 polynomials Y_m Y_m' with l <= 3),
+    and x, w independent N(0, 1), whose average is again the sum of squares of the coefficients."""
+    plan = oracle.make_plan("1x0e+1x1o+1x2e+1x3o", "1x0e+1x1o+1x2e+1x3o", lmax_out=3)
+    t, tw = np.polynomial.legendre.leggauss(6)
+    phi = np.arange(12) * (2 * np.pi / 12)
+    st = np.sqrt(1 - t * t)
+    dirs = np.stack([np.outer(st, np.cos(phi)).ravel(), np.outer(st, np.sin(phi)).ravel(),
+                     np.repeat(t, phi.size)], 1)
+    qw = np.repeat(tw, phi.size) / (2 * phi.size)  # weights sum to 1: the average over the sphere
+    Y = real_sh_all(3, dirs)
+    T = _trilinear_coefficients(plan)  # [k, i, j, q]
+    # out_k(x, w | y) = sum_{i,q} (sum_j T[k,i,j,q] y_j) x_i w_q
+    Ty = np.einsum("kijq,nj->nkiq", T, Y)
+    moment = np.einsum("n,nkiq->k", qw, Ty * Ty)
+    np.testing.assert_allclose(moment, 1.0, rtol=1e-12)
+
+
+def test_default_path_weight_closed_forms_1x1():
+    """1o x 1o with unit weights.  The outer product a b^T splits into its trace part, its
+    antisymmetric part and its symmetric traceless part (e3nn course, lesson 03a: the dot, cross
+    and symmetric traceless products); with the default path weights (1, sqrt(3), sqrt(5)) each
+    output block is an isometric image of one part, so its norm equals that part's Frobenius
+    norm, the three squared norms add up to |a|^2 |b|^2, and the scalar block is a.b/sqrt(3)."""
+    plan = oracle.make_plan("1x1o", "1x1o", lmax_out=2)
+    rng = np.random.default_rng(21)
+    for _ in range(5):
+        a, b = rng.standard_normal(3), rng.standard_normal(3)
+        out = oracle.tp_forward(plan, a[None], b[None], np.ones((1, 3)))[0]
+        M = np.outer(a, b)
+        tr = np.trace(M) / 3 * np.eye(3)
+        anti = 0.5 * (M - M.T)
+        sym = 0.5 * (M + M.T) - tr
+        assert abs(out[0] - a @ b / math.sqrt(3)) < 1e-14
+        assert abs(np.linalg.norm(out[1:4]) - np.linalg.norm(anti)) < 1e-14
+        assert abs(np.linalg.norm(out[4:9]) - np.linalg.norm(sym)) < 1e-14
+        assert abs(out @ out - (a @ a) * (b @ b)) < 1e-12
+
+
 def test_default_path_enumeration_counts():
     p0 = oracle.make_plan("8x0e+8x1o", "1x0e+1x1o+1x2e", lmax_out=2)
     assert [(plan_l(p0, i)) for i in range(p0.n_paths)] == [
