@@ -306,7 +306,8 @@ E3_API e3_status e3_conv_forward(const e3_plan* plan, int64_t N, int64_t E, cons
  * get zero grad_y and grad_w rows.  Senders with more than 256 out-edges are split into
  * 256-edge segments like the forward's rows.  topo and workspace: as for e3_conv_forward.  No atomics on the gradients: the path groups of
  * a sender run in a fixed order, so results are bitwise repeatable.  A group that waits for
- * its predecessor longer than about a second records E3_ERR_TIMEOUT.  Shared weights are not
+ * its predecessor longer than the wait limit (one second; e3_set_test_knobs) records
+ * E3_ERR_TIMEOUT.  Shared weights are not
  * supported. */
 E3_API e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E, const int32_t* row_ptr_dst,
                            const int32_t* src, const int32_t* dst, const int32_t* row_ptr_src,
@@ -315,6 +316,20 @@ E3_API e3_status e3_conv_backward(const e3_plan* plan, int64_t N, int64_t E, con
                            const void* grad_out, double out_scale, void* grad_x, void* grad_y,
                            void* grad_w, const void* topo, void* workspace, size_t workspace_bytes,
                            void* stream);
+
+/* No counterpart in the paper: failure-detection hooks for tests.  Every later convolution and
+ * tensor-product launch in this process uses these values:
+ *   wait_limit_ns  limit of every bounded device wait (a copy completion, a path group waiting
+ *                  for its predecessor, a row segment waiting for the earlier ones); after it the
+ *                  kernel records E3_ERR_TIMEOUT, stops waiting and returns normally.  0 restores
+ *                  the default of one second.
+ *   first_ticket   first ticket the ticketed kernels draw (default 0).  Raising it to k withholds
+ *                  the first k work items of a launch (group-major order: group 0's units first),
+ *                  so whatever waits for them times out: this is how a test makes a bounded wait
+ *                  run out without faulting anything.  Results are then unspecified.
+ * Process-global; not for concurrent use with production calls.  Negative values return
+ * E3_ERR_INVALID_ARG. */
+E3_API e3_status e3_set_test_knobs(int64_t wait_limit_ns, int32_t first_ticket);
 
 /* Message of the last non-OK status returned on the calling thread ("" if none). */
 E3_API const char* e3_last_error(void);

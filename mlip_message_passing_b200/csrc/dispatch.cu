@@ -2,6 +2,7 @@
 // translation unit compiled for its path set.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 #include <vector>
@@ -59,6 +60,12 @@ e3_status device_status_ptr(int** ptr) {
   return E3_OK;
 }
 
+static std::atomic<long long> g_wait_limit_ns{1000000000ll};
+static std::atomic<int> g_first_ticket{0};
+
+unsigned long long test_wait_limit_ns() { return static_cast<unsigned long long>(g_wait_limit_ns.load()); }
+int test_first_ticket() { return g_first_ticket.load(); }
+
 int sm_count() {
   int dev = 0;
   cudaGetDevice(&dev);
@@ -83,3 +90,11 @@ e3_status launch_backward(const e3_plan* plan, const BwdArgs& a, bool conv) {
 }
 
 }  // namespace e3b
+
+extern "C" e3_status e3_set_test_knobs(int64_t wait_limit_ns, int32_t first_ticket) {
+  e3b::clear_error();
+  if (wait_limit_ns < 0 || first_ticket < 0) return e3b::fail(E3_ERR_INVALID_ARG, "negative knob");
+  e3b::g_wait_limit_ns.store(wait_limit_ns == 0 ? 1000000000ll : wait_limit_ns);
+  e3b::g_first_ticket.store(first_ticket);
+  return E3_OK;
+}

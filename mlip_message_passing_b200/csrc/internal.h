@@ -42,6 +42,10 @@ e3_status ensure_device_tables();
 e3_status device_status_ptr(int** ptr);
 // Number of SMs of the current device.
 int sm_count();
+// Limit of every bounded device wait (nanoseconds) and the first ticket the ticketed kernels
+// draw, as set by e3_set_test_knobs (defaults: one second, 0).
+unsigned long long test_wait_limit_ns();
+int test_first_ticket();
 
 // Launchers (dispatch.cu, per path set in tp_conv_l*.cu).  Arguments are validated by the caller.
 struct FwdArgs {

@@ -325,6 +325,8 @@ struct KFwd {
   const int32_t* unseg;
   const int32_t* n_units;
   int64_t units_max;
+  unsigned long long wait_ns;  // limit of every bounded wait
+  int first_ticket;            // first ticket drawn (0; a test withholds tickets by raising it)
   double pscale[MAXP];  // scale * alpha_p
 };
 
@@ -493,11 +495,9 @@ struct FwdAcc {
 // ------------------------------------------------------------ async copy machinery ---
 // One thread per CTA streams the weight and x slices of upcoming edges into a ring of shared
 // memory stages with cp.async.bulk (1-D TMA, no multicast); completion is tracked by one
-// mbarrier per stage (transaction bytes).  Every wait is bounded: after WAIT_NS nanoseconds
-// of the global timer (WAIT_LIMIT polls for the progress counters of the backward) the kernel
-// records E3_ERR_TIMEOUT and stops issuing work.
-constexpr long long WAIT_LIMIT = 1ll << 24;
-constexpr unsigned long long WAIT_NS = 1000000000ull;
+// mbarrier per stage (transaction bytes).  Every wait is bounded: after the launch's wait_ns
+// nanoseconds of the global timer (one second unless a test sets it lower) the kernel records
+// E3_ERR_TIMEOUT and stops issuing work.
 constexpr int FWD_WIN = 64;  // in-edges whose sender ids and harmonics are staged at once
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -546,17 +546,33 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// bounded wait; false after WAIT_NS (the error is recorded).  The common case -- the copy
+// bounded wait; false after wait_ns (the error is recorded).  The common case -- the copy
 // landed while the previous stage was being consumed -- costs one test.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, unsigned long long wait_ns) {
   if (mbar_test_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   do {
     for (int i = 0; i < 16; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-  } while (global_ns() - t0 < WAIT_NS);
+  } while (global_ns() - t0 < wait_ns);
   record_error(status, E3_ERR_TIMEOUT);
   return false;
+}
+
+// Bounded wait (one thread) until *flag >= v (acquire); false after wait_ns nanoseconds of the
+// global timer, with E3_ERR_TIMEOUT recorded.
+__device__ __forceinline__ bool wait_flag_geq(const int* flag, int v, int* status, unsigned long long wait_ns) {
+  const unsigned long long t0 = global_ns();
+  int cur;
+  while (true) {
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(cur) : "l"(flag) : "memory");
+    if (cur >= v) return true;
+    if (global_ns() - t0 > wait_ns) {
+      record_error(status, E3_ERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(64);
+  }
 }
 
 template <typename T, int N>
@@ -726,7 +742,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, int64_t e
 
     for (int st = 0; st < steps; ++st) {
       const int slot = cons_slot;
-      const bool ok = mbar_wait(&bars[slot], cons_phase, a.status);
+      const bool ok = mbar_wait(&bars[slot], cons_phase, a.status, a.wait_ns);
       if (!ok) *s_abort = 1;
       cons_slot = cons_slot + 1 == S ? 0 : cons_slot + 1;
       if (cons_slot == 0) cons_phase ^= 1u;
@@ -760,7 +776,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, int64_t e
   if (!alive) {
     // a wait gave up: let the copies in flight land (bounded) before the CTA exits
     if (tid == 0)
-      for (uint32_t q = consumed - 1; q < issued; ++q) mbar_wait(&bars[q % S], (q / S) & 1u, a.status);
+      for (uint32_t q = consumed - 1; q < issued; ++q) mbar_wait(&bars[q % S], (q / S) & 1u, a.status, a.wait_ns);
     __syncthreads();
     if (seg_flag != nullptr && tid == 0)  // later segments must not wait for this one in vain
       asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(seg_flag), "r"(int(seg + 1)) : "memory");
@@ -780,19 +796,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, int64_t e
       // wait (bounded) until the earlier segments of this row and group have added theirs; the
       // segment that waits drew a later ticket than those it waits for, so they are resident or
       // finished
-      if (tid == 0 && seg > 0) {
-        const unsigned long long t0 = global_ns();
-        int v;
-        while (true) {
-          asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(seg_flag) : "memory");
-          if (v >= seg) break;
-          if (global_ns() - t0 > WAIT_NS) {
-            record_error(a.status, E3_ERR_TIMEOUT);
-            break;
-          }
-          __nanosleep(64);
-        }
-      }
+      if (tid == 0 && seg > 0) wait_flag_geq(seg_flag, int(seg), a.status, a.wait_ns);
       __syncthreads();
       if (slice == 0) {
         if (seg == 0)
@@ -823,7 +827,7 @@ __global__ void __launch_bounds__(256, fwd_min_blocks<CF>()) fwd_kernel(const __
     // a ticket per CTA (tickets follow the order CTAs start in): group, then row segment; a row's
     // later segments wait for its earlier ones, which hold earlier tickets
     __shared__ int s_ticket;
-    if (threadIdx.x == 0) s_ticket = atomicAdd(a.ticket, 1);
+    if (threadIdx.x == 0) s_ticket = atomicAdd(a.ticket, 1) + a.first_ticket;
     __syncthreads();
     const int t = s_ticket;
     const int g = int(t / a.units_max);
@@ -866,6 +870,8 @@ struct KBwd {
   const int4* uinfo;    // convolution: sender units of the topology buffer
   const int32_t* unseg;
   const int32_t* n_units;
+  unsigned long long wait_ns;  // limit of every bounded wait
+  int first_ticket;            // first ticket drawn (0; a test withholds tickets by raising it)
   double scale;
   double alpha[MAXP];
   float alpha_f[MAXP];  // the same path weights rounded once, for the float kernels
@@ -1203,19 +1209,7 @@ __device__ __forceinline__ void bwd_put_dx(typename CF::T* __restrict__ row, con
 // finished and the chain ends at group 0: no deadlock, whatever order the hardware schedules
 // CTAs in.  The wait is bounded; on timeout the error is recorded and the group proceeds.
 __device__ __forceinline__ void bwd_wait_turn(const KBwd& a, int64_t unit, int gi) {
-  if (gi > 0 && threadIdx.x == 0) {
-    long long it = 0;
-    int v;
-    while (true) {
-      asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a.done + unit) : "memory");
-      if (v >= gi) break;
-      if (++it >= WAIT_LIMIT) {
-        record_error(a.status, E3_ERR_TIMEOUT);
-        break;
-      }
-      __nanosleep(64);
-    }
-  }
+  if (gi > 0 && threadIdx.x == 0) wait_flag_geq(a.done + unit, gi, a.status, a.wait_ns);
   __syncwarp();
   // later bulk copies (async proxy) read what the earlier group wrote (generic proxy)
   asm volatile("fence.proxy.async;" ::: "memory");
@@ -1361,7 +1355,7 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const 
         if (lane < NS && rp < cnt) prefetch_l2(w + max(eid[rp], 0) * wrow + size_t(GR::PB) * C, WB);
       }
       const int slot = cons_slot;
-      const bool okw = mbar_wait(&bars[slot], cons_phase, a.status);
+      const bool okw = mbar_wait(&bars[slot], cons_phase, a.status, a.wait_ns);
       if (!okw) *s_abort = 1;
       cons_slot = cons_slot + 1 == S ? 0 : cons_slot + 1;
       if (cons_slot == 0) cons_phase ^= 1u;
@@ -1457,7 +1451,7 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const 
   if (!alive) {
     // a wait gave up: let the copies in flight land (bounded) before the CTA exits
     if (lane == 0)
-      for (uint32_t q = consumed - 1; q < issued; ++q) mbar_wait(&bars[q % S], (q / S) & 1u, a.status);
+      for (uint32_t q = consumed - 1; q < issued; ++q) mbar_wait(&bars[q % S], (q / S) & 1u, a.status, a.wait_ns);
     __syncthreads();
     if (chain != nullptr && lane == 0)  // later pairs must not wait for this one in vain
       asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(chain), "r"(pos + 1) : "memory");
@@ -1471,21 +1465,9 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const 
         for (int k = 0; k < K; ++k)
 #pragma unroll
           for (int j = 0; j < GR::NXG; ++j) dx[k][j] += __shfl_xor_sync(0xffffffffu, dx[k][j], off);
-      if (chain != nullptr && lane == 0 && pos > 0) {
-        // wait (bounded) for the earlier (group, segment) pairs of this sender; they drew
-        // earlier tickets, so they are resident or finished
-        const unsigned long long t0 = global_ns();
-        int v;
-        while (true) {
-          asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(chain) : "memory");
-          if (v >= pos) break;
-          if (global_ns() - t0 > WAIT_NS) {
-            record_error(a.status, E3_ERR_TIMEOUT);
-            break;
-          }
-          __nanosleep(64);
-        }
-      }
+      // wait (bounded) for the earlier (group, segment) pairs of this sender; they drew
+      // earlier tickets, so they are resident or finished
+      if (chain != nullptr && lane == 0 && pos > 0) wait_flag_geq(chain, pos, a.status, a.wait_ns);
       __syncwarp();
       if (slice == 0) bwd_put_dx<CF, GI>(gx + size_t(n) * xrow, dx, C, cb, scale, seg == 0);
       if (chain != nullptr) {
@@ -1515,7 +1497,7 @@ template <class CF, bool CONV, int CC>
 __global__ void __launch_bounds__(32, bwd_min_blocks<CF>()) bwd_kernel(const __grid_constant__ KBwd a) {
   extern __shared__ __align__(128) unsigned char smem[];
   int t = 0;
-  if (threadIdx.x == 0) t = atomicAdd(a.ticket, 1);
+  if (threadIdx.x == 0) t = atomicAdd(a.ticket, 1) + a.first_ticket;
   t = __shfl_sync(0xffffffffu, t, 0);
   const int g = int(t / a.units);
   const int64_t u = t % a.units;
@@ -1556,6 +1538,8 @@ e3_status launch_fwd_cc(const e3_plan* plan, const FwdArgs& h, bool conv) {
   a.sh_norm = h.sh_norm;
   e3_status st = device_status_ptr(&a.status);
   if (st != E3_OK) return st;
+  a.wait_ns = test_wait_limit_ns();
+  a.first_ticket = test_first_ticket();
   for (int p = 0; p < plan->n_paths; ++p) a.pscale[p] = h.scale * plan->alpha[p];
   const int CB = plan->C / 4;
   const int threads = CB >= 32 ? CB : 32;
@@ -1637,6 +1621,8 @@ e3_status launch_bwd_cc(const e3_plan* plan, const BwdArgs& h, bool conv) {
   a.scale = h.scale;
   e3_status st = device_status_ptr(&a.status);
   if (st != E3_OK) return st;
+  a.wait_ns = test_wait_limit_ns();
+  a.first_ticket = test_first_ticket();
   for (int p = 0; p < plan->n_paths; ++p) {
     a.alpha[p] = plan->alpha[p];
     a.alpha_f[p] = float(plan->alpha[p]);

@@ -28,7 +28,7 @@ SYMBOLS = [
     "e3_conv_forward", "e3_conv_backward", "e3_last_error", "e3_csr_build_static",
     "e3_backward_workspace_size", "e3_spherical_harmonics_backward", "e3_morton_workspace_size",
     "e3_morton_order", "e3_invert_permutation", "e3_remap_ids", "e3_conv_workspace_size",
-    "e3_conv_topology_size", "e3_conv_topology_build",
+    "e3_conv_topology_size", "e3_conv_topology_build", "e3_set_test_knobs",
 ]
 
 
@@ -81,6 +81,7 @@ def _load():
                             VP],
         "e3_invert_permutation": [I64, VP, VP, VP],
         "e3_remap_ids": [I64, VP, I64, VP, VP, VP],
+        "e3_set_test_knobs": [I64, I32],
         "e3_last_error": [],
     }
     for name, args in sig.items():

@@ -162,7 +162,8 @@ def graph_inputs(N, mul, lx, ly, lo, seed, dtype=np.float32, weights="host", dev
     """Water-box-like graph: src, dst (int32, sorted by (src, dst)), vec [E, 3] (dtype), x, w.
 
     weights="host" evaluates the radial MLP with numpy; "torch" evaluates it on `device` and
-    returns a torch tensor (for edge counts whose weights do not fit comfortably on the host).
+    returns a torch tensor (for edge counts whose weights do not fit comfortably on the host);
+    "none" skips it (w is None; mlp_apply on the returned parameters gives any subset of rows).
     """
     rng = np.random.default_rng(seed)
     side = box_side(N)
@@ -173,6 +174,8 @@ def graph_inputs(N, mul, lx, ly, lo, seed, dtype=np.float32, weights="host", dev
     feat = bessel_envelope(np.linalg.norm(vec, axis=1))
     if weights == "host":
         w = mlp_apply(feat, w1, w2, dtype)
+    elif weights == "none":
+        w = None
     else:
         import torch
         w = mlp_apply_torch(feat, w1, w2, torch.float32 if dtype == np.float32 else torch.float64, device)

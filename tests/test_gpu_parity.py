@@ -564,7 +564,9 @@ def test_conv_waterbox_full_size_sampled(e3b):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
 def test_conv_large_sampled(e3b, dtype):
-    """24000 nodes, ~1.26M edges, 128 channels, l <= 3: 256 sampled receivers."""
+    """24000 nodes, ~1.26M edges, 128 channels, l <= 3, at full size in the benchmark's launch
+    configuration: the forward on 256 sampled receivers (all their in-edges), the backward's grad_x
+    on 40 sampled senders (all their out-edges) and grad_y / grad_w on those out-edges."""
     cfg = W.CONFIGS["conv_large"]
     n, mul, lx, ly, lo = cfg["N"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
     torch.cuda.empty_cache()
@@ -573,14 +575,34 @@ def test_conv_large_sampled(e3b, dtype):
     s = 1 / math.sqrt(52)
     vec, x = graph.to_receiver_order(t(g["vec"])), t(g["x"])
     wr = graph.to_receiver_order(w)
+    del w  # rows the oracle needs are read from the receiver-ordered copy
+    torch.cuda.empty_cache()
+    perm = graph.perm_dst.cpu().numpy()
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(len(perm))
+
+    def w_rows(sel):
+        return h(wr[torch.as_tensor(inv[sel], device=DEV)])
+
     out = e3b.conv_forward(p, graph, x, wr, edge_vec=vec, out_scale=s)
     nodes = np.sort(np.random.default_rng(1).choice(n, 256, replace=False))
     sel = np.flatnonzero(np.isin(g["dst"], nodes))
-    w_sel = h(w[torch.as_tensor(sel, device=DEV)])
     Y = oracle.real_sh_all(ly, g["vec"][sel].astype(np.float64))
-    ref = oracle.conv_forward(q, n, g["src"][sel], g["dst"][sel], g["x"], Y, w_sel, s)
+    ref = oracle.conv_forward(q, n, g["src"][sel], g["dst"][sel], g["x"], Y, w_rows(sel), s)
     assert rel_err(h(out[torch.as_tensor(nodes, device=DEV)]), ref[nodes]) <= TOL[dtype]
-    del w, wr, out
+    del out
+    torch.cuda.empty_cache()
+    go = W.grad_out(n, q.irreps_out.dim, 5, dtype=NP[dtype])
+    gx, gy, gw = e3b.conv_backward(p, graph, x, wr, t(go), edge_vec=vec, out_scale=s)
+    senders = np.sort(np.random.default_rng(2).choice(n, 40, replace=False))
+    sel = np.flatnonzero(np.isin(g["src"], senders))
+    Y = oracle.real_sh_all(ly, g["vec"][sel].astype(np.float64))
+    rx, ry, rw = oracle.conv_backward(q, n, g["src"][sel], g["dst"][sel], g["x"], Y, w_rows(sel), go, s)
+    assert rel_err(h(gx[torch.as_tensor(senders, device=DEV)]), rx[senders]) <= TOL[dtype]
+    pos = torch.as_tensor(inv[sel], device=DEV)
+    assert rel_err(h(gy[pos]), ry) <= TOL[dtype]
+    assert rel_err(h(gw[pos]), rw) <= TOL[dtype]
+    del wr, gx, gy, gw
     torch.cuda.empty_cache()
 
 

@@ -146,3 +146,11 @@ def test_c_abi_from_plain_c(e3b, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "FAIL" not in r.stdout
+
+
+def test_test_knobs_validate_and_reset(e3b):
+    # host-only: negative values are refused before anything changes; (0, 0) restores the defaults
+    assert e3b.lib.e3_set_test_knobs(-1, 0) == e3b.E3_ERR_INVALID_ARG
+    assert e3b.lib.e3_set_test_knobs(0, -3) == e3b.E3_ERR_INVALID_ARG
+    assert e3b.lib.e3_set_test_knobs(5_000_000, 1) == e3b.E3_OK
+    assert e3b.lib.e3_set_test_knobs(0, 0) == e3b.E3_OK
