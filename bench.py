@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--no-tp", action="store_true", help="skip the tensor-product (no graph) measurement")
     ap.add_argument("--no-waterbox", action="store_true", help="skip the second (water-box) block")
     ap.add_argument("--no-scrub", action="store_true", help="skip the L2-scrubbed per-kernel statistics")
+    ap.add_argument("--shard", action="store_true",
+                    help="shard ONE graph over the ranks (receiver ranges, NCCL halo exchange; strong scaling) "
+                         "instead of one independent graph per rank")
     return ap.parse_args()
 
 
@@ -568,6 +571,79 @@ def measure_e2e(case, steps, world, dist, dev):
             "overlap": "two streams: step k's device-to-host copies overlap step k+1's host-to-device copies"}
 
 
+def run_sharded(args):
+    """Strong scaling: the ranks share one graph (receiver ranges; x halo rows and grad_x partials
+    cross ranks through NCCL all-to-all).  A step is the sharded forward + backward; value = the
+    graph's edges over the slowest rank's step time."""
+    import torch
+    import torch.distributed as dist
+    from mlip_message_passing_b200 import e3b, shard as S, workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    cfg, irreps_x, irreps_y = workload_spec(args.workload)
+    N, mul, lx, ly, lo = cfg["N"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
+    g = W.graph_inputs(N, mul, lx, ly, lo, cfg["seed"], weights="none")  # the same graph on every rank
+    order = np.argsort(g["dst"], kind="stable")
+    src, dst, vec = g["src"][order], g["dst"][order], g["vec"][order]
+    row_ptr = np.concatenate([[0], np.cumsum(np.bincount(dst, minlength=N))])
+    sh = S.ShardPlan(N, src, dst, row_ptr, rank, world)
+    plan = e3b.Plan(irreps_x, irreps_y, lmax_out=lo)
+    conv = S.ShardedConv(sh, S.TorchComm(), S.CudaBackend(plan, sh, dev))
+    e = slice(sh.e_lo, sh.e_hi)
+    feat = W.bessel_envelope(np.linalg.norm(vec[e].astype(np.float64), axis=1))
+    w = W.mlp_apply_torch(feat, *g["mlp"], torch.float32, dev)
+    v = torch.as_tensor(vec[e], device=dev)
+    x = torch.as_tensor(g["x"][sh.lo:sh.hi], device=dev)
+    go = torch.as_tensor(W.grad_out(N, plan.dim_out, cfg.get("grad_seed", 4))[sh.lo:sh.hi], device=dev)
+    s = 1.0 / math.sqrt(52.0)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        conv.forward(x, w, v, s)
+        conv.backward(x, w, v, go, s)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e3b.device_status()
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+    e3b.device_status()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dist, dev) / args.steps
+    halo = max_over_ranks(sh.halo.shape[0], world, dist, dev)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    E = int(row_ptr[-1])
+    line = {"metric": METRIC, "value": E / (ms * 1e-3), "unit": "edges/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{args.workload}_fwd_bwd_sharded", "nodes": N, "edges": E,
+                       "parallelism": f"receiver ranges over {world} ranks, NCCL all-to-all halo exchange",
+                       "max_halo_rows": int(halo)},
+            "gpu_launches": None, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -680,6 +756,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.shard:
+        return run_sharded(args)
     return run_native(args)
 
 

@@ -233,6 +233,15 @@ E3_API e3_status e3_csr_build_static(int64_t N, int64_t E, const int32_t* src, c
 E3_API e3_status e3_gather_rows(int64_t n_rows, int64_t n_in_rows, int64_t row_bytes,
                          const int32_t* perm, const void* in, void* out, void* stream);
 
+/* Rows of `in` added into rows of `out`: out[idx[i], :] += in[i, :] for i < n_rows, each row
+ * row_elems elements of `dtype`; out has n_out_rows rows.  The indices of one call must be
+ * distinct (then no two threads touch one element and the result is deterministic).  This is the
+ * reduction step of a sharded backward (E3J summary, section E.2.2: receiver-partitioned work):
+ * a rank adds the grad_x partial rows other ranks computed for its senders, one source rank per
+ * call, in a fixed order.  An index out of range records E3_ERR_INDEX and that row is skipped. */
+E3_API e3_status e3_add_rows(int64_t n_rows, int64_t n_out_rows, int64_t row_elems, e3_dtype dtype,
+                             const int32_t* idx, const void* in, void* out, void* stream);
+
 /* ------------------------------------------------------------------- node reordering --- */
 
 /* Sparse, irregular gathers bound message passing (Sobek: Streaming Equivariant Tensor Product

@@ -163,6 +163,24 @@ __global__ void gather_rows_kernel(int64_t n_rows, int64_t n_in_rows, int64_t ro
   }
 }
 
+// out[idx[r], :] += in[r, :] for rows r < n_rows of `words` elements of T; the indices of one call
+// are distinct (the caller's contract), so no two threads touch one element and the result does
+// not depend on scheduling.
+template <typename T>
+__global__ void add_rows_kernel(int64_t n_rows, int64_t n_out_rows, int64_t words, const int32_t* __restrict__ idx,
+                                const T* __restrict__ in, T* __restrict__ out, int* status) {
+  const int64_t total = n_rows * words;
+  for (int64_t q = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; q < total; q += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = q / words, c = q % words;
+    const int32_t d = __ldg(idx + r);
+    if (d < 0 || d >= n_out_rows) {
+      rs_error(status, E3_ERR_INDEX);
+      continue;
+    }
+    out[int64_t(d) * words + c] += in[q];
+  }
+}
+
 // ------------------------------------------------------------------- node reordering ---
 // Morton (Z-order) code of a position: each coordinate quantised to 10 bits inside the box
 // (scale = 1024 / extent in double, floor, clamp), bit b of axis k goes to bit 3 b + k.
@@ -408,6 +426,33 @@ extern "C" e3_status e3_gather_rows(int64_t n_rows, int64_t n_in_rows, int64_t r
       n_rows, n_in_rows, words, vec16, perm, static_cast<const uint32_t*>(in), static_cast<uint32_t*>(out), status);
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "gather launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+extern "C" e3_status e3_add_rows(int64_t n_rows, int64_t n_out_rows, int64_t row_elems, e3_dtype dtype,
+                                 const int32_t* idx, const void* in, void* out, void* stream) {
+  clear_error();
+  if (n_rows < 0 || n_out_rows < 0 || row_elems < 0) return fail(E3_ERR_SHAPE, "negative size");
+  if (dtype != E3_F32 && dtype != E3_F64) return fail(E3_ERR_INVALID_ARG, "bad dtype %d", int(dtype));
+  if (n_rows == 0 || row_elems == 0) return E3_OK;
+  if (idx == nullptr || in == nullptr || out == nullptr) return fail(E3_ERR_INVALID_ARG, "NULL pointer");
+  const size_t es = dtype == E3_F64 ? 8 : 4;
+  if ((reinterpret_cast<uintptr_t>(in) % es) || (reinterpret_cast<uintptr_t>(out) % es))
+    return fail(E3_ERR_INVALID_ARG, "in/out not aligned to the element size");
+  int* status = nullptr;
+  e3_status st = device_status_ptr(&status);
+  if (st != E3_OK) return st;
+  const int64_t total = n_rows * row_elems;
+  const int blocks = int(std::min<int64_t>((total + 255) / 256, 148 * 16));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == E3_F32)
+    add_rows_kernel<float><<<blocks, 256, 0, s>>>(n_rows, n_out_rows, row_elems, idx, static_cast<const float*>(in),
+                                                  static_cast<float*>(out), status);
+  else
+    add_rows_kernel<double><<<blocks, 256, 0, s>>>(n_rows, n_out_rows, row_elems, idx,
+                                                   static_cast<const double*>(in), static_cast<double*>(out), status);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "add_rows launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
 }
 

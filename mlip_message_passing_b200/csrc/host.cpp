@@ -572,7 +572,7 @@ extern "C" e3_status e3_conv_workspace_size(const e3_plan* plan, int64_t N, int6
   clear_error();
   if (plan == nullptr || bytes == nullptr) return fail(E3_ERR_INVALID_ARG, "plan or bytes is NULL");
   if (N < 0 || E < 0 || N >= (int64_t(1) << 31) || E >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N or E out of range");
-  *bytes = conv_counters(N, E, plan_groups(plan)).total;
+  *bytes = conv_workspace_bytes(plan, N, E, plan_groups(plan));
   return E3_OK;
 }
 
@@ -582,7 +582,7 @@ static e3_status check_conv_workspace(const e3_plan* plan, int64_t N, int64_t E,
   if (reinterpret_cast<uintptr_t>(topo) % 16 != 0) return fail(E3_ERR_INVALID_ARG, "topology buffer is not 16-byte aligned");
   if (ws == nullptr) return fail(E3_ERR_INVALID_ARG, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(ws) % 16 != 0) return fail(E3_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
-  const size_t need = conv_counters(N, E, plan_groups(plan)).total;
+  const size_t need = conv_workspace_bytes(plan, N, E, plan_groups(plan));
   if (ws_bytes < need) return fail(E3_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", ws_bytes, need);
   return E3_OK;
 }

@@ -137,6 +137,16 @@ inline ConvCounters conv_counters(int64_t N, int64_t E, int G) {
 }
 // path groups of a plan's kernels
 int plan_groups(const e3_plan* plan);
+// Workspace of one convolution call: the counters, then, for float plans, room for a
+// component-major copy of x (forward) or of grad_out (backward), which the paired kernels stage.
+inline size_t conv_workspace_bytes(const e3_plan* plan, int64_t N, int64_t E, int groups) {
+  size_t b = conv_counters(N, E, groups).total;
+  if (plan->dtype == E3_F32) {
+    const int64_t row = plan->dim1 > plan->dim_out ? plan->dim1 : plan->dim_out;
+    b += (size_t(N) * size_t(row) * 4 + 255) & ~size_t(255);
+  }
+  return b;
+}
 e3_status launch_backward(const e3_plan* plan, const BwdArgs& a, bool conv);
 // Zero rows [*first_row, n_rows) of a row-major array of row_bytes-byte rows (first_row read on
 // the device: the padding positions after the last CSR row).

@@ -143,6 +143,9 @@ __device__ __forceinline__ T a_entry(const T (&Y)[NY]) {
   return v;
 }
 
+__device__ __forceinline__ float2 lo2(float4 v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(float4 v) { return make_float2(v.z, v.w); }
+
 // ----------------------------------------------------------------- memory helpers ---
 // 16-byte vector moves between global memory and register arrays.
 template <typename T, int N>
@@ -490,7 +493,147 @@ struct FwdAcc {
       st16(orow + size_t(C) * PC::OUT + size_t(4 * cb) * D3, t);
     });
   }
+
+  // sum over the slices of a warp (lanes that differ in the bits from CB up), fixed butterfly
+  __device__ __forceinline__ void reduce_slices(int CB) {
+    for (int off = CB; off < 32; off <<= 1)
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int o = 0; o < GR::NOG; ++o) acc[k][o] += __shfl_xor_sync(0xffffffffu, acc[k][o], off);
+  }
 };
+
+// The forward accumulator of the float convolution with paired FP32 arithmetic: acc[q][o] holds
+// channels (4cb + 2q, 4cb + 2q + 1) of output o in one register pair, so each fma.rn.f32x2 does
+// the work of two FFMA (the kernels are bound by FP32 issue).  The staged x slices are
+// component-major inside each degree block ([m][u], see transpose_blocks_kernel), so one 16-byte
+// shared load gives two channel pairs of one component.  An entry A[m1, m3] is built once per
+// thread with scalar FMAs (constant-bank coefficients) and duplicated into a pair; keeping the
+// harmonics scalar saves the registers a duplicated copy would hold (measured faster).  The loop
+// runs over m1 outside and m3 inside, so the accumulators of one row are independent; per channel
+// every operation and its order are those of FwdAcc, so the results are bitwise the same.
+template <class CF, int GI>
+struct FwdAcc2 {
+  using GR = Grp<CF, GI>;
+  float2 acc[2][GR::NOG];
+
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+      for (int o = 0; o < GR::NOG; ++o) acc[q][o] = make_float2(0.f, 0.f);
+  }
+
+  // sw: the group's weight slice ([path][u]); sx: x blocks L1A..L1B, each [m][u]
+  __device__ __forceinline__ void edge_smem(const float* sw, const float* sx, const float (&Y)[CF::NY], int C,
+                                            int cb) {
+    static_for<GR::PB, GR::PE>([&](auto pc) {
+      constexpr int P = decltype(pc)::value;
+      using PC = PathC<CF, P>;
+      constexpr int L1 = PC::L1, L2 = PC::L2, L3 = PC::L3, D1 = PC::D1, D3 = PC::D3;
+      constexpr int OO = PC::OUT - GR::OB;
+      const float4 w4 = *reinterpret_cast<const float4*>(sw + size_t(P - GR::PB) * C + 4 * cb);
+      const float2 w2[2] = {lo2(w4), hi2(w4)};
+      float2 x2[2][D1];
+#pragma unroll
+      for (int m1 = 0; m1 < D1; ++m1) {
+        const float4 v = *reinterpret_cast<const float4*>(sx + size_t(C) * (L1 * L1 - GR::XB + m1) + 4 * cb);
+        x2[0][m1] = lo2(v);
+        x2[1][m1] = hi2(v);
+      }
+      if constexpr (D1 < D3) {
+        static_for<0, D1>([&](auto m1c) {
+          constexpr int M1I = decltype(m1c)::value;
+          const float2 xs[2] = {__fmul2_rn(w2[0], x2[0][M1I]), __fmul2_rn(w2[1], x2[1][M1I])};
+          static_for<0, D3>([&](auto m3c) {
+            constexpr int M3I = decltype(m3c)::value;
+            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) {
+              const float a1 = a_entry<float, L1, L2, L3, M1I - L1, M3I - L3>(Y);
+              const float2 a = make_float2(a1, a1);
+              acc[0][OO + M3I] = __ffma2_rn(a, xs[0], acc[0][OO + M3I]);
+              acc[1][OO + M3I] = __ffma2_rn(a, xs[1], acc[1][OO + M3I]);
+            }
+          });
+        });
+      } else {
+        float2 t[2][D3];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int m3 = 0; m3 < D3; ++m3) t[q][m3] = make_float2(0.f, 0.f);
+        static_for<0, D1>([&](auto m1c) {
+          constexpr int M1I = decltype(m1c)::value;
+          static_for<0, D3>([&](auto m3c) {
+            constexpr int M3I = decltype(m3c)::value;
+            if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) {
+              const float a1 = a_entry<float, L1, L2, L3, M1I - L1, M3I - L3>(Y);
+              const float2 a = make_float2(a1, a1);
+              t[0][M3I] = __ffma2_rn(a, x2[0][M1I], t[0][M3I]);
+              t[1][M3I] = __ffma2_rn(a, x2[1][M1I], t[1][M3I]);
+            }
+          });
+        });
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int m3 = 0; m3 < D3; ++m3) acc[q][OO + m3] = __ffma2_rn(w2[q], t[q][m3], acc[q][OO + m3]);
+      }
+    });
+  }
+
+  __device__ __forceinline__ float ch(int k, int o) const { return (k & 1) ? acc[k >> 1][o].y : acc[k >> 1][o].x; }
+
+  __device__ __forceinline__ void store_add(float* __restrict__ orow, int C, int cb, const double* pscale) {
+    static_for<GR::PB, GR::PE>([&](auto pc) {
+      constexpr int P = decltype(pc)::value;
+      using PC = PathC<CF, P>;
+      constexpr int D3 = PC::D3, OO = PC::OUT - GR::OB;
+      const float s = float(pscale[P]);
+      float* p = orow + size_t(C) * PC::OUT + size_t(4 * cb) * D3;
+      float t[K * D3];
+      ld16_l2(t, p);
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int m = 0; m < D3; ++m) t[k * D3 + m] += s * ch(k, OO + m);
+      st16(p, t);
+    });
+  }
+
+  __device__ __forceinline__ void store(float* __restrict__ orow, int C, int cb, const double* pscale) {
+    static_for<GR::PB, GR::PE>([&](auto pc) {
+      constexpr int P = decltype(pc)::value;
+      using PC = PathC<CF, P>;
+      constexpr int D3 = PC::D3, OO = PC::OUT - GR::OB;
+      const float s = float(pscale[P]);
+      float t[K * D3];
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int m = 0; m < D3; ++m) t[k * D3 + m] = s * ch(k, OO + m);
+      st16(orow + size_t(C) * PC::OUT + size_t(4 * cb) * D3, t);
+    });
+  }
+
+  __device__ __forceinline__ void reduce_slices(int CB) {
+    for (int off = CB; off < 32; off <<= 1)
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int o = 0; o < GR::NOG; ++o) {
+          acc[q][o].x += __shfl_xor_sync(0xffffffffu, acc[q][o].x, off);
+          acc[q][o].y += __shfl_xor_sync(0xffffffffu, acc[q][o].y, off);
+        }
+  }
+};
+
+// Paired arithmetic is used by the float convolution (its x and grad_out are transposed to
+// component-major blocks first); double precision and the tensor product keep FwdAcc.
+template <class CF, bool CONV>
+constexpr bool paired() {
+  return CONV && std::is_same<typename CF::T, float>::value;
+}
 
 // ------------------------------------------------------------ async copy machinery ---
 // One thread per CTA streams the weight and x slices of upcoming edges into a ring of shared
@@ -702,7 +845,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, int64_t e
   }
   __syncthreads();
 
-  FwdAcc<CF, GI> f;
+  typename std::conditional<paired<CF, CONV>(), FwdAcc2<CF, GI>, FwdAcc<CF, GI>>::type f;
   f.zero();
   T Y[CF::NY];
   // ring state: identical in every thread, advanced uniformly
@@ -783,13 +926,7 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, int64_t e
     return;
   }
   if constexpr (CONV) {
-    if (CB < 32) {
-      for (int off = CB; off < 32; off <<= 1)
-#pragma unroll
-        for (int k = 0; k < K; ++k)
-#pragma unroll
-          for (int o = 0; o < GR::NOG; ++o) f.acc[k][o] += __shfl_xor_sync(0xffffffffu, f.acc[k][o], off);
-    }
+    if (CB < 32) f.reduce_slices(CB);
     if (seg_flag == nullptr) {
       if (slice == 0) f.store(out + size_t(unit) * orow, C, cb, a.pscale);
     } else {
@@ -874,7 +1011,9 @@ struct KBwd {
   int first_ticket;            // first ticket drawn (0; a test withholds tickets by raising it)
   double scale;
   double alpha[MAXP];
-  float alpha_f[MAXP];  // the same path weights rounded once, for the float kernels
+  float alpha_f[MAXP];    // the same path weights rounded once, for the float kernels
+  float2 alpha_f2[MAXP];  // {alpha_f, alpha_f}: operands of the paired float arithmetic
+  float2 salpha_f2[MAXP]; // {float(scale) * alpha_f, same}: the grad_w factor, rounded as the scalar code rounds it
 };
 
 // Which path groups touch x block l1 / harmonics block l2 (the first toucher stores, later
@@ -1053,6 +1192,110 @@ __device__ __forceinline__ void bwd_edge(const typename CF::T (&xr)[K][Grp<CF, G
               if constexpr (cg_nz(L1, L2, L3, M1I - L1, M2, M3I - L3)) {
                 constexpr int I = cg_index(L1, L2, L3, M1I - L1, M2, M3I - L3);
                 dY[L2 * L2 + L2 + M2] = fma(CGT<T>::template get<I>(), z, dY[L2 * L2 + L2 + M2]);
+              }
+            });
+          }
+        });
+      });
+    }
+  });
+}
+
+// Per-edge backward of group GI for the float convolution with paired FP32 arithmetic (see
+// FwdAcc2): xr2 and dx2 hold channels (4cb + 2q, 4cb + 2q + 1) of one x component in a register
+// pair, and the staged grad_out slice sg is component-major inside each path block ([m3][u]).
+// Per channel the operations and their order are those of bwd_edge, except the grad_y product,
+// whose sum over the thread's four channels is formed as two pair sums added at the end.
+template <class CF, int GI, int FL>
+__device__ __forceinline__ void bwd_edge2(const float2 (&xr2)[2][Grp<CF, GI>::NXG], const float* sw,
+                                          const float (&Y)[CF::NY], const float* sg,
+                                          float2 (&dx2)[2][Grp<CF, GI>::NXG], float (&dY)[CF::NY], bool want_dy,
+                                          float* __restrict__ gw, int C, int cb, const float2* alpha2,
+                                          const float2* salpha2) {
+  using GR = Grp<CF, GI>;
+#pragma unroll
+  for (int i = 0; i < CF::NY; ++i) dY[i] = 0.f;
+  static_for<GR::PB, GR::PE>([&](auto pc) {
+    constexpr int P = decltype(pc)::value;
+    using PC = PathC<CF, P>;
+    constexpr int L1 = PC::L1, L2 = PC::L2, L3 = PC::L3, D1 = PC::D1, D3 = PC::D3;
+    constexpr int XO = L1 * L1 - GR::XB, PW = P - GR::PB;
+    const float4 w4 = *reinterpret_cast<const float4*>(sw + size_t(PW) * C + 4 * cb);
+    float2 g2[2][D3];
+#pragma unroll
+    for (int m3 = 0; m3 < D3; ++m3) {
+      const float4 v = *reinterpret_cast<const float4*>(sg + size_t(C) * (PC::OUT - GR::OB + m3) + 4 * cb);
+      g2[0][m3] = lo2(v);
+      g2[1][m3] = hi2(v);
+    }
+    const float2 wa2[2] = {__fmul2_rn(alpha2[P], lo2(w4)), __fmul2_rn(alpha2[P], hi2(w4))};
+    // t[q][m1] = sum_m3 A[m1, m3] g[q][m3]
+    float2 t2[2][D1];
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+      for (int m1 = 0; m1 < D1; ++m1) t2[q][m1] = make_float2(0.f, 0.f);
+    static_for<0, D3>([&](auto m3c) {
+      constexpr int M3I = decltype(m3c)::value;
+      float2 a[D1];
+      static_for<0, D1>([&](auto m1c) {
+        constexpr int M1I = decltype(m1c)::value;
+        if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) {
+          const float a1 = a_entry<float, L1, L2, L3, M1I - L1, M3I - L3>(Y);
+          a[M1I] = make_float2(a1, a1);
+        }
+      });
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        static_for<0, D1>([&](auto m1c) {
+          constexpr int M1I = decltype(m1c)::value;
+          if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) t2[q][M1I] = __ffma2_rn(a[M1I], g2[q][M3I], t2[q][M1I]);
+        });
+    });
+    if (FL == 1 || gw != nullptr) {  // grad_w[e, p, u] = scale alpha_p sum_m1 x[u, m1] t[u, m1]
+      float2 o2[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int m1 = 0; m1 < D1; ++m1) s2 = __ffma2_rn(xr2[q][XO + m1], t2[q][m1], s2);
+        o2[q] = __fmul2_rn(salpha2[P], s2);
+      }
+      __stcs(reinterpret_cast<float4*>(gw + size_t(P) * C + 4 * cb), make_float4(o2[0].x, o2[0].y, o2[1].x, o2[1].y));
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q)  // grad_x += alpha_p w t
+#pragma unroll
+      for (int m1 = 0; m1 < D1; ++m1) dx2[q][XO + m1] = __ffma2_rn(wa2[q], t2[q][m1], dx2[q][XO + m1]);
+    if (FL == 1 || want_dy) {  // grad_y[m2] += sum_{m1,m3} C[m1,m2,m3] sum_u alpha_p w_u x_u[m1] g_u[m3]
+      constexpr bool SX = D1 <= D3;  // the weight scales the shorter of the x and grad_out blocks
+      float2 xw2[2][SX ? D1 : 1], gw2[2][SX ? 1 : D3];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if constexpr (SX) {
+#pragma unroll
+          for (int m1 = 0; m1 < D1; ++m1) xw2[q][m1] = __fmul2_rn(wa2[q], xr2[q][XO + m1]);
+        } else {
+#pragma unroll
+          for (int m3 = 0; m3 < D3; ++m3) gw2[q][m3] = __fmul2_rn(wa2[q], g2[q][m3]);
+        }
+      }
+      static_for<0, D1>([&](auto m1c) {
+        constexpr int M1I = decltype(m1c)::value;
+        static_for<0, D3>([&](auto m3c) {
+          constexpr int M3I = decltype(m3c)::value;
+          if constexpr (a_nz(L1, L2, L3, M1I - L1, M3I - L3)) {
+            float2 z2;
+            if constexpr (SX)
+              z2 = __ffma2_rn(xw2[1][M1I], g2[1][M3I], __fmul2_rn(xw2[0][M1I], g2[0][M3I]));
+            else
+              z2 = __ffma2_rn(xr2[1][XO + M1I], gw2[1][M3I], __fmul2_rn(xr2[0][XO + M1I], gw2[0][M3I]));
+            const float z = z2.x + z2.y;
+            static_for<-L2, L2 + 1>([&](auto m2c) {
+              constexpr int M2 = decltype(m2c)::value;
+              if constexpr (cg_nz(L1, L2, L3, M1I - L1, M2, M3I - L3)) {
+                constexpr int I = cg_index(L1, L2, L3, M1I - L1, M2, M3I - L3);
+                dY[L2 * L2 + L2 + M2] = fmaf(c_cg32[I], z, dY[L2 * L2 + L2 + M2]);
               }
             });
           }
@@ -1281,11 +1524,21 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const 
   __syncthreads();
 
   T xr[K][GR::NXG], dx[K][GR::NXG], Y[CF::NY], dY[CF::NY];
+  float2 xr2[2][GR::NXG], dx2[2][GR::NXG];  // paired float convolution: channel pairs of x, grad_x
 #pragma unroll
   for (int k = 0; k < K; ++k)
 #pragma unroll
     for (int j = 0; j < GR::NXG; ++j) dx[k][j] = T(0);
   if constexpr (CONV) load_x<CF, GR>(xr, x + size_t(n) * xrow, C, cb);
+  if constexpr (paired<CF, CONV>()) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+      for (int j = 0; j < GR::NXG; ++j) {
+        xr2[q][j] = make_float2(xr[2 * q][j], xr[2 * q + 1][j]);
+        dx2[q][j] = make_float2(0.f, 0.f);
+      }
+  }
   // grad_y components this lane writes after the per-edge reduction (fixed per lane)
   const int ybase = reduce_scatter_base<YUse<CF, GI>::VP>(CB, cb);
   const int yheld = YUse<CF, GI>::VP >= CB ? YUse<CF, GI>::VP / CB : 1;
@@ -1388,9 +1641,12 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const 
 #pragma unroll
           for (int m = 0; m < CF::NY; ++m) Y[m] = yp[m];
         }
-        bwd_edge<CF, GI, FL>(xr, sl, Y, sl + WB / sizeof(T), dx, dY, want_dy,
-                             (FL == 1 || gwp) ? gwp + e * wrow : nullptr, C, cb,
-                         a.alpha, a.alpha_f, scale);
+        if constexpr (paired<CF, CONV>())
+          bwd_edge2<CF, GI, FL>(xr2, sl, Y, sl + WB / sizeof(T), dx2, dY, want_dy,
+                                (FL == 1 || gwp) ? gwp + e * wrow : nullptr, C, cb, a.alpha_f2, a.salpha_f2);
+        else
+          bwd_edge<CF, GI, FL>(xr, sl, Y, sl + WB / sizeof(T), dx, dY, want_dy,
+                               (FL == 1 || gwp) ? gwp + e * wrow : nullptr, C, cb, a.alpha, a.alpha_f, scale);
       } else {
 #pragma unroll
         for (int m = 0; m < CF::NY; ++m) dY[m] = T(0);
@@ -1460,11 +1716,29 @@ __device__ __forceinline__ void bwd_group(const KBwd& a, const int64_t u, const 
   }
   if constexpr (CONV) {
     if (gx != nullptr) {
-      for (int off = CB; off < 32; off <<= 1)
+      if constexpr (paired<CF, CONV>()) {
+        for (int off = CB; off < 32; off <<= 1)
 #pragma unroll
-        for (int k = 0; k < K; ++k)
+          for (int q = 0; q < 2; ++q)
 #pragma unroll
-          for (int j = 0; j < GR::NXG; ++j) dx[k][j] += __shfl_xor_sync(0xffffffffu, dx[k][j], off);
+            for (int j = 0; j < GR::NXG; ++j) {
+              dx2[q][j].x += __shfl_xor_sync(0xffffffffu, dx2[q][j].x, off);
+              dx2[q][j].y += __shfl_xor_sync(0xffffffffu, dx2[q][j].y, off);
+            }
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int j = 0; j < GR::NXG; ++j) {
+            dx[2 * q][j] = dx2[q][j].x;
+            dx[2 * q + 1][j] = dx2[q][j].y;
+          }
+      } else {
+        for (int off = CB; off < 32; off <<= 1)
+#pragma unroll
+          for (int k = 0; k < K; ++k)
+#pragma unroll
+            for (int j = 0; j < GR::NXG; ++j) dx[k][j] += __shfl_xor_sync(0xffffffffu, dx[k][j], off);
+      }
       // wait (bounded) for the earlier (group, segment) pairs of this sender; they drew
       // earlier tickets, so they are resident or finished
       if (chain != nullptr && lane == 0 && pos > 0) wait_flag_geq(chain, pos, a.status, a.wait_ns);
@@ -1520,6 +1794,64 @@ __global__ void __launch_bounds__(32, bwd_min_blocks<CF>()) bwd_kernel(const __g
   }
 }
 
+// ============================================================ layout transposition ===
+// Rows of blocks, block b holding C channels x D_b components.  in: mul_ir ([u][m] inside a
+// block, the boundary's layout); out: component-major ([m][u] inside a block, the same block
+// offsets).  The paired float kernels stage these copies, so that one 16-byte shared-memory load
+// gives two channel pairs of one component.  Each thread writes 4 consecutive channels of one
+// component (a 16-byte store); the reads of a block hit L1 after its first touch.
+struct TransposeArgs {
+  const float* in;
+  float* out;
+  int64_t rows;
+  int row_len;  // floats per row
+  int C;
+  int nblk;
+  int D[MAXP];
+  int off[MAXP];  // float offset of block b in a row
+};
+
+static __global__ void __launch_bounds__(128) transpose_blocks_kernel(const __grid_constant__ TransposeArgs a) {
+  for (int64_t r = blockIdx.x; r < a.rows; r += gridDim.x) {
+    const float* __restrict__ in = a.in + r * a.row_len;
+    float* __restrict__ out = a.out + r * a.row_len;
+    for (int b = 0; b < a.nblk; ++b) {
+      const int D = a.D[b], n = a.C * D;
+      const float* __restrict__ ib = in + a.off[b];
+      float* __restrict__ ob = out + a.off[b];
+      for (int i = 4 * int(threadIdx.x); i < n; i += 4 * int(blockDim.x)) {
+        const int m = i / a.C, u = i - m * a.C;  // C % 4 == 0: i .. i + 3 share m
+        const float* p = ib + u * D + m;
+        __stcg(reinterpret_cast<float4*>(ob + i), make_float4(__ldg(p), __ldg(p + D), __ldg(p + 2 * D), __ldg(p + 3 * D)));
+      }
+    }
+  }
+}
+
+// Component-major copy of `rows` rows whose blocks have the given degrees, on `stream`.
+static inline e3_status transpose_blocks(const float* in, float* out, int64_t rows, int C, const int* degs, int nblk,
+                                         cudaStream_t stream) {
+  if (rows <= 0) return E3_OK;
+  TransposeArgs t{};
+  t.in = in;
+  t.out = out;
+  t.rows = rows;
+  t.C = C;
+  t.nblk = nblk;
+  int off = 0;
+  for (int b = 0; b < nblk; ++b) {
+    t.D[b] = 2 * degs[b] + 1;
+    t.off[b] = off;
+    off += C * t.D[b];
+  }
+  t.row_len = off;
+  const int64_t grid = std::min<int64_t>(rows, int64_t(sm_count()) * 16);
+  transpose_blocks_kernel<<<unsigned(grid), 128, 0, stream>>>(t);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "transpose launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
 // =================================================================== host launchers ===
 template <class CF, int CC>
 e3_status launch_fwd_cc(const e3_plan* plan, const FwdArgs& h, bool conv) {
@@ -1573,6 +1905,15 @@ e3_status launch_fwd_cc(const e3_plan* plan, const FwdArgs& h, bool conv) {
     a.units_max = seg_units_max(h.n_rows, h.n_edges);
     cudaError_t e2 = cudaMemsetAsync(ws, 0, Cn.chain, static_cast<cudaStream_t>(h.stream));
     if (e2 != cudaSuccess) return fail(E3_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e2));
+    if constexpr (paired<CF, true>()) {  // x in component-major blocks, after the counters
+      int degs[CF::LX + 1];
+      for (int l = 0; l <= CF::LX; ++l) degs[l] = l;
+      float* xt = reinterpret_cast<float*>(ws + Cn.total);
+      st = transpose_blocks(static_cast<const float*>(h.x), xt, h.n_rows, plan->C, degs, CF::LX + 1,
+                            static_cast<cudaStream_t>(h.stream));
+      if (st != E3_OK) return st;
+      a.x = xt;
+    }
     units = a.units_max;
     a.n_chunks = 0;
   } else {
@@ -1626,6 +1967,9 @@ e3_status launch_bwd_cc(const e3_plan* plan, const BwdArgs& h, bool conv) {
   for (int p = 0; p < plan->n_paths; ++p) {
     a.alpha[p] = plan->alpha[p];
     a.alpha_f[p] = float(plan->alpha[p]);
+    a.alpha_f2[p] = make_float2(a.alpha_f[p], a.alpha_f[p]);
+    const float sal = float(h.scale) * a.alpha_f[p];
+    a.salpha_f2[p] = make_float2(sal, sal);
   }
   const int CB = plan->C / 4;
   if (CB > 32) return fail(E3_ERR_UNSUPPORTED, "the backward kernels need a multiplicity of at most 128");
@@ -1649,6 +1993,14 @@ e3_status launch_bwd_cc(const e3_plan* plan, const BwdArgs& h, bool conv) {
     a.n_units = reinterpret_cast<const int32_t*>(topo + T.units);
     err = cudaMemsetAsync(ws, 0, Cn.total, s);
     if (err != cudaSuccess) return fail(E3_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
+    if constexpr (paired<CF, true>()) {  // grad_out in component-major path blocks, after the counters
+      int degs[CF::P];
+      for (int p = 0; p < CF::P; ++p) degs[p] = CF::PT.l3[p];
+      float* gt = reinterpret_cast<float*>(ws + Cn.total);
+      st = transpose_blocks(static_cast<const float*>(h.grad_out), gt, h.n_nodes, plan->C, degs, CF::P, s);
+      if (st != E3_OK) return st;
+      a.grad_out = gt;
+    }
   } else {
     const int64_t n_units = (h.n_nodes + NS - 1) / NS;
     units = std::min<int64_t>(n_units, int64_t(sm_count()) * 16);

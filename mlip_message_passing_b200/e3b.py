@@ -28,7 +28,7 @@ SYMBOLS = [
     "e3_conv_forward", "e3_conv_backward", "e3_last_error", "e3_csr_build_static",
     "e3_backward_workspace_size", "e3_spherical_harmonics_backward", "e3_morton_workspace_size",
     "e3_morton_order", "e3_invert_permutation", "e3_remap_ids", "e3_conv_workspace_size",
-    "e3_conv_topology_size", "e3_conv_topology_build", "e3_set_test_knobs",
+    "e3_conv_topology_size", "e3_conv_topology_build", "e3_set_test_knobs", "e3_add_rows",
 ]
 
 
@@ -69,6 +69,7 @@ def _load():
         "e3_csr_build": [I64, I64, VP, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP],
         "e3_csr_build_static": [I64, I64, VP, VP, VP, VP, VP, VP, VP],
         "e3_gather_rows": [I64, I64, I64, VP, VP, VP, VP],
+        "e3_add_rows": [I64, I64, I64, ctypes.c_int, VP, VP, VP, VP],
         "e3_conv_forward": [VP, I64, I64, VP, VP, VP, VP, VP, ctypes.c_int, VP, D, VP, VP, VP, ctypes.c_size_t,
                             VP],
         "e3_conv_workspace_size": [VP, I64, I64, ctypes.POINTER(ctypes.c_size_t)],
@@ -372,6 +373,20 @@ def gather_rows(perm, t, out=None):
         out = torch.empty((n,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
     row_bytes = t.element_size() * (t[0].numel() if t.dim() > 1 else 1)
     _check(lib.e3_gather_rows(n, t.shape[0], row_bytes, _ptr(perm), _ptr(t), _ptr(out), _stream()))
+    return out
+
+
+def add_rows_(out, idx, t):
+    """out[idx[i]] += t[i] for distinct int32 indices (e3_add_rows); returns out."""
+    n = idx.shape[0]
+    _need(idx, "idx", torch.int32, (n,), out.device)
+    if out.dtype not in _DTYPES:
+        raise ValueError("out must be float32 or float64")
+    _need(t, "t", out.dtype, (n,) + tuple(out.shape[1:]), out.device)
+    if not out.is_contiguous():
+        raise ValueError("out must be contiguous")
+    row = out[0].numel() if out.dim() > 1 else 1
+    _check(lib.e3_add_rows(n, out.shape[0], row, _DTYPES[out.dtype], _ptr(idx), _ptr(t), _ptr(out), _stream()))
     return out
 
 
