@@ -282,6 +282,20 @@ E3_API e3_status e3_conv_topology_size(int64_t N, int64_t E, size_t* bytes);
 E3_API e3_status e3_conv_topology_build(int64_t N, int64_t E, const int32_t* row_ptr_dst,
                                  const int32_t* row_ptr_src, void* topo, size_t topo_bytes, void* stream);
 
+/* The same units laid out in a processing order: order [N] (device int32) is a permutation of the
+ * nodes, and the kernels then work through rows (receivers in the forward, senders in the
+ * backward) in that order, each row's segments together and in segment order.  The numbering of
+ * the nodes, and so every array's layout and every result, is unchanged (bitwise): only which
+ * rows are in flight together changes.  With spatially random node ids and node rows larger than
+ * L2, an order that follows space (e.g. e3_morton_order of the positions) makes the rows in flight
+ * neighbours, so the x rows the forward gathers and the grad_out rows the backward gathers are
+ * reused from L2 (Sobek: Streaming Equivariant Tensor Product Convolutions, abstract: sparse,
+ * irregular gathers bound message passing).  An entry out of [0, N) records E3_ERR_INDEX and its
+ * row gets no work; an order that is not a permutation gives unspecified results. */
+E3_API e3_status e3_conv_topology_build_ordered(int64_t N, int64_t E, const int32_t* row_ptr_dst,
+                                                const int32_t* row_ptr_src, const int32_t* order, void* topo,
+                                                size_t topo_bytes, void* stream);
+
 /* out[n] = out_scale * sum_{e : dst_e = n} TP(x[src_e], Y_e, w_e)   [CONV][TP]
  * Edge arrays are in receiver order (apply perm_dst once per topology):
  *   row_ptr_dst [N+1] (row_ptr_dst[0] == 0, non-decreasing; row_ptr_dst[N] <= E, the positions

@@ -150,9 +150,11 @@ E3_HD constexpr int path_cost(int LX, int LY, int LO, int p) {
 }
 
 // Path groups.  Each thread accumulates 4 channels x the outputs of one group of paths in
-// registers, so a group is capped at a number of outputs per channel (the forward and the
-// backward use different caps).  Groups are contiguous runs of paths in enumeration order,
-// cut greedily when the next path would exceed the cap.
+// registers, so a group is capped at a number of outputs per channel.  Groups are contiguous runs
+// of paths in enumeration order, cut greedily when the next path would exceed the cap or would
+// make the group's x components per channel (its degree span l1) exceed 7: a backward thread holds
+// x and grad_x of that span in registers, and the merged kernel's register need is its largest
+// group's (measured on the l <= 3 set: the span 2..3, 12 components, made the backward spill).
 constexpr int GROUP_OUT_CAP = 20;
 
 // Everything the kernels need to know about a path set, computed once per (LX, LY, LO).
@@ -178,12 +180,15 @@ E3_HD constexpr PathTable make_path_table(int LX, int LY, int LO, int cap) {
   int outs = 0;
   t.gbegin[0] = 0;
   t.ngroups = 1;
+  int l1_first = 0;  // lowest x degree of the current group
   for (int p = 0; p < t.n; ++p) {
     const int d = 2 * t.l3[p] + 1;
-    if (outs > 0 && outs + d > cap) {
+    const int nx = (t.l1[p] + 1) * (t.l1[p] + 1) - l1_first * l1_first;  // x components if p joins
+    if (outs > 0 && (outs + d > cap || nx > 7)) {
       t.gbegin[t.ngroups++] = p;
       outs = 0;
     }
+    if (outs == 0) l1_first = t.l1[p];
     outs += d;
   }
   t.gbegin[t.ngroups] = t.n;

@@ -229,37 +229,61 @@ __global__ void remap_ids_kernel(int64_t n, const int32_t* __restrict__ ids, int
   }
 }
 
-// segments per row (at least one, so that every row is written), seg_start[N] = 0 for the scan
-__global__ void seg_count_kernel(int64_t N, const int32_t* __restrict__ row_ptr, int32_t* __restrict__ seg_start) {
-  for (int64_t n = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; n <= N; n += int64_t(gridDim.x) * blockDim.x) {
-    if (n == N) {
+// Segments per row, in processing order: entry i counts the segments of row order[i] (row i
+// without an order); at least one, so that every row is written; seg_start[N] = 0 for the scan.
+// A row whose pointers are out of range, or an order entry out of range, counts one (empty)
+// segment.
+__global__ void seg_count_kernel(int64_t N, int64_t E, const int32_t* __restrict__ row_ptr,
+                                 const int32_t* __restrict__ order, int32_t* __restrict__ seg_start) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i <= N; i += int64_t(gridDim.x) * blockDim.x) {
+    if (i == N) {
       seg_start[N] = 0;
       continue;
     }
-    const int64_t deg = int64_t(row_ptr[n + 1]) - row_ptr[n];
-    seg_start[n] = deg <= SEG_EDGES ? 1 : int32_t((deg + SEG_EDGES - 1) / SEG_EDGES);
+    const int64_t n = order != nullptr ? int64_t(order[i]) : i;
+    int64_t deg = 0;
+    if (n >= 0 && n < N) {
+      const int64_t r0 = row_ptr[n], r1 = row_ptr[n + 1];
+      if (r0 >= 0 && r1 >= r0 && r1 <= E) deg = r1 - r0;
+    }
+    seg_start[i] = deg <= SEG_EDGES ? 1 : int32_t((deg + SEG_EDGES - 1) / SEG_EDGES);
   }
 }
 
-// the units of each row: {row, first edge, end edge, segment} and the row's segment count; the
-// number of units goes to *units.  Rows whose pointers are out of range get empty units.
-__global__ void unit_fill_kernel(int64_t N, int64_t E, const int32_t* __restrict__ row_ptr,
-                                 const int32_t* __restrict__ seg_start, int4* __restrict__ info,
-                                 int32_t* __restrict__ nseg, int32_t* __restrict__ units, int* status) {
-  for (int64_t n = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; n < N; n += int64_t(gridDim.x) * blockDim.x) {
-    int64_t r0 = row_ptr[n], r1 = row_ptr[n + 1];
-    if (r0 < 0 || r1 < r0 || r1 > E) {
+// The units of each row in processing order: {row, first edge, end edge, segment} and the row's
+// segment count; the number of units goes to *units.  Rows whose pointers are out of range, and
+// order entries out of range, record E3_ERR_INDEX and get empty units; units beyond units_max
+// (row pointers that overlap) record E3_ERR_INDEX and are dropped.
+__global__ void unit_fill_kernel(int64_t N, int64_t E, int64_t units_max, const int32_t* __restrict__ row_ptr,
+                                 const int32_t* __restrict__ order, const int32_t* __restrict__ seg_start,
+                                 int4* __restrict__ info, int32_t* __restrict__ nseg, int32_t* __restrict__ units,
+                                 int* status) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < N; i += int64_t(gridDim.x) * blockDim.x) {
+    int64_t n = order != nullptr ? int64_t(order[i]) : i;
+    int64_t r0 = 0, r1 = 0;
+    if (n < 0 || n >= N) {
       atomicCAS(status, 0, int(E3_ERR_INDEX));
-      r0 = r1 = 0;
+      n = 0;
+    } else {
+      r0 = row_ptr[n];
+      r1 = row_ptr[n + 1];
+      if (r0 < 0 || r1 < r0 || r1 > E) {
+        atomicCAS(status, 0, int(E3_ERR_INDEX));
+        r0 = r1 = 0;
+      }
     }
-    const int32_t u0 = seg_start[n], k = seg_start[n + 1] - u0;
+    const int32_t u0 = seg_start[i], k = seg_start[i + 1] - u0;
     for (int32_t s = 0; s < k; ++s) {
+      if (u0 < 0 || int64_t(u0) + s >= units_max) {
+        atomicCAS(status, 0, int(E3_ERR_INDEX));
+        break;
+      }
       const int64_t e0 = r0 + int64_t(s) * SEG_EDGES;
       const int64_t e1 = e0 + SEG_EDGES < r1 ? e0 + SEG_EDGES : r1;
       info[u0 + s] = make_int4(int(n), int(e0 < e1 ? e0 : e1), int(e1), s);
       nseg[u0 + s] = k;
     }
-    if (n == N - 1) *units = seg_start[N];
+    if (i == N - 1) *units = int32_t(seg_start[N] < units_max ? seg_start[N] : units_max);
   }
 }
 
@@ -316,8 +340,8 @@ static e3_status radix_sort(const int32_t* keys, const int32_t* other, const int
   return E3_OK;
 }
 
-e3_status build_topo_part(int64_t N, int64_t E, const int32_t* row_ptr, unsigned char* base, const TopoPart& t,
-                          void* stream) {
+e3_status build_topo_part(int64_t N, int64_t E, const int32_t* row_ptr, const int32_t* order, unsigned char* base,
+                          const TopoPart& t, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* units = reinterpret_cast<int32_t*>(base + t.units);
   cudaError_t err = cudaMemsetAsync(units, 0, 16, s);
@@ -328,9 +352,10 @@ e3_status build_topo_part(int64_t N, int64_t E, const int32_t* row_ptr, unsigned
   if (st != E3_OK) return st;
   int32_t* seg_start = reinterpret_cast<int32_t*>(base + t.seg_start);
   const int blocks = int(std::min<int64_t>((N + 256) / 256, 148 * 8));
-  seg_count_kernel<<<blocks, 256, 0, s>>>(N, row_ptr, seg_start);
+  seg_count_kernel<<<blocks, 256, 0, s>>>(N, E, row_ptr, order, seg_start);
   exclusive_scan_1cta<<<1, 1024, 0, s>>>(seg_start, N + 1, nullptr);
-  unit_fill_kernel<<<blocks, 256, 0, s>>>(N, E, row_ptr, seg_start, reinterpret_cast<int4*>(base + t.info),
+  unit_fill_kernel<<<blocks, 256, 0, s>>>(N, E, seg_units_max(N, E), row_ptr, order, seg_start,
+                                          reinterpret_cast<int4*>(base + t.info),
                                           reinterpret_cast<int32_t*>(base + t.nseg), units, status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "topology launch failed: %s", cudaGetErrorString(err));
@@ -603,6 +628,12 @@ extern "C" e3_status e3_conv_topology_size(int64_t N, int64_t E, size_t* bytes) 
 
 extern "C" e3_status e3_conv_topology_build(int64_t N, int64_t E, const int32_t* row_ptr_dst, const int32_t* row_ptr_src,
                                             void* topo, size_t topo_bytes_, void* stream) {
+  return e3_conv_topology_build_ordered(N, E, row_ptr_dst, row_ptr_src, nullptr, topo, topo_bytes_, stream);
+}
+
+extern "C" e3_status e3_conv_topology_build_ordered(int64_t N, int64_t E, const int32_t* row_ptr_dst,
+                                                    const int32_t* row_ptr_src, const int32_t* order, void* topo,
+                                                    size_t topo_bytes_, void* stream) {
   clear_error();
   if (N < 0 || E < 0 || N >= (int64_t(1) << 31) || E >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N or E out of range");
   if (topo == nullptr || (reinterpret_cast<uintptr_t>(topo) & 15u) != 0)
@@ -610,7 +641,7 @@ extern "C" e3_status e3_conv_topology_build(int64_t N, int64_t E, const int32_t*
   if (topo_bytes_ < topo_bytes(N, E)) return fail(E3_ERR_SHAPE, "topology buffer of %zu bytes, need %zu", topo_bytes_, topo_bytes(N, E));
   if (N > 0 && (row_ptr_dst == nullptr || row_ptr_src == nullptr)) return fail(E3_ERR_INVALID_ARG, "row_ptr array is NULL");
   unsigned char* base = static_cast<unsigned char*>(topo);
-  e3_status st = build_topo_part(N, E, row_ptr_dst, base, topo_dst(N, E), stream);
+  e3_status st = build_topo_part(N, E, row_ptr_dst, order, base, topo_dst(N, E), stream);
   if (st != E3_OK) return st;
-  return build_topo_part(N, E, row_ptr_src, base, topo_src(N, E), stream);
+  return build_topo_part(N, E, row_ptr_src, order, base, topo_src(N, E), stream);
 }

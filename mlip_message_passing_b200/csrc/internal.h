@@ -118,10 +118,11 @@ inline TopoPart topo_part(int64_t N, int64_t E, size_t base) {
 inline TopoPart topo_dst(int64_t N, int64_t E) { return topo_part(N, E, 0); }
 inline TopoPart topo_src(int64_t N, int64_t E) { return topo_part(N, E, topo_dst(N, E).end); }
 inline size_t topo_bytes(int64_t N, int64_t E) { return (topo_src(N, E).end + 255) & ~size_t(255); }
-// Fill one direction's part from row_ptr [N + 1] (rows with out-of-range pointers record
-// E3_ERR_INDEX and get empty units); stream-ordered.
-e3_status build_topo_part(int64_t N, int64_t E, const int32_t* row_ptr, unsigned char* base, const TopoPart& t,
-                          void* stream);
+// Fill one direction's part from row_ptr [N + 1], rows in the processing order `order` (a
+// permutation of 0..N-1, or NULL for 0..N-1); rows with out-of-range pointers record E3_ERR_INDEX
+// and get empty units; stream-ordered.
+e3_status build_topo_part(int64_t N, int64_t E, const int32_t* row_ptr, const int32_t* order, unsigned char* base,
+                          const TopoPart& t, void* stream);
 
 // Per-call counters of a convolution launch (zeroed by the call):
 //   ticket (16 B) | flags [units_max * G] int | chain [N] int

@@ -949,14 +949,20 @@ __device__ __forceinline__ void fwd_group(const KFwd& a, int64_t unit, int64_t e
 }
 
 // Register budget of the forward: path sets with output degree <= 2 fit in 128 registers per
-// thread (16 resident warps per SM); the l <= 3 set keeps the compiler's choice (spills at 128).
+// thread (16 resident warps per SM, CTAs of up to 256 threads, multiplicity <= 1024); the l <= 3
+// set gets 168 (12 warps per SM, CTAs of up to 64 threads, multiplicity <= 256): measured on the
+// large convolution, 7.9 ms against 9.0 ms with the compiler's choice of 252.
+template <class CF>
+constexpr int fwd_max_threads() {
+  return CF::LO <= 2 ? 256 : 64;
+}
 template <class CF>
 constexpr int fwd_min_blocks() {
-  return CF::LO <= 2 ? 2 : 1;
+  return CF::LO <= 2 ? 2 : 6;
 }
 
 template <class CF, bool CONV, int CC>
-__global__ void __launch_bounds__(256, fwd_min_blocks<CF>()) fwd_kernel(const __grid_constant__ KFwd a) {
+__global__ void __launch_bounds__(fwd_max_threads<CF>(), fwd_min_blocks<CF>()) fwd_kernel(const __grid_constant__ KFwd a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   // group-major order, so the CTAs resident on an SM at any time mostly run the same path group
   // and share its (large, fully unrolled) code
@@ -1876,6 +1882,9 @@ e3_status launch_fwd_cc(const e3_plan* plan, const FwdArgs& h, bool conv) {
   const int CB = plan->C / 4;
   const int threads = CB >= 32 ? CB : 32;
   const int NS = CB >= 32 ? 1 : 32 / CB;
+  if (threads > fwd_max_threads<CF>())
+    return fail(E3_ERR_UNSUPPORTED, "forward: multiplicity %d needs %d threads per CTA, at most %d compiled", plan->C,
+                threads, fwd_max_threads<CF>());
   // ring depth: as deep as 3 stages while the CTAs that fit by registers also fit in shared memory
   auto kern = conv ? fwd_kernel<CF, true, CC> : fwd_kernel<CF, false, CC>;
   cudaFuncAttributes fa{};

@@ -29,6 +29,7 @@ SYMBOLS = [
     "e3_backward_workspace_size", "e3_spherical_harmonics_backward", "e3_morton_workspace_size",
     "e3_morton_order", "e3_invert_permutation", "e3_remap_ids", "e3_conv_workspace_size",
     "e3_conv_topology_size", "e3_conv_topology_build", "e3_set_test_knobs", "e3_add_rows",
+    "e3_conv_topology_build_ordered",
 ]
 
 
@@ -75,6 +76,7 @@ def _load():
         "e3_conv_workspace_size": [VP, I64, I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_conv_topology_size": [I64, I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_conv_topology_build": [I64, I64, VP, VP, VP, ctypes.c_size_t, VP],
+        "e3_conv_topology_build_ordered": [I64, I64, VP, VP, VP, VP, ctypes.c_size_t, VP],
         "e3_conv_backward": [VP, I64, I64, VP, VP, VP, VP, VP, VP, VP, VP, ctypes.c_int, VP, VP, D, VP, VP, VP,
                              VP, VP, ctypes.c_size_t, VP],
         "e3_morton_workspace_size": [I64, ctypes.POINTER(ctypes.c_size_t)],
@@ -393,9 +395,11 @@ def add_rows_(out, idx, t):
 class Graph:
     """A fixed topology in receiver order: CSR arrays plus src/dst permuted once (E3J,
     section E.2.2: CSR receiver aggregation).  ``perm_dst[i]`` is the original id of the
-    i-th edge in receiver order; use ``to_receiver_order`` on per-edge arrays."""
+    i-th edge in receiver order; use ``to_receiver_order`` on per-edge arrays.  ``order``: an
+    optional int32 permutation of the nodes in which the kernels process rows (for example the
+    Morton order of the positions, ``morton_order``); results do not depend on it."""
 
-    def __init__(self, n_nodes, src, dst):
+    def __init__(self, n_nodes, src, dst, order=None):
         self.n_nodes = int(n_nodes)
         self.n_edges = int(src.shape[0])
         self.perm_dst, self.row_ptr_dst, self.perm_src, self.row_ptr_src = csr_build(self.n_nodes, src, dst)
@@ -405,8 +409,11 @@ class Graph:
         nbytes = ctypes.c_size_t()
         _check(lib.e3_conv_topology_size(self.n_nodes, self.n_edges, ctypes.byref(nbytes)))
         self.topo = torch.empty(nbytes.value, dtype=torch.uint8, device=src.device)
-        _check(lib.e3_conv_topology_build(self.n_nodes, self.n_edges, _ptr(self.row_ptr_dst), _ptr(self.row_ptr_src),
-                                          _ptr(self.topo), self.topo.numel(), _stream()))
+        if order is not None:
+            _need(order, "order", torch.int32, (self.n_nodes,), src.device)
+        _check(lib.e3_conv_topology_build_ordered(self.n_nodes, self.n_edges, _ptr(self.row_ptr_dst),
+                                                  _ptr(self.row_ptr_src), _ptr(order), _ptr(self.topo),
+                                                  self.topo.numel(), _stream()))
 
     def to_receiver_order(self, t):
         return gather_rows(self.perm_dst, t.contiguous())

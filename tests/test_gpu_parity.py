@@ -693,3 +693,44 @@ def test_autograd_wrapper(e3b):
     out.backward(go)
     gx, gy, gw = e3b.conv_backward(p, graph, x.detach(), wr.detach(), go, y=Y, out_scale=0.3)
     assert torch.equal(x.grad, gx) and torch.equal(y.grad, gy) and torch.equal(wr.grad, gw)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float64])
+def test_processing_order_changes_nothing(e3b, dtype):
+    """Rows processed in another order (a random permutation, and the Morton order of the
+    positions) give bitwise the results of node-id order, also for hub rows cut into segments;
+    an order entry out of range is reported, not dereferenced."""
+    n, mul, lx, ly, lo = 400, 32, 2, 3, 2
+    g = W.graph_inputs(n, mul, lx, ly, lo, 21, dtype=NP[dtype])
+    rng = np.random.default_rng(22)
+    hub = 600  # node 7 receives and sends 600 extra edges: three segments each way
+    src = np.concatenate([g["src"], rng.integers(0, n, hub), np.full(hub, 7)]).astype(np.int32)
+    dst = np.concatenate([g["dst"], np.full(hub, 7), rng.integers(0, n, hub)]).astype(np.int32)
+    keep = src != dst
+    src, dst = src[keep], dst[keep]
+    vec = rng.standard_normal((src.shape[0], 3)).astype(NP[dtype])
+    p = gplan(e3b, mul, lx, ly, lo, dtype)
+    w = rng.standard_normal((src.shape[0], p.weight_numel)).astype(NP[dtype])
+    go = t(rng.standard_normal((n, p.dim_out)).astype(NP[dtype]))
+    x = t(g["x"])
+
+    def run(order):
+        graph = e3b.Graph(n, t(src), t(dst), order=order)
+        v, wr = graph.to_receiver_order(t(vec)), graph.to_receiver_order(t(w))
+        out = e3b.conv_forward(p, graph, x, wr, edge_vec=v, out_scale=0.3)
+        grads = e3b.conv_backward(p, graph, x, wr, go, edge_vec=v, out_scale=0.3)
+        e3b.device_status()
+        return [out, *grads]
+
+    base = run(None)
+    perm = torch.as_tensor(rng.permutation(n).astype(np.int32), device=DEV)
+    morton = e3b.morton_order(t(g["pos"]), (0.0, 0.0, 0.0), (g["side"],) * 3)
+    for order in (perm, morton):
+        for a, b in zip(run(order), base):
+            assert torch.equal(a, b)
+    bad = perm.clone()
+    bad[3] = n + 5
+    graph = e3b.Graph(n, t(src), t(dst), order=bad)
+    with pytest.raises(e3b.E3Error) as err:
+        e3b.device_status()
+    assert err.value.status == e3b.E3_ERR_INDEX
