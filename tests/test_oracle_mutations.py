@@ -240,3 +240,35 @@ def test_right_default_path_weight_passes(monkeypatch):
     # the harness itself: the stated formula re-applied leaves every pin green
     _patch_alpha(monkeypatch, lambda l3, mv, no: np.sqrt((2 * l3 + 1) / (mv * no)))
     assert not _caught(ALPHA_PINS)
+
+
+def _patch_radial(monkeypatch, name, fn):
+    import oracle.radial as orad
+    monkeypatch.setattr(orad, name, fn)
+    monkeypatch.setattr(oracle, name, fn)
+
+
+def test_bessel_without_normalisation(monkeypatch):
+    import oracle.radial as orad
+    orig = orad.bessel_basis
+    _patch_radial(monkeypatch, "bessel_basis", lambda r, c, n: orig(r, c, n) / np.sqrt(2.0 / c))
+    assert _caught([pins.test_bessel_basis_orthonormal_and_limits])
+
+
+def test_bessel_wrong_frequency(monkeypatch):
+    import oracle.radial as orad
+    orig = orad.bessel_basis
+    _patch_radial(monkeypatch, "bessel_basis", lambda r, c, n: orig(r, 2 * c, n))
+    assert _caught([pins.test_bessel_basis_orthonormal_and_limits])
+
+
+@pytest.mark.parametrize("which", ["sign", "order"])
+def test_envelope_wrong_polynomial(monkeypatch, which):
+    import oracle.radial as orad
+    orig = orad.polynomial_envelope
+    if which == "sign":
+        bad = lambda d, p: np.where(np.asarray(d) < 1, 1.0 - (orig(d, p) - 1.0) * 0.9 - 0.1 * np.asarray(d) ** p, 0.0)
+    else:
+        bad = lambda d, p: orig(d, p - 1) if p > 3 else 1 - np.asarray(d)
+    _patch_radial(monkeypatch, "polynomial_envelope", bad)
+    assert _caught([lambda: pins.test_polynomial_envelope_smooth_at_cutoff(6)])

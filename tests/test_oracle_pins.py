@@ -618,3 +618,69 @@ def test_invert_permutation():
     perm = np.random.default_rng(61).permutation(50).astype(np.int32)
     inv = oracle.invert_permutation(perm)
     assert np.array_equal(perm[inv], np.arange(50)) and np.array_equal(inv[perm], np.arange(50))
+
+
+# ----------------------------------------------------------------- radial network ---
+def test_bessel_basis_orthonormal_and_limits():
+    """sqrt(2/c) sin(n pi r / c) / r are orthonormal on [0, c] with weight r^2 (Gauss-Legendre,
+    exact for the trigonometric products to rounding at this order), vanish at r = c and tend to
+    sqrt(2/c) n pi / c at r = 0."""
+    c, nb = 5.0, 8
+    t, wq = np.polynomial.legendre.leggauss(200)
+    r = 0.5 * c * (t + 1.0)
+    b = oracle.bessel_basis(r, c, nb)
+    gram = (b * (r * r * 0.5 * c * wq)[:, None]).T @ b
+    np.testing.assert_allclose(gram, np.eye(nb), atol=1e-12)
+    np.testing.assert_allclose(oracle.bessel_basis(np.array([c]), c, nb), 0.0, atol=1e-14)
+    lim = np.sqrt(2 / c) * np.arange(1, nb + 1) * np.pi / c
+    np.testing.assert_allclose(oracle.bessel_basis(np.array([0.0]), c, nb)[0], lim, rtol=1e-15)
+    np.testing.assert_allclose(oracle.bessel_basis(np.array([1e-7]), c, nb)[0], lim, rtol=1e-10)
+
+
+@pytest.mark.parametrize("p", [3, 5, 6, 8])
+def test_polynomial_envelope_smooth_at_cutoff(p):
+    """The envelope itself (no formula retyped): u(0) = 1; near the cutoff u(1 - e) shrinks like
+    e^3, i.e. u, u' and u'' all vanish at d = 1 (C^2, more than the C^1 the forces need); zero
+    from the cutoff on; decreasing on [0, 1)."""
+    u = lambda d: oracle.polynomial_envelope(np.asarray(d, dtype=np.float64), p)
+    assert u([0.0])[0] == 1.0
+    e = np.array([2e-3, 1e-3, 5e-4])
+    ratio = u(1.0 - e) / e ** 3
+    np.testing.assert_allclose(ratio[1:], ratio[:-1], rtol=0.02)  # cubic order
+    # near d = 0 the envelope leaves 1 at order p (the order the reading fixes)
+    d0 = np.array([0.02, 0.01])
+    slope = np.log((1 - u(d0[0:1])[0]) / (1 - u(d0[1:2])[0])) / np.log(2.0)
+    assert abs(slope - p) < 0.1
+    assert np.all(u([1.0, 1.5, 7.0]) == 0.0)
+    d = np.linspace(0, 0.999, 200)
+    assert np.all(np.diff(u(d)) <= 0) and np.all(np.diff(u(np.linspace(0.2, 0.999, 100))) < 0)
+
+
+def test_silu_closed_forms():
+    x = np.array([-30.0, -1.0, 0.0, 1.0, 30.0])
+    np.testing.assert_allclose(oracle.silu(x), x / (1 + np.exp(-x)), rtol=1e-15)
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    np.testing.assert_allclose(oracle.silu(np.array([40.0])), 40.0, rtol=1e-15)
+    h = 1e-6  # SiLU'(0) = 1/2
+    assert abs((oracle.silu(np.array([h]))[0] - oracle.silu(np.array([-h]))[0]) / (2 * h) - 0.5) < 1e-9
+
+
+def test_radial_weights_brute_force_and_cutoff():
+    rng = np.random.default_rng(31)
+    vec = rng.standard_normal((7, 3)) * 2.0
+    vec[0] = [5.5, 0.0, 0.0]  # beyond the cutoff: envelope 0, SiLU(0) = 0, so w = 0
+    w1 = rng.standard_normal((8, 6))
+    w2 = rng.standard_normal((6, 5))
+    got = oracle.radial_weights(vec, 5.0, 8, 6, w1, w2)
+    for e in range(vec.shape[0]):
+        r = math.sqrt(sum(v * v for v in vec[e]))
+        d = r / 5.0
+        u = 1 - 28 * d ** 6 + 48 * d ** 7 - 21 * d ** 8 if d < 1 else 0.0
+        f = [math.sqrt(2 / 5.0) * math.sin(n * math.pi * r / 5.0) / r * u for n in range(1, 9)]
+        h = []
+        for j in range(6):
+            a = sum(f[n] * w1[n, j] for n in range(8))
+            h.append(a / (1 + math.exp(-a)))
+        for k in range(5):
+            assert abs(got[e, k] - sum(h[j] * w2[j, k] for j in range(6))) < 1e-13
+    assert np.all(got[0] == 0.0)
