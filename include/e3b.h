@@ -269,6 +269,28 @@ E3_API e3_status e3_invert_permutation(int64_t N, const int32_t* perm, int32_t* 
 E3_API e3_status e3_remap_ids(int64_t n, const int32_t* ids, int64_t N, const int32_t* map, int32_t* out,
                        void* stream);
 
+/* ------------------------------------------------------------------- radial network --- */
+
+/* The per-edge path weights of the convolution as a learned function of the edge length (e3nn
+ * course, "Curriculum at a glance", lesson 06a: m_ij = (R(|r_ij|) Y(r_ij)) (x)_w h_j; lesson 05b:
+ * a Bessel basis times a polynomial envelope that keeps the energy smooth at the cutoff):
+ *   f_n = sqrt(2/c) sin(n pi r / c) / r * u(r / c),  n = 1 .. n_basis  (r = |edge_vec|; r -> 0: limit)
+ *   u(d) = 1 - (p+1)(p+2)/2 d^p + p (p+2) d^(p+1) - p (p+1)/2 d^(p+2) for d < 1, else 0
+ *   w = SiLU(f W1) W2,  SiLU(x) = x / (1 + e^-x),  no biases.
+ * The second layer ([E, hidden] x [hidden, n_out]) runs on the tensor cores (tcgen05, tf32 inputs
+ * split into high and low parts, three passes, float32 accumulation: float32-level accuracy).
+ * Float32 only.  W2 is first laid out once per weight update by e3_radial_prepare.
+ *   hidden: a multiple of 8 in [8, 64]; n_out: a multiple of 4; n_basis in [1, 16]; p in [1, 32].
+ *   edge_vec [E, 3], W1 [n_basis, hidden] row-major (device, 4-byte aligned); W2 [hidden, n_out]
+ *   row-major (device); prep: device buffer of e3_radial_prep_size bytes, 16-byte aligned, owned
+ *   by the caller; w [E, n_out] (device, 16-byte aligned, overwritten).  E == 0 is a no-op. */
+E3_API e3_status e3_radial_prep_size(int32_t hidden, int32_t n_out, size_t* bytes);
+E3_API e3_status e3_radial_prepare(int32_t hidden, int32_t n_out, const float* w2, void* prep, size_t prep_bytes,
+                                   void* stream);
+E3_API e3_status e3_radial_weights(int64_t E, const float* edge_vec, double cutoff, int32_t n_basis,
+                                   int32_t envelope_p, int32_t hidden, const float* w1, const void* prep,
+                                   int32_t n_out, float* w, void* stream);
+
 /* ----------------------------------------------------------------------- convolution --- */
 
 /* Work units of the convolution for one topology [CONV]: each receiver's in-edges (receiver CSR)

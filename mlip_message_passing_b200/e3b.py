@@ -29,7 +29,7 @@ SYMBOLS = [
     "e3_backward_workspace_size", "e3_spherical_harmonics_backward", "e3_morton_workspace_size",
     "e3_morton_order", "e3_invert_permutation", "e3_remap_ids", "e3_conv_workspace_size",
     "e3_conv_topology_size", "e3_conv_topology_build", "e3_set_test_knobs", "e3_add_rows",
-    "e3_conv_topology_build_ordered",
+    "e3_conv_topology_build_ordered", "e3_radial_prep_size", "e3_radial_prepare", "e3_radial_weights",
 ]
 
 
@@ -71,6 +71,9 @@ def _load():
         "e3_csr_build_static": [I64, I64, VP, VP, VP, VP, VP, VP, VP],
         "e3_gather_rows": [I64, I64, I64, VP, VP, VP, VP],
         "e3_add_rows": [I64, I64, I64, ctypes.c_int, VP, VP, VP, VP],
+        "e3_radial_prep_size": [I32, I32, ctypes.POINTER(ctypes.c_size_t)],
+        "e3_radial_prepare": [I32, I32, VP, VP, ctypes.c_size_t, VP],
+        "e3_radial_weights": [I64, VP, D, I32, I32, I32, VP, VP, I32, VP, VP],
         "e3_conv_forward": [VP, I64, I64, VP, VP, VP, VP, VP, ctypes.c_int, VP, D, VP, VP, VP, ctypes.c_size_t,
                             VP],
         "e3_conv_workspace_size": [VP, I64, I64, ctypes.POINTER(ctypes.c_size_t)],
@@ -390,6 +393,36 @@ def add_rows_(out, idx, t):
     row = out[0].numel() if out.dim() > 1 else 1
     _check(lib.e3_add_rows(n, out.shape[0], row, _DTYPES[out.dtype], _ptr(idx), _ptr(t), _ptr(out), _stream()))
     return out
+
+
+class Radial:
+    """The radial network w = SiLU(f(|v|) W1) W2 (Bessel basis x polynomial envelope) with W2 laid
+    out once for the tensor cores (e3_radial_prepare); call ``weights(edge_vec)`` per step."""
+
+    def __init__(self, w1, w2, cutoff, envelope_p=6):
+        if w1.dtype != torch.float32 or w2.dtype != torch.float32:
+            raise ValueError("the radial network runs in float32")
+        if not (w1.is_contiguous() and w2.is_contiguous()) or w1.device != w2.device or w1.device.type != "cuda":
+            raise ValueError("w1, w2 must be contiguous CUDA tensors on one device")
+        self.n_basis, self.hidden = w1.shape
+        if w2.shape[0] != self.hidden:
+            raise ValueError("w2 must be [hidden, n_out]")
+        self.n_out = w2.shape[1]
+        self.cutoff, self.p, self.w1 = float(cutoff), int(envelope_p), w1
+        nbytes = ctypes.c_size_t()
+        _check(lib.e3_radial_prep_size(self.hidden, self.n_out, ctypes.byref(nbytes)))
+        self.prep = torch.empty(nbytes.value, dtype=torch.uint8, device=w1.device)
+        _check(lib.e3_radial_prepare(self.hidden, self.n_out, _ptr(w2), _ptr(self.prep), nbytes.value, _stream()))
+
+    def weights(self, edge_vec, out=None):
+        E = edge_vec.shape[0]
+        _need(edge_vec, "edge_vec", torch.float32, (E, 3), self.w1.device)
+        if out is None:
+            out = torch.empty((E, self.n_out), dtype=torch.float32, device=self.w1.device)
+        _need(out, "out", torch.float32, (E, self.n_out), self.w1.device)
+        _check(lib.e3_radial_weights(E, _ptr(edge_vec), self.cutoff, self.n_basis, self.p, self.hidden, _ptr(self.w1),
+                                     _ptr(self.prep), self.n_out, _ptr(out), _stream()))
+        return out
 
 
 class Graph:
