@@ -64,6 +64,7 @@ def parse():
     ap.add_argument("--no-tp", action="store_true", help="skip the tensor-product (no graph) measurement")
     ap.add_argument("--no-waterbox", action="store_true", help="skip the second (water-box) block")
     ap.add_argument("--no-scrub", action="store_true", help="skip the L2-scrubbed per-kernel statistics")
+    ap.add_argument("--no-radial", action="store_true", help="skip the radial-network (tensor core) measurement")
     ap.add_argument("--shard", action="store_true",
                     help="shard ONE graph over the ranks (receiver ranges, NCCL halo exchange; strong scaling) "
                          "instead of one independent graph per rank")
@@ -353,6 +354,7 @@ class ConvCase:
         N, mul, lx, ly, lo = cfg["N"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
         # weak scaling: every rank owns an independent box of the same size (its own seed)
         g = W.graph_inputs(N, mul, lx, ly, lo, rank_seed(cfg["seed"], rank), weights="torch", device=dev)
+        g_mlp = g["mlp"]
         self.plan = e3b.Plan(self.irreps_x, self.irreps_y, lmax_out=lo)
         src_t, dst_t = torch.as_tensor(g["src"], device=dev), torch.as_tensor(g["dst"], device=dev)
         x = torch.as_tensor(g["x"], device=dev)
@@ -384,6 +386,7 @@ class ConvCase:
         self.w = self.graph.to_receiver_order(w_t)
         del g, vec_t, w_t
         self.x, self.go = x, go
+        self.mlp = g_mlp
         self.scale = 1.0 / math.sqrt(52.0)
         self.out = torch.empty((N, self.plan.dim_out), device=dev)
         self.gx = torch.empty_like(x)
@@ -500,6 +503,44 @@ class ConvCase:
                            "algorithmic_bytes": dom_bytes,
                            "achieved_from": "mean launch time over the timed steps (CUDA events)"}
         return out
+
+    def radial_stats(self, reps=SCRUB_REPS):
+        """The radial network on the tensor cores (e3_radial_weights) for this graph's edges: the
+        same weights the convolution streams, written into the grad_w buffer (scratch here);
+        median / p10 / p90 of `reps` launches, each after an L2 scrub."""
+        import torch
+        from mlip_message_passing_b200 import e3b, workloads as W
+        w1, w2 = (torch.as_tensor(m.astype(np.float32), device=self.dev) for m in self.mlp)
+        rad = e3b.Radial(w1, w2, W.CUTOFF, W.ENVELOPE_P)
+        out = self.gw
+        stream = torch.cuda.current_stream()
+        scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=self.dev)
+        for _ in range(3):
+            rad.weights(self.vec, out)
+        ev = []
+        for _ in range(reps):
+            scrub.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            rad.weights(self.vec, out)
+            b.record(stream)
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        e3b.device_status()
+        del scrub
+        t = [a.elapsed_time(b) for a, b in ev]
+        ms = statistics.median(t)
+        E, K, n_out = self.E, rad.hidden, rad.n_out
+        nbytes = E * (12 + 4 * n_out) + 4 * (w1.numel() + w2.numel())
+        flops = 3 * 2 * E * K * (128 * ((n_out + 127) // 128))  # three tf32 passes, 128-column tiles
+        peak, peak_kind = hbm_peak()
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"workload": f"radial network: {E} edges, 8 Bessel x envelope -> SiLU({K}) -> {n_out} weights, fp32 "
+                            f"out, tf32x3 on tcgen05", "median_ms": ms, "p10_ms": percentile(t, 10),
+                "p90_ms": percentile(t, 90), "launches": reps, "edges_per_s": E / (ms * 1e-3), "GBps": gbs,
+                "frac_of_hbm": gbs / peak, "frac_of_nominal": gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": nbytes,
+                "bound": "hbm (the weight write)", "tensor_tflops": flops / (ms * 1e-3) / 1e12,
+                "tensor_flops_per_launch": flops}
 
     def describe(self):
         c = self.cfg
@@ -679,6 +720,7 @@ def run_native(args):
     value = job_throughput(case.E_work, world, ms_step)
     stats = None if args.no_scrub else case.scrubbed_stats()
     head = case.block(fwd_ms, bwd_ms, stats, peak, peak_kind)
+    radial = None if args.no_radial else case.radial_stats()
     w_mb = case.w.numel() * case.w.element_size() / 1e6
     N, E, E_work, plan = case.N, case.E, case.E_work, case.plan
 
@@ -757,6 +799,7 @@ def run_native(args):
                            "L2 scrubbed before each launch"},
         "waterbox": water,
         "tp": tp,
+        "radial": radial,
         "roofline": head["roofline"],
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -34,10 +34,13 @@ namespace {
 
 constexpr int RT_M = 128;         // edges per tile: the MMA's M, one TMEM lane per edge
 constexpr int RT_N = 128;         // output columns per tile: the MMA's N
+constexpr int RT_STAGES = 2;      // B tiles in flight (ring of shared-memory stages)
+constexpr int RT_ACC = 2;         // TMEM accumulators (one per stage)
 constexpr int RT_KMAX = 64;       // hidden width (the MMA's K) at most
 constexpr int RT_BASIS_MAX = 16;  // Bessel functions at most
-constexpr int RT_THREADS = 128;   // four warps; warp w reads TMEM lanes 32w .. 32w + 31
-constexpr int RT_TMEM_COLS = 2 * RT_N;
+constexpr int RT_MATH_WARPS = 8;  // warps w and w + 4 read TMEM lanes 32 (w % 4) .. + 31
+constexpr int RT_THREADS = 32 * RT_MATH_WARPS + 64;  // + one MMA warp + one B producer warp
+constexpr int RT_TMEM_COLS = RT_ACC * RT_N;
 
 // Byte offset of element (row, k) of a K-major operand block with K columns, in the canonical
 // no-swizzle layout: 8-row x 16-byte core matrices; the core matrices along K are LBO = 128 bytes
@@ -124,8 +127,9 @@ __device__ __forceinline__ void mma_commit(uint64_t* b) {
 __device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 consecutive accumulator columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+// 32 consecutive accumulator columns of this thread's TMEM lane (the caller waits with
+// tcgen05.wait::ld before reading v).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
       "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -134,7 +138,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
         "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 struct RadialArgs {
@@ -153,9 +156,15 @@ struct RadialSmem {
   static __host__ __device__ size_t a_bytes(int K) { return size_t(RT_M) * K * 4; }   // one of hi, lo
   static __host__ __device__ size_t b_bytes(int K) { return size_t(2) * RT_N * K * 4; }  // a tile: hi + lo
   static __host__ __device__ size_t b_off(int K) { return 2 * a_bytes(K); }
-  static __host__ __device__ size_t w1_off(int K) { return b_off(K) + 2 * b_bytes(K); }
-  static __host__ __device__ size_t bar_off(int K) { return w1_off(K) + size_t(RT_BASIS_MAX) * RT_KMAX * 4; }
-  static __host__ __device__ size_t total(int K) { return bar_off(K) + 64; }
+  static __host__ __device__ size_t w1_off(int K) { return b_off(K) + RT_STAGES * b_bytes(K); }  // (W1 is read through L1)
+  static __host__ __device__ size_t stage_off(int K) { return w1_off(K); }
+  // per warp, a 32-row x 32-column block of the accumulator on its way to global memory; the
+  // 16-byte chunk j of row r sits at chunk j ^ (r % 8), so writes by row and reads by column group
+  // are both free of bank conflicts
+  static constexpr int STAGE_LD = 32;
+  static __host__ __device__ size_t stage_bytes() { return size_t(RT_MATH_WARPS) * 32 * STAGE_LD * 4; }
+  static __host__ __device__ size_t bar_off(int K) { return stage_off(K) + stage_bytes(); }
+  static __host__ __device__ size_t total(int K) { return bar_off(K) + 8 * (2 * RT_STAGES + 2 * RT_ACC + 2) + 16; }
 };
 
 // Bessel features times the envelope of edge e (zeros past the last edge).
@@ -181,67 +190,99 @@ __device__ __forceinline__ void radial_features(const RadialArgs& a, int64_t e, 
   }
 }
 
-// Thread 0: bulk copy of B tile nt into the next stage of the ring (copies counts the requests).
-__device__ __forceinline__ void request_tile(unsigned char* Bs, const unsigned char* prep, int nt, uint32_t bbytes,
-                                             uint64_t* bbar, uint32_t& copies) {
-  const uint32_t s = copies & 1u;
-  bulk_copy(Bs + size_t(s) * bbytes, prep + size_t(nt) * bbytes, bbytes, &bbar[s]);
-  ++copies;
+// The same wait by every lane of a warp, with one verdict for the warp: the lanes leave it
+// converged (the TMEM loads that follow are warp-collective) and agree on a timeout.
+// Lane 0 polls (32 lanes polling one barrier serialise in shared memory); once it has seen the
+// phase complete, every lane tests it once more, which succeeds at once and gives each lane its
+// own acquire of what the phase publishes (the phase cannot advance before this warp signals).
+__device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, int* status, unsigned long long wait_ns) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = bar_wait(b, parity, status, wait_ns);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok) ok = bar_test(b, parity);
+  return __all_sync(0xffffffffu, ok) != 0;
 }
 
-// Thread 0: the three-pass product of column tile number qq (stage and accumulator qq & 1) once
-// its B tile has landed; false if that wait gave up.
-__device__ __forceinline__ bool issue_tile(const RadialArgs& a, uint32_t qq, uint32_t tmem, uint32_t idesc,
-                                           uint32_t a_hi, uint32_t a_lo, unsigned char* Bs, uint32_t bbytes,
-                                           uint64_t* bbar, uint64_t* mbar, int64_t& last_commit) {
-  const uint32_t s = qq & 1u;
-  if (!bar_wait(&bbar[s], (qq >> 1) & 1u, a.status, a.wait_ns)) return false;
-  fence_after_sync();
-  const uint32_t b_hi = saddr(Bs + size_t(s) * bbytes), b_lo = b_hi + bbytes / 2;
-  const uint32_t d = tmem + s * RT_N;
+// The abort flag as one value for the whole warp.
+__device__ __forceinline__ bool warp_aborted(volatile int* flag) { return __any_sync(0xffffffffu, *flag != 0) != 0; }
+
+// Bulk copy of B tile nt into stage s (one thread).
+__device__ __forceinline__ void request_tile(unsigned char* Bs, const unsigned char* prep, int nt, uint32_t s,
+                                             uint32_t bbytes, uint64_t* bfull) {
+  bulk_copy(Bs + size_t(s) * bbytes, prep + size_t(nt) * bbytes, bbytes, &bfull[s]);
+}
+
+// The three-pass product of one column tile (one thread): B stage s, accumulator ac.
+__device__ __forceinline__ void issue_mma(const RadialArgs& a, uint32_t tmem, uint32_t idesc, uint32_t a_hi,
+                                          uint32_t a_lo, uint32_t b_hi, uint32_t b_lo, uint32_t ac) {
+  const uint32_t d = tmem + ac * RT_N;
   for (int ks = 0; ks < a.K / 8; ++ks) {
     const uint32_t o = uint32_t(ks) * 256;  // one K step: two 128-byte core matrices along K
     mma_tf32(d, smem_desc(a_hi + o, a.K), smem_desc(b_hi + o, a.K), idesc, ks > 0 ? 1u : 0u);
     mma_tf32(d, smem_desc(a_hi + o, a.K), smem_desc(b_lo + o, a.K), idesc, 1u);
     mma_tf32(d, smem_desc(a_lo + o, a.K), smem_desc(b_hi + o, a.K), idesc, 1u);
   }
-  mma_commit(&mbar[s]);
-  last_commit = int64_t(qq);
-  return true;
 }
 
-// Every thread: the 128 accumulator columns of its TMEM lane (edge e) to w[e, 128 nt ..]; the
-// loads are warp-collective, so threads past the last edge load too and store nothing.
-__device__ __forceinline__ void store_tile(const RadialArgs& a, int64_t e, int nt, uint32_t lane_base) {
+// The RT_N / 2 accumulator columns [cbeg, cbeg + RT_N / 2) of this warp's 32 TMEM lanes (edges
+// e0 .. e0 + 31) to w[e, RT_N nt + cbeg ..], 32 columns at a time: each thread loads its lane's
+// values (warp-collective: every thread takes part) and writes them as a row of the warp's
+// staging block; then each store instruction of the warp writes four whole 128-byte row segments
+// (lane l: row l / 8 + 4 i, columns 4 (l % 8) ..), so no sector of w is written in parts.
+__device__ __forceinline__ void store_tile(const RadialArgs& a, int64_t e0, int nt, int cbeg, uint32_t lane_base,
+                                           float* stage) {
+  const int lane = threadIdx.x & 31;
   const int c0 = nt * RT_N;
-  float* orow = a.out + (e < a.E ? e : 0) * a.n_out;
+  constexpr int LD = RadialSmem::STAGE_LD;
+  constexpr int H = RT_N / 64;  // 32-column chunks of this warp's half of the tile
+  uint32_t v[H][32];
 #pragma unroll
-  for (int c = 0; c < RT_N; c += 32) {
-    uint32_t v[32];
-    tmem_ld32(lane_base + uint32_t(c), v);
-    if (e < a.E) {
+  for (int h = 0; h < H; ++h) tmem_ld32_nowait(lane_base + uint32_t(cbeg + 32 * h), v[h]);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const int col = c0 + c + j;
-        if (col < a.n_out)  // n_out % 4 == 0: a group of 4 is all in or all out
-          __stcs(reinterpret_cast<float4*>(orow + col),
-                 make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                             __uint_as_float(v[j + 3])));
-      }
+  for (int h = 0; h < H; ++h) {
+    const int c = cbeg + 32 * h;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(stage + lane * LD + 4 * (j ^ (lane & 7))) =
+          make_float4(__uint_as_float(v[h][4 * j]), __uint_as_float(v[h][4 * j + 1]), __uint_as_float(v[h][4 * j + 2]),
+                      __uint_as_float(v[h][4 * j + 3]));
+    __syncwarp();
+    const int col = c0 + c + 4 * (lane & 7);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int row = (lane >> 3) + 4 * i;
+      const int64_t e = e0 + row;
+      if (e < a.E && col < a.n_out)  // n_out % 4 == 0: a group of 4 is all in or all out
+        *reinterpret_cast<float4*>(a.out + e * a.n_out + col) =
+            *reinterpret_cast<const float4*>(stage + row * LD + 4 * ((lane & 7) ^ (row & 7)));
     }
+    __syncwarp();
   }
 }
 
+// Warp-specialised: warps 0 .. RT_MATH_WARPS-1 compute the hidden layer into the A operand and
+// drain the accumulators to w; warp RT_MATH_WARPS issues the MMAs; the next warp streams the B
+// tiles.  They meet only on mbarriers, each wait bounded:
+//   bfull[s] / bempty[s]      B stage s landed / read by its MMAs (tcgen05.commit)
+//   accfull[c] / accempty[c]  accumulator c written (tcgen05.commit) / drained (one arrive per math warp)
+//   afull / aempty            A of an edge tile written (one arrive per math warp) / read by its MMAs
+// A consumer waits on parity (use & 1) of a full barrier; a producer waits on parity
+// ((use & 1) ^ 1) of an empty one, which a fresh barrier passes at once.
 __global__ void __launch_bounds__(RT_THREADS, 1) radial_kernel(const __grid_constant__ RadialArgs a) {
   extern __shared__ __align__(1024) unsigned char sm[];
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = a.K;
   unsigned char* As = sm;
   unsigned char* Bs = sm + RadialSmem::b_off(K);
-  float* w1s = reinterpret_cast<float*>(sm + RadialSmem::w1_off(K));
-  uint64_t* bbar = reinterpret_cast<uint64_t*>(sm + RadialSmem::bar_off(K));  // B tile landed, per stage
-  uint64_t* mbar = bbar + 2;                                                 // MMAs done, per accumulator
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bbar + 4);
+  float* stage = reinterpret_cast<float*>(sm + RadialSmem::stage_off(K));
+  uint64_t* bfull = reinterpret_cast<uint64_t*>(sm + RadialSmem::bar_off(K));
+  uint64_t* bempty = bfull + RT_STAGES;
+  uint64_t* accfull = bempty + RT_STAGES;
+  uint64_t* accempty = accfull + RT_ACC;
+  uint64_t* afull = accempty + RT_ACC;
+  uint64_t* aempty = afull + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(aempty + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tslot + 1);
   const uint32_t ABYTES = uint32_t(RadialSmem::a_bytes(K)), BBYTES = uint32_t(RadialSmem::b_bytes(K));
 
@@ -251,94 +292,140 @@ __global__ void __launch_bounds__(RT_THREADS, 1) radial_kernel(const __grid_cons
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) bar_init(&bbar[i], 1);
+    for (int i = 0; i < RT_STAGES; ++i) {
+      bar_init(&bfull[i], 1);
+      bar_init(&bempty[i], 1);
+    }
+    for (int i = 0; i < RT_ACC; ++i) {
+      bar_init(&accfull[i], 1);
+      bar_init(&accempty[i], RT_MATH_WARPS);
+    }
+    bar_init(afull, RT_MATH_WARPS);
+    bar_init(aempty, 1);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int i = tid; i < a.n_basis * K; i += RT_THREADS) w1s[i] = __ldg(a.w1 + i);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tslot;
-  const uint32_t idesc = idesc_tf32(RT_M, RT_N);
-  const uint32_t a_hi = saddr(As), a_lo = saddr(As + ABYTES);
-
-  uint32_t q = 0;            // (edge tile, column tile) pairs started by this CTA: identical in every thread
-  uint32_t copies = 0;       // B tiles requested (thread 0's count)
-  int64_t last_commit = -1;  // sequence number of the last committed MMA group (thread 0's)
-  bool alive = true;
   const int64_t n_etiles = (a.E + RT_M - 1) / RT_M;
-  for (int64_t et = blockIdx.x; et < n_etiles && alive; et += gridDim.x) {
-    // ---- features of this thread's edge, then its hidden layer four units at a time, written as
-    // the A operand rows (tf32 hi / lo).  Every MMA that read A has completed: each column tile's
-    // completion was waited for in the previous edge tile.
-    const int64_t e = et * RT_M + tid;
-    float f[RT_BASIS_MAX];
-    radial_features(a, e, f);
-    for (int k = 0; k < K; k += 4) {
-      float hk[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float s = 0.f;
-#pragma unroll
-        for (int n = 0; n < RT_BASIS_MAX; ++n)
-          if (n < a.n_basis) s = fmaf(f[n], w1s[n * K + k + j], s);
-        hk[j] = e < a.E ? s / (1.f + expf(-s)) : 0.f;
-      }
-      float4 hi, lo;
-      hi.x = to_tf32(hk[0]);
-      hi.y = to_tf32(hk[1]);
-      hi.z = to_tf32(hk[2]);
-      hi.w = to_tf32(hk[3]);
-      lo.x = to_tf32(hk[0] - hi.x);
-      lo.y = to_tf32(hk[1] - hi.y);
-      lo.z = to_tf32(hk[2] - hi.z);
-      lo.w = to_tf32(hk[3] - hi.w);
-      *reinterpret_cast<float4*>(As + kmajor_off(tid, k, K)) = hi;
-      *reinterpret_cast<float4*>(As + ABYTES + kmajor_off(tid, k, K)) = lo;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the tensor core reads A through the async proxy
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
 
-    // ---- column tiles: MMA(nt + 1) is issued before the epilogue of nt
-    const uint32_t q0 = q;
-    if (tid == 0) {
-      request_tile(Bs, a.prep, 0, BBYTES, bbar, copies);
-      if (a.n_tiles > 1) request_tile(Bs, a.prep, 1, BBYTES, bbar, copies);
-      if (!issue_tile(a, q0, tmem, idesc, a_hi, a_lo, Bs, BBYTES, bbar, mbar, last_commit)) *s_abort = 1;
-    }
-    for (int nt = 0; nt < a.n_tiles; ++nt) {
-      const uint32_t qq = q0 + uint32_t(nt), s = qq & 1u;
-      if (tid == 0 && !*s_abort && nt + 1 < a.n_tiles &&
-          !issue_tile(a, qq + 1, tmem, idesc, a_hi, a_lo, Bs, BBYTES, bbar, mbar, last_commit))
+  if (warp < RT_MATH_WARPS) {
+    // ------------------------------------------------------------- math warps
+    uint32_t qq = 0, etn = 0;
+    for (int64_t et = blockIdx.x; et < n_etiles && !warp_aborted(s_abort); et += gridDim.x, ++etn) {
+      // A of the previous edge tile has been read by all its MMAs
+      if (!warp_wait(aempty, (etn & 1u) ^ 1u, a.status, a.wait_ns)) {
         *s_abort = 1;
-      // this tile's MMAs done: its accumulator is readable and its B stage is free.  The flag
-      // is made uniform over the CTA, so the warp-collective TMEM loads below are taken by all
-      // threads or by none.
-      const bool done = __syncthreads_and(bar_wait(&mbar[s], (qq >> 1) & 1u, a.status, a.wait_ns) ? 1 : 0) != 0;
-      if (!done) *s_abort = 1;
-      fence_after_sync();
-      if (tid == 0 && done && nt + 2 < a.n_tiles) request_tile(Bs, a.prep, nt + 2, BBYTES, bbar, copies);
-      if (done) store_tile(a, e, nt, tmem + (uint32_t(warp * 32) << 16) + s * RT_N);
-      fence_before_sync();
-      __syncthreads();
-      fence_after_sync();
-      if (*s_abort) {
-        alive = false;
         break;
       }
+      const int row = tid & (RT_M - 1);  // two threads per edge: each writes half of the hidden units
+      const int64_t e = et * RT_M + row;
+      float f[RT_BASIS_MAX];
+      radial_features(a, e, f);
+      const int kh = K / 2;  // a multiple of 4
+      for (int k = (tid >> 7) * kh; k < (tid >> 7) * kh + kh; k += 4) {
+        float hk[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float sum = 0.f;
+#pragma unroll
+          for (int n = 0; n < RT_BASIS_MAX; ++n)
+            if (n < a.n_basis) sum = fmaf(f[n], __ldg(a.w1 + n * K + k + j), sum);
+          hk[j] = e < a.E ? sum / (1.f + expf(-sum)) : 0.f;
+        }
+        float4 hi, lo;
+        hi.x = to_tf32(hk[0]);
+        hi.y = to_tf32(hk[1]);
+        hi.z = to_tf32(hk[2]);
+        hi.w = to_tf32(hk[3]);
+        lo.x = to_tf32(hk[0] - hi.x);
+        lo.y = to_tf32(hk[1] - hi.y);
+        lo.z = to_tf32(hk[2] - hi.z);
+        lo.w = to_tf32(hk[3] - hi.w);
+        *reinterpret_cast<float4*>(As + kmajor_off(row, k, K)) = hi;
+        *reinterpret_cast<float4*>(As + ABYTES + kmajor_off(row, k, K)) = lo;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the tensor core reads A through the async proxy
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(afull)) : "memory");
+      for (int nt = 0; nt < a.n_tiles; ++nt, ++qq) {
+        const uint32_t ac = qq % RT_ACC;
+        if (!warp_wait(&accfull[ac], (qq / RT_ACC) & 1u, a.status, a.wait_ns)) {
+          *s_abort = 1;
+          break;
+        }
+        fence_after_sync();
+        // warps w and w + 4 share TMEM lanes 32 (w % 4) ..; each takes half of the columns
+        store_tile(a, et * RT_M + (warp & 3) * 32, nt, (warp >> 2) * (RT_N / 2),
+                   tmem + (uint32_t((warp & 3) * 32) << 16) + ac * RT_N, stage + warp * 32 * RadialSmem::STAGE_LD);
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(&accempty[ac])) : "memory");
+      }
     }
-    q += uint32_t(a.n_tiles);
-  }
-  if (!alive && tid == 0) {
-    // a wait gave up: let the last copy of each stage and the last committed MMA group (whose
-    // completion implies every earlier one) finish, bounded, before the tensor memory is released
-    for (uint32_t i = copies >= 2 ? copies - 2 : 0; i < copies; ++i)
-      bar_wait(&bbar[i & 1u], (i >> 1) & 1u, a.status, a.wait_ns);
-    if (last_commit >= 0)
-      bar_wait(&mbar[uint32_t(last_commit) & 1u], (uint32_t(last_commit) >> 1) & 1u, a.status, a.wait_ns);
+    __syncwarp();
+  } else if (warp == RT_MATH_WARPS) {
+    // ------------------------------------------------------------- MMA warp (one thread)
+    if (lane == 0) {
+      const uint32_t idesc = idesc_tf32(RT_M, RT_N);
+      const uint32_t a_hi = saddr(As), a_lo = saddr(As + ABYTES);
+      uint32_t qq = 0, etn = 0;
+      int64_t last = -1;  // 0: the last commit went to aempty, else accfull / bempty of tile last - 1
+      for (int64_t et = blockIdx.x; et < n_etiles && !*s_abort; et += gridDim.x, ++etn) {
+        if (!bar_wait(afull, etn & 1u, a.status, a.wait_ns)) {
+          *s_abort = 1;
+          break;
+        }
+        fence_after_sync();
+        for (int nt = 0; nt < a.n_tiles && !*s_abort; ++nt, ++qq) {
+          const uint32_t s = qq % RT_STAGES, ac = qq % RT_ACC;
+          if (!bar_wait(&bfull[s], (qq / RT_STAGES) & 1u, a.status, a.wait_ns) ||
+              !bar_wait(&accempty[ac], ((qq / RT_ACC) & 1u) ^ 1u, a.status, a.wait_ns)) {
+            *s_abort = 1;
+            break;
+          }
+          fence_after_sync();
+          const uint32_t b_hi = saddr(Bs + size_t(s) * BBYTES), b_lo = b_hi + BBYTES / 2;
+          issue_mma(a, tmem, idesc, a_hi, a_lo, b_hi, b_lo, ac);
+          mma_commit(&bempty[s]);
+          mma_commit(&accfull[ac]);
+          last = int64_t(qq) + 1;
+        }
+        if (*s_abort) break;
+        mma_commit(aempty);
+        last = 0;
+      }
+      if (*s_abort && last > 0) {
+        // let the last committed MMA group finish (bounded) before the tensor memory is released
+        const uint32_t lq = uint32_t(last - 1);
+        bar_wait(&accfull[lq % RT_ACC], (lq / RT_ACC) & 1u, a.status, a.wait_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- B producer (one thread)
+    if (lane == 0) {
+      uint32_t i = 0;
+      for (int64_t et = blockIdx.x; et < n_etiles && !*s_abort; et += gridDim.x) {
+        for (int nt = 0; nt < a.n_tiles; ++nt, ++i) {
+          const uint32_t s = i % RT_STAGES;
+          if (!bar_wait(&bempty[s], ((i / RT_STAGES) & 1u) ^ 1u, a.status, a.wait_ns)) {
+            *s_abort = 1;
+            break;
+          }
+          request_tile(Bs, a.prep, nt, s, BBYTES, bfull);
+        }
+        if (*s_abort) break;
+      }
+      if (*s_abort) {
+        // let the copies in flight land (bounded) before the CTA exits
+        for (uint32_t k = i >= RT_STAGES ? i - RT_STAGES : 0; k < i; ++k)
+          bar_wait(&bfull[k % RT_STAGES], (k / RT_STAGES) & 1u, a.status, a.wait_ns);
+      }
+    }
+    __syncwarp();
   }
   fence_before_sync();
   __syncthreads();
