@@ -43,6 +43,10 @@
  *     edge is skipped, never dereferenced.
  *   - Results are deterministic: the same inputs give bitwise the same outputs (no atomics
  *     on floating-point data).
+ *   - Per-device state (the status word, the coefficient tables, the address of the static CSR
+ *     scratch) is set up on a device's first use and kept for the life of the process: after
+ *     cudaDeviceReset, or after the primary context is destroyed, the library must not be called
+ *     again in that process (the cached device addresses would be stale).
  */
 #ifndef E3B_H
 #define E3B_H
