@@ -189,6 +189,17 @@ E3_API e3_status e3_spherical_harmonics(int32_t lmax, int64_t n, const void* vec
 E3_API e3_status e3_spherical_harmonics_backward(int32_t lmax, int64_t n, const void* vec, e3_sh_norm sh_norm,
                                           const void* grad_y, e3_dtype dtype, void* grad_vec, void* stream);
 
+/* The backward of e3_spherical_harmonics_backward, so that forces can be trained through the
+ * harmonics (xnn, "Run Models on Fused GPU Kernels", Training: the fast paths are twice
+ * differentiable).  With grad_vec = J(vec)^T grad_y and u [n, 3] an upstream gradient for grad_vec:
+ *   d_grad_y[i] = J(vec_i) u_i                          ([n, (lmax+1)^2]: derivative of Y along u)
+ *   d_vec[i]    = grad over vec_i of grad_y_i . J(vec_i) u_i   ([n, 3]: a Hessian-vector product)
+ * Both outputs overwritten; same layouts, dtype and limits as e3_spherical_harmonics_backward; a
+ * zero vector gets zeros. */
+E3_API e3_status e3_spherical_harmonics_double_backward(int32_t lmax, int64_t n, const void* vec, e3_sh_norm sh_norm,
+                                                        const void* grad_y, const void* u, e3_dtype dtype,
+                                                        void* d_grad_y, void* d_vec, void* stream);
+
 /* ------------------------------------------------------------------ CSR segmentation --- */
 
 /* Bytes of device workspace that e3_csr_build needs for N nodes and E edges. */

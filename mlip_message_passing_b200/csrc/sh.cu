@@ -79,6 +79,121 @@ __global__ void sh_bwd_kernel(int64_t n, const T* __restrict__ vec, int norm, co
   }
 }
 
+// Second order.  For upstream u (a gradient with respect to grad_vec), the backward of
+// grad_vec = J(vec)^T gy is
+//     d/dgy  = J(vec) u                       (the harmonics' directional derivative along u)
+//     d/dvec = grad_vec (gy . J(vec) u)       (a Hessian-vector product)
+// Both come from evaluating Y on nested dual numbers: the outer number carries the derivative
+// along u, its parts are Dual3 numbers carrying the three derivatives with respect to vec; the
+// direction vec / |vec| is formed on these numbers (1 / sqrt by its own derivative rules), so
+// the radial projection of the first order is included.
+template <typename T>
+struct DualU {  // a + b e with e^2 = 0, parts of type T
+  T a, b;
+};
+template <typename T>
+__device__ __forceinline__ DualU<T> operator+(const DualU<T>& x, const DualU<T>& y) { return {x.a + y.a, x.b + y.b}; }
+template <typename T>
+__device__ __forceinline__ DualU<T> operator-(const DualU<T>& x, const DualU<T>& y) { return {x.a - y.a, x.b - y.b}; }
+template <typename T>
+__device__ __forceinline__ DualU<T> operator*(const DualU<T>& x, const DualU<T>& y) {
+  return {x.a * y.a, x.a * y.b + x.b * y.a};
+}
+template <typename T>
+struct DualUCast {  // constants of sh_poly as nested duals
+  static __device__ __forceinline__ DualU<Dual3<T>> make(double c) { return {Dual3<T>(c), Dual3<T>(0.0)}; }
+};
+template <typename T>
+struct DU {  // DualU<Dual3<T>> with the constructor from a double that sh_poly needs
+  DualU<Dual3<T>> q;
+  __device__ DU() {}
+  __device__ DU(double c) : q{Dual3<T>(c), Dual3<T>(0.0)} {}
+  __device__ DU(const DualU<Dual3<T>>& v) : q(v) {}
+};
+template <typename T>
+__device__ __forceinline__ DU<T> operator+(const DU<T>& x, const DU<T>& y) { return DU<T>(x.q + y.q); }
+template <typename T>
+__device__ __forceinline__ DU<T> operator-(const DU<T>& x, const DU<T>& y) { return DU<T>(x.q - y.q); }
+template <typename T>
+__device__ __forceinline__ DU<T> operator*(const DU<T>& x, const DU<T>& y) { return DU<T>(x.q * y.q); }
+
+// 1 / sqrt(s) on a Dual3 (value and its three derivatives).
+template <typename T>
+__device__ __forceinline__ Dual3<T> rsqrt_d3(const Dual3<T>& s) {
+  Dual3<T> r;
+  r.v = rsqrt_t(s.v);
+  const T dv = T(-0.5) * r.v * r.v * r.v;  // d(s^-1/2)/ds
+#pragma unroll
+  for (int k = 0; k < 3; ++k) r.d[k] = dv * s.d[k];
+  return r;
+}
+// 1 / sqrt(s) on the nested dual: the outer derivative scales by the same first derivative, taken
+// as a Dual3 so that its own vec-derivatives are right.
+template <typename T>
+__device__ __forceinline__ DU<T> rsqrt_du(const DU<T>& s) {
+  const Dual3<T> r = rsqrt_d3(s.q.a);
+  // d(s^-1/2)/ds = -1/2 s^-3/2 = -1/2 r^3 (a Dual3)
+  const Dual3<T> d = Dual3<T>(-0.5) * r * r * r;
+  return DU<T>(DualU<Dual3<T>>{r, d * s.q.b});
+}
+
+template <int LY, typename T>
+__global__ void sh_bwd2_kernel(int64_t n, const T* __restrict__ vec, int norm, const T* __restrict__ gy,
+                               const T* __restrict__ u, T* __restrict__ d_gy, T* __restrict__ d_vec) {
+  constexpr int NY = (LY + 1) * (LY + 1);
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    DU<T> c[3];
+    T r2 = T(0);
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const T vk = vec[3 * i + k];
+      r2 += vk * vk;
+      c[k] = DU<T>(DualU<Dual3<T>>{Dual3<T>(vk, k), Dual3<T>(0.0)});
+      c[k].q.b.v = u[3 * i + k];  // the derivative along u
+    }
+    DU<T> Y[NY];
+    if (r2 > T(0)) {
+      const DU<T> inv = rsqrt_du(c[0] * c[0] + c[1] * c[1] + c[2] * c[2]);
+      sh_poly<LY, DU<T>>(c[0] * inv, c[1] * inv, c[2] * inv, Y);
+    } else {  // Y^0 = 1, Y^(l>0) = 0 at the origin: no derivatives
+#pragma unroll
+      for (int m = 0; m < NY; ++m) Y[m] = DU<T>(m == 0 ? 1.0 : 0.0);
+    }
+    T hv[3] = {T(0), T(0), T(0)};
+#pragma unroll
+    for (int l = 0; l <= LY; ++l) {
+      const T cn = sh_norm_factor<T>(norm, l);
+#pragma unroll
+      for (int m = 0; m < 2 * l + 1; ++m) {
+        const int j = l * l + m;
+        d_gy[i * NY + j] = cn * Y[j].q.b.v;  // (J u)_j
+        const T g = cn * gy[i * NY + j];
+#pragma unroll
+        for (int k = 0; k < 3; ++k) hv[k] = fma(g, Y[j].q.b.d[k], hv[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 3; ++k) d_vec[3 * i + k] = hv[k];
+  }
+}
+
+template <typename T>
+static void sh_bwd2_launch(int lmax, int64_t n, const void* vec, int norm, const void* gy, const void* u, void* dgy,
+                           void* dvec, cudaStream_t s) {
+  const int blocks = int(std::min<int64_t>((n + 255) / 256, int64_t(sm_count()) * 16));
+  const T* v = static_cast<const T*>(vec);
+  const T* g = static_cast<const T*>(gy);
+  const T* uu = static_cast<const T*>(u);
+  T* a = static_cast<T*>(dgy);
+  T* b = static_cast<T*>(dvec);
+  switch (lmax) {
+    case 0: sh_bwd2_kernel<0, T><<<blocks, 256, 0, s>>>(n, v, norm, g, uu, a, b); break;
+    case 1: sh_bwd2_kernel<1, T><<<blocks, 256, 0, s>>>(n, v, norm, g, uu, a, b); break;
+    case 2: sh_bwd2_kernel<2, T><<<blocks, 256, 0, s>>>(n, v, norm, g, uu, a, b); break;
+    default: sh_bwd2_kernel<3, T><<<blocks, 256, 0, s>>>(n, v, norm, g, uu, a, b); break;
+  }
+}
+
 template <typename T>
 static void sh_bwd_launch(int lmax, int64_t n, const void* vec, int norm, const void* gy, void* gv, cudaStream_t s) {
   const int blocks = int(std::min<int64_t>((n + 255) / 256, int64_t(sm_count()) * 16));
@@ -157,5 +272,33 @@ extern "C" e3_status e3_spherical_harmonics_backward(int32_t lmax, int64_t n, co
     sh_bwd_launch<double>(lmax, n, vec, sh_norm, grad_y, grad_vec, s);
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "harmonics backward launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+extern "C" e3_status e3_spherical_harmonics_double_backward(int32_t lmax, int64_t n, const void* vec,
+                                                            e3_sh_norm sh_norm, const void* grad_y,
+                                                            const void* u, e3_dtype dtype, void* d_grad_y,
+                                                            void* d_vec, void* stream) {
+  clear_error();
+  if (lmax < 0 || lmax > E3_LMAX) return fail(E3_ERR_UNSUPPORTED, "lmax %d not in [0, %d]", lmax, E3_LMAX);
+  if (n < 0) return fail(E3_ERR_SHAPE, "n < 0");
+  if (dtype != E3_F32 && dtype != E3_F64) return fail(E3_ERR_INVALID_ARG, "bad dtype");
+  if (sh_norm < E3_SH_COMPONENT || sh_norm > E3_SH_NORM) return fail(E3_ERR_INVALID_ARG, "bad sh_norm");
+  if (n == 0) return E3_OK;
+  const size_t es = dtype == E3_F64 ? 8 : 4;
+  const void* ptrs[5] = {vec, grad_y, u, d_grad_y, d_vec};
+  for (const void* q : ptrs) {
+    if (q == nullptr) return fail(E3_ERR_INVALID_ARG, "NULL pointer");
+    if (reinterpret_cast<uintptr_t>(q) % es) return fail(E3_ERR_INVALID_ARG, "pointer not aligned to its element size");
+  }
+  e3_status st = ensure_device_tables();
+  if (st != E3_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == E3_F32)
+    sh_bwd2_launch<float>(lmax, n, vec, sh_norm, grad_y, u, d_grad_y, d_vec, s);
+  else
+    sh_bwd2_launch<double>(lmax, n, vec, sh_norm, grad_y, u, d_grad_y, d_vec, s);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "harmonics double backward launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
 }

@@ -30,6 +30,7 @@ SYMBOLS = [
     "e3_morton_order", "e3_invert_permutation", "e3_remap_ids", "e3_conv_workspace_size",
     "e3_conv_topology_size", "e3_conv_topology_build", "e3_set_test_knobs", "e3_add_rows",
     "e3_conv_topology_build_ordered", "e3_radial_prep_size", "e3_radial_prepare", "e3_radial_weights",
+    "e3_spherical_harmonics_double_backward",
 ]
 
 
@@ -66,6 +67,7 @@ def _load():
         "e3_backward_workspace_size": [I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_spherical_harmonics": [I32, I64, VP, ctypes.c_int, ctypes.c_int, VP, VP],
         "e3_spherical_harmonics_backward": [I32, I64, VP, ctypes.c_int, VP, ctypes.c_int, VP, VP],
+        "e3_spherical_harmonics_double_backward": [I32, I64, VP, ctypes.c_int, VP, VP, ctypes.c_int, VP, VP, VP],
         "e3_csr_workspace_size": [I64, I64, ctypes.POINTER(ctypes.c_size_t)],
         "e3_csr_build": [I64, I64, VP, VP, VP, VP, VP, VP, VP, ctypes.c_size_t, VP],
         "e3_csr_build_static": [I64, I64, VP, VP, VP, VP, VP, VP, VP],
@@ -288,6 +290,19 @@ def spherical_harmonics_backward(lmax, vec, grad_y, sh_norm="component", out=Non
     return out
 
 
+def spherical_harmonics_double_backward(lmax, vec, grad_y, u, sh_norm="component"):
+    """(d_grad_y, d_vec): the backward of grad_vec = J(vec)^T grad_y for upstream u
+    (e3_spherical_harmonics_double_backward)."""
+    n = vec.shape[0]
+    for t_, nm, sh_ in ((vec, "vec", (n, 3)), (grad_y, "grad_y", (n, (lmax + 1) ** 2)), (u, "u", (n, 3))):
+        _need(t_, nm, vec.dtype, sh_, vec.device)
+    d_gy = torch.empty((n, (lmax + 1) ** 2), dtype=vec.dtype, device=vec.device)
+    d_vec = torch.empty((n, 3), dtype=vec.dtype, device=vec.device)
+    _check(lib.e3_spherical_harmonics_double_backward(lmax, n, _ptr(vec), _SH_NORMS[sh_norm], _ptr(grad_y), _ptr(u),
+                                                      _DTYPES[vec.dtype], _ptr(d_gy), _ptr(d_vec), _stream()))
+    return d_gy, d_vec
+
+
 class _ShFn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, vec, lmax, sh_norm):
@@ -298,11 +313,27 @@ class _ShFn(torch.autograd.Function):
     @staticmethod
     def backward(ctx, g):
         (vec,) = ctx.saved_tensors
-        return spherical_harmonics_backward(ctx.lmax, vec, g.contiguous(), ctx.sh_norm), None, None
+        return _ShBwdFn.apply(vec, g.contiguous(), ctx.lmax, ctx.sh_norm), None, None
+
+
+class _ShBwdFn(torch.autograd.Function):
+    """grad_vec = J(vec)^T grad_y as a differentiable function of (vec, grad_y)."""
+
+    @staticmethod
+    def forward(ctx, vec, gy, lmax, sh_norm):
+        ctx.lmax, ctx.sh_norm = lmax, sh_norm
+        ctx.save_for_backward(vec, gy)
+        return spherical_harmonics_backward(lmax, vec, gy, sh_norm)
+
+    @staticmethod
+    def backward(ctx, u):
+        vec, gy = ctx.saved_tensors
+        d_gy, d_vec = spherical_harmonics_double_backward(ctx.lmax, vec, gy, u.contiguous(), ctx.sh_norm)
+        return d_vec, d_gy, None, None
 
 
 def sh(lmax, vec, sh_norm="component"):
-    """Differentiable real harmonics of vec [n, 3]."""
+    """Twice-differentiable real harmonics of vec [n, 3]."""
     return _ShFn.apply(vec, lmax, sh_norm)
 
 
@@ -500,6 +531,17 @@ def conv_backward(plan, graph, x, w, grad_out, y=None, edge_vec=None, sh_norm="c
     return gx, gy, gw
 
 
+def _accumulate(acc, t):
+    """acc + t for same-shape tensors through the library (e3_add_rows with the identity rows)."""
+    if t is None:
+        return acc
+    if acc is None:
+        return t.contiguous().clone()
+    n = acc.shape[0]
+    idx = torch.arange(n, dtype=torch.int32, device=acc.device)
+    return add_rows_(acc.contiguous(), idx, t.contiguous())
+
+
 class _ConvFn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, x, y, w, plan, graph, out_scale):
@@ -510,14 +552,61 @@ class _ConvFn(torch.autograd.Function):
     @staticmethod
     def backward(ctx, g):
         x, y, w = ctx.saved_tensors
-        gx, gy, gw = conv_backward(ctx.plan, ctx.graph, x, w, g.contiguous(), y=y, out_scale=ctx.out_scale,
-                                   need_x=ctx.needs_input_grad[0], need_y=ctx.needs_input_grad[1],
-                                   need_w=ctx.needs_input_grad[2])
+        gx, gy, gw = _ConvBwdFn.apply(x, y, w, g.contiguous(), ctx.plan, ctx.graph, ctx.out_scale,
+                                      tuple(ctx.needs_input_grad[:3]))
         return gx, gy, gw, None, None, None
 
 
+class _ConvBwdFn(torch.autograd.Function):
+    """The convolution's backward as a differentiable function of (x, y, w, grad_out), so that the
+    convolution is twice differentiable (xnn, "Run Models on Fused GPU Kernels", Training: force
+    training runs through the fast path).  The convolution F(x, y, w) is linear in each argument,
+    so with B_x, B_y, B_w its three gradients and upstream (u_x, u_y, u_w) for them,
+        d/dg = F(u_x, y, w) + F(x, u_y, w) + F(x, y, u_w)
+        d/dx = B_x(x, u_y, w, g) + B_x(x, y, u_w, g)
+        d/dy = B_y(u_x, y, w, g) + B_y(x, y, u_w, g)
+        d/dw = B_w(u_x, y, w, g) + B_w(x, u_y, w, g)
+    (e.g. <u_y, B_y(x, w, g)> = <g, F(x, u_y, w)>, whose x-gradient is B_x with y -> u_y), each
+    term one call of the library's forward or backward kernels, sums by e3_add_rows."""
+
+    @staticmethod
+    def forward(ctx, x, y, w, g, plan, graph, out_scale, needs):
+        ctx.plan, ctx.graph, ctx.out_scale = plan, graph, out_scale
+        ctx.save_for_backward(x, y, w, g)
+        gx, gy, gw = conv_backward(plan, graph, x, w, g, y=y, out_scale=out_scale, need_x=needs[0], need_y=needs[1],
+                                   need_w=needs[2])
+        return gx, gy, gw
+
+    @staticmethod
+    def backward(ctx, ux, uy, uw):
+        x, y, w, g = ctx.saved_tensors
+        P, G, s = ctx.plan, ctx.graph, ctx.out_scale
+        nx, ny, nw, ng = ctx.needs_input_grad[:4]
+        ux = None if ux is None else ux.contiguous()
+        uy = None if uy is None else uy.contiguous()
+        uw = None if uw is None else uw.contiguous()
+        dx = dy = dw = dg = None
+        if ng:
+            if ux is not None:
+                dg = _accumulate(dg, conv_forward(P, G, ux, w, y=y, out_scale=s))
+            if uy is not None:
+                dg = _accumulate(dg, conv_forward(P, G, x, w, y=uy, out_scale=s))
+            if uw is not None:
+                dg = _accumulate(dg, conv_forward(P, G, x, uw, y=y, out_scale=s))
+        if uy is not None and (nx or nw):  # y -> u_y: its x- and w-gradients
+            bx, _, bw = conv_backward(P, G, x, w, g, y=uy, out_scale=s, need_x=nx, need_y=False, need_w=nw)
+            dx, dw = _accumulate(dx, bx), _accumulate(dw, bw)
+        if uw is not None and (nx or ny):  # w -> u_w: its x- and y-gradients
+            bx, by, _ = conv_backward(P, G, x, uw, g, y=y, out_scale=s, need_x=nx, need_y=ny, need_w=False)
+            dx, dy = _accumulate(dx, bx), _accumulate(dy, by)
+        if ux is not None and (ny or nw):  # x -> u_x: its y- and w-gradients
+            _, by, bw = conv_backward(P, G, ux, w, g, y=y, out_scale=s, need_x=False, need_y=ny, need_w=nw)
+            dy, dw = _accumulate(dy, by), _accumulate(dw, bw)
+        return dx, dy, dw, dg, None, None, None, None
+
+
 def conv(plan, graph, x, y, w, out_scale=1.0):
-    """Differentiable convolution with respect to x, y (harmonics) and w."""
+    """Twice-differentiable convolution with respect to x, y (harmonics) and w."""
     return _ConvFn.apply(x, y, w, plan, graph, out_scale)
 
 
