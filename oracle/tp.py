@@ -1,4 +1,4 @@
-"""Weighted channelwise ("uvu") tensor product in float64 (oracle side; test infrastructure only).
+"""Weighted tensor product in float64 (oracle side; test infrastructure only).
 
 e3nn course, "Curriculum at a glance", lesson 03b: a learnable tensor product x (x)_w y is a list
 of instructions (i1, i2, i_out); each instruction couples irrep i1 of x with irrep i2 of y into
@@ -9,6 +9,17 @@ channels v of y with one weight per (u, v):
     out[b, i_out, u, m3] += alpha_p * sum_v w[b, p, u, v]
                             * sum_{m1, m2} C_p[m1, m2, m3] x[b, i1, u, m1] y[b, i2, v, m2]
 
+"uuu" ties all three channels (both inputs and the output have the same multiplicity), one weight
+per (p, u):
+
+    out[b, i_out, u, m3] += alpha_p * w[b, p, u] * sum_{m1, m2} C_p[m1, m2, m3] x[b, i1, u, m1] y[b, i2, u, m2]
+
+"uvw" (fully connected) mixes every pair of input channels into every output channel, one weight
+per (p, u, v, w):
+
+    out[b, i_out, w, m3] += alpha_p * sum_{u, v} W[b, p, u, v, w]
+                            * sum_{m1, m2} C_p[m1, m2, m3] x[b, i1, u, m1] y[b, i2, v, m2]
+
 Lesson 03a fixes the parity rule p3 = p1 p2 and the triangle rule |l1-l2| <= l3 <= l1+l2.
 The sum over (m1, m2, m3) is written densely (no use of sparsity).  Readings taken where the
 sources are silent:
@@ -17,9 +28,11 @@ sources are silent:
   |l1-l2| to min(l1+l2, lmax_out): one instruction with its own output block ("uncollapsed"
   output, irrep (mul_x, l3, p1 p2)); E3J summary, section B.3, treats collapsed (shared) output
   blocks as a special case, which explicit instruction lists may request by sharing i_out;
-* weights: ``w[b, p, u, v]`` flattened path-major, then u, then v (one weight per (u, v));
-* alpha_p = sqrt((2 l3 + 1) / (mul_y * n_out)), n_out = number of instructions writing i_out,
-  so that unit-variance inputs give unit-variance outputs; an instruction may override it.
+* weights flattened path-major, then the mode's channel indices in the order written above
+  (uvu: u, v; uuu: u; uvw: u, v, w);
+* alpha_p = sqrt((2 l3 + 1) / (fan_in * n_out)), n_out = number of instructions writing i_out and
+  fan_in the channel sum of one output element (uvu: mul_y; uuu: 1; uvw: mul_x * mul_y), so that
+  unit-variance inputs give unit-variance outputs; an instruction may override it.
 """
 
 from dataclasses import dataclass, field
@@ -49,6 +62,7 @@ class TPPlan:
     weight_offsets: list = field(default_factory=list)
     weight_numel: int = 0
     shared_weights: bool = False
+    mode: str = "uvu"
 
     @property
     def n_paths(self):
@@ -66,8 +80,10 @@ def _enumerate(ir1, ir2, lmax_out):
 
 
 def make_plan(irreps_in1, irreps_in2, irreps_out=None, instructions=None, lmax_out=None,
-              shared_weights=False):
+              shared_weights=False, mode="uvu"):
     """Build the oracle's plan.  ``irreps_out``/``instructions`` None -> default enumeration."""
+    if mode not in ("uvu", "uuu", "uvw"):
+        raise ValueError(f"unknown connection mode {mode!r}")
     ir1 = parse_irreps(irreps_in1) if isinstance(irreps_in1, str) else irreps_in1
     ir2 = parse_irreps(irreps_in2) if isinstance(irreps_in2, str) else irreps_in2
     if instructions is None:
@@ -83,22 +99,25 @@ def make_plan(irreps_in1, irreps_in2, irreps_out=None, instructions=None, lmax_o
             raise ValueError(f"instruction {ins_} breaks the triangle rule")
         if c.p != a.p * b.p:
             raise ValueError(f"instruction {ins_} breaks the parity rule p3 = p1 p2")
-        if c.mul != a.mul:
-            raise ValueError(f"uvu instruction {ins_} needs mul_out == mul_in1")
+        if mode in ("uvu", "uuu") and c.mul != a.mul:
+            raise ValueError(f"{mode} instruction {ins_} needs mul_out == mul_in1")
+        if mode == "uuu" and b.mul != a.mul:
+            raise ValueError(f"uuu instruction {ins_} needs mul_in2 == mul_in1")
     n_out = {}
     for ins_ in ins:
         n_out[ins_.i_out] = n_out.get(ins_.i_out, 0) + 1
     alphas, woffs, wn = [], [], 0
     for ins_ in ins:
         a, b, c = ir1[ins_.i_in1], ir2[ins_.i_in2], irout[ins_.i_out]
+        fan_in = {"uvu": b.mul, "uuu": 1, "uvw": a.mul * b.mul}[mode]
         if ins_.path_weight >= 0:
             alphas.append(float(ins_.path_weight))
         else:
-            alphas.append(float(np.sqrt((2 * c.l + 1) / (b.mul * n_out[ins_.i_out]))))
+            alphas.append(float(np.sqrt((2 * c.l + 1) / (fan_in * n_out[ins_.i_out]))))
         woffs.append(wn)
         if ins_.has_weight:
-            wn += a.mul * b.mul
-    return TPPlan(ir1, ir2, irout, ins, alphas, woffs, wn, shared_weights)
+            wn += {"uvu": a.mul * b.mul, "uuu": a.mul, "uvw": a.mul * b.mul * c.mul}[mode]
+    return TPPlan(ir1, ir2, irout, ins, alphas, woffs, wn, shared_weights, mode)
 
 
 def _blocks(plan, p):
@@ -111,13 +130,24 @@ def _blocks(plan, p):
 
 
 def _weights(plan, w, p, bsz):
-    ins, a, b = plan.instructions[p], plan.irreps_in1[plan.instructions[p].i_in1], plan.irreps_in2[plan.instructions[p].i_in2]
+    """The path's weights as [B, u, v] (uvu), [B, u] (uuu) or [B, u, v, w] (uvw)."""
+    ins = plan.instructions[p]
+    a, b, c = plan.irreps_in1[ins.i_in1], plan.irreps_in2[ins.i_in2], plan.irreps_out[ins.i_out]
+    shape = {"uvu": (a.mul, b.mul), "uuu": (a.mul,), "uvw": (a.mul, b.mul, c.mul)}[plan.mode]
+    size = int(np.prod(shape))
     if not ins.has_weight:
-        return np.ones((bsz, a.mul, b.mul))
+        return np.ones((bsz,) + shape)
     off = plan.weight_offsets[p]
     if plan.shared_weights:
-        return np.broadcast_to(w[off:off + a.mul * b.mul].reshape(1, a.mul, b.mul), (bsz, a.mul, b.mul))
-    return w[:, off:off + a.mul * b.mul].reshape(bsz, a.mul, b.mul)
+        return np.broadcast_to(w[off:off + size].reshape((1,) + shape), (bsz,) + shape)
+    return w[:, off:off + size].reshape((bsz,) + shape)
+
+
+# einsum of each mode: x "bui", y "bvj", C "ijk", weights, output "b?k"
+_FWD = {"uvu": "bui,bvj,ijk,buv->buk", "uuu": "bui,buj,ijk,bu->buk", "uvw": "bui,bvj,ijk,buvw->bwk"}
+_DX = {"uvu": "bvj,ijk,buv,buk->bui", "uuu": "buj,ijk,bu,buk->bui", "uvw": "bvj,ijk,buvw,bwk->bui"}
+_DY = {"uvu": "bui,ijk,buv,buk->bvj", "uuu": "bui,ijk,bu,buk->buj", "uvw": "bui,ijk,buvw,bwk->bvj"}
+_DW = {"uvu": "bui,bvj,ijk,buk->buv", "uuu": "bui,buj,ijk,buk->bu", "uvw": "bui,bvj,ijk,bwk->buvw"}
 
 
 def tp_forward(plan, x, y, w):
@@ -133,7 +163,7 @@ def tp_forward(plan, x, y, w):
         xs = x[:, o1:o1 + a.dim].reshape(bsz, a.mul, 2 * a.l + 1)
         ys = y[:, o2:o2 + b.dim].reshape(bsz, b.mul, 2 * b.l + 1)
         ws = _weights(plan, w, p, bsz)
-        blk = plan.alphas[p] * np.einsum("bui,bvj,ijk,buv->buk", xs, ys, C, ws, optimize=True)
+        blk = plan.alphas[p] * np.einsum(_FWD[plan.mode], xs, ys, C, ws, optimize=True)
         out[:, o3:o3 + c.dim] += blk.reshape(bsz, -1)
     return out
 
@@ -156,13 +186,13 @@ def tp_backward(plan, x, y, w, grad_out):
         ys = y[:, o2:o2 + b.dim].reshape(bsz, b.mul, 2 * b.l + 1)
         gs = g[:, o3:o3 + c.dim].reshape(bsz, c.mul, 2 * c.l + 1)
         ws = _weights(plan, w, p, bsz)
-        dx[:, o1:o1 + a.dim] += al * np.einsum("bvj,ijk,buv,buk->bui", ys, C, ws, gs, optimize=True).reshape(bsz, -1)
-        dy[:, o2:o2 + b.dim] += al * np.einsum("bui,ijk,buv,buk->bvj", xs, C, ws, gs, optimize=True).reshape(bsz, -1)
+        dx[:, o1:o1 + a.dim] += al * np.einsum(_DX[plan.mode], ys, C, ws, gs, optimize=True).reshape(bsz, -1)
+        dy[:, o2:o2 + b.dim] += al * np.einsum(_DY[plan.mode], xs, C, ws, gs, optimize=True).reshape(bsz, -1)
         if ins.has_weight:
             off = plan.weight_offsets[p]
-            dwp = al * np.einsum("bui,bvj,ijk,buk->buv", xs, ys, C, gs, optimize=True).reshape(bsz, -1)
+            dwp = al * np.einsum(_DW[plan.mode], xs, ys, C, gs, optimize=True).reshape(bsz, -1)
             if plan.shared_weights:
-                dw[off:off + a.mul * b.mul] += dwp.sum(axis=0)
+                dw[off:off + dwp.shape[1]] += dwp.sum(axis=0)
             else:
-                dw[:, off:off + a.mul * b.mul] += dwp
+                dw[:, off:off + dwp.shape[1]] += dwp
     return dx, dy, dw

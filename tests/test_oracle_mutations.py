@@ -16,11 +16,15 @@ from tests import test_oracle_pins as pins
 
 
 def _caught(checks):
+    """True when one check fails an assertion.  A check that raises ValueError (a mutation that
+    breaks the shapes of that check's inputs) does not count as catching it."""
     for fn in checks:
         try:
             fn()
         except AssertionError:
             return True
+        except ValueError:
+            continue
     return False
 
 
@@ -124,7 +128,7 @@ def test_backward_dropped_alpha_in_dy(monkeypatch):
         return dx, dy * 0.5, dw
 
     monkeypatch.setattr(oracle, "tp_backward", bad)
-    assert _caught([pins.test_tp_backward_euler_identities_and_fd])
+    assert _caught([lambda: pins.test_tp_backward_euler_identities_and_fd("uvu")])
 
 
 def test_conv_double_scale(monkeypatch):
@@ -240,6 +244,75 @@ def test_right_default_path_weight_passes(monkeypatch):
     # the harness itself: the stated formula re-applied leaves every pin green
     _patch_alpha(monkeypatch, lambda l3, mv, no: np.sqrt((2 * l3 + 1) / (mv * no)))
     assert not _caught(ALPHA_PINS)
+
+
+MODE_PINS = [lambda: pins.test_tp_modes_brute_force("uuu"), lambda: pins.test_tp_modes_brute_force("uvw"),
+             lambda: pins.test_tp_modes_brute_force("uvw_fans"),
+             lambda: pins.test_default_path_weight_gives_unit_second_moment("uvw_fans"),
+             pins.test_modes_coincide_at_multiplicity_one, pins.test_uuu_is_uvu_on_the_diagonal,
+             pins.test_scalar_path_modes_closed_forms,
+             lambda: pins.test_default_path_weight_gives_unit_second_moment("uuu"),
+             lambda: pins.test_default_path_weight_gives_unit_second_moment("uvw"),
+             lambda: pins.test_tp_modes_equivariance_o3("uuu"), lambda: pins.test_tp_modes_equivariance_o3("uvw"),
+             lambda: pins.test_tp_backward_euler_identities_and_fd("uuu"),
+             lambda: pins.test_tp_backward_euler_identities_and_fd("uvw")]
+
+
+@pytest.mark.parametrize("mode,eq", [
+    ("uuu", "bui,bvj,ijk,bu->buk"),      # y summed over all channels instead of tied
+    ("uvw", "bui,bvj,ijk,bvuw->bwk"),    # u and v of the weights transposed
+])
+def test_mode_forward_wrong_contraction(monkeypatch, mode, eq):
+    monkeypatch.setitem(otp._FWD, mode, eq)
+    assert _caught(MODE_PINS)
+
+
+@pytest.mark.parametrize("mode", ["uuu", "uvw"])
+def test_mode_weights_reversed(monkeypatch, mode):
+    orig = otp._weights
+
+    def bad(plan, w, p, bsz):
+        ws = orig(plan, w, p, bsz)
+        if plan.mode != mode:
+            return ws
+        return np.ascontiguousarray(ws.reshape(bsz, -1)[:, ::-1]).reshape(ws.shape)
+
+    monkeypatch.setattr(otp, "_weights", bad)
+    assert _caught(MODE_PINS)
+
+
+@pytest.mark.parametrize("mode,table,eq", [
+    ("uuu", "_DX", "bvj,ijk,bu,buk->bui"),      # y summed over channels
+    ("uuu", "_DW", "bui,bvj,ijk,buk->bu"),      # y summed over channels
+    ("uvw", "_DY", "bui,ijk,bvuw,bwk->bvj"),    # weights' u and v transposed (square paths)
+    ("uvw", "_DW", "bui,bvj,ijk,bwk->bvuw"),    # weights' u and v transposed (square paths)
+])
+def test_mode_backward_wrong_contraction(monkeypatch, mode, table, eq):
+    monkeypatch.setitem(getattr(otp, table), mode, eq)
+    assert _caught(MODE_PINS)
+
+
+@pytest.mark.parametrize("mode,fan_in,wrong", [
+    ("uuu", lambda a, b: b, True), ("uvw", lambda a, b: b, True), ("uvw", lambda a, b: a, True),
+    ("uuu", lambda a, b: 1, False), ("uvw", lambda a, b: a * b, False),   # the harness: the stated fans pass
+])
+def test_mode_wrong_default_path_weight(monkeypatch, mode, fan_in, wrong):
+    orig = otp.make_plan
+
+    def bad(*args, **kwargs):
+        plan = orig(*args, **kwargs)
+        if plan.mode == mode:
+            n_out = {}
+            for ins in plan.instructions:
+                n_out[ins.i_out] = n_out.get(ins.i_out, 0) + 1
+            plan.alphas = [np.sqrt((2 * plan.irreps_out[i.i_out].l + 1)
+                                   / (fan_in(plan.irreps_in1[i.i_in1].mul, plan.irreps_in2[i.i_in2].mul) * n_out[i.i_out]))
+                           for i in plan.instructions]
+        return plan
+
+    monkeypatch.setattr(otp, "make_plan", bad)
+    monkeypatch.setattr(oracle, "make_plan", bad)
+    assert _caught(MODE_PINS) == wrong
 
 
 def _patch_radial(monkeypatch, name, fn):

@@ -240,6 +240,18 @@ def test_real_cg_gaunt_property(l1, l2):
 
 
 # --------------------------------------------------------------- tensor product ---
+def _channel_triples(mode, a, bb, c):
+    """(u, v, w_out, weight index within the path) of every channel coupling of one instruction:
+    uvu ties w_out = u and sums v; uuu ties all three; uvw couples every (u, v) with every w_out
+    (e3nn course, lesson 03b: the connection mode of an instruction)."""
+    if mode == "uvu":
+        return [(u, v, u, u * bb.mul + v) for u in range(a.mul) for v in range(bb.mul)]
+    if mode == "uuu":
+        return [(u, u, u, u) for u in range(a.mul)]
+    return [(u, v, k, (u * bb.mul + v) * c.mul + k)
+            for u in range(a.mul) for v in range(bb.mul) for k in range(c.mul)]
+
+
 def brute_tp(plan, x, y, w):
     """Pure-Python loops over every index of the definition (tiny inputs only)."""
     out = np.zeros((x.shape[0], plan.irreps_out.dim))
@@ -249,17 +261,31 @@ def brute_tp(plan, x, y, w):
             a, c = plan.irreps_in1[ins.i_in1], plan.irreps_out[ins.i_out]
             bb = plan.irreps_in2[ins.i_in2]
             C = real_cg(a.l, bb.l, c.l)
-            for u in range(a.mul):
-                for v in range(bb.mul):
-                    wt = w[b, plan.weight_offsets[p] + u * bb.mul + v]
-                    for i in range(2 * a.l + 1):
-                        for j in range(2 * bb.l + 1):
-                            for k in range(2 * c.l + 1):
-                                out[b, o3s[ins.i_out] + u * (2 * c.l + 1) + k] += (
-                                    plan.alphas[p] * wt * C[i, j, k]
-                                    * x[b, o1s[ins.i_in1] + u * (2 * a.l + 1) + i]
-                                    * y[b, o2s[ins.i_in2] + v * (2 * bb.l + 1) + j])
+            for u, v, wo, q in _channel_triples(plan.mode, a, bb, c):
+                wt = w[b, plan.weight_offsets[p] + q]
+                for i in range(2 * a.l + 1):
+                    for j in range(2 * bb.l + 1):
+                        for k in range(2 * c.l + 1):
+                            out[b, o3s[ins.i_out] + wo * (2 * c.l + 1) + k] += (
+                                plan.alphas[p] * wt * C[i, j, k]
+                                * x[b, o1s[ins.i_in1] + u * (2 * a.l + 1) + i]
+                                * y[b, o2s[ins.i_in2] + v * (2 * bb.l + 1) + j])
     return out
+
+
+def mode_plan(mode):
+    """A small plan of each connection mode: several channels, a collapsed output (two paths into
+    one block), and for uvw output multiplicities that differ from the inputs'."""
+    if mode == "uuu":
+        return oracle.make_plan("2x0e+2x1o+2x2e", "2x0e+2x1o+2x2e", lmax_out=2, mode="uuu")
+    if mode == "uvw":
+        return oracle.make_plan("2x0e+2x1o", "2x1o+2x0e", "1x1o+3x0e+2x1e",
+                                instructions=[(0, 0, 0), (1, 1, 0), (1, 0, 1), (1, 0, 2)], mode="uvw")
+    if mode == "uvw_fans":  # two paths into one block with channel fans 2 x 3 and 1 x 2
+        return oracle.make_plan("2x0e+1x1o", "3x1o+2x0e", "1x1o+3x0e+2x1e",
+                                instructions=[(0, 0, 0), (1, 1, 0), (1, 0, 1), (1, 0, 2)], mode="uvw")
+    return oracle.make_plan("2x0e+2x1o", "3x1o", "2x1o+2x0e+2x1e",
+                            instructions=[(0, 0, 0), (1, 0, 1), (1, 0, 2)], mode="uvu")
 
 
 def test_tp_matches_brute_force_loops():
@@ -279,6 +305,72 @@ def test_tp_multiplicity_two_inputs_brute_force():
     y = rng.standard_normal((2, plan.irreps_in2.dim))
     w = rng.standard_normal((2, plan.weight_numel))
     np.testing.assert_allclose(oracle.tp_forward(plan, x, y, w), brute_tp(plan, x, y, w), atol=1e-13)
+
+
+@pytest.mark.parametrize("mode", ["uvu", "uuu", "uvw", "uvw_fans"])
+def test_tp_modes_brute_force(mode):
+    rng = np.random.default_rng(7)
+    plan = mode_plan(mode)
+    x = rng.standard_normal((2, plan.irreps_in1.dim))
+    y = rng.standard_normal((2, plan.irreps_in2.dim))
+    w = rng.standard_normal((2, plan.weight_numel))
+    assert plan.weight_numel == sum(len(_channel_triples(plan.mode, plan.irreps_in1[i.i_in1], plan.irreps_in2[i.i_in2],
+                                                         plan.irreps_out[i.i_out])) for i in plan.instructions)
+    np.testing.assert_allclose(oracle.tp_forward(plan, x, y, w), brute_tp(plan, x, y, w), atol=1e-13)
+
+
+def test_modes_coincide_at_multiplicity_one():
+    """With one channel everywhere the three connection modes are the same map, default path
+    weights included (each output element then sums exactly one channel product)."""
+    rng = np.random.default_rng(8)
+    plans = [oracle.make_plan("1x0e+1x1o+1x2e", "1x0e+1x1o+1x2e", lmax_out=2, mode=m) for m in ("uvu", "uuu", "uvw")]
+    x = rng.standard_normal((3, plans[0].irreps_in1.dim))
+    y = rng.standard_normal((3, plans[0].irreps_in2.dim))
+    w = rng.standard_normal((3, plans[0].weight_numel))
+    outs = [oracle.tp_forward(p, x, y, w) for p in plans]
+    assert plans[0].alphas == plans[1].alphas == plans[2].alphas
+    np.testing.assert_allclose(outs[1], outs[0], atol=1e-14)
+    np.testing.assert_allclose(outs[2], outs[0], atol=1e-14)
+
+
+def test_uuu_is_uvu_on_the_diagonal():
+    """uuu equals uvu whose weight matrix per path is diagonal in (u, v), up to the default path
+    weight: uvu normalises by the channel count of y, uuu by one channel."""
+    rng = np.random.default_rng(9)
+    pu = oracle.make_plan("3x0e+3x1o", "3x0e+3x1o", lmax_out=1, mode="uuu")
+    pv = oracle.make_plan("3x0e+3x1o", "3x0e+3x1o", lmax_out=1, mode="uvu")
+    x = rng.standard_normal((2, pu.irreps_in1.dim))
+    y = rng.standard_normal((2, pu.irreps_in2.dim))
+    wu = rng.standard_normal((2, pu.weight_numel))
+    wv = np.zeros((2, pv.weight_numel))
+    for p in range(pu.n_paths):
+        for u in range(3):
+            wv[:, pv.weight_offsets[p] + u * 3 + u] = wu[:, pu.weight_offsets[p] + u] * pu.alphas[p] / pv.alphas[p]
+    np.testing.assert_allclose(oracle.tp_forward(pu, x, y, wu), oracle.tp_forward(pv, x, y, wv), atol=1e-13)
+    assert all(abs(a / b - math.sqrt(3)) < 1e-14 for a, b in zip(pu.alphas, pv.alphas))
+
+
+def test_scalar_path_modes_closed_forms():
+    """0e x 0e -> 0e with C = 1: uuu is the channelwise product w_u x_u y_u (alpha 1); uvw is the
+    bilinear form sum_uv W_uvw x_u y_v / sqrt(mul_x mul_y)."""
+    rng = np.random.default_rng(10)
+    x, y = rng.standard_normal((4, 3)), rng.standard_normal((4, 3))
+    pu = oracle.make_plan("3x0e", "3x0e", lmax_out=0, mode="uuu")
+    w = rng.standard_normal((4, 3))
+    np.testing.assert_allclose(oracle.tp_forward(pu, x, y, w), w * x * y, atol=1e-15)
+    pw = oracle.make_plan("3x0e", "3x0e", "2x0e", instructions=[(0, 0, 0)], mode="uvw")
+    W = rng.standard_normal((4, 3, 3, 2))
+    want = np.einsum("buvw,bu,bv->bw", W, x, y) / 3.0
+    np.testing.assert_allclose(oracle.tp_forward(pw, x, y, W.reshape(4, -1)), want, atol=1e-14)
+
+
+def test_mode_validation():
+    with pytest.raises(ValueError):
+        oracle.make_plan("2x1o", "3x1o", lmax_out=2, mode="uuu")  # uuu ties x and y channels
+    with pytest.raises(ValueError):
+        oracle.make_plan("2x1o", "1x1o", "3x0e", instructions=[(0, 0, 0)], mode="uvu")  # uvu ties x and out
+    with pytest.raises(ValueError):
+        oracle.make_plan("1x1o", "1x1o", lmax_out=2, mode="uvv")
 
 
 def test_tp_scalar_path():
@@ -303,7 +395,7 @@ def _trilinear_coefficients(plan):
     return T
 
 
-@pytest.mark.parametrize("case", ["uncollapsed", "collapsed", "mul_y2"])
+@pytest.mark.parametrize("case", ["uncollapsed", "collapsed", "mul_y2", "uuu", "uvw", "uvw_fans"])
 def test_default_path_weight_gives_unit_second_moment(case):
     """The default path weight alpha_p is fixed by one property (e3nn course, lesson 03b: paths
     are normalised so that the output keeps the scale of the inputs): when every component of x,
@@ -315,9 +407,11 @@ def test_default_path_weight_gives_unit_second_moment(case):
     elif case == "collapsed":  # two paths share each output block: n_out = 2
         plan = oracle.make_plan("1x1o+1x2o", "1x1o", "1x1e+1x2e",
                                 instructions=[(0, 0, 0), (1, 0, 0), (1, 0, 1)])
-    else:  # uvu with two channels of y: sum over v with a weight per (u, v)
+    elif case == "mul_y2":  # uvu with two channels of y: sum over v with a weight per (u, v)
         plan = oracle.make_plan("2x1o", "2x1o+2x2e", "2x0e+2x1e+2x2o+2x3o",
                                 instructions=[(0, 0, 0), (0, 0, 1), (0, 1, 2), (0, 1, 3)])
+    else:  # the other connection modes (uuu: one channel per output; uvw: mul_x * mul_y)
+        plan = mode_plan(case)
     T = _trilinear_coefficients(plan)
     moment = (T * T).sum(axis=(1, 2, 3))
     np.testing.assert_allclose(moment, 1.0, rtol=1e-12)
@@ -418,9 +512,29 @@ def test_tp_equivariance_o3(flip):
     np.testing.assert_allclose(out_rot, _rep(plan.irreps_out, Ds, flip, out), atol=1e-12)
 
 
-def test_tp_backward_euler_identities_and_fd():
+@pytest.mark.parametrize("mode", ["uuu", "uvw"])
+def test_tp_modes_equivariance_o3(mode):
+    """Rotating (and reflecting) both inputs of a uuu or uvw product rotates its output; y here is
+    a general feature (several channels), not only harmonics."""
+    rng = np.random.default_rng(13)
+    plan = (oracle.make_plan("2x0e+2x1o+2x2e+2x3o", "2x0e+2x1o+2x2e+2x3o", lmax_out=3, mode="uuu") if mode == "uuu"
+            else oracle.make_plan("2x0e+2x1o+1x2e", "2x1o+1x2o", lmax_out=3, mode="uvw"))
+    R = rand_rot(rng)
+    Ds = {l: wigner_real(l, R, rng) for l in range(4)}
+    x = rng.standard_normal((3, plan.irreps_in1.dim))
+    y = rng.standard_normal((3, plan.irreps_in2.dim))
+    w = rng.standard_normal((3, plan.weight_numel))
+    out = oracle.tp_forward(plan, x, y, w)
+    for flip in (False, True):
+        out_rot = oracle.tp_forward(plan, _rep(plan.irreps_in1, Ds, flip, x), _rep(plan.irreps_in2, Ds, flip, y), w)
+        np.testing.assert_allclose(out_rot, _rep(plan.irreps_out, Ds, flip, out), atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", ["uvu", "uuu", "uvw"])
+def test_tp_backward_euler_identities_and_fd(mode):
     rng = np.random.default_rng(12)
-    plan = oracle.make_plan("2x0e+2x1o+2x2e", "1x0e+1x1o+1x2e+1x3o", lmax_out=2)
+    plan = {"uvu": lambda: oracle.make_plan("2x0e+2x1o+2x2e", "1x0e+1x1o+1x2e+1x3o", lmax_out=2),
+            "uuu": lambda: mode_plan("uuu"), "uvw": lambda: mode_plan("uvw")}[mode]()
     B = 4
     x = rng.standard_normal((B, plan.irreps_in1.dim))
     y = rng.standard_normal((B, plan.irreps_in2.dim))
