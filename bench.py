@@ -62,6 +62,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-tp", action="store_true", help="skip the tensor-product (no graph) measurement")
+    ap.add_argument("--no-uuu", action="store_true", help="skip the channelwise (uuu) tensor-product measurement")
     ap.add_argument("--no-waterbox", action="store_true", help="skip the second (water-box) block")
     ap.add_argument("--no-scrub", action="store_true", help="skip the L2-scrubbed per-kernel statistics")
     ap.add_argument("--no-radial", action="store_true", help="skip the radial-network (tensor core) measurement")
@@ -282,19 +283,26 @@ def run_reference(args):
     return 0
 
 
-def measure_tp(args, dev):
-    """Tensor product without a graph (per-sample x, harmonics and weights) on the batched
-    workload, forward and backward, CUDA events; inputs (several GB) are larger than L2."""
+def measure_tp(args, dev, name="tp_batched"):
+    """Tensor product without a graph, forward and backward, CUDA events; inputs (several GB) are
+    larger than L2.  tp_batched: uvu with per-sample x, harmonics and weights; tp_uuu: the
+    channelwise mode with per-sample x, y (128 channels each) and weights."""
     import torch
     from mlip_message_passing_b200 import e3b, workloads as W
 
-    cfg = W.CONFIGS["tp_batched"]
+    cfg = W.CONFIGS[name]
     B, mul, lx, ly, lo = cfg["B"], cfg["mul"], cfg["lx"], cfg["ly"], cfg["lo"]
-    plan = e3b.Plan(W.irreps_str(mul, lx), W.sh_irreps(ly), lmax_out=lo)
     gen = torch.Generator(device=dev).manual_seed(cfg["seed"])
-    vec = torch.randn(B, 3, generator=gen, device=dev)
-    vec /= vec.norm(dim=1, keepdim=True)
-    y = e3b.spherical_harmonics(ly, vec)
+    if name == "tp_uuu":
+        irreps_y = W.irreps_str(mul, ly)
+        plan = e3b.Plan(W.irreps_str(mul, lx), irreps_y, lmax_out=lo, mode="uuu")
+        y = torch.randn(B, plan.dim_in2, generator=gen, device=dev)
+    else:
+        irreps_y = W.sh_irreps(ly)
+        plan = e3b.Plan(W.irreps_str(mul, lx), irreps_y, lmax_out=lo)
+        vec = torch.randn(B, 3, generator=gen, device=dev)
+        vec /= vec.norm(dim=1, keepdim=True)
+        y = e3b.spherical_harmonics(ly, vec)
     x = torch.randn(B, plan.dim_in1, generator=gen, device=dev)
     w = torch.randn(B, plan.weight_numel, generator=gen, device=dev)
     go = torch.randn(B, plan.dim_out, generator=gen, device=dev)
@@ -312,7 +320,7 @@ def measure_tp(args, dev):
                                e3b._stream())
 
     res = {}
-    for name, fn in (("fwd", fwd), ("bwd", bwd)):
+    for part, fn in (("fwd", fwd), ("bwd", bwd)):
         for _ in range(args.warmup):
             fn()
         torch.cuda.synchronize()
@@ -325,17 +333,17 @@ def measure_tp(args, dev):
             ev.append((a, b))
         torch.cuda.synchronize()
         e3b.device_status()
-        res[name] = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+        res[part] = statistics.fmean(a.elapsed_time(b) for a, b in ev)
     dx, dy, dw, do = plan.dim_in1, plan.dim_in2, plan.weight_numel, plan.dim_out
     nbytes = {"fwd": 4 * B * (dx + dy + dw + do), "bwd": 4 * B * (2 * dx + 2 * dy + 2 * dw + do)}
     peak, _ = hbm_peak()
-    line = {"workload": f"tp_batched: B={B}, {W.irreps_str(mul, lx)} x {W.sh_irreps(ly)} -> l<={lo}, "
-                        f"{plan.n_paths} paths, fp32"}
-    for name in ("fwd", "bwd"):
-        ms = res[name]
-        gbs = nbytes[name] / (ms * 1e-3) / 1e9
-        line[name] = {"ms": ms, "samples_per_s": B / (ms * 1e-3), "GBps": gbs, "frac_of_hbm": gbs / peak,
-                      "frac_of_nominal": gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": nbytes[name]}
+    line = {"workload": f"{name}: B={B}, {W.irreps_str(mul, lx)} x {irreps_y} -> l<={lo}, "
+                        f"{plan.n_paths} paths, {'uuu' if name == 'tp_uuu' else 'uvu'}, fp32"}
+    for part in ("fwd", "bwd"):
+        ms = res[part]
+        gbs = nbytes[part] / (ms * 1e-3) / 1e9
+        line[part] = {"ms": ms, "samples_per_s": B / (ms * 1e-3), "GBps": gbs, "frac_of_hbm": gbs / peak,
+                      "frac_of_nominal": gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": nbytes[part]}
     del x, y, w, go, out, gx, gy, gw, ws
     torch.cuda.empty_cache()
     return line
@@ -767,6 +775,7 @@ def run_native(args):
         return 0
 
     tp = None if args.no_tp else measure_tp(args, dev)
+    uuu = None if args.no_uuu else measure_tp(args, dev, "tp_uuu")
     cfg, irreps_x, irreps_y = workload_spec(args.workload)
     cpu = None
     if not args.no_cpu_baseline:
@@ -799,6 +808,7 @@ def run_native(args):
                            "L2 scrubbed before each launch"},
         "waterbox": water,
         "tp": tp,
+        "uuu": uuu,
         "radial": radial,
         "roofline": head["roofline"],
         "cpu_baseline": cpu,

@@ -78,7 +78,10 @@ typedef enum {
 
 typedef enum { E3_F32 = 0, E3_F64 = 1 } e3_dtype;
 
-/* Connection modes of lesson 03b [TP].  Only E3_UVU has kernels; others -> UNSUPPORTED. */
+/* Connection modes of lesson 03b [TP]: which channel indices an instruction ties.
+ *   E3_UVU  out[u] = sum_v w[u,v] (x[u] (x) y[v])            tensor product and convolution
+ *   E3_UUU  out[u] = w[u] (x[u] (x) y[u])                      tensor product only
+ *   E3_UVW, E3_UUW                                             no kernels -> UNSUPPORTED */
 typedef enum { E3_UVU = 0, E3_UVW = 1, E3_UUU = 2, E3_UUW = 3 } e3_mode;
 
 /* SH normalisations of lesson 02b [SH]: component (sum_m Y^2 = 2l+1), integral
@@ -104,6 +107,11 @@ typedef struct e3_plan e3_plan;
  *               l = 0..Lx in ascending order (any parities), one common multiplicity C with
  *               C % 4 == 0, Lx <= 3.
  *   irreps_in2  edge attributes, e.g. "1x0e+1x1o+1x2e+1x3o": multiplicity 1, l = 0..Ly, Ly <= 3.
+ *               In the uuu mode the multiplicity is C (one y channel per x channel), and C
+ *               may be any positive number.
+ *   mode        E3_UVU or E3_UUU.  Weights per path: C (uvu with one y channel, one weight per
+ *               (u, v)) or C (uuu, one per u); default alpha_p = sqrt((2 l3 + 1) / (fan * n_out))
+ *               with fan = mul_in2 (uvu) or 1 (uuu), n_out = instructions writing the block.
  *   irreps_out  with n_instr == 0: a filter listing the output irreps allowed (multiplicities
  *               ignored; NULL or "" = all); instructions are then enumerated as
  *               for i1, for i2, for l3 = |l1-l2| .. l1+l2 with (l3, p1 p2) in the filter,

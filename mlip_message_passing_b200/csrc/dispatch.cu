@@ -12,7 +12,6 @@
 
 namespace e3b {
 
-#define E3_CONFIGS(X) X(1, 1, 2) X(1, 2, 2) X(2, 3, 2) X(3, 3, 3)
 #define E3_DECL(A, B, C)                                                              \
   e3_status upload_tables_l##A##B##C(const double* t64, const float* t32);            \
   e3_status launch_fwd_l##A##B##C(const e3_plan* plan, const FwdArgs& a, bool conv);   \
@@ -42,6 +41,10 @@ e3_status ensure_device_tables() {
   }
   E3_CONFIGS(E3_UP)
 #undef E3_UP
+  {
+    const e3_status st = upload_tables_uuu(t.data(), tf.data());
+    if (st != E3_OK) return st;
+  }
   const int zero = 0;
   cudaError_t err = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
   if (err == cudaSuccess) err = cudaGetSymbolAddress(reinterpret_cast<void**>(&g_status_ptr[dev]), g_status);

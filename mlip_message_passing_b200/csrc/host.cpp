@@ -356,7 +356,7 @@ extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_i
           for (const auto& f : irf) ok = ok || (f.l == l3 && f.p == p3);
           if (!ok) continue;
           ins.push_back({i1, i2, int(out_irreps.size()), -1.0});
-          out_irreps.push_back({a.mul, l3, p3});  // uvu: output channel u of x
+          out_irreps.push_back({a.mul, l3, p3});  // uvu and uuu: output channel u of x
         }
       }
     if (ins.empty()) return fail(E3_ERR_INSTRUCTION, "no allowed path between the inputs and the output filter");
@@ -373,14 +373,17 @@ extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_i
                     q, a.l, b.l, c.l);
       if (c.p != a.p * b.p)
         return fail(E3_ERR_INSTRUCTION, "instruction %d: parity rule p3 = p1 p2 fails", q);
-      if (mode == E3_UVU && c.mul != a.mul)
-        return fail(E3_ERR_INSTRUCTION, "instruction %d: uvu needs mul_out == mul_in1", q);
+      if ((mode == E3_UVU || mode == E3_UUU) && c.mul != a.mul)
+        return fail(E3_ERR_INSTRUCTION, "instruction %d: %s needs mul_out == mul_in1", q, mode == E3_UVU ? "uvu" : "uuu");
+      if (mode == E3_UUU && b.mul != a.mul)
+        return fail(E3_ERR_INSTRUCTION, "instruction %d: uuu needs mul_in2 == mul_in1", q);
       if (!s.has_weight)
         return fail(E3_ERR_UNSUPPORTED, "instruction %d: paths without weights have no kernel", q);
       ins.push_back({s.i_in1, s.i_in2, s.i_out, s.path_weight});
     }
   }
-  if (mode != E3_UVU) return fail(E3_ERR_UNSUPPORTED, "only the uvu connection mode has kernels");
+  if (mode != E3_UVU && mode != E3_UUU)
+    return fail(E3_ERR_UNSUPPORTED, "the uvu and uuu connection modes have kernels; this mode has none");
 
   // layout the kernels are compiled for
   const int C = ir1[0].mul;
@@ -388,11 +391,13 @@ extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_i
     if (ir1[i].l != i || ir1[i].mul != C)
       return fail(E3_ERR_UNSUPPORTED,
                   "irreps_in1 must be Cx0+Cx1+..+CxLx (one block per degree, ascending, common multiplicity)");
+  const int mul2 = mode == E3_UUU ? C : 1;
   for (int i = 0; i < int(ir2.size()); ++i)
-    if (ir2[i].l != i || ir2[i].mul != 1)
-      return fail(E3_ERR_UNSUPPORTED, "irreps_in2 must be 1x0+1x1+..+1xLy");
+    if (ir2[i].l != i || ir2[i].mul != mul2)
+      return fail(E3_ERR_UNSUPPORTED, mode == E3_UUU ? "irreps_in2 must be Cx0+Cx1+..+CxLy in the uuu mode"
+                                                      : "irreps_in2 must be 1x0+1x1+..+1xLy");
   const int LX = int(ir1.size()) - 1, LY = int(ir2.size()) - 1;
-  if (C % 4 != 0 || !((C / 4) <= 32 ? (32 % (C / 4) == 0) : ((C / 4) % 32 == 0)))
+  if (mode == E3_UVU && (C % 4 != 0 || !((C / 4) <= 32 ? (32 % (C / 4) == 0) : ((C / 4) % 32 == 0))))
     return fail(E3_ERR_UNSUPPORTED, "multiplicity %d: kernels need C in {4, 8, 16, 32, 64} or a multiple of 128", C);
   int LO = 0;
   for (const auto& s : ins) LO = std::max(LO, out_irreps[s.io].l);
@@ -421,6 +426,7 @@ extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_i
   }
   plan->dtype = dtype;
   plan->wmode = wmode;
+  plan->mode = mode;
   plan->C = C;
   plan->LX = LX;
   plan->LY = LY;
@@ -433,7 +439,10 @@ extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_i
     plan->l1.push_back(ir1[ins[p].i1].l);
     plan->l2.push_back(b.l);
     plan->l3.push_back(c.l);
-    plan->alpha.push_back(ins[p].pw >= 0 ? ins[p].pw : std::sqrt((2.0 * c.l + 1.0) / (b.mul * n_out[ins[p].io])));
+    // default path weight: unit second moment of every output component for unit-variance
+    // inputs; the fan-in of one output element is mul_in2 channels in uvu and one in uuu
+    const double fan_in = mode == E3_UUU ? 1.0 : double(b.mul);
+    plan->alpha.push_back(ins[p].pw >= 0 ? ins[p].pw : std::sqrt((2.0 * c.l + 1.0) / (fan_in * n_out[ins[p].io])));
   }
   for (const auto& a : ir1) plan->dim1 += int64_t(a.mul) * (2 * a.l + 1);
   for (const auto& b : ir2) plan->dim2 += int64_t(b.mul) * (2 * b.l + 1);
@@ -533,6 +542,23 @@ static e3_status check_plan_device(const e3_plan* plan) {
       return fail(E3_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);        \
   } while (0)
 
+static UuuArgs uuu_args(const e3_plan* plan, int64_t B, const void* x, const void* y, const void* w,
+                        int64_t w_stride, void* stream) {
+  UuuArgs u{};
+  u.B = B;
+  u.C = plan->C;
+  u.dim1 = plan->dim1;
+  u.dim2 = plan->dim2;
+  u.dim_out = plan->dim_out;
+  u.x = x;
+  u.y = y;
+  u.w = w;
+  u.w_stride = w_stride;
+  u.stream = stream;
+  for (int p = 0; p < plan->n_paths && p < UUU_MAXP; ++p) u.alpha[p] = plan->alpha[p];
+  return u;
+}
+
 extern "C" e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x, const void* y, const void* w,
                                    void* out, void* stream) {
   clear_error();
@@ -555,6 +581,11 @@ extern "C" e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x
   a.scale = 1.0;
   a.out = out;
   a.stream = stream;
+  if (plan->mode == E3_UUU) {
+    UuuArgs u = uuu_args(plan, B, x, y, w, a.w_stride, stream);
+    u.out = out;
+    return launch_uuu(plan, u, false);
+  }
   return launch_forward(plan, a, false);
 }
 
@@ -572,6 +603,7 @@ extern "C" e3_status e3_conv_workspace_size(const e3_plan* plan, int64_t N, int6
   clear_error();
   if (plan == nullptr || bytes == nullptr) return fail(E3_ERR_INVALID_ARG, "plan or bytes is NULL");
   if (N < 0 || E < 0 || N >= (int64_t(1) << 31) || E >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N or E out of range");
+  if (plan->mode != E3_UVU) return fail(E3_ERR_UNSUPPORTED, "the convolution has kernels for the uvu mode only");
   *bytes = conv_workspace_bytes(plan, N, E, plan_groups(plan));
   return E3_OK;
 }
@@ -629,11 +661,20 @@ extern "C" e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* 
   a.grad_y = grad_y;
   a.grad_w = grad_w;
   a.stream = stream;
+  if (plan->mode == E3_UUU) {
+    UuuArgs u = uuu_args(plan, B, x, y, w, plan->weight_numel, stream);
+    u.grad_out = grad_out;
+    u.grad_x = grad_x;
+    u.grad_y = grad_y;
+    u.grad_w = grad_w;
+    return launch_uuu(plan, u, true);
+  }
   return launch_backward(plan, a, false);
 }
 
 static e3_status check_conv_common(const e3_plan* plan, int64_t N, int64_t E, const void* y, const void* vec,
                                    e3_sh_norm sh_norm) {
+  if (plan->mode != E3_UVU) return fail(E3_ERR_UNSUPPORTED, "the convolution has kernels for the uvu mode only");
   if (N < 0 || N >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "N = %lld out of range", (long long)N);
   if (E < 0 || E >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "E = %lld out of range", (long long)E);
   if (E > 0 && (y == nullptr) == (vec == nullptr)) return fail(E3_ERR_INVALID_ARG, "give exactly one of y and edge_vec");

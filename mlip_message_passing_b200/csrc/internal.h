@@ -11,7 +11,8 @@ struct e3_plan {
   int device = 0;
   e3_dtype dtype = E3_F32;
   e3_weight_mode wmode = E3_W_PER_SAMPLE;
-  int C = 0;                      // common multiplicity of the x irreps
+  e3_mode mode = E3_UVU;
+  int C = 0;                      // common multiplicity of the x irreps (and of y in uuu)
   int LX = 0, LY = 0, LO = 0;     // degree range of x, y and the output
   int n_paths = 0;
   std::vector<int> l1, l2, l3;    // per path
@@ -21,6 +22,9 @@ struct e3_plan {
 };
 
 namespace e3b {
+
+// Path sets (LX, LY, LO) with compiled kernels.
+#define E3_CONFIGS(X) X(1, 1, 2) X(1, 2, 2) X(2, 3, 2) X(3, 3, 3)
 
 // Thread-local error message; returns `st` so callers can `return fail(st, ...)`.
 e3_status fail(e3_status st, const char* fmt, ...);
@@ -149,6 +153,27 @@ inline size_t conv_workspace_bytes(const e3_plan* plan, int64_t N, int64_t E, in
   return b;
 }
 e3_status launch_backward(const e3_plan* plan, const BwdArgs& a, bool conv);
+
+// uuu tensor product (tp_uuu.cu): one thread per (sample, channel).
+constexpr int UUU_MAXP = 64;
+struct UuuArgs {
+  int64_t B;
+  int C;
+  int64_t dim1, dim2, dim_out;
+  const void* x;
+  const void* y;
+  const void* w;
+  int64_t w_stride;          // weight_numel, or 0 for shared weights (forward only)
+  void* out;                 // forward
+  const void* grad_out;      // backward
+  void* grad_x;              // backward, each optional
+  void* grad_y;
+  void* grad_w;
+  void* stream;
+  double alpha[UUU_MAXP];
+};
+e3_status upload_tables_uuu(const double* t64, const float* t32);
+e3_status launch_uuu(const e3_plan* plan, const UuuArgs& a, bool backward);
 // Zero rows [*first_row, n_rows) of a row-major array of row_bytes-byte rows (first_row read on
 // the device: the padding positions after the last CSR row).
 e3_status zero_rows_after(const int32_t* first_row, int64_t n_rows, int64_t row_bytes, void* ptr, void* stream);

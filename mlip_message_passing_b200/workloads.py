@@ -6,6 +6,7 @@ the smoke check so that the CUDA path and the float64 oracle see the same bytes.
 
 Recipes (numpy PCG64, ``default_rng(seed)``; draws in the order listed):
 
+* channelwise (uuu) product: x, y, w ~ N(0, 1) in that order;
 * batched product: edge-like vectors ~ N(0, 1) (or uniform on the sphere), then x ~ N(0, 1)
   [B, dim_x], then w ~ N(0, 1) [B, weight_numel];
 * water-box-like graph: N positions uniform in a periodic cube of side (N / 0.1)^(1/3) Angstrom
@@ -134,6 +135,8 @@ CONFIGS = {
     "conv_waterbox": dict(kind="conv", N=3000, mul=64, lx=2, ly=3, lo=2, seed=2),
     "conv_large": dict(kind="conv", N=24_000, mul=128, lx=3, ly=3, lo=3, seed=3),
     "conv_waterbox_bwd": dict(kind="conv", N=3000, mul=64, lx=2, ly=3, lo=2, seed=2, grad_seed=4),
+    # channelwise (uuu) product of two node-feature sets of 128 channels, degrees 0..3
+    "tp_uuu": dict(kind="tp_uuu", B=32_768, mul=128, lx=3, ly=3, lo=3, seed=5),
 }
 
 
@@ -156,6 +159,16 @@ def tp_inputs(B, mul, lx, ly, lo, seed, vectors="normal", dtype=np.float32):
     x = rng.standard_normal((B, mul * (lx + 1) ** 2)).astype(dtype)
     w = rng.standard_normal((B, n_paths(lx, ly, lo) * mul)).astype(dtype)
     return dict(vec=v, x=x, w=w)
+
+
+def channel_inputs(B, mul, lx, ly, lo, seed, dtype=np.float32):
+    """Inputs of a channelwise (uuu) product: x [B, mul (lx+1)^2], y [B, mul (ly+1)^2] and
+    w [B, P mul], all N(0, 1), drawn in that order."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, mul * (lx + 1) ** 2)).astype(dtype)
+    y = rng.standard_normal((B, mul * (ly + 1) ** 2)).astype(dtype)
+    w = rng.standard_normal((B, n_paths(lx, ly, lo) * mul)).astype(dtype)
+    return dict(x=x, y=y, w=w)
 
 
 def graph_inputs(N, mul, lx, ly, lo, seed, dtype=np.float32, weights="host", device=None):

@@ -93,6 +93,18 @@ def test_plan_unsupported(e3b):
     st, msg = _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", "1x0e+1x1o+1x2e")
     assert st == e3b.E3_ERR_UNSUPPORTED and "every path" in msg
     assert _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", dtype=7)[0] == e3b.E3_ERR_INVALID_ARG
+    assert _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", mode=3)[0] == e3b.E3_ERR_UNSUPPORTED
+    assert _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", mode=9)[0] == e3b.E3_ERR_INVALID_ARG
+
+
+def test_plan_uuu_validation(e3b):
+    # uuu ties the channels of both inputs: y needs the multiplicity of x
+    st, msg = _create(e3b, "8x0e+8x1o", "1x0e+1x1o", mode=2)
+    assert st == e3b.E3_ERR_UNSUPPORTED and "uuu" in msg
+    st, msg = _create(e3b, "8x1o", "4x1o", "8x0e", instr=[(0, 0, 0)], mode=2)
+    assert st == e3b.E3_ERR_INSTRUCTION and "mul_in2" in msg
+    st, msg = _create(e3b, "8x1o", "8x1o", "4x0e", instr=[(0, 0, 0)], mode=2)
+    assert st == e3b.E3_ERR_INSTRUCTION and "mul_out" in msg
 
 
 def test_supported_list(e3b):
