@@ -19,7 +19,7 @@ LIB = os.path.join(HERE, "libe3b.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVFLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include")]
-SOURCES = ["host.cpp", "dispatch.cu", "csr.cu", "sh.cu", "radial.cu", "tp_uuu.cu", "tp_conv_l112.cu", "tp_conv_l122.cu",
+SOURCES = ["host.cpp", "dispatch.cu", "csr.cu", "sh.cu", "radial.cu", "tp_uuu.cu", "tp_uvw.cu", "tp_conv_l112.cu", "tp_conv_l122.cu",
            "tp_conv_l232.cu", "tp_conv_l333.cu"]
 
 

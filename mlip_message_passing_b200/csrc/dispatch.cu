@@ -42,7 +42,8 @@ e3_status ensure_device_tables() {
   E3_CONFIGS(E3_UP)
 #undef E3_UP
   {
-    const e3_status st = upload_tables_uuu(t.data(), tf.data());
+    e3_status st = upload_tables_uuu(t.data(), tf.data());
+    if (st == E3_OK) st = upload_tables_uvw(t.data(), tf.data());
     if (st != E3_OK) return st;
   }
   const int zero = 0;

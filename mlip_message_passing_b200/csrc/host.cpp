@@ -3,6 +3,8 @@
 // launches work.  No CUDA kernels live here.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <climits>
 #include <cmath>
 #include <complex>
 #include <cstdarg>
@@ -314,6 +316,125 @@ extern "C" e3_status e3_cg_dense(int32_t l1, int32_t l2, int32_t l3, double* out
   return E3_OK;
 }
 
+e3_plan::~e3_plan() {
+  if (uvw_prep != nullptr) {
+    int cur = -1;
+    const bool restore = cudaGetDevice(&cur) == cudaSuccess && cur != device;
+    if (restore) cudaSetDevice(device);
+    cudaFree(uvw_prep);
+    if (restore) cudaSetDevice(cur);
+  }
+}
+
+// Plan of the fully connected (uvw) mode: x = Cx0+..+CxLx, y = 1x0+..+1xLy, output blocks of one
+// multiplicity Co; instructions given, or every (i1, i2, i_out) that the triangle and parity rules
+// allow, in that loop order.  Shared float32 weights W_p[u][w] (v has one value), alpha_p =
+// sqrt((2 l3 + 1) / (C n_out)).
+static e3_status create_uvw(const std::vector<IrrepT>& ir1, const std::vector<IrrepT>& ir2,
+                            const std::vector<IrrepT>& irf, bool have_out, const e3_instruction* instr,
+                            int32_t n_instr, e3_dtype dtype, e3_weight_mode wmode, e3_plan** plan_out) {
+  if (!have_out) return fail(E3_ERR_INSTRUCTION, "the uvw mode needs irreps_out");
+  struct Ins {
+    int i1, i2, io;
+    double pw;
+  };
+  std::vector<Ins> ins;
+  if (n_instr == 0) {
+    for (int i1 = 0; i1 < int(ir1.size()); ++i1)
+      for (int i2 = 0; i2 < int(ir2.size()); ++i2)
+        for (int io = 0; io < int(irf.size()); ++io)
+          if (triangle(ir1[i1].l, ir2[i2].l, irf[io].l) && irf[io].p == ir1[i1].p * ir2[i2].p)
+            ins.push_back({i1, i2, io, -1.0});
+  } else {
+    for (int q = 0; q < n_instr; ++q) {
+      const auto& s = instr[q];
+      if (s.i_in1 < 0 || s.i_in1 >= int(ir1.size()) || s.i_in2 < 0 || s.i_in2 >= int(ir2.size()) || s.i_out < 0 ||
+          s.i_out >= int(irf.size()))
+        return fail(E3_ERR_INSTRUCTION, "instruction %d: index out of range", q);
+      const auto &a = ir1[s.i_in1], &b = ir2[s.i_in2], &c = irf[s.i_out];
+      if (!triangle(a.l, b.l, c.l))
+        return fail(E3_ERR_INSTRUCTION, "instruction %d: triangle rule |l1-l2| <= l3 <= l1+l2 fails (%d,%d,%d)", q,
+                    a.l, b.l, c.l);
+      if (c.p != a.p * b.p) return fail(E3_ERR_INSTRUCTION, "instruction %d: parity rule p3 = p1 p2 fails", q);
+      if (!s.has_weight) return fail(E3_ERR_UNSUPPORTED, "instruction %d: paths without weights have no kernel", q);
+      ins.push_back({s.i_in1, s.i_in2, s.i_out, s.path_weight});
+    }
+  }
+  if (ins.empty()) return fail(E3_ERR_INSTRUCTION, "no allowed path between the inputs and irreps_out");
+  if (dtype != E3_F32) return fail(E3_ERR_UNSUPPORTED, "uvw kernels compute in float32 (tf32 tensor cores, three passes)");
+  if (wmode != E3_W_SHARED) return fail(E3_ERR_UNSUPPORTED, "uvw kernels take shared weights");
+  const int C = ir1[0].mul;
+  for (int i = 0; i < int(ir1.size()); ++i)
+    if (ir1[i].l != i || ir1[i].mul != C)
+      return fail(E3_ERR_UNSUPPORTED,
+                  "irreps_in1 must be Cx0+Cx1+..+CxLx (one block per degree, ascending, common multiplicity)");
+  for (int i = 0; i < int(ir2.size()); ++i)
+    if (ir2[i].l != i || ir2[i].mul != 1) return fail(E3_ERR_UNSUPPORTED, "irreps_in2 must be 1x0+1x1+..+1xLy");
+  const int Co = irf[0].mul;
+  for (const auto& c : irf)
+    if (c.mul != Co) return fail(E3_ERR_UNSUPPORTED, "uvw output blocks need one common multiplicity");
+  if (C % 32 != 0 || C > 128 || Co % 32 != 0 || Co > 128)
+    return fail(E3_ERR_UNSUPPORTED, "uvw kernels need multiplicities in {32, 64, 96, 128} (got %d and %d)", C, Co);
+  const int LX = int(ir1.size()) - 1, LY = int(ir2.size()) - 1;
+  int LO = 0;
+  for (const auto& c : irf) LO = std::max(LO, c.l);
+  if (LX > E3_LMAX || LY > E3_LMAX || LO > E3_LMAX) return fail(E3_ERR_UNSUPPORTED, "degrees above %d have no kernel", E3_LMAX);
+  if (int(ins.size()) > UVW_MAXP || int(irf.size()) > UVW_MAXT)
+    return fail(E3_ERR_UNSUPPORTED, "at most %d paths and %d output blocks", UVW_MAXP, UVW_MAXT);
+
+  auto* plan = new (std::nothrow) e3_plan();
+  if (plan == nullptr) return fail(E3_ERR_INVALID_ARG, "out of host memory");
+  if (cudaGetDevice(&plan->device) != cudaSuccess) {
+    delete plan;
+    return fail(E3_ERR_CUDA, "cudaGetDevice failed");
+  }
+  plan->dtype = dtype;
+  plan->wmode = wmode;
+  plan->mode = E3_UVW;
+  plan->C = C;
+  plan->Co = Co;
+  plan->LX = LX;
+  plan->LY = LY;
+  plan->LO = LO;
+  plan->n_paths = int(ins.size());
+  for (const auto& c : irf) {
+    plan->out_off.push_back(int(plan->dim_out));
+    plan->out_l.push_back(c.l);
+    plan->dim_out += int64_t(c.mul) * (2 * c.l + 1);
+  }
+  std::vector<int> n_out(irf.size(), 0);
+  for (const auto& s : ins) n_out[s.io] += 1;
+  for (const auto& s : ins) {
+    const int l1 = ir1[s.i1].l, l3 = irf[s.io].l;
+    plan->l1.push_back(l1);
+    plan->l2.push_back(ir2[s.i2].l);
+    plan->l3.push_back(l3);
+    plan->io.push_back(s.io);
+    plan->x_off.push_back(C * l1 * l1);
+    plan->g_off.push_back(plan->out_off[s.io]);
+    plan->alpha.push_back(s.pw >= 0 ? s.pw : std::sqrt((2.0 * l3 + 1.0) / (double(C) * n_out[s.io])));
+  }
+  plan->dim1 = int64_t(C) * (LX + 1) * (LX + 1);
+  plan->dim2 = int64_t(LY + 1) * (LY + 1);
+  plan->weight_numel = int64_t(plan->n_paths) * C * Co;
+  plan->irreps_out = irreps_to_string(irf);
+  packed_cg_table();
+  e3_status st = ensure_device_tables();
+  if (st == E3_OK) {
+    plan->uvw_prep_size = uvw_prep_bytes(plan->n_paths, C, Co);
+    if (cudaMalloc(&plan->uvw_prep, plan->uvw_prep_size) != cudaSuccess) {
+      plan->uvw_prep = nullptr;
+      st = fail(E3_ERR_CUDA, "allocating the weight staging buffer (%zu bytes) failed", plan->uvw_prep_size);
+    }
+  }
+  if (st != E3_OK) {
+    delete plan;
+    return st;
+  }
+  *plan_out = plan;
+  return E3_OK;
+}
+
 extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_in2,
                                     const char* irreps_out, const e3_instruction* instr,
                                     int32_t n_instr, e3_mode mode, e3_dtype dtype,
@@ -338,6 +459,7 @@ extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_i
     return fail(E3_ERR_IRREPS_PARSE, "irreps_out: %s", why.c_str());
   if (n_instr > 0 && !have_out)
     return fail(E3_ERR_INSTRUCTION, "explicit instructions need irreps_out");
+  if (mode == E3_UVW) return create_uvw(ir1, ir2, irf, have_out, instr, n_instr, dtype, wmode, plan_out);
 
   // instructions: (i1, i2, i_out, alpha_override); output irreps
   struct Ins {
@@ -383,7 +505,7 @@ extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_i
     }
   }
   if (mode != E3_UVU && mode != E3_UUU)
-    return fail(E3_ERR_UNSUPPORTED, "the uvu and uuu connection modes have kernels; this mode has none");
+    return fail(E3_ERR_UNSUPPORTED, "the uvu, uuu and uvw connection modes have kernels; this mode has none");
 
   // layout the kernels are compiled for
   const int C = ir1[0].mul;
@@ -559,6 +681,82 @@ static UuuArgs uuu_args(const e3_plan* plan, int64_t B, const void* x, const voi
   return u;
 }
 
+// Launch arguments of the uvw contraction.  Forward: targets are the output blocks, terms the paths
+// into each, input x.  grad_x: targets are the x blocks, terms the paths out of each, input grad_out.
+static e3_status uvw_gemm_args(const e3_plan* plan, int64_t B, bool fwd, const void* in, const void* y, void* out,
+                               UvwGemmArgs* a) {
+  *a = UvwGemmArgs{};
+  const int P = plan->n_paths, C = plan->C, Co = plan->Co;
+  a->B = B;
+  a->in = static_cast<const float*>(in);
+  a->in_stride = fwd ? plan->dim1 : plan->dim_out;
+  a->k_in = fwd ? C : Co;
+  a->y = static_cast<const float*>(y);
+  a->y_stride = plan->dim2;
+  a->out = static_cast<float*>(out);
+  a->out_stride = fwd ? plan->dim_out : plan->dim1;
+  a->N = fwd ? Co : C;
+  const size_t fwd_chunk = size_t(2) * Co * 32 * 4, bwd_chunk = size_t(2) * C * 32 * 4;
+  a->prep = static_cast<const unsigned char*>(plan->uvw_prep) + (fwd ? 0 : size_t(P) * (C / 32) * fwd_chunk);
+  a->b_chunk_bytes = uint32_t(fwd ? fwd_chunk : bwd_chunk);
+  const int nt = fwd ? int(plan->out_l.size()) : plan->LX + 1;
+  int64_t tiles = 0;
+  int nterm = 0;
+  for (int t = 0; t < nt; ++t) {
+    UvwTarget& tg = a->tg[t];
+    tg.l = fwd ? plan->out_l[t] : t;
+    tg.off = fwd ? plan->out_off[t] : C * t * t;
+    tg.bt = 128 / (2 * tg.l + 1);
+    tg.tile_begin = int32_t(tiles);
+    tg.term_begin = nterm;
+    for (int p = 0; p < P; ++p) {
+      if ((fwd ? plan->io[p] : plan->l1[p]) != t) continue;
+      UvwTerm& tm = a->term[nterm++];
+      tm.in_off = fwd ? plan->x_off[p] : plan->g_off[p];
+      tm.l_in = fwd ? plan->l1[p] : plan->l3[p];
+      tm.l2 = plan->l2[p];
+      tm.chunk0 = fwd ? p * (C / 32) : p * (Co / 32);
+      tm.alpha = float(plan->alpha[p]);
+    }
+    tg.term_end = nterm;
+    tiles += (B + tg.bt - 1) / tg.bt;
+  }
+  if (tiles >= INT32_MAX) return fail(E3_ERR_SHAPE, "B = %lld is too large", (long long)B);
+  a->n_targets = nt;
+  a->total_tiles = int32_t(tiles);
+  a->wait_ns = test_wait_limit_ns();
+  return device_status_ptr(&a->status);
+}
+
+static UvwBwdArgs uvw_bwd_args(const e3_plan* plan, int64_t B, const void* x, const void* y, const void* w,
+                               const void* g, void* grad_w, void* grad_y) {
+  UvwBwdArgs a{};
+  a.B = B;
+  a.C = plan->C;
+  a.Co = plan->Co;
+  a.P = plan->n_paths;
+  a.x = static_cast<const float*>(x);
+  a.dim1 = plan->dim1;
+  a.y = static_cast<const float*>(y);
+  a.dim2 = plan->dim2;
+  a.w = static_cast<const float*>(w);
+  a.g = static_cast<const float*>(g);
+  a.dim_out = plan->dim_out;
+  a.grad_w = static_cast<float*>(grad_w);
+  a.grad_y = static_cast<float*>(grad_y);
+  for (int p = 0; p < plan->n_paths; ++p) {
+    UvwPath& q = a.path[p];
+    q.l1 = plan->l1[p];
+    q.l2 = plan->l2[p];
+    q.l3 = plan->l3[p];
+    q.x_off = plan->x_off[p];
+    q.g_off = plan->g_off[p];
+    q.w_off = int64_t(p) * plan->C * plan->Co;
+    q.alpha = float(plan->alpha[p]);
+  }
+  return a;
+}
+
 extern "C" e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x, const void* y, const void* w,
                                    void* out, void* stream) {
   clear_error();
@@ -585,6 +783,14 @@ extern "C" e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x
     UuuArgs u = uuu_args(plan, B, x, y, w, a.w_stride, stream);
     u.out = out;
     return launch_uuu(plan, u, false);
+  }
+  if (plan->mode == E3_UVW) {
+    st = launch_uvw_prep(plan->n_paths, plan->C, plan->Co, static_cast<const float*>(w), plan->uvw_prep, stream);
+    if (st != E3_OK) return st;
+    UvwGemmArgs g;
+    st = uvw_gemm_args(plan, B, true, x, y, out, &g);
+    if (st != E3_OK) return st;
+    return launch_uvw_gemm(g, true, stream);
   }
   return launch_forward(plan, a, false);
 }
@@ -633,7 +839,8 @@ extern "C" e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* 
   clear_error();
   e3_status st = check_plan_device(plan);
   if (st != E3_OK) return st;
-  if (plan->wmode == E3_W_SHARED) return fail(E3_ERR_UNSUPPORTED, "backward with shared weights has no kernel");
+  if (plan->wmode == E3_W_SHARED && plan->mode != E3_UVW)
+    return fail(E3_ERR_UNSUPPORTED, "backward with shared weights has no kernel");
   if (B < 0 || B >= (int64_t(1) << 31)) return fail(E3_ERR_SHAPE, "B = %lld out of range", (long long)B);
   if (B == 0) return E3_OK;
   E3_REQ(x, "x");
@@ -661,6 +868,23 @@ extern "C" e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* 
   a.grad_y = grad_y;
   a.grad_w = grad_w;
   a.stream = stream;
+  if (plan->mode == E3_UVW) {
+    if (grad_x) {
+      st = launch_uvw_prep(plan->n_paths, plan->C, plan->Co, static_cast<const float*>(w), plan->uvw_prep, stream);
+      if (st != E3_OK) return st;
+      UvwGemmArgs g;
+      st = uvw_gemm_args(plan, B, false, grad_out, y, grad_x, &g);
+      if (st == E3_OK) st = launch_uvw_gemm(g, false, stream);
+      if (st != E3_OK) return st;
+    }
+    const UvwBwdArgs b = uvw_bwd_args(plan, B, x, y, w, grad_out, grad_w, grad_y);
+    if (grad_w) {
+      st = launch_uvw_grad_w(b, stream);
+      if (st != E3_OK) return st;
+    }
+    if (grad_y) return launch_uvw_grad_y(b, stream);
+    return E3_OK;
+  }
   if (plan->mode == E3_UUU) {
     UuuArgs u = uuu_args(plan, B, x, y, w, plan->weight_numel, stream);
     u.grad_out = grad_out;

@@ -19,6 +19,13 @@ struct e3_plan {
   std::vector<double> alpha;      // per path
   int64_t dim1 = 0, dim2 = 0, dim_out = 0, weight_numel = 0;
   std::string irreps_out;
+  // uvw: output channels, per path the output block and offsets, the weight staging buffer
+  int Co = 0;
+  std::vector<int> io, x_off, g_off;
+  std::vector<int> out_l, out_off;  // per output block
+  void* uvw_prep = nullptr;
+  size_t uvw_prep_size = 0;
+  ~e3_plan();
 };
 
 namespace e3b {
@@ -174,6 +181,70 @@ struct UuuArgs {
 };
 e3_status upload_tables_uuu(const double* t64, const float* t32);
 e3_status launch_uuu(const e3_plan* plan, const UuuArgs& a, bool backward);
+// uvw tensor product with shared weights (tp_uvw.cu).
+// The tcgen05 contraction: per target block (an output block in the forward, an x block for
+// grad_x) the sum over its terms (paths) of alpha_p (coupled input) x W_p.
+constexpr int UVW_MAXT = 16;
+constexpr int UVW_MAXP = 64;
+struct UvwTarget {
+  int32_t off;          // offset of the block in a row of the result
+  int32_t l;            // its degree
+  int32_t bt;           // samples per tile: floor(128 / (2 l + 1))
+  int32_t tile_begin;   // first tile of this target in the launch
+  int32_t term_begin, term_end;
+};
+struct UvwTerm {
+  int32_t in_off;       // offset of the input block (x block, or grad_out block) in an input row
+  int32_t l_in, l2;     // its degree and the degree of y
+  int32_t chunk0;       // first B chunk of the path in the prepared weights
+  float alpha;
+};
+struct UvwGemmArgs {
+  int64_t B;
+  const float* in;
+  int64_t in_stride;
+  int32_t k_in;         // input channels of every term (the K of one term)
+  const float* y;
+  int64_t y_stride;
+  float* out;
+  int64_t out_stride;
+  int32_t N;            // channels of the result (the MMA's N)
+  const unsigned char* prep;
+  uint32_t b_chunk_bytes;
+  int32_t n_targets, total_tiles;
+  UvwTarget tg[UVW_MAXT];
+  UvwTerm term[UVW_MAXP];
+  int* status;
+  unsigned long long wait_ns;
+};
+// grad_w and grad_y on the CUDA cores: every path's degrees and offsets.
+struct UvwPath {
+  int32_t l1, l2, l3;
+  int32_t x_off, g_off;  // offsets of the path's x block and output block in their rows
+  int64_t w_off;         // offset of W_p [C][Cout] in the shared weights
+  float alpha;
+};
+struct UvwBwdArgs {
+  int64_t B;
+  int32_t C, Co, P;
+  const float* x;
+  int64_t dim1;
+  const float* y;
+  int64_t dim2;
+  const float* w;
+  const float* g;
+  int64_t dim_out;
+  float* grad_w;
+  float* grad_y;
+  UvwPath path[UVW_MAXP];
+};
+e3_status upload_tables_uvw(const double* t64, const float* t32);
+size_t uvw_prep_bytes(int P, int C, int Co);
+e3_status launch_uvw_prep(int P, int C, int Co, const float* w, void* prep, void* stream);
+e3_status launch_uvw_gemm(const UvwGemmArgs& a, bool fwd, void* stream);
+e3_status launch_uvw_grad_w(const UvwBwdArgs& a, void* stream);
+e3_status launch_uvw_grad_y(const UvwBwdArgs& a, void* stream);
+
 // Zero rows [*first_row, n_rows) of a row-major array of row_bytes-byte rows (first_row read on
 // the device: the padding positions after the last CSR row).
 e3_status zero_rows_after(const int32_t* first_row, int64_t n_rows, int64_t row_bytes, void* ptr, void* stream);

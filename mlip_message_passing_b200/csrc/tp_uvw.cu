@@ -1,0 +1,650 @@
+// Fully connected ("uvw") tensor product with shared weights on the fifth-generation tensor cores.
+//
+// What is computed (e3nn course, "Curriculum at a glance", lesson 03b: in the uvw mode every
+// channel u of x and v of y feeds every output channel w, one weight per (path, u, v, w)).  With y
+// of one channel per degree (the harmonics of an edge, or any single-channel feature) this is
+//     out[b, o, w, m3] = sum_{p -> o} alpha_p sum_u W_p[u, w] T_p[b, u, m3],
+//     T_p[b, u, m3]   = sum_{m1, m2} C_p[m1, m2, m3] x[b, l1(p), u, m1] y[b, l2(p), m2],
+// for each output block o a dense contraction over K = (path, u): rows (sample, m3), columns w.
+// The backward's grad_x has the same shape with x and grad_out exchanged:
+//     grad_x[b, l1, u, m1] = sum_{p: l1(p) = l1} alpha_p sum_w W_p[u, w] S_p[b, w, m1],
+//     S_p[b, w, m1]       = sum_{m2, m3} C_p[m1, m2, m3] g[b, o(p), w, m3] y[b, l2(p), m2].
+// Both run in one warp-specialised tcgen05 kernel (uvw_gemm_kernel):
+//   * a tile is 128 accumulator rows of one target block of degree l: BT = floor(128 / D)
+//     samples x D = 2 l + 1 components, row b_local D + m;
+//   * eight math warps compute the A operand (alpha_p T_p, or alpha_p S_p) for 32 input channels
+//     at a time on the CUDA cores, as tf32 high and low parts, into a ring of shared-memory
+//     stages (K-major, the canonical no-swizzle layout of 8-row x 16-byte core matrices);
+//   * the weights, split per call into tf32 high and low parts and laid out as B operand chunks of
+//     32 input channels (uvw_prep_kernel), stream in by bulk copy (cp.async.bulk, no multicast);
+//   * one thread issues A_hi B_hi + A_hi B_lo + A_lo B_hi per 8-wide K step (the three-pass split
+//     product: float32 accuracy from tf32 inputs) into float32 accumulators in TMEM, 128 lanes x
+//     N columns each: the main products go round-robin by chunk into UV_NBIG accumulators and the
+//     two small correction products into one more, so that no accumulator takes more than a third
+//     of the additions of a long K (a tile sums up to ~1300 products, and every addition in the
+//     tensor core rounds); after the last chunk of a tile the math warps load and add the
+//     accumulators (tcgen05.ld, float32) and store the sum.
+// Every wait is bounded (E3_ERR_TIMEOUT) and TMEM is released before the CTA exits.
+// grad_w (a reduction over samples) and grad_y (a reduction over channels) run on the CUDA cores.
+#include <climits>
+
+#include "kernels.cuh"
+#include "tc_sm100.cuh"
+
+namespace e3b {
+namespace {
+
+constexpr int UV_M = 128;          // accumulator rows per tile (TMEM lanes)
+constexpr int UV_KC = 32;          // input channels per K chunk
+constexpr int UV_NMAX = 128;       // output channels (the MMA's N) at most
+constexpr int UV_STAGES = 3;       // A and B chunks in flight
+constexpr int UV_MATH_WARPS = 8;
+constexpr int UV_THREADS = 32 * UV_MATH_WARPS + 64;  // + one MMA warp + one B producer warp
+constexpr int UV_NBIG = 3;       // accumulators of the main products (round-robin by chunk)
+constexpr int UV_TMEM_COLS = 512;  // (UV_NBIG + 1) x UV_NMAX columns, rounded up to a power of two
+constexpr uint32_t UV_A_BYTES = UV_M * UV_KC * 4;             // one of hi, lo
+constexpr uint32_t UV_B_BYTES_MAX = 2 * UV_NMAX * UV_KC * 4;  // hi + lo
+
+struct UvwSmem {
+  static constexpr size_t a_off(int s) { return size_t(s) * 2 * UV_A_BYTES; }
+  static constexpr size_t b_off(int s) { return size_t(UV_STAGES) * 2 * UV_A_BYTES + size_t(s) * UV_B_BYTES_MAX; }
+  static constexpr size_t bar_off() { return b_off(UV_STAGES); }
+  // afull, aempty, bfull, bempty [UV_STAGES] each, accfull, accempty; then the TMEM slot and the abort flag
+  static constexpr size_t total() { return bar_off() + 8 * (4 * UV_STAGES + 2) + 16; }
+};
+
+__device__ __forceinline__ int find_target(const UvwGemmArgs& a, int tile) {
+  int t = 0;
+  while (t + 1 < a.n_targets && tile >= a.tg[t + 1].tile_begin) ++t;
+  return t;
+}
+
+// A operand of one chunk: 32 input channels [32 kc, 32 kc + 32) of term tm for the samples of a
+// tile.  Thread (warp w, lane): channels ul = 16 (w % 2) + 4 (lane / 8) .. + 3 of the chunk,
+// samples b_local = 8 (w / 2) + lane % 8 + 32 i.  The eight lanes of one store phase hold eight
+// consecutive samples, whose rows differ modulo 8 (D is odd), so the 16-byte stores are free of
+// bank conflicts.
+template <int LI, int L2, int LT, bool FWD>
+__device__ __forceinline__ void produce(const UvwGemmArgs& a, int bt, int64_t b0, const UvwTerm& tm, int kc,
+                                        unsigned char* As, int warp, int lane) {
+  constexpr int DI = 2 * LI + 1, DT = 2 * LT + 1, NY2 = (L2 + 1) * (L2 + 1);
+  const int ul = 16 * (warp & 1) + 4 * (lane >> 3);
+  const int64_t u = int64_t(kc) * UV_KC + ul;
+  const float alpha = tm.alpha;
+  for (int bl = 8 * (warp >> 1) + (lane & 7); bl < bt; bl += 32) {
+    const int64_t b = b0 + bl;
+    if (b >= a.B) break;
+    float Y[NY2];
+    const float* yb = a.y + b * a.y_stride + L2 * L2;
+#pragma unroll
+    for (int m = 0; m < 2 * L2 + 1; ++m) Y[L2 * L2 + m] = __ldg(yb + m);
+    // coupling of this sample: cm[i][t] = sum_m2 C[..] Y[m2] for input component i, target t
+    float cm[DI][DT];
+    static_for<0, DI>([&](auto ic) {
+      static_for<0, DT>([&](auto tc) {
+        constexpr int I = decltype(ic)::value, T = decltype(tc)::value;
+        if constexpr (FWD) {
+          if constexpr (a_nz(LI, L2, LT, I - LI, T - LT))
+            cm[I][T] = a_entry<float, LI, L2, LT, I - LI, T - LT>(Y);
+          else
+            cm[I][T] = 0.f;
+        } else {
+          if constexpr (a_nz(LT, L2, LI, T - LT, I - LI))
+            cm[I][T] = a_entry<float, LT, L2, LI, T - LT, I - LI>(Y);
+          else
+            cm[I][T] = 0.f;
+        }
+      });
+    });
+    float in[4 * DI];  // channels ul .. ul + 3, components contiguous: one run of 4 DI floats
+    const float4* ip = reinterpret_cast<const float4*>(a.in + b * a.in_stride + tm.in_off + u * DI);
+#pragma unroll
+    for (int j = 0; j < DI; ++j) {
+      const float4 v = __ldg(ip + j);
+      in[4 * j] = v.x;
+      in[4 * j + 1] = v.y;
+      in[4 * j + 2] = v.z;
+      in[4 * j + 3] = v.w;
+    }
+#pragma unroll
+    for (int t = 0; t < DT; ++t) {
+      float v[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < DI; ++i) s = fmaf(cm[i][t], in[c * DI + i], s);
+        v[c] = alpha * s;
+      }
+      float4 hi, lo;
+      hi.x = to_tf32(v[0]);
+      hi.y = to_tf32(v[1]);
+      hi.z = to_tf32(v[2]);
+      hi.w = to_tf32(v[3]);
+      lo.x = to_tf32(v[0] - hi.x);
+      lo.y = to_tf32(v[1] - hi.y);
+      lo.z = to_tf32(v[2] - hi.z);
+      lo.w = to_tf32(v[3] - hi.w);
+      const uint32_t off = kmajor_off(bl * DT + t, ul, UV_KC);
+      *reinterpret_cast<float4*>(As + off) = hi;
+      *reinterpret_cast<float4*>(As + UV_A_BYTES + off) = lo;
+    }
+  }
+}
+
+template <bool FWD>
+__device__ __forceinline__ void produce_chunk(const UvwGemmArgs& a, const UvwTarget& tg, int64_t b0,
+                                              const UvwTerm& tm, int kc, unsigned char* As, int warp, int lane) {
+  dispatch<E3_LMAX + 1>(tm.l_in, [&](auto lic) {
+    dispatch<E3_LMAX + 1>(tm.l2, [&](auto l2c) {
+      dispatch<E3_LMAX + 1>(tg.l, [&](auto ltc) {
+        constexpr int LI = decltype(lic)::value, L2 = decltype(l2c)::value, LT = decltype(ltc)::value;
+        if constexpr (triangle(LI, L2, LT)) produce<LI, L2, LT, FWD>(a, tg.bt, b0, tm, kc, As, warp, lane);
+      });
+    });
+  });
+}
+
+// Accumulator rows 32 (w % 4) + lane of this warp to the target block: warps w and w + 4 share
+// the lanes and take alternate 32-column groups; the value is the sum of the correction
+// accumulator and the nbig main accumulators in use.  Every lane joins each tcgen05.ld
+// (warp-collective); rows past the tile's samples store nothing.
+__device__ __forceinline__ void store_rows(const UvwGemmArgs& a, const UvwTarget& tg, int64_t b0, uint32_t tmem,
+                                           int nbig, int warp, int lane) {
+  const int D = 2 * tg.l + 1;
+  const int r = 32 * (warp & 3) + lane;
+  const int bl = r / D, m = r - bl * D;
+  const int64_t b = b0 + bl;
+  const bool ok = bl < tg.bt && b < a.B;
+  float* dst = a.out + (ok ? b * a.out_stride + tg.off + m : 0);
+  const uint32_t lane_base = tmem + (uint32_t(32 * (warp & 3)) << 16);
+  for (int c = 32 * (warp >> 2); c < a.N; c += 64) {
+    uint32_t v[32];
+    float sum[32];
+    tmem_ld32_nowait(lane_base + uint32_t(UV_NBIG * UV_NMAX + c), v);
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) sum[i] = __uint_as_float(v[i]);
+    for (int k = 0; k < nbig; ++k) {
+      tmem_ld32_nowait(lane_base + uint32_t(k * UV_NMAX + c), v);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int i = 0; i < 32; ++i) sum[i] += __uint_as_float(v[i]);
+    }
+    if (ok) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dst[int64_t(c + i) * D] = sum[i];
+    }
+  }
+}
+
+// A target block that no path writes: its rows are zero.
+__device__ __forceinline__ void zero_rows(const UvwGemmArgs& a, const UvwTarget& tg, int64_t b0, int tid) {
+  const int D = 2 * tg.l + 1;
+  const int64_t n = int64_t(tg.bt) * a.N * D;
+  for (int64_t i = tid; i < n; i += 32 * UV_MATH_WARPS) {
+    const int64_t bl = i / (int64_t(a.N) * D);
+    const int64_t b = b0 + bl;
+    if (b < a.B) a.out[b * a.out_stride + tg.off + (i - bl * a.N * D)] = 0.f;
+  }
+}
+
+// Warp-specialised: warps 0 .. 7 produce A chunks and drain the accumulator; warp 8 issues the
+// MMAs; warp 9 streams the B chunks.  They meet on mbarriers, each wait bounded:
+//   afull[s] / aempty[s]   A chunk in stage s written (one arrive per math warp) / read by its MMAs
+//   bfull[s] / bempty[s]   B chunk in stage s landed / read by its MMAs
+//   accfull / accempty     the tile's accumulator complete (tcgen05.commit) / drained
+// A consumer waits on parity (use & 1) of a full barrier; a producer on parity ((use & 1) ^ 1) of
+// an empty one, which a fresh barrier passes at once.  Tiles of targets without paths are zeroed
+// by the math warps and skipped by the other two roles (they count no barrier phases).
+template <bool FWD>
+__global__ void __launch_bounds__(UV_THREADS, 1) uvw_gemm_kernel(const __grid_constant__ UvwGemmArgs a) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t* afull = reinterpret_cast<uint64_t*>(sm + UvwSmem::bar_off());
+  uint64_t* aempty = afull + UV_STAGES;
+  uint64_t* bfull = aempty + UV_STAGES;
+  uint64_t* bempty = bfull + UV_STAGES;
+  uint64_t* accfull = bempty + UV_STAGES;
+  uint64_t* accempty = accfull + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(accempty + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tslot + 1);
+  const int nk = a.k_in / UV_KC;
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tslot)),
+                 "r"(UV_TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    for (int i = 0; i < UV_STAGES; ++i) {
+      bar_init(&afull[i], UV_MATH_WARPS);
+      bar_init(&aempty[i], 1);
+      bar_init(&bfull[i], 1);
+      bar_init(&bempty[i], 1);
+    }
+    bar_init(accfull, 1);
+    bar_init(accempty, UV_MATH_WARPS);
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tslot;
+
+  if (warp < UV_MATH_WARPS) {
+    // ------------------------------------------------------------- math warps
+    uint32_t q = 0, tn = 0;
+    for (int tile = blockIdx.x; tile < a.total_tiles && !warp_aborted(s_abort); tile += gridDim.x) {
+      const UvwTarget& tg = a.tg[find_target(a, tile)];
+      const int64_t b0 = int64_t(tile - tg.tile_begin) * tg.bt;
+      if (tg.term_begin == tg.term_end) {
+        zero_rows(a, tg, b0, tid);
+        continue;
+      }
+      bool ok = true;
+      for (int j = tg.term_begin; j < tg.term_end && ok; ++j) {
+        for (int kc = 0; kc < nk; ++kc, ++q) {
+          const uint32_t s = q % UV_STAGES;
+          if (!warp_wait(&aempty[s], ((q / UV_STAGES) & 1u) ^ 1u, a.status, a.wait_ns)) {
+            *s_abort = 1;
+            ok = false;
+            break;
+          }
+          produce_chunk<FWD>(a, tg, b0, a.term[j], kc, sm + UvwSmem::a_off(int(s)), warp, lane);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the tensor core reads A through the async proxy
+          __syncwarp();
+          if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(&afull[s])) : "memory");
+        }
+      }
+      if (!ok) break;
+      if (!warp_wait(accfull, tn & 1u, a.status, a.wait_ns)) {
+        *s_abort = 1;
+        break;
+      }
+      fence_after_sync();
+      const int chunks = (tg.term_end - tg.term_begin) * nk;
+      store_rows(a, tg, b0, tmem, chunks < UV_NBIG ? chunks : UV_NBIG, warp, lane);
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(accempty)) : "memory");
+      ++tn;
+    }
+    __syncwarp();
+  } else if (warp == UV_MATH_WARPS) {
+    // ------------------------------------------------------------- MMA warp (one thread)
+    if (lane == 0) {
+      const uint32_t idesc = idesc_tf32(UV_M, a.N);
+      const uint32_t bhalf = a.b_chunk_bytes / 2;
+      uint32_t q = 0, tn = 0;
+      int64_t last = -1;  // chunk index + 1 of the last commit (its aempty phase), or -1
+      for (int tile = blockIdx.x; tile < a.total_tiles && !*s_abort; tile += gridDim.x) {
+        const UvwTarget& tg = a.tg[find_target(a, tile)];
+        if (tg.term_begin == tg.term_end) continue;
+        if (!bar_wait(accempty, (tn & 1u) ^ 1u, a.status, a.wait_ns)) {
+          *s_abort = 1;
+          break;
+        }
+        fence_after_sync();
+        uint32_t ci = 0;  // chunk of this tile
+        for (int j = tg.term_begin; j < tg.term_end && !*s_abort; ++j) {
+          for (int kc = 0; kc < nk; ++kc, ++q, ++ci) {
+            const uint32_t s = q % UV_STAGES, ph = (q / UV_STAGES) & 1u;
+            if (!bar_wait(&afull[s], ph, a.status, a.wait_ns) || !bar_wait(&bfull[s], ph, a.status, a.wait_ns)) {
+              *s_abort = 1;
+              break;
+            }
+            fence_after_sync();
+            const uint32_t a_hi = saddr(sm + UvwSmem::a_off(int(s))), a_lo = a_hi + UV_A_BYTES;
+            const uint32_t b_hi = saddr(sm + UvwSmem::b_off(int(s))), b_lo = b_hi + bhalf;
+            const uint32_t big = tmem + (ci % UV_NBIG) * UV_NMAX, small = tmem + UV_NBIG * UV_NMAX;
+#pragma unroll
+            for (int ks = 0; ks < UV_KC / 8; ++ks) {
+              const uint32_t o = uint32_t(ks) * 256;  // one K step: two 128-byte core matrices along K
+              mma_tf32(big, smem_desc(a_hi + o, UV_KC), smem_desc(b_hi + o, UV_KC), idesc,
+                       (ci < UV_NBIG && ks == 0) ? 0u : 1u);
+              mma_tf32(small, smem_desc(a_hi + o, UV_KC), smem_desc(b_lo + o, UV_KC), idesc,
+                       (ci == 0 && ks == 0) ? 0u : 1u);
+              mma_tf32(small, smem_desc(a_lo + o, UV_KC), smem_desc(b_hi + o, UV_KC), idesc, 1u);
+            }
+            mma_commit(&aempty[s]);
+            mma_commit(&bempty[s]);
+            last = int64_t(q) + 1;
+          }
+        }
+        if (*s_abort) break;
+        mma_commit(accfull);
+        ++tn;
+      }
+      if (*s_abort && last > 0) {
+        // let the last committed MMA group finish (bounded) before the tensor memory is released
+        const uint32_t lq = uint32_t(last - 1);
+        bar_wait(&aempty[lq % UV_STAGES], (lq / UV_STAGES) & 1u, a.status, a.wait_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- B producer (one thread)
+    if (lane == 0) {
+      uint32_t q = 0;
+      for (int tile = blockIdx.x; tile < a.total_tiles && !*s_abort; tile += gridDim.x) {
+        const UvwTarget& tg = a.tg[find_target(a, tile)];
+        for (int j = tg.term_begin; j < tg.term_end && !*s_abort; ++j) {
+          for (int kc = 0; kc < nk; ++kc, ++q) {
+            const uint32_t s = q % UV_STAGES;
+            if (!bar_wait(&bempty[s], ((q / UV_STAGES) & 1u) ^ 1u, a.status, a.wait_ns)) {
+              *s_abort = 1;
+              break;
+            }
+            bulk_copy(sm + UvwSmem::b_off(int(s)), a.prep + size_t(a.term[j].chunk0 + kc) * a.b_chunk_bytes,
+                      a.b_chunk_bytes, &bfull[s]);
+          }
+        }
+      }
+      if (*s_abort) {
+        // let the copies in flight land (bounded) before the CTA exits
+        for (uint32_t k = q >= UV_STAGES ? q - UV_STAGES : 0; k < q; ++k)
+          bar_wait(&bfull[k % UV_STAGES], (k / UV_STAGES) & 1u, a.status, a.wait_ns);
+      }
+    }
+    __syncwarp();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(UV_TMEM_COLS));
+}
+
+// Shared weights W [P][C][Cout] -> B chunks of 32 input channels, tf32 high part then low part,
+// each [N rows x 32] K-major: the forward's chunks (p, kc) hold rows w, k = u - 32 kc; the
+// backward's (after all forward chunks) rows u, k = w - 32 kc.
+__global__ void uvw_prep_kernel(int P, int C, int Co, const float* __restrict__ w, unsigned char* __restrict__ prep) {
+  const int64_t total = int64_t(P) * C * Co;
+  const uint32_t fwd_bytes = 2u * uint32_t(Co) * UV_KC * 4, bwd_bytes = 2u * uint32_t(C) * UV_KC * 4;
+  unsigned char* bwd = prep + size_t(P) * (C / UV_KC) * fwd_bytes;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
+    const int wc = int(i % Co);
+    const int64_t pu = i / Co;
+    const int u = int(pu % C), p = int(pu / C);
+    const float v = __ldg(w + i);
+    const float hi = to_tf32(v), lo = to_tf32(v - hi);
+    unsigned char* f = prep + (size_t(p) * (C / UV_KC) + u / UV_KC) * fwd_bytes;
+    *reinterpret_cast<float*>(f + kmajor_off(wc, u % UV_KC, UV_KC)) = hi;
+    *reinterpret_cast<float*>(f + fwd_bytes / 2 + kmajor_off(wc, u % UV_KC, UV_KC)) = lo;
+    unsigned char* g = bwd + (size_t(p) * (Co / UV_KC) + wc / UV_KC) * bwd_bytes;
+    *reinterpret_cast<float*>(g + kmajor_off(u, wc % UV_KC, UV_KC)) = hi;
+    *reinterpret_cast<float*>(g + bwd_bytes / 2 + kmajor_off(u, wc % UV_KC, UV_KC)) = lo;
+  }
+}
+
+// ------------------------------------------------------------------ grad_w (CUDA cores) ---
+// grad_W_p[u, w] = alpha_p sum_{b, m3} T_p[b, u, m3] g[b, o(p), w, m3]: a CTA takes one path and a
+// range of samples, in chunks of SB = floor(32 / D3) samples: it writes T_p of the chunk (rows
+// (sample, m3), columns u) and the chunk's grad_out block (rows (sample, m3), columns w) to shared
+// memory, then each thread accumulates an 8 x 8 block of (u, w) over the rows; the partial sums of
+// all CTAs of a path are added into grad_w (zeroed first) with atomics.
+constexpr int GW_THREADS = 256;
+constexpr int GW_ROWS = 32;
+
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void gw_path(const UvwBwdArgs& a, const UvwPath& pp, int64_t bbeg, int64_t bend, float* Ts,
+                                        float* Gs, float (&acc)[8][8], int tu, int tw, bool active) {
+  constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, NY2 = (L2 + 1) * (L2 + 1), SB = GW_ROWS / D3;
+  const int C = a.C, Co = a.Co;
+  for (int64_t b0 = bbeg; b0 < bend; b0 += SB) {
+    const int ns = int(b0 + SB <= bend ? SB : bend - b0);
+    for (int i = threadIdx.x; i < SB * C; i += GW_THREADS) {
+      const int s = i / C, u = i - s * C;
+      float T[D3];
+#pragma unroll
+      for (int m = 0; m < D3; ++m) T[m] = 0.f;
+      if (s < ns) {
+        const int64_t b = b0 + s;
+        float Y[NY2], xv[D1];
+#pragma unroll
+        for (int m = 0; m < 2 * L2 + 1; ++m) Y[L2 * L2 + m] = __ldg(a.y + b * a.dim2 + L2 * L2 + m);
+#pragma unroll
+        for (int m = 0; m < D1; ++m) xv[m] = __ldg(a.x + b * a.dim1 + pp.x_off + int64_t(u) * D1 + m);
+        static_for<0, D3>([&](auto tc) {
+          static_for<0, D1>([&](auto ic) {
+            constexpr int M3 = decltype(tc)::value - L3, M1 = decltype(ic)::value - L1;
+            if constexpr (a_nz(L1, L2, L3, M1, M3))
+              T[M3 + L3] = fmaf(a_entry<float, L1, L2, L3, M1, M3>(Y), xv[M1 + L1], T[M3 + L3]);
+          });
+        });
+      }
+#pragma unroll
+      for (int m = 0; m < D3; ++m) Ts[(s * D3 + m) * C + u] = T[m];
+    }
+    for (int i = threadIdx.x; i < SB * Co * D3; i += GW_THREADS) {
+      const int s = i / (Co * D3), r = i - s * (Co * D3);  // r = w D3 + m3, the block's memory order
+      const int w = r / D3, m = r - w * D3;
+      Gs[(s * D3 + m) * Co + w] = s < ns ? __ldg(a.g + (b0 + s) * a.dim_out + pp.g_off + r) : 0.f;
+    }
+    __syncthreads();
+    if (active) {
+      for (int r = 0; r < SB * D3; ++r) {
+        float av[8], bv[8];
+        const float4* ap = reinterpret_cast<const float4*>(Ts + r * C + tu * 8);
+        const float4* bp = reinterpret_cast<const float4*>(Gs + r * Co + tw * 8);
+        const float4 a0 = ap[0], a1 = ap[1], b0v = bp[0], b1v = bp[1];
+        av[0] = a0.x, av[1] = a0.y, av[2] = a0.z, av[3] = a0.w, av[4] = a1.x, av[5] = a1.y, av[6] = a1.z, av[7] = a1.w;
+        bv[0] = b0v.x, bv[1] = b0v.y, bv[2] = b0v.z, bv[3] = b0v.w, bv[4] = b1v.x, bv[5] = b1v.y, bv[6] = b1v.z,
+        bv[7] = b1v.w;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(GW_THREADS) uvw_grad_w_kernel(const __grid_constant__ UvwBwdArgs a, int64_t per_split) {
+  __shared__ __align__(16) float Ts[GW_ROWS * UV_NMAX];
+  __shared__ __align__(16) float Gs[GW_ROWS * UV_NMAX];
+  const UvwPath& pp = a.path[blockIdx.x];
+  const int nw = a.Co / 8;
+  const int tu = threadIdx.x / nw, tw = threadIdx.x - tu * nw;
+  const bool active = tu < a.C / 8;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  const int64_t bbeg = int64_t(blockIdx.y) * per_split;
+  const int64_t bend = bbeg + per_split < a.B ? bbeg + per_split : a.B;
+  if (bbeg < bend) {
+    dispatch<E3_LMAX + 1>(pp.l1, [&](auto l1c) {
+      dispatch<E3_LMAX + 1>(pp.l2, [&](auto l2c) {
+        dispatch<E3_LMAX + 1>(pp.l3, [&](auto l3c) {
+          constexpr int L1 = decltype(l1c)::value, L2 = decltype(l2c)::value, L3 = decltype(l3c)::value;
+          if constexpr (triangle(L1, L2, L3)) gw_path<L1, L2, L3>(a, pp, bbeg, bend, Ts, Gs, acc, tu, tw, active);
+        });
+      });
+    });
+  }
+  if (active && bbeg < bend) {
+    float* dst = a.grad_w + pp.w_off + int64_t(tu * 8) * a.Co + tw * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) atomicAdd(dst + int64_t(i) * a.Co + j, pp.alpha * acc[i][j]);
+  }
+}
+
+// ------------------------------------------------------------------ grad_y (CUDA cores) ---
+// grad_y[b, l2, m2] = sum_p alpha_p sum_{m1, m3} C_p[m1, m2, m3] sum_u x[b, u, m1] Z_p[b, u, m3],
+// Z_p[b, u, m3] = sum_w W_p[u, w] g[b, o(p), w, m3].  A CTA of C threads (thread u) takes GY_SB
+// samples and walks every path: it keeps the samples' grad_out block in shared memory (reloaded when
+// the block changes), forms Z_p for its channel from the weight row W_p[u, :] (32 columns at a time
+// in registers), contracts with its x and the coefficients, and sums over the channels with warp
+// shuffles and shared-memory atomics into the samples' grad_y, which it then writes (each sample
+// belongs to one CTA: no global atomics).
+constexpr int GY_SB = 8;
+constexpr int GY_NY = (E3_LMAX + 1) * (E3_LMAX + 1);
+
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void gy_path(const UvwBwdArgs& a, const UvwPath& pp, int64_t b0, int ns, const float* gS,
+                                        float* qS) {
+  constexpr int D1 = 2 * L1 + 1, D2 = 2 * L2 + 1, D3 = 2 * L3 + 1, NY2 = (L2 + 1) * (L2 + 1);
+  const int u = threadIdx.x, Co = a.Co;
+  float Z[GY_SB][D3];
+#pragma unroll
+  for (int s = 0; s < GY_SB; ++s)
+#pragma unroll
+    for (int m = 0; m < D3; ++m) Z[s][m] = 0.f;
+  const float* wrow = a.w + pp.w_off + int64_t(u) * Co;
+  for (int w0 = 0; w0 < Co; w0 += 32) {
+    float wr[32];
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(wrow + w0 + j));
+      wr[j] = v.x, wr[j + 1] = v.y, wr[j + 2] = v.z, wr[j + 3] = v.w;
+    }
+#pragma unroll
+    for (int s = 0; s < GY_SB; ++s) {
+      const float* gs = gS + s * (Co * D3) + w0 * D3;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+#pragma unroll
+        for (int m = 0; m < D3; ++m) Z[s][m] = fmaf(wr[j], gs[j * D3 + m], Z[s][m]);
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < GY_SB; ++s) {
+    if (s >= ns) break;
+    const int64_t b = b0 + s;
+    float xv[D1];
+#pragma unroll
+    for (int m = 0; m < D1; ++m) xv[m] = __ldg(a.x + b * a.dim1 + pp.x_off + int64_t(u) * D1 + m);
+    float c[D2];
+#pragma unroll
+    for (int m = 0; m < D2; ++m) c[m] = 0.f;
+    static_for<-L1, L1 + 1>([&](auto m1c) {
+      static_for<-L2, L2 + 1>([&](auto m2c) {
+        static_for<-L3, L3 + 1>([&](auto m3c) {
+          constexpr int M1 = decltype(m1c)::value, M2 = decltype(m2c)::value, M3 = decltype(m3c)::value;
+          if constexpr (cg_nz(L1, L2, L3, M1, M2, M3)) {
+            constexpr int I = cg_index(L1, L2, L3, M1, M2, M3);
+            c[M2 + L2] = fmaf(CGT<float>::template get<I>() * xv[M1 + L1], Z[s][M3 + L3], c[M2 + L2]);
+          }
+        });
+      });
+    });
+#pragma unroll
+    for (int m = 0; m < D2; ++m) {
+      float v = pp.alpha * c[m];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if ((threadIdx.x & 31) == 0) atomicAdd(&qS[s * GY_NY + L2 * L2 + m], v);
+    }
+  }
+  (void)NY2;
+}
+
+__global__ void __launch_bounds__(UV_NMAX) uvw_grad_y_kernel(const __grid_constant__ UvwBwdArgs a) {
+  __shared__ __align__(16) float gS[GY_SB * UV_NMAX * 7];
+  __shared__ float qS[GY_SB * GY_NY];
+  const int64_t b0 = int64_t(blockIdx.x) * GY_SB;
+  const int ns = int(b0 + GY_SB <= a.B ? GY_SB : a.B - b0);
+  for (int i = threadIdx.x; i < GY_SB * GY_NY; i += blockDim.x) qS[i] = 0.f;
+  int loaded = -1;
+  for (int p = 0; p < a.P; ++p) {
+    const UvwPath& pp = a.path[p];
+    const int D3 = 2 * pp.l3 + 1, n = a.Co * D3;
+    if (pp.g_off != loaded) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < GY_SB * n; i += blockDim.x) {
+        const int s = i / n;
+        gS[i] = s < ns ? __ldg(a.g + (b0 + s) * a.dim_out + pp.g_off + (i - s * n)) : 0.f;
+      }
+      __syncthreads();
+      loaded = pp.g_off;
+    }
+    dispatch<E3_LMAX + 1>(pp.l1, [&](auto l1c) {
+      dispatch<E3_LMAX + 1>(pp.l2, [&](auto l2c) {
+        dispatch<E3_LMAX + 1>(pp.l3, [&](auto l3c) {
+          constexpr int L1 = decltype(l1c)::value, L2 = decltype(l2c)::value, L3 = decltype(l3c)::value;
+          if constexpr (triangle(L1, L2, L3)) gy_path<L1, L2, L3>(a, pp, b0, ns, gS, qS);
+        });
+      });
+    });
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < ns * int(a.dim2); i += blockDim.x) {
+    const int s = i / int(a.dim2), m = i - s * int(a.dim2);
+    a.grad_y[(b0 + s) * a.dim2 + m] = qS[s * GY_NY + m];
+  }
+}
+
+}  // namespace
+
+e3_status upload_tables_uvw(const double* t64, const float* t32) {
+  const cudaError_t err = upload_tables(t64, t32);
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uploading the CG table failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+size_t uvw_prep_bytes(int P, int C, int Co) { return size_t(16) * P * C * Co; }
+
+e3_status launch_uvw_prep(int P, int C, int Co, const float* w, void* prep, void* stream) {
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t total = int64_t(P) * C * Co;
+  const int blocks = int(std::min<int64_t>((total + 255) / 256, 4 * 148));
+  uvw_prep_kernel<<<blocks, 256, 0, s>>>(P, C, Co, w, static_cast<unsigned char*>(prep));
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw prep launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+e3_status launch_uvw_gemm(const UvwGemmArgs& a, bool fwd, void* stream) {
+  if (a.total_tiles <= 0 || a.B == 0) return E3_OK;
+  if (a.N % 32 != 0 || a.N > UV_NMAX || a.k_in % UV_KC != 0) return fail(E3_ERR_UNSUPPORTED, "uvw channel counts");
+  const size_t smem = UvwSmem::total();
+  cudaError_t err =
+      fwd ? cudaFuncSetAttribute(uvw_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))
+          : cudaFuncSetAttribute(uvw_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw smem attribute: %s", cudaGetErrorString(err));
+  const int grid = std::min(a.total_tiles, sm_count());
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fwd)
+    uvw_gemm_kernel<true><<<grid, UV_THREADS, smem, s>>>(a);
+  else
+    uvw_gemm_kernel<false><<<grid, UV_THREADS, smem, s>>>(a);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+}  // namespace e3b
+
+namespace e3b {
+
+e3_status launch_uvw_grad_w(const UvwBwdArgs& a, void* stream) {
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaMemsetAsync(a.grad_w, 0, sizeof(float) * size_t(a.P) * a.C * a.Co, s);
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "zeroing grad_w failed: %s", cudaGetErrorString(err));
+  if (a.B == 0) return E3_OK;
+  // about four CTAs per SM over all paths, each a contiguous range of samples
+  const int64_t splits = std::max<int64_t>(1, std::min<int64_t>((4 * int64_t(sm_count()) + a.P - 1) / a.P, (a.B + 7) / 8));
+  const int64_t per_split = (a.B + splits - 1) / splits;
+  uvw_grad_w_kernel<<<dim3(unsigned(a.P), unsigned(splits)), GW_THREADS, 0, s>>>(a, per_split);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw grad_w launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+e3_status launch_uvw_grad_y(const UvwBwdArgs& a, void* stream) {
+  if (a.B == 0) return E3_OK;
+  const int64_t blocks = (a.B + GY_SB - 1) / GY_SB;
+  if (blocks > INT_MAX) return fail(E3_ERR_SHAPE, "B too large");
+  uvw_grad_y_kernel<<<unsigned(blocks), a.C, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw grad_y launch failed: %s", cudaGetErrorString(err));
+  return E3_OK;
+}
+
+}  // namespace e3b

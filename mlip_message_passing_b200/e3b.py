@@ -236,7 +236,7 @@ def tp_backward(plan, x, y, w, grad_out, need_x=True, need_y=True, need_w=True):
     dev, dt = plan.device, plan.dtype
     _need(x, "x", dt, (B, plan.dim_in1), dev)
     _need(y, "y", dt, (B, plan.dim_in2), dev)
-    _need(w, "w", dt, (B, plan.weight_numel), dev)
+    _need(w, "w", dt, plan._w_shape(B), dev)
     _need(grad_out, "grad_out", dt, (B, plan.dim_out), dev)
     gx = torch.empty_like(x) if need_x else None
     gy = torch.empty_like(y) if need_y else None

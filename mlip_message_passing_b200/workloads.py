@@ -7,6 +7,7 @@ the smoke check so that the CUDA path and the float64 oracle see the same bytes.
 Recipes (numpy PCG64, ``default_rng(seed)``; draws in the order listed):
 
 * channelwise (uuu) product: x, y, w ~ N(0, 1) in that order;
+* fully connected (uvw) product, shared weights: x, y, w ~ N(0, 1) in that order;
 * batched product: edge-like vectors ~ N(0, 1) (or uniform on the sphere), then x ~ N(0, 1)
   [B, dim_x], then w ~ N(0, 1) [B, weight_numel];
 * water-box-like graph: N positions uniform in a periodic cube of side (N / 0.1)^(1/3) Angstrom
@@ -137,6 +138,10 @@ CONFIGS = {
     "conv_waterbox_bwd": dict(kind="conv", N=3000, mul=64, lx=2, ly=3, lo=2, seed=2, grad_seed=4),
     # channelwise (uuu) product of two node-feature sets of 128 channels, degrees 0..3
     "tp_uuu": dict(kind="tp_uuu", B=32_768, mul=128, lx=3, ly=3, lo=3, seed=5),
+    # fully connected (uvw) product, shared weights: 128 channels of degrees 0..3 with one
+    # harmonic-like channel of degrees 0..3 into 128 channels of every (l3 <= 3, parity) block
+    "tp_uvw": dict(kind="tp_uvw", B=65_536, mul=128, lx=3, ly=3, seed=6,
+                   irreps_out="128x0e+128x1o+128x1e+128x2e+128x2o+128x3o+128x3e"),
 }
 
 
@@ -168,6 +173,16 @@ def channel_inputs(B, mul, lx, ly, lo, seed, dtype=np.float32):
     x = rng.standard_normal((B, mul * (lx + 1) ** 2)).astype(dtype)
     y = rng.standard_normal((B, mul * (ly + 1) ** 2)).astype(dtype)
     w = rng.standard_normal((B, n_paths(lx, ly, lo) * mul)).astype(dtype)
+    return dict(x=x, y=y, w=w)
+
+
+def uvw_inputs(B, dim_x, dim_y, weight_numel, seed, dtype=np.float32):
+    """Inputs of a fully connected product with shared weights: x [B, dim_x], y [B, dim_y] and
+    w [weight_numel], all N(0, 1), drawn in that order."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, dim_x)).astype(dtype)
+    y = rng.standard_normal((B, dim_y)).astype(dtype)
+    w = rng.standard_normal(weight_numel).astype(dtype)
     return dict(x=x, y=y, w=w)
 
 
