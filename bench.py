@@ -63,6 +63,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-tp", action="store_true", help="skip the tensor-product (no graph) measurement")
     ap.add_argument("--no-uuu", action="store_true", help="skip the channelwise (uuu) tensor-product measurement")
+    ap.add_argument("--no-uvw", action="store_true", help="skip the fully connected (uvw) tensor-product measurement")
     ap.add_argument("--no-waterbox", action="store_true", help="skip the second (water-box) block")
     ap.add_argument("--no-scrub", action="store_true", help="skip the L2-scrubbed per-kernel statistics")
     ap.add_argument("--no-radial", action="store_true", help="skip the radial-network (tensor core) measurement")
@@ -344,6 +345,83 @@ def measure_tp(args, dev, name="tp_batched"):
         gbs = nbytes[part] / (ms * 1e-3) / 1e9
         line[part] = {"ms": ms, "samples_per_s": B / (ms * 1e-3), "GBps": gbs, "frac_of_hbm": gbs / peak,
                       "frac_of_nominal": gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": nbytes[part]}
+    del x, y, w, go, out, gx, gy, gw, ws
+    torch.cuda.empty_cache()
+    return line
+
+
+def tf32_peak():
+    """Dense tf32 tensor peak: the measured bf16 burst peak times the nominal tf32 / bf16 ratio
+    (1.1 / 2.25 PFLOP/s)."""
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["bf16_tflops"]) * 1.1 / 2.25, "measured bf16 x nominal tf32/bf16"
+    except (OSError, KeyError, ValueError):
+        return 1590.0 * 1.1 / 2.25, "fallback bf16 x nominal tf32/bf16"
+
+
+def measure_uvw(args, dev):
+    """Fully connected (uvw) product with shared weights on the tp_uvw workload: the forward (weight
+    split + tcgen05 contraction), and each backward part alone, CUDA events after warm-up; inputs
+    (2.6 GB) larger than L2.  The contraction's algorithmic FLOPs are 2 B C Co sum_p D(p) (D the
+    target degree's dimension); the tensor cores execute three tf32 products per FLOP counted."""
+    import torch
+    from mlip_message_passing_b200 import e3b, workloads as W
+
+    cfg = W.CONFIGS["tp_uvw"]
+    B = cfg["B"]
+    ir1, ir2, irout = W.irreps_str(cfg["mul"], cfg["lx"]), W.sh_irreps(cfg["ly"]), cfg["irreps_out"]
+    plan = e3b.Plan(ir1, ir2, irout, mode="uvw", shared_weights=True)
+    gen = torch.Generator(device=dev).manual_seed(cfg["seed"])
+    x = torch.randn(B, plan.dim_in1, generator=gen, device=dev)
+    y = torch.randn(B, plan.dim_in2, generator=gen, device=dev)
+    w = torch.randn(plan.weight_numel, generator=gen, device=dev)
+    go = torch.randn(B, plan.dim_out, generator=gen, device=dev)
+    out = torch.empty(B, plan.dim_out, device=dev)
+    gx, gy, gw = torch.empty_like(x), torch.empty_like(y), torch.empty_like(w)
+    ws = e3b.backward_workspace(B, dev)
+    stream = torch.cuda.current_stream()
+    P = e3b._ptr
+
+    def bwd(nx, ny, nw):
+        e3b.lib.e3_tp_backward(plan.handle, B, P(x), P(y), P(w), P(go), P(gx) if nx else None, P(gy) if ny else None,
+                               P(gw) if nw else None, P(ws), ws.numel(), e3b._stream())
+
+    parts = {"fwd": lambda: e3b.lib.e3_tp_forward(plan.handle, B, P(x), P(y), P(w), P(out), e3b._stream()),
+             "grad_x": lambda: bwd(True, False, False), "grad_w": lambda: bwd(False, False, True),
+             "grad_y": lambda: bwd(False, True, False), "bwd": lambda: bwd(True, True, True)}
+    res = {}
+    for part, fn in parts.items():
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        ev = []
+        for _ in range(max(3, args.steps)):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        e3b.device_status()
+        res[part] = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    d3 = sum(2 * l3 + 1 for (_, _, l3) in plan.paths)
+    d1 = sum(2 * l1 + 1 for (l1, _, _) in plan.paths)
+    c_out = int(irout.split("x")[0])
+    base = 2.0 * B * cfg["mul"] * c_out
+    flops = {"fwd": base * d3, "grad_x": base * d1, "grad_w": base * d3, "grad_y": base * d3}
+    flops["bwd"] = flops["grad_x"] + flops["grad_w"] + flops["grad_y"]
+    peak, peak_kind = tf32_peak()
+    line = {"workload": f"tp_uvw: B={B}, {ir1} x {ir2} -> {irout}, {plan.n_paths} paths, shared weights, fp32 "
+                        "(three tf32 passes on the tensor cores for fwd and grad_x; CUDA cores for grad_w, grad_y)",
+            "tf32_peak_tflops": peak, "peak_kind": peak_kind}
+    for part in parts:
+        ms = res[part]
+        tf = flops[part] / (ms * 1e-3) / 1e12
+        entry = {"ms": ms, "samples_per_s": B / (ms * 1e-3), "TFLOPs": tf, "algorithmic_flops": flops[part]}
+        if part in ("fwd", "grad_x"):
+            entry["tensor_frac"] = 3 * tf / peak  # three tf32 products per counted FLOP
+        line[part] = entry
     del x, y, w, go, out, gx, gy, gw, ws
     torch.cuda.empty_cache()
     return line
@@ -776,6 +854,7 @@ def run_native(args):
 
     tp = None if args.no_tp else measure_tp(args, dev)
     uuu = None if args.no_uuu else measure_tp(args, dev, "tp_uuu")
+    uvw = None if args.no_uvw else measure_uvw(args, dev)
     cfg, irreps_x, irreps_y = workload_spec(args.workload)
     cpu = None
     if not args.no_cpu_baseline:
@@ -809,6 +888,7 @@ def run_native(args):
         "waterbox": water,
         "tp": tp,
         "uuu": uuu,
+        "uvw": uvw,
         "radial": radial,
         "roofline": head["roofline"],
         "cpu_baseline": cpu,

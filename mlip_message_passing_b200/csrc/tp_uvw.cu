@@ -14,7 +14,8 @@
 //     samples x D = 2 l + 1 components, row b_local D + m;
 //   * eight math warps compute the A operand (alpha_p T_p, or alpha_p S_p) for 32 input channels
 //     at a time on the CUDA cores, as tf32 high and low parts, into a ring of shared-memory
-//     stages (K-major, the canonical no-swizzle layout of 8-row x 16-byte core matrices);
+//     stages (K-major, the canonical no-swizzle layout of 8-row x 16-byte core matrices); a
+//     thread keeps its samples' coupling sum_m2 C y in registers over all chunks of a term;
 //   * the weights, split per call into tf32 high and low parts and laid out as B operand chunks of
 //     32 input channels (uvw_prep_kernel), stream in by bulk copy (cp.async.bulk, no multicast);
 //   * one thread issues A_hi B_hi + A_hi B_lo + A_lo B_hi per 8-wide K step (the three-pass split
@@ -59,90 +60,118 @@ __device__ __forceinline__ int find_target(const UvwGemmArgs& a, int tile) {
   return t;
 }
 
-// A operand of one chunk: 32 input channels [32 kc, 32 kc + 32) of term tm for the samples of a
-// tile.  Thread (warp w, lane): channels ul = 16 (w % 2) + 4 (lane / 8) .. + 3 of the chunk,
-// samples b_local = 8 (w / 2) + lane % 8 + 32 i.  The eight lanes of one store phase hold eight
+// A operand of every chunk of one term (32 input channels [32 kc, 32 kc + 32) per chunk) for the
+// samples of a tile.  Thread (warp w, lane): channels ul = 16 (w % 2) + 4 (lane / 8) .. + 3 of a
+// chunk, samples b_local = 8 (w / 2) + lane % 8 + 32 i (i < NSLOT).  The coupling of each of its
+// samples, cm[i][t] = sum_m2 C[..] y[m2] (input component i, target component t), is formed once
+// and kept in registers for the term's chunks.  The eight lanes of one store phase hold eight
 // consecutive samples, whose rows differ modulo 8 (D is odd), so the 16-byte stores are free of
-// bank conflicts.
+// bank conflicts.  Returns false when a wait gave up (the abort flag is then set).
 template <int LI, int L2, int LT, bool FWD>
-__device__ __forceinline__ void produce(const UvwGemmArgs& a, int bt, int64_t b0, const UvwTerm& tm, int kc,
-                                        unsigned char* As, int warp, int lane) {
+__device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64_t b0, const UvwTerm& tm, int nk,
+                                             unsigned char* sm, uint64_t* aempty, uint64_t* afull, uint32_t& q,
+                                             volatile int* s_abort, int warp, int lane) {
   constexpr int DI = 2 * LI + 1, DT = 2 * LT + 1, NY2 = (L2 + 1) * (L2 + 1);
+  constexpr int NSLOT = (UV_M / DT + 31) / 32;
   const int ul = 16 * (warp & 1) + 4 * (lane >> 3);
-  const int64_t u = int64_t(kc) * UV_KC + ul;
-  const float alpha = tm.alpha;
-  for (int bl = 8 * (warp >> 1) + (lane & 7); bl < bt; bl += 32) {
-    const int64_t b = b0 + bl;
-    if (b >= a.B) break;
-    float Y[NY2];
-    const float* yb = a.y + b * a.y_stride + L2 * L2;
+  float cm[NSLOT][DI][DT];
+  const float* inrow[NSLOT];
+  bool valid[NSLOT];
 #pragma unroll
-    for (int m = 0; m < 2 * L2 + 1; ++m) Y[L2 * L2 + m] = __ldg(yb + m);
-    // coupling of this sample: cm[i][t] = sum_m2 C[..] Y[m2] for input component i, target t
-    float cm[DI][DT];
+  for (int k = 0; k < NSLOT; ++k) {
+    const int bl = 8 * (warp >> 1) + (lane & 7) + 32 * k;
+    const int64_t b = b0 + bl;
+    valid[k] = bl < bt && b < a.B;
+    inrow[k] = a.in + (valid[k] ? b * a.in_stride + tm.in_off : 0);
+    float Y[NY2];
+#pragma unroll
+    for (int m = 0; m < 2 * L2 + 1; ++m) Y[L2 * L2 + m] = valid[k] ? __ldg(a.y + b * a.y_stride + L2 * L2 + m) : 0.f;
     static_for<0, DI>([&](auto ic) {
       static_for<0, DT>([&](auto tc) {
         constexpr int I = decltype(ic)::value, T = decltype(tc)::value;
         if constexpr (FWD) {
           if constexpr (a_nz(LI, L2, LT, I - LI, T - LT))
-            cm[I][T] = a_entry<float, LI, L2, LT, I - LI, T - LT>(Y);
+            cm[k][I][T] = tm.alpha * a_entry<float, LI, L2, LT, I - LI, T - LT>(Y);
           else
-            cm[I][T] = 0.f;
+            cm[k][I][T] = 0.f;
         } else {
           if constexpr (a_nz(LT, L2, LI, T - LT, I - LI))
-            cm[I][T] = a_entry<float, LT, L2, LI, T - LT, I - LI>(Y);
+            cm[k][I][T] = tm.alpha * a_entry<float, LT, L2, LI, T - LT, I - LI>(Y);
           else
-            cm[I][T] = 0.f;
+            cm[k][I][T] = 0.f;
         }
       });
     });
-    float in[4 * DI];  // channels ul .. ul + 3, components contiguous: one run of 4 DI floats
-    const float4* ip = reinterpret_cast<const float4*>(a.in + b * a.in_stride + tm.in_off + u * DI);
-#pragma unroll
-    for (int j = 0; j < DI; ++j) {
-      const float4 v = __ldg(ip + j);
-      in[4 * j] = v.x;
-      in[4 * j + 1] = v.y;
-      in[4 * j + 2] = v.z;
-      in[4 * j + 3] = v.w;
-    }
-#pragma unroll
-    for (int t = 0; t < DT; ++t) {
-      float v[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < DI; ++i) s = fmaf(cm[i][t], in[c * DI + i], s);
-        v[c] = alpha * s;
-      }
-      float4 hi, lo;
-      hi.x = to_tf32(v[0]);
-      hi.y = to_tf32(v[1]);
-      hi.z = to_tf32(v[2]);
-      hi.w = to_tf32(v[3]);
-      lo.x = to_tf32(v[0] - hi.x);
-      lo.y = to_tf32(v[1] - hi.y);
-      lo.z = to_tf32(v[2] - hi.z);
-      lo.w = to_tf32(v[3] - hi.w);
-      const uint32_t off = kmajor_off(bl * DT + t, ul, UV_KC);
-      *reinterpret_cast<float4*>(As + off) = hi;
-      *reinterpret_cast<float4*>(As + UV_A_BYTES + off) = lo;
-    }
   }
+  for (int kc = 0; kc < nk; ++kc, ++q) {
+    const uint32_t s = q % UV_STAGES;
+    if (!warp_wait(&aempty[s], ((q / UV_STAGES) & 1u) ^ 1u, a.status, a.wait_ns)) {
+      *s_abort = 1;
+      return false;
+    }
+    unsigned char* As = sm + UvwSmem::a_off(int(s));
+    const int64_t u = int64_t(kc) * UV_KC + ul;
+#pragma unroll
+    for (int k = 0; k < NSLOT; ++k) {
+      if (!valid[k]) continue;
+      const int bl = 8 * (warp >> 1) + (lane & 7) + 32 * k;
+      float in[4 * DI];  // channels u .. u + 3, components contiguous: one run of 4 DI floats
+      const float4* ip = reinterpret_cast<const float4*>(inrow[k] + u * DI);
+#pragma unroll
+      for (int j = 0; j < DI; ++j) {
+        const float4 v = __ldg(ip + j);
+        in[4 * j] = v.x;
+        in[4 * j + 1] = v.y;
+        in[4 * j + 2] = v.z;
+        in[4 * j + 3] = v.w;
+      }
+#pragma unroll
+      for (int t = 0; t < DT; ++t) {
+        float v[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float acc = 0.f;
+#pragma unroll
+          for (int i = 0; i < DI; ++i) acc = fmaf(cm[k][i][t], in[c * DI + i], acc);
+          v[c] = acc;
+        }
+        float4 hi, lo;
+        hi.x = to_tf32(v[0]);
+        hi.y = to_tf32(v[1]);
+        hi.z = to_tf32(v[2]);
+        hi.w = to_tf32(v[3]);
+        lo.x = to_tf32(v[0] - hi.x);
+        lo.y = to_tf32(v[1] - hi.y);
+        lo.z = to_tf32(v[2] - hi.z);
+        lo.w = to_tf32(v[3] - hi.w);
+        const uint32_t off = kmajor_off(bl * DT + t, ul, UV_KC);
+        *reinterpret_cast<float4*>(As + off) = hi;
+        *reinterpret_cast<float4*>(As + UV_A_BYTES + off) = lo;
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the tensor core reads A through the async proxy
+    __syncwarp();
+    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(&afull[s])) : "memory");
+  }
+  return true;
 }
 
 template <bool FWD>
-__device__ __forceinline__ void produce_chunk(const UvwGemmArgs& a, const UvwTarget& tg, int64_t b0,
-                                              const UvwTerm& tm, int kc, unsigned char* As, int warp, int lane) {
+__device__ __forceinline__ bool produce_term_any(const UvwGemmArgs& a, const UvwTarget& tg, int64_t b0,
+                                                 const UvwTerm& tm, int nk, unsigned char* sm, uint64_t* aempty,
+                                                 uint64_t* afull, uint32_t& q, volatile int* s_abort, int warp,
+                                                 int lane) {
+  bool ok = true;
   dispatch<E3_LMAX + 1>(tm.l_in, [&](auto lic) {
     dispatch<E3_LMAX + 1>(tm.l2, [&](auto l2c) {
       dispatch<E3_LMAX + 1>(tg.l, [&](auto ltc) {
         constexpr int LI = decltype(lic)::value, L2 = decltype(l2c)::value, LT = decltype(ltc)::value;
-        if constexpr (triangle(LI, L2, LT)) produce<LI, L2, LT, FWD>(a, tg.bt, b0, tm, kc, As, warp, lane);
+        if constexpr (triangle(LI, L2, LT))
+          ok = produce_term<LI, L2, LT, FWD>(a, tg.bt, b0, tm, nk, sm, aempty, afull, q, s_abort, warp, lane);
       });
     });
   });
+  return ok;
 }
 
 // Accumulator rows 32 (w % 4) + lane of this warp to the target block: warps w and w + 4 share
@@ -244,20 +273,8 @@ __global__ void __launch_bounds__(UV_THREADS, 1) uvw_gemm_kernel(const __grid_co
         continue;
       }
       bool ok = true;
-      for (int j = tg.term_begin; j < tg.term_end && ok; ++j) {
-        for (int kc = 0; kc < nk; ++kc, ++q) {
-          const uint32_t s = q % UV_STAGES;
-          if (!warp_wait(&aempty[s], ((q / UV_STAGES) & 1u) ^ 1u, a.status, a.wait_ns)) {
-            *s_abort = 1;
-            ok = false;
-            break;
-          }
-          produce_chunk<FWD>(a, tg, b0, a.term[j], kc, sm + UvwSmem::a_off(int(s)), warp, lane);
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the tensor core reads A through the async proxy
-          __syncwarp();
-          if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(&afull[s])) : "memory");
-        }
-      }
+      for (int j = tg.term_begin; j < tg.term_end && ok; ++j)
+        ok = produce_term_any<FWD>(a, tg, b0, a.term[j], nk, sm, aempty, afull, q, s_abort, warp, lane);
       if (!ok) break;
       if (!warp_wait(accfull, tn & 1u, a.status, a.wait_ns)) {
         *s_abort = 1;
