@@ -110,13 +110,22 @@ __device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64
       return false;
     }
     unsigned char* As = sm + UvwSmem::a_off(int(s));
-    const int64_t u = int64_t(kc) * UV_KC + ul;
+    if (kc + 1 < nk) {
+      // ask L2 for the next chunk's runs now, so that their loads do not wait on HBM
+#pragma unroll
+      for (int k = 0; k < NSLOT; ++k) {
+        if (!valid[k]) continue;
+        const float* ip = inrow[k] + (int64_t(kc + 1) * UV_KC + ul) * DI;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(ip));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(ip + 4 * DI - 1));
+      }
+    }
 #pragma unroll
     for (int k = 0; k < NSLOT; ++k) {
       if (!valid[k]) continue;
       const int bl = 8 * (warp >> 1) + (lane & 7) + 32 * k;
       float in[4 * DI];  // channels u .. u + 3, components contiguous: one run of 4 DI floats
-      const float4* ip = reinterpret_cast<const float4*>(inrow[k] + u * DI);
+      const float4* ip = reinterpret_cast<const float4*>(inrow[k] + (int64_t(kc) * UV_KC + ul) * DI);
 #pragma unroll
       for (int j = 0; j < DI; ++j) {
         const float4 v = __ldg(ip + j);
