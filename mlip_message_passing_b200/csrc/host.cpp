@@ -317,11 +317,12 @@ extern "C" e3_status e3_cg_dense(int32_t l1, int32_t l2, int32_t l3, double* out
 }
 
 e3_plan::~e3_plan() {
-  if (uvw_prep != nullptr) {
+  if (uvw_prep != nullptr || uvw_z != nullptr) {
     int cur = -1;
     const bool restore = cudaGetDevice(&cur) == cudaSuccess && cur != device;
     if (restore) cudaSetDevice(device);
-    cudaFree(uvw_prep);
+    if (uvw_prep != nullptr) cudaFree(uvw_prep);
+    if (uvw_z != nullptr) cudaFree(uvw_z);
     if (restore) cudaSetDevice(cur);
   }
 }
@@ -406,6 +407,8 @@ static e3_status create_uvw(const std::vector<IrrepT>& ir1, const std::vector<Ir
   for (const auto& s : ins) n_out[s.io] += 1;
   for (const auto& s : ins) {
     const int l1 = ir1[s.i1].l, l3 = irf[s.io].l;
+    plan->z_off.push_back(int(plan->uvw_z_row));
+    plan->uvw_z_row += 2 * l3 + 1;
     plan->l1.push_back(l1);
     plan->l2.push_back(ir2[s.i2].l);
     plan->l3.push_back(l3);
@@ -425,6 +428,15 @@ static e3_status create_uvw(const std::vector<IrrepT>& ir1, const std::vector<Ir
     if (cudaMalloc(&plan->uvw_prep, plan->uvw_prep_size) != cudaSuccess) {
       plan->uvw_prep = nullptr;
       st = fail(E3_ERR_CUDA, "allocating the weight staging buffer (%zu bytes) failed", plan->uvw_prep_size);
+    }
+  }
+  if (st == E3_OK) {
+    // grad_y goes through Z_p = W_p g for every path, a batch of samples at a time (<= 256 MiB)
+    plan->uvw_z_row *= C;
+    plan->uvw_z_batch = std::max<int64_t>(128, std::min<int64_t>(16384, (int64_t(1) << 28) / (4 * plan->uvw_z_row)));
+    if (cudaMalloc(&plan->uvw_z, size_t(plan->uvw_z_batch) * plan->uvw_z_row * 4) != cudaSuccess) {
+      plan->uvw_z = nullptr;
+      st = fail(E3_ERR_CUDA, "allocating the grad_y staging buffer failed");
     }
   }
   if (st != E3_OK) {
@@ -683,9 +695,16 @@ static UuuArgs uuu_args(const e3_plan* plan, int64_t B, const void* x, const voi
 
 // Launch arguments of the uvw contraction.  Forward: targets are the output blocks, terms the paths
 // into each, input x.  grad_x: targets are the x blocks, terms the paths out of each, input grad_out.
-static e3_status uvw_gemm_args(const e3_plan* plan, int64_t B, bool fwd, const void* in, const void* y, void* out,
+// Roles of the uvw contraction kernel.
+enum { UVW_FWD = 0, UVW_GX = 1, UVW_PLAIN = 2 };
+
+// Launch arguments of the uvw contraction.  Forward: targets are the output blocks, terms the paths
+// into each, input x.  grad_x: targets are the x blocks, terms the paths out of each, input grad_out.
+// Plain (for grad_y): one target per path, its Z_p block (C channels), input grad_out.
+static e3_status uvw_gemm_args(const e3_plan* plan, int64_t B, int role, const void* in, const void* y, void* out,
                                UvwGemmArgs* a) {
   *a = UvwGemmArgs{};
+  const bool fwd = role == UVW_FWD;
   const int P = plan->n_paths, C = plan->C, Co = plan->Co;
   a->B = B;
   a->in = static_cast<const float*>(in);
@@ -694,29 +713,29 @@ static e3_status uvw_gemm_args(const e3_plan* plan, int64_t B, bool fwd, const v
   a->y = static_cast<const float*>(y);
   a->y_stride = plan->dim2;
   a->out = static_cast<float*>(out);
-  a->out_stride = fwd ? plan->dim_out : plan->dim1;
+  a->out_stride = fwd ? plan->dim_out : (role == UVW_GX ? plan->dim1 : plan->uvw_z_row);
   a->N = fwd ? Co : C;
   const size_t fwd_chunk = size_t(2) * Co * 32 * 4, bwd_chunk = size_t(2) * C * 32 * 4;
   a->prep = static_cast<const unsigned char*>(plan->uvw_prep) + (fwd ? 0 : size_t(P) * (C / 32) * fwd_chunk);
   a->b_chunk_bytes = uint32_t(fwd ? fwd_chunk : bwd_chunk);
-  const int nt = fwd ? int(plan->out_l.size()) : plan->LX + 1;
+  const int nt = fwd ? int(plan->out_l.size()) : (role == UVW_GX ? plan->LX + 1 : P);
   int64_t tiles = 0;
   int nterm = 0;
   for (int t = 0; t < nt; ++t) {
     UvwTarget& tg = a->tg[t];
-    tg.l = fwd ? plan->out_l[t] : t;
-    tg.off = fwd ? plan->out_off[t] : C * t * t;
+    tg.l = fwd ? plan->out_l[t] : (role == UVW_GX ? t : plan->l3[t]);
+    tg.off = fwd ? plan->out_off[t] : (role == UVW_GX ? C * t * t : C * plan->z_off[t]);
     tg.bt = 128 / (2 * tg.l + 1);
     tg.tile_begin = int32_t(tiles);
     tg.term_begin = nterm;
     for (int p = 0; p < P; ++p) {
-      if ((fwd ? plan->io[p] : plan->l1[p]) != t) continue;
+      if ((fwd ? plan->io[p] : (role == UVW_GX ? plan->l1[p] : p)) != t) continue;
       UvwTerm& tm = a->term[nterm++];
       tm.in_off = fwd ? plan->x_off[p] : plan->g_off[p];
       tm.l_in = fwd ? plan->l1[p] : plan->l3[p];
-      tm.l2 = plan->l2[p];
+      tm.l2 = role == UVW_PLAIN ? 0 : plan->l2[p];
       tm.chunk0 = fwd ? p * (C / 32) : p * (Co / 32);
-      tm.alpha = float(plan->alpha[p]);
+      tm.alpha = role == UVW_PLAIN ? 1.f : float(plan->alpha[p]);
     }
     tg.term_end = nterm;
     tiles += (B + tg.bt - 1) / tg.bt;
@@ -751,6 +770,7 @@ static UvwBwdArgs uvw_bwd_args(const e3_plan* plan, int64_t B, const void* x, co
     q.l3 = plan->l3[p];
     q.x_off = plan->x_off[p];
     q.g_off = plan->g_off[p];
+    q.z_off = plan->z_off[p];
     q.w_off = int64_t(p) * plan->C * plan->Co;
     q.alpha = float(plan->alpha[p]);
   }
@@ -788,9 +808,9 @@ extern "C" e3_status e3_tp_forward(const e3_plan* plan, int64_t B, const void* x
     st = launch_uvw_prep(plan->n_paths, plan->C, plan->Co, static_cast<const float*>(w), plan->uvw_prep, stream);
     if (st != E3_OK) return st;
     UvwGemmArgs g;
-    st = uvw_gemm_args(plan, B, true, x, y, out, &g);
+    st = uvw_gemm_args(plan, B, UVW_FWD, x, y, out, &g);
     if (st != E3_OK) return st;
-    return launch_uvw_gemm(g, true, stream);
+    return launch_uvw_gemm(g, UVW_FWD, stream);
   }
   return launch_forward(plan, a, false);
 }
@@ -869,12 +889,14 @@ extern "C" e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* 
   a.grad_w = grad_w;
   a.stream = stream;
   if (plan->mode == E3_UVW) {
-    if (grad_x) {
+    if (grad_x || grad_y) {
       st = launch_uvw_prep(plan->n_paths, plan->C, plan->Co, static_cast<const float*>(w), plan->uvw_prep, stream);
       if (st != E3_OK) return st;
+    }
+    if (grad_x) {
       UvwGemmArgs g;
-      st = uvw_gemm_args(plan, B, false, grad_out, y, grad_x, &g);
-      if (st == E3_OK) st = launch_uvw_gemm(g, false, stream);
+      st = uvw_gemm_args(plan, B, UVW_GX, grad_out, y, grad_x, &g);
+      if (st == E3_OK) st = launch_uvw_gemm(g, UVW_GX, stream);
       if (st != E3_OK) return st;
     }
     const UvwBwdArgs b = uvw_bwd_args(plan, B, x, y, w, grad_out, grad_w, grad_y);
@@ -882,7 +904,19 @@ extern "C" e3_status e3_tp_backward(const e3_plan* plan, int64_t B, const void* 
       st = launch_uvw_grad_w(b, stream);
       if (st != E3_OK) return st;
     }
-    if (grad_y) return launch_uvw_grad_y(b, stream);
+    if (grad_y) {
+      // Z_p = W_p g for a batch of samples on the tensor cores, then the contraction with x
+      for (int64_t b0 = 0; b0 < B; b0 += plan->uvw_z_batch) {
+        const int64_t nb = std::min<int64_t>(plan->uvw_z_batch, B - b0);
+        UvwGemmArgs g;
+        st = uvw_gemm_args(plan, nb, UVW_PLAIN, static_cast<const float*>(grad_out) + b0 * plan->dim_out, y,
+                           plan->uvw_z, &g);
+        if (st == E3_OK) st = launch_uvw_gemm(g, UVW_PLAIN, stream);
+        if (st == E3_OK)
+          st = launch_uvw_grad_y(b, static_cast<const float*>(plan->uvw_z), plan->uvw_z_row, b0, nb, stream);
+        if (st != E3_OK) return st;
+      }
+    }
     return E3_OK;
   }
   if (plan->mode == E3_UUU) {

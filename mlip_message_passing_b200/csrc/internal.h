@@ -21,10 +21,12 @@ struct e3_plan {
   std::string irreps_out;
   // uvw: output channels, per path the output block and offsets, the weight staging buffer
   int Co = 0;
-  std::vector<int> io, x_off, g_off;
+  std::vector<int> io, x_off, g_off, z_off;
   std::vector<int> out_l, out_off;  // per output block
   void* uvw_prep = nullptr;
   size_t uvw_prep_size = 0;
+  void* uvw_z = nullptr;            // Z of a batch of samples for grad_y
+  int64_t uvw_z_row = 0, uvw_z_batch = 0;
   ~e3_plan();
 };
 
@@ -184,7 +186,7 @@ e3_status launch_uuu(const e3_plan* plan, const UuuArgs& a, bool backward);
 // uvw tensor product with shared weights (tp_uvw.cu).
 // The tcgen05 contraction: per target block (an output block in the forward, an x block for
 // grad_x) the sum over its terms (paths) of alpha_p (coupled input) x W_p.
-constexpr int UVW_MAXT = 16;
+constexpr int UVW_MAXT = 64;
 constexpr int UVW_MAXP = 64;
 struct UvwTarget {
   int32_t off;          // offset of the block in a row of the result
@@ -221,6 +223,7 @@ struct UvwGemmArgs {
 struct UvwPath {
   int32_t l1, l2, l3;
   int32_t x_off, g_off;  // offsets of the path's x block and output block in their rows
+  int32_t z_off;         // per-channel offset of the path's block in a row of Z (sum of earlier 2 l3 + 1)
   int64_t w_off;         // offset of W_p [C][Cout] in the shared weights
   float alpha;
 };
@@ -241,9 +244,12 @@ struct UvwBwdArgs {
 e3_status upload_tables_uvw(const double* t64, const float* t32);
 size_t uvw_prep_bytes(int P, int C, int Co);
 e3_status launch_uvw_prep(int P, int C, int Co, const float* w, void* prep, void* stream);
-e3_status launch_uvw_gemm(const UvwGemmArgs& a, bool fwd, void* stream);
+// role: 0 forward (A = alpha C-coupled x), 1 grad_x (A = alpha C-coupled grad_out), 2 plain (A = the input)
+e3_status launch_uvw_gemm(const UvwGemmArgs& a, int role, void* stream);
 e3_status launch_uvw_grad_w(const UvwBwdArgs& a, void* stream);
-e3_status launch_uvw_grad_y(const UvwBwdArgs& a, void* stream);
+// grad_y of samples [b0, b0 + nb) from Z (row r = sample b0 + r, z_stride floats per row)
+e3_status launch_uvw_grad_y(const UvwBwdArgs& a, const float* z, int64_t z_stride, int64_t b0, int64_t nb,
+                            void* stream);
 
 // Zero rows [*first_row, n_rows) of a row-major array of row_bytes-byte rows (first_row read on
 // the device: the padding positions after the last CSR row).

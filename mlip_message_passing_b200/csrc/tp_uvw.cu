@@ -46,6 +46,9 @@ constexpr int UV_TMEM_COLS = 512;  // (UV_NBIG + 1) x UV_NMAX columns, rounded u
 constexpr uint32_t UV_A_BYTES = UV_M * UV_KC * 4;             // one of hi, lo
 constexpr uint32_t UV_B_BYTES_MAX = 2 * UV_NMAX * UV_KC * 4;  // hi + lo
 
+// What the math warps put into the A operand (see produce_term).
+enum UvwRole { ROLE_FWD = 0, ROLE_GX = 1, ROLE_PLAIN = 2 };
+
 struct UvwSmem {
   static constexpr size_t a_off(int s) { return size_t(s) * 2 * UV_A_BYTES; }
   static constexpr size_t b_off(int s) { return size_t(UV_STAGES) * 2 * UV_A_BYTES + size_t(s) * UV_B_BYTES_MAX; }
@@ -67,7 +70,7 @@ __device__ __forceinline__ int find_target(const UvwGemmArgs& a, int tile) {
 // and kept in registers for the term's chunks.  The eight lanes of one store phase hold eight
 // consecutive samples, whose rows differ modulo 8 (D is odd), so the 16-byte stores are free of
 // bank conflicts.  Returns false when a wait gave up (the abort flag is then set).
-template <int LI, int L2, int LT, bool FWD>
+template <int LI, int L2, int LT, int ROLE>
 __device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64_t b0, const UvwTerm& tm, int nk,
                                              unsigned char* sm, uint64_t* aempty, uint64_t* afull, uint32_t& q,
                                              volatile int* s_abort, int warp, int lane) {
@@ -85,11 +88,14 @@ __device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64
     inrow[k] = a.in + (valid[k] ? b * a.in_stride + tm.in_off : 0);
     float Y[NY2];
 #pragma unroll
-    for (int m = 0; m < 2 * L2 + 1; ++m) Y[L2 * L2 + m] = valid[k] ? __ldg(a.y + b * a.y_stride + L2 * L2 + m) : 0.f;
+    for (int m = 0; m < 2 * L2 + 1; ++m)
+      Y[L2 * L2 + m] = (ROLE != ROLE_PLAIN && valid[k]) ? __ldg(a.y + b * a.y_stride + L2 * L2 + m) : 0.f;
     static_for<0, DI>([&](auto ic) {
       static_for<0, DT>([&](auto tc) {
         constexpr int I = decltype(ic)::value, T = decltype(tc)::value;
-        if constexpr (FWD) {
+        if constexpr (ROLE == ROLE_PLAIN) {
+          cm[k][I][T] = I == T ? tm.alpha : 0.f;  // the input itself (DT == DI)
+        } else if constexpr (ROLE == ROLE_FWD) {
           if constexpr (a_nz(LI, L2, LT, I - LI, T - LT))
             cm[k][I][T] = tm.alpha * a_entry<float, LI, L2, LT, I - LI, T - LT>(Y);
           else
@@ -139,10 +145,14 @@ __device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64
         float v[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float acc = 0.f;
+          if constexpr (ROLE == ROLE_PLAIN) {
+            v[c] = tm.alpha * in[c * DI + t];
+          } else {
+            float acc = 0.f;
 #pragma unroll
-          for (int i = 0; i < DI; ++i) acc = fmaf(cm[k][i][t], in[c * DI + i], acc);
-          v[c] = acc;
+            for (int i = 0; i < DI; ++i) acc = fmaf(cm[k][i][t], in[c * DI + i], acc);
+            v[c] = acc;
+          }
         }
         float4 hi, lo;
         hi.x = to_tf32(v[0]);
@@ -165,21 +175,28 @@ __device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64
   return true;
 }
 
-template <bool FWD>
+template <int ROLE>
 __device__ __forceinline__ bool produce_term_any(const UvwGemmArgs& a, const UvwTarget& tg, int64_t b0,
                                                  const UvwTerm& tm, int nk, unsigned char* sm, uint64_t* aempty,
                                                  uint64_t* afull, uint32_t& q, volatile int* s_abort, int warp,
                                                  int lane) {
   bool ok = true;
-  dispatch<E3_LMAX + 1>(tm.l_in, [&](auto lic) {
-    dispatch<E3_LMAX + 1>(tm.l2, [&](auto l2c) {
-      dispatch<E3_LMAX + 1>(tg.l, [&](auto ltc) {
-        constexpr int LI = decltype(lic)::value, L2 = decltype(l2c)::value, LT = decltype(ltc)::value;
-        if constexpr (triangle(LI, L2, LT))
-          ok = produce_term<LI, L2, LT, FWD>(a, tg.bt, b0, tm, nk, sm, aempty, afull, q, s_abort, warp, lane);
+  if constexpr (ROLE == ROLE_PLAIN) {
+    dispatch<E3_LMAX + 1>(tm.l_in, [&](auto lic) {
+      constexpr int LI = decltype(lic)::value;
+      ok = produce_term<LI, 0, LI, ROLE>(a, tg.bt, b0, tm, nk, sm, aempty, afull, q, s_abort, warp, lane);
+    });
+  } else {
+    dispatch<E3_LMAX + 1>(tm.l_in, [&](auto lic) {
+      dispatch<E3_LMAX + 1>(tm.l2, [&](auto l2c) {
+        dispatch<E3_LMAX + 1>(tg.l, [&](auto ltc) {
+          constexpr int LI = decltype(lic)::value, L2 = decltype(l2c)::value, LT = decltype(ltc)::value;
+          if constexpr (triangle(LI, L2, LT))
+            ok = produce_term<LI, L2, LT, ROLE>(a, tg.bt, b0, tm, nk, sm, aempty, afull, q, s_abort, warp, lane);
+        });
       });
     });
-  });
+  }
   return ok;
 }
 
@@ -235,7 +252,7 @@ __device__ __forceinline__ void zero_rows(const UvwGemmArgs& a, const UvwTarget&
 // A consumer waits on parity (use & 1) of a full barrier; a producer on parity ((use & 1) ^ 1) of
 // an empty one, which a fresh barrier passes at once.  Tiles of targets without paths are zeroed
 // by the math warps and skipped by the other two roles (they count no barrier phases).
-template <bool FWD>
+template <int ROLE>
 __global__ void __launch_bounds__(UV_THREADS, 1) uvw_gemm_kernel(const __grid_constant__ UvwGemmArgs a) {
   extern __shared__ __align__(1024) unsigned char sm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -283,7 +300,7 @@ __global__ void __launch_bounds__(UV_THREADS, 1) uvw_gemm_kernel(const __grid_co
       }
       bool ok = true;
       for (int j = tg.term_begin; j < tg.term_end && ok; ++j)
-        ok = produce_term_any<FWD>(a, tg, b0, a.term[j], nk, sm, aempty, afull, q, s_abort, warp, lane);
+        ok = produce_term_any<ROLE>(a, tg, b0, a.term[j], nk, sm, aempty, afull, q, s_abort, warp, lane);
       if (!ok) break;
       if (!warp_wait(accfull, tn & 1u, a.status, a.wait_ns)) {
         *s_abort = 1;
@@ -501,109 +518,66 @@ __global__ void __launch_bounds__(GW_THREADS) uvw_grad_w_kernel(const __grid_con
   }
 }
 
-// ------------------------------------------------------------------ grad_y (CUDA cores) ---
+// ------------------------------------------------------------------ grad_y ---
 // grad_y[b, l2, m2] = sum_p alpha_p sum_{m1, m3} C_p[m1, m2, m3] sum_u x[b, u, m1] Z_p[b, u, m3],
-// Z_p[b, u, m3] = sum_w W_p[u, w] g[b, o(p), w, m3].  A CTA of C threads (thread u) takes GY_SB
-// samples and walks every path: it keeps the samples' grad_out block in shared memory (reloaded when
-// the block changes), forms Z_p for its channel from the weight row W_p[u, :] (32 columns at a time
-// in registers), contracts with its x and the coefficients, and sums over the channels with warp
-// shuffles and shared-memory atomics into the samples' grad_y, which it then writes (each sample
-// belongs to one CTA: no global atomics).
-constexpr int GY_SB = 8;
+// Z_p[b, u, m3] = sum_w W_p[u, w] g[b, o(p), w, m3].  Z (every path, a batch of samples) comes from
+// the tensor-core kernel in its plain role; here a CTA of C threads (thread u) takes one sample,
+// contracts its x and Z rows with the coefficients path by path, and sums over the channels with
+// warp shuffles and shared-memory atomics into the sample's grad_y.
 constexpr int GY_NY = (E3_LMAX + 1) * (E3_LMAX + 1);
 
 template <int L1, int L2, int L3>
-__device__ __forceinline__ void gy_path(const UvwBwdArgs& a, const UvwPath& pp, int64_t b0, int ns, const float* gS,
-                                        float* qS) {
-  constexpr int D1 = 2 * L1 + 1, D2 = 2 * L2 + 1, D3 = 2 * L3 + 1, NY2 = (L2 + 1) * (L2 + 1);
-  const int u = threadIdx.x, Co = a.Co;
-  float Z[GY_SB][D3];
+__device__ __forceinline__ void gy_path(const UvwBwdArgs& a, const UvwPath& pp, int64_t b, const float* zrow, float* qS) {
+  constexpr int D1 = 2 * L1 + 1, D2 = 2 * L2 + 1, D3 = 2 * L3 + 1;
+  const int u = threadIdx.x;
+  float xv[D1], zv[D3];
 #pragma unroll
-  for (int s = 0; s < GY_SB; ++s)
+  for (int m = 0; m < D1; ++m) xv[m] = __ldg(a.x + b * a.dim1 + pp.x_off + int64_t(u) * D1 + m);
 #pragma unroll
-    for (int m = 0; m < D3; ++m) Z[s][m] = 0.f;
-  const float* wrow = a.w + pp.w_off + int64_t(u) * Co;
-  for (int w0 = 0; w0 < Co; w0 += 32) {
-    float wr[32];
+  for (int m = 0; m < D3; ++m) zv[m] = __ldg(zrow + int64_t(pp.z_off) * a.C + int64_t(u) * D3 + m);
+  float c[D2];
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(wrow + w0 + j));
-      wr[j] = v.x, wr[j + 1] = v.y, wr[j + 2] = v.z, wr[j + 3] = v.w;
-    }
-#pragma unroll
-    for (int s = 0; s < GY_SB; ++s) {
-      const float* gs = gS + s * (Co * D3) + w0 * D3;
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-#pragma unroll
-        for (int m = 0; m < D3; ++m) Z[s][m] = fmaf(wr[j], gs[j * D3 + m], Z[s][m]);
-    }
-  }
-#pragma unroll
-  for (int s = 0; s < GY_SB; ++s) {
-    if (s >= ns) break;
-    const int64_t b = b0 + s;
-    float xv[D1];
-#pragma unroll
-    for (int m = 0; m < D1; ++m) xv[m] = __ldg(a.x + b * a.dim1 + pp.x_off + int64_t(u) * D1 + m);
-    float c[D2];
-#pragma unroll
-    for (int m = 0; m < D2; ++m) c[m] = 0.f;
-    static_for<-L1, L1 + 1>([&](auto m1c) {
-      static_for<-L2, L2 + 1>([&](auto m2c) {
-        static_for<-L3, L3 + 1>([&](auto m3c) {
-          constexpr int M1 = decltype(m1c)::value, M2 = decltype(m2c)::value, M3 = decltype(m3c)::value;
-          if constexpr (cg_nz(L1, L2, L3, M1, M2, M3)) {
-            constexpr int I = cg_index(L1, L2, L3, M1, M2, M3);
-            c[M2 + L2] = fmaf(CGT<float>::template get<I>() * xv[M1 + L1], Z[s][M3 + L3], c[M2 + L2]);
-          }
-        });
+  for (int m = 0; m < D2; ++m) c[m] = 0.f;
+  static_for<-L1, L1 + 1>([&](auto m1c) {
+    static_for<-L2, L2 + 1>([&](auto m2c) {
+      static_for<-L3, L3 + 1>([&](auto m3c) {
+        constexpr int M1 = decltype(m1c)::value, M2 = decltype(m2c)::value, M3 = decltype(m3c)::value;
+        if constexpr (cg_nz(L1, L2, L3, M1, M2, M3)) {
+          constexpr int I = cg_index(L1, L2, L3, M1, M2, M3);
+          c[M2 + L2] = fmaf(CGT<float>::template get<I>() * xv[M1 + L1], zv[M3 + L3], c[M2 + L2]);
+        }
       });
     });
+  });
 #pragma unroll
-    for (int m = 0; m < D2; ++m) {
-      float v = pp.alpha * c[m];
+  for (int m = 0; m < D2; ++m) {
+    float v = pp.alpha * c[m];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if ((threadIdx.x & 31) == 0) atomicAdd(&qS[s * GY_NY + L2 * L2 + m], v);
-    }
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&qS[L2 * L2 + m], v);
   }
-  (void)NY2;
 }
 
-__global__ void __launch_bounds__(UV_NMAX) uvw_grad_y_kernel(const __grid_constant__ UvwBwdArgs a) {
-  __shared__ __align__(16) float gS[GY_SB * UV_NMAX * 7];
-  __shared__ float qS[GY_SB * GY_NY];
-  const int64_t b0 = int64_t(blockIdx.x) * GY_SB;
-  const int ns = int(b0 + GY_SB <= a.B ? GY_SB : a.B - b0);
-  for (int i = threadIdx.x; i < GY_SB * GY_NY; i += blockDim.x) qS[i] = 0.f;
-  int loaded = -1;
+__global__ void __launch_bounds__(UV_NMAX) uvw_grad_y_kernel(const __grid_constant__ UvwBwdArgs a, const float* z,
+                                                             int64_t z_stride, int64_t b0) {
+  __shared__ float qS[GY_NY];
+  const int64_t b = b0 + blockIdx.x;
+  if (threadIdx.x < GY_NY) qS[threadIdx.x] = 0.f;
+  __syncthreads();
+  const float* zrow = z + int64_t(blockIdx.x) * z_stride;
   for (int p = 0; p < a.P; ++p) {
     const UvwPath& pp = a.path[p];
-    const int D3 = 2 * pp.l3 + 1, n = a.Co * D3;
-    if (pp.g_off != loaded) {
-      __syncthreads();
-      for (int i = threadIdx.x; i < GY_SB * n; i += blockDim.x) {
-        const int s = i / n;
-        gS[i] = s < ns ? __ldg(a.g + (b0 + s) * a.dim_out + pp.g_off + (i - s * n)) : 0.f;
-      }
-      __syncthreads();
-      loaded = pp.g_off;
-    }
     dispatch<E3_LMAX + 1>(pp.l1, [&](auto l1c) {
       dispatch<E3_LMAX + 1>(pp.l2, [&](auto l2c) {
         dispatch<E3_LMAX + 1>(pp.l3, [&](auto l3c) {
           constexpr int L1 = decltype(l1c)::value, L2 = decltype(l2c)::value, L3 = decltype(l3c)::value;
-          if constexpr (triangle(L1, L2, L3)) gy_path<L1, L2, L3>(a, pp, b0, ns, gS, qS);
+          if constexpr (triangle(L1, L2, L3)) gy_path<L1, L2, L3>(a, pp, b, zrow, qS);
         });
       });
     });
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < ns * int(a.dim2); i += blockDim.x) {
-    const int s = i / int(a.dim2), m = i - s * int(a.dim2);
-    a.grad_y[(b0 + s) * a.dim2 + m] = qS[s * GY_NY + m];
-  }
+  if (threadIdx.x < a.dim2) a.grad_y[b * a.dim2 + threadIdx.x] = qS[threadIdx.x];
 }
 
 }  // namespace
@@ -626,20 +600,23 @@ e3_status launch_uvw_prep(int P, int C, int Co, const float* w, void* prep, void
   return E3_OK;
 }
 
-e3_status launch_uvw_gemm(const UvwGemmArgs& a, bool fwd, void* stream) {
+e3_status launch_uvw_gemm(const UvwGemmArgs& a, int role, void* stream) {
   if (a.total_tiles <= 0 || a.B == 0) return E3_OK;
   if (a.N % 32 != 0 || a.N > UV_NMAX || a.k_in % UV_KC != 0) return fail(E3_ERR_UNSUPPORTED, "uvw channel counts");
   const size_t smem = UvwSmem::total();
   cudaError_t err =
-      fwd ? cudaFuncSetAttribute(uvw_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))
-          : cudaFuncSetAttribute(uvw_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      role == ROLE_FWD  ? cudaFuncSetAttribute(uvw_gemm_kernel<ROLE_FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))
+      : role == ROLE_GX ? cudaFuncSetAttribute(uvw_gemm_kernel<ROLE_GX>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))
+                        : cudaFuncSetAttribute(uvw_gemm_kernel<ROLE_PLAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw smem attribute: %s", cudaGetErrorString(err));
   const int grid = std::min(a.total_tiles, sm_count());
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (fwd)
-    uvw_gemm_kernel<true><<<grid, UV_THREADS, smem, s>>>(a);
+  if (role == ROLE_FWD)
+    uvw_gemm_kernel<ROLE_FWD><<<grid, UV_THREADS, smem, s>>>(a);
+  else if (role == ROLE_GX)
+    uvw_gemm_kernel<ROLE_GX><<<grid, UV_THREADS, smem, s>>>(a);
   else
-    uvw_gemm_kernel<false><<<grid, UV_THREADS, smem, s>>>(a);
+    uvw_gemm_kernel<ROLE_PLAIN><<<grid, UV_THREADS, smem, s>>>(a);
   err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
@@ -663,11 +640,11 @@ e3_status launch_uvw_grad_w(const UvwBwdArgs& a, void* stream) {
   return E3_OK;
 }
 
-e3_status launch_uvw_grad_y(const UvwBwdArgs& a, void* stream) {
-  if (a.B == 0) return E3_OK;
-  const int64_t blocks = (a.B + GY_SB - 1) / GY_SB;
-  if (blocks > INT_MAX) return fail(E3_ERR_SHAPE, "B too large");
-  uvw_grad_y_kernel<<<unsigned(blocks), a.C, 0, static_cast<cudaStream_t>(stream)>>>(a);
+e3_status launch_uvw_grad_y(const UvwBwdArgs& a, const float* z, int64_t z_stride, int64_t b0, int64_t nb,
+                            void* stream) {
+  if (nb <= 0) return E3_OK;
+  if (nb > INT_MAX) return fail(E3_ERR_SHAPE, "batch too large");
+  uvw_grad_y_kernel<<<unsigned(nb), a.C, 0, static_cast<cudaStream_t>(stream)>>>(a, z, z_stride, b0);
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw grad_y launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
