@@ -82,12 +82,14 @@ def hbm_peak():
 
 
 def kernel_source_hash():
-    """Hash of the library's code with comments and whitespace removed (a comment edit leaves the
-    kernels, and so the recorded DRAM traffic, unchanged; any code change changes the hash)."""
+    """Hash of the convolution kernels' code (kernels.cuh, cg_pattern.h, internal.h and the per-path-set
+    units tp_conv_l*.cu) with comments and whitespace removed: a comment edit leaves the kernels, and
+    so the recorded DRAM traffic, unchanged; any code change to them changes the hash."""
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mlip_message_passing_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    conv = lambda n: n in ("kernels.cuh", "cg_pattern.h", "internal.h") or (n.startswith("tp_conv_l") and n.endswith(".cu"))
+    for name in sorted(n for n in os.listdir(csrc) if conv(n)):
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)

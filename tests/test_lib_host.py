@@ -83,8 +83,7 @@ def test_plan_instruction_errors(e3b):
 
 
 def test_plan_unsupported(e3b):
-    # uvw mode, unsupported layouts, degrees without compiled kernels
-    assert _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", mode=1)[0] == e3b.E3_ERR_UNSUPPORTED
+    # unsupported layouts, degrees without compiled kernels
     assert _create(e3b, "8x0e+4x1o", "1x0e+1x1o+1x2e")[0] == e3b.E3_ERR_UNSUPPORTED
     assert _create(e3b, "8x1o+8x0e", "1x0e+1x1o+1x2e")[0] == e3b.E3_ERR_UNSUPPORTED
     assert _create(e3b, "6x0e+6x1o", "1x0e+1x1o+1x2e")[0] == e3b.E3_ERR_UNSUPPORTED
@@ -95,6 +94,24 @@ def test_plan_unsupported(e3b):
     assert _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", dtype=7)[0] == e3b.E3_ERR_INVALID_ARG
     assert _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", mode=3)[0] == e3b.E3_ERR_UNSUPPORTED
     assert _create(e3b, "8x0e+8x1o", "1x0e+1x1o+1x2e", mode=9)[0] == e3b.E3_ERR_INVALID_ARG
+
+
+def test_plan_uvw_validation(e3b):
+    # the fully connected mode needs output blocks, shared float32 weights and multiplicities in {32..128}
+    st, msg = _create(e3b, "32x0e+32x1o", "1x0e+1x1o", mode=1)
+    assert st == e3b.E3_ERR_INSTRUCTION and "irreps_out" in msg
+    st, msg = _create(e3b, "32x0e+32x1o", "1x0e+1x1o", "32x0e+32x1o", mode=1)
+    assert st == e3b.E3_ERR_UNSUPPORTED and "shared" in msg
+    st, msg = _create(e3b, "32x0e+32x1o", "1x0e+1x1o", "32x0e+32x1o", mode=1, wmode=1, dtype=1)
+    assert st == e3b.E3_ERR_UNSUPPORTED and "float32" in msg
+    st, msg = _create(e3b, "16x0e+16x1o", "1x0e+1x1o", "32x0e+32x1o", mode=1, wmode=1)
+    assert st == e3b.E3_ERR_UNSUPPORTED and "multiplicities" in msg
+    st, msg = _create(e3b, "32x0e+32x1o", "1x0e+1x1o", "32x0e+64x1o", mode=1, wmode=1)
+    assert st == e3b.E3_ERR_UNSUPPORTED and "common multiplicity" in msg
+    st, msg = _create(e3b, "32x0e", "1x0e", "32x1o", mode=1, wmode=1)
+    assert st == e3b.E3_ERR_INSTRUCTION and "no allowed path" in msg
+    st, msg = _create(e3b, "32x1o", "1x1o", "32x0o", instr=[(0, 0, 0)], mode=1, wmode=1)
+    assert st == e3b.E3_ERR_INSTRUCTION and "parity" in msg
 
 
 def test_plan_uuu_validation(e3b):
