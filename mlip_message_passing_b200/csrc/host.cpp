@@ -763,6 +763,8 @@ static UvwBwdArgs uvw_bwd_args(const e3_plan* plan, int64_t B, const void* x, co
   a.dim_out = plan->dim_out;
   a.grad_w = static_cast<float*>(grad_w);
   a.grad_y = static_cast<float*>(grad_y);
+  a.wait_ns = test_wait_limit_ns();
+  device_status_ptr(&a.status);
   for (int p = 0; p < plan->n_paths; ++p) {
     UvwPath& q = a.path[p];
     q.l1 = plan->l1[p];

@@ -226,6 +226,8 @@ struct UvwPath {
   int32_t z_off;         // per-channel offset of the path's block in a row of Z (sum of earlier 2 l3 + 1)
   int64_t w_off;         // offset of W_p [C][Cout] in the shared weights
   float alpha;
+  int64_t chunks;        // grad_w: K chunks of this path (filled by the launcher)
+  int32_t tile_begin;    // grad_w: first tile of this path
 };
 struct UvwBwdArgs {
   int64_t B;
@@ -239,6 +241,9 @@ struct UvwBwdArgs {
   int64_t dim_out;
   float* grad_w;
   float* grad_y;
+  int* status;
+  unsigned long long wait_ns;
+  int32_t total_tiles;   // grad_w (filled by the launcher)
   UvwPath path[UVW_MAXP];
 };
 e3_status upload_tables_uvw(const double* t64, const float* t32);

@@ -26,7 +26,8 @@
 //     tensor core rounds); after the last chunk of a tile the math warps load and add the
 //     accumulators (tcgen05.ld, float32) and store the sum.
 // Every wait is bounded (E3_ERR_TIMEOUT) and TMEM is released before the CTA exits.
-// grad_w (a reduction over samples) and grad_y (a reduction over channels) run on the CUDA cores.
+// grad_w, a contraction over samples, runs in a second tcgen05 kernel (both operands written by the
+// math warps); grad_y contracts Z_p = W_p g (this kernel, plain role) with x on the CUDA cores.
 #include <climits>
 
 #include "kernels.cuh"
@@ -421,101 +422,275 @@ __global__ void uvw_prep_kernel(int P, int C, int Co, const float* __restrict__ 
   }
 }
 
-// ------------------------------------------------------------------ grad_w (CUDA cores) ---
-// grad_W_p[u, w] = alpha_p sum_{b, m3} T_p[b, u, m3] g[b, o(p), w, m3]: a CTA takes one path and a
-// range of samples, in chunks of SB = floor(32 / D3) samples: it writes T_p of the chunk (rows
-// (sample, m3), columns u) and the chunk's grad_out block (rows (sample, m3), columns w) to shared
-// memory, then each thread accumulates an 8 x 8 block of (u, w) over the rows; the partial sums of
-// all CTAs of a path are added into grad_w (zeroed first) with atomics.
-constexpr int GW_THREADS = 256;
-constexpr int GW_ROWS = 32;
+// ------------------------------------------------------------- grad_w (tensor cores) ---
+// grad_W_p[u, w] = alpha_p sum_k T_p[k, u] g_p[k, w] over k = (sample, m3): a contraction whose K runs
+// over the samples.  A tile is one path and GT_CHUNKS chunks of K; a chunk holds SK = floor(32 / D3)
+// samples' D3 components (the last 32 - SK D3 positions stay zero).  The math warps write both
+// operands of a chunk (A[u][k] = T_p, B[w][k] = the grad_out block, tf32 high and low parts) after
+// putting the chunk's couplings sum_m2 C y in shared memory; one thread issues the three-pass MMAs
+// into four TMEM accumulators as in the forward; after a tile the math warps add the accumulators
+// and add alpha_p times them into grad_w (zeroed first) with atomics.  A tile sums at most
+// 64 x 32 products per accumulator row, so no accumulator takes more than ~90 additions.
+constexpr int GT_CHUNKS = 64;
+constexpr int GT_STAGES = 3;
+constexpr int GT_THREADS = 32 * UV_MATH_WARPS + 32;  // + the MMA warp
+constexpr uint32_t GT_A_BYTES = UV_M * UV_KC * 4;     // one of hi, lo
+constexpr uint32_t GT_B_BYTES = UV_NMAX * UV_KC * 4;  // one of hi, lo
+constexpr int GT_CM = 32 * 7 * 7;                     // couplings of one chunk: SK x DI x D3 <= 32 x 7 x 7 floats
 
+struct GtSmem {
+  static constexpr size_t a_off(int s) { return size_t(s) * 2 * (GT_A_BYTES + GT_B_BYTES); }
+  static constexpr size_t b_off(int s) { return a_off(s) + 2 * GT_A_BYTES; }
+  static constexpr size_t cm_off() { return a_off(GT_STAGES); }                  // two buffers
+  static constexpr size_t bar_off() { return cm_off() + 2 * GT_CM * 4; }
+  // full, empty [GT_STAGES] each, accfull, accempty; then the TMEM slot and the abort flag
+  static constexpr size_t total() { return bar_off() + 8 * (2 * GT_STAGES + 2) + 16; }
+};
+
+__device__ __forceinline__ int gt_find_path(const UvwBwdArgs& a, int tile) {
+  int p = 0;
+  while (p + 1 < a.P && tile >= a.path[p + 1].tile_begin) ++p;
+  return p;
+}
+
+// One chunk (chunk index ch of the path) of path pp: couplings, then A and B into stage As / Bs.
 template <int L1, int L2, int L3>
-__device__ __forceinline__ void gw_path(const UvwBwdArgs& a, const UvwPath& pp, int64_t bbeg, int64_t bend, float* Ts,
-                                        float* Gs, float (&acc)[8][8], int tu, int tw, bool active) {
-  constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, NY2 = (L2 + 1) * (L2 + 1), SB = GW_ROWS / D3;
-  const int C = a.C, Co = a.Co;
-  for (int64_t b0 = bbeg; b0 < bend; b0 += SB) {
-    const int ns = int(b0 + SB <= bend ? SB : bend - b0);
-    for (int i = threadIdx.x; i < SB * C; i += GW_THREADS) {
-      const int s = i / C, u = i - s * C;
-      float T[D3];
+__device__ __noinline__ void gt_chunk(const UvwBwdArgs& a, const UvwPath& pp, int64_t ch, unsigned char* As,
+                                      unsigned char* Bs, float* cmS, int tid) {
+  constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, NY2 = (L2 + 1) * (L2 + 1), SK = UV_KC / D3;
+  const int64_t bbase = ch * SK;
+  if (tid < SK) {
+    // couplings of sample tid: cm[i][t] = sum_m2 C[i, m2, t] y[m2]
+    const int64_t b = bbase + tid;
+    float Y[NY2];
 #pragma unroll
-      for (int m = 0; m < D3; ++m) T[m] = 0.f;
-      if (s < ns) {
-        const int64_t b = b0 + s;
-        float Y[NY2], xv[D1];
+    for (int m = 0; m < 2 * L2 + 1; ++m) Y[L2 * L2 + m] = b < a.B ? __ldg(a.y + b * a.dim2 + L2 * L2 + m) : 0.f;
+    float* cm = cmS + tid * D1 * D3;
+    static_for<0, D1>([&](auto ic) {
+      static_for<0, D3>([&](auto tc) {
+        constexpr int I = decltype(ic)::value, T = decltype(tc)::value;
+        if constexpr (a_nz(L1, L2, L3, I - L1, T - L3))
+          cm[I * D3 + T] = a_entry<float, L1, L2, L3, I - L1, T - L3>(Y);
+        else
+          cm[I * D3 + T] = 0.f;
+      });
+    });
+  } else {
+    // the next chunk's x and grad_out rows into L2 (one 128-byte line per thread and pass)
+    const int64_t nb = bbase + SK;
+    const int xl = (a.C * D1 * 4 + 127) / 128, gl = (a.Co * D3 * 4 + 127) / 128;
+    for (int i = tid - SK; i < SK * (xl + gl); i += 32 * UV_MATH_WARPS - SK) {
+      const int sl = i / (xl + gl), j = i - sl * (xl + gl);
+      const int64_t b = nb + sl;
+      if (b >= a.B) continue;
+      const float* ptr = j < xl ? a.x + b * a.dim1 + pp.x_off + 32 * j : a.g + b * a.dim_out + pp.g_off + 32 * (j - xl);
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(32 * UV_MATH_WARPS) : "memory");
+  // A[u][s D3 + m3] = T_p[b_s, u, m3] for channels u, u + 1 of sample s
+  const int nq = a.C / 2;
+  for (int task = tid; task < SK * nq; task += 32 * UV_MATH_WARPS) {
+    const int sl = task / nq, u = 2 * (task - sl * nq);
+    const int64_t b = bbase + sl;
+    float T[2][D3];
 #pragma unroll
-        for (int m = 0; m < 2 * L2 + 1; ++m) Y[L2 * L2 + m] = __ldg(a.y + b * a.dim2 + L2 * L2 + m);
+    for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int m = 0; m < D1; ++m) xv[m] = __ldg(a.x + b * a.dim1 + pp.x_off + int64_t(u) * D1 + m);
-        static_for<0, D3>([&](auto tc) {
-          static_for<0, D1>([&](auto ic) {
-            constexpr int M3 = decltype(tc)::value - L3, M1 = decltype(ic)::value - L1;
-            if constexpr (a_nz(L1, L2, L3, M1, M3))
-              T[M3 + L3] = fmaf(a_entry<float, L1, L2, L3, M1, M3>(Y), xv[M1 + L1], T[M3 + L3]);
-          });
-        });
+      for (int t = 0; t < D3; ++t) T[c][t] = 0.f;
+    if (b < a.B) {
+      const float2* xp = reinterpret_cast<const float2*>(a.x + b * a.dim1 + pp.x_off + int64_t(u) * D1);
+      float xv[2 * D1];
+#pragma unroll
+      for (int j = 0; j < D1; ++j) {
+        const float2 v = __ldg(xp + j);
+        xv[2 * j] = v.x, xv[2 * j + 1] = v.y;
       }
+      const float* cm = cmS + sl * D1 * D3;
 #pragma unroll
-      for (int m = 0; m < D3; ++m) Ts[(s * D3 + m) * C + u] = T[m];
+      for (int i = 0; i < D1; ++i)
+#pragma unroll
+        for (int t = 0; t < D3; ++t) {
+          const float cv = cm[i * D3 + t];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) T[c][t] = fmaf(cv, xv[c * D1 + i], T[c][t]);
+        }
     }
-    for (int i = threadIdx.x; i < SB * Co * D3; i += GW_THREADS) {
-      const int s = i / (Co * D3), r = i - s * (Co * D3);  // r = w D3 + m3, the block's memory order
-      const int w = r / D3, m = r - w * D3;
-      Gs[(s * D3 + m) * Co + w] = s < ns ? __ldg(a.g + (b0 + s) * a.dim_out + pp.g_off + r) : 0.f;
-    }
-    __syncthreads();
-    if (active) {
-      for (int r = 0; r < SB * D3; ++r) {
-        float av[8], bv[8];
-        const float4* ap = reinterpret_cast<const float4*>(Ts + r * C + tu * 8);
-        const float4* bp = reinterpret_cast<const float4*>(Gs + r * Co + tw * 8);
-        const float4 a0 = ap[0], a1 = ap[1], b0v = bp[0], b1v = bp[1];
-        av[0] = a0.x, av[1] = a0.y, av[2] = a0.z, av[3] = a0.w, av[4] = a1.x, av[5] = a1.y, av[6] = a1.z, av[7] = a1.w;
-        bv[0] = b0v.x, bv[1] = b0v.y, bv[2] = b0v.z, bv[3] = b0v.w, bv[4] = b1v.x, bv[5] = b1v.y, bv[6] = b1v.z,
-        bv[7] = b1v.w;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+    for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      for (int t = 0; t < D3; ++t) {
+        const float hi = to_tf32(T[c][t]), lo = to_tf32(T[c][t] - hi);
+        const uint32_t off = kmajor_off(u + c, sl * D3 + t, UV_KC);
+        *reinterpret_cast<float*>(As + off) = hi;
+        *reinterpret_cast<float*>(As + GT_A_BYTES + off) = lo;
       }
+  }
+  // B[w][s D3 + m3] = g[b_s, o(p), w, m3]
+  for (int task = tid; task < SK * a.Co; task += 32 * UV_MATH_WARPS) {
+    const int sl = task / a.Co, w = task - sl * a.Co;
+    const int64_t b = bbase + sl;
+    const float* gp = a.g + (b < a.B ? b * a.dim_out + pp.g_off + int64_t(w) * D3 : 0);
+#pragma unroll
+    for (int t = 0; t < D3; ++t) {
+      const float v = b < a.B ? __ldg(gp + t) : 0.f;
+      const float hi = to_tf32(v), lo = to_tf32(v - hi);
+      const uint32_t off = kmajor_off(w, sl * D3 + t, UV_KC);
+      *reinterpret_cast<float*>(Bs + off) = hi;
+      *reinterpret_cast<float*>(Bs + GT_B_BYTES + off) = lo;
     }
-    __syncthreads();
   }
 }
 
-__global__ void __launch_bounds__(GW_THREADS) uvw_grad_w_kernel(const __grid_constant__ UvwBwdArgs a, int64_t per_split) {
-  __shared__ __align__(16) float Ts[GW_ROWS * UV_NMAX];
-  __shared__ __align__(16) float Gs[GW_ROWS * UV_NMAX];
-  const UvwPath& pp = a.path[blockIdx.x];
-  const int nw = a.Co / 8;
-  const int tu = threadIdx.x / nw, tw = threadIdx.x - tu * nw;
-  const bool active = tu < a.C / 8;
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  const int64_t bbeg = int64_t(blockIdx.y) * per_split;
-  const int64_t bend = bbeg + per_split < a.B ? bbeg + per_split : a.B;
-  if (bbeg < bend) {
-    dispatch<E3_LMAX + 1>(pp.l1, [&](auto l1c) {
-      dispatch<E3_LMAX + 1>(pp.l2, [&](auto l2c) {
-        dispatch<E3_LMAX + 1>(pp.l3, [&](auto l3c) {
-          constexpr int L1 = decltype(l1c)::value, L2 = decltype(l2c)::value, L3 = decltype(l3c)::value;
-          if constexpr (triangle(L1, L2, L3)) gw_path<L1, L2, L3>(a, pp, bbeg, bend, Ts, Gs, acc, tu, tw, active);
+__global__ void __launch_bounds__(GT_THREADS, 1) uvw_grad_w_tc_kernel(const __grid_constant__ UvwBwdArgs a) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + GtSmem::bar_off());
+  uint64_t* empty = full + GT_STAGES;
+  uint64_t* accfull = empty + GT_STAGES;
+  uint64_t* accempty = accfull + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(accempty + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tslot + 1);
+  float* cmS = reinterpret_cast<float*>(sm + GtSmem::cm_off());
+
+  // the operand positions no chunk writes (k past SK D3, rows past C or Co) stay zero
+  for (size_t i = size_t(tid) * 16; i < GtSmem::cm_off(); i += size_t(GT_THREADS) * 16)
+    *reinterpret_cast<float4*>(sm + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tslot)),
+                 "r"(UV_TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    for (int i = 0; i < GT_STAGES; ++i) {
+      bar_init(&full[i], UV_MATH_WARPS);
+      bar_init(&empty[i], 1);
+    }
+    bar_init(accfull, 1);
+    bar_init(accempty, UV_MATH_WARPS);
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tslot;
+
+  // tiles in stride: a CTA's tiles mix paths of every degree (a contiguous range would leave the
+  // CTAs with degree-0 paths, whose chunks hold 32 samples, far behind: measured 2x slower)
+  if (warp < UV_MATH_WARPS) {
+    uint32_t q = 0, tn = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < a.total_tiles && ok; tile += gridDim.x, ++tn) {
+      const UvwPath& pp = a.path[gt_find_path(a, tile)];
+      const int64_t ch0 = int64_t(tile - pp.tile_begin) * GT_CHUNKS;
+      const int nck = int(pp.chunks - ch0 < GT_CHUNKS ? pp.chunks - ch0 : GT_CHUNKS);
+      for (int c = 0; c < nck; ++c, ++q) {
+        const uint32_t s = q % GT_STAGES;
+        // every math warp takes the same waits in the same order, so the block barrier inside the
+        // chunk is reached by all of them or (after an abort flag, read once per chunk) by none
+        const bool wok = warp_wait(&empty[s], ((q / GT_STAGES) & 1u) ^ 1u, a.status, a.wait_ns);
+        if (!wok) *s_abort = 1;
+        asm volatile("bar.sync 2, %0;" ::"r"(32 * UV_MATH_WARPS) : "memory");
+        if (*s_abort) {
+          ok = false;
+          break;
+        }
+        unsigned char* As = sm + GtSmem::a_off(int(s));
+        unsigned char* Bs = sm + GtSmem::b_off(int(s));
+        float* cm = cmS + (q & 1u) * GT_CM;
+        dispatch<E3_LMAX + 1>(pp.l1, [&](auto l1c) {
+          dispatch<E3_LMAX + 1>(pp.l2, [&](auto l2c) {
+            dispatch<E3_LMAX + 1>(pp.l3, [&](auto l3c) {
+              constexpr int L1 = decltype(l1c)::value, L2 = decltype(l2c)::value, L3 = decltype(l3c)::value;
+              if constexpr (triangle(L1, L2, L3)) gt_chunk<L1, L2, L3>(a, pp, ch0 + c, As, Bs, cm, tid);
+            });
+          });
         });
-      });
-    });
-  }
-  if (active && bbeg < bend) {
-    float* dst = a.grad_w + pp.w_off + int64_t(tu * 8) * a.Co + tw * 8;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the tensor core reads through the async proxy
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(&full[s])) : "memory");
+      }
+      if (!ok) break;
+      const bool aok = warp_wait(accfull, tn & 1u, a.status, a.wait_ns);
+      if (!aok) *s_abort = 1;
+      asm volatile("bar.sync 2, %0;" ::"r"(32 * UV_MATH_WARPS) : "memory");  // one verdict for all math warps
+      if (*s_abort) break;
+      fence_after_sync();
+      const int u = 32 * (warp & 3) + lane;
+      const int nbig = nck < UV_NBIG ? nck : UV_NBIG;
+      const uint32_t lane_base = tmem + (uint32_t(32 * (warp & 3)) << 16);
+      for (int cc = 32 * (warp >> 2); cc < a.Co; cc += 64) {
+        uint32_t v[32];
+        float sum[32];
+        tmem_ld32_nowait(lane_base + uint32_t(UV_NBIG * UV_NMAX + cc), v);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 32; ++i) sum[i] = __uint_as_float(v[i]);
+        for (int k = 0; k < nbig; ++k) {
+          tmem_ld32_nowait(lane_base + uint32_t(k * UV_NMAX + cc), v);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-      for (int j = 0; j < 8; ++j) atomicAdd(dst + int64_t(i) * a.Co + j, pp.alpha * acc[i][j]);
+          for (int i = 0; i < 32; ++i) sum[i] += __uint_as_float(v[i]);
+        }
+        if (u < a.C) {
+          float* dst = a.grad_w + pp.w_off + int64_t(u) * a.Co + cc;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) atomicAdd(dst + i, pp.alpha * sum[i]);
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(accempty)) : "memory");
+    }
+    __syncwarp();
+  } else if (lane == 0) {
+    // ------------------------------------------------------------- MMA thread
+    const uint32_t idesc = idesc_tf32(UV_M, a.Co);
+    uint32_t q = 0, tn = 0;
+    int64_t last = -1;
+    for (int tile = blockIdx.x; tile < a.total_tiles && !*s_abort; tile += gridDim.x, ++tn) {
+      const UvwPath& pp = a.path[gt_find_path(a, tile)];
+      const int64_t ch0 = int64_t(tile - pp.tile_begin) * GT_CHUNKS;
+      const int nck = int(pp.chunks - ch0 < GT_CHUNKS ? pp.chunks - ch0 : GT_CHUNKS);
+      if (!bar_wait(accempty, (tn & 1u) ^ 1u, a.status, a.wait_ns)) {
+        *s_abort = 1;
+        break;
+      }
+      fence_after_sync();
+      for (int c = 0; c < nck; ++c, ++q) {
+        const uint32_t s = q % GT_STAGES;
+        if (!bar_wait(&full[s], (q / GT_STAGES) & 1u, a.status, a.wait_ns)) {
+          *s_abort = 1;
+          break;
+        }
+        fence_after_sync();
+        const uint32_t a_hi = saddr(sm + GtSmem::a_off(int(s))), a_lo = a_hi + GT_A_BYTES;
+        const uint32_t b_hi = saddr(sm + GtSmem::b_off(int(s))), b_lo = b_hi + GT_B_BYTES;
+        const uint32_t big = tmem + (uint32_t(c) % UV_NBIG) * UV_NMAX, small = tmem + UV_NBIG * UV_NMAX;
+#pragma unroll
+        for (int ks = 0; ks < UV_KC / 8; ++ks) {
+          const uint32_t o = uint32_t(ks) * 256;
+          mma_tf32(big, smem_desc(a_hi + o, UV_KC), smem_desc(b_hi + o, UV_KC), idesc, (c < UV_NBIG && ks == 0) ? 0u : 1u);
+          mma_tf32(small, smem_desc(a_hi + o, UV_KC), smem_desc(b_lo + o, UV_KC), idesc, (c == 0 && ks == 0) ? 0u : 1u);
+          mma_tf32(small, smem_desc(a_lo + o, UV_KC), smem_desc(b_hi + o, UV_KC), idesc, 1u);
+        }
+        mma_commit(&empty[s]);
+        last = int64_t(q) + 1;
+      }
+      if (*s_abort) break;
+      mma_commit(accfull);
+    }
+    if (*s_abort && last > 0) {
+      const uint32_t lq = uint32_t(last - 1);
+      bar_wait(&empty[lq % GT_STAGES], (lq / GT_STAGES) & 1u, a.status, a.wait_ns);
+    }
   }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(UV_TMEM_COLS));
 }
 
 // ------------------------------------------------------------------ grad_y ---
@@ -626,15 +801,26 @@ e3_status launch_uvw_gemm(const UvwGemmArgs& a, int role, void* stream) {
 
 namespace e3b {
 
-e3_status launch_uvw_grad_w(const UvwBwdArgs& a, void* stream) {
+e3_status launch_uvw_grad_w(const UvwBwdArgs& in, void* stream) {
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t err = cudaMemsetAsync(a.grad_w, 0, sizeof(float) * size_t(a.P) * a.C * a.Co, s);
+  cudaError_t err = cudaMemsetAsync(in.grad_w, 0, sizeof(float) * size_t(in.P) * in.C * in.Co, s);
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "zeroing grad_w failed: %s", cudaGetErrorString(err));
-  if (a.B == 0) return E3_OK;
-  // about four CTAs per SM over all paths, each a contiguous range of samples
-  const int64_t splits = std::max<int64_t>(1, std::min<int64_t>((4 * int64_t(sm_count()) + a.P - 1) / a.P, (a.B + 7) / 8));
-  const int64_t per_split = (a.B + splits - 1) / splits;
-  uvw_grad_w_kernel<<<dim3(unsigned(a.P), unsigned(splits)), GW_THREADS, 0, s>>>(a, per_split);
+  if (in.B == 0) return E3_OK;
+  UvwBwdArgs a = in;
+  int64_t tiles = 0;
+  for (int p = 0; p < a.P; ++p) {
+    const int64_t sk = UV_KC / (2 * a.path[p].l3 + 1);
+    a.path[p].chunks = (a.B + sk - 1) / sk;
+    a.path[p].tile_begin = int32_t(tiles);
+    tiles += (a.path[p].chunks + GT_CHUNKS - 1) / GT_CHUNKS;
+  }
+  if (tiles >= INT_MAX) return fail(E3_ERR_SHAPE, "B too large");
+  a.total_tiles = int32_t(tiles);
+  const size_t smem = GtSmem::total();
+  err = cudaFuncSetAttribute(uvw_grad_w_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw grad_w smem attribute: %s", cudaGetErrorString(err));
+  const int grid = int(std::min<int64_t>(tiles, sm_count()));
+  uvw_grad_w_tc_kernel<<<grid, GT_THREADS, smem, s>>>(a);
   err = cudaGetLastError();
   if (err != cudaSuccess) return fail(E3_ERR_CUDA, "uvw grad_w launch failed: %s", cudaGetErrorString(err));
   return E3_OK;
