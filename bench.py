@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="conv_large", choices=["conv_waterbox", "conv_large"])
+    ap.add_argument("--kernel-case", choices=sorted(KERNEL_CASES), default=None,
+                    help="run one small case of a kernel a few times and exit (the target of profiler captures)")
     ap.add_argument("--reorder", default="none", choices=["none", "morton"],
                     help="renumber nodes along the Morton curve of their positions before timing")
     ap.add_argument("--order", default="morton", choices=["none", "morton"],
@@ -902,8 +904,69 @@ def run_native(args):
     return 0
 
 
+def case_radial(torch, e3b, W, dev):
+    """e3_radial_weights on 131 072 edges x 4352 weights (2.3 GB written: larger than L2), 4 launches."""
+    gen = torch.Generator(device=dev).manual_seed(0)
+    vec = torch.randn(131072, 3, generator=gen, device=dev) * 2.0
+    w1 = torch.randn(W.N_BASIS, W.HIDDEN, generator=gen, device=dev) / W.N_BASIS ** 0.5
+    w2 = torch.randn(W.HIDDEN, 4352, generator=gen, device=dev) / W.HIDDEN ** 0.5
+    rad = e3b.Radial(w1, w2, cutoff=W.CUTOFF, envelope_p=W.ENVELOPE_P)
+    for _ in range(4):
+        out = rad.weights(vec)
+    return float(out.abs().mean())
+
+
+def case_uvw(torch, e3b, W, dev):
+    """Fully connected product, 8192 samples of tp_uvw's shapes: 3 forward launches, then one backward."""
+    cfg = W.CONFIGS["tp_uvw"]
+    p = e3b.Plan(W.irreps_str(cfg["mul"], cfg["lx"]), W.sh_irreps(cfg["ly"]), cfg["irreps_out"], mode="uvw",
+                 shared_weights=True)
+    gen = torch.Generator(device=dev).manual_seed(0)
+    B = 8192
+    x = torch.randn(B, p.dim_in1, generator=gen, device=dev)
+    y = torch.randn(B, p.dim_in2, generator=gen, device=dev)
+    w = torch.randn(p.weight_numel, generator=gen, device=dev)
+    for _ in range(3):
+        out = e3b.tp_forward(p, x, y, w)
+    gx, gy, gw = e3b.tp_backward(p, x, y, w, torch.randn_like(out))
+    return float(out.abs().mean() + gw.abs().mean())
+
+
+def case_uuu(torch, e3b, W, dev):
+    """Channelwise product, 8192 samples of tp_uuu's shapes: 2 x (forward, backward)."""
+    cfg = W.CONFIGS["tp_uuu"]
+    ir = W.irreps_str(cfg["mul"], cfg["lx"])
+    p = e3b.Plan(ir, W.irreps_str(cfg["mul"], cfg["ly"]), lmax_out=cfg["lo"], mode="uuu")
+    gen = torch.Generator(device=dev).manual_seed(0)
+    B = 8192
+    x = torch.randn(B, p.dim_in1, generator=gen, device=dev)
+    y = torch.randn(B, p.dim_in2, generator=gen, device=dev)
+    w = torch.randn(B, p.weight_numel, generator=gen, device=dev)
+    go = torch.randn(B, p.dim_out, generator=gen, device=dev)
+    for _ in range(2):
+        out = e3b.tp_forward(p, x, y, w)
+        gx, gy, gw = e3b.tp_backward(p, x, y, w, go)
+    return float(out.abs().mean() + gx.abs().mean())
+
+
+KERNEL_CASES = {"radial": case_radial, "uvw": case_uvw, "uuu": case_uuu}
+
+
+def run_kernel_case(name):
+    import torch
+    from mlip_message_passing_b200 import e3b, workloads as W
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    v = KERNEL_CASES[name](torch, e3b, W, dev)
+    e3b.device_status()
+    print(json.dumps({"kernel_case": name, "checksum": v}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.kernel_case:
+        return run_kernel_case(args.kernel_case)
     if args.impl == "reference":
         return run_reference(args)
     if args.shard:
