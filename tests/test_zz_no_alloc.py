@@ -56,3 +56,35 @@ def test_static_csr_rejects_too_many_edges():
     st = e3b.lib.e3_csr_build_static(10, limit + 1, None, None, None, None, None, None, None)
     assert st == e3b.E3_ERR_SHAPE
     assert "limit" in e3b.lib.e3_last_error().decode()
+
+
+def test_static_csr_runs_inside_a_stream_capture():
+    """The reason the entry point exists: a call recorded into a CUDA graph (stream capture fails on
+    any allocation or synchronisation inside it) and replayed gives the workspace build's arrays, and
+    an ordinary call changes torch's allocated device memory by nothing."""
+    from mlip_message_passing_b200 import e3b
+    dev = torch.device("cuda", 0)
+    rng = np.random.default_rng(5)
+    n, e = 5000, 60000
+    src = torch.as_tensor(rng.integers(0, n, e).astype(np.int32), device=dev)
+    dst = torch.as_tensor(rng.integers(0, n, e).astype(np.int32), device=dev)
+    ref = e3b.csr_build(n, src, dst)
+    _static_build(e3b, n, src, dst)                           # warm-up: device state set up once
+    torch.cuda.synchronize()
+    bufs = [torch.full((e,), -7, dtype=torch.int32, device=dev), torch.full((n + 1,), -7, dtype=torch.int32, device=dev),
+            torch.full((e,), -7, dtype=torch.int32, device=dev), torch.full((n + 1,), -7, dtype=torch.int32, device=dev)]
+    before = torch.cuda.memory_allocated(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        st = e3b.lib.e3_csr_build_static(n, e, e3b._ptr(src), e3b._ptr(dst), e3b._ptr(bufs[0]), e3b._ptr(bufs[1]),
+                                         e3b._ptr(bufs[2]), e3b._ptr(bufs[3]), e3b._stream())
+    assert st == e3b.E3_OK, e3b.lib.e3_last_error().decode()
+    for b in bufs:
+        b.fill_(-7)
+    graph.replay()
+    torch.cuda.synchronize()
+    e3b.device_status()
+    for got, want in zip(bufs, ref):
+        assert torch.equal(got, want)
+    assert torch.cuda.memory_allocated(dev) == before
+    del graph
