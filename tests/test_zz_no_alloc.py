@@ -59,9 +59,9 @@ def test_static_csr_rejects_too_many_edges():
 
 
 def test_static_csr_runs_inside_a_stream_capture():
-    """The reason the entry point exists: a call recorded into a CUDA graph (stream capture fails on
-    any allocation or synchronisation inside it) and replayed gives the workspace build's arrays, and
-    an ordinary call changes torch's allocated device memory by nothing."""
+    """The reason the entry point exists: an ordinary call changes torch's allocated device memory by
+    nothing, and a call recorded into a CUDA graph (stream capture fails on any allocation or
+    synchronisation inside it) and replayed gives the workspace build's arrays."""
     from mlip_message_passing_b200 import e3b
     dev = torch.device("cuda", 0)
     rng = np.random.default_rng(5)
@@ -73,7 +73,12 @@ def test_static_csr_runs_inside_a_stream_capture():
     torch.cuda.synchronize()
     bufs = [torch.full((e,), -7, dtype=torch.int32, device=dev), torch.full((n + 1,), -7, dtype=torch.int32, device=dev),
             torch.full((e,), -7, dtype=torch.int32, device=dev), torch.full((n + 1,), -7, dtype=torch.int32, device=dev)]
+    # an ordinary call into preallocated outputs leaves torch's allocated device memory unchanged
     before = torch.cuda.memory_allocated(dev)
+    st = e3b.lib.e3_csr_build_static(n, e, e3b._ptr(src), e3b._ptr(dst), e3b._ptr(bufs[0]), e3b._ptr(bufs[1]),
+                                     e3b._ptr(bufs[2]), e3b._ptr(bufs[3]), e3b._stream())
+    torch.cuda.synchronize()
+    assert st == e3b.E3_OK and torch.cuda.memory_allocated(dev) == before
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         st = e3b.lib.e3_csr_build_static(n, e, e3b._ptr(src), e3b._ptr(dst), e3b._ptr(bufs[0]), e3b._ptr(bufs[1]),
@@ -86,5 +91,4 @@ def test_static_csr_runs_inside_a_stream_capture():
     e3b.device_status()
     for got, want in zip(bufs, ref):
         assert torch.equal(got, want)
-    assert torch.cuda.memory_allocated(dev) == before
     del graph
