@@ -38,11 +38,14 @@
  *     instructions writing the same output block (uncollapsed: sqrt(2 l3 + 1)).
  *   - Errors are returned before any launch when they can be seen on the host; the message
  *     is available from e3_last_error().  Errors seen on the device (an index out of range,
- *     a bounded wait that gave up) are recorded in one status word per device, shared by
- *     every call on that device, and read (and cleared) by e3_device_status(); the offending
- *     edge is skipped, never dereferenced.
+ *     a bounded wait that gave up) are recorded in a status word: the plan's own for calls
+ *     that take a plan (read and cleared by e3_plan_status()), one per device for the others
+ *     (CSR, harmonics, radial network); e3_device_status() reads and clears the device's word
+ *     and the words of every live plan on the device.  The offending edge is skipped, never
+ *     dereferenced.
  *   - Results are deterministic: the same inputs give bitwise the same outputs (no atomics
- *     on floating-point data).
+ *     on floating-point data), except the uvw mode's grad_w and grad_y, which add partial sums
+ *     with float atomics (their last bits may differ from run to run).
  *   - Per-device state (the status word, the coefficient tables, the address of the static CSR
  *     scratch) is set up on a device's first use and kept for the life of the process: after
  *     cudaDeviceReset, or after the primary context is destroyed, the library must not be called
@@ -142,9 +145,15 @@ E3_API e3_status e3_plan_irreps_out(const e3_plan* plan, char* buf, size_t buf_l
  * n_paths entries; either may be NULL). */
 E3_API e3_status e3_plan_paths(const e3_plan* plan, int32_t* lls, double* alpha);
 
-/* Synchronise `stream`, return the current device's status word (E3_OK, E3_ERR_INDEX or
- * E3_ERR_TIMEOUT; the first error recorded since the last read) and clear it. */
+/* Synchronise `stream`, return the current device's status (E3_OK, E3_ERR_INDEX or
+ * E3_ERR_TIMEOUT; the first error recorded since the last read by the calls without a plan or by
+ * any live plan on the device) and clear it. */
 E3_API e3_status e3_device_status(void* stream);
+
+/* Synchronise `stream`, return the status word of `plan` (errors recorded by the kernels of calls
+ * made with this plan since the last read) and clear it.  Calls on other plans, concurrent or not,
+ * do not touch it; calls on this plan from several streams share it. */
+E3_API e3_status e3_plan_status(const e3_plan* plan, void* stream);
 
 /* Real CG table as generated for the plan's kernels: dense [2l1+1][2l2+1][2l3+1] doubles
  * for (l1, l2, l3), written to out (host).  Exposed for table-against-table checks. */

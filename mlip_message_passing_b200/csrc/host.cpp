@@ -316,15 +316,40 @@ extern "C" e3_status e3_cg_dense(int32_t l1, int32_t l2, int32_t l3, double* out
   return E3_OK;
 }
 
+// Live plans, so that e3_device_status can drain their status words too.
+static std::mutex g_plans_mu;
+static std::vector<e3_plan*> g_plans;
+
 e3_plan::~e3_plan() {
-  if (uvw_prep != nullptr || uvw_z != nullptr) {
+  {
+    std::lock_guard<std::mutex> lock(g_plans_mu);
+    for (size_t i = 0; i < g_plans.size(); ++i)
+      if (g_plans[i] == this) {
+        g_plans.erase(g_plans.begin() + long(i));
+        break;
+      }
+  }
+  if (uvw_prep != nullptr || uvw_z != nullptr || status != nullptr) {
     int cur = -1;
     const bool restore = cudaGetDevice(&cur) == cudaSuccess && cur != device;
     if (restore) cudaSetDevice(device);
     if (uvw_prep != nullptr) cudaFree(uvw_prep);
     if (uvw_z != nullptr) cudaFree(uvw_z);
+    if (status != nullptr) cudaFree(status);
     if (restore) cudaSetDevice(cur);
   }
+}
+
+// The plan's own status word (zeroed), and its entry in the list of live plans.
+static e3_status plan_attach_status(e3_plan* plan) {
+  if (cudaMalloc(reinterpret_cast<void**>(&plan->status), 256) != cudaSuccess) {
+    plan->status = nullptr;
+    return fail(E3_ERR_CUDA, "allocating the plan's status word failed");
+  }
+  if (cudaMemset(plan->status, 0, 256) != cudaSuccess) return fail(E3_ERR_CUDA, "zeroing the plan's status word failed");
+  std::lock_guard<std::mutex> lock(g_plans_mu);
+  g_plans.push_back(plan);
+  return E3_OK;
 }
 
 // Plan of the fully connected (uvw) mode: x = Cx0+..+CxLx, y = 1x0+..+1xLy, output blocks of one
@@ -439,6 +464,7 @@ static e3_status create_uvw(const std::vector<IrrepT>& ir1, const std::vector<Ir
       st = fail(E3_ERR_CUDA, "allocating the grad_y staging buffer failed");
     }
   }
+  if (st == E3_OK) st = plan_attach_status(plan);
   if (st != E3_OK) {
     delete plan;
     return st;
@@ -584,7 +610,8 @@ extern "C" e3_status e3_plan_create(const char* irreps_in1, const char* irreps_i
   plan->weight_numel = int64_t(P) * C;
   plan->irreps_out = irreps_to_string(out_irreps);
   packed_cg_table();
-  const e3_status st = ensure_device_tables();
+  e3_status st = ensure_device_tables();
+  if (st == E3_OK) st = plan_attach_status(plan);
   if (st != E3_OK) {
     delete plan;
     return st;
@@ -637,19 +664,48 @@ extern "C" e3_status e3_plan_paths(const e3_plan* plan, int32_t* lls, double* al
   return E3_OK;
 }
 
+static e3_status check_plan_device(const e3_plan* plan);
+
+// Read and clear the status words `words` (device pointers) in stream order after synchronising
+// `stream`; the first nonzero one is the result.
+static e3_status drain_status(const std::vector<int*>& words, void* stream, const char* who) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::vector<int> h(words.size(), 0);
+  for (size_t i = 0; i < words.size(); ++i)
+    if (cudaMemcpyAsync(&h[i], words[i], sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemsetAsync(words[i], 0, sizeof(int), s) != cudaSuccess)
+      return fail(E3_ERR_CUDA, "reading a status word failed: %s", cudaGetErrorString(cudaGetLastError()));
+  if (cudaStreamSynchronize(s) != cudaSuccess)
+    return fail(E3_ERR_CUDA, "reading a status word failed: %s", cudaGetErrorString(cudaGetLastError()));
+  for (int v : h)
+    if (v != E3_OK)
+      return fail(static_cast<e3_status>(v), "%s reported %s", who,
+                  v == E3_ERR_INDEX ? "an index out of range" : (v == E3_ERR_TIMEOUT ? "a wait that gave up" : "an error"));
+  return E3_OK;
+}
+
 extern "C" e3_status e3_device_status(void* stream) {
   clear_error();
   int* d = nullptr;
   e3_status st = device_status_ptr(&d);
   if (st != E3_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int h = 0;
-  if (cudaMemcpyAsync(&h, d, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaMemsetAsync(d, 0, sizeof(int), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
-    return fail(E3_ERR_CUDA, "reading the device status word failed: %s", cudaGetErrorString(cudaGetLastError()));
-  if (h == E3_OK) return E3_OK;
-  return fail(static_cast<e3_status>(h), "device reported %s",
-              h == E3_ERR_INDEX ? "an index out of range" : (h == E3_ERR_TIMEOUT ? "a wait that gave up" : "an error"));
+  int dev = -1;
+  cudaGetDevice(&dev);
+  std::vector<int*> words{d};
+  {
+    std::lock_guard<std::mutex> lock(g_plans_mu);
+    for (e3_plan* p : g_plans)
+      if (p->device == dev && p->status != nullptr) words.push_back(p->status);
+  }
+  return drain_status(words, stream, "device");
+}
+
+extern "C" e3_status e3_plan_status(const e3_plan* plan, void* stream) {
+  clear_error();
+  const e3_status st = check_plan_device(plan);
+  if (st != E3_OK) return st;
+  if (plan->status == nullptr) return fail(E3_ERR_INVALID_ARG, "plan has no status word");
+  return drain_status({plan->status}, stream, "plan");
 }
 
 // ========================================================= C ABI: compute entry points ===
@@ -744,7 +800,8 @@ static e3_status uvw_gemm_args(const e3_plan* plan, int64_t B, int role, const v
   a->n_targets = nt;
   a->total_tiles = int32_t(tiles);
   a->wait_ns = test_wait_limit_ns();
-  return device_status_ptr(&a->status);
+  a->status = plan->status;
+  return E3_OK;
 }
 
 static UvwBwdArgs uvw_bwd_args(const e3_plan* plan, int64_t B, const void* x, const void* y, const void* w,
@@ -764,7 +821,7 @@ static UvwBwdArgs uvw_bwd_args(const e3_plan* plan, int64_t B, const void* x, co
   a.grad_w = static_cast<float*>(grad_w);
   a.grad_y = static_cast<float*>(grad_y);
   a.wait_ns = test_wait_limit_ns();
-  device_status_ptr(&a.status);
+  a.status = plan->status;
   for (int p = 0; p < plan->n_paths; ++p) {
     UvwPath& q = a.path[p];
     q.l1 = plan->l1[p];

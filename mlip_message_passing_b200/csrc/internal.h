@@ -27,6 +27,7 @@ struct e3_plan {
   size_t uvw_prep_size = 0;
   void* uvw_z = nullptr;            // Z of a batch of samples for grad_y
   int64_t uvw_z_row = 0, uvw_z_batch = 0;
+  int* status = nullptr;            // this plan's device status word (its kernels record errors here)
   ~e3_plan();
 };
 

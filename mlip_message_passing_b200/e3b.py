@@ -30,7 +30,7 @@ SYMBOLS = [
     "e3_morton_order", "e3_invert_permutation", "e3_remap_ids", "e3_conv_workspace_size",
     "e3_conv_topology_size", "e3_conv_topology_build", "e3_set_test_knobs", "e3_add_rows",
     "e3_conv_topology_build_ordered", "e3_radial_prep_size", "e3_radial_prepare", "e3_radial_weights",
-    "e3_spherical_harmonics_double_backward",
+    "e3_spherical_harmonics_double_backward", "e3_plan_status",
 ]
 
 
@@ -60,6 +60,7 @@ def _load():
         "e3_plan_irreps_out": [VP, ctypes.c_char_p, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)],
         "e3_plan_paths": [VP, ctypes.POINTER(I32), ctypes.POINTER(D)],
         "e3_device_status": [VP],
+        "e3_plan_status": [VP, VP],
         "e3_cg_dense": [I32, I32, I32, ctypes.POINTER(D)],
         "e3_supported": [],
         "e3_tp_forward": [VP, I64, VP, VP, VP, VP, VP],
@@ -211,6 +212,11 @@ class Plan:
     @property
     def handle(self):
         return self._handle
+
+    def status(self):
+        """Synchronise the current stream; raise E3Error if a kernel of a call made with this plan
+        recorded an error since the last read (e3_plan_status)."""
+        _check(lib.e3_plan_status(self._handle, _stream()))
 
     def _w_shape(self, rows):
         return (self.weight_numel,) if self.shared_weights else (rows, self.weight_numel)

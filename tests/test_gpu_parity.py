@@ -517,6 +517,37 @@ def test_conv_bad_index_is_reported_not_dereferenced(e3b):
     e3b.device_status()
 
 
+def test_errors_are_attributed_to_the_plan(e3b):
+    """Two plans used one after the other on one stream: the index error raised by a call on the
+    first plan is reported by that plan's status only; the second plan's status stays clean, and the
+    device-wide status is clean once the plan's word has been read."""
+    pa = gplan(e3b, 8, 1, 2, 2, torch.float32)
+    pb = gplan(e3b, 8, 1, 2, 2, torch.float32)
+    n = 4
+    src = np.array([0, 1, 2, 3], dtype=np.int32)
+    dst = np.array([1, 2, 3, 0], dtype=np.int32)
+    bad = e3b.Graph(n, t(src), t(dst))
+    bad.src[2] = 1000  # a sender id out of range, after the CSR was built
+    good = e3b.Graph(n, t(src), t(dst))
+    x = torch.randn(n, pa.dim_in1, device=DEV)
+    w = torch.randn(4, pa.weight_numel, device=DEV)
+    vec = torch.randn(4, 3, device=DEV)
+    e3b.conv_forward(pa, bad, x, w, edge_vec=vec)
+    e3b.conv_forward(pb, good, x, w, edge_vec=vec)
+    pb.status()  # clean
+    with pytest.raises(e3b.E3Error) as ei:
+        pa.status()
+    assert ei.value.status == e3b.E3_ERR_INDEX
+    pa.status()  # read and cleared
+    e3b.device_status()
+    # the device-wide read also drains a plan's word
+    e3b.conv_forward(pa, bad, x, w, edge_vec=vec)
+    with pytest.raises(e3b.E3Error) as ei:
+        e3b.device_status()
+    assert ei.value.status == e3b.E3_ERR_INDEX
+    pa.status()
+
+
 def test_conv_deterministic(e3b):
     g, graph, w = conv_setup(e3b, 400, 64, 2, 3, 2, 22, torch.float32)
     p = gplan(e3b, 64, 2, 3, 2, torch.float32)
