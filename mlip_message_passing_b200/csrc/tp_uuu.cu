@@ -150,6 +150,17 @@ __global__ void __launch_bounds__(UUU_THREADS) uuu_bwd_kernel(const UuuArgs a) {
   const T* w = static_cast<const T*>(a.w) + b * a.w_stride + u;
   const T* g = static_cast<const T*>(a.grad_out) + b * a.dim_out;
   T* gw = a.grad_w ? static_cast<T*>(a.grad_w) + b * a.w_stride + u : nullptr;
+  if constexpr (RUN) {
+    // ask L2 for every path's grad_out run and weight line of this warp now: the loop below reads
+    // them one path after the other, and each would otherwise wait on HBM in turn
+    static_for<0, CF::P>([&](auto pc) {
+      constexpr int P = decltype(pc)::value;
+      using PC = PathC<CF, P>;
+      const T* run = g + int64_t(a.C) * PC::OUT + int64_t(u - lane) * PC::D3;
+      if (lane * 128 < int(32 * PC::D3 * sizeof(T))) asm volatile("prefetch.global.L2 [%0];" ::"l"(run + lane * 128 / int(sizeof(T))));
+      if (lane == 31) asm volatile("prefetch.global.L2 [%0];" ::"l"(w + int64_t(P) * a.C));
+    });
+  }
   static_for<0, CF::P>([&](auto pc) {
     constexpr int P = decltype(pc)::value;
     using PC = PathC<CF, P>;
