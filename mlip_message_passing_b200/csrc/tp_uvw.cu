@@ -72,9 +72,9 @@ __device__ __forceinline__ int find_target(const UvwGemmArgs& a, int tile) {
 // consecutive samples, whose rows differ modulo 8 (D is odd), so the 16-byte stores are free of
 // bank conflicts.  Returns false when a wait gave up (the abort flag is then set).
 template <int LI, int L2, int LT, int ROLE>
-__device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64_t b0, const UvwTerm& tm, int nk,
-                                             unsigned char* sm, uint64_t* aempty, uint64_t* afull, uint32_t& q,
-                                             volatile int* s_abort, int warp, int lane) {
+__device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64_t b0, const UvwTerm& tm,
+                                             const UvwTerm* next, int nk, unsigned char* sm, uint64_t* aempty,
+                                             uint64_t* afull, uint32_t& q, volatile int* s_abort, int warp, int lane) {
   constexpr int DI = 2 * LI + 1, DT = 2 * LT + 1, NY2 = (L2 + 1) * (L2 + 1);
   constexpr int NSLOT = (UV_M / DT + 31) / 32;
   const int ul = 16 * (warp & 1) + 4 * (lane >> 3);
@@ -125,6 +125,16 @@ __device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64
         const float* ip = inrow[k] + (int64_t(kc + 1) * UV_KC + ul) * DI;
         asm volatile("prefetch.global.L2 [%0];" ::"l"(ip));
         asm volatile("prefetch.global.L2 [%0];" ::"l"(ip + 4 * DI - 1));
+      }
+    } else if (next != nullptr) {
+      // the last chunk of this term: the next term's first chunk (same samples, another block)
+      const int dn = 2 * next->l_in + 1;
+#pragma unroll
+      for (int k = 0; k < NSLOT; ++k) {
+        if (!valid[k]) continue;
+        const float* ip = inrow[k] - tm.in_off + next->in_off + int64_t(ul) * dn;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(ip));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(ip + 4 * dn - 1));
       }
     }
 #pragma unroll
@@ -178,14 +188,14 @@ __device__ __forceinline__ bool produce_term(const UvwGemmArgs& a, int bt, int64
 
 template <int ROLE>
 __device__ __forceinline__ bool produce_term_any(const UvwGemmArgs& a, const UvwTarget& tg, int64_t b0,
-                                                 const UvwTerm& tm, int nk, unsigned char* sm, uint64_t* aempty,
-                                                 uint64_t* afull, uint32_t& q, volatile int* s_abort, int warp,
-                                                 int lane) {
+                                                 const UvwTerm& tm, const UvwTerm* next, int nk, unsigned char* sm,
+                                                 uint64_t* aempty, uint64_t* afull, uint32_t& q,
+                                                 volatile int* s_abort, int warp, int lane) {
   bool ok = true;
   if constexpr (ROLE == ROLE_PLAIN) {
     dispatch<E3_LMAX + 1>(tm.l_in, [&](auto lic) {
       constexpr int LI = decltype(lic)::value;
-      ok = produce_term<LI, 0, LI, ROLE>(a, tg.bt, b0, tm, nk, sm, aempty, afull, q, s_abort, warp, lane);
+      ok = produce_term<LI, 0, LI, ROLE>(a, tg.bt, b0, tm, next, nk, sm, aempty, afull, q, s_abort, warp, lane);
     });
   } else {
     dispatch<E3_LMAX + 1>(tm.l_in, [&](auto lic) {
@@ -193,7 +203,8 @@ __device__ __forceinline__ bool produce_term_any(const UvwGemmArgs& a, const Uvw
         dispatch<E3_LMAX + 1>(tg.l, [&](auto ltc) {
           constexpr int LI = decltype(lic)::value, L2 = decltype(l2c)::value, LT = decltype(ltc)::value;
           if constexpr (triangle(LI, L2, LT))
-            ok = produce_term<LI, L2, LT, ROLE>(a, tg.bt, b0, tm, nk, sm, aempty, afull, q, s_abort, warp, lane);
+            ok = produce_term<LI, L2, LT, ROLE>(a, tg.bt, b0, tm, next, nk, sm, aempty, afull, q, s_abort, warp,
+                                                lane);
         });
       });
     });
@@ -301,7 +312,8 @@ __global__ void __launch_bounds__(UV_THREADS, 1) uvw_gemm_kernel(const __grid_co
       }
       bool ok = true;
       for (int j = tg.term_begin; j < tg.term_end && ok; ++j)
-        ok = produce_term_any<ROLE>(a, tg, b0, a.term[j], nk, sm, aempty, afull, q, s_abort, warp, lane);
+        ok = produce_term_any<ROLE>(a, tg, b0, a.term[j], j + 1 < tg.term_end ? &a.term[j + 1] : nullptr, nk, sm,
+                                    aempty, afull, q, s_abort, warp, lane);
       if (!ok) break;
       if (!warp_wait(accfull, tn & 1u, a.status, a.wait_ns)) {
         *s_abort = 1;
