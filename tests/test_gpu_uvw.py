@@ -143,3 +143,20 @@ def test_uvw_unsupported(e3b):
     p = e3b.Plan("32x0e+32x1o", "1x0e+1x1o", "32x0e+32x1o", mode="uvw", shared_weights=True)
     with pytest.raises(e3b.E3Error, match="UNSUPPORTED"):
         e3b.conv_workspace(p, 10, 20, DEV)
+
+
+def test_uvw_explicit_instructions_and_path_weight(e3b):
+    """An explicit instruction list (a subset of the fully connected one, out of loop order, one
+    path weight given) goes through the library's explicit path: same plan as the oracle's."""
+    ir1, ir2, irout = "32x0e+32x1o+32x2e", "1x0e+1x1o+1x2e", "64x1o+64x0e+64x2e"
+    ins = [(2, 1, 0), (0, 0, 1), (1, 1, 1, 0.7), (1, 0, 0), (2, 2, 2), (0, 2, 2)]
+    p = e3b.Plan(ir1, ir2, irout, instructions=ins, mode="uvw", shared_weights=True)
+    q = oracle.make_plan(ir1, ir2, irout, instructions=[oracle.Instruction(*i[:3], True, i[3] if len(i) > 3 else -1.0)
+                                                         for i in ins], mode="uvw", shared_weights=True)
+    assert p.n_paths == q.n_paths == len(ins) and p.weight_numel == q.weight_numel
+    np.testing.assert_allclose(p.alphas, q.alphas, rtol=1e-15)
+    x, y, w = inputs(p, 77, seed=4)
+    assert rel_err(h(e3b.tp_forward(p, t(x), t(y), t(w))), oracle.tp_forward(q, x, y, w)) <= 1e-5
+    g = np.random.default_rng(5).standard_normal((77, p.dim_out)).astype(np.float32)
+    for got, want in zip(e3b.tp_backward(p, t(x), t(y), t(w), t(g)), oracle.tp_backward(q, x, y, w, g)):
+        assert rel_err(h(got), want) <= 1e-5
