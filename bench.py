@@ -645,13 +645,16 @@ class ConvCase:
 
 
 def measure_e2e(case, steps, world, dist, dev):
-    """End to end through the public API (e3b.conv_forward / e3b.conv_backward) from pinned host
-    memory: every step copies its inputs in and all its results out.  Steps alternate between two
-    streams with their own device buffers, so step k's results travel to the host while step
-    k+1's inputs travel in; the device-to-host copies of consecutive steps are ordered (one set of
-    host result buffers)."""
+    """End to end through the public API: the step a training loop runs on one batch of this graph.
+    Per step the batch's data -- node features x and the edge vectors -- come in from pinned host
+    memory; the model's parameters stay on the device: the radial network's W1, W2 (laid out once by
+    e3b.Radial) and a fixed linear readout R of the output (loss = <R, out>, so grad_out = R).  The
+    step evaluates the path weights (e3b.Radial.weights, tcgen05), the convolution forward
+    (e3b.conv_forward), the loss, the convolution backward (e3b.conv_backward: grad_x, grad_y,
+    grad_w) and copies the loss back.  The input copies run on their own stream into two alternating
+    buffer sets, so the next step's inputs travel in while this step computes."""
     import torch
-    from mlip_message_passing_b200 import e3b
+    from mlip_message_passing_b200 import e3b, workloads as W
     stream = torch.cuda.current_stream()
     plan, graph, s = case.plan, case.graph, case.scale
 
@@ -660,29 +663,43 @@ def measure_e2e(case, steps, world, dist, dev):
         h.copy_(t)
         return h
 
-    hin = tuple(pinned_copy(t) for t in (case.x, case.vec, case.w, case.go))
-    shapes = [case.out.shape, case.x.shape, case.gy.shape, case.w.shape]
-    case.free()  # the headline buffers are no longer needed: room for two device sets
-    hout = tuple(torch.empty(sh, dtype=torch.float32, pin_memory=True) for sh in shapes)
-    streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
+    hin = (pinned_copy(case.x), pinned_copy(case.vec))
+    R = case.go
+    w1, w2 = (torch.as_tensor(m.astype(np.float32), device=dev) for m in case.mlp)
+    rad = e3b.Radial(w1, w2, W.CUTOFF, W.ENVELOPE_P)
+    n_out = rad.n_out
+    E = case.E
+    case.go = None
+    case.free()  # keep R (the readout) and the graph; the headline's other buffers go
+    case.graph = graph
+    w_buf = torch.empty((E, n_out), dtype=torch.float32, device=dev)
+    out_buf = torch.empty((case.N, plan.dim_out), dtype=torch.float32, device=dev)
     dev_in = [tuple(torch.empty_like(t, device=dev) for t in hin) for _ in range(2)]
-    d2h_done = [None]
+    loss_dev = torch.zeros(1, dtype=torch.float32, device=dev)
+    loss_host = torch.zeros(1, dtype=torch.float32, pin_memory=True)
+    copy_stream, comp_stream = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    consumed = [None, None]  # per buffer set: the compute of the last step that read it
 
     def e2e_step(k):
-        dx_, dvec_, dw_, dgo_ = dev_in[k % 2]
-        st = streams[k % 2]
-        with torch.cuda.stream(st):
-            for d_, h_ in zip(dev_in[k % 2], hin):
+        j = k % 2
+        with torch.cuda.stream(copy_stream):
+            if consumed[j] is not None:
+                copy_stream.wait_event(consumed[j])
+            for d_, h_ in zip(dev_in[j], hin):
                 d_.copy_(h_, non_blocking=True)
-            o = e3b.conv_forward(plan, graph, dx_, dw_, edge_vec=dvec_, out_scale=s)
-            r = e3b.conv_backward(plan, graph, dx_, dw_, dgo_, edge_vec=dvec_, out_scale=s)
-            if d2h_done[0] is not None:
-                st.wait_event(d2h_done[0])
-            for h_, d_ in zip(hout, (o, r[0], r[1], r[2])):
-                h_.copy_(d_, non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(st)
-            d2h_done[0] = ev
+            landed = torch.cuda.Event()
+            landed.record(copy_stream)
+        with torch.cuda.stream(comp_stream):
+            comp_stream.wait_event(landed)
+            x_, vec_ = dev_in[j]
+            rad.weights(vec_, w_buf)
+            e3b.conv_forward(plan, graph, x_, w_buf, edge_vec=vec_, out_scale=s, out=out_buf)
+            loss_dev.copy_(torch.dot(out_buf.view(-1), R.view(-1)).reshape(1))
+            e3b.conv_backward(plan, graph, x_, w_buf, R, edge_vec=vec_, out_scale=s)
+            loss_host.copy_(loss_dev, non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(comp_stream)
+            consumed[j] = done
 
     e2e_step(0)
     e2e_step(1)
@@ -691,14 +708,14 @@ def measure_e2e(case, steps, world, dist, dev):
         dist.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for st_ in streams:
-        st_.wait_event(a)
+    copy_stream.wait_event(a)
+    comp_stream.wait_event(a)
     for k in range(steps):
         e2e_step(k)
-    for st_ in streams:
-        done = torch.cuda.Event()
-        done.record(st_)
-        stream.wait_event(done)
+    for st_ in (copy_stream, comp_stream):
+        fin = torch.cuda.Event()
+        fin.record(st_)
+        stream.wait_event(fin)
     b.record(stream)
     torch.cuda.synchronize()
     e3b.device_status()
@@ -706,12 +723,17 @@ def measure_e2e(case, steps, world, dist, dev):
         dist.barrier()
     e_ms = max_over_ranks(a.elapsed_time(b) / steps, world, dist, dev)
     h2d = sum(t.numel() * t.element_size() for t in hin)
-    d2h = sum(t.numel() * t.element_size() for t in hout)
-    del dev_in, hin, hout
+    d2h = loss_host.numel() * loss_host.element_size()
+    loss = float(loss_host[0])
+    del dev_in, hin, w_buf, out_buf, rad
+    case.go = None
     torch.cuda.empty_cache()
     return {"value": job_throughput(case.E_work, world, e_ms), "unit": "edges/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": e_ms,
-            "overlap": "two streams: step k's device-to-host copies overlap step k+1's host-to-device copies"}
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": e_ms, "loss": loss,
+            "step": "h2d of x and the edge vectors (pinned), radial weights (tcgen05), conv forward, "
+                    "loss = <R, out>, conv backward (grad_x, grad_y, grad_w), d2h of the loss; radial "
+                    "parameters and the readout R resident on the device",
+            "overlap": "the next step's inputs are copied on their own stream into the other of two buffer sets"}
 
 
 def run_sharded(args):
