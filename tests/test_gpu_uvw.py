@@ -160,3 +160,25 @@ def test_uvw_explicit_instructions_and_path_weight(e3b):
     g = np.random.default_rng(5).standard_normal((77, p.dim_out)).astype(np.float32)
     for got, want in zip(e3b.tp_backward(p, t(x), t(y), t(w), t(g)), oracle.tp_backward(q, x, y, w, g)):
         assert rel_err(h(got), want) <= 1e-5
+
+
+def test_uvw_as_a_per_irrep_linear(e3b):
+    """The channel-mixing linear of a layer (per irrep, out_l = x_l W_l / sqrt(C)) is the fully
+    connected product with y = 1x0e of ones: checked against plain float64 matrix products, at the
+    shapes of the large graph's node features (128 -> 128 channels, degrees 0..3)."""
+    ir = W.irreps_str(128, 3)
+    p = e3b.Plan(ir, "1x0e", ir, mode="uvw", shared_weights=True)
+    assert p.n_paths == 4
+    rng = np.random.default_rng(15)
+    B = 3000
+    x = rng.standard_normal((B, p.dim_in1)).astype(np.float32)
+    Wl = [rng.standard_normal((128, 128)).astype(np.float32) for _ in range(4)]
+    w = np.concatenate([m.ravel() for m in Wl])
+    out = h(e3b.tp_forward(p, t(x), t(np.ones((B, 1), np.float32)), t(w)))
+    want, o = [], 0
+    for l in range(4):
+        d = 2 * l + 1
+        xl = x[:, o:o + 128 * d].reshape(B, 128, d).astype(np.float64)
+        want.append((np.einsum("uw,bum->bwm", Wl[l].astype(np.float64), xl) / np.sqrt(128.0)).reshape(B, -1))
+        o += 128 * d
+    assert rel_err(out, np.concatenate(want, axis=1)) <= 1e-5

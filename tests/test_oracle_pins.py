@@ -364,6 +364,29 @@ def test_scalar_path_modes_closed_forms():
     np.testing.assert_allclose(oracle.tp_forward(pw, x, y, W.reshape(4, -1)), want, atol=1e-14)
 
 
+def test_uvw_with_scalar_y_is_a_per_irrep_linear():
+    """With y = 1x0e the only paths are l x 0 -> l, whose coefficients are delta(m1, m3)/sqrt(2l+1)
+    (course 03a: coupling with a scalar), and the fan of an output element is mul_x: the fully
+    connected product is then the per-irrep channel mixing out_l[w, m] = sum_u W_l[u, w] x_l[u, m] y /
+    sqrt(mul_x), written here with plain matrix products."""
+    rng = np.random.default_rng(14)
+    ir1, irout = "4x0e+4x1o+4x2e", "3x0e+3x1o+3x2e"
+    plan = oracle.make_plan(ir1, "1x0e", irout, instructions=[(0, 0, 0), (1, 0, 1), (2, 0, 2)], mode="uvw")
+    B = 5
+    x = rng.standard_normal((B, plan.irreps_in1.dim))
+    y = rng.standard_normal((B, 1))
+    W = [rng.standard_normal((4, 3)) for _ in range(3)]
+    w = np.concatenate([m.ravel() for m in W])[None].repeat(B, axis=0)
+    got = oracle.tp_forward(plan, x, y, w)
+    want, o1 = [], 0
+    for l in range(3):
+        d = 2 * l + 1
+        xl = x[:, o1:o1 + 4 * d].reshape(B, 4, d)
+        want.append((np.einsum("uw,bum->bwm", W[l], xl) * y[:, :, None] / 2.0).reshape(B, -1))
+        o1 += 4 * d
+    np.testing.assert_allclose(got, np.concatenate(want, axis=1), atol=1e-13)
+
+
 def test_mode_validation():
     with pytest.raises(ValueError):
         oracle.make_plan("2x1o", "3x1o", lmax_out=2, mode="uuu")  # uuu ties x and y channels
